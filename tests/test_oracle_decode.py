@@ -1,0 +1,206 @@
+"""Pins for the oracle's paged decode attention: textbook attention on
+FP4-exact inputs, split/merge invariance, and closed forms of the fused
+probability quantization with and without underflow-aware scaling."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+E2M1_POS = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def _exact_fp4(rng, shape_blocks, beta, axis_len):
+    """Values that NVFP4 represents exactly with a unit tensor scale: every
+    beta-block along the last axis holds one +-6*2^j and E2M1 points * 2^j."""
+    vals = rng.choice(E2M1_POS, size=shape_blocks + (axis_len,)) * rng.choice([-1, 1], size=shape_blocks + (axis_len,))
+    nb = axis_len // beta
+    j = rng.integers(-3, 3, size=shape_blocks + (nb,))
+    pos = rng.integers(0, beta, size=shape_blocks + (nb,))
+    for idx in np.ndindex(*shape_blocks, nb):
+        blk = idx[-1]
+        vals[idx[:-1] + (blk * beta + pos[idx],)] = 6.0 * rng.choice([-1, 1])
+    scale = np.repeat(2.0 ** j, beta, axis=-1)
+    return (vals * scale).astype(np.float32)
+
+
+def _bf16(a):
+    return torch.tensor(np.asarray(a, np.float32)).to(torch.bfloat16)
+
+
+def _pages(seq_lens, rng):
+    npages = [(n + 63) // 64 for n in seq_lens]
+    num_pages = max(1, sum(npages))
+    perm = rng.permutation(num_pages)
+    maxp = max(1, max(npages))
+    bt = np.zeros((len(seq_lens), maxp), np.int32)
+    off = 0
+    slots = []
+    for b, n in enumerate(seq_lens):
+        bt[b, : npages[b]] = perm[off: off + npages[b]]
+        off += npages[b]
+        t = np.arange(n)
+        slots.append(bt[b, t // 64].astype(np.int64) * 64 + t % 64)
+    return bt, num_pages, np.concatenate(slots) if slots else np.zeros(0, np.int64)
+
+
+def _exact_case(rng, seq_lens, H_q, H_kv, d, fmt=0):
+    beta = 16 if fmt == 0 else 32
+    T = int(sum(seq_lens))
+    k = _exact_fp4(rng, (T, H_kv), beta, d)
+    # V blocks run along tokens: build per (head, channel) along the token axis,
+    # block-aligned per sequence (pages start at token 0 of each sequence)
+    v = np.zeros((T, H_kv, d), np.float32)
+    off = 0
+    for n in seq_lens:
+        npad = ((n + beta - 1) // beta) * beta
+        if npad:
+            vv = _exact_fp4(rng, (H_kv, d), beta, npad)        # [H_kv, d, npad]
+            if n % beta:
+                # the last block is partial: move its +-6*2^j onto a valid token
+                last = npad - beta
+                blk = vv[:, :, last:]
+                big = np.argmax(np.abs(blk), axis=-1)
+                for h in range(H_kv):
+                    for c in range(d):
+                        val = blk[h, c, big[h, c]]
+                        blk[h, c, big[h, c]] = blk[h, c, 0]
+                        blk[h, c, 0] = val
+            v[off: off + n] = np.transpose(vv, (2, 0, 1))[:n]
+        off += n
+    q = _exact_fp4(rng, (len(seq_lens), H_q), beta, d)
+    return q, k, v
+
+
+@pytest.mark.parametrize("G,seq_lens", [(4, [1000]), (8, [129, 0, 77, 513]), (1, [64, 300])])
+def test_exact_inputs_match_textbook_attention(ora, G, seq_lens):
+    rng = np.random.default_rng(G)
+    H_kv, d = 2, 128
+    H_q = G * H_kv
+    q, k, v = _exact_case(rng, seq_lens, H_q, H_kv, d)
+    bt, num_pages, sm = _pages(seq_lens, rng)
+    ones = np.ones((H_kv, d), np.float32)
+    g = np.ones(H_kv, np.float32)
+    cache = ora.empty_cache(num_pages, H_kv, d, d, ora.NVFP4)
+    fl = ora.FLAG_NO_HADAMARD
+    ora.quantize_kv(_bf16(k), _bf16(v), sm, cache, H_kv, ora.NVFP4, ones, g, g, num_pages, flags=fl)
+    # the cache holds the inputs exactly
+    t = 0
+    for b, n in enumerate(seq_lens):
+        for i in range(0, n, 37):
+            page, slot = bt[b, i // 64], i % 64
+            for h in range(H_kv):
+                assert np.array_equal(ora.dequant_key_row(cache, 0, page, h, H_kv, d, slot), k[t + i, h])
+                assert np.array_equal(ora.dequant_value_row(cache, 0, page, h, H_kv, d, slot), v[t + i, h])
+        t += n
+    sm_scale = 1 / math.sqrt(d) / 8
+    cu = np.concatenate([[0], np.cumsum(seq_lens)])
+    ref = ora.attention_ref(_bf16(q), _bf16(k), _bf16(v), cu, H_kv, sm_scale)
+    outs = []
+    for chunk in (1, 2, 1000):
+        o16, o64 = ora.decode(_bf16(q), cache, bt, np.array(seq_lens), H_kv, d, ora.NVFP4, ones, g, g,
+                              sm_scale, chunk, num_pages, flags=fl | ora.FLAG_EXACT_P)
+        scale = np.abs(ref).max() + 1e-30
+        assert np.max(np.abs(o64 - ref)) <= 1e-6 * scale, chunk
+        outs.append(o64)
+    # splits do not change the (unquantized-P) result
+    assert np.allclose(outs[0], outs[2], rtol=0, atol=1e-12 * (np.abs(ref).max() + 1e-30))
+    # empty sequence -> zeros
+    for b, n in enumerate(seq_lens):
+        if n == 0:
+            assert np.all(outs[0][b] == 0)
+
+
+def _uniform_case(ora, fmt, flags):
+    rng = np.random.default_rng(42)
+    H_kv, G, d, N = 1, 4, 128, 300
+    q = np.zeros((1, G, d), np.float32)
+    _, k, v = _exact_case(rng, [N], G, H_kv, d, fmt)
+    bt, num_pages, sm = _pages([N], rng)
+    ones = np.ones((H_kv, d), np.float32)
+    g = np.ones(H_kv, np.float32)
+    cache = ora.empty_cache(num_pages, H_kv, d, d, fmt)
+    ora.quantize_kv(_bf16(k), _bf16(v), sm, cache, H_kv, fmt, ones, g, g, num_pages, flags=ora.FLAG_NO_HADAMARD)
+    o16, o64 = ora.decode(_bf16(q), cache, bt, np.array([N]), H_kv, d, fmt, ones, g, g, 0.1, 1, num_pages,
+                          flags=ora.FLAG_NO_HADAMARD | flags)
+    return o64, v
+
+
+@pytest.mark.parametrize("fmt,flags,pscale", [
+    (0, 0, 1.03125),                      # p = 1 -> E4M3(2048/6)=352, E2M1(5.82)=6 -> 6*352/2048
+    (0, 8, 1.03125),                      # vanilla: E4M3(1/6)=0.171875 -> 6*0.171875
+    (1, 0, 1.0),                          # MXFP4: X = 2^-2, 1/X = 4 exactly
+])
+def test_uniform_logits_closed_form(ora, fmt, flags, pscale):
+    # q = 0 -> every logit is 0 -> p = 1 for every token; l counts tokens
+    o64, v = _uniform_case(ora, fmt, flags)
+    expect = pscale * v[:, 0].astype(np.float64).mean(0)
+    for h in range(4):
+        assert np.allclose(o64[0, h], expect, rtol=1e-12, atol=1e-12)
+
+
+def _sink_case(ora, fmt, flags, N=300, chunk=1000):
+    """One key with logit 10, the rest 0: p = 1 and e^-10 per token."""
+    rng = np.random.default_rng(7)
+    H_kv, G, d = 1, 2, 128
+    q = np.zeros((1, G, d), np.float32)
+    q[0, :, 0] = 6.0
+    k = np.zeros((N, H_kv, d), np.float32)
+    k[0, 0, 0] = 6.0
+    _, _, v = _exact_case(rng, [N], G, H_kv, d, fmt)
+    bt, num_pages, sm = _pages([N], rng)
+    ones = np.ones((H_kv, d), np.float32)
+    g = np.ones(H_kv, np.float32)
+    cache = ora.empty_cache(num_pages, H_kv, d, d, fmt)
+    ora.quantize_kv(_bf16(k), _bf16(v), sm, cache, H_kv, fmt, ones, g, g, num_pages, flags=ora.FLAG_NO_HADAMARD)
+    o16, o64 = ora.decode(_bf16(q), cache, bt, np.array([N]), H_kv, d, fmt, ones, g, g, 10.0 / 36.0, chunk,
+                          num_pages, flags=ora.FLAG_NO_HADAMARD | flags)
+    return o64, v[:, 0].astype(np.float64)
+
+
+def test_underflow_aware_scaling_closed_form(ora):
+    N = 300
+    l = 1.0 + (N - 1) * math.exp(-10.0)
+    # alpha = 2^11: tiny blocks get E4M3 scale 2^-6 and code 6 -> 6 * 2^-6 / 2048
+    o, v = _sink_case(ora, 0, 0, N)
+    tail = 6 * 2.0 ** -6 / 2048
+    expect = (1.03125 * v[0] + tail * v[16:].sum(0)) / l
+    assert np.allclose(o[0, 0], expect, rtol=1e-5, atol=1e-9)
+    # vanilla alpha = 1: every block without the sink collapses (E4M3(e^-10/6) = 0)
+    o, v = _sink_case(ora, 0, ora.FLAG_NO_UNDERFLOW, N)
+    assert np.allclose(o[0, 0], 1.03125 * v[0] / l, rtol=1e-5, atol=1e-9)
+    # MXFP4: E8M0 scale 2^-17 keeps the tail, block of the sink is 32 tokens
+    o, v = _sink_case(ora, 1, 0, N)
+    expect = (1.0 * v[0] + 6 * 2.0 ** -17 * v[32:].sum(0)) / l
+    assert np.allclose(o[0, 0], expect, rtol=1e-5, atol=1e-9)
+
+
+def test_split_kv_quantizes_probabilities_per_split(ora):
+    """With one tile per split, the tiles after the sink's tile run their own
+    softmax (their max is 0, so p = 1 and P^ = 1.03125 p) and the merge
+    weights them by e^(0 - 10); l stays the unquantized sum."""
+    N = 300
+    l = 1.0 + (N - 1) * math.exp(-10.0)
+    o, v = _sink_case(ora, 0, 0, N, chunk=1)
+    tail = 6 * 2.0 ** -6 / 2048
+    expect = (1.03125 * v[0] + tail * v[16:128].sum(0) + 1.03125 * math.exp(-10.0) * v[128:].sum(0)) / l
+    assert np.allclose(o[0, 0], expect, rtol=1e-5, atol=1e-9)
+
+
+def test_quantized_probabilities_stay_close_on_random_data(ora):
+    """With FP4 P the output stays within a few percent of the exact-P output
+    (a sanity bound, not a pin of any constant)."""
+    rng = np.random.default_rng(9)
+    H_kv, G, d, N = 1, 4, 128, 700
+    q, k, v = _exact_case(rng, [N], G, H_kv, d)
+    q = q / 4
+    bt, num_pages, sm = _pages([N], rng)
+    ones = np.ones((H_kv, d), np.float32)
+    g = np.ones(H_kv, np.float32)
+    cache = ora.empty_cache(num_pages, H_kv, d, d, 0)
+    ora.quantize_kv(_bf16(k), _bf16(v), sm, cache, H_kv, 0, ones, g, g, num_pages, flags=ora.FLAG_NO_HADAMARD)
+    args = (_bf16(q), cache, bt, np.array([N]), H_kv, d, 0, ones, g, g, 0.05, 2, num_pages)
+    _, exact = ora.decode(*args, flags=ora.FLAG_NO_HADAMARD | ora.FLAG_EXACT_P)
+    _, quant = ora.decode(*args, flags=ora.FLAG_NO_HADAMARD)
+    rel = np.linalg.norm(quant - exact) / np.linalg.norm(exact)
+    assert 0 < rel < 0.1
