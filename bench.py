@@ -1,0 +1,385 @@
+"""Benchmark of the FP4 paged decode-attention step on B200.
+
+One step = one decode step of a serving batch through the whole hot path:
+append-quantize each sequence's open value block (its newest token and the
+earlier tokens of the same 16/32-slot block, kept in bf16 by the caller) into
+the paged FP4 cache, then decode attention for one query token per sequence
+(query transform + dual-residual FP4, paged tile fetch, QK^T, transposed
+softmax with fused underflow-aware P quantization, P.V, split merge).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config qwen3_4b]
+                  [--fmt nvfp4|mxfp4] [--impl ours|reference]
+
+`value` is KV tokens per second (sum of context lengths per step / step
+time), device-timed with CUDA events; under torchrun each rank runs its own
+batch (weak scaling) and rank 0 reports the whole job over the slowest rank.
+`--impl reference` times the CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+CONFIG_TEXT = {
+    "qwen3_4b": "Qwen3-4B-shaped layer decode: B=16, 32 query / 8 KV heads, d=128, context 32768 each, page 64, "
+                "shuffled block table",
+    "qwen3_30b_a3b": "Qwen3-30B-A3B-shaped layer decode: B=64, 32 query / 4 KV heads, d=128, context U[8192,131072], "
+                     "page 64",
+    "underflow": "long-context underflow stress: B=4, 32/8 heads, d=128, context 131072, keys N(0,0.05^2)",
+    "mla": "MLA-shaped decode: B=32, 128 heads over one latent head, d_k=576, d_v=512, context 16384",
+    "tiny": "tiny decode: B=1, 4/1 heads, d=128, context 1024",
+}
+
+
+def algorithmic_bytes(sp, seq_lens, fmt: int) -> int:
+    """Packed KV + scales + block table + Q and O in bf16 for one decode."""
+    beta = 16 if fmt == 0 else 32
+    tok = int(np.sum(seq_lens))
+    per_tok = sp.H_kv * (sp.d_k // 2 + sp.d_k // beta + sp.d_v // 2 + sp.d_v // beta)
+    pages = int(np.sum((np.asarray(seq_lens) + 63) // 64))
+    return tok * per_tok + pages * 4 + sp.B * sp.H_q * (sp.d_k + sp.d_v) * 2
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu, self.proc, self.path = gpu_index, None, None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "100"], stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def setup_ours(sp, fmt, rank, device):
+    """Untimed: draw the workload on the GPU, calibrate, prefill-quantize the cache."""
+    import torch
+
+    from fp4_kv_cache_quant_b200 import bdfp4
+    from fp4_kv_cache_quant_b200.workloads import Workload
+
+    wl = Workload(sp, seed=rank)
+    beta = 16 if fmt == 0 else 32
+    kc, qc, vc = wl.calibration(device)
+    kv = bdfp4.bdfp4_calibrate(kc, qc, vc, sp.H_q, sp.H_kv)
+    cache = bdfp4.FP4Cache.empty(wl.num_pages, sp.H_kv, sp.d_k, sp.d_v, fmt, device=device)
+    status = torch.zeros(1, dtype=torch.int32, device=device)
+    tails_k, tails_v, tails_sm = [], [], []
+    q_bytes = 0
+    t_quant, quant_bytes = 0.0, 0
+    for b in range(sp.B):
+        n = int(wl.seq_lens[b])
+        k = wl.keys(b, device)
+        v = wl.values(b, device)
+        sm = torch.from_numpy(wl.slot_mapping(b)).to(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        bdfp4.bdfp4_quantize_kv(k, v, sm, kv, cache, dev_status=status)
+        e1.record()
+        torch.cuda.synchronize()
+        t_quant += e0.elapsed_time(e1) / 1e3
+        quant_bytes += (k.numel() + v.numel()) * 2 + n * sp.H_kv * (sp.d_k // 2 + sp.d_k // beta + sp.d_v // 2 +
+                                                                  sp.d_v // beta)
+        # the open value block of the newest token, kept in bf16 for the next append
+        r = ((n - 1) % beta) + 1 if n > 0 else 0
+        tails_k.append(k[n - r:].clone())
+        tails_v.append(v[n - r:].clone())
+        tails_sm.append(sm[n - r:].clone())
+        del k, v
+    assert int(status.item()) == 0
+    tail_k = torch.cat(tails_k)
+    tail_v = torch.cat(tails_v)
+    tail_sm = torch.cat(tails_sm)
+    q = wl.queries(device)
+    bt = torch.from_numpy(wl.block_table).to(device)
+    sl = torch.from_numpy(wl.seq_lens).to(device)
+    num_sms = torch.cuda.get_device_properties(device).multi_processor_count
+    chunk = bdfp4.bdfp4_decode_plan(wl.seq_lens, sp.H_kv, num_sms)
+    ws = bdfp4.workspace_for(sp.B, sp.H_q, sp.d_v, wl.max_pages, chunk, device=device)
+    out = torch.empty((sp.B, sp.H_q, sp.d_v), dtype=torch.bfloat16, device=device)
+    return dict(wl=wl, kv=kv, cache=cache, status=status, tail_k=tail_k, tail_v=tail_v, tail_sm=tail_sm, q=q, bt=bt,
+                sl=sl, chunk=chunk, ws=ws, out=out, quant_gbs=quant_bytes / t_quant / 1e9, num_sms=num_sms)
+
+
+def run_ours(args, sp, fmt):
+    import torch
+    import torch.distributed as dist
+
+    from fp4_kv_cache_quant_b200 import bdfp4
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+
+    S = setup_ours(sp, fmt, rank, device)
+    wl, kv, cache = S["wl"], S["kv"], S["cache"]
+    stream = torch.cuda.current_stream(device)
+
+    def step(q):
+        bdfp4.bdfp4_quantize_kv(S["tail_k"], S["tail_v"], S["tail_sm"], kv, cache, dev_status=S["status"])
+        bdfp4.bdfp4_decode(q, cache, S["bt"], S["sl"], kv, sp.sm_scale, S["chunk"], S["ws"], S["out"],
+                           dev_status=S["status"])
+
+    for _ in range(max(args.warmup, 3)):
+        step(S["q"])
+    torch.cuda.synchronize()
+
+    # per-launch decode timing (events on the launching stream) inside the timed region
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        bdfp4.bdfp4_quantize_kv(S["tail_k"], S["tail_v"], S["tail_sm"], kv, cache, dev_status=S["status"])
+        ev[i][0].record(stream)
+        bdfp4.bdfp4_decode(S["q"], cache, S["bt"], S["sl"], kv, sp.sm_scale, S["chunk"], S["ws"], S["out"],
+                           dev_status=S["status"])
+        ev[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    step_s = t0.elapsed_time(t1) / 1e3 / args.steps
+    dec_s = statistics.mean(a.elapsed_time(b) for a, b in ev) / 1e3
+    assert int(S["status"].item()) == 0, "device status set"
+
+    # end to end through the C ABI with host buffers: H2D of q and the tail rows,
+    # D2H of the output, every step
+    q_host = S["q"].cpu().pin_memory()
+    tk_host = S["tail_k"].cpu().pin_memory()
+    tv_host = S["tail_v"].cpu().pin_memory()
+    out_host = torch.empty(S["out"].shape, dtype=S["out"].dtype).pin_memory()
+    q_dev = torch.empty_like(S["q"])
+    e2e_steps = max(3, args.steps // 2)
+    for it in range(2 + e2e_steps):
+        if it == 2:
+            torch.cuda.synchronize()
+            s0 = torch.cuda.Event(enable_timing=True)
+            s1 = torch.cuda.Event(enable_timing=True)
+            s0.record(stream)
+        q_dev.copy_(q_host, non_blocking=True)
+        S["tail_k"].copy_(tk_host, non_blocking=True)
+        S["tail_v"].copy_(tv_host, non_blocking=True)
+        step(q_dev)
+        out_host.copy_(S["out"], non_blocking=True)
+    s1.record(stream)
+    torch.cuda.synchronize()
+    e2e_s = s0.elapsed_time(s1) / 1e3 / e2e_steps
+
+    tokens = float(np.sum(wl.seq_lens))
+    if world > 1:
+        t = torch.tensor([step_s, dec_s, e2e_s], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        step_s, dec_s, e2e_s = t.tolist()
+        tokens *= world
+    launches_per_step = 2 + 1 + (1 if S["chunk"] < (wl.max_pages * 64 + 127) // 128 else 0)
+    alg = algorithmic_bytes(sp, wl.seq_lens, fmt)
+    peaks_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(peaks_path):
+        peak, peak_src = json.load(open(peaks_path))["hbm_gbs"], "measured"
+    else:
+        peak, peak_src = 6650.0, "fallback"
+    traffic = None
+    tr_path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    if os.path.exists(tr_path):
+        rec = json.load(open(tr_path)).get(f"{args.config}_{args.fmt}")
+        if rec:
+            traffic = rec.get("bytes_per_launch")
+    result = {
+        "metric": "FP4 paged decode-attn KV tokens/s",
+        "value": tokens / step_s,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": max(args.warmup, 3),
+        "ms_per_step": step_s * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "nvfp4" if fmt == 0 else "mxfp4",
+        "data": "synthetic (seeded N(0,1) bf16 with outlier key channels; calibrated smoothing)",
+        "config": {"workload": CONFIG_TEXT[args.config], "name": args.config, "fmt": args.fmt,
+                   "global_batch": sp.B * world, "seq_len": int(np.max(wl.seq_lens)),
+                   "kv_tokens_per_step_per_gpu": int(tokens / world), "chunk_tiles": S["chunk"],
+                   "parallelism": f"replicas x{world} (no data-path collective)",
+                   "l2": f"inputs larger than L2 (FP4 cache {cache.nbytes() / 1e6:.0f} MB per GPU)",
+                   "accumulate": "fp32"},
+        "hbm_gbs": alg / dec_s / 1e9,
+        "decode_us": dec_s * 1e6,
+        "quantize_prefill_gbs": S["quant_gbs"],
+        "roofline": {"bound": "hbm", "achieved": alg / dec_s / 1e9, "peak": peak, "unit": "GB/s",
+                     "frac": alg / dec_s / 1e9 / peak, "traffic": traffic,
+                     "kernel": "decode_fp4_kernel + merge_splits_kernel (events bracket both)",
+                     "peak_source": f"{peak_src} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                     "algorithmic_bytes_per_launch": alg},
+        "e2e": {"value": tokens / e2e_s, "unit": "tokens/s",
+                "h2d_bytes_per_step": int(q_host.numel() * 2 + tk_host.numel() * 2 + tv_host.numel() * 2),
+                "d2h_bytes_per_step": int(out_host.numel() * 2)},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(sp, fmt, budget_s=args.cpu_budget)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def cpu_baseline(sp, fmt, budget_s: float = 15.0, seed: int = 0) -> dict:
+    """The oracle as it stands, timed on this host's cores on a bounded sample
+    of the same workload: decode (with the tail append) of the first few
+    sequences; prefill of the sample is untimed setup."""
+    import oracle
+    from fp4_kv_cache_quant_b200.workloads import Workload
+
+    wl = Workload(sp, seed=seed)
+    beta = 16 if fmt == 0 else 32
+    kc, qc, vc = wl.calibration("cpu")
+    smooth, kg, vg = oracle.calibrate(kc, qc, vc, sp.H_q, sp.H_kv)
+    q_all = wl.queries("cpu")
+    done_tokens, elapsed, nseq = 0, 0.0, 0
+    for b in range(sp.B):
+        n = int(wl.seq_lens[b])
+        k, v = wl.keys(b), wl.values(b)
+        sm = wl.slot_mapping(b)
+        cache = oracle.empty_cache(wl.num_pages, sp.H_kv, sp.d_k, sp.d_v, fmt)
+        oracle.quantize_kv(k, v, sm, cache, sp.H_kv, fmt, smooth, kg, vg, wl.num_pages)
+        r = ((n - 1) % beta) + 1
+        t0 = time.perf_counter()
+        oracle.quantize_kv(k[n - r:], v[n - r:], sm[n - r:], cache, sp.H_kv, fmt, smooth, kg, vg, wl.num_pages)
+        oracle.decode(q_all[b:b + 1], cache, wl.block_table[b:b + 1], wl.seq_lens[b:b + 1], sp.H_kv, sp.d_v, fmt,
+                      smooth, kg, vg, sp.sm_scale, 1 << 20, wl.num_pages)
+        elapsed += time.perf_counter() - t0
+        done_tokens += n
+        nseq += 1
+        if elapsed >= budget_s:
+            break
+    return {"value": done_tokens / elapsed, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{nseq} of {sp.B} sequences ({done_tokens} KV tokens, all heads): tail append + decode, "
+                      f"{elapsed:.1f} s"}
+
+
+def run_reference(args, sp, fmt):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    from fp4_kv_cache_quant_b200.workloads import Workload
+
+    wl = Workload(sp, seed=0)
+    beta = 16 if fmt == 0 else 32
+    kc, qc, vc = wl.calibration("cpu")
+    smooth, kg, vg = oracle.calibrate(kc, qc, vc, sp.H_q, sp.H_kv)
+    q_all = wl.queries("cpu")
+    # bounded sample per step: one sequence, its tail append and its decode
+    b = 0
+    n = int(wl.seq_lens[b])
+    k, v = wl.keys(b), wl.values(b)
+    sm = wl.slot_mapping(b)
+    cache = oracle.empty_cache(wl.num_pages, sp.H_kv, sp.d_k, sp.d_v, fmt)
+    oracle.quantize_kv(k, v, sm, cache, sp.H_kv, fmt, smooth, kg, vg, wl.num_pages)
+    r = ((n - 1) % beta) + 1
+
+    def step():
+        oracle.quantize_kv(k[n - r:], v[n - r:], sm[n - r:], cache, sp.H_kv, fmt, smooth, kg, vg, wl.num_pages)
+        oracle.decode(q_all[b:b + 1], cache, wl.block_table[b:b + 1], wl.seq_lens[b:b + 1], sp.H_kv, sp.d_v, fmt,
+                      smooth, kg, vg, sp.sm_scale, 1 << 20, wl.num_pages)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = (time.perf_counter() - t0) / args.steps
+    val = n / el
+    print(json.dumps({
+        "impl": "reference", "metric": "FP4 paged decode-attn KV tokens/s", "value": val, "unit": "tokens/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": el * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": CONFIG_TEXT[args.config], "name": args.config, "fmt": args.fmt},
+        "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": f"sequence 0 of {sp.B} ({n} KV tokens, all heads) per step: tail append + decode"},
+        "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="qwen3_4b", choices=list(CONFIG_TEXT))
+    ap.add_argument("--fmt", default="nvfp4", choices=["nvfp4", "mxfp4"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    from fp4_kv_cache_quant_b200.workloads import spec
+    sp = spec(args.config)
+    fmt = 0 if args.fmt == "nvfp4" else 1
+    if args.impl == "reference":
+        run_reference(args, sp, fmt)
+    else:
+        run_ours(args, sp, fmt)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,207 @@
+"""Thin ctypes binding of the bdfp4 C ABI (include/bdfp4.h).
+
+Argument marshalling only: every step of the path runs in libbdfp4.so's CUDA
+kernels.  torch provides device memory and streams.  The library is loaded
+from this package's directory; importing this module on a machine where it
+is missing raises, there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libbdfp4.so")
+
+NVFP4, MXFP4 = 0, 1
+FLAG_NO_HADAMARD = 1
+FLAG_NO_SCALE_SEARCH = 2
+FLAG_SINGLE_QUERY = 4
+FLAG_NO_UNDERFLOW = 8
+
+DEV_BAD_PAGE, DEV_BAD_SEQLEN, DEV_BAD_SLOT = 1, 2, 4
+
+PAGE_SLOTS = 64
+TILE_TOKENS = 128
+
+#: names of every entry point declared in include/bdfp4.h
+ENTRY_POINTS = ("bdfp4_calibrate", "bdfp4_quantize_kv", "bdfp4_quantize_q", "bdfp4_decode_plan",
+                "bdfp4_decode_workspace_size", "bdfp4_decode", "bdfp4_status_string")
+
+
+class BDFP4Error(RuntimeError):
+    pass
+
+
+class _KVParams(ctypes.Structure):
+    _fields_ = [("smooth", ctypes.c_void_p), ("k_gscale", ctypes.c_void_p), ("v_gscale", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libbdfp4.so (raises OSError if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise OSError(f"{LIB_PATH} is missing: build it with `python -m fp4_kv_cache_quant_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    i, i64, p, f, sz = ctypes.c_int, ctypes.c_int64, ctypes.c_void_p, ctypes.c_float, ctypes.c_size_t
+    kvp = ctypes.POINTER(_KVParams)
+    L.bdfp4_calibrate.argtypes = [p, p, p, i, i, i, i, i, i, i, p, p, p, p]
+    L.bdfp4_calibrate.restype = i
+    L.bdfp4_quantize_kv.argtypes = [p, p, p, i, i, i, i, i, i, kvp, p, p, p, p, i64, p, p]
+    L.bdfp4_quantize_kv.restype = i
+    L.bdfp4_quantize_q.argtypes = [p, i, i, i, i, i, i, p, p, p, p, p, p, p]
+    L.bdfp4_quantize_q.restype = i
+    L.bdfp4_decode_plan.argtypes = [p, i, i, i]
+    L.bdfp4_decode_plan.restype = i
+    L.bdfp4_decode_workspace_size.argtypes = [i, i, i, i, i]
+    L.bdfp4_decode_workspace_size.restype = sz
+    L.bdfp4_decode.argtypes = [p, p, p, p, p, p, p, i, i, i, i, i, i, i64, i, i, kvp, f, i, p, sz, p, p, p]
+    L.bdfp4_decode.restype = i
+    L.bdfp4_status_string.argtypes = [i]
+    L.bdfp4_status_string.restype = ctypes.c_char_p
+    _lib = L
+    return L
+
+
+def bdfp4_status_string(status: int) -> str:
+    return load().bdfp4_status_string(int(status)).decode()
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise BDFP4Error(f"{what}: {bdfp4_status_string(rc)} ({rc})")
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    assert t.is_contiguous(), "tensors passed to bdfp4 must be contiguous"
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def beta(fmt: int) -> int:
+    return 16 if fmt == NVFP4 else 32
+
+
+@dataclass
+class KVParams:
+    """Static per-layer parameters: smoothing factors and FP32 tensor scales."""
+    smooth: torch.Tensor    # [H_kv, d_k] fp32
+    k_gscale: torch.Tensor  # [H_kv] fp32
+    v_gscale: torch.Tensor  # [H_kv] fp32
+
+    def _c(self) -> _KVParams:
+        return _KVParams(self.smooth.data_ptr(), self.k_gscale.data_ptr(), self.v_gscale.data_ptr())
+
+
+@dataclass
+class FP4Cache:
+    """The paged FP4 KV cache arrays (layout in include/bdfp4.h)."""
+    k_pages: torch.Tensor
+    k_scales: torch.Tensor
+    v_pages: torch.Tensor
+    v_scales: torch.Tensor
+    num_pages: int
+    H_kv: int
+    d_k: int
+    d_v: int
+    fmt: int
+
+    @staticmethod
+    def empty(num_pages: int, H_kv: int, d_k: int, d_v: int, fmt: int, device="cuda") -> "FP4Cache":
+        b = beta(fmt)
+        mk = lambda n: torch.zeros(n, dtype=torch.uint8, device=device)  # noqa: E731
+        return FP4Cache(mk(num_pages * H_kv * PAGE_SLOTS * d_k // 2), mk(num_pages * H_kv * PAGE_SLOTS * d_k // b),
+                        mk(num_pages * H_kv * d_v * PAGE_SLOTS // 2), mk(num_pages * H_kv * d_v * PAGE_SLOTS // b),
+                        num_pages, H_kv, d_k, d_v, fmt)
+
+    def nbytes(self) -> int:
+        return sum(t.numel() for t in (self.k_pages, self.k_scales, self.v_pages, self.v_scales))
+
+
+def bdfp4_calibrate(k_cal: torch.Tensor, q_cal: torch.Tensor, v_cal: torch.Tensor, H_q: int, H_kv: int,
+                    flags: int = 0, stream=None) -> KVParams:
+    Tc, _, d_k = k_cal.shape
+    d_v = v_cal.shape[2]
+    dev = k_cal.device
+    kv = KVParams(torch.empty((H_kv, d_k), dtype=torch.float32, device=dev),
+                  torch.empty(H_kv, dtype=torch.float32, device=dev), torch.empty(H_kv, dtype=torch.float32, device=dev))
+    rc = load().bdfp4_calibrate(_ptr(k_cal), _ptr(q_cal), _ptr(v_cal), Tc, q_cal.shape[0], H_q, H_kv, d_k, d_v, flags,
+                                _ptr(kv.smooth), _ptr(kv.k_gscale), _ptr(kv.v_gscale), _stream(stream))
+    _check(rc, "bdfp4_calibrate")
+    return kv
+
+
+def bdfp4_quantize_kv(k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor, kv: KVParams, cache: FP4Cache,
+                      flags: int = 0, dev_status: torch.Tensor | None = None, stream=None) -> None:
+    T = k.shape[0]
+    c = kv._c()
+    rc = load().bdfp4_quantize_kv(_ptr(k), _ptr(v), _ptr(slot_mapping), T, cache.H_kv, cache.d_k, cache.d_v,
+                                  cache.fmt, flags, ctypes.byref(c), _ptr(cache.k_pages), _ptr(cache.k_scales),
+                                  _ptr(cache.v_pages), _ptr(cache.v_scales), cache.num_pages, _ptr(dev_status),
+                                  _stream(stream))
+    _check(rc, "bdfp4_quantize_kv")
+
+
+def bdfp4_quantize_q(q: torch.Tensor, H_kv: int, fmt: int, smooth: torch.Tensor, flags: int = 0,
+                     stream=None) -> dict:
+    B, H_q, d_k = q.shape
+    nb = d_k // beta(fmt)
+    dev = q.device
+    out = dict(q1_codes=torch.empty((B, H_q, d_k), dtype=torch.uint8, device=dev),
+               q1_scales=torch.empty((B, H_q, nb), dtype=torch.uint8, device=dev),
+               q2_codes=torch.empty((B, H_q, d_k), dtype=torch.uint8, device=dev),
+               q2_scales=torch.empty((B, H_q, nb), dtype=torch.uint8, device=dev),
+               g_q=torch.empty((B, H_q), dtype=torch.float32, device=dev))
+    rc = load().bdfp4_quantize_q(_ptr(q), B, H_q, H_kv, d_k, fmt, flags, _ptr(smooth), _ptr(out["q1_codes"]),
+                                 _ptr(out["q1_scales"]), _ptr(out["q2_codes"]), _ptr(out["q2_scales"]),
+                                 _ptr(out["g_q"]), _stream(stream))
+    _check(rc, "bdfp4_quantize_q")
+    return out
+
+
+def bdfp4_decode_plan(host_seq_lens, H_kv: int, num_sms: int) -> int:
+    import numpy as np
+    sl = np.ascontiguousarray(host_seq_lens, dtype=np.int32)
+    rc = load().bdfp4_decode_plan(ctypes.c_void_p(sl.ctypes.data), sl.shape[0], H_kv, num_sms)
+    if rc < 0:
+        _check(rc, "bdfp4_decode_plan")
+    return rc
+
+
+def bdfp4_decode_workspace_size(B: int, H_q: int, d_v: int, max_pages_per_seq: int, chunk_tiles: int) -> int:
+    return int(load().bdfp4_decode_workspace_size(B, H_q, d_v, max_pages_per_seq, chunk_tiles))
+
+
+def bdfp4_decode(q: torch.Tensor, cache: FP4Cache, block_table: torch.Tensor, seq_lens: torch.Tensor, kv: KVParams,
+                 sm_scale: float, chunk_tiles: int, workspace: torch.Tensor | None, out: torch.Tensor,
+                 flags: int = 0, dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    B, H_q, d_k = q.shape
+    c = kv._c()
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = load().bdfp4_decode(_ptr(q), _ptr(cache.k_pages), _ptr(cache.k_scales), _ptr(cache.v_pages),
+                             _ptr(cache.v_scales), _ptr(block_table), _ptr(seq_lens), B, H_q, cache.H_kv, d_k,
+                             cache.d_v, block_table.shape[1], cache.num_pages, cache.fmt, flags, ctypes.byref(c),
+                             float(sm_scale), int(chunk_tiles), _ptr(workspace), ws_bytes, _ptr(out),
+                             _ptr(dev_status), _stream(stream))
+    _check(rc, "bdfp4_decode")
+    return out
+
+
+def workspace_for(B: int, H_q: int, d_v: int, max_pages_per_seq: int, chunk_tiles: int, device="cuda"):
+    n = bdfp4_decode_workspace_size(B, H_q, d_v, max_pages_per_seq, chunk_tiles)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)

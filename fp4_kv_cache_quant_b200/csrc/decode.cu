@@ -1,0 +1,469 @@
+// decode.cu -- FP4 paged decode attention with split-KV and a log-sum-exp
+// merge (BitDecoding-FP4, Article Summary: dual-residual query, transposed
+// softmax with fused, underflow-aware probability quantization, paged KV).
+//
+// One CTA of 128 threads per (sequence, KV head, head chunk, split).  The
+// softmax is transposed: thread t owns token t of the current 128-token tile
+// (two pages) for every query head of the group, so row maxima and sums are
+// warp-shuffle reductions, and the FP4 quantization of the probabilities
+// (beta-token blocks) is a 4- or 5-step shuffle max inside the owning lanes.
+// For P.V the threads switch to owning value channels, reading each page's
+// channel-major FP4 block with 16-byte loads.
+
+#include <algorithm>
+
+#include "bdfp4_device.cuh"
+#include "host_common.h"
+#include "quant_device.cuh"
+
+namespace bdfp4 {
+
+struct DecodeArgs {
+    const __nv_bfloat16* q;
+    const uint8_t* k_pages;
+    const uint8_t* k_scales;
+    const uint8_t* v_pages;
+    const uint8_t* v_scales;
+    const int32_t* block_table;
+    const int32_t* seq_lens;
+    const float* smooth;
+    const float* k_gscale;
+    const float* v_gscale;
+    float* ws_o;   // [B][H_q][max_splits][d_v] unnormalised partial outputs
+    float* ws_ml;  // [B][H_q][max_splits][2]  (m in log2 units, l)
+    __nv_bfloat16* out;
+    int32_t* dev_status;
+    int B, H_q, H_kv, max_pages, flags, chunk_tiles, max_splits;
+    int64_t num_pages;
+    float sm_scale;
+};
+
+constexpr int kThreads = 128;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Splits of a sequence of N tokens.
+__host__ __device__ __forceinline__ int num_splits(int N, int chunk_tiles) {
+    const int ntiles = (N + kTileTokens - 1) / kTileTokens;
+    return (ntiles + chunk_tiles - 1) / chunk_tiles;
+}
+
+template <int FMT, int DK, int DV, int HG>
+__global__ void __launch_bounds__(kThreads) decode_fp4_kernel(const DecodeArgs a) {
+    constexpr int B = Fmt<FMT>::beta;
+    constexpr int NCH = DV / kThreads;   // value channels per thread
+    using RG = RowGeom<FMT, DK>;
+
+    __shared__ __align__(16) float dq[HG][DK];            // dequantized q1 + q2 (scale values, no g)
+    __shared__ __align__(16) float ph[HG][kTileTokens];   // quantized probabilities (times alpha)
+    __shared__ float2 lut[256];                            // E2M1 byte -> (low, high) values
+    __shared__ float red[4][HG];
+    __shared__ float lsc[HG];                              // sm_scale g_q g_k log2(e)
+    __shared__ int row_amax[kThreads];
+    __shared__ int pages[2];
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int split = blockIdx.x;
+    const int G = a.H_q / a.H_kv;
+    const int chunks = G / HG;
+    const int hk = blockIdx.y / chunks;
+    const int h0 = hk * G + (blockIdx.y % chunks) * HG;   // first query head of this CTA
+    const int b = blockIdx.z;
+
+    int N = a.seq_lens[b];
+    if (N < 0 || N > a.max_pages * kPageSlots) {
+        if (tid == 0 && split == 0) set_status(a.dev_status, BDFP4_DEV_BAD_SEQLEN);
+        N = 0;
+    }
+    const int ntiles = (N + kTileTokens - 1) / kTileTokens;
+    const int nspl = (ntiles + a.chunk_tiles - 1) / a.chunk_tiles;
+    if (split > 0 && split >= nspl) return;
+    if (N == 0) {  // empty sequence: zeros
+        for (int i = tid; i < HG * DV; i += kThreads)
+            a.out[((int64_t)b * a.H_q + h0 + i / DV) * DV + i % DV] = __float2bfloat16(0.0f);
+        return;
+    }
+
+    // ---------------------------------------------------------------- prologue
+    for (uint32_t by = tid; by < 256u; by += kThreads) lut[by] = make_float2(e2m1_value(by & 15u), e2m1_value(by >> 4));
+    const bool hadamard = !(a.flags & BDFP4_FLAG_NO_HADAMARD);
+    const bool dual = !(a.flags & BDFP4_FLAG_SINGLE_QUERY);
+    constexpr int rows_per_pass = kThreads / RG::rt;
+    for (int r0 = 0; r0 < HG; r0 += rows_per_pass) {
+        const int j = tid % RG::rt, rl = tid / RG::rt, r = r0 + rl;
+        const bool active = r < HG && j < RG::tpr;
+        row_amax[tid] = 0;
+        float x[B];
+        if (active) {
+            load_bf16_block<B>(a.q + ((int64_t)b * a.H_q + h0 + r) * DK, j * B, x);
+        } else {
+#pragma unroll
+            for (int i = 0; i < B; ++i) x[i] = 0.0f;
+        }
+        transform_block<FMT, DK, false>(x, a.smooth + (int64_t)hk * DK, j, hadamard);
+        __syncthreads();
+        if (active) atomicMax(&row_amax[rl], __float_as_int(block_amax<B>(x)));
+        __syncthreads();
+        if (active) {
+            const float amax = __int_as_float(row_amax[rl]);
+            const float gq = FMT == BDFP4_NVFP4 ? (amax > 0.0f ? __fdiv_rn(amax, 2688.0f) : 1.0f) : 1.0f;
+            uint32_t c1, c2, p1[B / 8], p2[B / 8];
+            quantize_query_block<FMT, DK>(x, gq, dual, c1, p1, c2, p2);
+            const float s1 = scale_value<FMT>(c1), s2 = scale_value<FMT>(c2);
+#pragma unroll
+            for (int i = 0; i < B; ++i) {
+                const uint32_t e1 = (p1[i / 8] >> (4 * (i % 8))) & 15u, e2 = (p2[i / 8] >> (4 * (i % 8))) & 15u;
+                dq[r][j * B + i] = e2m1_value(e1) * s1 + e2m1_value(e2) * s2;
+            }
+            if (j == 0) {
+                const float gk = FMT == BDFP4_NVFP4 ? a.k_gscale[hk] : 1.0f;
+                lsc[r] = a.sm_scale * gq * gk * kLog2e;
+            }
+        }
+        __syncthreads();
+    }
+
+    const float alpha = (FMT == BDFP4_NVFP4 && !(a.flags & BDFP4_FLAG_NO_UNDERFLOW)) ? kAlphaNV : 1.0f;
+    const float vg = FMT == BDFP4_NVFP4 ? a.v_gscale[hk] : 1.0f;
+    const int64_t kv_stride_k = (int64_t)kPageSlots * DK / 2, kv_stride_ks = (int64_t)kPageSlots * DK / B;
+    const int64_t kv_stride_v = (int64_t)DV * kPageSlots / 2, kv_stride_vs = (int64_t)DV * kPageSlots / B;
+
+    float m_run[HG], l_part[HG], o[HG][NCH];
+#pragma unroll
+    for (int g = 0; g < HG; ++g) {
+        m_run[g] = -INFINITY;
+        l_part[g] = 0.0f;
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) o[g][c] = 0.0f;
+    }
+
+    const int tile0 = split * a.chunk_tiles;
+    const int tile1 = min(tile0 + a.chunk_tiles, ntiles);
+    for (int tile = tile0; tile < tile1; ++tile) {
+        // ------------------------------------------------ logits (thread = token)
+        const int token = tile * kTileTokens + tid;
+        bool valid = token < N;
+        float s[HG];
+#pragma unroll
+        for (int g = 0; g < HG; ++g) s[g] = -INFINITY;
+        if (tid < 2) {
+            int pg = -1;
+            const int pi = tile * 2 + tid;
+            if (pi * kPageSlots < N) {
+                pg = a.block_table[(int64_t)b * a.max_pages + pi];
+                if (pg < 0 || pg >= a.num_pages) {
+                    set_status(a.dev_status, BDFP4_DEV_BAD_PAGE);
+                    pg = -1;
+                }
+            }
+            pages[tid] = pg;
+        }
+        __syncthreads();
+        const int page = pages[tid >> 6];
+        valid = valid && page >= 0;
+        if (valid) {
+            const int slot = tid & 63;
+            const uint8_t* kp = a.k_pages + ((int64_t)page * a.H_kv + hk) * kv_stride_k;
+            const uint8_t* ks = a.k_scales + ((int64_t)page * a.H_kv + hk) * kv_stride_ks;
+            float acc[HG];
+#pragma unroll
+            for (int g = 0; g < HG; ++g) acc[g] = 0.0f;
+#pragma unroll 2
+            for (int kc = 0; kc < DK / 32; ++kc) {
+                const uint4 w = __ldg(reinterpret_cast<const uint4*>(kp + k_nib_offset(DK, slot, kc * 32)));
+                const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int half = 0; half < 32 / B; ++half) {
+                    const int blk = (kc * 32) / B + half;
+                    const float sc = scale_value<FMT>(__ldg(ks + k_scale_offset<B>(DK, slot, blk)));
+#pragma unroll
+                    for (int wi = 0; wi < B / 8; ++wi) {
+                        const uint32_t word = words[half * (B / 8) + wi];
+#pragma unroll
+                        for (int by = 0; by < 4; ++by) {
+                            const float2 v2 = lut[(word >> (8 * by)) & 0xffu];
+                            const int e = kc * 32 + half * B + wi * 8 + by * 2;
+                            const float k0 = v2.x * sc, k1 = v2.y * sc;
+#pragma unroll
+                            for (int g = 0; g < HG; ++g) {
+                                const float2 qq = *reinterpret_cast<const float2*>(&dq[g][e]);
+                                acc[g] = fmaf(qq.x, k0, acc[g]);
+                                acc[g] = fmaf(qq.y, k1, acc[g]);
+                            }
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int g = 0; g < HG; ++g) s[g] = acc[g] * lsc[g];
+        }
+        // ------------------------------------------------ transposed online softmax
+        float p[HG], corr[HG];
+#pragma unroll
+        for (int g = 0; g < HG; ++g) {
+            float mx = s[g];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            if (lane == 0) red[warp][g] = mx;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int g = 0; g < HG; ++g) {
+            const float mt = fmaxf(fmaxf(red[0][g], red[1][g]), fmaxf(red[2][g], red[3][g]));
+            const float mn = fmaxf(m_run[g], mt);
+            corr[g] = exp2f(m_run[g] - mn);   // 0 on the split's first tile
+            m_run[g] = mn;
+            p[g] = valid ? exp2f(s[g] - mn) : 0.0f;
+            l_part[g] = l_part[g] * corr[g] + p[g];
+            // fused probability quantization over beta-token blocks of lanes
+            const float y = p[g] * alpha;
+            float am = y;
+#pragma unroll
+            for (int off = B / 2; off > 0; off >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
+            float sigma;
+            if constexpr (FMT == BDFP4_NVFP4) {
+                sigma = am > 0.0f ? e4m3_value(e4m3_encode(__fdiv_rn(am, 6.0f))) : 0.0f;
+            } else {
+                sigma = e8m0_value(mx_scale_code(am));
+            }
+            const uint32_t e = sigma > 0.0f ? e2m1_encode(__fdiv_rn(y, sigma)) : 0u;
+            ph[g][tid] = e2m1_value(e) * sigma;
+        }
+        __syncthreads();
+        // ------------------------------------------------ P.V (thread = value channel)
+#pragma unroll
+        for (int g = 0; g < HG; ++g)
+#pragma unroll
+            for (int c = 0; c < NCH; ++c) o[g][c] *= corr[g];
+        const int n_valid = min(kTileTokens, N - tile * kTileTokens);
+#pragma unroll
+        for (int pp = 0; pp < 2; ++pp) {
+            const int pg = pages[pp];
+            const int nv = min(kPageSlots, n_valid - pp * kPageSlots);
+            if (pg < 0 || nv <= 0) continue;
+            const uint8_t* vp = a.v_pages + ((int64_t)pg * a.H_kv + hk) * kv_stride_v;
+            const uint8_t* vs = a.v_scales + ((int64_t)pg * a.H_kv + hk) * kv_stride_vs;
+#pragma unroll
+            for (int c = 0; c < NCH; ++c) {
+                const int ch = tid + c * kThreads;
+#pragma unroll
+                for (int kc = 0; kc < 2; ++kc) {
+                    const uint4 w = __ldg(reinterpret_cast<const uint4*>(vp + v_nib_offset(ch, kc * 32)));
+                    const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int wi = 0; wi < 4; ++wi) {
+#pragma unroll
+                        for (int by = 0; by < 4; ++by) {
+                            const int sl = kc * 32 + wi * 8 + by * 2;   // slot of the low nibble
+                            if (sl >= nv) continue;                      // masked slots: select, never multiply
+                            const float sc = scale_value<FMT>(__ldg(vs + v_scale_offset<B>(ch, sl / B)));
+                            const float2 v2 = lut[(words[wi] >> (8 * by)) & 0xffu];
+                            const float v0 = v2.x * sc;
+                            const float v1 = (sl + 1 < nv) ? v2.y * sc : 0.0f;
+                            const int tt = pp * kPageSlots + sl;
+#pragma unroll
+                            for (int g = 0; g < HG; ++g) {
+                                const float2 pq = *reinterpret_cast<const float2*>(&ph[g][tt]);
+                                o[g][c] = fmaf(pq.x, v0, o[g][c]);
+                                o[g][c] = fmaf(pq.y, v1, o[g][c]);
+                            }
+                        }
+                    }
+                }
+            }
+        }
+        __syncthreads();
+    }
+
+    // ---------------------------------------------------------------- epilogue
+    // l = sum over the tile threads of their partial sums (warp shuffle + smem)
+    __shared__ float lsum[4][HG];
+#pragma unroll
+    for (int g = 0; g < HG; ++g) {
+        float v = l_part[g];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        if (lane == 0) lsum[warp][g] = v;
+    }
+    __syncthreads();
+    const float oscale = vg / alpha;
+    const bool single = nspl == 1;
+#pragma unroll
+    for (int g = 0; g < HG; ++g) {
+        const float l = lsum[0][g] + lsum[1][g] + lsum[2][g] + lsum[3][g];
+        const int64_t row = (int64_t)b * a.H_q + h0 + g;
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+            const int ch = tid + c * kThreads;
+            if (single) {
+                a.out[row * DV + ch] = __float2bfloat16(l > 0.0f ? o[g][c] * oscale / l : 0.0f);
+            } else {
+                a.ws_o[(row * a.max_splits + split) * DV + ch] = o[g][c] * oscale;
+            }
+        }
+        if (!single && tid == 0) {
+            a.ws_ml[(row * a.max_splits + split) * 2 + 0] = m_run[g];
+            a.ws_ml[(row * a.max_splits + split) * 2 + 1] = l;
+        }
+    }
+}
+
+// Log-sum-exp merge of the splits of one (sequence, query head); m in log2 units.
+template <int DV>
+__global__ void __launch_bounds__(128) merge_splits_kernel(const float* __restrict__ ws_o,
+                                                           const float* __restrict__ ws_ml,
+                                                           const int32_t* __restrict__ seq_lens, int H_q,
+                                                           int max_pages, int chunk_tiles, int max_splits,
+                                                           __nv_bfloat16* out) {
+    const int row = blockIdx.x;
+    const int b = row / H_q;
+    int N = seq_lens[b];
+    if (N < 0 || N > max_pages * kPageSlots) N = 0;
+    const int ns = num_splits(N, chunk_tiles);
+    if (ns <= 1) return;   // written by the decode kernel
+    float M = -INFINITY;
+    for (int s = 0; s < ns; ++s) M = fmaxf(M, ws_ml[((int64_t)row * max_splits + s) * 2]);
+    float L = 0.0f;
+    for (int s = 0; s < ns; ++s) {
+        const float* ml = ws_ml + ((int64_t)row * max_splits + s) * 2;
+        L += ml[1] * exp2f(ml[0] - M);
+    }
+    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+    for (int c = threadIdx.x; c < DV; c += blockDim.x) {
+        float acc = 0.0f;
+        for (int s = 0; s < ns; ++s)
+            acc += ws_o[((int64_t)row * max_splits + s) * DV + c] * exp2f(ws_ml[((int64_t)row * max_splits + s) * 2] - M);
+        out[(int64_t)row * DV + c] = __float2bfloat16(acc * inv);
+    }
+}
+
+}  // namespace bdfp4
+
+using namespace bdfp4;
+
+static int max_splits_for(int max_pages, int chunk_tiles) {
+    const int ntiles = (max_pages * kPageSlots + kTileTokens - 1) / kTileTokens;
+    return std::max(1, (ntiles + chunk_tiles - 1) / chunk_tiles);
+}
+
+extern "C" size_t bdfp4_decode_workspace_size(int B, int H_q, int d_v, int max_pages_per_seq, int chunk_tiles) {
+    if (B <= 0 || H_q <= 0 || d_v <= 0 || max_pages_per_seq <= 0 || chunk_tiles <= 0) return 0;
+    const size_t ms = (size_t)max_splits_for(max_pages_per_seq, chunk_tiles);
+    const size_t o_bytes = (size_t)B * H_q * ms * d_v * sizeof(float);
+    const size_t ml_bytes = (size_t)B * H_q * ms * 2 * sizeof(float);
+    return ((o_bytes + 255) / 256) * 256 + ml_bytes;
+}
+
+extern "C" int bdfp4_decode_plan(const int32_t* host_seq_lens, int B, int H_kv, int num_sms) {
+    if (!host_seq_lens || B <= 0 || H_kv <= 0 || num_sms <= 0) return BDFP4_ERR_ARG;
+    int64_t total_tiles = 0;
+    int max_tiles = 1;
+    for (int b = 0; b < B; ++b) {
+        const int n = host_seq_lens[b] > 0 ? host_seq_lens[b] : 0;
+        const int t = (n + kTileTokens - 1) / kTileTokens;
+        total_tiles += (int64_t)t * H_kv;
+        max_tiles = std::max(max_tiles, t);
+    }
+    // about 16 work items per SM keeps the tail short; at least 4 tiles per
+    // split keeps the merge traffic small next to the KV bytes
+    int64_t chunk = (total_tiles + 16LL * num_sms - 1) / (16LL * num_sms);
+    chunk = std::max<int64_t>(chunk, 4);
+    chunk = std::min<int64_t>(chunk, max_tiles);
+    return (int)std::max<int64_t>(chunk, 1);
+}
+
+template <int FMT, int DK, int DV>
+static int launch_decode(const DecodeArgs& a, int G, cudaStream_t st) {
+    int hg = G >= 16 ? 16 : G;
+    dim3 grid(a.max_splits, a.H_kv * (G / hg), a.B);
+    switch (hg) {
+        case 1: decode_fp4_kernel<FMT, DK, DV, 1><<<grid, kThreads, 0, st>>>(a); break;
+        case 2: decode_fp4_kernel<FMT, DK, DV, 2><<<grid, kThreads, 0, st>>>(a); break;
+        case 4: decode_fp4_kernel<FMT, DK, DV, 4><<<grid, kThreads, 0, st>>>(a); break;
+        case 8: decode_fp4_kernel<FMT, DK, DV, 8><<<grid, kThreads, 0, st>>>(a); break;
+        case 16: decode_fp4_kernel<FMT, DK, DV, 16><<<grid, kThreads, 0, st>>>(a); break;
+        default: return BDFP4_ERR_UNSUPPORTED;
+    }
+    if (a.max_splits > 1)
+        merge_splits_kernel<DV><<<a.B * a.H_q, 128, 0, st>>>(a.ws_o, a.ws_ml, a.seq_lens, a.H_q, a.max_pages,
+                                                             a.chunk_tiles, a.max_splits, a.out);
+    return launch_status();
+}
+
+extern "C" int bdfp4_decode(const void* q, const void* k_pages, const void* k_scales, const void* v_pages,
+                            const void* v_scales, const int32_t* block_table, const int32_t* seq_lens, int B, int H_q,
+                            int H_kv, int d_k, int d_v, int max_pages_per_seq, int64_t num_pages, bdfp4_fmt fmt,
+                            int flags, const bdfp4_kv_params* kv, float sm_scale, int chunk_tiles, void* workspace,
+                            size_t workspace_bytes, void* out, int32_t* dev_status, void* stream) {
+    if (B < 0 || H_q <= 0 || H_kv <= 0 || max_pages_per_seq <= 0 || num_pages < 0) return BDFP4_ERR_ARG;
+    if (fmt != BDFP4_NVFP4 && fmt != BDFP4_MXFP4) return BDFP4_ERR_ARG;
+    if (H_q % H_kv) return BDFP4_ERR_SHAPE;
+    if (!supported_dims(d_k, d_v)) return BDFP4_ERR_UNSUPPORTED;
+    const int G = H_q / H_kv;
+    if (G > 16 ? (G % 16 != 0 || G > 128) : (G & (G - 1)) != 0) return BDFP4_ERR_UNSUPPORTED;
+    if (B == 0) return BDFP4_OK;
+    if (!q || !k_pages || !k_scales || !v_pages || !v_scales || !block_table || !seq_lens || !out || !kv ||
+        !kv->smooth)
+        return BDFP4_ERR_ARG;
+    if (fmt == BDFP4_NVFP4 && (!kv->k_gscale || !kv->v_gscale)) return BDFP4_ERR_ARG;
+    if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_pages, 128) || !aligned(k_scales, 128) ||
+        !aligned(v_pages, 128) || !aligned(v_scales, 128))
+        return BDFP4_ERR_ALIGN;
+    if (chunk_tiles <= 0) {
+        // no host sequence lengths: plan for the longest possible sequence
+        int dev = 0, sms = 148;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return BDFP4_ERR_CUDA;
+        const int ntiles = (max_pages_per_seq * kPageSlots + kTileTokens - 1) / kTileTokens;
+        const int64_t total = (int64_t)B * H_kv * ntiles;
+        const int64_t chunk = std::max<int64_t>(4, (total + 16LL * sms - 1) / (16LL * sms));
+        chunk_tiles = (int)std::min<int64_t>(chunk, ntiles);
+    }
+    DecodeArgs a{};
+    a.max_splits = max_splits_for(max_pages_per_seq, chunk_tiles);
+    if (a.max_splits > 1) {
+        const size_t need = bdfp4_decode_workspace_size(B, H_q, d_v, max_pages_per_seq, chunk_tiles);
+        if (!workspace || workspace_bytes < need) return BDFP4_ERR_WORKSPACE;
+        if (!aligned(workspace, 128)) return BDFP4_ERR_ALIGN;
+        const size_t o_bytes = (size_t)B * H_q * a.max_splits * d_v * sizeof(float);
+        a.ws_o = (float*)workspace;
+        a.ws_ml = (float*)((char*)workspace + ((o_bytes + 255) / 256) * 256);
+    }
+    a.q = (const __nv_bfloat16*)q;
+    a.k_pages = (const uint8_t*)k_pages;
+    a.k_scales = (const uint8_t*)k_scales;
+    a.v_pages = (const uint8_t*)v_pages;
+    a.v_scales = (const uint8_t*)v_scales;
+    a.block_table = block_table;
+    a.seq_lens = seq_lens;
+    a.smooth = kv->smooth;
+    a.k_gscale = kv->k_gscale;
+    a.v_gscale = kv->v_gscale;
+    a.out = (__nv_bfloat16*)out;
+    a.dev_status = dev_status;
+    a.B = B;
+    a.H_q = H_q;
+    a.H_kv = H_kv;
+    a.max_pages = max_pages_per_seq;
+    a.num_pages = num_pages;
+    a.flags = flags;
+    a.chunk_tiles = chunk_tiles;
+    a.sm_scale = sm_scale;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (fmt == BDFP4_NVFP4)
+        return d_k == 128 ? launch_decode<BDFP4_NVFP4, 128, 128>(a, G, st) : launch_decode<BDFP4_NVFP4, 576, 512>(a, G, st);
+    return d_k == 128 ? launch_decode<BDFP4_MXFP4, 128, 128>(a, G, st) : launch_decode<BDFP4_MXFP4, 576, 512>(a, G, st);
+}
+
+extern "C" const char* bdfp4_status_string(int status) {
+    switch (status) {
+        case BDFP4_OK: return "ok";
+        case BDFP4_ERR_ARG: return "invalid argument (null pointer, negative size or bad enum)";
+        case BDFP4_ERR_SHAPE: return "inconsistent shapes";
+        case BDFP4_ERR_ALIGN: return "pointer not aligned (cache arrays and workspace 128 B, bf16 16 B)";
+        case BDFP4_ERR_UNSUPPORTED: return "shape outside the compiled set";
+        case BDFP4_ERR_CUDA: return "CUDA launch failed";
+        case BDFP4_ERR_WORKSPACE: return "workspace too small for the split plan";
+        default: return "unknown status";
+    }
+}

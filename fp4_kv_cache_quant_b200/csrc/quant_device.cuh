@@ -1,0 +1,155 @@
+// quant_device.cuh -- device steps shared by the quantizer kernels and the
+// decode prologue: the key/query transform (smoothing + Hadamard), block
+// quantization with its fp64 squared error, the key scale search and the
+// dual-residual query quantization (BitDecoding-FP4, Article Summary).
+#pragma once
+
+#include "bdfp4_device.cuh"
+
+namespace bdfp4 {
+
+// Row geometry: threads per row (padded), active threads, segment split.
+template <int FMT, int DK>
+struct RowGeom {
+    static constexpr int beta = Fmt<FMT>::beta;
+    static constexpr int tpr = DK / beta;                        // active threads
+    static constexpr int seg0 = (DK == 576) ? 512 : DK;          // first Hadamard segment
+    static constexpr int seg0_thr = seg0 / beta;
+    static constexpr int seg1_thr = (DK - seg0) / beta;           // rope segment threads (MLA)
+    static constexpr int rt = (DK == 576) ? ((seg0_thr == 32) ? 64 : 32) : tpr;   // padded threads per row
+};
+
+// Loads `beta` bf16 values starting at element e0 of a row into x.
+template <int BETA>
+__device__ __forceinline__ void load_bf16_block(const __nv_bfloat16* row, int e0, float* x) {
+    const uint4* p = reinterpret_cast<const uint4*>(row + e0);
+#pragma unroll
+    for (int v = 0; v < BETA / 8; ++v) {
+        uint4 w = __ldg(p + v);
+        x[8 * v + 0] = bf16_lo(w.x);
+        x[8 * v + 1] = bf16_hi(w.x);
+        x[8 * v + 2] = bf16_lo(w.y);
+        x[8 * v + 3] = bf16_hi(w.y);
+        x[8 * v + 4] = bf16_lo(w.z);
+        x[8 * v + 5] = bf16_hi(w.z);
+        x[8 * v + 6] = bf16_lo(w.w);
+        x[8 * v + 7] = bf16_hi(w.w);
+    }
+}
+
+// Smoothing + Hadamard of one thread's block (in place).  j = thread index in
+// the row; all lanes of the warp must call this (shuffles are warp-wide).
+template <int FMT, int DK, bool IS_KEY>
+__device__ __forceinline__ void transform_block(float* x, const float* smooth_row, int j, bool hadamard) {
+    using RG = RowGeom<FMT, DK>;
+    constexpr int B = RG::beta;
+    const int e0 = j * B;
+    const bool active = j < RG::tpr;
+#pragma unroll
+    for (int i = 0; i < B; ++i) {
+        float s = active ? __ldg(smooth_row + e0 + i) : 1.0f;
+        x[i] = IS_KEY ? __fdiv_rn(x[i], s) : __fmul_rn(x[i], s);
+    }
+    if (!hadamard) return;
+    fwht_local<B>(x);
+    const int seg = (j >= RG::seg0_thr) ? 1 : 0;
+    const int seg_thr = seg ? RG::seg1_thr : RG::seg0_thr;
+#pragma unroll
+    for (int lb = 1; lb < RG::seg0_thr; lb <<= 1) {
+        // every lane shuffles; only lanes whose segment spans this stage keep the result
+        float y[B];
+#pragma unroll
+        for (int i = 0; i < B; ++i) y[i] = x[i];
+        fwht_cross<B>(y, lb, 0xffffffffu);
+        if (active && lb < seg_thr) {
+#pragma unroll
+            for (int i = 0; i < B; ++i) x[i] = y[i];
+        }
+    }
+    const float post = hadamard_post(seg ? (DK - RG::seg0) : RG::seg0, IS_KEY);
+#pragma unroll
+    for (int i = 0; i < B; ++i) x[i] = __fmul_rn(x[i], post);
+}
+
+// E2M1 codes of x / sigma (sigma = 0 -> zeros), packed two per byte (even
+// element low), and the block's squared error summed left to right in fp64.
+template <int B>
+__device__ __forceinline__ double quantize_block(const float* x, float sigma, uint32_t* packed /* B/8 words */) {
+    double err = 0.0;
+#pragma unroll
+    for (int w = 0; w < B / 8; ++w) packed[w] = 0u;
+#pragma unroll
+    for (int i = 0; i < B; i += 2) {
+        uint32_t pair = 0u;
+        if (sigma != 0.0f) pair = e2m1x2_encode(__fdiv_rn(x[i], sigma), __fdiv_rn(x[i + 1], sigma));
+        packed[i / 8] |= pair << (4 * (i % 8));
+        double d0 = __dsub_rn((double)x[i], __dmul_rn((double)e2m1_value(pair & 15u), (double)sigma));
+        err = __dadd_rn(err, __dmul_rn(d0, d0));
+        double d1 = __dsub_rn((double)x[i + 1], __dmul_rn((double)e2m1_value(pair >> 4), (double)sigma));
+        err = __dadd_rn(err, __dmul_rn(d1, d1));
+    }
+    return err;
+}
+
+template <int B>
+__device__ __forceinline__ float block_amax(const float* x) {
+    float a = 0.0f;
+#pragma unroll
+    for (int i = 0; i < B; ++i) a = fmaxf(a, fabsf(x[i]));
+    return a;
+}
+
+// Scale search window: NVFP4 c0+7 .. c0-2 (E4M3 codes, within [0, 126]);
+// MXFP4 c0+1, c0 (E8M0, within [0, 254]); least squared error, ties to the
+// larger code.  All-zero blocks keep code 0.
+template <int FMT>
+__device__ __forceinline__ uint32_t search_scale(const float* x, float g) {
+    constexpr int B = Fmt<FMT>::beta;
+    const float amax = block_amax<B>(x);
+    const int c0 = (int)plain_scale_code<FMT>(amax, g);
+    if (amax == 0.0f) return (uint32_t)c0;
+    const int top = FMT == BDFP4_NVFP4 ? 126 : 254;
+    int hi = c0 + (FMT == BDFP4_NVFP4 ? 7 : 1);
+    int lo = c0 - (FMT == BDFP4_NVFP4 ? 2 : 0);
+    hi = hi > top ? top : hi;
+    lo = lo < 0 ? 0 : lo;
+    int best = hi;
+    double best_err = 0.0;
+    uint32_t scratch[B / 8];
+    for (int c = hi; c >= lo; --c) {
+        double err = quantize_block<B>(x, block_sigma<FMT>((uint32_t)c, g), scratch);
+        if (c == hi || err < best_err) {
+            best = c;
+            best_err = err;
+        }
+    }
+    return (uint32_t)best;
+}
+
+// ---------------------------------------------------------------- query
+// Dual-residual quantization of one query row by its row thread group.  The
+// row amax (for g_q) is a max over the row's threads through shared memory.
+template <int FMT, int DK>
+__device__ __forceinline__ void quantize_query_block(float* x, float gq, bool dual, uint32_t& c1, uint32_t* p1,
+                                                     uint32_t& c2, uint32_t* p2) {
+    constexpr int B = Fmt<FMT>::beta;
+    c1 = plain_scale_code<FMT>(block_amax<B>(x), gq);
+    const float s1 = block_sigma<FMT>(c1, gq);
+    quantize_block<B>(x, s1, p1);
+    float r[B];
+#pragma unroll
+    for (int i = 0; i < B; ++i) {
+        const uint32_t e = (p1[i / 8] >> (4 * (i % 8))) & 15u;
+        r[i] = __fsub_rn(x[i], __fmul_rn(e2m1_value(e), s1));
+    }
+    if (dual) {
+        c2 = plain_scale_code<FMT>(block_amax<B>(r), gq);
+        quantize_block<B>(r, block_sigma<FMT>(c2, gq), p2);
+    } else {
+        c2 = 0u;
+#pragma unroll
+        for (int w = 0; w < B / 8; ++w) p2[w] = 0u;
+    }
+}
+
+}  // namespace bdfp4

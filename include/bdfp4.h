@@ -1,0 +1,188 @@
+/*
+ * bdfp4.h -- C ABI of a B200 (sm_100a) library for decode-time attention over
+ * a paged KV cache stored in native 4-bit microscaling formats.
+ *
+ * The method is BitDecoding-FP4 ("BitDecoding-FP4: Native FP4 KV Cache
+ * Decoding via Algorithm-System Co-Design", Article Summary): NVFP4 / MXFP4 KV
+ * cache; Outlier-Aware Key Quantization (static smoothing, Hadamard rotation,
+ * scale search) under token-wise scaling; Dual-Residual Query Quantization
+ * (q ~ q1 + q2, two FP4 tensors); Underflow-Aware Probability Scaling; a
+ * transposed softmax with fused probability quantization and stacked-query
+ * MMA on paged caches.  How each step is read where the pages leave it open
+ * is stated next to the entry point that performs it.
+ *
+ * Conventions for every entry point:
+ *  - All array pointers are DEVICE pointers unless the name says host_.  The
+ *    caller owns and allocates all memory; the library keeps no state between
+ *    calls and allocates nothing.
+ *  - Work is enqueued on `stream` (a cudaStream_t passed as void*, NULL = the
+ *    legacy default stream) and is asynchronous; the return code only reports
+ *    errors found on the host before launch, or a launch failure.
+ *  - Errors the kernels find (bad page index, bad sequence length, bad slot)
+ *    are OR-ed into *dev_status (an int32 the caller zeroes and reads after
+ *    synchronising); the offending token is skipped, never read or written
+ *    out of bounds.  No kernel traps.
+ *  - bf16 tensors are row-major with the last dimension contiguous.
+ *  - Base pointers of cache arrays and the workspace must be 128-byte aligned;
+ *    bf16 inputs 16-byte aligned.
+ *
+ * Cache layout (a "page" holds 64 token slots for every KV head; beta = 16
+ * for NVFP4, 32 for MXFP4; FP4 values are E2M1 codes, two per byte, the
+ * even-indexed element in the low nibble; scale codes are E4M3 (NVFP4) or
+ * E8M0 (MXFP4) bytes):
+ *   k_pages  [num_pages][H_kv][64 * d_k / 2] bytes; within (page, head):
+ *            [slot/8][elem/32][slot%8][16 bytes holding elements 32*(elem/32)..+31]
+ *   k_scales [num_pages][H_kv][64 * d_k / beta]; within (page, head), scale of
+ *            block blk (elements blk*beta..) of slot:
+ *            [slot%32][blk / (64/beta)][slot/32][blk % (64/beta)]
+ *   v_pages  [num_pages][H_kv][d_v * 64 / 2]; within (page, head):
+ *            [chan/8][slot/32][chan%8][16 bytes holding slots 32*(slot/32)..+31]
+ *   v_scales [num_pages][H_kv][d_v * 64 / beta]; scale of the beta-slot block
+ *            blk of channel chan: [chan/128][chan%32][(chan%128)/32][blk]
+ * K blocks run along the head dim of one token (token-wise scaling); V blocks
+ * run along beta consecutive slots of one page for one channel, because the
+ * PV product reduces over tokens.  These are the tcgen05 block-scaled MMA
+ * operand layouts, so pages move to shared memory with plain bulk copies.
+ *
+ * Supported shapes: (d_k, d_v) in {(128, 128), (576, 512)}; H_q / H_kv in
+ * {1, 2, 4, 8, 16} or a multiple of 16 up to 128; anything else returns
+ * BDFP4_ERR_UNSUPPORTED.
+ */
+#ifndef BDFP4_H
+#define BDFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BDFP4_API __attribute__((visibility("default")))
+#else
+#define BDFP4_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { BDFP4_NVFP4 = 0, BDFP4_MXFP4 = 1 } bdfp4_fmt;
+
+/* host return codes */
+#define BDFP4_OK 0
+#define BDFP4_ERR_ARG (-1)         /* null pointer, negative size, bad enum       */
+#define BDFP4_ERR_SHAPE (-2)       /* inconsistent sizes                           */
+#define BDFP4_ERR_ALIGN (-3)       /* pointer alignment                            */
+#define BDFP4_ERR_UNSUPPORTED (-4) /* shape outside the compiled set               */
+#define BDFP4_ERR_CUDA (-5)        /* a CUDA launch or query failed                */
+#define BDFP4_ERR_WORKSPACE (-6)   /* workspace too small for the split plan      */
+
+/* bits OR-ed into *dev_status by the kernels */
+#define BDFP4_DEV_BAD_PAGE 1       /* block_table entry outside [0, num_pages)     */
+#define BDFP4_DEV_BAD_SEQLEN 2     /* seq_len < 0 or > max_pages_per_seq * 64      */
+#define BDFP4_DEV_BAD_SLOT 4       /* slot_mapping entry >= num_pages * 64         */
+
+/* flags (ablation arms of the method; 0 = the method as described) */
+#define BDFP4_FLAG_NO_HADAMARD 1     /* no rotation of K and q (must match between quantize and decode) */
+#define BDFP4_FLAG_NO_SCALE_SEARCH 2 /* keys use the plain amax scale rule                               */
+#define BDFP4_FLAG_SINGLE_QUERY 4    /* vanilla single-FP4 query (q2 = 0)                               */
+#define BDFP4_FLAG_NO_UNDERFLOW 8    /* vanilla probability scaling (alpha = 1)                         */
+
+/* Static per-layer quantization parameters (device pointers), produced by
+ * bdfp4_calibrate or supplied by the caller. */
+typedef struct {
+    const float* smooth;   /* [H_kv][d_k]: s_c, each a power of two; keys are divided by s_c, queries multiplied */
+    const float* k_gscale; /* [H_kv]: NVFP4 FP32 tensor scale of keys (unused for MXFP4)   */
+    const float* v_gscale; /* [H_kv]: NVFP4 FP32 tensor scale of values (unused for MXFP4) */
+} bdfp4_kv_params;
+
+/*
+ * Static calibration of the Outlier-Aware Key Quantization parameters
+ * ("static smoothing", Article Summary), from a calibration draw.
+ * k_cal [Tc][H_kv][d_k], v_cal [Tc][H_kv][d_v], q_cal [Tq][H_q][d_k] bf16.
+ * Outputs smooth [H_kv][d_k], k_gscale [H_kv], v_gscale [H_kv] (fp32).
+ * Reading: s_c = 2^n, n = round-half-up(log2(kmax_c / qmax_c) / 2) clamped to
+ * [-20, 20] (0 when either maximum is 0), kmax over the calibration keys of
+ * the head and qmax over the queries of its group; g_k = fp32(amax / 2688) of
+ * the transformed calibration keys, g_v = fp32(amax / 2688) of the values
+ * (2688 = 6 * 448, the E2M1 and E4M3 maxima), 1 when the amax is 0.
+ * Query head h belongs to KV head h / (H_q / H_kv).
+ */
+BDFP4_API int bdfp4_calibrate(const void* k_cal, const void* q_cal, const void* v_cal, int Tc, int Tq, int H_q, int H_kv,
+                    int d_k, int d_v, int flags, float* smooth, float* k_gscale, float* v_gscale, void* stream);
+
+/*
+ * KV-append quantization into the paged cache (Outlier-Aware Key Quantization,
+ * Article Summary; "Analyse approfondie" of the French page for what each
+ * part does).  k [T][H_kv][d_k], v [T][H_kv][d_v] bf16; slot_mapping [T] int64
+ * = page * 64 + slot, or -1 to skip the token.
+ * Keys: x = H (k / s) * 2^-ceil(L/2) per power-of-two segment of length 2^L
+ * of the head dim (576 = 512 + 64), computed as fixed fp32 butterflies; then
+ * per block of beta channels a scale code is searched (NVFP4: E4M3 codes
+ * c0+7 .. c0-2 around the plain code c0 = E4M3(amax / (6 g_k)); MXFP4: E8M0
+ * codes c0+1, c0 around the OCP MX rule) minimising the block's squared error
+ * (fp64, left to right), ties to the larger code; elements are E2M1(x / sigma),
+ * sigma = fp32(E4M3(c) g_k) or 2^(c-127).
+ * Values: the beta-slot blocks of the call's tokens are (re)quantized with the
+ * plain rule; a block's tokens must form one run of consecutive tokens with
+ * consecutive slots in this call, and slots of a touched block outside the
+ * run become zero.  To append a token into a partly filled block, pass the
+ * block's earlier tokens again in the same call.
+ * Results are bit-identical to the stated fp32/fp64 operation sequence.
+ */
+BDFP4_API int bdfp4_quantize_kv(const void* k, const void* v, const int64_t* slot_mapping, int T, int H_kv, int d_k, int d_v,
+                      bdfp4_fmt fmt, int flags, const bdfp4_kv_params* kv, void* k_pages, void* k_scales,
+                      void* v_pages, void* v_scales, int64_t num_pages, int32_t* dev_status, void* stream);
+
+/*
+ * Dual-Residual Query Quantization on its own (Article Summary; the French
+ * page: the second FP4 tensor encodes the residual of the first), exactly as
+ * the decode prologue performs it.  q [B][H_q][d_k] bf16.  Query transform:
+ * x = H (q * s) * 2^-floor(L/2).  NVFP4: g_q = fp32(amax(x) / 2688) per query
+ * head (1 if 0); q1 = plain-rule FP4 of x; r = fp32(x - fp32(e1 * sigma1));
+ * q2 = plain-rule FP4 of r with the same g_q.  MXFP4: E8M0 scales, no g_q.
+ * Outputs (logical layout, one E2M1 code per byte): q1_codes, q2_codes
+ * [B][H_q][d_k]; q1_scales, q2_scales [B][H_q][d_k / beta]; g_q [B][H_q].
+ */
+BDFP4_API int bdfp4_quantize_q(const void* q, int B, int H_q, int H_kv, int d_k, bdfp4_fmt fmt, int flags, const float* smooth,
+                     uint8_t* q1_codes, uint8_t* q1_scales, uint8_t* q2_codes, uint8_t* q2_scales, float* g_q,
+                     void* stream);
+
+/*
+ * Split plan for bdfp4_decode: tiles (128 tokens) per split so that the
+ * (sequence, KV head, split) work items fill num_sms SMs several times over.
+ * host_seq_lens [B] is a HOST array.  Returns chunk_tiles >= 1, or a negative
+ * status.  Sequence b then has ceil(ceil(N_b / 128) / chunk_tiles) splits.
+ */
+BDFP4_API int bdfp4_decode_plan(const int32_t* host_seq_lens, int B, int H_kv, int num_sms);
+
+/* Bytes of workspace bdfp4_decode needs for this shape and chunk_tiles. */
+BDFP4_API size_t bdfp4_decode_workspace_size(int B, int H_q, int d_v, int max_pages_per_seq, int chunk_tiles);
+
+/*
+ * FP4 paged decode attention, one query token per sequence.
+ * q [B][H_q][d_k] bf16; block_table [B][max_pages_per_seq] int32 page ids;
+ * seq_lens [B] int32; out [B][H_q][d_v] bf16.
+ * Per (sequence, query head): the query is transformed and dual-residual
+ * quantized; logits s_t = sm_scale g_q g_k (q1 + q2) . k_t over the paged keys;
+ * an online softmax runs over 128-token tiles from the sequence start, cut
+ * into splits of chunk_tiles tiles; per tile p_t = exp(s_t - m_new), l sums the
+ * unquantized p, and P is quantized in beta-token blocks (NVFP4: alpha = 2^11
+ * underflow-aware pre-scale, divided out exactly; E4M3 block scale of
+ * amax(alpha p) / 6, code 0 collapses the block; MXFP4: E8M0, alpha = 1);
+ * O accumulates P^ V; splits merge by log-sum-exp.  An empty sequence gives
+ * zeros.  chunk_tiles <= 0 picks a plan from device seq_lens' upper bound
+ * (max_pages_per_seq * 64).  workspace: >= bdfp4_decode_workspace_size bytes.
+ */
+BDFP4_API int bdfp4_decode(const void* q, const void* k_pages, const void* k_scales, const void* v_pages,
+                 const void* v_scales, const int32_t* block_table, const int32_t* seq_lens, int B, int H_q, int H_kv,
+                 int d_k, int d_v, int max_pages_per_seq, int64_t num_pages, bdfp4_fmt fmt, int flags,
+                 const bdfp4_kv_params* kv, float sm_scale, int chunk_tiles, void* workspace,
+                 size_t workspace_bytes, void* out, int32_t* dev_status, void* stream);
+
+/* Human-readable text of a host return code. */
+BDFP4_API const char* bdfp4_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BDFP4_H */

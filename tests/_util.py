@@ -1,0 +1,97 @@
+"""Helpers shared by the GPU parity tests: move a seeded workload to the GPU,
+run the oracle on the same inputs, compare."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from fp4_kv_cache_quant_b200 import bdfp4
+from fp4_kv_cache_quant_b200.workloads import Workload
+
+# decode tolerance: output within max-abs 1e-2 and relative L2 5e-3 of the
+# oracle run on identical FP4 cache bytes
+MAX_ABS = 1e-2
+REL_L2 = 5e-3
+
+
+def bf16_to_np(bits: np.ndarray) -> np.ndarray:
+    return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def out_to_np(t: torch.Tensor) -> np.ndarray:
+    return t.float().cpu().numpy()
+
+
+def compare_outputs(gpu: np.ndarray, ref: np.ndarray):
+    """-> (max_abs, rel_l2)."""
+    g = gpu.astype(np.float64)
+    r = ref.astype(np.float64)
+    max_abs = float(np.max(np.abs(g - r))) if g.size else 0.0
+    rel = float(np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-30))
+    return max_abs, rel
+
+
+def kv_params_np(kv: bdfp4.KVParams):
+    return kv.smooth.cpu().numpy(), kv.k_gscale.cpu().numpy(), kv.v_gscale.cpu().numpy()
+
+
+def kv_params_gpu(smooth, kg, vg) -> bdfp4.KVParams:
+    f = lambda a: torch.from_numpy(np.ascontiguousarray(a, np.float32)).cuda()  # noqa: E731
+    return bdfp4.KVParams(f(smooth), f(kg), f(vg))
+
+
+def cache_to_np(cache: bdfp4.FP4Cache) -> dict:
+    return {n: getattr(cache, n).cpu().numpy() for n in ("k_pages", "k_scales", "v_pages", "v_scales")}
+
+
+def cache_from_np(c: dict, num_pages, H_kv, d_k, d_v, fmt) -> bdfp4.FP4Cache:
+    g = lambda a: torch.from_numpy(a).cuda()  # noqa: E731
+    return bdfp4.FP4Cache(g(c["k_pages"]), g(c["k_scales"]), g(c["v_pages"]), g(c["v_scales"]), num_pages, H_kv,
+                          d_k, d_v, fmt)
+
+
+def oracle_calibration(ora, wl: Workload, flags: int = 0):
+    kc, qc, vc = wl.calibration("cpu")
+    return ora.calibrate(kc, qc, vc, wl.spec.H_q, wl.spec.H_kv, flags=flags)
+
+
+def quantize_both(ora, wl: Workload, fmt: int, smooth, kg, vg, flags: int = 0):
+    """Quantize the whole workload on the GPU and in the oracle; returns
+    (gpu FP4Cache, oracle cache dict)."""
+    sp = wl.spec
+    k = wl.all_keys("cpu")
+    v = wl.all_values("cpu")
+    sm = wl.slot_mapping_all()
+    ocache = ora.empty_cache(wl.num_pages, sp.H_kv, sp.d_k, sp.d_v, fmt)
+    ora.quantize_kv(k, v, sm, ocache, sp.H_kv, fmt, smooth, kg, vg, wl.num_pages, flags=flags)
+    gcache = bdfp4.FP4Cache.empty(wl.num_pages, sp.H_kv, sp.d_k, sp.d_v, fmt)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    bdfp4.bdfp4_quantize_kv(k.cuda(), v.cuda(), torch.from_numpy(sm).cuda(), kv_params_gpu(smooth, kg, vg), gcache,
+                            flags=flags, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    return gcache, ocache
+
+
+def assert_bytes_equal(gpu: dict, ora: dict):
+    for name in ("k_pages", "k_scales", "v_pages", "v_scales"):
+        a, b = gpu[name], ora[name]
+        assert a.shape == b.shape, name
+        bad = np.nonzero(a != b)[0]
+        assert bad.size == 0, f"{name}: {bad.size} bytes differ, first at {bad[:8].tolist()}: " \
+                              f"gpu {a[bad[:8]].tolist()} oracle {b[bad[:8]].tolist()}"
+
+
+def run_gpu_decode(wl: Workload, cache: bdfp4.FP4Cache, q: torch.Tensor, kvp: bdfp4.KVParams, chunk_tiles: int,
+                   flags: int = 0, seq_lens=None, block_table=None):
+    sp = wl.spec
+    sl = torch.from_numpy(np.asarray(wl.seq_lens if seq_lens is None else seq_lens, np.int32)).cuda()
+    bt = torch.from_numpy(np.asarray(wl.block_table if block_table is None else block_table, np.int32)).cuda()
+    B = q.shape[0]
+    out = torch.empty((B, sp.H_q, sp.d_v), dtype=torch.bfloat16, device="cuda")
+    ws = bdfp4.workspace_for(B, sp.H_q, sp.d_v, bt.shape[1], max(chunk_tiles, 1))
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    bdfp4.bdfp4_decode(q.cuda(), cache, bt, sl, kvp, sp.sm_scale, chunk_tiles, ws, out, flags=flags,
+                       dev_status=status)
+    torch.cuda.synchronize()
+    return out, int(status.item())

@@ -1,0 +1,109 @@
+"""Host-only checks of the C ABI: the library loads, exports every entry point
+include/bdfp4.h declares, and rejects bad arguments before touching a GPU."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from fp4_kv_cache_quant_b200 import bdfp4
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from fp4_kv_cache_quant_b200 import build
+    build.build()
+    return bdfp4.load()
+
+
+def _declared():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"BDFP4_API\s+[\w\s\*]+?\b(bdfp4_\w+)\s*\(", src)
+    return names
+
+
+def test_exports_every_declared_entry_point(lib):
+    names = _declared()
+    assert set(bdfp4.ENTRY_POINTS) <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for code in range(-6, 1):
+        s = bdfp4.bdfp4_status_string(code)
+        assert s and s != "unknown status"
+    assert bdfp4.bdfp4_status_string(42) == "unknown status"
+
+
+def test_decode_plan_host_logic(lib):
+    # 16 sequences of 32768 tokens, 8 KV heads, 148 SMs: 256 tiles each,
+    # 32768 work tiles -> ceil(32768 / (16 * 148)) = 14 tiles per split
+    assert bdfp4.bdfp4_decode_plan(np.full(16, 32768), 8, 148) == 14
+    # at least 4 tiles per split, at most the longest sequence
+    assert bdfp4.bdfp4_decode_plan(np.array([1000]), 1, 148) == 4
+    assert bdfp4.bdfp4_decode_plan(np.array([100]), 1, 148) == 1
+    # 64 sequences of 131072 tokens x 4 heads = 262144 tiles -> 111 per split
+    assert bdfp4.bdfp4_decode_plan(np.full(64, 131072), 4, 148) == 111
+    assert bdfp4.bdfp4_decode_plan(np.array([0, 0]), 2, 148) == 1
+    with pytest.raises(bdfp4.BDFP4Error):
+        bdfp4.bdfp4_decode_plan(np.array([10]), 0, 148)
+
+
+def test_workspace_size(lib):
+    # B=2, H_q=4, d_v=128, 16 pages = 8 tiles, 2 tiles per split -> 4 splits
+    o = 2 * 4 * 4 * 128 * 4
+    assert bdfp4.bdfp4_decode_workspace_size(2, 4, 128, 16, 2) == ((o + 255) // 256) * 256 + 2 * 4 * 4 * 2 * 4
+    assert bdfp4.bdfp4_decode_workspace_size(0, 4, 128, 16, 2) == 0
+
+
+def _p(addr):
+    return ctypes.c_void_p(addr)
+
+
+def test_quantize_kv_argument_errors(lib):
+    kv = bdfp4._KVParams(0x1000, 0x2000, 0x3000)
+    a = _p(0x10000)
+    args = lambda d_k=128, d_v=128, fmt=0, k=a, kvp=ctypes.byref(kv): (  # noqa: E731
+        k, a, a, 10, 2, d_k, d_v, fmt, 0, kvp, a, a, a, a, 4, None, None)
+    assert lib.bdfp4_quantize_kv(*args(d_k=64)) == -4
+    assert lib.bdfp4_quantize_kv(*args(d_k=576, d_v=128)) == -4
+    assert lib.bdfp4_quantize_kv(*args(fmt=7)) == -1
+    assert lib.bdfp4_quantize_kv(*args(k=None)) == -1
+    assert lib.bdfp4_quantize_kv(*args(kvp=None)) == -1
+    assert lib.bdfp4_quantize_kv(*args(k=_p(0x10001))) == -3
+
+
+def test_decode_argument_errors(lib):
+    kv = bdfp4._KVParams(0x1000, 0x2000, 0x3000)
+    a = _p(0x10000)
+
+    def call(H_q=8, H_kv=2, d_k=128, d_v=128, chunk=1, ws=None, ws_bytes=0, q=a, max_pages=4):
+        return lib.bdfp4_decode(q, a, a, a, a, a, a, 2, H_q, H_kv, d_k, d_v, max_pages, 16, 0, 0, ctypes.byref(kv),
+                                0.1, chunk, ws, ws_bytes, a, None, None)
+    assert call(H_q=6, H_kv=2) == -4      # group of 3
+    assert call(H_q=7, H_kv=2) == -2      # not a multiple
+    assert call(d_k=256) == -4
+    assert call(q=None) == -1
+    assert call(q=_p(0x10008)) == -3
+    assert call(chunk=1) == -6            # 2 splits need a workspace
+    n = bdfp4.bdfp4_decode_workspace_size(2, 8, 128, 4, 1)
+    assert call(chunk=1, ws=_p(0x20000), ws_bytes=n - 1) == -6
+
+
+def test_product_code_does_not_touch_the_oracle():
+    """The CUDA library and its binding share no code with the oracle."""
+    pkg = os.path.join(ROOT, "fp4_kv_cache_quant_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in re.sub(r"#.*|//.*", "", src).lower() or f == "workloads.py", f
+    osrc = open(os.path.join(ROOT, "oracle", "bdfp4_oracle.c")).read()
+    assert "#include \"" not in osrc

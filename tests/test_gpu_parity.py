@@ -1,0 +1,192 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Quantized bytes (cache, query codes, calibration) must match bit for bit;
+decode outputs within max-abs 1e-2 and relative L2 5e-3 of the oracle run on
+the same FP4 cache bytes."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from _util import (MAX_ABS, REL_L2, assert_bytes_equal, bf16_to_np, cache_from_np, cache_to_np, compare_outputs,
+                   kv_params_gpu, oracle_calibration, out_to_np, quantize_both, run_gpu_decode)
+from fp4_kv_cache_quant_b200 import bdfp4
+from fp4_kv_cache_quant_b200.workloads import Workload, spec
+
+pytestmark = pytest.mark.gpu
+
+NV, MX = 0, 1
+
+SMALL = {
+    # name: (spec, fmt)
+    "tiny_nv": (spec("tiny"), NV),
+    "tiny_mx": (spec("tiny"), MX),
+    "ragged_g8_nv": (spec("qwen3_30b_a3b", B=4, ctx=("list", (1000, 77, 129, 513))), NV),
+    "ragged_g8_mx": (spec("qwen3_30b_a3b", B=4, ctx=("list", (1000, 77, 129, 513))), MX),
+    "g1_nv": (spec("tiny", H_q=2, H_kv=2, ctx=("fixed", 300)), NV),
+    "g16_nv": (spec("tiny", B=2, H_q=16, H_kv=1, ctx=("list", (200, 1)), n_outlier=2), NV),
+    "mla_nv": (spec("mla", B=2, H_q=16, ctx=("list", (300, 130))), NV),
+    "mla_mx": (spec("mla", B=2, H_q=16, ctx=("list", (300, 130))), MX),
+}
+
+
+@pytest.fixture(scope="module")
+def lib():
+    assert torch.cuda.is_available()
+    bdfp4.load()
+    return bdfp4
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_calibration_bit_exact(ora, lib, name):
+    sp, fmt = SMALL[name]
+    wl = Workload(sp, seed=1)
+    smooth, kg, vg = oracle_calibration(ora, wl)
+    kc, qc, vc = wl.calibration("cpu")
+    kv = bdfp4.bdfp4_calibrate(kc.cuda(), qc.cuda(), vc.cuda(), sp.H_q, sp.H_kv)
+    torch.cuda.synchronize()
+    assert np.array_equal(kv.smooth.cpu().numpy(), smooth)
+    assert np.array_equal(kv.k_gscale.cpu().numpy(), kg)
+    assert np.array_equal(kv.v_gscale.cpu().numpy(), vg)
+
+
+@pytest.mark.parametrize("flags", [0, bdfp4.FLAG_NO_HADAMARD | bdfp4.FLAG_NO_SCALE_SEARCH])
+@pytest.mark.parametrize("name", list(SMALL))
+def test_quantize_kv_bit_exact(ora, lib, name, flags):
+    sp, fmt = SMALL[name]
+    wl = Workload(sp, seed=2)
+    smooth, kg, vg = oracle_calibration(ora, wl, flags)
+    gcache, ocache = quantize_both(ora, wl, fmt, smooth, kg, vg, flags)
+    assert_bytes_equal(cache_to_np(gcache), ocache)
+
+
+@pytest.mark.parametrize("fmt", [NV, MX])
+def test_quantize_kv_adversarial_values(ora, lib, fmt):
+    """Exact E2M1 midpoints (ties), zero blocks, tiny and huge values, runs
+    that start mid-block, skipped tokens (-1), partial pages."""
+    rng = np.random.default_rng(3)
+    H_kv, d, T = 2, 128, 150
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.0, 7.0, 0.0])
+    k = rng.choice(mids, size=(T, H_kv, d)) * rng.choice([-1, 1], size=(T, H_kv, d)) * 2.0 ** rng.integers(-3, 3, size=(T, H_kv, 1))
+    v = rng.choice(mids, size=(T, H_kv, d)) * rng.choice([-1, 1], size=(T, H_kv, d)) * 2.0 ** rng.integers(-3, 3, size=(T, H_kv, 1))
+    k[5] = 0.0
+    v[20:40] = 0.0
+    k[7] *= 1e-30
+    v[9] *= 1e20
+    k = torch.tensor(k, dtype=torch.float32).to(torch.bfloat16)
+    v = torch.tensor(v, dtype=torch.float32).to(torch.bfloat16)
+    # slots: a run starting mid-block, a skipped token, a run into a second page
+    sm = np.concatenate([np.arange(3, 3 + 100), [-1], np.arange(64 * 2 + 10, 64 * 2 + 10 + 49)]).astype(np.int64)
+    num_pages = 4
+    for flags in (0, bdfp4.FLAG_NO_HADAMARD):
+        smooth = (2.0 ** rng.integers(-2, 3, size=(H_kv, d))).astype(np.float32)
+        kg = np.array([0.37, 0.011], np.float32)
+        vg = np.array([0.05, 1.3], np.float32)
+        ocache = ora.empty_cache(num_pages, H_kv, d, d, fmt)
+        ora.quantize_kv(k, v, sm, ocache, H_kv, fmt, smooth, kg, vg, num_pages, flags=flags)
+        gcache = bdfp4.FP4Cache.empty(num_pages, H_kv, d, d, fmt)
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        bdfp4.bdfp4_quantize_kv(k.cuda(), v.cuda(), torch.from_numpy(sm).cuda(), kv_params_gpu(smooth, kg, vg), gcache,
+                                flags=flags, dev_status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        assert_bytes_equal(cache_to_np(gcache), ocache)
+
+
+@pytest.mark.parametrize("flags", [0, bdfp4.FLAG_SINGLE_QUERY, bdfp4.FLAG_NO_HADAMARD])
+@pytest.mark.parametrize("name", ["tiny_nv", "tiny_mx", "ragged_g8_nv", "mla_nv", "mla_mx"])
+def test_quantize_q_bit_exact(ora, lib, name, flags):
+    sp, fmt = SMALL[name]
+    wl = Workload(sp, seed=4)
+    smooth, _, _ = oracle_calibration(ora, wl, flags)
+    q = wl.queries("cpu")
+    ref = ora.quantize_q(q, sp.H_kv, fmt, smooth, flags=flags)
+    got = bdfp4.bdfp4_quantize_q(q.cuda(), sp.H_kv, fmt, torch.from_numpy(smooth).cuda(), flags=flags)
+    torch.cuda.synchronize()
+    for key in ("q1_codes", "q1_scales", "q2_codes", "q2_scales", "g_q"):
+        assert np.array_equal(got[key].cpu().numpy(), ref[key]), key
+
+
+def _decode_case(ora, name, chunk_tiles, flags, seed=5):
+    sp, fmt = SMALL[name]
+    wl = Workload(sp, seed=seed)
+    smooth, kg, vg = oracle_calibration(ora, wl, flags & bdfp4.FLAG_NO_HADAMARD)
+    q = wl.queries("cpu")
+    ocache = ora.empty_cache(wl.num_pages, sp.H_kv, sp.d_k, sp.d_v, fmt)
+    ora.quantize_kv(wl.all_keys(), wl.all_values(), wl.slot_mapping_all(), ocache, sp.H_kv, fmt, smooth, kg, vg,
+                    wl.num_pages, flags=flags & bdfp4.FLAG_NO_HADAMARD)
+    if chunk_tiles <= 0:
+        chunk_tiles = bdfp4.bdfp4_decode_plan(wl.seq_lens, sp.H_kv, torch.cuda.get_device_properties(0).multi_processor_count)
+    ref16, _ = ora.decode(q, ocache, wl.block_table, wl.seq_lens, sp.H_kv, sp.d_v, fmt, smooth, kg, vg, sp.sm_scale,
+                          chunk_tiles, wl.num_pages, flags=flags)
+    gcache = cache_from_np(ocache, wl.num_pages, sp.H_kv, sp.d_k, sp.d_v, fmt)
+    out, status = run_gpu_decode(wl, gcache, q, kv_params_gpu(smooth, kg, vg), chunk_tiles, flags)
+    assert status == 0
+    return out_to_np(out), bf16_to_np(ref16), wl
+
+
+@pytest.mark.parametrize("chunk", [0, 1, 3])
+@pytest.mark.parametrize("name", list(SMALL))
+def test_decode_matches_oracle(ora, lib, name, chunk):
+    got, ref, wl = _decode_case(ora, name, chunk, 0)
+    max_abs, rel = compare_outputs(got, ref)
+    assert max_abs <= MAX_ABS and rel <= REL_L2, (max_abs, rel)
+    for b, n in enumerate(wl.seq_lens):
+        if n == 0:
+            assert np.all(got[b] == 0)
+
+
+@pytest.mark.parametrize("flags", [bdfp4.FLAG_SINGLE_QUERY, bdfp4.FLAG_NO_UNDERFLOW, bdfp4.FLAG_NO_HADAMARD,
+                                   bdfp4.FLAG_SINGLE_QUERY | bdfp4.FLAG_NO_UNDERFLOW])
+@pytest.mark.parametrize("name", ["tiny_nv", "ragged_g8_nv", "ragged_g8_mx"])
+def test_decode_ablation_flags_match_oracle(ora, lib, name, flags):
+    got, ref, _ = _decode_case(ora, name, 2, flags)
+    max_abs, rel = compare_outputs(got, ref)
+    assert max_abs <= MAX_ABS and rel <= REL_L2, (max_abs, rel)
+
+
+def test_decode_empty_and_single_token(ora, lib):
+    sp = spec("tiny", B=3, ctx=("list", (0, 1, 65)))
+    SMALL["edge"] = (sp, NV)
+    try:
+        got, ref, wl = _decode_case(ora, "edge", 1, 0)
+    finally:
+        del SMALL["edge"]
+    assert np.all(got[0] == 0)
+    max_abs, rel = compare_outputs(got, ref)
+    assert max_abs <= MAX_ABS and rel <= REL_L2, (max_abs, rel)
+
+
+def test_device_status_on_bad_block_table(ora, lib):
+    """An out-of-range page id is reported through dev_status and skipped."""
+    sp, fmt = SMALL["tiny_nv"]
+    wl = Workload(sp, seed=6)
+    smooth, kg, vg = oracle_calibration(ora, wl)
+    gcache, _ = quantize_both(ora, wl, fmt, smooth, kg, vg)
+    bt = wl.block_table.copy()
+    bt[0, 3] = wl.num_pages + 100
+    out, status = run_gpu_decode(wl, gcache, wl.queries(), kv_params_gpu(smooth, kg, vg), 2, block_table=bt)
+    assert status & bdfp4.DEV_BAD_PAGE
+    assert np.isfinite(out_to_np(out)).all()
+    # a sequence longer than the table allows is reported too
+    out, status = run_gpu_decode(wl, gcache, wl.queries(), kv_params_gpu(smooth, kg, vg), 2,
+                                 seq_lens=[sp.ctx[1] + 10**6])
+    assert status & bdfp4.DEV_BAD_SEQLEN
+
+
+def test_quantize_then_decode_end_to_end(ora, lib):
+    """GPU quantizer -> GPU decode against oracle quantizer -> oracle decode."""
+    sp, fmt = SMALL["ragged_g8_nv"]
+    wl = Workload(sp, seed=7)
+    kc, qc, vc = wl.calibration("cpu")
+    kv = bdfp4.bdfp4_calibrate(kc.cuda(), qc.cuda(), vc.cuda(), sp.H_q, sp.H_kv)
+    smooth, kg, vg = oracle_calibration(ora, wl)
+    gcache, ocache = quantize_both(ora, wl, fmt, smooth, kg, vg)
+    q = wl.queries()
+    chunk = bdfp4.bdfp4_decode_plan(wl.seq_lens, sp.H_kv, torch.cuda.get_device_properties(0).multi_processor_count)
+    out, status = run_gpu_decode(wl, gcache, q, kv, chunk)
+    ref16, _ = ora.decode(q, ocache, wl.block_table, wl.seq_lens, sp.H_kv, sp.d_v, fmt, smooth, kg, vg, sp.sm_scale,
+                          chunk, wl.num_pages)
+    max_abs, rel = compare_outputs(out_to_np(out), bf16_to_np(ref16))
+    assert status == 0 and max_abs <= MAX_ABS and rel <= REL_L2, (max_abs, rel)
