@@ -29,7 +29,10 @@ TILE_TOKENS = 128
 
 #: names of every entry point declared in include/bdfp4.h
 ENTRY_POINTS = ("bdfp4_calibrate", "bdfp4_quantize_kv", "bdfp4_quantize_q", "bdfp4_decode_plan",
-                "bdfp4_decode_workspace_size", "bdfp4_decode", "bdfp4_status_string")
+                "bdfp4_decode_workspace_size", "bdfp4_decode", "bdfp4_decode_noalloc", "bdfp4_status_string")
+
+#: size of the library's built-in scratch used by bdfp4_decode_noalloc
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class BDFP4Error(RuntimeError):
@@ -65,6 +68,8 @@ def load() -> ctypes.CDLL:
     L.bdfp4_decode_workspace_size.restype = sz
     L.bdfp4_decode.argtypes = [p, p, p, p, p, p, p, i, i, i, i, i, i, i64, i, i, kvp, f, i, p, sz, p, p, p]
     L.bdfp4_decode.restype = i
+    L.bdfp4_decode_noalloc.argtypes = [p, p, p, p, p, p, p, i, i, i, i, i, i, i64, i, i, kvp, f, i, p, p, p]
+    L.bdfp4_decode_noalloc.restype = i
     L.bdfp4_status_string.argtypes = [i]
     L.bdfp4_status_string.restype = ctypes.c_char_p
     _lib = L
@@ -205,3 +210,20 @@ def bdfp4_decode(q: torch.Tensor, cache: FP4Cache, block_table: torch.Tensor, se
 def workspace_for(B: int, H_q: int, d_v: int, max_pages_per_seq: int, chunk_tiles: int, device="cuda"):
     n = bdfp4_decode_workspace_size(B, H_q, d_v, max_pages_per_seq, chunk_tiles)
     return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def bdfp4_decode_noalloc(q: torch.Tensor, cache: FP4Cache, block_table: torch.Tensor, seq_lens: torch.Tensor,
+                         kv: KVParams, sm_scale: float, chunk_tiles: int, out: torch.Tensor, flags: int = 0,
+                         dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """bdfp4_decode for callers that cannot allocate device memory: the split
+    partials use the library's built-in scratch (NOALLOC_SCRATCH_BYTES), so no
+    workspace is passed.  Calls that overlap on the GPU race on that scratch."""
+    B, H_q, d_k = q.shape
+    c = kv._c()
+    rc = load().bdfp4_decode_noalloc(_ptr(q), _ptr(cache.k_pages), _ptr(cache.k_scales), _ptr(cache.v_pages),
+                                     _ptr(cache.v_scales), _ptr(block_table), _ptr(seq_lens), B, H_q, cache.H_kv,
+                                     d_k, cache.d_v, block_table.shape[1], cache.num_pages, cache.fmt, flags,
+                                     ctypes.byref(c), float(sm_scale), int(chunk_tiles), _ptr(out),
+                                     _ptr(dev_status), _stream(stream))
+    _check(rc, "bdfp4_decode_noalloc")
+    return out

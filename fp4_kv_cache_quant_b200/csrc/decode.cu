@@ -11,6 +11,7 @@
 // channel-major FP4 block with 16-byte loads.
 
 #include <algorithm>
+#include <mutex>
 
 #include "bdfp4_device.cuh"
 #include "host_common.h"
@@ -453,6 +454,60 @@ extern "C" int bdfp4_decode(const void* q, const void* k_pages, const void* k_sc
     if (fmt == BDFP4_NVFP4)
         return d_k == 128 ? launch_decode<BDFP4_NVFP4, 128, 128>(a, G, st) : launch_decode<BDFP4_NVFP4, 576, 512>(a, G, st);
     return d_k == 128 ? launch_decode<BDFP4_MXFP4, 128, 128>(a, G, st) : launch_decode<BDFP4_MXFP4, 576, 512>(a, G, st);
+}
+
+// ---------------------------------------------------------------- no-allocation variant
+// Scratch for the split partials of bdfp4_decode_noalloc: a file-scope device
+// array (held by every GPU that loads the library).  Host code must not pass
+// the symbol itself to a kernel -- on the host it is only a stand-in -- so its
+// device address is looked up once per device with that device current.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[BDFP4_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mutex;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (nullptr on failure).
+void* noalloc_scratch_address() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (!g_scratch_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+        g_scratch_ptr[dev] = p;
+    }
+    return g_scratch_ptr[dev];
+}
+}  // namespace
+
+extern "C" int bdfp4_decode_noalloc(const void* q, const void* k_pages, const void* k_scales, const void* v_pages,
+                                    const void* v_scales, const int32_t* block_table, const int32_t* seq_lens, int B,
+                                    int H_q, int H_kv, int d_k, int d_v, int max_pages_per_seq, int64_t num_pages,
+                                    bdfp4_fmt fmt, int flags, const bdfp4_kv_params* kv, float sm_scale,
+                                    int chunk_tiles, void* out, int32_t* dev_status, void* stream) {
+    if (B <= 0 || H_q <= 0 || d_v <= 0 || max_pages_per_seq <= 0)
+        return bdfp4_decode(q, k_pages, k_scales, v_pages, v_scales, block_table, seq_lens, B, H_q, H_kv, d_k, d_v,
+                            max_pages_per_seq, num_pages, fmt, flags, kv, sm_scale, chunk_tiles, nullptr, 0, out,
+                            dev_status, stream);
+    if (chunk_tiles <= 0) {
+        int dev = 0, sms = 148;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return BDFP4_ERR_CUDA;
+        const int ntiles = (max_pages_per_seq * kPageSlots + kTileTokens - 1) / kTileTokens;
+        const int64_t total = (int64_t)B * (H_kv > 0 ? H_kv : 1) * ntiles;
+        const int64_t chunk = std::max<int64_t>(4, (total + 16LL * sms - 1) / (16LL * sms));
+        chunk_tiles = (int)std::min<int64_t>(chunk, ntiles);
+    }
+    if (bdfp4_decode_workspace_size(B, H_q, d_v, max_pages_per_seq, chunk_tiles) > BDFP4_NOALLOC_SCRATCH_BYTES)
+        return BDFP4_ERR_WORKSPACE;
+    void* scratch = noalloc_scratch_address();
+    if (!scratch) return BDFP4_ERR_CUDA;
+    return bdfp4_decode(q, k_pages, k_scales, v_pages, v_scales, block_table, seq_lens, B, H_q, H_kv, d_k, d_v,
+                        max_pages_per_seq, num_pages, fmt, flags, kv, sm_scale, chunk_tiles, scratch,
+                        BDFP4_NOALLOC_SCRATCH_BYTES, out, dev_status, stream);
 }
 
 extern "C" const char* bdfp4_status_string(int status) {

@@ -178,6 +178,35 @@ BDFP4_API int bdfp4_decode(const void* q, const void* k_pages, const void* k_sca
                  const bdfp4_kv_params* kv, float sm_scale, int chunk_tiles, void* workspace,
                  size_t workspace_bytes, void* out, int32_t* dev_status, void* stream);
 
+/*
+ * bdfp4_decode without a caller-provided workspace.  The paper has no
+ * counterpart: this entry point exists for callers that cannot allocate
+ * device memory themselves -- for example an operator plugged into a host
+ * framework that hands it only its inputs and outputs (no workspace hook), or
+ * a latency-critical serving loop that must not call into an allocator.
+ * The split-KV partials go to a scratch array compiled into the library
+ * (a file-scope __device__ array of BDFP4_NOALLOC_SCRATCH_BYTES bytes that
+ * every GPU loading the library holds until the process exits); nothing is
+ * allocated by this call.  Arguments are those of bdfp4_decode without
+ * workspace / workspace_bytes.
+ *  - If the split plan (chunk_tiles, or the automatic plan when chunk_tiles
+ *    <= 0) needs more scratch than BDFP4_NOALLOC_SCRATCH_BYTES, the call
+ *    returns BDFP4_ERR_WORKSPACE; pass a larger chunk_tiles to fit.
+ *  - The first call on each device looks up the scratch array's device
+ *    address (cudaGetSymbolAddress) with that device current; make that first
+ *    call before any stream capture.  A failed lookup returns BDFP4_ERR_CUDA.
+ *  - All calls share the one array and it keeps the last call's contents (no
+ *    part of it needs to start at zero: every partial is written before it is
+ *    read).  Calls that overlap on the GPU -- on different streams, or from
+ *    different host threads without ordering -- race on it.
+ */
+#define BDFP4_NOALLOC_SCRATCH_BYTES (16u << 20)
+BDFP4_API int bdfp4_decode_noalloc(const void* q, const void* k_pages, const void* k_scales, const void* v_pages,
+                                   const void* v_scales, const int32_t* block_table, const int32_t* seq_lens, int B,
+                                   int H_q, int H_kv, int d_k, int d_v, int max_pages_per_seq, int64_t num_pages,
+                                   bdfp4_fmt fmt, int flags, const bdfp4_kv_params* kv, float sm_scale,
+                                   int chunk_tiles, void* out, int32_t* dev_status, void* stream);
+
 /* Human-readable text of a host return code. */
 BDFP4_API const char* bdfp4_status_string(int status);
 
