@@ -22,14 +22,14 @@ FLAG_NO_SCALE_SEARCH = 2
 FLAG_SINGLE_QUERY = 4
 FLAG_NO_UNDERFLOW = 8
 
-DEV_BAD_PAGE, DEV_BAD_SEQLEN, DEV_BAD_SLOT = 1, 2, 4
+DEV_BAD_PAGE, DEV_BAD_SEQLEN, DEV_BAD_SLOT, DEV_TIMEOUT = 1, 2, 4, 8
 
 PAGE_SLOTS = 64
 TILE_TOKENS = 128
 
 #: names of every entry point declared in include/bdfp4.h
 ENTRY_POINTS = ("bdfp4_calibrate", "bdfp4_quantize_kv", "bdfp4_quantize_q", "bdfp4_decode_plan",
-                "bdfp4_decode_workspace_size", "bdfp4_decode", "bdfp4_decode_noalloc", "bdfp4_status_string")
+                "bdfp4_decode_workspace_size", "bdfp4_decode", "bdfp4_decode_noalloc", "bdfp4_status_string", "bdfp4_last_error")
 
 #: size of the library's built-in scratch used by bdfp4_decode_noalloc
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -72,6 +72,8 @@ def load() -> ctypes.CDLL:
     L.bdfp4_decode_noalloc.restype = i
     L.bdfp4_status_string.argtypes = [i]
     L.bdfp4_status_string.restype = ctypes.c_char_p
+    L.bdfp4_last_error.argtypes = []
+    L.bdfp4_last_error.restype = ctypes.c_char_p
     _lib = L
     return L
 
@@ -80,9 +82,14 @@ def bdfp4_status_string(status: int) -> str:
     return load().bdfp4_status_string(int(status)).decode()
 
 
+def bdfp4_last_error() -> str:
+    return load().bdfp4_last_error().decode()
+
+
 def _check(rc: int, what: str):
     if rc != 0:
-        raise BDFP4Error(f"{what}: {bdfp4_status_string(rc)} ({rc})")
+        detail = f" [{bdfp4_last_error()}]" if rc == -5 else ""
+        raise BDFP4Error(f"{what}: {bdfp4_status_string(rc)} ({rc}){detail}")
 
 
 def _ptr(t: torch.Tensor | None):

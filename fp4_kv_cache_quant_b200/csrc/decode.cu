@@ -11,42 +11,15 @@
 // channel-major FP4 block with 16-byte loads.
 
 #include <algorithm>
+#include <cstdio>
 #include <mutex>
 
 #include "bdfp4_device.cuh"
 #include "host_common.h"
 #include "quant_device.cuh"
+#include "decode_common.cuh"
 
 namespace bdfp4 {
-
-struct DecodeArgs {
-    const __nv_bfloat16* q;
-    const uint8_t* k_pages;
-    const uint8_t* k_scales;
-    const uint8_t* v_pages;
-    const uint8_t* v_scales;
-    const int32_t* block_table;
-    const int32_t* seq_lens;
-    const float* smooth;
-    const float* k_gscale;
-    const float* v_gscale;
-    float* ws_o;   // [B][H_q][max_splits][d_v] unnormalised partial outputs
-    float* ws_ml;  // [B][H_q][max_splits][2]  (m in log2 units, l)
-    __nv_bfloat16* out;
-    int32_t* dev_status;
-    int B, H_q, H_kv, max_pages, flags, chunk_tiles, max_splits;
-    int64_t num_pages;
-    float sm_scale;
-};
-
-constexpr int kThreads = 128;
-constexpr float kLog2e = 1.4426950408889634f;
-
-// Splits of a sequence of N tokens.
-__host__ __device__ __forceinline__ int num_splits(int N, int chunk_tiles) {
-    const int ntiles = (N + kTileTokens - 1) / kTileTokens;
-    return (ntiles + chunk_tiles - 1) / chunk_tiles;
-}
 
 template <int FMT, int DK, int DV, int HG>
 __global__ void __launch_bounds__(kThreads) decode_fp4_kernel(const DecodeArgs a) {
@@ -374,6 +347,15 @@ extern "C" int bdfp4_decode_plan(const int32_t* host_seq_lens, int B, int H_kv, 
 
 template <int FMT, int DK, int DV>
 static int launch_decode(const DecodeArgs& a, int G, cudaStream_t st) {
+    if (DK == 128 && G <= 16) {
+        // tensor-core path (decode_tc.cu)
+        const int rc = launch_decode_tc(a, FMT, G, st);
+        if (rc != BDFP4_OK) return rc;
+        if (a.max_splits > 1)
+            merge_splits_kernel<DV><<<a.B * a.H_q, 128, 0, st>>>(a.ws_o, a.ws_ml, a.seq_lens, a.H_q, a.max_pages,
+                                                                 a.chunk_tiles, a.max_splits, a.out);
+        return launch_status();
+    }
     int hg = G >= 16 ? 16 : G;
     dim3 grid(a.max_splits, a.H_kv * (G / hg), a.B);
     switch (hg) {
@@ -509,6 +491,15 @@ extern "C" int bdfp4_decode_noalloc(const void* q, const void* k_pages, const vo
                         max_pages_per_seq, num_pages, fmt, flags, kv, sm_scale, chunk_tiles, scratch,
                         BDFP4_NOALLOC_SCRATCH_BYTES, out, dev_status, stream);
 }
+
+namespace bdfp4 {
+static thread_local char g_last_error[256] = "no CUDA error recorded";
+void record_cuda_error(cudaError_t e) {
+    snprintf(g_last_error, sizeof(g_last_error), "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+}
+}  // namespace bdfp4
+
+extern "C" const char* bdfp4_last_error(void) { return bdfp4::g_last_error; }
 
 extern "C" const char* bdfp4_status_string(int status) {
     switch (status) {

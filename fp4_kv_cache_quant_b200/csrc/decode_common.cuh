@@ -1,0 +1,43 @@
+// decode_common.cuh -- arguments and split arithmetic shared by the decode
+// kernels (CUDA-core path for MLA shapes, tcgen05 path for d = 128).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "bdfp4_device.cuh"
+
+namespace bdfp4 {
+
+struct DecodeArgs {
+    const __nv_bfloat16* q;
+    const uint8_t* k_pages;
+    const uint8_t* k_scales;
+    const uint8_t* v_pages;
+    const uint8_t* v_scales;
+    const int32_t* block_table;
+    const int32_t* seq_lens;
+    const float* smooth;
+    const float* k_gscale;
+    const float* v_gscale;
+    float* ws_o;   // [B][H_q][max_splits][d_v] unnormalised partial outputs
+    float* ws_ml;  // [B][H_q][max_splits][2]  (m in log2 units, l)
+    __nv_bfloat16* out;
+    int32_t* dev_status;
+    int B, H_q, H_kv, max_pages, flags, chunk_tiles, max_splits;
+    int64_t num_pages;
+    float sm_scale;
+};
+
+constexpr int kThreads = 128;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Splits of a sequence of N tokens.
+__host__ __device__ __forceinline__ int num_splits(int N, int chunk_tiles) {
+    const int ntiles = (N + kTileTokens - 1) / kTileTokens;
+    return (ntiles + chunk_tiles - 1) / chunk_tiles;
+}
+
+// tcgen05 decode for d_k = d_v = 128 (decode_tc.cu); returns a host status.
+int launch_decode_tc(const DecodeArgs& a, int fmt, int G, cudaStream_t st);
+
+}  // namespace bdfp4

@@ -1,0 +1,539 @@
+// decode_tc.cu -- FP4 paged decode attention on the sm_100a tensor cores
+// (BitDecoding-FP4, Article Summary: stacked query MMA on paged KV caches,
+// transposed softmax with fused probability quantization, dual-residual
+// query, underflow-aware probability scaling), for d_k = d_v = 128.
+//
+// One CTA per (sequence, KV head, split); six warps:
+//   warp 4      producer: reads the block table and bulk-copies each 128-token
+//               tile (two pages: K nibbles, K scales, V nibbles, V scales) into
+//               a 4-stage shared-memory ring (mbarrier complete_tx);
+//   warp 5      MMA issuer (one lane) and TMEM owner:
+//                 S^T[token, q-row] = K_tile . [q1; q2]^T   (M = 128 tokens,
+//                 N = 2G stacked query rows, block-scaled E2M1, fp32 in TMEM),
+//                 O^T[chan, head]  += V^T . P^T             (M = 128 channels,
+//                 N = G heads, K = the tile's tokens, one MMA per page);
+//   warps 0..3  softmax: thread t owns token t of the tile (TMEM lane t), so
+//               the softmax is transposed -- per-head maxima are warp
+//               reductions, the FP4 quantization of P (beta-token blocks) is a
+//               shuffle max over the lanes of a block, and the P codes go
+//               straight into the shared-memory operand of the PV MMA.  The
+//               same threads write the block-scale factors into TMEM and fold
+//               each tile's O into registers with the online-softmax rescale.
+// Every wait is bounded; a timeout sets BDFP4_DEV_TIMEOUT and the CTA unwinds.
+
+#include "bdfp4_device.cuh"
+#include "decode_common.cuh"
+#include "host_common.h"
+#include "quant_device.cuh"
+#include "tc_ptx.cuh"
+
+namespace bdfp4 {
+
+template <int FMT, int G>
+struct TcCfg {
+    static constexpr int B = Fmt<FMT>::beta;
+    static constexpr int DK = 128, DV = 128;
+    static constexpr int NQ = (2 * G < 8) ? 8 : 2 * G;  // N of the QK MMA (q1 rows, q2 rows, padding)
+    static constexpr int NP = (G < 8) ? 8 : G;          // N of the PV MMA
+    static constexpr int KS = DK / 64;                   // MMA K steps of QK
+    static constexpr int NS = 4;                         // pipeline stages
+    static constexpr int K_PAGE = kPageSlots * DK / 2;   // 4096
+    static constexpr int KS_PAGE = kPageSlots * DK / B;  // 512 (NVFP4) / 256 (MXFP4)
+    static constexpr int V_PAGE = DV * kPageSlots / 2;   // 4096
+    static constexpr int VS_PAGE = DV * kPageSlots / B;
+    static constexpr int OFF_K = 0;
+    static constexpr int OFF_V = 2 * K_PAGE;
+    static constexpr int OFF_KS = OFF_V + 2 * V_PAGE;
+    static constexpr int OFF_VS = OFF_KS + 2 * KS_PAGE;
+    static constexpr int STAGE = OFF_VS + 2 * VS_PAGE;
+    static constexpr int Q_BYTES = (NQ / 8) * (DK / 32) * 128;
+    static constexpr int P_PAGE = (NP / 8) * 256;
+    static constexpr int P_BUF = 2 * P_PAGE;
+    static constexpr int SPB = 64 / B;                   // scale blocks per 64 tokens / elements
+    // shared memory map
+    static constexpr int SM_STAGES = 0;
+    static constexpr int SM_Q = SM_STAGES + NS * STAGE;
+    static constexpr int SM_P = SM_Q + Q_BYTES;
+    static constexpr int SM_QSC = SM_P + 2 * P_BUF;            // [NQ][8] query scale codes
+    static constexpr int SM_PSC = SM_QSC + NQ * 8;             // [2][G][8] probability scale codes
+    static constexpr int SM_RED = SM_PSC + 2 * G * 8;          // [4][G] floats
+    static constexpr int SM_LSC = SM_RED + 4 * G * 4;          // [G] floats
+    static constexpr int SM_AMAX = SM_LSC + G * 4;             // [128] ints (row amax during the prologue)
+    static constexpr int SM_PAGES = SM_AMAX + 128 * 4;         // [NS][2] ints
+    static constexpr int SM_BARS = (SM_PAGES + NS * 2 * 4 + 7) / 8 * 8;
+    static constexpr int NBARS = 2 * NS + 8;
+    static constexpr int SM_MISC = SM_BARS + NBARS * 8;        // tmem slot, abort flags
+    static constexpr int SMEM = SM_MISC + 16;
+    // TMEM column map
+    static constexpr int T_S = 0;
+    static constexpr int T_O = 2 * NQ;
+    static constexpr int T_SFK = ((T_O + 2 * NP + 3) / 4) * 4;   // 2 x (4 per K step x KS)
+    static constexpr int T_SFV = T_SFK + 2 * 4 * KS;             // 2 x (4 per page x 2 pages)
+    // every scale-factor operand starts on a 4-column boundary (one 32-bit
+    // column per 32 rows of a 128-row chunk), B operands included
+    static constexpr int T_SFQ = T_SFV + 2 * 8;                  // KS x 4 columns
+    static constexpr int T_SFP = T_SFQ + 4 * KS;                 // 2 buffers x 2 pages x 4 columns
+    static constexpr int T_USED = T_SFP + 16;
+    static constexpr int T_ALLOC = T_USED <= 32 ? 32 : T_USED <= 64 ? 64 : T_USED <= 128 ? 128 : 256;
+};
+
+constexpr long long kWaitLimit = 1LL << 32;   // clock cycles (about 2 s)
+
+template <int FMT, int G>
+__global__ void __launch_bounds__(192, 1) decode_tc_kernel(const DecodeArgs a) {
+    using C = TcCfg<FMT, G>;
+    constexpr bool MX = FMT == BDFP4_MXFP4;
+    constexpr int B = C::B;
+    using RG = RowGeom<FMT, 128>;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t* q_op = smem + C::SM_Q;
+    uint8_t* p_op = smem + C::SM_P;
+    uint8_t* qsc = smem + C::SM_QSC;
+    uint8_t* psc = smem + C::SM_PSC;
+    float* red = reinterpret_cast<float*>(smem + C::SM_RED);
+    float* lsc = reinterpret_cast<float*>(smem + C::SM_LSC);
+    int* row_amax = reinterpret_cast<int*>(smem + C::SM_AMAX);
+    int* page_ids = reinterpret_cast<int*>(smem + C::SM_PAGES);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SM_BARS);
+    uint64_t* full = bars;                    // [NS] producer -> consumers
+    uint64_t* empty = bars + C::NS;           // [NS] PV done -> producer
+    uint64_t* sfk_ready = bars + 2 * C::NS;   // [2] K scale factors in TMEM -> MMA
+    uint64_t* s_full = sfk_ready + 2;         // [2] QK done -> softmax
+    uint64_t* p_ready = s_full + 2;           // [2] P + scale factors ready -> MMA
+    uint64_t* o_full = p_ready + 2;           // [2] PV done -> softmax
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SM_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::SM_MISC + 4);   // any role gave up
+    volatile int* sm_abort = reinterpret_cast<volatile int*>(smem + C::SM_MISC + 8);     // softmax warps' decision
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+    const int h0 = hk * G;
+
+    int N = a.seq_lens[b];
+    if (N < 0 || N > a.max_pages * kPageSlots) {
+        if (tid == 0 && split == 0) set_status(a.dev_status, BDFP4_DEV_BAD_SEQLEN);
+        N = 0;
+    }
+    const int ntiles = (N + kTileTokens - 1) / kTileTokens;
+    const int nspl = (ntiles + a.chunk_tiles - 1) / a.chunk_tiles;
+    if (split > 0 && split >= nspl) return;
+    if (N == 0) {
+        for (int i = tid; i < G * C::DV; i += blockDim.x)
+            a.out[((int64_t)b * a.H_q + h0 + i / C::DV) * C::DV + i % C::DV] = __float2bfloat16(0.0f);
+        return;
+    }
+    const int tile0 = split * a.chunk_tiles;
+    const int n = min(a.chunk_tiles, ntiles - tile0);   // tiles of this split (>= 1)
+
+    if (tid == 0) {
+        for (int s = 0; s < C::NS; ++s) {
+            tc::mbar_init(&full[s], 1);
+            tc::mbar_init(&empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(&sfk_ready[i], 4);
+            tc::mbar_init(&s_full[i], 1);
+            tc::mbar_init(&p_ready[i], 4);
+            tc::mbar_init(&o_full[i], 1);
+        }
+        *abort_flag = 0;
+        *sm_abort = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == 5) {
+        tc::tmem_alloc(tmem_slot, C::T_ALLOC);
+        tc::tmem_relinquish();
+    }
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+
+    if (warp == 4) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            for (int j = 0; j < n; ++j) {
+                const int s = j % C::NS;
+                if (j >= C::NS && !tc::mbar_wait(&empty[s], ((j / C::NS) - 1) & 1, abort_flag, kWaitLimit)) {
+                    *abort_flag = 1;
+                    break;
+                }
+                const int tile = tile0 + j;
+                int pg[2];
+                uint32_t bytes = 0;
+                for (int p = 0; p < 2; ++p) {
+                    pg[p] = -1;
+                    const int pi = tile * 2 + p;
+                    if (pi * kPageSlots < N) {
+                        const int v = a.block_table[(int64_t)b * a.max_pages + pi];
+                        if (v >= 0 && v < a.num_pages) {
+                            pg[p] = v;
+                            bytes += C::K_PAGE + C::KS_PAGE + C::V_PAGE + C::VS_PAGE;
+                        } else {
+                            set_status(a.dev_status, BDFP4_DEV_BAD_PAGE);
+                        }
+                    }
+                    page_ids[s * 2 + p] = pg[p];
+                }
+                tc::mbar_arrive_expect_tx(&full[s], bytes);
+                uint8_t* st = smem + C::SM_STAGES + s * C::STAGE;
+                for (int p = 0; p < 2; ++p) {
+                    if (pg[p] < 0) continue;
+                    const int64_t ph = (int64_t)pg[p] * a.H_kv + hk;
+                    tc::bulk_g2s(st + C::OFF_K + p * C::K_PAGE, a.k_pages + ph * C::K_PAGE, C::K_PAGE, &full[s]);
+                    tc::bulk_g2s(st + C::OFF_KS + p * C::KS_PAGE, a.k_scales + ph * C::KS_PAGE, C::KS_PAGE, &full[s]);
+                    tc::bulk_g2s(st + C::OFF_V + p * C::V_PAGE, a.v_pages + ph * C::V_PAGE, C::V_PAGE, &full[s]);
+                    tc::bulk_g2s(st + C::OFF_VS + p * C::VS_PAGE, a.v_scales + ph * C::VS_PAGE, C::VS_PAGE, &full[s]);
+                }
+            }
+        }
+    } else if (warp == 5) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = tc::idesc_fp4(C::NQ, MX);
+            constexpr uint32_t idesc_pv = tc::idesc_fp4(C::NP, MX);
+            const uint32_t q_addr = tc::smem_u32(q_op);
+            const uint32_t p_addr = tc::smem_u32(p_op);
+            const uint32_t st_addr = tc::smem_u32(smem + C::SM_STAGES);
+            auto issue_qk = [&](int j) -> bool {
+                const int s = j % C::NS, buf = j & 1;
+                if (!tc::mbar_wait(&full[s], (j / C::NS) & 1, abort_flag, kWaitLimit)) return false;
+                if (!tc::mbar_wait(&sfk_ready[buf], (j >> 1) & 1, abort_flag, kWaitLimit)) return false;
+                tc::tc_fence_after();
+                const uint32_t kt = st_addr + s * C::STAGE + C::OFF_K;
+#pragma unroll
+                for (int ks = 0; ks < C::KS; ++ks) {
+                    tc::mma_fp4<MX>(tbase + C::T_S + buf * C::NQ, tc::smem_desc(kt + ks * 256, 128, 512),
+                                    tc::smem_desc(q_addr + ks * 256, 128, 512), idesc_qk,
+                                    tbase + C::T_SFK + buf * 4 * C::KS + ks * 4, tbase + C::T_SFQ + ks * 4, ks > 0);
+                }
+                tc::mma_commit(&s_full[buf]);
+                return true;
+            };
+            bool ok = issue_qk(0);
+            for (int j = 0; ok && j < n; ++j) {
+                if (j + 1 < n && !(ok = issue_qk(j + 1))) break;
+                const int s = j % C::NS, buf = j & 1;
+                if (!(ok = tc::mbar_wait(&p_ready[buf], (j >> 1) & 1, abort_flag, kWaitLimit))) break;
+                tc::tc_fence_after();
+                const uint32_t vt = st_addr + s * C::STAGE + C::OFF_V;
+#pragma unroll
+                for (int p = 0; p < 2; ++p) {
+                    tc::mma_fp4<MX>(tbase + C::T_O + buf * C::NP, tc::smem_desc(vt + p * C::V_PAGE, 128, 256),
+                                    tc::smem_desc(p_addr + buf * C::P_BUF + p * C::P_PAGE, 128, 256), idesc_pv,
+                                    tbase + C::T_SFV + buf * 8 + p * 4, tbase + C::T_SFP + (buf * 2 + p) * 4, p > 0);
+                }
+                tc::mma_commit(&o_full[buf]);
+                tc::mma_commit(&empty[s]);
+            }
+            if (!ok) *abort_flag = 1;
+        }
+    } else {
+        // ------------------------------------------------------------ softmax warps 0..3
+        const uint32_t tq = tbase + ((uint32_t)(32 * warp) << 16);   // this warp's TMEM lane quadrant
+        const bool hadamard = !(a.flags & BDFP4_FLAG_NO_HADAMARD);
+        const bool dual = !(a.flags & BDFP4_FLAG_SINGLE_QUERY);
+        const float alpha = (FMT == BDFP4_NVFP4 && !(a.flags & BDFP4_FLAG_NO_UNDERFLOW)) ? kAlphaNV : 1.0f;
+        bool bad = false;
+
+        // query prologue: transform + dual-residual FP4 straight into the QK operand
+        for (int i = tid; i < C::Q_BYTES / 16; i += 128) reinterpret_cast<uint4*>(q_op)[i] = make_uint4(0, 0, 0, 0);
+        for (int i = tid; i < C::NQ * 8; i += 128) qsc[i] = 0;
+        row_amax[tid] = 0;
+        tc::named_bar_sync(1, 128);
+        {
+            const int j = tid % RG::rt, r = tid / RG::rt;
+            const bool active = r < G && j < RG::tpr;
+            float x[B];
+            if (active) {
+                load_bf16_block<B>(a.q + ((int64_t)b * a.H_q + h0 + r) * C::DK, j * B, x);
+            } else {
+#pragma unroll
+                for (int i = 0; i < B; ++i) x[i] = 0.0f;
+            }
+            transform_block<FMT, 128, false>(x, a.smooth + (int64_t)hk * C::DK, j, hadamard);
+            if (active) atomicMax(&row_amax[r], __float_as_int(block_amax<B>(x)));
+            tc::named_bar_sync(1, 128);
+            if (active) {
+                const float amax = __int_as_float(row_amax[r]);
+                const float gq = FMT == BDFP4_NVFP4 ? (amax > 0.0f ? __fdiv_rn(amax, 2688.0f) : 1.0f) : 1.0f;
+                uint32_t c1, c2, p1[B / 8], p2[B / 8];
+                quantize_query_block<FMT, 128>(x, gq, dual, c1, p1, c2, p2);
+                // rows: q1 of head r -> r, q2 -> G + r; element e -> chunk e/32, byte (e%32)/2
+                const int e0 = j * B;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    const int row = half ? G + r : r;
+                    const uint32_t* pk = half ? p2 : p1;
+                    uint8_t* dst = q_op + (row / 8) * 512 + (e0 / 32) * 128 + (row % 8) * 16 + (e0 % 32) / 2;
+                    if constexpr (B == 16) *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
+                    else *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    qsc[row * 8 + j] = (uint8_t)(half ? c2 : c1);
+                }
+                if (j == 0) {
+                    const float gk = FMT == BDFP4_NVFP4 ? a.k_gscale[hk] : 1.0f;
+                    lsc[r] = a.sm_scale * gq * gk * kLog2e;
+                }
+            }
+            tc::fence_proxy_async_smem();
+            tc::named_bar_sync(1, 128);
+        }
+        // query scale factors (SFB of QK): lane n <- row n, one column per K step, all quadrants
+        {
+            uint32_t col[C::KS];
+#pragma unroll
+            for (int ks = 0; ks < C::KS; ++ks) {
+                uint32_t v = 0;
+                if (lane < C::NQ) {
+                    if constexpr (B == 16) v = *reinterpret_cast<const uint32_t*>(qsc + lane * 8 + ks * 4);
+                    else v = (uint32_t)qsc[lane * 8 + ks * 2] | ((uint32_t)qsc[lane * 8 + ks * 2 + 1] << 8);
+                }
+                col[ks] = v;
+            }
+#pragma unroll
+            for (int ks = 0; ks < C::KS; ++ks) tc::tmem_st4(tq + C::T_SFQ + ks * 4, col[ks], 0u, 0u, 0u);
+        }
+        // K scale factors of tile j (SFA of QK): TMEM lane i, column m1 (+4 per K step) <- row 32*m1 + i
+        auto write_sfk = [&](int j) -> bool {
+            const int s = j % C::NS;
+            if (!tc::mbar_wait(&full[s], (j / C::NS) & 1, abort_flag, kWaitLimit)) return false;
+            const uint8_t* ks = smem + C::SM_STAGES + s * C::STAGE + C::OFF_KS;
+            uint32_t v[8];
+            if constexpr (B == 16) {
+                const uint4 p0 = *reinterpret_cast<const uint4*>(ks + 16 * lane);
+                const uint4 p1 = *reinterpret_cast<const uint4*>(ks + C::KS_PAGE + 16 * lane);
+                v[0] = p0.x; v[1] = p0.y; v[2] = p1.x; v[3] = p1.y;
+                v[4] = p0.z; v[5] = p0.w; v[6] = p1.z; v[7] = p1.w;
+            } else {
+                const uint2 p0 = *reinterpret_cast<const uint2*>(ks + 8 * lane);
+                const uint2 p1 = *reinterpret_cast<const uint2*>(ks + C::KS_PAGE + 8 * lane);
+                v[0] = p0.x & 0xffffu; v[1] = p0.x >> 16; v[2] = p1.x & 0xffffu; v[3] = p1.x >> 16;
+                v[4] = p0.y & 0xffffu; v[5] = p0.y >> 16; v[6] = p1.y & 0xffffu; v[7] = p1.y >> 16;
+            }
+            tc::tmem_st8(tq + C::T_SFK + (j & 1) * 4 * C::KS, v);
+            tc::tmem_wait_st();
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&sfk_ready[j & 1]);
+            return true;
+        };
+        bad |= !write_sfk(0);
+
+        float m_run[G], l_part[G], o_acc[G], corr_prev[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            m_run[g] = -INFINITY;
+            l_part[g] = 0.0f;
+            o_acc[g] = 0.0f;
+            corr_prev[g] = 0.0f;
+        }
+        const int tok_in_tile = 32 * warp + lane;
+        auto fold_o = [&](int j) -> bool {
+            if (!tc::mbar_wait(&o_full[j & 1], (j >> 1) & 1, abort_flag, kWaitLimit)) return false;
+            tc::tc_fence_after();
+            uint32_t ov[C::NP];
+            tc::tmem_ld<C::NP>(tq + C::T_O + (j & 1) * C::NP, ov);
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int g = 0; g < G; ++g) o_acc[g] = o_acc[g] * corr_prev[g] + __uint_as_float(ov[g]);
+            return true;
+        };
+
+        for (int j = 0; j < n; ++j) {
+            const int s = j % C::NS, buf = j & 1, tile = tile0 + j;
+            if (j + 1 < n) bad |= !write_sfk(j + 1);
+            // logits of this thread's token
+            if (!tc::mbar_wait(&s_full[buf], (j >> 1) & 1, abort_flag, kWaitLimit)) bad = true;
+            tc::tc_fence_after();
+            uint32_t sr[C::NQ];
+            tc::tmem_ld<C::NQ>(tq + C::T_S + buf * C::NQ, sr);
+            tc::tmem_wait_ld();
+            const int token = tile * kTileTokens + tok_in_tile;
+            const bool valid = token < N && page_ids[s * 2 + (warp >> 1)] >= 0;
+            float sv[G];
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+                sv[g] = valid ? (__uint_as_float(sr[g]) + __uint_as_float(sr[G + g])) * lsc[g] : -INFINITY;
+            // per-head tile maximum: warp reduction, then across the four warps
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                float mx = sv[g];
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                if (lane == 0) red[warp * G + g] = mx;
+            }
+            // one decision for all four warps: sm_abort is written only before this barrier
+            if (bad || *abort_flag) *sm_abort = 1;
+            tc::named_bar_sync(1, 128);
+            if (*sm_abort) break;
+            float corr[G];
+            uint8_t* pb = p_op + buf * C::P_BUF + (warp >> 1) * C::P_PAGE + (warp & 1) * 128 + (lane >> 3) * 4;
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const float mt = fmaxf(fmaxf(red[g], red[G + g]), fmaxf(red[2 * G + g], red[3 * G + g]));
+                const float mn = fmaxf(m_run[g], mt);
+                corr[g] = exp2f(m_run[g] - mn);   // 0 on the split's first tile
+                m_run[g] = mn;
+                const float p = valid ? exp2f(sv[g] - mn) : 0.0f;
+                l_part[g] = l_part[g] * corr[g] + p;
+                // fused FP4 quantization of p over beta-token blocks (lanes)
+                const float y = p * alpha;
+                float am = y;
+#pragma unroll
+                for (int off = B / 2; off > 0; off >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
+                uint32_t c;
+                float sigma;
+                if constexpr (FMT == BDFP4_NVFP4) {
+                    c = am > 0.0f ? e4m3_encode(__fdiv_rn(am, 6.0f)) : 0u;
+                    sigma = e4m3_value(c);
+                } else {
+                    c = mx_scale_code(am);
+                    sigma = e8m0_value(c);
+                }
+                const uint32_t e = sigma > 0.0f ? e2m1_encode(__fdiv_rn(y, sigma)) : 0u;
+                uint32_t word = e << (4 * (lane & 7));
+                word |= __shfl_xor_sync(0xffffffffu, word, 1);
+                word |= __shfl_xor_sync(0xffffffffu, word, 2);
+                word |= __shfl_xor_sync(0xffffffffu, word, 4);
+                if ((lane & 7) == 0) *reinterpret_cast<uint32_t*>(pb + (g >> 3) * 256 + (g & 7) * 16) = word;
+                if ((lane & (B - 1)) == 0) psc[(buf * G + g) * 8 + tok_in_tile / B] = (uint8_t)c;
+            }
+            tc::fence_proxy_async_smem();
+            tc::named_bar_sync(1, 128);
+            // P scale factors (SFB of PV): lane g <- head g, one column per page
+            {
+                uint32_t c0 = 0, c1 = 0;
+                if (lane < G) {
+                    const uint8_t* ps = psc + (buf * G + lane) * 8;
+                    if constexpr (B == 16) {
+                        c0 = *reinterpret_cast<const uint32_t*>(ps);
+                        c1 = *reinterpret_cast<const uint32_t*>(ps + 4);
+                    } else {
+                        c0 = (uint32_t)ps[0] | ((uint32_t)ps[1] << 8);
+                        c1 = (uint32_t)ps[2] | ((uint32_t)ps[3] << 8);
+                    }
+                }
+                tc::tmem_st4(tq + C::T_SFP + buf * 8, c0, 0u, 0u, 0u);
+                tc::tmem_st4(tq + C::T_SFP + buf * 8 + 4, c1, 0u, 0u, 0u);
+            }
+            // V scale factors (SFA of PV): lane i, column m1 (+4 per page) <- channel 32*m1 + i;
+            // blocks past the sequence end are zeroed (never multiplied by garbage)
+            {
+                const uint8_t* vs = smem + C::SM_STAGES + s * C::STAGE + C::OFF_VS;
+                uint32_t v[8];
+#pragma unroll
+                for (int p = 0; p < 2; ++p) {
+                    const int t0 = tile * kTileTokens + p * kPageSlots;
+                    int nvb = page_ids[s * 2 + p] >= 0 ? (N - t0 + B - 1) / B : 0;
+                    nvb = nvb < 0 ? 0 : (nvb > C::SPB ? C::SPB : nvb);
+                    if constexpr (B == 16) {
+                        const uint32_t mask = nvb >= 4 ? 0xffffffffu : ((1u << (8 * nvb)) - 1u);
+                        const uint4 w = *reinterpret_cast<const uint4*>(vs + p * C::VS_PAGE + 16 * lane);
+                        v[p * 4 + 0] = w.x & mask;
+                        v[p * 4 + 1] = w.y & mask;
+                        v[p * 4 + 2] = w.z & mask;
+                        v[p * 4 + 3] = w.w & mask;
+                    } else {
+                        const uint32_t mask = nvb >= 2 ? 0xffffu : ((1u << (8 * nvb)) - 1u);
+                        const uint2 w = *reinterpret_cast<const uint2*>(vs + p * C::VS_PAGE + 8 * lane);
+                        v[p * 4 + 0] = w.x & mask;
+                        v[p * 4 + 1] = (w.x >> 16) & mask;
+                        v[p * 4 + 2] = w.y & mask;
+                        v[p * 4 + 3] = (w.y >> 16) & mask;
+                    }
+                }
+                tc::tmem_st8(tq + C::T_SFV + buf * 8, v);
+            }
+            tc::tmem_wait_st();
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&p_ready[buf]);
+            // fold the previous tile's O into registers
+            if (j >= 1) bad |= !fold_o(j - 1);
+#pragma unroll
+            for (int g = 0; g < G; ++g) corr_prev[g] = corr[g];
+        }
+        if (!*sm_abort && !fold_o(n - 1)) bad = true;
+        if (bad || *abort_flag) *sm_abort = 1;
+
+        // ------------------------------------------------------------ epilogue (thread = channel)
+        tc::named_bar_sync(1, 128);
+        if (*sm_abort) *abort_flag = 1;
+        if (!*sm_abort) {
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                float v = l_part[g];
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+                if (lane == 0) red[warp * G + g] = v;
+            }
+            tc::named_bar_sync(1, 128);
+            const float vg = FMT == BDFP4_NVFP4 ? a.v_gscale[hk] : 1.0f;
+            const float oscale = vg / alpha;
+            const int ch = tok_in_tile;
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const float l = red[g] + red[G + g] + red[2 * G + g] + red[3 * G + g];
+                const int64_t row = (int64_t)b * a.H_q + h0 + g;
+                if (nspl == 1) {
+                    a.out[row * C::DV + ch] = __float2bfloat16(l > 0.0f ? o_acc[g] * oscale / l : 0.0f);
+                } else {
+                    a.ws_o[(row * a.max_splits + split) * C::DV + ch] = o_acc[g] * oscale;
+                    if (tid == 0) {
+                        a.ws_ml[(row * a.max_splits + split) * 2 + 0] = m_run[g];
+                        a.ws_ml[(row * a.max_splits + split) * 2 + 1] = l;
+                    }
+                }
+            }
+        }
+    }
+
+    tc::tc_fence_before();
+    __syncthreads();
+    if (*abort_flag && tid == 0) set_status(a.dev_status, BDFP4_DEV_TIMEOUT);
+    if (warp == 5) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tbase, C::T_ALLOC);
+    }
+}
+
+template <int FMT, int G>
+static int launch_tc(const DecodeArgs& a, cudaStream_t st) {
+    using C = TcCfg<FMT, G>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        const cudaError_t e =
+            cudaFuncSetAttribute(decode_tc_kernel<FMT, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        if (e != cudaSuccess) {
+            record_cuda_error(e);
+            return BDFP4_ERR_CUDA;
+        }
+        attr_set = true;
+    }
+    dim3 grid(a.max_splits, a.H_kv, a.B);
+    decode_tc_kernel<FMT, G><<<grid, 192, C::SMEM, st>>>(a);
+    return launch_status();
+}
+
+int launch_decode_tc(const DecodeArgs& a, int fmt, int G, cudaStream_t st) {
+    if (fmt == BDFP4_NVFP4) {
+        switch (G) {
+            case 1: return launch_tc<BDFP4_NVFP4, 1>(a, st);
+            case 2: return launch_tc<BDFP4_NVFP4, 2>(a, st);
+            case 4: return launch_tc<BDFP4_NVFP4, 4>(a, st);
+            case 8: return launch_tc<BDFP4_NVFP4, 8>(a, st);
+            case 16: return launch_tc<BDFP4_NVFP4, 16>(a, st);
+        }
+    } else {
+        switch (G) {
+            case 1: return launch_tc<BDFP4_MXFP4, 1>(a, st);
+            case 2: return launch_tc<BDFP4_MXFP4, 2>(a, st);
+            case 4: return launch_tc<BDFP4_MXFP4, 4>(a, st);
+            case 8: return launch_tc<BDFP4_MXFP4, 8>(a, st);
+            case 16: return launch_tc<BDFP4_MXFP4, 16>(a, st);
+        }
+    }
+    return BDFP4_ERR_UNSUPPORTED;
+}
+
+}  // namespace bdfp4

@@ -79,6 +79,7 @@ typedef enum { BDFP4_NVFP4 = 0, BDFP4_MXFP4 = 1 } bdfp4_fmt;
 #define BDFP4_DEV_BAD_PAGE 1       /* block_table entry outside [0, num_pages)     */
 #define BDFP4_DEV_BAD_SEQLEN 2     /* seq_len < 0 or > max_pages_per_seq * 64      */
 #define BDFP4_DEV_BAD_SLOT 4       /* slot_mapping entry >= num_pages * 64         */
+#define BDFP4_DEV_TIMEOUT 8        /* a bounded in-kernel wait gave up (the CTA unwound) */
 
 /* flags (ablation arms of the method; 0 = the method as described) */
 #define BDFP4_FLAG_NO_HADAMARD 1     /* no rotation of K and q (must match between quantize and decode) */
@@ -209,6 +210,11 @@ BDFP4_API int bdfp4_decode_noalloc(const void* q, const void* k_pages, const voi
 
 /* Human-readable text of a host return code. */
 BDFP4_API const char* bdfp4_status_string(int status);
+
+/* Name and text of the last CUDA error this thread's calls into the library
+ * met (the detail behind BDFP4_ERR_CUDA); the string stays valid until the
+ * thread's next failing call. */
+BDFP4_API const char* bdfp4_last_error(void);
 
 #ifdef __cplusplus
 }
