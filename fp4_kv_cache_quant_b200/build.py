@@ -28,15 +28,17 @@ def _stale() -> bool:
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
-    if not force and not _stale():
+def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None, out: str | None = None) -> str:
+    """Compile csrc/*.cu into libbdfp4.so (or `out`) unless it is up to date."""
+    target = out or LIB
+    if not force and out is None and not _stale():
         return LIB
-    cmd = [NVCC, *FLAGS, *(extra or []), "-o", LIB + ".tmp", *sources()]
+    cmd = [NVCC, *FLAGS, *(extra or []), "-o", target + ".tmp", *sources()]
     if verbose:
         print(" ".join(cmd), flush=True)
     subprocess.run(cmd, check=True)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(target + ".tmp", target)
+    return target
 
 
 if __name__ == "__main__":

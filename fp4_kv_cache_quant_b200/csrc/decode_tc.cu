@@ -27,6 +27,10 @@
 #include "quant_device.cuh"
 #include "tc_ptx.cuh"
 
+#ifndef BDFP4_TC_STAGES
+#define BDFP4_TC_STAGES 3
+#endif
+
 namespace bdfp4 {
 
 template <int FMT, int G>
@@ -36,7 +40,7 @@ struct TcCfg {
     static constexpr int NQ = (2 * G < 8) ? 8 : 2 * G;  // N of the QK MMA (q1 rows, q2 rows, padding)
     static constexpr int NP = (G < 8) ? 8 : G;          // N of the PV MMA
     static constexpr int KS = DK / 64;                   // MMA K steps of QK
-    static constexpr int NS = 4;                         // pipeline stages
+    static constexpr int NS = BDFP4_TC_STAGES;           // pipeline stages
     static constexpr int K_PAGE = kPageSlots * DK / 2;   // 4096
     static constexpr int KS_PAGE = kPageSlots * DK / B;  // 512 (NVFP4) / 256 (MXFP4)
     static constexpr int V_PAGE = DV * kPageSlots / 2;   // 4096
@@ -55,9 +59,9 @@ struct TcCfg {
     static constexpr int SM_Q = SM_STAGES + NS * STAGE;
     static constexpr int SM_P = SM_Q + Q_BYTES;
     static constexpr int SM_QSC = SM_P + 2 * P_BUF;            // [NQ][8] query scale codes
-    static constexpr int SM_PSC = SM_QSC + NQ * 8;             // [2][G][8] probability scale codes
-    static constexpr int SM_RED = SM_PSC + 2 * G * 8;          // [4][G] floats
-    static constexpr int SM_LSC = SM_RED + 4 * G * 4;          // [G] floats
+    static constexpr int SM_PSF = (SM_QSC + NQ * 8 + 127) / 128 * 128;   // [2 buf][2 page][32 rows][16 B] P scales
+    static constexpr int SM_RED = SM_PSF + 2 * 2 * 512;                  // [2][G][4] per-warp maxima (floats)
+    static constexpr int SM_LSC = SM_RED + 2 * G * 4 * 4;               // [G] floats
     static constexpr int SM_AMAX = SM_LSC + G * 4;             // [128] ints (row amax during the prologue)
     static constexpr int SM_PAGES = SM_AMAX + 128 * 4;         // [NS][2] ints
     static constexpr int SM_BARS = (SM_PAGES + NS * 2 * 4 + 7) / 8 * 8;
@@ -75,6 +79,13 @@ struct TcCfg {
     static constexpr int T_SFP = T_SFQ + 4 * KS;                 // 2 buffers x 2 pages x 4 columns
     static constexpr int T_USED = T_SFP + 16;
     static constexpr int T_ALLOC = T_USED <= 32 ? 32 : T_USED <= 64 ? 64 : T_USED <= 128 ? 128 : 256;
+    // TMEM holds 512 columns per SM; request enough shared memory that one CTA
+    // more than TMEM can serve never becomes resident (it would only wait in
+    // tcgen05.alloc): with k = 512 / T_ALLOC CTAs per SM, (k + 1) * (smem + 1 KB)
+    // must exceed the 228 KB of an SM
+    static constexpr int MAX_CTAS = 512 / T_ALLOC;
+    static constexpr int SMEM_MIN = 233472 / (MAX_CTAS + 1) - 1024 + 16;
+    static constexpr int SMEM_LAUNCH = SMEM > SMEM_MIN ? SMEM : SMEM_MIN;
 };
 
 constexpr long long kWaitLimit = 1LL << 32;   // clock cycles (about 2 s)
@@ -89,7 +100,7 @@ __global__ void __launch_bounds__(192, 1) decode_tc_kernel(const DecodeArgs a) {
     uint8_t* q_op = smem + C::SM_Q;
     uint8_t* p_op = smem + C::SM_P;
     uint8_t* qsc = smem + C::SM_QSC;
-    uint8_t* psc = smem + C::SM_PSC;
+    uint8_t* psf = smem + C::SM_PSF;
     float* red = reinterpret_cast<float*>(smem + C::SM_RED);
     float* lsc = reinterpret_cast<float*>(smem + C::SM_LSC);
     int* row_amax = reinterpret_cast<int*>(smem + C::SM_AMAX);
@@ -151,42 +162,61 @@ __global__ void __launch_bounds__(192, 1) decode_tc_kernel(const DecodeArgs a) {
 
     if (warp == 4) {
         // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            for (int j = 0; j < n; ++j) {
-                const int s = j % C::NS;
-                if (j >= C::NS && !tc::mbar_wait(&empty[s], ((j / C::NS) - 1) & 1, abort_flag, kWaitLimit)) {
-                    *abort_flag = 1;
-                    break;
-                }
-                const int tile = tile0 + j;
-                int pg[2];
-                uint32_t bytes = 0;
+        // The warp reads the page ids of 32 tiles at once (one tile per lane),
+        // so the dependent block-table load is off the per-tile path; lane 0
+        // then waits for a free stage and issues the tile's bulk copies.
+        bool ok = true;
+        for (int j0 = 0; ok && j0 < n; j0 += 32) {
+            int pg_l[2] = {-1, -1};
+            if (j0 + lane < n) {
+                const int tile = tile0 + j0 + lane;
+#pragma unroll
                 for (int p = 0; p < 2; ++p) {
-                    pg[p] = -1;
                     const int pi = tile * 2 + p;
                     if (pi * kPageSlots < N) {
                         const int v = a.block_table[(int64_t)b * a.max_pages + pi];
-                        if (v >= 0 && v < a.num_pages) {
-                            pg[p] = v;
-                            bytes += C::K_PAGE + C::KS_PAGE + C::V_PAGE + C::VS_PAGE;
-                        } else {
-                            set_status(a.dev_status, BDFP4_DEV_BAD_PAGE);
-                        }
+                        if (v >= 0 && v < a.num_pages) pg_l[p] = v;
+                        else set_status(a.dev_status, BDFP4_DEV_BAD_PAGE);
                     }
-                    page_ids[s * 2 + p] = pg[p];
-                }
-                tc::mbar_arrive_expect_tx(&full[s], bytes);
-                uint8_t* st = smem + C::SM_STAGES + s * C::STAGE;
-                for (int p = 0; p < 2; ++p) {
-                    if (pg[p] < 0) continue;
-                    const int64_t ph = (int64_t)pg[p] * a.H_kv + hk;
-                    tc::bulk_g2s(st + C::OFF_K + p * C::K_PAGE, a.k_pages + ph * C::K_PAGE, C::K_PAGE, &full[s]);
-                    tc::bulk_g2s(st + C::OFF_KS + p * C::KS_PAGE, a.k_scales + ph * C::KS_PAGE, C::KS_PAGE, &full[s]);
-                    tc::bulk_g2s(st + C::OFF_V + p * C::V_PAGE, a.v_pages + ph * C::V_PAGE, C::V_PAGE, &full[s]);
-                    tc::bulk_g2s(st + C::OFF_VS + p * C::VS_PAGE, a.v_scales + ph * C::VS_PAGE, C::VS_PAGE, &full[s]);
                 }
             }
+            const int kmax = min(32, n - j0);
+            for (int k = 0; k < kmax; ++k) {
+                const int j = j0 + k;
+                const int pg0 = __shfl_sync(0xffffffffu, pg_l[0], k);
+                const int pg1 = __shfl_sync(0xffffffffu, pg_l[1], k);
+                if (lane == 0) {
+                    const int s = j % C::NS;
+                    if (j >= C::NS && !tc::mbar_wait(&empty[s], ((j / C::NS) - 1) & 1, abort_flag, kWaitLimit)) {
+                        ok = false;
+                    } else {
+                        const int pg[2] = {pg0, pg1};
+                        uint32_t bytes = 0;
+#pragma unroll
+                        for (int p = 0; p < 2; ++p) {
+                            page_ids[s * 2 + p] = pg[p];
+                            if (pg[p] >= 0) bytes += C::K_PAGE + C::KS_PAGE + C::V_PAGE + C::VS_PAGE;
+                        }
+                        tc::mbar_arrive_expect_tx(&full[s], bytes);
+                        uint8_t* st = smem + C::SM_STAGES + s * C::STAGE;
+#pragma unroll
+                        for (int p = 0; p < 2; ++p) {
+                            if (pg[p] < 0) continue;
+                            const int64_t ph = (int64_t)pg[p] * a.H_kv + hk;
+                            tc::bulk_g2s(st + C::OFF_K + p * C::K_PAGE, a.k_pages + ph * C::K_PAGE, C::K_PAGE, &full[s]);
+                            tc::bulk_g2s(st + C::OFF_KS + p * C::KS_PAGE, a.k_scales + ph * C::KS_PAGE, C::KS_PAGE,
+                                         &full[s]);
+                            tc::bulk_g2s(st + C::OFF_V + p * C::V_PAGE, a.v_pages + ph * C::V_PAGE, C::V_PAGE, &full[s]);
+                            tc::bulk_g2s(st + C::OFF_VS + p * C::VS_PAGE, a.v_scales + ph * C::VS_PAGE, C::VS_PAGE,
+                                         &full[s]);
+                        }
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+            }
         }
+        if (!ok && lane == 0) *abort_flag = 1;
     } else if (warp == 5) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -195,6 +225,7 @@ __global__ void __launch_bounds__(192, 1) decode_tc_kernel(const DecodeArgs a) {
             const uint32_t q_addr = tc::smem_u32(q_op);
             const uint32_t p_addr = tc::smem_u32(p_op);
             const uint32_t st_addr = tc::smem_u32(smem + C::SM_STAGES);
+            const uint32_t psf_addr = tc::smem_u32(psf);
             auto issue_qk = [&](int j) -> bool {
                 const int s = j % C::NS, buf = j & 1;
                 if (!tc::mbar_wait(&full[s], (j / C::NS) & 1, abort_flag, kWaitLimit)) return false;
@@ -217,6 +248,16 @@ __global__ void __launch_bounds__(192, 1) decode_tc_kernel(const DecodeArgs a) {
                 if (!(ok = tc::mbar_wait(&p_ready[buf], (j >> 1) & 1, abort_flag, kWaitLimit))) break;
                 tc::tc_fence_after();
                 const uint32_t vt = st_addr + s * C::STAGE + C::OFF_V;
+                // scale factors of P (written by the softmax warps) and, for NVFP4, of V
+                // (the page's scale block is already in the 32 x 16-byte copy layout)
+#pragma unroll
+                for (int p = 0; p < 2; ++p) {
+                    tc::tmem_cp_32x128b_x4(tbase + C::T_SFP + (buf * 2 + p) * 4,
+                                           tc::smem_desc(psf_addr + (buf * 2 + p) * 512, 128, 128));
+                    if constexpr (!MX)
+                        tc::tmem_cp_32x128b_x4(tbase + C::T_SFV + buf * 8 + p * 4,
+                                               tc::smem_desc(vt - C::OFF_V + C::OFF_VS + p * C::VS_PAGE, 128, 128));
+                }
 #pragma unroll
                 for (int p = 0; p < 2; ++p) {
                     tc::mma_fp4<MX>(tbase + C::T_O + buf * C::NP, tc::smem_desc(vt + p * C::V_PAGE, 128, 256),
@@ -239,6 +280,7 @@ __global__ void __launch_bounds__(192, 1) decode_tc_kernel(const DecodeArgs a) {
         // query prologue: transform + dual-residual FP4 straight into the QK operand
         for (int i = tid; i < C::Q_BYTES / 16; i += 128) reinterpret_cast<uint4*>(q_op)[i] = make_uint4(0, 0, 0, 0);
         for (int i = tid; i < C::NQ * 8; i += 128) qsc[i] = 0;
+        for (int i = tid; i < 2 * 2 * 512 / 16; i += 128) reinterpret_cast<uint4*>(psf)[i] = make_uint4(0, 0, 0, 0);
         row_amax[tid] = 0;
         tc::named_bar_sync(1, 128);
         {
@@ -339,6 +381,13 @@ __global__ void __launch_bounds__(192, 1) decode_tc_kernel(const DecodeArgs a) {
             return true;
         };
 
+        // alpha * exp2(s - m), the scaled probability; the same instruction
+        // sequence serves a token and its block maximum, so the block scale is
+        // the one its largest member picks
+        auto scaled_prob = [&](float sv, float mn) -> float { return __fmul_rn(exp2f(__fsub_rn(sv, mn)), alpha); };
+        const int page_of_thread = warp >> 1;
+        const int blk_in_page = (tok_in_tile & 63) / B;
+
         for (int j = 0; j < n; ++j) {
             const int s = j % C::NS, buf = j & 1, tile = tile0 + j;
             if (j + 1 < n) bad |= !write_sfk(j + 1);
@@ -349,103 +398,84 @@ __global__ void __launch_bounds__(192, 1) decode_tc_kernel(const DecodeArgs a) {
             tc::tmem_ld<C::NQ>(tq + C::T_S + buf * C::NQ, sr);
             tc::tmem_wait_ld();
             const int token = tile * kTileTokens + tok_in_tile;
-            const bool valid = token < N && page_ids[s * 2 + (warp >> 1)] >= 0;
-            float sv[G];
-#pragma unroll
-            for (int g = 0; g < G; ++g)
-                sv[g] = valid ? (__uint_as_float(sr[g]) + __uint_as_float(sr[G + g])) * lsc[g] : -INFINITY;
-            // per-head tile maximum: warp reduction, then across the four warps
+            const bool valid = token < N && page_ids[s * 2 + page_of_thread] >= 0;
+            float sv[G], bmax[G];
+            float* rb = red + buf * G * 4;   // [G][4 warps] maxima of this tile
 #pragma unroll
             for (int g = 0; g < G; ++g) {
-                float mx = sv[g];
+                sv[g] = valid ? (__uint_as_float(sr[g]) + __uint_as_float(sr[G + g])) * lsc[g] : -INFINITY;
+                // maximum over this thread's probability block (beta lanes), then the warp
+                float v = sv[g];
 #pragma unroll
-                for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-                if (lane == 0) red[warp * G + g] = mx;
+                for (int off = 1; off < B; off <<= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+                bmax[g] = v;
+                if constexpr (B < 32) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+                if (lane == 0) rb[g * 4 + warp] = v;
             }
             // one decision for all four warps: sm_abort is written only before this barrier
             if (bad || *abort_flag) *sm_abort = 1;
             tc::named_bar_sync(1, 128);
             if (*sm_abort) break;
             float corr[G];
-            uint8_t* pb = p_op + buf * C::P_BUF + (warp >> 1) * C::P_PAGE + (warp & 1) * 128 + (lane >> 3) * 4;
+            uint8_t* pb = p_op + buf * C::P_BUF + page_of_thread * C::P_PAGE + (warp & 1) * 128 + (lane >> 3) * 4;
+            uint8_t* sfb = psf + (buf * 2 + page_of_thread) * 512 + blk_in_page;
 #pragma unroll
             for (int g = 0; g < G; ++g) {
-                const float mt = fmaxf(fmaxf(red[g], red[G + g]), fmaxf(red[2 * G + g], red[3 * G + g]));
-                const float mn = fmaxf(m_run[g], mt);
+                const float4 m4 = *reinterpret_cast<const float4*>(rb + g * 4);
+                const float mn = fmaxf(m_run[g], fmaxf(fmaxf(m4.x, m4.y), fmaxf(m4.z, m4.w)));
                 corr[g] = exp2f(m_run[g] - mn);   // 0 on the split's first tile
                 m_run[g] = mn;
-                const float p = valid ? exp2f(sv[g] - mn) : 0.0f;
-                l_part[g] = l_part[g] * corr[g] + p;
-                // fused FP4 quantization of p over beta-token blocks (lanes)
-                const float y = p * alpha;
-                float am = y;
-#pragma unroll
-                for (int off = B / 2; off > 0; off >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
+                const float y = scaled_prob(sv[g], mn);    // 0 for masked tokens (sv = -inf)
+                l_part[g] = l_part[g] * corr[g] + y;       // l in units of alpha (cancels at the end)
+                // fused FP4 quantization of the probabilities over beta-token blocks
+                const float am = scaled_prob(bmax[g], mn);
                 uint32_t c;
-                float sigma;
-                if constexpr (FMT == BDFP4_NVFP4) {
-                    c = am > 0.0f ? e4m3_encode(__fdiv_rn(am, 6.0f)) : 0u;
-                    sigma = e4m3_value(c);
-                } else {
-                    c = mx_scale_code(am);
-                    sigma = e8m0_value(c);
-                }
-                const uint32_t e = sigma > 0.0f ? e2m1_encode(__fdiv_rn(y, sigma)) : 0u;
+                if constexpr (FMT == BDFP4_NVFP4) c = e4m3_encode(__fmul_rn(am, 1.0f / 6.0f));
+                else c = mx_scale_code(am);
+                const float sigma = scale_value<FMT>(c);
+                const uint32_t e = sigma > 0.0f ? e2m1_encode(__fdividef(y, sigma)) : 0u;
                 uint32_t word = e << (4 * (lane & 7));
                 word |= __shfl_xor_sync(0xffffffffu, word, 1);
                 word |= __shfl_xor_sync(0xffffffffu, word, 2);
                 word |= __shfl_xor_sync(0xffffffffu, word, 4);
                 if ((lane & 7) == 0) *reinterpret_cast<uint32_t*>(pb + (g >> 3) * 256 + (g & 7) * 16) = word;
-                if ((lane & (B - 1)) == 0) psc[(buf * G + g) * 8 + tok_in_tile / B] = (uint8_t)c;
+                if ((lane & (B - 1)) == 0) sfb[g * 16] = (uint8_t)c;   // SFB row g of this page
             }
-            tc::fence_proxy_async_smem();
-            tc::named_bar_sync(1, 128);
-            // P scale factors (SFB of PV): lane g <- head g, one column per page
-            {
-                uint32_t c0 = 0, c1 = 0;
-                if (lane < G) {
-                    const uint8_t* ps = psc + (buf * G + lane) * 8;
-                    if constexpr (B == 16) {
-                        c0 = *reinterpret_cast<const uint32_t*>(ps);
-                        c1 = *reinterpret_cast<const uint32_t*>(ps + 4);
-                    } else {
-                        c0 = (uint32_t)ps[0] | ((uint32_t)ps[1] << 8);
-                        c1 = (uint32_t)ps[2] | ((uint32_t)ps[3] << 8);
+            // V scale factors: blocks past the sequence end (or of a page that was not
+            // loaded) are zeroed, so stale bytes are never multiplied
+            const bool tail = (tile + 1) * kTileTokens > N || page_ids[s * 2] < 0 || page_ids[s * 2 + 1] < 0;
+            uint8_t* vs = smem + C::SM_STAGES + s * C::STAGE + C::OFF_VS;
+            if constexpr (B == 16) {
+                if (tail) {
+                    const int ch = tok_in_tile;   // thread = channel
+#pragma unroll
+                    for (int p = 0; p < 2; ++p) {
+                        const int t0 = tile * kTileTokens + p * kPageSlots;
+                        int nvb = page_ids[s * 2 + p] >= 0 ? (N - t0 + B - 1) / B : 0;
+                        nvb = nvb < 0 ? 0 : (nvb > C::SPB ? C::SPB : nvb);
+                        for (int bb = nvb; bb < C::SPB; ++bb)
+                            vs[p * C::VS_PAGE + (ch & 31) * 16 + (ch >> 5) * 4 + bb] = 0;
                     }
                 }
-                tc::tmem_st4(tq + C::T_SFP + buf * 8, c0, 0u, 0u, 0u);
-                tc::tmem_st4(tq + C::T_SFP + buf * 8 + 4, c1, 0u, 0u, 0u);
-            }
-            // V scale factors (SFA of PV): lane i, column m1 (+4 per page) <- channel 32*m1 + i;
-            // blocks past the sequence end are zeroed (never multiplied by garbage)
-            {
-                const uint8_t* vs = smem + C::SM_STAGES + s * C::STAGE + C::OFF_VS;
+            } else {
                 uint32_t v[8];
 #pragma unroll
                 for (int p = 0; p < 2; ++p) {
                     const int t0 = tile * kTileTokens + p * kPageSlots;
                     int nvb = page_ids[s * 2 + p] >= 0 ? (N - t0 + B - 1) / B : 0;
                     nvb = nvb < 0 ? 0 : (nvb > C::SPB ? C::SPB : nvb);
-                    if constexpr (B == 16) {
-                        const uint32_t mask = nvb >= 4 ? 0xffffffffu : ((1u << (8 * nvb)) - 1u);
-                        const uint4 w = *reinterpret_cast<const uint4*>(vs + p * C::VS_PAGE + 16 * lane);
-                        v[p * 4 + 0] = w.x & mask;
-                        v[p * 4 + 1] = w.y & mask;
-                        v[p * 4 + 2] = w.z & mask;
-                        v[p * 4 + 3] = w.w & mask;
-                    } else {
-                        const uint32_t mask = nvb >= 2 ? 0xffffu : ((1u << (8 * nvb)) - 1u);
-                        const uint2 w = *reinterpret_cast<const uint2*>(vs + p * C::VS_PAGE + 8 * lane);
-                        v[p * 4 + 0] = w.x & mask;
-                        v[p * 4 + 1] = (w.x >> 16) & mask;
-                        v[p * 4 + 2] = w.y & mask;
-                        v[p * 4 + 3] = (w.y >> 16) & mask;
-                    }
+                    const uint32_t mask = nvb >= 2 ? 0xffffu : ((1u << (8 * nvb)) - 1u);
+                    const uint2 w = *reinterpret_cast<const uint2*>(vs + p * C::VS_PAGE + 8 * lane);
+                    v[p * 4 + 0] = w.x & mask;
+                    v[p * 4 + 1] = (w.x >> 16) & mask;
+                    v[p * 4 + 2] = w.y & mask;
+                    v[p * 4 + 3] = (w.y >> 16) & mask;
                 }
                 tc::tmem_st8(tq + C::T_SFV + buf * 8, v);
+                tc::tmem_wait_st();
+                tc::tc_fence_before();
             }
-            tc::tmem_wait_st();
-            tc::tc_fence_before();
+            tc::fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&p_ready[buf]);
             // fold the previous tile's O into registers
@@ -468,8 +498,8 @@ __global__ void __launch_bounds__(192, 1) decode_tc_kernel(const DecodeArgs a) {
                 if (lane == 0) red[warp * G + g] = v;
             }
             tc::named_bar_sync(1, 128);
-            const float vg = FMT == BDFP4_NVFP4 ? a.v_gscale[hk] : 1.0f;
-            const float oscale = vg / alpha;
+            // O and l both carry the factor alpha (P^ is alpha p quantized), so it cancels
+            const float oscale = FMT == BDFP4_NVFP4 ? a.v_gscale[hk] : 1.0f;
             const int ch = tok_in_tile;
 #pragma unroll
             for (int g = 0; g < G; ++g) {
@@ -503,7 +533,7 @@ static int launch_tc(const DecodeArgs& a, cudaStream_t st) {
     static bool attr_set = false;
     if (!attr_set) {
         const cudaError_t e =
-            cudaFuncSetAttribute(decode_tc_kernel<FMT, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+            cudaFuncSetAttribute(decode_tc_kernel<FMT, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_LAUNCH);
         if (e != cudaSuccess) {
             record_cuda_error(e);
             return BDFP4_ERR_CUDA;
@@ -511,7 +541,7 @@ static int launch_tc(const DecodeArgs& a, cudaStream_t st) {
         attr_set = true;
     }
     dim3 grid(a.max_splits, a.H_kv, a.B);
-    decode_tc_kernel<FMT, G><<<grid, 192, C::SMEM, st>>>(a);
+    decode_tc_kernel<FMT, G><<<grid, 192, C::SMEM_LAUNCH, st>>>(a);
     return launch_status();
 }
 

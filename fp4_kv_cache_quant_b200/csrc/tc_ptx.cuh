@@ -31,18 +31,39 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// try_wait suspends the thread until the phase completes or a hardware time
+// limit passes, so a waiting warp issues almost nothing.
+__device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
 // Bounded wait on a phase: gives up after `limit` clock cycles or when
 // *abort is set; returns false then.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, long long limit) {
+#ifdef BDFP4_SPIN_WAIT
     if (mbar_test(bar, parity)) return true;
     const long long t0 = clock64();
     for (uint32_t it = 0;; ++it) {
         if (mbar_test(bar, parity)) return true;
-        if ((it & 255u) == 255u) {
+        if ((it & 63u) == 63u) {
             if (*abort) return false;
             if (clock64() - t0 > limit) return false;
         }
     }
+#else
+    if (mbar_try(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try(bar, parity)) return true;
+        if (*abort) return false;
+        if (clock64() - t0 > limit) return false;
+    }
+#endif
 }
 
 // ------------------------------------------------------------------ bulk copy
@@ -151,6 +172,13 @@ __device__ __forceinline__ void mma_fp4(uint32_t d_tmem, uint64_t a_desc, uint64
             "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
             : "memory");
     }
+}
+
+// Copy 32 rows x 16 bytes from shared memory (described like an MMA operand:
+// 8-row x 16-byte core blocks, sbo between them) into 4 TMEM columns of lanes
+// 0..31, replicated into all four lane quadrants.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
 // Arrive on an mbarrier once every tcgen05 operation issued so far by this thread completes.
