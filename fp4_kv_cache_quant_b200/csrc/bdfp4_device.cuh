@@ -12,6 +12,7 @@
 
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include "../../include/bdfp4.h"
@@ -66,6 +67,13 @@ __device__ __forceinline__ float e4m3_value(uint32_t code) {
     uint32_t e = (code >> 3) & 15u, m = code & 7u;
     float mag = (e == 0) ? (float)m * 0.001953125f : __uint_as_float(((e + 120u) << 23) | (m << 20));
     return (code & 0x80u) ? -mag : mag;
+}
+
+// E4M3 value through the hardware conversion (exact: E4M3 is a subset of fp16).
+__device__ __forceinline__ float e4m3_value_hw(uint32_t code) {
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((unsigned short)(code & 0xffu)));
+    return __half2float(__ushort_as_half((unsigned short)(h2 & 0xffffu)));
 }
 
 // Unsigned E4M3 encode: nearest, ties to even, >= 448 saturates to 448.

@@ -30,6 +30,9 @@
 #ifndef BDFP4_TC_STAGES
 #define BDFP4_TC_STAGES 3
 #endif
+#ifndef BDFP4_TC_MIN_CTAS
+#define BDFP4_TC_MIN_CTAS 3
+#endif
 
 namespace bdfp4 {
 
@@ -41,6 +44,16 @@ struct TcCfg {
     static constexpr int NP = (G < 8) ? 8 : G;          // N of the PV MMA
     static constexpr int KS = DK / 64;                   // MMA K steps of QK
     static constexpr int NS = BDFP4_TC_STAGES;           // pipeline stages
+    // softmax warpgroups: warps w and w + 4 read the same TMEM lanes (tokens), so
+    // two groups split the query heads of every tile between them
+    static constexpr int NSG = G >= 2 ? 2 : 1;
+    static constexpr int HG = G / NSG;                   // heads per group
+    static constexpr int NSW = 4 * NSG;                  // softmax warps
+    static constexpr int PRODUCER = NSW, MMA_WARP = NSW + 1;
+    static constexpr int THREADS = 32 * (NSW + 2);
+    // CTAs per SM the register budget is shaped for (3 x 10 warps fit in 64 K
+    // registers at 64 per thread)
+    static constexpr int MIN_CTAS = BDFP4_TC_MIN_CTAS;
     static constexpr int K_PAGE = kPageSlots * DK / 2;   // 4096
     static constexpr int KS_PAGE = kPageSlots * DK / B;  // 512 (NVFP4) / 256 (MXFP4)
     static constexpr int V_PAGE = DV * kPageSlots / 2;   // 4096
@@ -58,15 +71,14 @@ struct TcCfg {
     static constexpr int SM_STAGES = 0;
     static constexpr int SM_Q = SM_STAGES + NS * STAGE;
     static constexpr int SM_P = SM_Q + Q_BYTES;
-    static constexpr int SM_QSC = SM_P + 2 * P_BUF;            // [NQ][8] query scale codes
+    static constexpr int SM_QSC = SM_P + 2 * P_BUF;                      // [NQ][8] query scale codes
     static constexpr int SM_PSF = (SM_QSC + NQ * 8 + 127) / 128 * 128;   // [2 buf][2 page][32 rows][16 B] P scales
     static constexpr int SM_RED = SM_PSF + 2 * 2 * 512;                  // [2][G][4] per-warp maxima (floats)
     static constexpr int SM_LSC = SM_RED + 2 * G * 4 * 4;               // [G] floats
-    static constexpr int SM_AMAX = SM_LSC + G * 4;             // [128] ints (row amax during the prologue)
-    static constexpr int SM_PAGES = SM_AMAX + 128 * 4;         // [NS][2] ints
+    static constexpr int SM_PAGES = SM_LSC + G * 4;                      // [NS][2] ints
     static constexpr int SM_BARS = (SM_PAGES + NS * 2 * 4 + 7) / 8 * 8;
     static constexpr int NBARS = 2 * NS + 8;
-    static constexpr int SM_MISC = SM_BARS + NBARS * 8;        // tmem slot, abort flags
+    static constexpr int SM_MISC = SM_BARS + NBARS * 8;                  // tmem slot, abort flags
     static constexpr int SMEM = SM_MISC + 16;
     // TMEM column map
     static constexpr int T_S = 0;
@@ -91,10 +103,11 @@ struct TcCfg {
 constexpr long long kWaitLimit = 1LL << 32;   // clock cycles (about 2 s)
 
 template <int FMT, int G>
-__global__ void __launch_bounds__(192, 1) decode_tc_kernel(const DecodeArgs a) {
+__global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTAS) decode_tc_kernel(const DecodeArgs a) {
     using C = TcCfg<FMT, G>;
     constexpr bool MX = FMT == BDFP4_MXFP4;
     constexpr int B = C::B;
+    constexpr int HG = C::HG;
     using RG = RowGeom<FMT, 128>;
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t* q_op = smem + C::SM_Q;
@@ -103,7 +116,6 @@ __global__ void __launch_bounds__(192, 1) decode_tc_kernel(const DecodeArgs a) {
     uint8_t* psf = smem + C::SM_PSF;
     float* red = reinterpret_cast<float*>(smem + C::SM_RED);
     float* lsc = reinterpret_cast<float*>(smem + C::SM_LSC);
-    int* row_amax = reinterpret_cast<int*>(smem + C::SM_AMAX);
     int* page_ids = reinterpret_cast<int*>(smem + C::SM_PAGES);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SM_BARS);
     uint64_t* full = bars;                    // [NS] producer -> consumers
@@ -114,7 +126,7 @@ __global__ void __launch_bounds__(192, 1) decode_tc_kernel(const DecodeArgs a) {
     uint64_t* o_full = p_ready + 2;           // [2] PV done -> softmax
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SM_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::SM_MISC + 4);   // any role gave up
-    volatile int* sm_abort = reinterpret_cast<volatile int*>(smem + C::SM_MISC + 8);     // softmax warps' decision
+    volatile int* sm_abort = reinterpret_cast<volatile int*>(smem + C::SM_MISC + 8);     // [NSG] group decisions
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
@@ -142,16 +154,17 @@ __global__ void __launch_bounds__(192, 1) decode_tc_kernel(const DecodeArgs a) {
             tc::mbar_init(&empty[s], 1);
         }
         for (int i = 0; i < 2; ++i) {
-            tc::mbar_init(&sfk_ready[i], 4);
+            tc::mbar_init(&sfk_ready[i], C::NSW);
             tc::mbar_init(&s_full[i], 1);
-            tc::mbar_init(&p_ready[i], 4);
+            tc::mbar_init(&p_ready[i], C::NSW);
             tc::mbar_init(&o_full[i], 1);
         }
         *abort_flag = 0;
-        *sm_abort = 0;
+        sm_abort[0] = 0;
+        sm_abort[1] = 0;
         tc::fence_mbar_init();
     }
-    if (warp == 5) {
+    if (warp == C::MMA_WARP) {
         tc::tmem_alloc(tmem_slot, C::T_ALLOC);
         tc::tmem_relinquish();
     }
@@ -160,7 +173,7 @@ __global__ void __launch_bounds__(192, 1) decode_tc_kernel(const DecodeArgs a) {
     tc::tc_fence_after();
     const uint32_t tbase = *tmem_slot;
 
-    if (warp == 4) {
+    if (warp == C::PRODUCER) {
         // ------------------------------------------------------------ producer
         // The warp reads the page ids of 32 tiles at once (one tile per lane),
         // so the dependent block-table load is off the per-tile path; lane 0
@@ -217,7 +230,7 @@ __global__ void __launch_bounds__(192, 1) decode_tc_kernel(const DecodeArgs a) {
             }
         }
         if (!ok && lane == 0) *abort_flag = 1;
-    } else if (warp == 5) {
+    } else if (warp == C::MMA_WARP) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_qk = tc::idesc_fp4(C::NQ, MX);
@@ -270,19 +283,23 @@ __global__ void __launch_bounds__(192, 1) decode_tc_kernel(const DecodeArgs a) {
             if (!ok) *abort_flag = 1;
         }
     } else {
-        // ------------------------------------------------------------ softmax warps 0..3
-        const uint32_t tq = tbase + ((uint32_t)(32 * warp) << 16);   // this warp's TMEM lane quadrant
+        // ------------------------------------------------------------ softmax warps
+        const int grp = warp >> 2;                 // head group
+        const int qd = warp & 3;                   // TMEM lane quadrant = tokens 32 qd .. 32 qd + 31
+        const int gb = grp * HG;                   // first head of the group
+        const int bar_id = 1 + grp;                // named barrier of the group (128 threads)
+        const uint32_t tq = tbase + ((uint32_t)(32 * qd) << 16);
         const bool hadamard = !(a.flags & BDFP4_FLAG_NO_HADAMARD);
         const bool dual = !(a.flags & BDFP4_FLAG_SINGLE_QUERY);
         const float alpha = (FMT == BDFP4_NVFP4 && !(a.flags & BDFP4_FLAG_NO_UNDERFLOW)) ? kAlphaNV : 1.0f;
         bool bad = false;
 
-        // query prologue: transform + dual-residual FP4 straight into the QK operand
-        for (int i = tid; i < C::Q_BYTES / 16; i += 128) reinterpret_cast<uint4*>(q_op)[i] = make_uint4(0, 0, 0, 0);
-        for (int i = tid; i < C::NQ * 8; i += 128) qsc[i] = 0;
-        for (int i = tid; i < 2 * 2 * 512 / 16; i += 128) reinterpret_cast<uint4*>(psf)[i] = make_uint4(0, 0, 0, 0);
-        row_amax[tid] = 0;
-        tc::named_bar_sync(1, 128);
+        // query prologue (all softmax warps): transform + dual-residual FP4 straight into the QK operand
+        int* row_amax = reinterpret_cast<int*>(psf);   // the P scale buffers are free until the first tile
+        for (int i = tid; i < C::Q_BYTES / 16; i += 32 * C::NSW) reinterpret_cast<uint4*>(q_op)[i] = make_uint4(0, 0, 0, 0);
+        for (int i = tid; i < C::NQ * 8; i += 32 * C::NSW) qsc[i] = 0;
+        if (tid < 32) row_amax[tid] = 0;
+        tc::named_bar_sync(1 + C::NSG, 32 * C::NSW);
         {
             const int j = tid % RG::rt, r = tid / RG::rt;
             const bool active = r < G && j < RG::tpr;
@@ -295,7 +312,7 @@ __global__ void __launch_bounds__(192, 1) decode_tc_kernel(const DecodeArgs a) {
             }
             transform_block<FMT, 128, false>(x, a.smooth + (int64_t)hk * C::DK, j, hadamard);
             if (active) atomicMax(&row_amax[r], __float_as_int(block_amax<B>(x)));
-            tc::named_bar_sync(1, 128);
+            tc::named_bar_sync(1 + C::NSG, 32 * C::NSW);
             if (active) {
                 const float amax = __int_as_float(row_amax[r]);
                 const float gq = FMT == BDFP4_NVFP4 ? (amax > 0.0f ? __fdiv_rn(amax, 2688.0f) : 1.0f) : 1.0f;
@@ -318,11 +335,12 @@ __global__ void __launch_bounds__(192, 1) decode_tc_kernel(const DecodeArgs a) {
                 }
             }
             tc::fence_proxy_async_smem();
-            tc::named_bar_sync(1, 128);
+            tc::named_bar_sync(1 + C::NSG, 32 * C::NSW);
+            // the P scale-factor buffers: zero (rows of absent heads must stay zero)
+            for (int i = tid; i < 2 * 2 * 512 / 16; i += 32 * C::NSW) reinterpret_cast<uint4*>(psf)[i] = make_uint4(0, 0, 0, 0);
         }
-        // query scale factors (SFB of QK): lane n <- row n, one column per K step, all quadrants
-        {
-            uint32_t col[C::KS];
+        // query scale factors (SFB of QK): lane n <- row n, one 4-column chunk per K step
+        if (grp == 0) {
 #pragma unroll
             for (int ks = 0; ks < C::KS; ++ks) {
                 uint32_t v = 0;
@@ -330,29 +348,32 @@ __global__ void __launch_bounds__(192, 1) decode_tc_kernel(const DecodeArgs a) {
                     if constexpr (B == 16) v = *reinterpret_cast<const uint32_t*>(qsc + lane * 8 + ks * 4);
                     else v = (uint32_t)qsc[lane * 8 + ks * 2] | ((uint32_t)qsc[lane * 8 + ks * 2 + 1] << 8);
                 }
-                col[ks] = v;
+                tc::tmem_st4(tq + C::T_SFQ + ks * 4, v, 0u, 0u, 0u);
             }
-#pragma unroll
-            for (int ks = 0; ks < C::KS; ++ks) tc::tmem_st4(tq + C::T_SFQ + ks * 4, col[ks], 0u, 0u, 0u);
         }
-        // K scale factors of tile j (SFA of QK): TMEM lane i, column m1 (+4 per K step) <- row 32*m1 + i
+        tc::fence_proxy_async_smem();
+        tc::named_bar_sync(1 + C::NSG, 32 * C::NSW);   // psf zeroed before any tile writes it
+        // K scale factors of tile j (SFA of QK): TMEM lane i, column m1 (+4 per K step) <- token 32*m1 + i.
+        // Each group writes its share of the K steps.
         auto write_sfk = [&](int j) -> bool {
             const int s = j % C::NS;
             if (!tc::mbar_wait(&full[s], (j / C::NS) & 1, abort_flag, kWaitLimit)) return false;
             const uint8_t* ks = smem + C::SM_STAGES + s * C::STAGE + C::OFF_KS;
-            uint32_t v[8];
-            if constexpr (B == 16) {
-                const uint4 p0 = *reinterpret_cast<const uint4*>(ks + 16 * lane);
-                const uint4 p1 = *reinterpret_cast<const uint4*>(ks + C::KS_PAGE + 16 * lane);
-                v[0] = p0.x; v[1] = p0.y; v[2] = p1.x; v[3] = p1.y;
-                v[4] = p0.z; v[5] = p0.w; v[6] = p1.z; v[7] = p1.w;
-            } else {
-                const uint2 p0 = *reinterpret_cast<const uint2*>(ks + 8 * lane);
-                const uint2 p1 = *reinterpret_cast<const uint2*>(ks + C::KS_PAGE + 8 * lane);
-                v[0] = p0.x & 0xffffu; v[1] = p0.x >> 16; v[2] = p1.x & 0xffffu; v[3] = p1.x >> 16;
-                v[4] = p0.y & 0xffffu; v[5] = p0.y >> 16; v[6] = p1.y & 0xffffu; v[7] = p1.y >> 16;
+#pragma unroll
+            for (int kk = 0; kk < C::KS / C::NSG; ++kk) {
+                const int kstep = grp * (C::KS / C::NSG) + kk;
+                uint32_t v0, v1, v2, v3;
+                if constexpr (B == 16) {
+                    const uint2 p0 = *reinterpret_cast<const uint2*>(ks + 16 * lane + 8 * kstep);
+                    const uint2 p1 = *reinterpret_cast<const uint2*>(ks + C::KS_PAGE + 16 * lane + 8 * kstep);
+                    v0 = p0.x; v1 = p0.y; v2 = p1.x; v3 = p1.y;
+                } else {
+                    const uint32_t p0 = *reinterpret_cast<const uint32_t*>(ks + 8 * lane + 4 * kstep);
+                    const uint32_t p1 = *reinterpret_cast<const uint32_t*>(ks + C::KS_PAGE + 8 * lane + 4 * kstep);
+                    v0 = p0 & 0xffffu; v1 = p0 >> 16; v2 = p1 & 0xffffu; v3 = p1 >> 16;
+                }
+                tc::tmem_st4(tq + C::T_SFK + (j & 1) * 4 * C::KS + kstep * 4, v0, v1, v2, v3);
             }
-            tc::tmem_st8(tq + C::T_SFK + (j & 1) * 4 * C::KS, v);
             tc::tmem_wait_st();
             tc::tc_fence_before();
             __syncwarp();
@@ -361,23 +382,23 @@ __global__ void __launch_bounds__(192, 1) decode_tc_kernel(const DecodeArgs a) {
         };
         bad |= !write_sfk(0);
 
-        float m_run[G], l_part[G], o_acc[G], corr_prev[G];
+        float m_run[HG], l_part[HG], o_acc[HG], corr_prev[HG];
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
+        for (int g = 0; g < HG; ++g) {
             m_run[g] = -INFINITY;
             l_part[g] = 0.0f;
             o_acc[g] = 0.0f;
             corr_prev[g] = 0.0f;
         }
-        const int tok_in_tile = 32 * warp + lane;
+        const int tok_in_tile = 32 * qd + lane;
         auto fold_o = [&](int j) -> bool {
             if (!tc::mbar_wait(&o_full[j & 1], (j >> 1) & 1, abort_flag, kWaitLimit)) return false;
             tc::tc_fence_after();
-            uint32_t ov[C::NP];
-            tc::tmem_ld<C::NP>(tq + C::T_O + (j & 1) * C::NP, ov);
+            uint32_t ov[HG];
+            tc::tmem_ld<HG>(tq + C::T_O + (j & 1) * C::NP + gb, ov);
             tc::tmem_wait_ld();
 #pragma unroll
-            for (int g = 0; g < G; ++g) o_acc[g] = o_acc[g] * corr_prev[g] + __uint_as_float(ov[g]);
+            for (int g = 0; g < HG; ++g) o_acc[g] = o_acc[g] * corr_prev[g] + __uint_as_float(ov[g]);
             return true;
         };
 
@@ -385,43 +406,45 @@ __global__ void __launch_bounds__(192, 1) decode_tc_kernel(const DecodeArgs a) {
         // sequence serves a token and its block maximum, so the block scale is
         // the one its largest member picks
         auto scaled_prob = [&](float sv, float mn) -> float { return __fmul_rn(exp2f(__fsub_rn(sv, mn)), alpha); };
-        const int page_of_thread = warp >> 1;
+        const int page_of_thread = qd >> 1;
         const int blk_in_page = (tok_in_tile & 63) / B;
 
         for (int j = 0; j < n; ++j) {
             const int s = j % C::NS, buf = j & 1, tile = tile0 + j;
             if (j + 1 < n) bad |= !write_sfk(j + 1);
-            // logits of this thread's token
+            // logits of this thread's token for the group's heads (q1 and q2 columns)
             if (!tc::mbar_wait(&s_full[buf], (j >> 1) & 1, abort_flag, kWaitLimit)) bad = true;
             tc::tc_fence_after();
-            uint32_t sr[C::NQ];
-            tc::tmem_ld<C::NQ>(tq + C::T_S + buf * C::NQ, sr);
+            uint32_t s1[HG], s2[HG];
+            tc::tmem_ld<HG>(tq + C::T_S + buf * C::NQ + gb, s1);
+            tc::tmem_ld<HG>(tq + C::T_S + buf * C::NQ + G + gb, s2);
             tc::tmem_wait_ld();
             const int token = tile * kTileTokens + tok_in_tile;
             const bool valid = token < N && page_ids[s * 2 + page_of_thread] >= 0;
-            float sv[G], bmax[G];
-            float* rb = red + buf * G * 4;   // [G][4 warps] maxima of this tile
+            float sv[HG], bmax[HG];
+            float* rb = red + buf * G * 4;   // [G][4 quadrants] maxima of this tile
 #pragma unroll
-            for (int g = 0; g < G; ++g) {
-                sv[g] = valid ? (__uint_as_float(sr[g]) + __uint_as_float(sr[G + g])) * lsc[g] : -INFINITY;
+            for (int g = 0; g < HG; ++g) {
+                sv[g] = valid ? (__uint_as_float(s1[g]) + __uint_as_float(s2[g])) * lsc[gb + g] : -INFINITY;
                 // maximum over this thread's probability block (beta lanes), then the warp
                 float v = sv[g];
 #pragma unroll
                 for (int off = 1; off < B; off <<= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
                 bmax[g] = v;
                 if constexpr (B < 32) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-                if (lane == 0) rb[g * 4 + warp] = v;
+                if (lane == 0) rb[(gb + g) * 4 + qd] = v;
             }
-            // one decision for all four warps: sm_abort is written only before this barrier
-            if (bad || *abort_flag) *sm_abort = 1;
-            tc::named_bar_sync(1, 128);
-            if (*sm_abort) break;
-            float corr[G];
-            uint8_t* pb = p_op + buf * C::P_BUF + page_of_thread * C::P_PAGE + (warp & 1) * 128 + (lane >> 3) * 4;
+            // one decision for the group's four warps: its flag is written only before this barrier
+            if (bad || *abort_flag) sm_abort[grp] = 1;
+            tc::named_bar_sync(bar_id, 128);
+            if (sm_abort[grp]) break;
+            float corr[HG];
+            uint8_t* pb = p_op + buf * C::P_BUF + page_of_thread * C::P_PAGE + (qd & 1) * 128 + (lane >> 3) * 4;
             uint8_t* sfb = psf + (buf * 2 + page_of_thread) * 512 + blk_in_page;
 #pragma unroll
-            for (int g = 0; g < G; ++g) {
-                const float4 m4 = *reinterpret_cast<const float4*>(rb + g * 4);
+            for (int g = 0; g < HG; ++g) {
+                const int hh = gb + g;
+                const float4 m4 = *reinterpret_cast<const float4*>(rb + hh * 4);
                 const float mn = fmaxf(m_run[g], fmaxf(fmaxf(m4.x, m4.y), fmaxf(m4.z, m4.w)));
                 corr[g] = exp2f(m_run[g] - mn);   // 0 on the split's first tile
                 m_run[g] = mn;
@@ -430,50 +453,57 @@ __global__ void __launch_bounds__(192, 1) decode_tc_kernel(const DecodeArgs a) {
                 // fused FP4 quantization of the probabilities over beta-token blocks
                 const float am = scaled_prob(bmax[g], mn);
                 uint32_t c;
-                if constexpr (FMT == BDFP4_NVFP4) c = e4m3_encode(__fmul_rn(am, 1.0f / 6.0f));
-                else c = mx_scale_code(am);
-                const float sigma = scale_value<FMT>(c);
+                float sigma;
+                if constexpr (FMT == BDFP4_NVFP4) {
+                    c = e4m3_encode(__fmul_rn(am, 1.0f / 6.0f));
+                    sigma = e4m3_value_hw(c);
+                } else {
+                    c = mx_scale_code(am);
+                    sigma = e8m0_value(c);
+                }
                 const uint32_t e = sigma > 0.0f ? e2m1_encode(__fdividef(y, sigma)) : 0u;
                 uint32_t word = e << (4 * (lane & 7));
                 word |= __shfl_xor_sync(0xffffffffu, word, 1);
                 word |= __shfl_xor_sync(0xffffffffu, word, 2);
                 word |= __shfl_xor_sync(0xffffffffu, word, 4);
-                if ((lane & 7) == 0) *reinterpret_cast<uint32_t*>(pb + (g >> 3) * 256 + (g & 7) * 16) = word;
-                if ((lane & (B - 1)) == 0) sfb[g * 16] = (uint8_t)c;   // SFB row g of this page
+                if ((lane & 7) == 0) *reinterpret_cast<uint32_t*>(pb + (hh >> 3) * 256 + (hh & 7) * 16) = word;
+                if ((lane & (B - 1)) == 0) sfb[hh * 16] = (uint8_t)c;   // SFB row hh of this page
             }
-            // V scale factors: blocks past the sequence end (or of a page that was not
-            // loaded) are zeroed, so stale bytes are never multiplied
-            const bool tail = (tile + 1) * kTileTokens > N || page_ids[s * 2] < 0 || page_ids[s * 2 + 1] < 0;
-            uint8_t* vs = smem + C::SM_STAGES + s * C::STAGE + C::OFF_VS;
-            if constexpr (B == 16) {
-                if (tail) {
-                    const int ch = tok_in_tile;   // thread = channel
+            // V scale factors (group 0): blocks past the sequence end (or of a page that
+            // was not loaded) are zeroed, so stale bytes are never multiplied
+            if (grp == 0) {
+                const bool tail = (tile + 1) * kTileTokens > N || page_ids[s * 2] < 0 || page_ids[s * 2 + 1] < 0;
+                uint8_t* vs = smem + C::SM_STAGES + s * C::STAGE + C::OFF_VS;
+                if constexpr (B == 16) {
+                    if (tail) {
+                        const int ch = tok_in_tile;   // thread = channel
+#pragma unroll
+                        for (int p = 0; p < 2; ++p) {
+                            const int t0 = tile * kTileTokens + p * kPageSlots;
+                            int nvb = page_ids[s * 2 + p] >= 0 ? (N - t0 + B - 1) / B : 0;
+                            nvb = nvb < 0 ? 0 : (nvb > C::SPB ? C::SPB : nvb);
+                            for (int bb = nvb; bb < C::SPB; ++bb)
+                                vs[p * C::VS_PAGE + (ch & 31) * 16 + (ch >> 5) * 4 + bb] = 0;
+                        }
+                    }
+                } else {
+                    uint32_t v[8];
 #pragma unroll
                     for (int p = 0; p < 2; ++p) {
                         const int t0 = tile * kTileTokens + p * kPageSlots;
                         int nvb = page_ids[s * 2 + p] >= 0 ? (N - t0 + B - 1) / B : 0;
                         nvb = nvb < 0 ? 0 : (nvb > C::SPB ? C::SPB : nvb);
-                        for (int bb = nvb; bb < C::SPB; ++bb)
-                            vs[p * C::VS_PAGE + (ch & 31) * 16 + (ch >> 5) * 4 + bb] = 0;
+                        const uint32_t mask = nvb >= 2 ? 0xffffu : ((1u << (8 * nvb)) - 1u);
+                        const uint2 w = *reinterpret_cast<const uint2*>(vs + p * C::VS_PAGE + 8 * lane);
+                        v[p * 4 + 0] = w.x & mask;
+                        v[p * 4 + 1] = (w.x >> 16) & mask;
+                        v[p * 4 + 2] = w.y & mask;
+                        v[p * 4 + 3] = (w.y >> 16) & mask;
                     }
+                    tc::tmem_st8(tq + C::T_SFV + buf * 8, v);
+                    tc::tmem_wait_st();
+                    tc::tc_fence_before();
                 }
-            } else {
-                uint32_t v[8];
-#pragma unroll
-                for (int p = 0; p < 2; ++p) {
-                    const int t0 = tile * kTileTokens + p * kPageSlots;
-                    int nvb = page_ids[s * 2 + p] >= 0 ? (N - t0 + B - 1) / B : 0;
-                    nvb = nvb < 0 ? 0 : (nvb > C::SPB ? C::SPB : nvb);
-                    const uint32_t mask = nvb >= 2 ? 0xffffu : ((1u << (8 * nvb)) - 1u);
-                    const uint2 w = *reinterpret_cast<const uint2*>(vs + p * C::VS_PAGE + 8 * lane);
-                    v[p * 4 + 0] = w.x & mask;
-                    v[p * 4 + 1] = (w.x >> 16) & mask;
-                    v[p * 4 + 2] = w.y & mask;
-                    v[p * 4 + 3] = (w.y >> 16) & mask;
-                }
-                tc::tmem_st8(tq + C::T_SFV + buf * 8, v);
-                tc::tmem_wait_st();
-                tc::tc_fence_before();
             }
             tc::fence_proxy_async_smem();
             __syncwarp();
@@ -481,35 +511,37 @@ __global__ void __launch_bounds__(192, 1) decode_tc_kernel(const DecodeArgs a) {
             // fold the previous tile's O into registers
             if (j >= 1) bad |= !fold_o(j - 1);
 #pragma unroll
-            for (int g = 0; g < G; ++g) corr_prev[g] = corr[g];
+            for (int g = 0; g < HG; ++g) corr_prev[g] = corr[g];
         }
-        if (!*sm_abort && !fold_o(n - 1)) bad = true;
-        if (bad || *abort_flag) *sm_abort = 1;
+        if (!sm_abort[grp] && !fold_o(n - 1)) bad = true;
+        if (bad || *abort_flag) sm_abort[grp] = 1;
 
         // ------------------------------------------------------------ epilogue (thread = channel)
-        tc::named_bar_sync(1, 128);
-        if (*sm_abort) *abort_flag = 1;
-        if (!*sm_abort) {
+        tc::named_bar_sync(bar_id, 128);
+        if (sm_abort[grp]) *abort_flag = 1;
+        if (!sm_abort[grp]) {
+            float* rl = red;   // [G][4] partial sums (the tile maxima are no longer read)
 #pragma unroll
-            for (int g = 0; g < G; ++g) {
+            for (int g = 0; g < HG; ++g) {
                 float v = l_part[g];
 #pragma unroll
                 for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-                if (lane == 0) red[warp * G + g] = v;
+                if (lane == 0) rl[(gb + g) * 4 + qd] = v;
             }
-            tc::named_bar_sync(1, 128);
+            tc::named_bar_sync(bar_id, 128);
             // O and l both carry the factor alpha (P^ is alpha p quantized), so it cancels
             const float oscale = FMT == BDFP4_NVFP4 ? a.v_gscale[hk] : 1.0f;
             const int ch = tok_in_tile;
 #pragma unroll
-            for (int g = 0; g < G; ++g) {
-                const float l = red[g] + red[G + g] + red[2 * G + g] + red[3 * G + g];
-                const int64_t row = (int64_t)b * a.H_q + h0 + g;
+            for (int g = 0; g < HG; ++g) {
+                const int hh = gb + g;
+                const float l = rl[hh * 4] + rl[hh * 4 + 1] + rl[hh * 4 + 2] + rl[hh * 4 + 3];
+                const int64_t row = (int64_t)b * a.H_q + h0 + hh;
                 if (nspl == 1) {
                     a.out[row * C::DV + ch] = __float2bfloat16(l > 0.0f ? o_acc[g] * oscale / l : 0.0f);
                 } else {
                     a.ws_o[(row * a.max_splits + split) * C::DV + ch] = o_acc[g] * oscale;
-                    if (tid == 0) {
+                    if (tok_in_tile == 0) {
                         a.ws_ml[(row * a.max_splits + split) * 2 + 0] = m_run[g];
                         a.ws_ml[(row * a.max_splits + split) * 2 + 1] = l;
                     }
@@ -521,7 +553,7 @@ __global__ void __launch_bounds__(192, 1) decode_tc_kernel(const DecodeArgs a) {
     tc::tc_fence_before();
     __syncthreads();
     if (*abort_flag && tid == 0) set_status(a.dev_status, BDFP4_DEV_TIMEOUT);
-    if (warp == 5) {
+    if (warp == C::MMA_WARP) {
         tc::tc_fence_after();
         tc::tmem_dealloc(tbase, C::T_ALLOC);
     }
@@ -541,7 +573,7 @@ static int launch_tc(const DecodeArgs& a, cudaStream_t st) {
         attr_set = true;
     }
     dim3 grid(a.max_splits, a.H_kv, a.B);
-    decode_tc_kernel<FMT, G><<<grid, 192, C::SMEM_LAUNCH, st>>>(a);
+    decode_tc_kernel<FMT, G><<<grid, C::THREADS, C::SMEM_LAUNCH, st>>>(a);
     return launch_status();
 }
 
