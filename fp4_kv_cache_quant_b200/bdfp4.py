@@ -137,7 +137,7 @@ class FP4Cache:
     def empty(num_pages: int, H_kv: int, d_k: int, d_v: int, fmt: int, device="cuda") -> "FP4Cache":
         b = beta(fmt)
         mk = lambda n: torch.zeros(n, dtype=torch.uint8, device=device)  # noqa: E731
-        return FP4Cache(mk(num_pages * H_kv * PAGE_SLOTS * d_k // 2), mk(num_pages * H_kv * PAGE_SLOTS * d_k // b),
+        return FP4Cache(mk(num_pages * H_kv * PAGE_SLOTS * d_k // 2), mk(num_pages * H_kv * 256 * ((d_k // b + 3) // 4)),
                         mk(num_pages * H_kv * d_v * PAGE_SLOTS // 2), mk(num_pages * H_kv * d_v * PAGE_SLOTS // b),
                         num_pages, H_kv, d_k, d_v, fmt)
 

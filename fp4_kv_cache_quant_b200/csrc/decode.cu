@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(kThreads) decode_fp4_kernel(const DecodeArgs a
 
     const float alpha = (FMT == BDFP4_NVFP4 && !(a.flags & BDFP4_FLAG_NO_UNDERFLOW)) ? kAlphaNV : 1.0f;
     const float vg = FMT == BDFP4_NVFP4 ? a.v_gscale[hk] : 1.0f;
-    const int64_t kv_stride_k = (int64_t)kPageSlots * DK / 2, kv_stride_ks = (int64_t)kPageSlots * DK / B;
+    const int64_t kv_stride_k = (int64_t)kPageSlots * DK / 2, kv_stride_ks = k_scale_page_bytes(DK, B);
     const int64_t kv_stride_v = (int64_t)DV * kPageSlots / 2, kv_stride_vs = (int64_t)DV * kPageSlots / B;
 
     float m_run[HG], l_part[HG], o[HG][NCH];

@@ -55,9 +55,14 @@ struct TcCfg {
     // registers at 64 per thread)
     static constexpr int MIN_CTAS = BDFP4_TC_MIN_CTAS;
     static constexpr int K_PAGE = kPageSlots * DK / 2;   // 4096
-    static constexpr int KS_PAGE = kPageSlots * DK / B;  // 512 (NVFP4) / 256 (MXFP4)
+    static constexpr int NKG = (DK / B + 3) / 4;         // 4-block K scale groups per token (2 / 1)
+    static constexpr int KPG = KS / NKG;                 // K steps per scale group (1 NVFP4, 2 MXFP4)
+    static constexpr int KS_PAGE = 256 * NKG;            // K scale bytes per page (512 / 256)
     static constexpr int V_PAGE = DV * kPageSlots / 2;   // 4096
     static constexpr int VS_PAGE = DV * kPageSlots / B;
+    // a stage holds one 128-token tile: K [m1][page][1 KB] (MMA row 32 m1 + i <- slot
+    // (i%16) + 16 m1 of page i/16), V [page][4 KB], K scales [group][page][256 B],
+    // V scales [page][VS_PAGE]
     static constexpr int OFF_K = 0;
     static constexpr int OFF_V = 2 * K_PAGE;
     static constexpr int OFF_KS = OFF_V + 2 * V_PAGE;
@@ -73,18 +78,18 @@ struct TcCfg {
     static constexpr int SM_P = SM_Q + Q_BYTES;
     static constexpr int SM_QSC = SM_P + 2 * P_BUF;                      // [NQ][8] query scale codes
     static constexpr int SM_PSF = (SM_QSC + NQ * 8 + 127) / 128 * 128;   // [2 buf][2 page][32 rows][16 B] P scales
-    static constexpr int SM_RED = SM_PSF + 2 * 2 * 512;                  // [2][G][4] per-warp maxima (floats)
-    static constexpr int SM_LSC = SM_RED + 2 * G * 4 * 4;               // [G] floats
+    static constexpr int SM_RED = SM_PSF + 2 * 2 * 512;                  // [2][G][8] 16-token maxima (floats)
+    static constexpr int SM_LSC = SM_RED + 2 * G * 8 * 4;               // [G] floats
     static constexpr int SM_PAGES = SM_LSC + G * 4;                      // [NS][2] ints
     static constexpr int SM_BARS = (SM_PAGES + NS * 2 * 4 + 7) / 8 * 8;
-    static constexpr int NBARS = 2 * NS + 8;
+    static constexpr int NBARS = 2 * NS + 9;
     static constexpr int SM_MISC = SM_BARS + NBARS * 8;                  // tmem slot, abort flags
     static constexpr int SMEM = SM_MISC + 16;
     // TMEM column map
     static constexpr int T_S = 0;
     static constexpr int T_O = 2 * NQ;
-    static constexpr int T_SFK = ((T_O + 2 * NP + 3) / 4) * 4;   // 2 x (4 per K step x KS)
-    static constexpr int T_SFV = T_SFK + 2 * 4 * KS;             // 2 x (4 per page x 2 pages)
+    static constexpr int T_SFK = ((T_O + 2 * NP + 3) / 4) * 4;   // 2 x (4 per K scale group x NKG)
+    static constexpr int T_SFV = T_SFK + 2 * 4 * NKG;            // 2 x (4 per page x 2 pages)
     // every scale-factor operand starts on a 4-column boundary (one 32-bit
     // column per 32 rows of a 128-row chunk), B operands included
     static constexpr int T_SFQ = T_SFV + 2 * 8;                  // KS x 4 columns
@@ -120,10 +125,10 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SM_BARS);
     uint64_t* full = bars;                    // [NS] producer -> consumers
     uint64_t* empty = bars + C::NS;           // [NS] PV done -> producer
-    uint64_t* sfk_ready = bars + 2 * C::NS;   // [2] K scale factors in TMEM -> MMA
-    uint64_t* s_full = sfk_ready + 2;         // [2] QK done -> softmax
+    uint64_t* s_full = bars + 2 * C::NS;      // [2] QK done -> softmax
     uint64_t* p_ready = s_full + 2;           // [2] P + scale factors ready -> MMA
     uint64_t* o_full = p_ready + 2;           // [2] PV done -> softmax
+    uint64_t* q_ready = o_full + 2;           // query operand and its scale factors -> MMA
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SM_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::SM_MISC + 4);   // any role gave up
     volatile int* sm_abort = reinterpret_cast<volatile int*>(smem + C::SM_MISC + 8);     // [NSG] group decisions
@@ -154,11 +159,11 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
             tc::mbar_init(&empty[s], 1);
         }
         for (int i = 0; i < 2; ++i) {
-            tc::mbar_init(&sfk_ready[i], C::NSW);
             tc::mbar_init(&s_full[i], 1);
             tc::mbar_init(&p_ready[i], C::NSW);
             tc::mbar_init(&o_full[i], 1);
         }
+        tc::mbar_init(q_ready, C::NSW);
         *abort_flag = 0;
         sm_abort[0] = 0;
         sm_abort[1] = 0;
@@ -216,9 +221,14 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                         for (int p = 0; p < 2; ++p) {
                             if (pg[p] < 0) continue;
                             const int64_t ph = (int64_t)pg[p] * a.H_kv + hk;
-                            tc::bulk_g2s(st + C::OFF_K + p * C::K_PAGE, a.k_pages + ph * C::K_PAGE, C::K_PAGE, &full[s]);
-                            tc::bulk_g2s(st + C::OFF_KS + p * C::KS_PAGE, a.k_scales + ph * C::KS_PAGE, C::KS_PAGE,
-                                         &full[s]);
+#pragma unroll
+                            for (int c = 0; c < 4; ++c)   // slot groups 2c, 2c+1 -> MMA row groups 4c + 2p, +1
+                                tc::bulk_g2s(st + C::OFF_K + c * 2048 + p * 1024, a.k_pages + ph * C::K_PAGE + c * 1024,
+                                             1024, &full[s]);
+#pragma unroll
+                            for (int kg = 0; kg < C::NKG; ++kg)
+                                tc::bulk_g2s(st + C::OFF_KS + kg * 512 + p * 256, a.k_scales + ph * C::KS_PAGE + kg * 256,
+                                             256, &full[s]);
                             tc::bulk_g2s(st + C::OFF_V + p * C::V_PAGE, a.v_pages + ph * C::V_PAGE, C::V_PAGE, &full[s]);
                             tc::bulk_g2s(st + C::OFF_VS + p * C::VS_PAGE, a.v_scales + ph * C::VS_PAGE, C::VS_PAGE,
                                          &full[s]);
@@ -242,19 +252,30 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
             auto issue_qk = [&](int j) -> bool {
                 const int s = j % C::NS, buf = j & 1;
                 if (!tc::mbar_wait(&full[s], (j / C::NS) & 1, abort_flag, kWaitLimit)) return false;
-                if (!tc::mbar_wait(&sfk_ready[buf], (j >> 1) & 1, abort_flag, kWaitLimit)) return false;
                 tc::tc_fence_after();
                 const uint32_t kt = st_addr + s * C::STAGE + C::OFF_K;
+                // K scale factors: each 512-byte group chunk (16 rows of page 0, then of
+                // page 1) is already in the 32 x 16-byte copy layout
+#pragma unroll
+                for (int kg = 0; kg < C::NKG; ++kg)
+                    tc::tmem_cp_32x128b_x4(tbase + C::T_SFK + (buf * C::NKG + kg) * 4,
+                                           tc::smem_desc(kt - C::OFF_K + C::OFF_KS + kg * 512, 128, 128));
 #pragma unroll
                 for (int ks = 0; ks < C::KS; ++ks) {
+                    // MXFP4 packs two K steps per scale column: byte offset 2 (sf id) for the odd step
+                    const uint32_t sfid = (uint32_t)(ks % C::KPG) * 2u;
                     tc::mma_fp4<MX>(tbase + C::T_S + buf * C::NQ, tc::smem_desc(kt + ks * 256, 128, 512),
-                                    tc::smem_desc(q_addr + ks * 256, 128, 512), idesc_qk,
-                                    tbase + C::T_SFK + buf * 4 * C::KS + ks * 4, tbase + C::T_SFQ + ks * 4, ks > 0);
+                                    tc::smem_desc(q_addr + ks * 256, 128, 512), idesc_qk | (sfid << 29),
+                                    (tbase + C::T_SFK + (buf * C::NKG + ks / C::KPG) * 4) | (sfid << 30),
+                                    tbase + C::T_SFQ + ks * 4, ks > 0);
                 }
                 tc::mma_commit(&s_full[buf]);
                 return true;
             };
-            bool ok = issue_qk(0);
+            // the softmax warps quantize the query into shared memory and TMEM first
+            bool ok = tc::mbar_wait(q_ready, 0, abort_flag, kWaitLimit);
+            if (ok) tc::tc_fence_after();
+            ok = ok && issue_qk(0);
             for (int j = 0; ok && j < n; ++j) {
                 if (j + 1 < n && !(ok = issue_qk(j + 1))) break;
                 const int s = j % C::NS, buf = j & 1;
@@ -350,38 +371,12 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                 }
                 tc::tmem_st4(tq + C::T_SFQ + ks * 4, v, 0u, 0u, 0u);
             }
+            tc::tmem_wait_st();
         }
+        tc::tc_fence_before();
         tc::fence_proxy_async_smem();
         tc::named_bar_sync(1 + C::NSG, 32 * C::NSW);   // psf zeroed before any tile writes it
-        // K scale factors of tile j (SFA of QK): TMEM lane i, column m1 (+4 per K step) <- token 32*m1 + i.
-        // Each group writes its share of the K steps.
-        auto write_sfk = [&](int j) -> bool {
-            const int s = j % C::NS;
-            if (!tc::mbar_wait(&full[s], (j / C::NS) & 1, abort_flag, kWaitLimit)) return false;
-            const uint8_t* ks = smem + C::SM_STAGES + s * C::STAGE + C::OFF_KS;
-#pragma unroll
-            for (int kk = 0; kk < C::KS / C::NSG; ++kk) {
-                const int kstep = grp * (C::KS / C::NSG) + kk;
-                uint32_t v0, v1, v2, v3;
-                if constexpr (B == 16) {
-                    const uint2 p0 = *reinterpret_cast<const uint2*>(ks + 16 * lane + 8 * kstep);
-                    const uint2 p1 = *reinterpret_cast<const uint2*>(ks + C::KS_PAGE + 16 * lane + 8 * kstep);
-                    v0 = p0.x; v1 = p0.y; v2 = p1.x; v3 = p1.y;
-                } else {
-                    const uint32_t p0 = *reinterpret_cast<const uint32_t*>(ks + 8 * lane + 4 * kstep);
-                    const uint32_t p1 = *reinterpret_cast<const uint32_t*>(ks + C::KS_PAGE + 8 * lane + 4 * kstep);
-                    v0 = p0 & 0xffffu; v1 = p0 >> 16; v2 = p1 & 0xffffu; v3 = p1 >> 16;
-                }
-                tc::tmem_st4(tq + C::T_SFK + (j & 1) * 4 * C::KS + kstep * 4, v0, v1, v2, v3);
-            }
-            tc::tmem_wait_st();
-            tc::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&sfk_ready[j & 1]);
-            return true;
-        };
-        bad |= !write_sfk(0);
-
+        if (lane == 0) tc::mbar_arrive(q_ready);
         float m_run[HG], l_part[HG], o_acc[HG], corr_prev[HG];
 #pragma unroll
         for (int g = 0; g < HG; ++g) {
@@ -390,7 +385,11 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
             o_acc[g] = 0.0f;
             corr_prev[g] = 0.0f;
         }
-        const int tok_in_tile = 32 * qd + lane;
+        // TMEM lane 32 qd + lane holds slot (lane % 16) + 16 qd of page lane / 16 of the tile
+        const int page_of_thread = lane >> 4;
+        const int pos_in_page = 16 * qd + (lane & 15);
+        const int tok_in_tile = page_of_thread * kPageSlots + pos_in_page;
+        const int chan = 32 * qd + lane;   // O^T lane = value channel
         auto fold_o = [&](int j) -> bool {
             if (!tc::mbar_wait(&o_full[j & 1], (j >> 1) & 1, abort_flag, kWaitLimit)) return false;
             tc::tc_fence_after();
@@ -406,12 +405,12 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
         // sequence serves a token and its block maximum, so the block scale is
         // the one its largest member picks
         auto scaled_prob = [&](float sv, float mn) -> float { return __fmul_rn(exp2f(__fsub_rn(sv, mn)), alpha); };
-        const int page_of_thread = qd >> 1;
-        const int blk_in_page = (tok_in_tile & 63) / B;
 
         for (int j = 0; j < n; ++j) {
             const int s = j % C::NS, buf = j & 1, tile = tile0 + j;
-            if (j + 1 < n) bad |= !write_sfk(j + 1);
+            // the stage's bytes and page ids (producer writes) become visible to this thread
+            // through the stage barrier; it completed before QK(j), so this does not wait
+            if (!tc::mbar_wait(&full[s], (j / C::NS) & 1, abort_flag, kWaitLimit)) bad = true;
             // logits of this thread's token for the group's heads (q1 and q2 columns)
             if (!tc::mbar_wait(&s_full[buf], (j >> 1) & 1, abort_flag, kWaitLimit)) bad = true;
             tc::tc_fence_after();
@@ -421,37 +420,43 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
             tc::tmem_wait_ld();
             const int token = tile * kTileTokens + tok_in_tile;
             const bool valid = token < N && page_ids[s * 2 + page_of_thread] >= 0;
-            float sv[HG], bmax[HG];
-            float* rb = red + buf * G * 4;   // [G][4 quadrants] maxima of this tile
+            float sv[HG], hmax[HG];
+            float* rb = red + buf * G * 8;   // [G][page][qd] maxima of 16 consecutive tokens
 #pragma unroll
             for (int g = 0; g < HG; ++g) {
                 sv[g] = valid ? (__uint_as_float(s1[g]) + __uint_as_float(s2[g])) * lsc[gb + g] : -INFINITY;
-                // maximum over this thread's probability block (beta lanes), then the warp
+                // maximum over the 16 lanes (consecutive slots) of this half warp
                 float v = sv[g];
 #pragma unroll
-                for (int off = 1; off < B; off <<= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-                bmax[g] = v;
-                if constexpr (B < 32) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-                if (lane == 0) rb[(gb + g) * 4 + qd] = v;
+                for (int off = 1; off < 16; off <<= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+                hmax[g] = v;
+                if ((lane & 15) == 0) rb[(gb + g) * 8 + page_of_thread * 4 + qd] = v;
             }
             // one decision for the group's four warps: its flag is written only before this barrier
             if (bad || *abort_flag) sm_abort[grp] = 1;
             tc::named_bar_sync(bar_id, 128);
             if (sm_abort[grp]) break;
             float corr[HG];
-            uint8_t* pb = p_op + buf * C::P_BUF + page_of_thread * C::P_PAGE + (qd & 1) * 128 + (lane >> 3) * 4;
-            uint8_t* sfb = psf + (buf * 2 + page_of_thread) * 512 + blk_in_page;
+            // P operand: token pos of page p is K index pos -> 16-byte chunk pos/32, byte (pos%32)/2
+            uint8_t* pb = p_op + buf * C::P_BUF + page_of_thread * C::P_PAGE + (qd >> 1) * 128 + (qd & 1) * 8 +
+                          ((lane & 15) >> 3) * 4;
+            uint8_t* sfb = psf + (buf * 2 + page_of_thread) * 512 + pos_in_page / B;
 #pragma unroll
             for (int g = 0; g < HG; ++g) {
                 const int hh = gb + g;
-                const float4 m4 = *reinterpret_cast<const float4*>(rb + hh * 4);
-                const float mn = fmaxf(m_run[g], fmaxf(fmaxf(m4.x, m4.y), fmaxf(m4.z, m4.w)));
+                const float4 ma = *reinterpret_cast<const float4*>(rb + hh * 8);
+                const float4 mb = *reinterpret_cast<const float4*>(rb + hh * 8 + 4);
+                const float mt = fmaxf(fmaxf(fmaxf(ma.x, ma.y), fmaxf(ma.z, ma.w)), fmaxf(fmaxf(mb.x, mb.y), fmaxf(mb.z, mb.w)));
+                const float mn = fmaxf(m_run[g], mt);
                 corr[g] = exp2f(m_run[g] - mn);   // 0 on the split's first tile
                 m_run[g] = mn;
                 const float y = scaled_prob(sv[g], mn);    // 0 for masked tokens (sv = -inf)
                 l_part[g] = l_part[g] * corr[g] + y;       // l in units of alpha (cancels at the end)
-                // fused FP4 quantization of the probabilities over beta-token blocks
-                const float am = scaled_prob(bmax[g], mn);
+                // fused FP4 quantization of the probabilities over beta-token blocks: a
+                // 16-token block is this half warp; a 32-token block adds the neighbour warp's half
+                float bm = hmax[g];
+                if constexpr (B == 32) bm = fmaxf(bm, rb[hh * 8 + page_of_thread * 4 + (qd ^ 1)]);
+                const float am = scaled_prob(bm, mn);
                 uint32_t c;
                 float sigma;
                 if constexpr (FMT == BDFP4_NVFP4) {
@@ -467,7 +472,7 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                 word |= __shfl_xor_sync(0xffffffffu, word, 2);
                 word |= __shfl_xor_sync(0xffffffffu, word, 4);
                 if ((lane & 7) == 0) *reinterpret_cast<uint32_t*>(pb + (hh >> 3) * 256 + (hh & 7) * 16) = word;
-                if ((lane & (B - 1)) == 0) sfb[hh * 16] = (uint8_t)c;   // SFB row hh of this page
+                if ((lane & 15) == 0 && (B == 16 || (qd & 1) == 0)) sfb[hh * 16] = (uint8_t)c;   // SFB row hh
             }
             // V scale factors (group 0): blocks past the sequence end (or of a page that
             // was not loaded) are zeroed, so stale bytes are never multiplied
@@ -476,14 +481,13 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                 uint8_t* vs = smem + C::SM_STAGES + s * C::STAGE + C::OFF_VS;
                 if constexpr (B == 16) {
                     if (tail) {
-                        const int ch = tok_in_tile;   // thread = channel
 #pragma unroll
                         for (int p = 0; p < 2; ++p) {
                             const int t0 = tile * kTileTokens + p * kPageSlots;
                             int nvb = page_ids[s * 2 + p] >= 0 ? (N - t0 + B - 1) / B : 0;
                             nvb = nvb < 0 ? 0 : (nvb > C::SPB ? C::SPB : nvb);
                             for (int bb = nvb; bb < C::SPB; ++bb)
-                                vs[p * C::VS_PAGE + (ch & 31) * 16 + (ch >> 5) * 4 + bb] = 0;
+                                vs[p * C::VS_PAGE + (chan & 31) * 16 + (chan >> 5) * 4 + bb] = 0;
                         }
                     }
                 } else {
@@ -520,28 +524,28 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
         tc::named_bar_sync(bar_id, 128);
         if (sm_abort[grp]) *abort_flag = 1;
         if (!sm_abort[grp]) {
-            float* rl = red;   // [G][4] partial sums (the tile maxima are no longer read)
+            float* rl = red;   // [G][8] partial sums (the tile maxima are no longer read)
 #pragma unroll
             for (int g = 0; g < HG; ++g) {
                 float v = l_part[g];
 #pragma unroll
                 for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-                if (lane == 0) rl[(gb + g) * 4 + qd] = v;
+                if (lane == 0) rl[(gb + g) * 8 + qd] = v;
             }
             tc::named_bar_sync(bar_id, 128);
             // O and l both carry the factor alpha (P^ is alpha p quantized), so it cancels
             const float oscale = FMT == BDFP4_NVFP4 ? a.v_gscale[hk] : 1.0f;
-            const int ch = tok_in_tile;
+            const int ch = chan;
 #pragma unroll
             for (int g = 0; g < HG; ++g) {
                 const int hh = gb + g;
-                const float l = rl[hh * 4] + rl[hh * 4 + 1] + rl[hh * 4 + 2] + rl[hh * 4 + 3];
+                const float l = rl[hh * 8] + rl[hh * 8 + 1] + rl[hh * 8 + 2] + rl[hh * 8 + 3];
                 const int64_t row = (int64_t)b * a.H_q + h0 + hh;
                 if (nspl == 1) {
                     a.out[row * C::DV + ch] = __float2bfloat16(l > 0.0f ? o_acc[g] * oscale / l : 0.0f);
                 } else {
                     a.ws_o[(row * a.max_splits + split) * C::DV + ch] = o_acc[g] * oscale;
-                    if (tok_in_tile == 0) {
+                    if (chan == 0) {
                         a.ws_ml[(row * a.max_splits + split) * 2 + 0] = m_run[g];
                         a.ws_ml[(row * a.max_splits + split) * 2 + 1] = l;
                     }

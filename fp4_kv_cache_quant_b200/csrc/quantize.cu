@@ -61,7 +61,7 @@ __global__ void __launch_bounds__(256) quantize_k_kernel(const __nv_bfloat16* __
     } else {
         *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
     }
-    uint8_t* ks = k_scales + (page * H_kv + h) * (int64_t)(kPageSlots * DK / B);
+    uint8_t* ks = k_scales + (page * H_kv + h) * (int64_t)k_scale_page_bytes(DK, B);
     ks[k_scale_offset<B>(DK, slot, j)] = (uint8_t)code;
 }
 

@@ -32,9 +32,9 @@
  * E8M0 (MXFP4) bytes):
  *   k_pages  [num_pages][H_kv][64 * d_k / 2] bytes; within (page, head):
  *            [slot/8][elem/32][slot%8][16 bytes holding elements 32*(elem/32)..+31]
- *   k_scales [num_pages][H_kv][64 * d_k / beta]; within (page, head), scale of
- *            block blk (elements blk*beta..) of slot:
- *            [slot%32][blk / (64/beta)][slot/32][blk % (64/beta)]
+ *   k_scales [num_pages][H_kv][256 * ceil(d_k / (4 beta))]; within (page, head),
+ *            the scale of block blk (elements blk*beta..) of slot sits at
+ *            [blk/4][slot%16][slot/16][blk%4] (256-byte chunks)
  *   v_pages  [num_pages][H_kv][d_v * 64 / 2]; within (page, head):
  *            [chan/8][slot/32][chan%8][16 bytes holding slots 32*(slot/32)..+31]
  *   v_scales [num_pages][H_kv][d_v * 64 / beta]; scale of the beta-slot block
@@ -42,7 +42,10 @@
  * K blocks run along the head dim of one token (token-wise scaling); V blocks
  * run along beta consecutive slots of one page for one channel, because the
  * PV product reduces over tokens.  These are the tcgen05 block-scaled MMA
- * operand layouts, so pages move to shared memory with plain bulk copies.
+ * operand and scale-factor layouts: pages move to shared memory with plain
+ * bulk copies and scale chunks move on into tensor memory with tcgen05.cp
+ * (a 128-token tile takes MMA row 32*m + i from slot (i%16) + 16*m of page
+ * i/16, so each page contributes whole 16-byte scale rows).
  *
  * Supported shapes: (d_k, d_v) in {(128, 128), (576, 512)}; H_q / H_kv in
  * {1, 2, 4, 8, 16} or a multiple of 16 up to 128; anything else returns

@@ -224,7 +224,7 @@ def calibrate(k_cal, q_cal, v_cal, H_q: int, H_kv: int, flags: int = 0):
 def cache_sizes(num_pages: int, H_kv: int, d_k: int, d_v: int, fmt: int) -> dict:
     b = beta(fmt)
     return dict(k_pages=num_pages * H_kv * PAGE_SLOTS * d_k // 2,
-                k_scales=num_pages * H_kv * PAGE_SLOTS * d_k // b,
+                k_scales=num_pages * H_kv * 256 * ((d_k // b + 3) // 4),
                 v_pages=num_pages * H_kv * d_v * PAGE_SLOTS // 2,
                 v_scales=num_pages * H_kv * d_v * PAGE_SLOTS // b)
 

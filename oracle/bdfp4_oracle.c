@@ -204,15 +204,19 @@ static size_t k_nib_byte(int64_t page, int head, int H_kv, int d_k, int slot, in
     return base + in;
 }
 
-/* K scales of (page, head): d_k/beta codes per slot, grouped by 64-element
- * K step: [slot%32][kstep][slot/32][scale within kstep]. */
+/* K scales of (page, head): groups of four consecutive block codes of a slot
+ * share a 4-byte word; 256-byte chunks per group index:
+ * [blk/4][slot%16][slot/16][blk%4], i.e. 64 * 4 * ceil(d_k / (4 beta)) bytes
+ * per (page, head). */
+static size_t k_scale_page_bytes(int d_k, int beta)
+{
+    return (size_t)256 * (size_t)((d_k / beta + 3) / 4);
+}
+
 static size_t k_scale_byte(int64_t page, int head, int H_kv, int d_k, int beta, int slot, int blk)
 {
-    int per_step = 64 / beta, nsteps = d_k / 64;
-    size_t base = ((size_t)page * H_kv + head) * (size_t)(PAGE_SLOTS * d_k / beta);
-    size_t in = (size_t)(slot % 32) * (size_t)(2 * nsteps * per_step)
-              + (size_t)(blk / per_step) * (size_t)(2 * per_step)
-              + (size_t)(slot / 32) * (size_t)per_step + (size_t)(blk % per_step);
+    size_t base = ((size_t)page * H_kv + head) * k_scale_page_bytes(d_k, beta);
+    size_t in = (size_t)(blk / 4) * 256 + (size_t)(slot % 16) * 16 + (size_t)(slot / 16) * 4 + (size_t)(blk % 4);
     return base + in;
 }
 
