@@ -78,8 +78,10 @@ struct TcCfg {
     static constexpr int SM_P = SM_Q + Q_BYTES;
     static constexpr int SM_QSC = SM_P + 2 * P_BUF;                      // [NQ][8] query scale codes
     static constexpr int SM_PSF = (SM_QSC + NQ * 8 + 127) / 128 * 128;   // [2 buf][2 page][32 rows][16 B] P scales
-    static constexpr int SM_RED = SM_PSF + 2 * 2 * 512;                  // [2][G][8] 16-token maxima (floats)
-    static constexpr int SM_LSC = SM_RED + 2 * G * 8 * 4;               // [G] floats
+    // per S buffer: [G][4] warp maxima, then (MXFP4) [G][4][2] half-warp maxima (floats)
+    static constexpr int RED_BUF = (B == 32 ? 12 : 4) * G;
+    static constexpr int SM_RED = SM_PSF + 2 * 2 * 512;
+    static constexpr int SM_LSC = SM_RED + 2 * RED_BUF * 4;             // [G] floats
     static constexpr int SM_PAGES = SM_LSC + G * 4;                      // [NS][2] ints
     static constexpr int SM_BARS = (SM_PAGES + NS * 2 * 4 + 7) / 8 * 8;
     static constexpr int NBARS = 2 * NS + 9;
@@ -339,11 +341,13 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                 const float gq = FMT == BDFP4_NVFP4 ? (amax > 0.0f ? __fdiv_rn(amax, 2688.0f) : 1.0f) : 1.0f;
                 uint32_t c1, c2, p1[B / 8], p2[B / 8];
                 quantize_query_block<FMT, 128>(x, gq, dual, c1, p1, c2, p2);
-                // rows: q1 of head r -> r, q2 -> G + r; element e -> chunk e/32, byte (e%32)/2
+                // rows: group (r / HG) owns 2 HG consecutive rows, q1 of its heads then q2, so a
+                // softmax warp loads both logits of its heads with one TMEM load;
+                // element e -> chunk e/32, byte (e%32)/2
                 const int e0 = j * B;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
-                    const int row = half ? G + r : r;
+                    const int row = (r / HG) * 2 * HG + half * HG + r % HG;
                     const uint32_t* pk = half ? p2 : p1;
                     uint8_t* dst = q_op + (row / 8) * 512 + (e0 / 32) * 128 + (row % 8) * 16 + (e0 % 32) / 2;
                     if constexpr (B == 16) *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
@@ -401,78 +405,113 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
             return true;
         };
 
-        // alpha * exp2(s - m), the scaled probability; the same instruction
-        // sequence serves a token and its block maximum, so the block scale is
-        // the one its largest member picks
-        auto scaled_prob = [&](float sv, float mn) -> float { return __fmul_rn(exp2f(__fsub_rn(sv, mn)), alpha); };
+        // log2 of alpha: alpha * 2^(x - m) is evaluated as 2^(x - (m - log2 alpha))
+        const float la = alpha == kAlphaNV ? 11.0f : 0.0f;
+        float lsr[HG];
+#pragma unroll
+        for (int g = 0; g < HG; ++g) lsr[g] = lsc[gb + g];
+        const bool lo_half = lane < 16;
+        // P operand bytes: a lane pair (tokens 2i, 2i + 1 of a half warp) fills one byte of
+        // each head row; with two heads per pair step the even lane writes head g, the odd
+        // lane head g + 1.  Token pos of page p is K index pos: 16-byte chunk pos/32, byte (pos%32)/2
+        const int hsel = HG >= 2 ? (lane & 1) : 0;
+        const bool pstore = HG >= 2 || (lane & 1) == 0;
+        const bool sfstore = (lane & 15) < (HG >= 2 ? 2 : 1) && (B == 16 || (qd & 1) == 0);
+        const uint32_t psel = (lane & 1) ? 0x0004u : 0x0040u;   // byte 0 <- token 2i, byte 1 <- token 2i + 1
+        uint8_t* const pbyte = p_op + page_of_thread * C::P_PAGE + (qd >> 1) * 128 + (qd & 1) * 8 + ((lane & 15) >> 1) +
+                               hsel * 16;
+        uint8_t* const sfbyte = psf + page_of_thread * 512 + pos_in_page / B + hsel * 16;
 
         for (int j = 0; j < n; ++j) {
             const int s = j % C::NS, buf = j & 1, tile = tile0 + j;
             // the stage's bytes and page ids (producer writes) become visible to this thread
             // through the stage barrier; it completed before QK(j), so this does not wait
             if (!tc::mbar_wait(&full[s], (j / C::NS) & 1, abort_flag, kWaitLimit)) bad = true;
-            // logits of this thread's token for the group's heads (q1 and q2 columns)
+            // logits of this thread's token for the group's heads (q1 then q2 columns)
             if (!tc::mbar_wait(&s_full[buf], (j >> 1) & 1, abort_flag, kWaitLimit)) bad = true;
             tc::tc_fence_after();
-            uint32_t s1[HG], s2[HG];
-            tc::tmem_ld<HG>(tq + C::T_S + buf * C::NQ + gb, s1);
-            tc::tmem_ld<HG>(tq + C::T_S + buf * C::NQ + G + gb, s2);
+            uint32_t sr[2 * HG];
+            tc::tmem_ld<2 * HG>(tq + C::T_S + buf * C::NQ + 2 * gb, sr);
             tc::tmem_wait_ld();
             const int token = tile * kTileTokens + tok_in_tile;
             const bool valid = token < N && page_ids[s * 2 + page_of_thread] >= 0;
-            float sv[HG], hmax[HG];
-            float* rb = red + buf * G * 8;   // [G][page][qd] maxima of 16 consecutive tokens
+            // raw logits q1.k + q2.k (the positive factor lsc is applied later, so maxima
+            // commute with it) and their maxima over each half warp (16 consecutive slots)
+            float t[HG], hm_lo[HG], hm_hi[HG];
 #pragma unroll
             for (int g = 0; g < HG; ++g) {
-                sv[g] = valid ? (__uint_as_float(s1[g]) + __uint_as_float(s2[g])) * lsc[gb + g] : -INFINITY;
-                // maximum over the 16 lanes (consecutive slots) of this half warp
-                float v = sv[g];
+                t[g] = valid ? __uint_as_float(sr[g]) + __uint_as_float(sr[HG + g]) : -INFINITY;
+                hm_lo[g] = tc::redux_max_f32(lo_half ? t[g] : -INFINITY, 0xffffffffu);
+                hm_hi[g] = tc::redux_max_f32(lo_half ? -INFINITY : t[g], 0xffffffffu);
+            }
+            float* rw = red + buf * C::RED_BUF;
+            if (lane == 0) {
 #pragma unroll
-                for (int off = 1; off < 16; off <<= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-                hmax[g] = v;
-                if ((lane & 15) == 0) rb[(gb + g) * 8 + page_of_thread * 4 + qd] = v;
+                for (int g = 0; g < HG; ++g) {
+                    rw[(gb + g) * 4 + qd] = fmaxf(hm_lo[g], hm_hi[g]);
+                    if constexpr (MX)
+                        *reinterpret_cast<float2*>(rw + 4 * G + ((gb + g) * 4 + qd) * 2) = make_float2(hm_lo[g], hm_hi[g]);
+                }
             }
             // one decision for the group's four warps: its flag is written only before this barrier
             if (bad || *abort_flag) sm_abort[grp] = 1;
             tc::named_bar_sync(bar_id, 128);
             if (sm_abort[grp]) break;
-            float corr[HG];
-            // P operand: token pos of page p is K index pos -> 16-byte chunk pos/32, byte (pos%32)/2
-            uint8_t* pb = p_op + buf * C::P_BUF + page_of_thread * C::P_PAGE + (qd >> 1) * 128 + (qd & 1) * 8 +
-                          ((lane & 15) >> 3) * 4;
-            uint8_t* sfb = psf + (buf * 2 + page_of_thread) * 512 + pos_in_page / B;
+            float y[HG], am[HG], corr[HG];
+            uint32_t mxc[HG];   // MXFP4 block scale codes
 #pragma unroll
             for (int g = 0; g < HG; ++g) {
-                const int hh = gb + g;
-                const float4 ma = *reinterpret_cast<const float4*>(rb + hh * 8);
-                const float4 mb = *reinterpret_cast<const float4*>(rb + hh * 8 + 4);
-                const float mt = fmaxf(fmaxf(fmaxf(ma.x, ma.y), fmaxf(ma.z, ma.w)), fmaxf(fmaxf(mb.x, mb.y), fmaxf(mb.z, mb.w)));
-                const float mn = fmaxf(m_run[g], mt);
-                corr[g] = exp2f(m_run[g] - mn);   // 0 on the split's first tile
+                const float4 w4 = *reinterpret_cast<const float4*>(rw + (gb + g) * 4);
+                const float mt = fmaxf(fmaxf(w4.x, w4.y), fmaxf(w4.z, w4.w));
+                const float mn = fmaxf(m_run[g], mt * lsr[g]);
+                const float mz = mn == -INFINITY ? 0.0f : mn;
+                corr[g] = tc::ex2_approx(m_run[g] - mz);   // 0 on the split's first tile
                 m_run[g] = mn;
-                const float y = scaled_prob(sv[g], mn);    // 0 for masked tokens (sv = -inf)
-                l_part[g] = l_part[g] * corr[g] + y;       // l in units of alpha (cancels at the end)
-                // fused FP4 quantization of the probabilities over beta-token blocks: a
-                // 16-token block is this half warp; a 32-token block adds the neighbour warp's half
-                float bm = hmax[g];
-                if constexpr (B == 32) bm = fmaxf(bm, rb[hh * 8 + page_of_thread * 4 + (qd ^ 1)]);
-                const float am = scaled_prob(bm, mn);
-                uint32_t c;
-                float sigma;
-                if constexpr (FMT == BDFP4_NVFP4) {
-                    c = e4m3_encode(__fmul_rn(am, 1.0f / 6.0f));
-                    sigma = e4m3_value_hw(c);
+                const float base = mz - la;
+                // the same two instructions give a token's scaled probability and its block's
+                // maximum, so the block scale is the one its largest member picks
+                y[g] = tc::ex2_approx(fmaf(t[g], lsr[g], -base));   // 0 for masked tokens
+                l_part[g] = fmaf(l_part[g], corr[g], y[g]);         // l in units of alpha (cancels at the end)
+                float bm = lo_half ? hm_lo[g] : hm_hi[g];
+                if constexpr (!MX) {
+                    am[g] = tc::ex2_approx(fmaf(bm, lsr[g], -base));
                 } else {
-                    c = mx_scale_code(am);
-                    sigma = e8m0_value(c);
+                    // a 32-token block adds the neighbour warp's half of the same page.  The
+                    // OCP MX shared exponent is taken in the log domain: the block maximum is
+                    // 2^d with d = x_b - m, so floor(log2) = floor(d) exactly (d = 0 for the
+                    // tile's largest logit), and the element is 2^(x - m - e) for the scale 2^e
+                    bm = fmaxf(bm, rw[4 * G + ((gb + g) * 4 + (qd ^ 1)) * 2 + page_of_thread]);
+                    const float d = __fsub_rn(__fmul_rn(bm, lsr[g]), mz);
+                    const int c = max(__float2int_rd(fmaxf(d, -256.0f)) + 125, 0);
+                    mxc[g] = (uint32_t)c;
+                    am[g] = tc::ex2_approx(fmaf(t[g], lsr[g], -(mz + (float)(c - 127))));
                 }
-                const uint32_t e = sigma > 0.0f ? e2m1_encode(__fdividef(y, sigma)) : 0u;
-                uint32_t word = e << (4 * (lane & 7));
-                word |= __shfl_xor_sync(0xffffffffu, word, 1);
-                word |= __shfl_xor_sync(0xffffffffu, word, 2);
-                word |= __shfl_xor_sync(0xffffffffu, word, 4);
-                if ((lane & 7) == 0) *reinterpret_cast<uint32_t*>(pb + (hh >> 3) * 256 + (hh & 7) * 16) = word;
-                if ((lane & 15) == 0 && (B == 16 || (qd & 1) == 0)) sfb[hh * 16] = (uint8_t)c;   // SFB row hh
+            }
+            // fused FP4 quantization of the probabilities, two heads per conversion
+            uint8_t* const pb = pbyte + buf * C::P_BUF;
+            uint8_t* const sfb = sfbyte + buf * 2 * 512;
+#pragma unroll
+            for (int g = 0; g < HG; g += 2) {
+                const int g1 = HG >= 2 ? g + 1 : g;
+                uint32_t codes;
+                float q0, q1;
+                if constexpr (FMT == BDFP4_NVFP4) {
+                    codes = tc::e4m3x2_encode(__fmul_rn(am[g], 1.0f / 6.0f), __fmul_rn(am[g1], 1.0f / 6.0f));
+                    const float2 sg = tc::e4m3x2_value(codes);
+                    // a zero scale zeroes the whole block inside the MMA, whatever the element codes
+                    q0 = y[g] * tc::rcp_approx(sg.x);
+                    q1 = y[g1] * tc::rcp_approx(sg.y);
+                } else {
+                    codes = mxc[g] | (mxc[g1] << 8);
+                    q0 = am[g];    // the element already divided by its block scale
+                    q1 = am[g1];
+                }
+                const uint32_t mine = e2m1x2_encode(q0, q1);   // head g in bits 0..3, head g1 in 4..7
+                const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
+                const uint32_t w = __byte_perm(mine, other, psel) >> (4 * hsel);
+                const int hr = gb + g;
+                if (pstore) pb[(hr >> 3) * 256 + (hr & 7) * 16] = (uint8_t)((w & 0xfu) | ((w >> 4) & 0xf0u));
+                if (sfstore) sfb[hr * 16] = (uint8_t)(codes >> (8 * hsel));   // SFB rows hr, hr + 1
             }
             // V scale factors (group 0): blocks past the sequence end (or of a page that
             // was not loaded) are zeroed, so stale bytes are never multiplied

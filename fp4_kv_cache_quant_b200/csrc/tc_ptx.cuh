@@ -4,6 +4,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda_fp16.h>
 
 namespace bdfp4 {
 namespace tc {
@@ -200,6 +201,41 @@ __device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdes
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                  : "memory");
+}
+
+// Maximum of v over the lanes of membermask (every lane of the mask must take part).
+__device__ __forceinline__ float redux_max_f32(float v, uint32_t mask) {
+    float r;
+    asm volatile("redux.sync.max.f32 %0, %1, %2;" : "=f"(r) : "f"(v), "r"(mask));
+    return r;
+}
+
+// 2^x by the special-function unit (approximate, subnormal results flushed to 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+// Two unsigned fp32 values to E4M3FN (nearest, ties to even, saturating):
+// lo's code in bits 0..7, hi's in bits 8..15.
+__device__ __forceinline__ uint32_t e4m3x2_encode(float lo, float hi) {
+    uint16_t packed;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(packed) : "f"(hi), "f"(lo));
+    return packed;
+}
+
+// Values of the two E4M3 codes in bits 0..7 and 8..15 (exact through fp16).
+__device__ __forceinline__ float2 e4m3x2_value(uint32_t codes) {
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((unsigned short)(codes & 0xffffu)));
+    return __half22float2(*reinterpret_cast<const __half2*>(&h2));
+}
+
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
