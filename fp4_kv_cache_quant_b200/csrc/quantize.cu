@@ -6,8 +6,9 @@
 // Thread mapping: one thread per scale block of a row (beta = 16 or 32
 // consecutive channels), so the Hadamard butterflies of stages below beta run
 // in registers and the wider stages are lane shuffles inside the row's thread
-// group; the scale search of a block then runs sequentially in its thread,
-// which fixes the fp64 error sum to left-to-right order.
+// group.  The key scale search then gives every candidate code of a block its
+// own thread (each fp64 error summed left to right) and one thread picks the
+// winner in window order.
 
 #include "bdfp4_device.cuh"
 #include "host_common.h"
@@ -16,6 +17,27 @@
 namespace bdfp4 {
 
 // ---------------------------------------------------------------- K append
+// Work split of the K append: every scale block of a row gets NC lanes, one per
+// candidate code of its search window (10 for NVFP4, 2 for MXFP4, padded), so
+// the window is searched in parallel; R rows share a 256-thread CTA.
+template <int FMT, int DK>
+struct KGeom {
+    using RG = RowGeom<FMT, DK>;
+    static constexpr int B = RG::beta;
+    static constexpr int NB = DK / B;                                  // scale blocks per row
+    static constexpr int NC = FMT == BDFP4_NVFP4 ? 16 : 2;             // candidate lanes per block
+    static constexpr int R = 256 / (NB * NC) >= 1 ? 256 / (NB * NC) : 1;
+    static constexpr int PAIRS = R * NB * NC;                           // (block, candidate) pairs
+    static constexpr int PAIRS_PAD = (PAIRS + 255) / 256 * 256;
+    static constexpr int T1 = (R * RG::rt + 31) / 32 * 32;             // transform threads (whole warps)
+    static_assert(T1 <= 256, "transform threads exceed the CTA");
+};
+
+// Phase 1 transforms R rows into shared memory (thread per block, butterflies
+// across the row's threads); phase 2 quantizes every block under every code of
+// its window and keeps the fp64 squared errors (each summed left to right);
+// phase 3 scans each window from its largest code down, keeping the first
+// least error, and stores the winner.  The choice is the sequential search's.
 template <int FMT, int DK>
 __global__ void __launch_bounds__(256) quantize_k_kernel(const __nv_bfloat16* __restrict__ k,
                                                          const int64_t* __restrict__ slot_mapping, int T, int H_kv,
@@ -23,93 +45,177 @@ __global__ void __launch_bounds__(256) quantize_k_kernel(const __nv_bfloat16* __
                                                          const float* __restrict__ k_gscale, uint8_t* k_pages,
                                                          uint8_t* k_scales, int64_t num_pages, int flags,
                                                          int32_t* dev_status) {
-    using RG = RowGeom<FMT, DK>;
-    constexpr int B = RG::beta;
-    constexpr int rows_per_block = 256 / RG::rt;
-    const int j = threadIdx.x % RG::rt;
-    const int64_t row = (int64_t)blockIdx.x * rows_per_block + threadIdx.x / RG::rt;
-    const bool in_range = row < (int64_t)T * H_kv;
-    const int t = (int)(in_range ? row / H_kv : 0);
-    const int h = (int)(in_range ? row % H_kv : 0);
-    int64_t sm = in_range ? __ldg(slot_mapping + t) : -1;
-    if (sm >= num_pages * kPageSlots) {
-        if (j == 0) set_status(dev_status, BDFP4_DEV_BAD_SLOT);
-        sm = -1;
-    }
-    // whole warps stay converged through the shuffles; inactive rows compute on zeros
-    const bool active = sm >= 0 && j < RG::tpr;
-    float x[B];
-    if (active) {
-        load_bf16_block<B>(k + ((int64_t)t * H_kv + h) * DK, j * B, x);
-    } else {
+    using KG = KGeom<FMT, DK>;
+    using RG = typename KG::RG;
+    constexpr int B = KG::B, NB = KG::NB, NC = KG::NC, R = KG::R;
+    __shared__ float xs[R][DK];
+    __shared__ double errs[KG::PAIRS_PAD];
+    __shared__ uint32_t pks[KG::PAIRS_PAD][B / 8];
+    __shared__ int win[R * NB];            // hi << 16 | lo
+    __shared__ long long slots[R];
+    __shared__ float gs[R];                // tensor scale of the row's head
+    const int tid = threadIdx.x;
+    const int64_t rows = (int64_t)T * H_kv;
+    const int64_t row0 = (int64_t)blockIdx.x * R;
+
+    if (tid < KG::T1) {
+        const int r = tid / RG::rt, j = tid % RG::rt;
+        const int64_t row = row0 + r;
+        const bool in_range = r < R && row < rows;
+        const int t = (int)(in_range ? row / H_kv : 0);
+        const int h = (int)(in_range ? row % H_kv : 0);
+        int64_t sm = in_range ? __ldg(slot_mapping + t) : -1;
+        if (sm >= num_pages * kPageSlots) {
+            if (j == 0) set_status(dev_status, BDFP4_DEV_BAD_SLOT);
+            sm = -1;
+        }
+        // whole warps stay converged through the shuffles; inactive rows compute on zeros
+        // the row is loaded whatever its slot id, so the two loads overlap
+        float x[B];
+        if (in_range && j < RG::tpr) {
+            load_bf16_block<B>(k + ((int64_t)t * H_kv + h) * DK, j * B, x);
+        } else {
 #pragma unroll
-        for (int i = 0; i < B; ++i) x[i] = 0.0f;
+            for (int i = 0; i < B; ++i) x[i] = 0.0f;
+        }
+        if (sm < 0) {
+#pragma unroll
+            for (int i = 0; i < B; ++i) x[i] = 0.0f;
+        }
+        const bool active = sm >= 0 && j < RG::tpr;
+        transform_block<FMT, DK, true>(x, smooth + (int64_t)h * DK, j, !(flags & BDFP4_FLAG_NO_HADAMARD));
+        if (active) {
+#pragma unroll
+            for (int i = 0; i < B; ++i) xs[r][j * B + i] = x[i];
+        }
+        if (r < R && j == 0) {
+            slots[r] = sm;
+            gs[r] = FMT == BDFP4_NVFP4 ? __ldg(k_gscale + h) : 1.0f;
+        }
     }
-    transform_block<FMT, DK, true>(x, smooth + (int64_t)h * DK, j, !(flags & BDFP4_FLAG_NO_HADAMARD));
-    if (!active) return;
-    const float g = FMT == BDFP4_NVFP4 ? __ldg(k_gscale + h) : 1.0f;
-    const uint32_t code = (flags & BDFP4_FLAG_NO_SCALE_SEARCH) ? plain_scale_code<FMT>(block_amax<B>(x), g)
-                                                                : search_scale<FMT>(x, g);
-    uint32_t packed[B / 8];
-    quantize_block<B>(x, block_sigma<FMT>(code, g), packed);
-    const int64_t page = sm / kPageSlots;
-    const int slot = (int)(sm % kPageSlots);
-    uint8_t* kp = k_pages + (page * H_kv + h) * (int64_t)(kPageSlots * DK / 2);
-    uint8_t* dst = kp + k_nib_offset(DK, slot, j * B);
-    if constexpr (B == 16) {
-        *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
-    } else {
-        *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    __syncthreads();
+
+    for (int p = tid; p < KG::PAIRS; p += 256) {
+        const int r = p / (NB * NC), bk = (p / NC) % NB, ci = p % NC;
+        if (slots[r] < 0) continue;
+        const float g = gs[r];
+        float x[B];
+#pragma unroll
+        for (int i = 0; i < B; ++i) x[i] = xs[r][bk * B + i];
+        const float amax = block_amax<B>(x);
+        const int c0 = (int)plain_scale_code<FMT>(amax, g);
+        int hi = c0, lo = c0;   // all-zero blocks and the plain rule keep c0
+        if (amax != 0.0f && !(flags & BDFP4_FLAG_NO_SCALE_SEARCH)) {
+            const int top = FMT == BDFP4_NVFP4 ? 126 : 254;
+            hi = min(c0 + (FMT == BDFP4_NVFP4 ? 7 : 1), top);
+            lo = max(c0 - (FMT == BDFP4_NVFP4 ? 2 : 0), 0);
+        }
+        if (ci == 0) win[r * NB + bk] = (hi << 16) | lo;
+        const int c = hi - ci;
+        if (c >= lo) errs[p] = quantize_block<B>(x, block_sigma<FMT>((uint32_t)c, g), pks[p]);
     }
-    uint8_t* ks = k_scales + (page * H_kv + h) * (int64_t)k_scale_page_bytes(DK, B);
-    ks[k_scale_offset<B>(DK, slot, j)] = (uint8_t)code;
+    __syncthreads();
+
+    for (int q = tid; q < R * NB; q += 256) {
+        const int r = q / NB, bk = q % NB;
+        const int64_t sm = slots[r];
+        if (sm < 0) continue;
+        const int h = (int)((row0 + r) % H_kv);
+        const int hi = win[q] >> 16, lo = win[q] & 0xffff;
+        const int base = q * NC;
+        int best = 0;
+        double best_err = errs[base];
+        for (int ci = 1; ci <= hi - lo; ++ci) {
+            if (errs[base + ci] < best_err) {
+                best = ci;
+                best_err = errs[base + ci];
+            }
+        }
+        const int64_t page = sm / kPageSlots;
+        const int slot = (int)(sm % kPageSlots);
+        uint8_t* kp = k_pages + (page * H_kv + h) * (int64_t)(kPageSlots * DK / 2);
+        uint8_t* dst = kp + k_nib_offset(DK, slot, bk * B);
+        const uint32_t* pk = pks[base + best];
+        if constexpr (B == 16) {
+            *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
+        } else {
+            *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+        uint8_t* ks = k_scales + (page * H_kv + h) * (int64_t)k_scale_page_bytes(DK, B);
+        ks[k_scale_offset<B>(DK, slot, bk)] = (uint8_t)(hi - best);
+    }
 }
 
 // ---------------------------------------------------------------- V append
-// One warp per (token, head); only the first token of each run within a
-// beta-slot block does work (see bdfp4_quantize_kv in bdfp4.h).
+// One thread per (token, head, channel); only the first token of each run
+// within a beta-slot block does work (see bdfp4_quantize_kv in bdfp4.h), for
+// the whole block of its channel.
+template <int DV>
+struct VGeom {
+    static constexpr int TPR = DV < 256 ? DV : 256;   // threads of a row in one CTA
+    static constexpr int RPC = 256 / TPR;             // rows per CTA
+    static constexpr int CPR = DV / TPR;              // CTAs per row
+};
+
 template <int FMT, int DV>
 __global__ void __launch_bounds__(256) quantize_v_kernel(const __nv_bfloat16* __restrict__ v,
                                                          const int64_t* __restrict__ slot_mapping, int T, int H_kv,
                                                          const float* __restrict__ v_gscale, uint8_t* v_pages,
                                                          uint8_t* v_scales, int64_t num_pages) {
     constexpr int B = Fmt<FMT>::beta;
-    const int lane = threadIdx.x & 31;
-    const int64_t row = (int64_t)blockIdx.x * 8 + threadIdx.x / 32;
+    using VG = VGeom<DV>;
+    const int64_t row = (int64_t)(blockIdx.x / VG::CPR) * VG::RPC + threadIdx.x / VG::TPR;
+    const int c = (int)(blockIdx.x % VG::CPR) * VG::TPR + threadIdx.x % VG::TPR;
     if (row >= (int64_t)T * H_kv) return;
     const int t = (int)(row / H_kv), h = (int)(row % H_kv);
+    // two rounds of independent loads: this token's and its predecessor's slot
+    // ids (the leader test), then the next B - 1 slot ids with the B rows a run can cover
     const int64_t sm = __ldg(slot_mapping + t);
+    const int64_t sm_prev = t > 0 ? __ldg(slot_mapping + t - 1) : -2;
     if (sm < 0 || sm >= num_pages * kPageSlots) return;  // bad slots are reported by the K kernel
     const int slot = (int)(sm % kPageSlots);
-    const bool leader = (slot % B == 0) || t == 0 || __ldg(slot_mapping + t - 1) != sm - 1;
+    const bool leader = (slot % B == 0) || t == 0 || sm_prev != sm - 1;
     if (!leader) return;
+    int64_t sm_next[B - 1];
+#pragma unroll
+    for (int i = 1; i < B; ++i) sm_next[i - 1] = t + i < T ? __ldg(slot_mapping + t + i) : -2;
+    const unsigned short* vb = reinterpret_cast<const unsigned short*>(v);
+    uint32_t raw[B];
+#pragma unroll
+    for (int i = 0; i < B; ++i) raw[i] = t + i < T ? (uint32_t)__ldg(vb + ((int64_t)(t + i) * H_kv + h) * DV + c) : 0u;
+    const float g = FMT == BDFP4_NVFP4 ? __ldg(v_gscale + h) : 1.0f;
+    // run: the following tokens on consecutive slots of the same block
     int n = 1;
-    while (t + n < T && __ldg(slot_mapping + t + n) == sm + n && (slot + n) / B == slot / B) ++n;
+    bool run = true;
+#pragma unroll
+    for (int i = 1; i < B; ++i) {
+        run = run && sm_next[i - 1] == sm + i && (slot + i) / B == slot / B;
+        n += run ? 1 : 0;
+    }
     const int first = slot - slot % B;
     const int64_t page = sm / kPageSlots;
-    const float g = FMT == BDFP4_NVFP4 ? __ldg(v_gscale + h) : 1.0f;
     uint8_t* vp = v_pages + (page * H_kv + h) * (int64_t)(DV * kPageSlots / 2);
     uint8_t* vs = v_scales + (page * H_kv + h) * (int64_t)(DV * kPageSlots / B);
-    const unsigned short* vb = reinterpret_cast<const unsigned short*>(v);
-    for (int c = lane; c < DV; c += 32) {
-        float x[B];
+    // slot first + i holds token t + (first + i - slot) when that lies in the run
+    float x[B];
 #pragma unroll
-        for (int i = 0; i < B; ++i) {
-            const int jt = first + i - slot;
-            x[i] = (jt >= 0 && jt < n) ? __uint_as_float((uint32_t)__ldg(vb + ((int64_t)(t + jt) * H_kv + h) * DV + c) << 16)
-                                       : 0.0f;
-        }
-        const uint32_t code = plain_scale_code<FMT>(block_amax<B>(x), g);
-        uint32_t packed[B / 8];
-        quantize_block<B>(x, block_sigma<FMT>(code, g), packed);
-        uint8_t* dst = vp + v_nib_offset(c, first);
-        if constexpr (B == 16) {
-            *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
-        } else {
-            *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-        }
-        vs[v_scale_offset<B>(c, first / B)] = (uint8_t)code;
+    for (int i = 0; i < B; ++i) {
+        const int jt = first + i - slot;
+        uint32_t w = 0u;
+#pragma unroll
+        for (int u = 0; u < B; ++u) w = (u == jt) ? raw[u] : w;
+        x[i] = (jt >= 0 && jt < n) ? __uint_as_float(w << 16) : 0.0f;
     }
+    const uint32_t code = plain_scale_code<FMT>(block_amax<B>(x), g);
+    uint32_t packed[B / 8];
+    quantize_block<B>(x, block_sigma<FMT>(code, g), packed);
+    uint8_t* dst = vp + v_nib_offset(c, first);
+    if constexpr (B == 16) {
+        *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+    } else {
+        *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    }
+    vs[v_scale_offset<B>(c, first / B)] = (uint8_t)code;
 }
 
 template <int FMT, int DK>
@@ -254,14 +360,13 @@ template <int FMT, int DK, int DV>
 static void launch_quantize_kv(const void* k, const void* v, const int64_t* slot_mapping, int T, int H_kv,
                                const bdfp4_kv_params* kv, void* k_pages, void* k_scales, void* v_pages,
                                void* v_scales, int64_t num_pages, int flags, int32_t* dev_status, cudaStream_t st) {
-    using RG = RowGeom<FMT, DK>;
     const int64_t rows = (int64_t)T * H_kv;
-    const int rows_per_block = 256 / RG::rt;
-    const int64_t kblocks = (rows + rows_per_block - 1) / rows_per_block;
+    const int64_t kblocks = (rows + KGeom<FMT, DK>::R - 1) / KGeom<FMT, DK>::R;
     quantize_k_kernel<FMT, DK><<<(unsigned)kblocks, 256, 0, st>>>(
         (const __nv_bfloat16*)k, slot_mapping, T, H_kv, kv->smooth, kv->k_gscale, (uint8_t*)k_pages,
         (uint8_t*)k_scales, num_pages, flags, dev_status);
-    const int64_t vblocks = (rows + 7) / 8;
+    using VG = VGeom<DV>;
+    const int64_t vblocks = (rows + VG::RPC - 1) / VG::RPC * VG::CPR;
     quantize_v_kernel<FMT, DV><<<(unsigned)vblocks, 256, 0, st>>>((const __nv_bfloat16*)v, slot_mapping, T, H_kv,
                                                                   kv->v_gscale, (uint8_t*)v_pages,
                                                                   (uint8_t*)v_scales, num_pages);
