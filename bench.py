@@ -49,6 +49,19 @@ def algorithmic_bytes(sp, seq_lens, fmt: int) -> int:
     return tok * per_tok + pages * 4 + sp.B * sp.H_q * (sp.d_k + sp.d_v) * 2
 
 
+DECODE_SOURCES = ("decode_tc.cu", "tc_ptx.cuh", "bdfp4_device.cuh", "quant_device.cuh", "decode_common.cuh")
+
+
+def decode_source_hash() -> str:
+    """sha256 over the sources of the tensor-core decode kernel."""
+    import hashlib
+    h = hashlib.sha256()
+    for name in DECODE_SOURCES:
+        with open(os.path.join(ROOT, "fp4_kv_cache_quant_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 class ClockSampler:
     """SM clock and clock-event (throttle) reasons polled through NVML in a
     background thread during the timed region (read-only queries)."""
@@ -247,7 +260,8 @@ def run_ours(args, sp, fmt):
     tr_path = os.path.join(ROOT, "profiles", "decode_traffic.json")
     if os.path.exists(tr_path):
         rec = json.load(open(tr_path)).get(f"{args.config}_{args.fmt}")
-        if rec:
+        # the counters describe the kernel as captured: null once its sources changed
+        if rec and rec.get("source_sha256") == decode_source_hash():
             traffic = rec.get("bytes_per_launch")
     result = {
         "metric": "FP4 paged decode-attn KV tokens/s",
