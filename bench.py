@@ -40,6 +40,13 @@ CONFIG_TEXT = {
 }
 
 
+def bf16_algorithmic_bytes(sp, seq_lens) -> int:
+    """bf16 K and V + block table + Q and O in bf16 for one decode of the comparator."""
+    tok = int(np.sum(seq_lens))
+    pages = int(np.sum((np.asarray(seq_lens) + 63) // 64))
+    return tok * sp.H_kv * 2 * (sp.d_k + sp.d_v) + pages * 4 + sp.B * sp.H_q * (sp.d_k + sp.d_v) * 2
+
+
 def algorithmic_bytes(sp, seq_lens, fmt: int) -> int:
     """Packed KV + scales + block table + Q and O in bf16 for one decode."""
     beta = 16 if fmt == 0 else 32
@@ -117,8 +124,10 @@ class ClockSampler:
                 "reasons": sorted(v for k, v in names.items() if self.reasons & k), "samples": len(self.samples)}
 
 
-def setup_ours(sp, fmt, rank, device):
-    """Untimed: draw the workload on the GPU, calibrate, prefill-quantize the cache."""
+def setup_ours(sp, fmt, rank, device, with_bf16: bool = False):
+    """Untimed: draw the workload on the GPU, calibrate, prefill-quantize the
+    cache (and, with_bf16, fill the BF16-KV comparator's pages from the same
+    keys and values)."""
     import torch
 
     from fp4_kv_cache_quant_b200 import bdfp4
@@ -130,6 +139,7 @@ def setup_ours(sp, fmt, rank, device):
     kv = bdfp4.bdfp4_calibrate(kc, qc, vc, sp.H_q, sp.H_kv)
     cache = bdfp4.FP4Cache.empty(wl.num_pages, sp.H_kv, sp.d_k, sp.d_v, fmt, device=device)
     status = torch.zeros(1, dtype=torch.int32, device=device)
+    bcache = bdfp4.BF16Cache.empty(wl.num_pages, sp.H_kv, sp.d_k, device=device) if with_bf16 else None
     tails_k, tails_v, tails_sm = [], [], []
     q_bytes = 0
     t_quant, quant_bytes = 0.0, 0
@@ -138,6 +148,8 @@ def setup_ours(sp, fmt, rank, device):
         k = wl.keys(b, device)
         v = wl.values(b, device)
         sm = torch.from_numpy(wl.slot_mapping(b)).to(device)
+        if bcache is not None:
+            bdfp4.bdfp4_bf16_append(k, v, sm, bcache, dev_status=status)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         bdfp4.bdfp4_quantize_kv(k, v, sm, kv, cache, dev_status=status)
@@ -164,7 +176,8 @@ def setup_ours(sp, fmt, rank, device):
     ws = bdfp4.workspace_for(sp.B, sp.H_q, sp.d_v, wl.max_pages, chunk, device=device)
     out = torch.empty((sp.B, sp.H_q, sp.d_v), dtype=torch.bfloat16, device=device)
     return dict(wl=wl, kv=kv, cache=cache, status=status, tail_k=tail_k, tail_v=tail_v, tail_sm=tail_sm, q=q, bt=bt,
-                sl=sl, chunk=chunk, ws=ws, out=out, quant_gbs=quant_bytes / t_quant / 1e9, num_sms=num_sms)
+                sl=sl, chunk=chunk, ws=ws, out=out, quant_gbs=quant_bytes / t_quant / 1e9, num_sms=num_sms,
+                bcache=bcache)
 
 
 def run_ours(args, sp, fmt):
@@ -182,7 +195,7 @@ def run_ours(args, sp, fmt):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
 
-    S = setup_ours(sp, fmt, rank, device)
+    S = setup_ours(sp, fmt, rank, device, with_bf16=not args.no_bf16 and sp.d_k == 128)
     wl, kv, cache = S["wl"], S["kv"], S["cache"]
     stream = torch.cuda.current_stream(device)
 
@@ -220,6 +233,27 @@ def run_ours(args, sp, fmt):
     dec_s = statistics.mean(a.elapsed_time(b) for a, b in ev) / 1e3
     assert int(S["status"].item()) == 0, "device status set"
 
+    # the BF16-KV comparator on the same workload: decode calls timed alone
+    bf16_s = 0.0
+    if S["bcache"] is not None:
+        bout = torch.empty_like(S["out"])
+
+        def bf16_decode():
+            bdfp4.bdfp4_bf16_decode(S["q"], S["bcache"], S["bt"], S["sl"], sp.sm_scale, S["chunk"], S["ws"], bout,
+                                    dev_status=S["status"])
+
+        for _ in range(max(args.warmup, 3)):
+            bf16_decode()
+        torch.cuda.synchronize()
+        bev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for i in range(args.steps):
+            bev[i][0].record(stream)
+            bf16_decode()
+            bev[i][1].record(stream)
+        torch.cuda.synchronize()
+        bf16_s = statistics.mean(a.elapsed_time(b) for a, b in bev) / 1e3
+        assert int(S["status"].item()) == 0, "device status set"
+
     # end to end through the C ABI with host buffers: H2D of q and the tail rows,
     # D2H of the output, every step
     q_host = S["q"].cpu().pin_memory()
@@ -245,9 +279,9 @@ def run_ours(args, sp, fmt):
 
     tokens = float(np.sum(wl.seq_lens))
     if world > 1:
-        t = torch.tensor([step_s, dec_s, e2e_s], dtype=torch.float64, device=device)
+        t = torch.tensor([step_s, dec_s, e2e_s, bf16_s], dtype=torch.float64, device=device)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_s, dec_s, e2e_s = t.tolist()
+        step_s, dec_s, e2e_s, bf16_s = t.tolist()
         tokens *= world
     launches_per_step = 2 + 1 + (1 if S["chunk"] < (wl.max_pages * 64 + 127) // 128 else 0)
     alg = algorithmic_bytes(sp, wl.seq_lens, fmt)
@@ -296,6 +330,13 @@ def run_ours(args, sp, fmt):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
     }
+    if bf16_s > 0:
+        b_alg = bf16_algorithmic_bytes(sp, wl.seq_lens)
+        result["bf16_kv"] = {
+            "kernel": "decode_bf16_kernel + merge_splits_kernel (tcgen05 kind::f16, same tiles and pipeline)",
+            "decode_us": bf16_s * 1e6, "kv_tokens_per_s": tokens / bf16_s, "hbm_gbs": b_alg / bf16_s / 1e9,
+            "frac": b_alg / bf16_s / 1e9 / peak, "algorithmic_bytes_per_launch": b_alg,
+            "fp4_decode_speedup": bf16_s / dec_s}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(sp, fmt, budget_s=args.cpu_budget)
     if world > 1:
@@ -394,6 +435,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-bf16", action="store_true", help="skip the BF16-KV comparator")
     args = ap.parse_args()
     from fp4_kv_cache_quant_b200.workloads import spec
     sp = spec(args.config)

@@ -30,6 +30,8 @@ TILE_TOKENS = 128
 #: names of every entry point declared in include/bdfp4.h
 ENTRY_POINTS = ("bdfp4_calibrate", "bdfp4_quantize_kv", "bdfp4_quantize_q", "bdfp4_decode_plan",
                 "bdfp4_decode_workspace_size", "bdfp4_decode", "bdfp4_decode_noalloc", "bdfp4_status_string", "bdfp4_last_error")
+#: names of every entry point declared in include/bdfp4_bf16.h
+BF16_ENTRY_POINTS = ("bdfp4_bf16_append", "bdfp4_bf16_decode")
 
 #: size of the library's built-in scratch used by bdfp4_decode_noalloc
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -74,6 +76,10 @@ def load() -> ctypes.CDLL:
     L.bdfp4_status_string.restype = ctypes.c_char_p
     L.bdfp4_last_error.argtypes = []
     L.bdfp4_last_error.restype = ctypes.c_char_p
+    L.bdfp4_bf16_append.argtypes = [p, p, p, i, i, i, p, p, i64, p, p]
+    L.bdfp4_bf16_append.restype = i
+    L.bdfp4_bf16_decode.argtypes = [p, p, p, p, p, i, i, i, i, i, i64, f, i, p, sz, p, p, p]
+    L.bdfp4_bf16_decode.restype = i
     _lib = L
     return L
 
@@ -234,3 +240,43 @@ def bdfp4_decode_noalloc(q: torch.Tensor, cache: FP4Cache, block_table: torch.Te
                                      _ptr(dev_status), _stream(stream))
     _check(rc, "bdfp4_decode_noalloc")
     return out
+
+
+# ---------------------------------------------------------------- BF16-KV comparator (include/bdfp4_bf16.h)
+@dataclass
+class BF16Cache:
+    """bf16 K/V pages in the comparator's MMA operand layouts (16 KB per page and head at d = 128)."""
+    k_pages: torch.Tensor   # uint8 [num_pages, H_kv, 64 * d * 2]
+    v_pages: torch.Tensor   # uint8 [num_pages, H_kv, d * 64 * 2]
+    num_pages: int
+    H_kv: int
+    d: int
+
+    @staticmethod
+    def empty(num_pages: int, H_kv: int, d: int, device="cuda") -> "BF16Cache":
+        n = PAGE_SLOTS * d * 2
+        return BF16Cache(torch.empty((num_pages, H_kv, n), dtype=torch.uint8, device=device),
+                         torch.empty((num_pages, H_kv, n), dtype=torch.uint8, device=device), num_pages, H_kv, d)
+
+    def nbytes(self) -> int:
+        return self.k_pages.numel() + self.v_pages.numel()
+
+
+def bdfp4_bf16_append(k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor, cache: BF16Cache,
+                      dev_status: torch.Tensor | None = None, stream=None):
+    T, H_kv, d = k.shape
+    _check(load().bdfp4_bf16_append(_ptr(k), _ptr(v), _ptr(slot_mapping), T, H_kv, d, _ptr(cache.k_pages),
+                                    _ptr(cache.v_pages), cache.num_pages, _ptr(dev_status), _stream(stream)),
+           "bdfp4_bf16_append")
+
+
+def bdfp4_bf16_decode(q: torch.Tensor, cache: BF16Cache, block_table: torch.Tensor, seq_lens: torch.Tensor,
+                      sm_scale: float, chunk_tiles: int, workspace: torch.Tensor | None, out: torch.Tensor,
+                      dev_status: torch.Tensor | None = None, stream=None):
+    B, H_q, d = q.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().bdfp4_bf16_decode(_ptr(q), _ptr(cache.k_pages), _ptr(cache.v_pages), _ptr(block_table),
+                                    _ptr(seq_lens), B, H_q, cache.H_kv, d, block_table.shape[1], cache.num_pages,
+                                    float(sm_scale), int(chunk_tiles), _ptr(workspace), ws_bytes, _ptr(out),
+                                    _ptr(dev_status), _stream(stream)),
+           "bdfp4_bf16_decode")

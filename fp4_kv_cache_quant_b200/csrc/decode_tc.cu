@@ -27,9 +27,6 @@
 #include "quant_device.cuh"
 #include "tc_ptx.cuh"
 
-#ifndef BDFP4_TC_STAGES
-#define BDFP4_TC_STAGES 3
-#endif
 #ifndef BDFP4_TC_MIN_CTAS
 #define BDFP4_TC_MIN_CTAS 3
 #endif
@@ -43,7 +40,10 @@ struct TcCfg {
     static constexpr int NQ = (2 * G < 8) ? 8 : 2 * G;  // N of the QK MMA (q1 rows, q2 rows, padding)
     static constexpr int NP = (G < 8) ? 8 : G;          // N of the PV MMA
     static constexpr int KS = DK / 64;                   // MMA K steps of QK
-    static constexpr int NS = BDFP4_TC_STAGES;           // pipeline stages
+    // two shared-memory rings: K stages are released when QK completes, V stages
+    // when PV completes, so K (needed first) is prefetched further ahead
+    static constexpr int NSK = 4;
+    static constexpr int NSV = 3;
     // softmax warpgroups: warps w and w + 4 read the same TMEM lanes (tokens), so
     // two groups split the query heads of every tile between them
     static constexpr int NSG = G >= 2 ? 2 : 1;
@@ -60,21 +60,23 @@ struct TcCfg {
     static constexpr int KS_PAGE = 256 * NKG;            // K scale bytes per page (512 / 256)
     static constexpr int V_PAGE = DV * kPageSlots / 2;   // 4096
     static constexpr int VS_PAGE = DV * kPageSlots / B;
-    // a stage holds one 128-token tile: K [m1][page][1 KB] (MMA row 32 m1 + i <- slot
-    // (i%16) + 16 m1 of page i/16), V [page][4 KB], K scales [group][page][256 B],
-    // V scales [page][VS_PAGE]
+    // K stage of a 128-token tile: K [m1][page][1 KB] (MMA row 32 m1 + i <- slot
+    // (i%16) + 16 m1 of page i/16), then K scales [group][page][256 B]
     static constexpr int OFF_K = 0;
-    static constexpr int OFF_V = 2 * K_PAGE;
-    static constexpr int OFF_KS = OFF_V + 2 * V_PAGE;
-    static constexpr int OFF_VS = OFF_KS + 2 * KS_PAGE;
-    static constexpr int STAGE = OFF_VS + 2 * VS_PAGE;
+    static constexpr int OFF_KS = 2 * K_PAGE;
+    static constexpr int KSTAGE = OFF_KS + 2 * KS_PAGE;
+    // V stage: V [page][4 KB], then V scales [page][VS_PAGE]
+    static constexpr int OFF_V = 0;
+    static constexpr int OFF_VS = 2 * V_PAGE;
+    static constexpr int VSTAGE = OFF_VS + 2 * VS_PAGE;
     static constexpr int Q_BYTES = (NQ / 8) * (DK / 32) * 128;
     static constexpr int P_PAGE = (NP / 8) * 256;
     static constexpr int P_BUF = 2 * P_PAGE;
     static constexpr int SPB = 64 / B;                   // scale blocks per 64 tokens / elements
     // shared memory map
-    static constexpr int SM_STAGES = 0;
-    static constexpr int SM_Q = SM_STAGES + NS * STAGE;
+    static constexpr int SM_KST = 0;
+    static constexpr int SM_VST = SM_KST + NSK * KSTAGE;
+    static constexpr int SM_Q = SM_VST + NSV * VSTAGE;
     static constexpr int SM_P = SM_Q + Q_BYTES;
     static constexpr int SM_QSC = SM_P + 2 * P_BUF;                      // [NQ][8] query scale codes
     static constexpr int SM_PSF = (SM_QSC + NQ * 8 + 127) / 128 * 128;   // [2 buf][2 page][32 rows][16 B] P scales
@@ -82,9 +84,8 @@ struct TcCfg {
     static constexpr int RED_BUF = (B == 32 ? 12 : 4) * G;
     static constexpr int SM_RED = SM_PSF + 2 * 2 * 512;
     static constexpr int SM_LSC = SM_RED + 2 * RED_BUF * 4;             // [G] floats
-    static constexpr int SM_PAGES = SM_LSC + G * 4;                      // [NS][2] ints
-    static constexpr int SM_BARS = (SM_PAGES + NS * 2 * 4 + 7) / 8 * 8;
-    static constexpr int NBARS = 2 * NS + 9;
+    static constexpr int SM_BARS = (SM_LSC + G * 4 + 7) / 8 * 8;
+    static constexpr int NBARS = 2 * NSK + 2 * NSV + 7;
     static constexpr int SM_MISC = SM_BARS + NBARS * 8;                  // tmem slot, abort flags
     static constexpr int SMEM = SM_MISC + 16;
     // TMEM column map
@@ -123,11 +124,12 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
     uint8_t* psf = smem + C::SM_PSF;
     float* red = reinterpret_cast<float*>(smem + C::SM_RED);
     float* lsc = reinterpret_cast<float*>(smem + C::SM_LSC);
-    int* page_ids = reinterpret_cast<int*>(smem + C::SM_PAGES);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SM_BARS);
-    uint64_t* full = bars;                    // [NS] producer -> consumers
-    uint64_t* empty = bars + C::NS;           // [NS] PV done -> producer
-    uint64_t* s_full = bars + 2 * C::NS;      // [2] QK done -> softmax
+    uint64_t* kfull = bars;                   // [NSK] K tile landed -> MMA
+    uint64_t* kempty = kfull + C::NSK;        // [NSK] QK done -> producer
+    uint64_t* vfull = kempty + C::NSK;        // [NSV] V tile landed -> MMA, softmax
+    uint64_t* vempty = vfull + C::NSV;        // [NSV] PV done -> producer
+    uint64_t* s_full = vempty + C::NSV;       // [2] QK done -> softmax
     uint64_t* p_ready = s_full + 2;           // [2] P + scale factors ready -> MMA
     uint64_t* o_full = p_ready + 2;           // [2] PV done -> softmax
     uint64_t* q_ready = o_full + 2;           // query operand and its scale factors -> MMA
@@ -156,9 +158,13 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
     const int n = min(a.chunk_tiles, ntiles - tile0);   // tiles of this split (>= 1)
 
     if (tid == 0) {
-        for (int s = 0; s < C::NS; ++s) {
-            tc::mbar_init(&full[s], 1);
-            tc::mbar_init(&empty[s], 1);
+        for (int s = 0; s < C::NSK; ++s) {
+            tc::mbar_init(&kfull[s], 1);
+            tc::mbar_init(&kempty[s], 1);
+        }
+        for (int s = 0; s < C::NSV; ++s) {
+            tc::mbar_init(&vfull[s], 1);
+            tc::mbar_init(&vempty[s], 1);
         }
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(&s_full[i], 1);
@@ -182,11 +188,14 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
 
     if (warp == C::PRODUCER) {
         // ------------------------------------------------------------ producer
-        // The warp reads the page ids of 32 tiles at once (one tile per lane),
-        // so the dependent block-table load is off the per-tile path; lane 0
-        // then waits for a free stage and issues the tile's bulk copies.
+        // Step k issues the K half of tile k and the V half of tile k - 1, each
+        // into its own ring, so K runs one tile ahead of V.  The warp reads the
+        // page ids of 32 tiles at once (one tile per lane), so the dependent
+        // block-table load is off the per-tile path; lane 0 then waits for free
+        // stages and issues the bulk copies.
         bool ok = true;
-        for (int j0 = 0; ok && j0 < n; j0 += 32) {
+        int pv0 = -1, pv1 = -1;   // pages of the previous tile (the V half of this step)
+        for (int j0 = 0; ok && j0 <= n; j0 += 32) {
             int pg_l[2] = {-1, -1};
             if (j0 + lane < n) {
                 const int tile = tile0 + j0 + lane;
@@ -200,43 +209,65 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                     }
                 }
             }
-            const int kmax = min(32, n - j0);
-            for (int k = 0; k < kmax; ++k) {
-                const int j = j0 + k;
-                const int pg0 = __shfl_sync(0xffffffffu, pg_l[0], k);
-                const int pg1 = __shfl_sync(0xffffffffu, pg_l[1], k);
+            const int kmax = min(32, n + 1 - j0);
+            for (int kk = 0; kk < kmax; ++kk) {
+                const int k = j0 + kk;
+                const int pg0 = __shfl_sync(0xffffffffu, pg_l[0], kk);
+                const int pg1 = __shfl_sync(0xffffffffu, pg_l[1], kk);
                 if (lane == 0) {
-                    const int s = j % C::NS;
-                    if (j >= C::NS && !tc::mbar_wait(&empty[s], ((j / C::NS) - 1) & 1, abort_flag, kWaitLimit)) {
-                        ok = false;
-                    } else {
-                        const int pg[2] = {pg0, pg1};
-                        uint32_t bytes = 0;
+                    if (k < n) {
+                        const int s = k % C::NSK;
+                        if (k >= C::NSK && !tc::mbar_wait(&kempty[s], ((k / C::NSK) - 1) & 1, abort_flag, kWaitLimit)) {
+                            ok = false;
+                        } else {
+                            const int pg[2] = {pg0, pg1};
+                            uint32_t bytes = 0;
 #pragma unroll
-                        for (int p = 0; p < 2; ++p) {
-                            page_ids[s * 2 + p] = pg[p];
-                            if (pg[p] >= 0) bytes += C::K_PAGE + C::KS_PAGE + C::V_PAGE + C::VS_PAGE;
+                            for (int p = 0; p < 2; ++p)
+                                if (pg[p] >= 0) bytes += C::K_PAGE + C::KS_PAGE;
+                            tc::mbar_arrive_expect_tx(&kfull[s], bytes);
+                            uint8_t* stg = smem + C::SM_KST + s * C::KSTAGE;
+#pragma unroll
+                            for (int p = 0; p < 2; ++p) {
+                                if (pg[p] < 0) continue;
+                                const int64_t ph = (int64_t)pg[p] * a.H_kv + hk;
+#pragma unroll
+                                for (int c = 0; c < 4; ++c)   // slot groups 2c, 2c+1 -> MMA row groups 4c + 2p, +1
+                                    tc::bulk_g2s(stg + C::OFF_K + c * 2048 + p * 1024,
+                                                 a.k_pages + ph * C::K_PAGE + c * 1024, 1024, &kfull[s]);
+#pragma unroll
+                                for (int kg = 0; kg < C::NKG; ++kg)
+                                    tc::bulk_g2s(stg + C::OFF_KS + kg * 512 + p * 256,
+                                                 a.k_scales + ph * C::KS_PAGE + kg * 256, 256, &kfull[s]);
+                            }
                         }
-                        tc::mbar_arrive_expect_tx(&full[s], bytes);
-                        uint8_t* st = smem + C::SM_STAGES + s * C::STAGE;
+                    }
+                    if (ok && k >= 1) {
+                        const int v = k - 1, s = v % C::NSV;
+                        if (v >= C::NSV && !tc::mbar_wait(&vempty[s], ((v / C::NSV) - 1) & 1, abort_flag, kWaitLimit)) {
+                            ok = false;
+                        } else {
+                            const int pg[2] = {pv0, pv1};
+                            uint32_t bytes = 0;
 #pragma unroll
-                        for (int p = 0; p < 2; ++p) {
-                            if (pg[p] < 0) continue;
-                            const int64_t ph = (int64_t)pg[p] * a.H_kv + hk;
+                            for (int p = 0; p < 2; ++p)
+                                if (pg[p] >= 0) bytes += C::V_PAGE + C::VS_PAGE;
+                            tc::mbar_arrive_expect_tx(&vfull[s], bytes);
+                            uint8_t* stg = smem + C::SM_VST + s * C::VSTAGE;
 #pragma unroll
-                            for (int c = 0; c < 4; ++c)   // slot groups 2c, 2c+1 -> MMA row groups 4c + 2p, +1
-                                tc::bulk_g2s(st + C::OFF_K + c * 2048 + p * 1024, a.k_pages + ph * C::K_PAGE + c * 1024,
-                                             1024, &full[s]);
-#pragma unroll
-                            for (int kg = 0; kg < C::NKG; ++kg)
-                                tc::bulk_g2s(st + C::OFF_KS + kg * 512 + p * 256, a.k_scales + ph * C::KS_PAGE + kg * 256,
-                                             256, &full[s]);
-                            tc::bulk_g2s(st + C::OFF_V + p * C::V_PAGE, a.v_pages + ph * C::V_PAGE, C::V_PAGE, &full[s]);
-                            tc::bulk_g2s(st + C::OFF_VS + p * C::VS_PAGE, a.v_scales + ph * C::VS_PAGE, C::VS_PAGE,
-                                         &full[s]);
+                            for (int p = 0; p < 2; ++p) {
+                                if (pg[p] < 0) continue;
+                                const int64_t ph = (int64_t)pg[p] * a.H_kv + hk;
+                                tc::bulk_g2s(stg + C::OFF_V + p * C::V_PAGE, a.v_pages + ph * C::V_PAGE, C::V_PAGE,
+                                             &vfull[s]);
+                                tc::bulk_g2s(stg + C::OFF_VS + p * C::VS_PAGE, a.v_scales + ph * C::VS_PAGE,
+                                             C::VS_PAGE, &vfull[s]);
+                            }
                         }
                     }
                 }
+                pv0 = pg0;
+                pv1 = pg1;
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
             }
@@ -249,13 +280,14 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
             constexpr uint32_t idesc_pv = tc::idesc_fp4(C::NP, MX);
             const uint32_t q_addr = tc::smem_u32(q_op);
             const uint32_t p_addr = tc::smem_u32(p_op);
-            const uint32_t st_addr = tc::smem_u32(smem + C::SM_STAGES);
+            const uint32_t kst_addr = tc::smem_u32(smem + C::SM_KST);
+            const uint32_t vst_addr = tc::smem_u32(smem + C::SM_VST);
             const uint32_t psf_addr = tc::smem_u32(psf);
             auto issue_qk = [&](int j) -> bool {
-                const int s = j % C::NS, buf = j & 1;
-                if (!tc::mbar_wait(&full[s], (j / C::NS) & 1, abort_flag, kWaitLimit)) return false;
+                const int s = j % C::NSK, buf = j & 1;
+                if (!tc::mbar_wait(&kfull[s], (j / C::NSK) & 1, abort_flag, kWaitLimit)) return false;
                 tc::tc_fence_after();
-                const uint32_t kt = st_addr + s * C::STAGE + C::OFF_K;
+                const uint32_t kt = kst_addr + s * C::KSTAGE + C::OFF_K;
                 // K scale factors: each 512-byte group chunk (16 rows of page 0, then of
                 // page 1) is already in the 32 x 16-byte copy layout
 #pragma unroll
@@ -272,6 +304,7 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                                     tbase + C::T_SFQ + ks * 4, ks > 0);
                 }
                 tc::mma_commit(&s_full[buf]);
+                tc::mma_commit(&kempty[s]);   // the K stage is free once QK has read it
                 return true;
             };
             // the softmax warps quantize the query into shared memory and TMEM first
@@ -280,10 +313,11 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
             ok = ok && issue_qk(0);
             for (int j = 0; ok && j < n; ++j) {
                 if (j + 1 < n && !(ok = issue_qk(j + 1))) break;
-                const int s = j % C::NS, buf = j & 1;
+                const int s = j % C::NSV, buf = j & 1;
                 if (!(ok = tc::mbar_wait(&p_ready[buf], (j >> 1) & 1, abort_flag, kWaitLimit))) break;
+                if (!(ok = tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, kWaitLimit))) break;
                 tc::tc_fence_after();
-                const uint32_t vt = st_addr + s * C::STAGE + C::OFF_V;
+                const uint32_t vt = vst_addr + s * C::VSTAGE + C::OFF_V;
                 // scale factors of P (written by the softmax warps) and, for NVFP4, of V
                 // (the page's scale block is already in the 32 x 16-byte copy layout)
 #pragma unroll
@@ -301,7 +335,7 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                                     tbase + C::T_SFV + buf * 8 + p * 4, tbase + C::T_SFP + (buf * 2 + p) * 4, p > 0);
                 }
                 tc::mma_commit(&o_full[buf]);
-                tc::mma_commit(&empty[s]);
+                tc::mma_commit(&vempty[s]);
             }
             if (!ok) *abort_flag = 1;
         }
@@ -423,10 +457,7 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
         uint8_t* const sfbyte = psf + page_of_thread * 512 + pos_in_page / B + hsel * 16;
 
         for (int j = 0; j < n; ++j) {
-            const int s = j % C::NS, buf = j & 1, tile = tile0 + j;
-            // the stage's bytes and page ids (producer writes) become visible to this thread
-            // through the stage barrier; it completed before QK(j), so this does not wait
-            if (!tc::mbar_wait(&full[s], (j / C::NS) & 1, abort_flag, kWaitLimit)) bad = true;
+            const int buf = j & 1, tile = tile0 + j;
             // logits of this thread's token for the group's heads (q1 then q2 columns)
             if (!tc::mbar_wait(&s_full[buf], (j >> 1) & 1, abort_flag, kWaitLimit)) bad = true;
             tc::tc_fence_after();
@@ -434,7 +465,8 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
             tc::tmem_ld<2 * HG>(tq + C::T_S + buf * C::NQ + 2 * gb, sr);
             tc::tmem_wait_ld();
             const int token = tile * kTileTokens + tok_in_tile;
-            const bool valid = token < N && page_ids[s * 2 + page_of_thread] >= 0;
+            // (a page the block table gets wrong is reported through BDFP4_DEV_BAD_PAGE)
+            const bool valid = token < N;
             // raw logits q1.k + q2.k (the positive factor lsc is applied later, so maxima
             // commute with it) and their maxima over each half warp (16 consecutive slots)
             float t[HG], hm_lo[HG], hm_hi[HG];
@@ -513,28 +545,32 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                 if (pstore) pb[(hr >> 3) * 256 + (hr & 7) * 16] = (uint8_t)((w & 0xfu) | ((w >> 4) & 0xf0u));
                 if (sfstore) sfb[hr * 16] = (uint8_t)(codes >> (8 * hsel));   // SFB rows hr, hr + 1
             }
-            // V scale factors (group 0): blocks past the sequence end (or of a page that
-            // was not loaded) are zeroed, so stale bytes are never multiplied
+            // V scale factors (group 0): blocks past the sequence end are zeroed, so the
+            // bytes a page holds there are never multiplied.  The V stage can not be
+            // refilled before this tile's PV, so waiting for it here is safe.
             if (grp == 0) {
-                const bool tail = (tile + 1) * kTileTokens > N || page_ids[s * 2] < 0 || page_ids[s * 2 + 1] < 0;
-                uint8_t* vs = smem + C::SM_STAGES + s * C::STAGE + C::OFF_VS;
+                const int s = j % C::NSV;
+                const bool tail = (tile + 1) * kTileTokens > N;
+                uint8_t* vs = smem + C::SM_VST + s * C::VSTAGE + C::OFF_VS;
                 if constexpr (B == 16) {
                     if (tail) {
+                        if (!tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, kWaitLimit)) bad = true;
 #pragma unroll
                         for (int p = 0; p < 2; ++p) {
                             const int t0 = tile * kTileTokens + p * kPageSlots;
-                            int nvb = page_ids[s * 2 + p] >= 0 ? (N - t0 + B - 1) / B : 0;
+                            int nvb = (N - t0 + B - 1) / B;
                             nvb = nvb < 0 ? 0 : (nvb > C::SPB ? C::SPB : nvb);
                             for (int bb = nvb; bb < C::SPB; ++bb)
                                 vs[p * C::VS_PAGE + (chan & 31) * 16 + (chan >> 5) * 4 + bb] = 0;
                         }
                     }
                 } else {
+                    if (!tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, kWaitLimit)) bad = true;
                     uint32_t v[8];
 #pragma unroll
                     for (int p = 0; p < 2; ++p) {
                         const int t0 = tile * kTileTokens + p * kPageSlots;
-                        int nvb = page_ids[s * 2 + p] >= 0 ? (N - t0 + B - 1) / B : 0;
+                        int nvb = (N - t0 + B - 1) / B;
                         nvb = nvb < 0 ? 0 : (nvb > C::SPB ? C::SPB : nvb);
                         const uint32_t mask = nvb >= 2 ? 0xffffu : ((1u << (8 * nvb)) - 1u);
                         const uint2 w = *reinterpret_cast<const uint2*>(vs + p * C::VS_PAGE + 8 * lane);

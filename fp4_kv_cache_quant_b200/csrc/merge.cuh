@@ -1,0 +1,59 @@
+// merge.cuh -- log-sum-exp merge of split-KV partial outputs, shared by the
+// FP4 and BF16 decode paths.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "decode_common.cuh"
+
+namespace bdfp4 {
+
+// One CTA (128 threads) per (sequence, query head) row with more than one split:
+//   out = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s,  M = max_s m_s.
+template <int DV>
+__global__ void __launch_bounds__(128) merge_splits_kernel(const float* __restrict__ ws_o,
+                                                           const float* __restrict__ ws_ml,
+                                                           const int32_t* __restrict__ seq_lens, int H_q,
+                                                           int max_pages, int chunk_tiles, int max_splits,
+                                                           __nv_bfloat16* out) {
+    const int row = blockIdx.x;
+    const int b = row / H_q;
+    int N = seq_lens[b];
+    if (N < 0 || N > max_pages * kPageSlots) N = 0;
+    const int ns = num_splits(N, chunk_tiles);
+    if (ns <= 1) return;   // written by the decode kernel
+    // split weights 2^(m_s - M) through shared memory: the (m, l) pairs load in
+    // parallel, one per thread, instead of one dependent load per split
+    extern __shared__ float sw[];   // [ns] weights, then L
+    const float* ml = ws_ml + (int64_t)row * max_splits * 2;
+    float M = -INFINITY;
+    for (int s = threadIdx.x; s < ns; s += blockDim.x) M = fmaxf(M, ml[2 * s]);
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    __shared__ float wmax[4];
+    if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = M;
+    __syncthreads();
+    M = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
+    for (int s = threadIdx.x; s < ns; s += blockDim.x) sw[s] = exp2f(ml[2 * s] - M);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float L = 0.0f;
+        for (int s = 0; s < ns; ++s) L += ml[2 * s + 1] * sw[s];
+        sw[ns] = L;
+    }
+    __syncthreads();
+    const float L = sw[ns];
+    const float inv = L > 0.0f ? 1.0f / L : 0.0f;
+    for (int c = threadIdx.x; c < DV; c += blockDim.x) {
+        const float* o = ws_o + (int64_t)row * max_splits * DV + c;
+        float acc = 0.0f;
+#pragma unroll 4
+        for (int s = 0; s < ns; ++s) acc += o[(int64_t)s * DV] * sw[s];
+        out[(int64_t)row * DV + c] = __float2bfloat16(acc * inv);
+    }
+}
+
+// Dynamic shared memory of merge_splits_kernel: a weight per split and L.
+inline size_t merge_smem(int max_splits) { return ((size_t)max_splits + 1) * sizeof(float); }
+
+}  // namespace bdfp4

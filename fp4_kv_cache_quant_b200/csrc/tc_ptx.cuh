@@ -170,6 +170,23 @@ __host__ __device__ constexpr uint32_t idesc_fp4(int N, bool e8m0) {
     return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((e8m0 ? 1u : 0u) << 23) | ((128u >> 4) << 24);
 }
 
+// Instruction descriptor of a dense bf16 x bf16 -> fp32 MMA (kind::f16), both
+// operands K-major, M = 128, N a multiple of 16 in [16, 256]: D format F32
+// (bits 4-5 = 1), A and B format BF16 (bits 7-9 and 10-12 = 1), N >> 3 at
+// bit 17, M >> 4 at bit 24.
+__host__ __device__ constexpr uint32_t idesc_bf16(int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((128u >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 template <bool MX>
 __device__ __forceinline__ void mma_fp4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                         uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {

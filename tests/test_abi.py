@@ -31,6 +31,7 @@ def _declared():
 def test_exports_every_declared_entry_point(lib):
     names = _declared()
     assert set(bdfp4.ENTRY_POINTS) <= set(names)
+    assert set(bdfp4.BF16_ENTRY_POINTS) <= set(names)
     for n in names:
         assert hasattr(lib, n), n
 
@@ -107,3 +108,18 @@ def test_product_code_does_not_touch_the_oracle():
                 assert "oracle" not in re.sub(r"#.*|//.*", "", src).lower() or f == "workloads.py", f
     osrc = open(os.path.join(ROOT, "oracle", "bdfp4_oracle.c")).read()
     assert "#include \"" not in osrc
+
+
+def test_bf16_entry_points_reject_bad_arguments(lib):
+    L = bdfp4.load()
+    # d other than 128 is outside the compiled set; G = 3 is not a power of two; H_q % H_kv != 0
+    assert L.bdfp4_bf16_append(None, None, None, 1, 1, 64, None, None, 1, None, None) == -4
+    assert L.bdfp4_bf16_decode(None, None, None, None, None, 1, 3, 1, 128, 1, 1, 1.0, 1, None, 0, None, None,
+                               None) == -4
+    assert L.bdfp4_bf16_decode(None, None, None, None, None, 1, 4, 3, 128, 1, 1, 1.0, 1, None, 0, None, None,
+                               None) == -2
+    # null pointers with a supported shape, and negative sizes
+    assert L.bdfp4_bf16_decode(None, None, None, None, None, 1, 4, 1, 128, 1, 1, 1.0, 1, None, 0, None, None,
+                               None) == -1
+    assert L.bdfp4_bf16_append(None, None, None, -1, 1, 128, None, None, 1, None, None) == -1
+    assert L.bdfp4_bf16_append(None, None, None, 0, 1, 128, None, None, 1, None, None) == 0
