@@ -192,7 +192,9 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
         // into its own ring, so K runs one tile ahead of V.  The warp reads the
         // page ids of 32 tiles at once (one tile per lane), so the dependent
         // block-table load is off the per-tile path; lane 0 then waits for free
-        // stages and issues the bulk copies.
+        // stages, and one lane per bulk copy issues a step's copies together (a
+        // single thread issuing them one after another is slower than the tiles
+        // are consumed).
         bool ok = true;
         int pv0 = -1, pv1 = -1;   // pages of the previous tile (the V half of this step)
         for (int j0 = 0; ok && j0 <= n; j0 += 32) {
@@ -214,62 +216,62 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                 const int k = j0 + kk;
                 const int pg0 = __shfl_sync(0xffffffffu, pg_l[0], kk);
                 const int pg1 = __shfl_sync(0xffffffffu, pg_l[1], kk);
-                if (lane == 0) {
-                    if (k < n) {
-                        const int s = k % C::NSK;
-                        if (k >= C::NSK && !tc::mbar_wait(&kempty[s], ((k / C::NSK) - 1) & 1, abort_flag, kWaitLimit)) {
+                const bool do_k = k < n, do_v = k >= 1;
+                const int ks = k % C::NSK, v = k - 1, vsi = (k + C::NSV - 1) % C::NSV;
+                // K half: lane 0 claims the stage and posts the byte count, then lanes 0-7
+                // copy the K pieces (1 KB each: slot groups 2c, 2c+1 of page p -> MMA row
+                // groups 4c + 2p, +1) and lanes 8.. the K scale chunks, all at once
+                if (do_k) {
+                    if (lane == 0) {
+                        if (k >= C::NSK && !tc::mbar_wait(&kempty[ks], ((k / C::NSK) - 1) & 1, abort_flag, kWaitLimit))
                             ok = false;
-                        } else {
-                            const int pg[2] = {pg0, pg1};
-                            uint32_t bytes = 0;
-#pragma unroll
-                            for (int p = 0; p < 2; ++p)
-                                if (pg[p] >= 0) bytes += C::K_PAGE + C::KS_PAGE;
-                            tc::mbar_arrive_expect_tx(&kfull[s], bytes);
-                            uint8_t* stg = smem + C::SM_KST + s * C::KSTAGE;
-#pragma unroll
-                            for (int p = 0; p < 2; ++p) {
-                                if (pg[p] < 0) continue;
-                                const int64_t ph = (int64_t)pg[p] * a.H_kv + hk;
-#pragma unroll
-                                for (int c = 0; c < 4; ++c)   // slot groups 2c, 2c+1 -> MMA row groups 4c + 2p, +1
-                                    tc::bulk_g2s(stg + C::OFF_K + c * 2048 + p * 1024,
-                                                 a.k_pages + ph * C::K_PAGE + c * 1024, 1024, &kfull[s]);
-#pragma unroll
-                                for (int kg = 0; kg < C::NKG; ++kg)
-                                    tc::bulk_g2s(stg + C::OFF_KS + kg * 512 + p * 256,
-                                                 a.k_scales + ph * C::KS_PAGE + kg * 256, 256, &kfull[s]);
-                            }
-                        }
+                        else
+                            tc::mbar_arrive_expect_tx(&kfull[ks], (pg0 >= 0 ? C::K_PAGE + C::KS_PAGE : 0) +
+                                                                      (pg1 >= 0 ? C::K_PAGE + C::KS_PAGE : 0));
                     }
-                    if (ok && k >= 1) {
-                        const int v = k - 1, s = v % C::NSV;
-                        if (v >= C::NSV && !tc::mbar_wait(&vempty[s], ((v / C::NSV) - 1) & 1, abort_flag, kWaitLimit)) {
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
+                    uint8_t* stg = smem + C::SM_KST + ks * C::KSTAGE;
+                    if (lane < 8) {
+                        const int c = lane & 3, p = lane >> 2, pg = p ? pg1 : pg0;
+                        if (pg >= 0)
+                            tc::bulk_g2s(stg + C::OFF_K + c * 2048 + p * 1024,
+                                         a.k_pages + ((int64_t)pg * a.H_kv + hk) * C::K_PAGE + c * 1024, 1024, &kfull[ks]);
+                    } else if (lane < 8 + 2 * C::NKG) {
+                        const int kg = (lane - 8) >> 1, p = (lane - 8) & 1, pg = p ? pg1 : pg0;
+                        if (pg >= 0)
+                            tc::bulk_g2s(stg + C::OFF_KS + kg * 512 + p * 256,
+                                         a.k_scales + ((int64_t)pg * a.H_kv + hk) * C::KS_PAGE + kg * 256, 256,
+                                         &kfull[ks]);
+                    }
+                }
+                // V half of the previous tile: lanes 0-1 copy the V pages, 2-3 their scales
+                if (do_v) {
+                    if (lane == 0) {
+                        if (v >= C::NSV && !tc::mbar_wait(&vempty[vsi], ((v / C::NSV) - 1) & 1, abort_flag, kWaitLimit))
                             ok = false;
-                        } else {
-                            const int pg[2] = {pv0, pv1};
-                            uint32_t bytes = 0;
-#pragma unroll
-                            for (int p = 0; p < 2; ++p)
-                                if (pg[p] >= 0) bytes += C::V_PAGE + C::VS_PAGE;
-                            tc::mbar_arrive_expect_tx(&vfull[s], bytes);
-                            uint8_t* stg = smem + C::SM_VST + s * C::VSTAGE;
-#pragma unroll
-                            for (int p = 0; p < 2; ++p) {
-                                if (pg[p] < 0) continue;
-                                const int64_t ph = (int64_t)pg[p] * a.H_kv + hk;
+                        else
+                            tc::mbar_arrive_expect_tx(&vfull[vsi], (pv0 >= 0 ? C::V_PAGE + C::VS_PAGE : 0) +
+                                                                       (pv1 >= 0 ? C::V_PAGE + C::VS_PAGE : 0));
+                    }
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
+                    uint8_t* stg = smem + C::SM_VST + vsi * C::VSTAGE;
+                    if (lane < 4) {
+                        const int p = lane & 1, pg = p ? pv1 : pv0;
+                        if (pg >= 0) {
+                            const int64_t ph = (int64_t)pg * a.H_kv + hk;
+                            if (lane < 2)
                                 tc::bulk_g2s(stg + C::OFF_V + p * C::V_PAGE, a.v_pages + ph * C::V_PAGE, C::V_PAGE,
-                                             &vfull[s]);
+                                             &vfull[vsi]);
+                            else
                                 tc::bulk_g2s(stg + C::OFF_VS + p * C::VS_PAGE, a.v_scales + ph * C::VS_PAGE,
-                                             C::VS_PAGE, &vfull[s]);
-                            }
+                                             C::VS_PAGE, &vfull[vsi]);
                         }
                     }
                 }
                 pv0 = pg0;
                 pv1 = pg1;
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) break;
             }
         }
         if (!ok && lane == 0) *abort_flag = 1;
