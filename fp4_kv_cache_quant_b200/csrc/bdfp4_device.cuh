@@ -134,12 +134,12 @@ __device__ __forceinline__ uint32_t k_nib_offset(int d_k, int slot, int e) {
     return (uint32_t)((slot >> 3) * (d_k / 32) * 128 + (e >> 5) * 128 + (slot & 7) * 16 + ((e & 31) >> 1));
 }
 // K scales: four consecutive block codes of a slot share a 32-bit word;
-// [blk/4][slot%16][slot/16][blk%4] in 256-byte chunks.
+// [blk/4][slot%32][slot/32][blk%4] in 256-byte chunks.
 __host__ __device__ __forceinline__ int k_scale_page_bytes(int d_k, int beta) { return 256 * ((d_k / beta + 3) / 4); }
 template <int BETA>
 __device__ __forceinline__ uint32_t k_scale_offset(int d_k, int slot, int blk) {
     (void)d_k;
-    return (uint32_t)((blk >> 2) * 256 + (slot & 15) * 16 + (slot >> 4) * 4 + (blk & 3));
+    return (uint32_t)((blk >> 2) * 256 + (slot & 31) * 8 + (slot >> 5) * 4 + (blk & 3));
 }
 __device__ __forceinline__ uint32_t v_nib_offset(int chan, int slot) {
     return (uint32_t)((chan >> 3) * 256 + (slot >> 5) * 128 + (chan & 7) * 16 + ((slot & 31) >> 1));

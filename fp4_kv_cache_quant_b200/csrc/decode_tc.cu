@@ -60,11 +60,12 @@ struct TcCfg {
     static constexpr int KS_PAGE = 256 * NKG;            // K scale bytes per page (512 / 256)
     static constexpr int V_PAGE = DV * kPageSlots / 2;   // 4096
     static constexpr int VS_PAGE = DV * kPageSlots / B;
-    // K stage of a 128-token tile: K [m1][page][1 KB] (MMA row 32 m1 + i <- slot
-    // (i%16) + 16 m1 of page i/16), then K scales [group][page][256 B]
+    // K stage of a 128-token tile: K of page 0 (MMA rows 0-63) and page 1 (rows
+    // 64-127), then per scale group the 32 x 16-byte tcgen05.cp source: row i
+    // holds the scale words of rows i, 32 + i, 64 + i, 96 + i
     static constexpr int OFF_K = 0;
     static constexpr int OFF_KS = 2 * K_PAGE;
-    static constexpr int KSTAGE = OFF_KS + 2 * KS_PAGE;
+    static constexpr int KSTAGE = OFF_KS + NKG * 512;
     // V stage: V [page][4 KB], then V scales [page][VS_PAGE]
     static constexpr int OFF_V = 0;
     static constexpr int OFF_VS = 2 * V_PAGE;
@@ -80,8 +81,8 @@ struct TcCfg {
     static constexpr int SM_P = SM_Q + Q_BYTES;
     static constexpr int SM_QSC = SM_P + 2 * P_BUF;                      // [NQ][8] query scale codes
     static constexpr int SM_PSF = (SM_QSC + NQ * 8 + 127) / 128 * 128;   // [2 buf][2 page][32 rows][16 B] P scales
-    // per S buffer: [G][4] warp maxima, then (MXFP4) [G][4][2] half-warp maxima (floats)
-    static constexpr int RED_BUF = (B == 32 ? 12 : 4) * G;
+    // per S buffer: [G][4] warp maxima (floats)
+    static constexpr int RED_BUF = 4 * G;
     static constexpr int SM_RED = SM_PSF + 2 * 2 * 512;
     static constexpr int SM_LSC = SM_RED + 2 * RED_BUF * 4;             // [G] floats
     static constexpr int SM_BARS = (SM_LSC + G * 4 + 7) / 8 * 8;
@@ -159,7 +160,7 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
 
     if (tid == 0) {
         for (int s = 0; s < C::NSK; ++s) {
-            tc::mbar_init(&kfull[s], 1);
+            tc::mbar_init(&kfull[s], 1 + 32);   // the byte count, then the producer lanes' cp.async
             tc::mbar_init(&kempty[s], 1);
         }
         for (int s = 0; s < C::NSV; ++s) {
@@ -218,32 +219,36 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                 const int pg1 = __shfl_sync(0xffffffffu, pg_l[1], kk);
                 const bool do_k = k < n, do_v = k >= 1;
                 const int ks = k % C::NSK, v = k - 1, vsi = (k + C::NSV - 1) % C::NSV;
-                // K half: lane 0 claims the stage and posts the byte count, then lanes 0-7
-                // copy the K pieces (1 KB each: slot groups 2c, 2c+1 of page p -> MMA row
-                // groups 4c + 2p, +1) and lanes 8.. the K scale chunks, all at once
+                // K half: lane 0 claims the stage and posts the byte count; lanes 0-1 bulk-copy
+                // the two K pages and every lane copies, with cp.async, the 8 scale bytes of
+                // slots lane and 32 + lane of each page and scale group into row lane of the
+                // group's tcgen05.cp source, then arrives on the stage barrier once they land
                 if (do_k) {
                     if (lane == 0) {
                         if (k >= C::NSK && !tc::mbar_wait(&kempty[ks], ((k / C::NSK) - 1) & 1, abort_flag, kWaitLimit))
                             ok = false;
                         else
-                            tc::mbar_arrive_expect_tx(&kfull[ks], (pg0 >= 0 ? C::K_PAGE + C::KS_PAGE : 0) +
-                                                                      (pg1 >= 0 ? C::K_PAGE + C::KS_PAGE : 0));
+                            tc::mbar_arrive_expect_tx(&kfull[ks], (pg0 >= 0 ? C::K_PAGE : 0) + (pg1 >= 0 ? C::K_PAGE : 0));
                     }
                     ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (!ok) break;
                     uint8_t* stg = smem + C::SM_KST + ks * C::KSTAGE;
-                    if (lane < 8) {
-                        const int c = lane & 3, p = lane >> 2, pg = p ? pg1 : pg0;
+                    if (lane < 2) {
+                        const int pg = lane ? pg1 : pg0;
                         if (pg >= 0)
-                            tc::bulk_g2s(stg + C::OFF_K + c * 2048 + p * 1024,
-                                         a.k_pages + ((int64_t)pg * a.H_kv + hk) * C::K_PAGE + c * 1024, 1024, &kfull[ks]);
-                    } else if (lane < 8 + 2 * C::NKG) {
-                        const int kg = (lane - 8) >> 1, p = (lane - 8) & 1, pg = p ? pg1 : pg0;
-                        if (pg >= 0)
-                            tc::bulk_g2s(stg + C::OFF_KS + kg * 512 + p * 256,
-                                         a.k_scales + ((int64_t)pg * a.H_kv + hk) * C::KS_PAGE + kg * 256, 256,
-                                         &kfull[ks]);
+                            tc::bulk_g2s(stg + C::OFF_K + lane * C::K_PAGE,
+                                         a.k_pages + ((int64_t)pg * a.H_kv + hk) * C::K_PAGE, C::K_PAGE, &kfull[ks]);
                     }
+#pragma unroll
+                    for (int p = 0; p < 2; ++p) {
+                        const int pg = p ? pg1 : pg0;
+                        if (pg < 0) continue;
+                        const uint8_t* ksrc = a.k_scales + ((int64_t)pg * a.H_kv + hk) * C::KS_PAGE + lane * 8;
+#pragma unroll
+                        for (int kg = 0; kg < C::NKG; ++kg)
+                            tc::cp_async_8(stg + C::OFF_KS + kg * 512 + lane * 16 + p * 8, ksrc + kg * 256);
+                    }
+                    tc::cp_async_mbar_arrive_noinc(&kfull[ks]);
                 }
                 // V half of the previous tile: lanes 0-1 copy the V pages, 2-3 their scales
                 if (do_v) {
@@ -289,9 +294,11 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                 const int s = j % C::NSK, buf = j & 1;
                 if (!tc::mbar_wait(&kfull[s], (j / C::NSK) & 1, abort_flag, kWaitLimit)) return false;
                 tc::tc_fence_after();
+                // the scale rows came through cp.async (generic proxy); tcgen05.cp reads them
+                // through the async proxy
+                tc::fence_proxy_async_smem();
                 const uint32_t kt = kst_addr + s * C::KSTAGE + C::OFF_K;
-                // K scale factors: each 512-byte group chunk (16 rows of page 0, then of
-                // page 1) is already in the 32 x 16-byte copy layout
+                // K scale factors: each 512-byte group chunk is the 32 x 16-byte copy source
 #pragma unroll
                 for (int kg = 0; kg < C::NKG; ++kg)
                     tc::tmem_cp_32x128b_x4(tbase + C::T_SFK + (buf * C::NKG + kg) * 4,
@@ -425,10 +432,11 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
             o_acc[g] = 0.0f;
             corr_prev[g] = 0.0f;
         }
-        // TMEM lane 32 qd + lane holds slot (lane % 16) + 16 qd of page lane / 16 of the tile
-        const int page_of_thread = lane >> 4;
-        const int pos_in_page = 16 * qd + (lane & 15);
-        const int tok_in_tile = page_of_thread * kPageSlots + pos_in_page;
+        // TMEM lane 32 qd + lane holds token 32 qd + lane of the tile: slot 32 (qd % 2) + lane
+        // of page qd / 2, so a warp owns 32 consecutive slots of one page
+        const int page_of_thread = qd >> 1;
+        const int pos_in_page = 32 * (qd & 1) + lane;
+        const int tok_in_tile = 32 * qd + lane;
         const int chan = 32 * qd + lane;   // O^T lane = value channel
         auto fold_o = [&](int j) -> bool {
             if (!tc::mbar_wait(&o_full[j & 1], (j >> 1) & 1, abort_flag, kWaitLimit)) return false;
@@ -452,10 +460,11 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
         // lane head g + 1.  Token pos of page p is K index pos: 16-byte chunk pos/32, byte (pos%32)/2
         const int hsel = HG >= 2 ? (lane & 1) : 0;
         const bool pstore = HG >= 2 || (lane & 1) == 0;
-        const bool sfstore = (lane & 15) < (HG >= 2 ? 2 : 1) && (B == 16 || (qd & 1) == 0);
+        // the lanes that write a block's scale byte: the first (two) of the half warp
+        // (NVFP4, 16-token blocks) or of the warp (MXFP4, 32-token blocks)
+        const bool sfstore = (lane & (B - 1)) < (HG >= 2 ? 2 : 1);
         const uint32_t psel = (lane & 1) ? 0x0004u : 0x0040u;   // byte 0 <- token 2i, byte 1 <- token 2i + 1
-        uint8_t* const pbyte = p_op + page_of_thread * C::P_PAGE + (qd >> 1) * 128 + (qd & 1) * 8 + ((lane & 15) >> 1) +
-                               hsel * 16;
+        uint8_t* const pbyte = p_op + page_of_thread * C::P_PAGE + (qd & 1) * 128 + (lane >> 1) + hsel * 16;
         uint8_t* const sfbyte = psf + page_of_thread * 512 + pos_in_page / B + hsel * 16;
 
         for (int j = 0; j < n; ++j) {
@@ -483,8 +492,6 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
 #pragma unroll
                 for (int g = 0; g < HG; ++g) {
                     rw[(gb + g) * 4 + qd] = fmaxf(hm_lo[g], hm_hi[g]);
-                    if constexpr (MX)
-                        *reinterpret_cast<float2*>(rw + 4 * G + ((gb + g) * 4 + qd) * 2) = make_float2(hm_lo[g], hm_hi[g]);
                 }
             }
             // one decision for the group's four warps: its flag is written only before this barrier
@@ -506,15 +513,16 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                 // maximum, so the block scale is the one its largest member picks
                 y[g] = tc::ex2_approx(fmaf(t[g], lsr[g], -base));   // 0 for masked tokens
                 l_part[g] = fmaf(l_part[g], corr[g], y[g]);         // l in units of alpha (cancels at the end)
-                float bm = lo_half ? hm_lo[g] : hm_hi[g];
                 if constexpr (!MX) {
+                    // a 16-token block is this half warp
+                    const float bm = lo_half ? hm_lo[g] : hm_hi[g];
                     am[g] = tc::ex2_approx(fmaf(bm, lsr[g], -base));
                 } else {
-                    // a 32-token block adds the neighbour warp's half of the same page.  The
-                    // OCP MX shared exponent is taken in the log domain: the block maximum is
-                    // 2^d with d = x_b - m, so floor(log2) = floor(d) exactly (d = 0 for the
-                    // tile's largest logit), and the element is 2^(x - m - e) for the scale 2^e
-                    bm = fmaxf(bm, rw[4 * G + ((gb + g) * 4 + (qd ^ 1)) * 2 + page_of_thread]);
+                    // a 32-token block is this warp.  The OCP MX shared exponent is taken in the
+                    // log domain: the block maximum is 2^d with d = x_b - m, so floor(log2) =
+                    // floor(d) exactly (d = 0 for the tile's largest logit), and the element is
+                    // 2^(x - m - e) for the scale 2^e
+                    const float bm = fmaxf(hm_lo[g], hm_hi[g]);
                     const float d = __fsub_rn(__fmul_rn(bm, lsr[g]), mz);
                     const int c = max(__float2int_rd(fmaxf(d, -256.0f)) + 125, 0);
                     mxc[g] = (uint32_t)c;

@@ -220,6 +220,18 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
                  : "memory");
 }
 
+// Asynchronous 8-byte global -> shared copy (both addresses 8-byte aligned).
+__device__ __forceinline__ void cp_async_8(void* dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
+// Arrive on an mbarrier once every cp.async this thread has issued completes.
+// The arrival is not added to the expected count: the barrier's init count
+// must include it.
+__device__ __forceinline__ void cp_async_mbar_arrive_noinc(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // Maximum of v over the lanes of membermask (every lane of the mask must take part).
 __device__ __forceinline__ float redux_max_f32(float v, uint32_t mask) {
     float r;

@@ -34,7 +34,7 @@
  *            [slot/8][elem/32][slot%8][16 bytes holding elements 32*(elem/32)..+31]
  *   k_scales [num_pages][H_kv][256 * ceil(d_k / (4 beta))]; within (page, head),
  *            the scale of block blk (elements blk*beta..) of slot sits at
- *            [blk/4][slot%16][slot/16][blk%4] (256-byte chunks)
+ *            [blk/4][slot%32][slot/32][blk%4] (256-byte chunks)
  *   v_pages  [num_pages][H_kv][d_v * 64 / 2]; within (page, head):
  *            [chan/8][slot/32][chan%8][16 bytes holding slots 32*(slot/32)..+31]
  *   v_scales [num_pages][H_kv][d_v * 64 / beta]; scale of the beta-slot block
@@ -42,10 +42,11 @@
  * K blocks run along the head dim of one token (token-wise scaling); V blocks
  * run along beta consecutive slots of one page for one channel, because the
  * PV product reduces over tokens.  These are the tcgen05 block-scaled MMA
- * operand and scale-factor layouts: pages move to shared memory with plain
- * bulk copies and scale chunks move on into tensor memory with tcgen05.cp
- * (a 128-token tile takes MMA row 32*m + i from slot (i%16) + 16*m of page
- * i/16, so each page contributes whole 16-byte scale rows).
+ * operand and scale-factor layouts: each page moves to shared memory with one
+ * bulk copy per array and scale chunks move on into tensor memory with
+ * tcgen05.cp (a 128-token tile takes MMA rows 0-63 from its first page and
+ * 64-127 from its second; lane i of a K scale chunk holds the words of slots
+ * i and 32 + i of both pages, 8 contiguous bytes per page).
  *
  * Supported shapes: (d_k, d_v) in {(128, 128), (576, 512)}; H_q / H_kv in
  * {1, 2, 4, 8, 16} or a multiple of 16 up to 128; anything else returns

@@ -206,7 +206,7 @@ static size_t k_nib_byte(int64_t page, int head, int H_kv, int d_k, int slot, in
 
 /* K scales of (page, head): groups of four consecutive block codes of a slot
  * share a 4-byte word; 256-byte chunks per group index:
- * [blk/4][slot%16][slot/16][blk%4], i.e. 64 * 4 * ceil(d_k / (4 beta)) bytes
+ * [blk/4][slot%32][slot/32][blk%4], i.e. 64 * 4 * ceil(d_k / (4 beta)) bytes
  * per (page, head). */
 static size_t k_scale_page_bytes(int d_k, int beta)
 {
@@ -216,7 +216,7 @@ static size_t k_scale_page_bytes(int d_k, int beta)
 static size_t k_scale_byte(int64_t page, int head, int H_kv, int d_k, int beta, int slot, int blk)
 {
     size_t base = ((size_t)page * H_kv + head) * k_scale_page_bytes(d_k, beta);
-    size_t in = (size_t)(blk / 4) * 256 + (size_t)(slot % 16) * 16 + (size_t)(slot / 16) * 4 + (size_t)(blk % 4);
+    size_t in = (size_t)(blk / 4) * 256 + (size_t)(slot % 32) * 8 + (size_t)(slot / 32) * 4 + (size_t)(blk % 4);
     return base + in;
 }
 

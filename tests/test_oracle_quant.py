@@ -74,7 +74,7 @@ def test_cache_layout_golden_offsets(ora):
     """One token with a single non-zero channel lands where the layout
     definition says (offsets worked out by hand from it):
     K nibble byte = ((page*H_kv+head)*64*d/2) + (slot/8)*(d/32)*128 + (e/32)*128 + (slot%8)*16 + (e%32)/2
-    K scale byte  = ((page*H_kv+head)*256*ceil(d/64)) + (blk/4)*256 + (slot%16)*16 + (slot/16)*4 + blk%4
+    K scale byte  = ((page*H_kv+head)*256*ceil(d/64)) + (blk/4)*256 + (slot%32)*8 + (slot/32)*4 + blk%4
     V nibble byte = ((page*H_kv+head)*d*32) + (c/8)*256 + (slot/32)*128 + (c%8)*16 + (slot%32)/2
     V scale byte  = ((page*H_kv+head)*d*4) + (c/128)*512 + (c%32)*16 + ((c%128)/32)*4 + slot/16
     page 2, head 1 of 2, slot 37, channel 77, value 6.0, d = 128, NVFP4, g = 1, plain scale rule."""
@@ -91,8 +91,8 @@ def test_cache_layout_golden_offsets(ora):
     nz = {name: [(int(i), int(cache[name][i])) for i in np.nonzero(cache[name])[0]] for name in cache}
     # hand-computed: 20480 + 4*4*128 + 2*128 + 5*16 + 6 = 22870, odd element -> high nibble of E2M1(6)=7
     assert nz["k_pages"] == [(22870, 0x70)]
-    # 5*512 + 1*256 + 5*16 + 2*4 + 0 = 2904, E4M3(1.0) = 0x38
-    assert nz["k_scales"] == [(2904, 0x38)]
+    # 5*512 + 1*256 + 5*8 + 1*4 + 0 = 2860, E4M3(1.0) = 0x38
+    assert nz["k_scales"] == [(2860, 0x38)]
     # 20480 + 9*256 + 1*128 + 5*16 + 2 = 22994, odd slot -> high nibble
     assert nz["v_pages"] == [(22994, 0x70)]
     # 2560 + 0 + 13*16 + 2*4 + 2 = 2778
