@@ -292,12 +292,28 @@ static int max_splits_for(int max_pages, int chunk_tiles) {
     return std::max(1, (ntiles + chunk_tiles - 1) / chunk_tiles);
 }
 
+// Workspace regions: split partials (fp32 O, then (m, l)) when a sequence can
+// have more than one split, then the query images of the tensor-core path
+// (at most kQueryImageBytes per query head).
+constexpr size_t kQueryImageBytes = 640;
+
+struct WorkspaceMap {
+    size_t o_bytes, ml_bytes, q_off, total;
+};
+
+static WorkspaceMap workspace_map(int B, int H_q, int d_v, int max_splits) {
+    WorkspaceMap m{};
+    const size_t ms = max_splits > 1 ? (size_t)max_splits : 0;
+    m.o_bytes = (size_t)B * H_q * ms * d_v * sizeof(float);
+    m.ml_bytes = (size_t)B * H_q * ms * 2 * sizeof(float);
+    m.q_off = ((m.o_bytes + 255) / 256) * 256 + ((m.ml_bytes + 255) / 256) * 256;
+    m.total = m.q_off + (size_t)B * H_q * kQueryImageBytes;
+    return m;
+}
+
 extern "C" size_t bdfp4_decode_workspace_size(int B, int H_q, int d_v, int max_pages_per_seq, int chunk_tiles) {
     if (B <= 0 || H_q <= 0 || d_v <= 0 || max_pages_per_seq <= 0 || chunk_tiles <= 0) return 0;
-    const size_t ms = (size_t)max_splits_for(max_pages_per_seq, chunk_tiles);
-    const size_t o_bytes = (size_t)B * H_q * ms * d_v * sizeof(float);
-    const size_t ml_bytes = (size_t)B * H_q * ms * 2 * sizeof(float);
-    return ((o_bytes + 255) / 256) * 256 + ml_bytes;
+    return workspace_map(B, H_q, d_v, max_splits_for(max_pages_per_seq, chunk_tiles)).total;
 }
 
 extern "C" int bdfp4_decode_plan(const int32_t* host_seq_lens, int B, int H_kv, int num_sms) {
@@ -377,13 +393,14 @@ extern "C" int bdfp4_decode(const void* q, const void* k_pages, const void* k_sc
     }
     DecodeArgs a{};
     a.max_splits = max_splits_for(max_pages_per_seq, chunk_tiles);
-    if (a.max_splits > 1) {
-        const size_t need = bdfp4_decode_workspace_size(B, H_q, d_v, max_pages_per_seq, chunk_tiles);
-        if (!workspace || workspace_bytes < need) return BDFP4_ERR_WORKSPACE;
+    const bool tensor_core_path = d_k == 128 && G <= 16;
+    if (a.max_splits > 1 || tensor_core_path) {
+        const WorkspaceMap m = workspace_map(B, H_q, d_v, a.max_splits);
+        if (!workspace || workspace_bytes < m.total) return BDFP4_ERR_WORKSPACE;
         if (!aligned(workspace, 128)) return BDFP4_ERR_ALIGN;
-        const size_t o_bytes = (size_t)B * H_q * a.max_splits * d_v * sizeof(float);
         a.ws_o = (float*)workspace;
-        a.ws_ml = (float*)((char*)workspace + ((o_bytes + 255) / 256) * 256);
+        a.ws_ml = (float*)((char*)workspace + ((m.o_bytes + 255) / 256) * 256);
+        a.qpack = (uint8_t*)workspace + m.q_off;
     }
     a.q = (const __nv_bfloat16*)q;
     a.k_pages = (const uint8_t*)k_pages;

@@ -21,6 +21,7 @@ struct DecodeArgs {
     const float* v_gscale;
     float* ws_o;   // [B][H_q][max_splits][d_v] unnormalised partial outputs
     float* ws_ml;  // [B][H_q][max_splits][2]  (m in log2 units, l)
+    uint8_t* qpack;  // [B][H_kv] query images of the tensor-core path (written before the decode)
     __nv_bfloat16* out;
     int32_t* dev_status;
     int B, H_q, H_kv, max_pages, flags, chunk_tiles, max_splits;

@@ -74,19 +74,24 @@ struct TcCfg {
     static constexpr int P_PAGE = (NP / 8) * 256;
     static constexpr int P_BUF = 2 * P_PAGE;
     static constexpr int SPB = 64 / B;                   // scale blocks per 64 tokens / elements
+    // the query image of a (sequence, KV head), copied into shared memory in one
+    // piece: QK operand, its scale codes [NQ][8], the per-head logit scales [G]
+    static constexpr int LSC_BYTES = (G * 4 + 15) / 16 * 16;
+    static constexpr int QPACK = Q_BYTES + NQ * 8 + LSC_BYTES;
+    static constexpr int QTHREADS = (G * RowGeom<FMT, 128>::rt + 31) / 32 * 32;   // threads of prep_query_kernel
     // shared memory map
     static constexpr int SM_KST = 0;
     static constexpr int SM_VST = SM_KST + NSK * KSTAGE;
     static constexpr int SM_Q = SM_VST + NSV * VSTAGE;
-    static constexpr int SM_P = SM_Q + Q_BYTES;
-    static constexpr int SM_QSC = SM_P + 2 * P_BUF;                      // [NQ][8] query scale codes
-    static constexpr int SM_PSF = (SM_QSC + NQ * 8 + 127) / 128 * 128;   // [2 buf][2 page][32 rows][16 B] P scales
+    static constexpr int SM_QSC = SM_Q + Q_BYTES;
+    static constexpr int SM_LSC = SM_QSC + NQ * 8;
+    static constexpr int SM_P = SM_Q + QPACK;
+    static constexpr int SM_PSF = (SM_P + 2 * P_BUF + 127) / 128 * 128;  // [2 buf][2 page][32 rows][16 B] P scales
     // per S buffer: [G][4] warp maxima (floats)
     static constexpr int RED_BUF = 4 * G;
     static constexpr int SM_RED = SM_PSF + 2 * 2 * 512;
-    static constexpr int SM_LSC = SM_RED + 2 * RED_BUF * 4;             // [G] floats
-    static constexpr int SM_BARS = (SM_LSC + G * 4 + 7) / 8 * 8;
-    static constexpr int NBARS = 2 * NSK + 2 * NSV + 7;
+    static constexpr int SM_BARS = (SM_RED + 2 * RED_BUF * 4 + 7) / 8 * 8;
+    static constexpr int NBARS = 2 * NSK + 2 * NSV + 8;
     static constexpr int SM_MISC = SM_BARS + NBARS * 8;                  // tmem slot, abort flags
     static constexpr int SMEM = SM_MISC + 16;
     // TMEM column map
@@ -111,13 +116,74 @@ struct TcCfg {
 
 constexpr long long kWaitLimit = 1LL << 32;   // clock cycles (about 2 s)
 
+// Query image of one (sequence, KV head): smoothing + Hadamard transform and
+// dual-residual FP4 of its G query heads, laid out as the decode CTA keeps them
+// in shared memory (QK operand rows: group (r / HG) owns 2 HG consecutive rows,
+// q1 of its heads then q2, so a softmax warp loads both logits of its heads with
+// one TMEM load; element e -> chunk e/32, byte (e%32)/2; then the scale codes
+// [NQ][8] and the logit scales sm_scale g_q g_k log2(e) per head).  Every split of
+// the sequence copies it instead of recomputing it.
+template <int FMT, int G>
+__global__ void __launch_bounds__(TcCfg<FMT, G>::QTHREADS) prep_query_kernel(const DecodeArgs a) {
+    using C = TcCfg<FMT, G>;
+    using RG = RowGeom<FMT, 128>;
+    constexpr int B = C::B, HG = C::HG;
+    // the decode grid may start now; it waits for this grid before copying the image
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    __shared__ __align__(16) uint8_t img[C::QPACK];
+    __shared__ int row_amax[G];
+    uint8_t* q_op = img;
+    uint8_t* qsc = img + C::Q_BYTES;
+    float* lsc = reinterpret_cast<float*>(img + C::Q_BYTES + C::NQ * 8);
+    const int tid = threadIdx.x, hk = blockIdx.x, b = blockIdx.y, h0 = hk * G;
+    const bool hadamard = !(a.flags & BDFP4_FLAG_NO_HADAMARD);
+    const bool dual = !(a.flags & BDFP4_FLAG_SINGLE_QUERY);
+    for (int i = tid; i < C::QPACK / 16; i += blockDim.x) reinterpret_cast<uint4*>(img)[i] = make_uint4(0, 0, 0, 0);
+    if (tid < G) row_amax[tid] = 0;
+    __syncthreads();
+    const int j = tid % RG::rt, r = tid / RG::rt;
+    const bool active = r < G && j < RG::tpr;
+    float x[B];
+    if (active) {
+        load_bf16_block<B>(a.q + ((int64_t)b * a.H_q + h0 + r) * C::DK, j * B, x);
+    } else {
+#pragma unroll
+        for (int i = 0; i < B; ++i) x[i] = 0.0f;
+    }
+    transform_block<FMT, 128, false>(x, a.smooth + (int64_t)hk * C::DK, j, hadamard);
+    if (active) atomicMax(&row_amax[r], __float_as_int(block_amax<B>(x)));
+    __syncthreads();
+    if (active) {
+        const float amax = __int_as_float(row_amax[r]);
+        const float gq = FMT == BDFP4_NVFP4 ? (amax > 0.0f ? __fdiv_rn(amax, 2688.0f) : 1.0f) : 1.0f;
+        uint32_t c1, c2, p1[B / 8], p2[B / 8];
+        quantize_query_block<FMT, 128>(x, gq, dual, c1, p1, c2, p2);
+        const int e0 = j * B;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const int row = (r / HG) * 2 * HG + half * HG + r % HG;
+            const uint32_t* pk = half ? p2 : p1;
+            uint8_t* dst = q_op + (row / 8) * 512 + (e0 / 32) * 128 + (row % 8) * 16 + (e0 % 32) / 2;
+            if constexpr (B == 16) *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
+            else *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            qsc[row * 8 + j] = (uint8_t)(half ? c2 : c1);
+        }
+        if (j == 0) {
+            const float gk = FMT == BDFP4_NVFP4 ? a.k_gscale[hk] : 1.0f;
+            lsc[r] = a.sm_scale * gq * gk * kLog2e;
+        }
+    }
+    __syncthreads();
+    uint4* out = reinterpret_cast<uint4*>(a.qpack + ((int64_t)b * a.H_kv + hk) * C::QPACK);
+    for (int i = tid; i < C::QPACK / 16; i += blockDim.x) out[i] = reinterpret_cast<const uint4*>(img)[i];
+}
+
 template <int FMT, int G>
 __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTAS) decode_tc_kernel(const DecodeArgs a) {
     using C = TcCfg<FMT, G>;
     constexpr bool MX = FMT == BDFP4_MXFP4;
     constexpr int B = C::B;
     constexpr int HG = C::HG;
-    using RG = RowGeom<FMT, 128>;
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t* q_op = smem + C::SM_Q;
     uint8_t* p_op = smem + C::SM_P;
@@ -134,6 +200,7 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
     uint64_t* p_ready = s_full + 2;           // [2] P + scale factors ready -> MMA
     uint64_t* o_full = p_ready + 2;           // [2] PV done -> softmax
     uint64_t* q_ready = o_full + 2;           // query operand and its scale factors -> MMA
+    uint64_t* q_full = q_ready + 1;           // query image landed -> softmax
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SM_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::SM_MISC + 4);   // any role gave up
     volatile int* sm_abort = reinterpret_cast<volatile int*>(smem + C::SM_MISC + 8);     // [NSG] group decisions
@@ -173,6 +240,7 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
             tc::mbar_init(&o_full[i], 1);
         }
         tc::mbar_init(q_ready, C::NSW);
+        tc::mbar_init(q_full, 1);
         *abort_flag = 0;
         sm_abort[0] = 0;
         sm_abort[1] = 0;
@@ -355,58 +423,20 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
         const int gb = grp * HG;                   // first head of the group
         const int bar_id = 1 + grp;                // named barrier of the group (128 threads)
         const uint32_t tq = tbase + ((uint32_t)(32 * qd) << 16);
-        const bool hadamard = !(a.flags & BDFP4_FLAG_NO_HADAMARD);
-        const bool dual = !(a.flags & BDFP4_FLAG_SINGLE_QUERY);
         const float alpha = (FMT == BDFP4_NVFP4 && !(a.flags & BDFP4_FLAG_NO_UNDERFLOW)) ? kAlphaNV : 1.0f;
         bool bad = false;
 
-        // query prologue (all softmax warps): transform + dual-residual FP4 straight into the QK operand
-        int* row_amax = reinterpret_cast<int*>(psf);   // the P scale buffers are free until the first tile
-        for (int i = tid; i < C::Q_BYTES / 16; i += 32 * C::NSW) reinterpret_cast<uint4*>(q_op)[i] = make_uint4(0, 0, 0, 0);
-        for (int i = tid; i < C::NQ * 8; i += 32 * C::NSW) qsc[i] = 0;
-        if (tid < 32) row_amax[tid] = 0;
-        tc::named_bar_sync(1 + C::NSG, 32 * C::NSW);
-        {
-            const int j = tid % RG::rt, r = tid / RG::rt;
-            const bool active = r < G && j < RG::tpr;
-            float x[B];
-            if (active) {
-                load_bf16_block<B>(a.q + ((int64_t)b * a.H_q + h0 + r) * C::DK, j * B, x);
-            } else {
-#pragma unroll
-                for (int i = 0; i < B; ++i) x[i] = 0.0f;
-            }
-            transform_block<FMT, 128, false>(x, a.smooth + (int64_t)hk * C::DK, j, hadamard);
-            if (active) atomicMax(&row_amax[r], __float_as_int(block_amax<B>(x)));
-            tc::named_bar_sync(1 + C::NSG, 32 * C::NSW);
-            if (active) {
-                const float amax = __int_as_float(row_amax[r]);
-                const float gq = FMT == BDFP4_NVFP4 ? (amax > 0.0f ? __fdiv_rn(amax, 2688.0f) : 1.0f) : 1.0f;
-                uint32_t c1, c2, p1[B / 8], p2[B / 8];
-                quantize_query_block<FMT, 128>(x, gq, dual, c1, p1, c2, p2);
-                // rows: group (r / HG) owns 2 HG consecutive rows, q1 of its heads then q2, so a
-                // softmax warp loads both logits of its heads with one TMEM load;
-                // element e -> chunk e/32, byte (e%32)/2
-                const int e0 = j * B;
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    const int row = (r / HG) * 2 * HG + half * HG + r % HG;
-                    const uint32_t* pk = half ? p2 : p1;
-                    uint8_t* dst = q_op + (row / 8) * 512 + (e0 / 32) * 128 + (row % 8) * 16 + (e0 % 32) / 2;
-                    if constexpr (B == 16) *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
-                    else *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                    qsc[row * 8 + j] = (uint8_t)(half ? c2 : c1);
-                }
-                if (j == 0) {
-                    const float gk = FMT == BDFP4_NVFP4 ? a.k_gscale[hk] : 1.0f;
-                    lsc[r] = a.sm_scale * gq * gk * kLog2e;
-                }
-            }
-            tc::fence_proxy_async_smem();
-            tc::named_bar_sync(1 + C::NSG, 32 * C::NSW);
-            // the P scale-factor buffers: zero (rows of absent heads must stay zero)
-            for (int i = tid; i < 2 * 2 * 512 / 16; i += 32 * C::NSW) reinterpret_cast<uint4*>(psf)[i] = make_uint4(0, 0, 0, 0);
+        // the query image (QK operand, scale codes, logit scales) of this (sequence, KV head)
+        // arrives in one bulk copy from prep_query_kernel, which this grid may overlap:
+        // griddepcontrol.wait holds the copy until that grid's writes are visible
+        if (tid == 0) {
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            tc::mbar_arrive_expect_tx(q_full, C::QPACK);
+            tc::bulk_g2s(q_op, a.qpack + ((int64_t)b * a.H_kv + hk) * C::QPACK, C::QPACK, q_full);
         }
+        // the P scale-factor buffers: zero (rows of absent heads must stay zero)
+        for (int i = tid; i < 2 * 2 * 512 / 16; i += 32 * C::NSW) reinterpret_cast<uint4*>(psf)[i] = make_uint4(0, 0, 0, 0);
+        if (!tc::mbar_wait(q_full, 0, abort_flag, kWaitLimit)) bad = true;
         // query scale factors (SFB of QK): lane n <- row n, one 4-column chunk per K step
         if (grp == 0) {
 #pragma unroll
@@ -661,8 +691,26 @@ static int launch_tc(const DecodeArgs& a, cudaStream_t st) {
         }
         attr_set = true;
     }
-    dim3 grid(a.max_splits, a.H_kv, a.B);
-    decode_tc_kernel<FMT, G><<<grid, C::THREADS, C::SMEM_LAUNCH, st>>>(a);
+    prep_query_kernel<FMT, G><<<dim3(a.H_kv, a.B), C::QTHREADS, 0, st>>>(a);
+    const int rc = launch_status();
+    if (rc != BDFP4_OK) return rc;
+    // programmatic dependent launch: the decode CTAs start (TMEM, barriers, K/V
+    // streaming) while the query images are computed
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.max_splits, a.H_kv, a.B);
+    cfg.blockDim = dim3(C::THREADS);
+    cfg.dynamicSmemBytes = C::SMEM_LAUNCH;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<FMT, G>, a);
+    if (e != cudaSuccess) {
+        record_cuda_error(e);
+        return BDFP4_ERR_CUDA;
+    }
     return launch_status();
 }
 

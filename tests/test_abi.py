@@ -58,9 +58,15 @@ def test_decode_plan_host_logic(lib):
 
 
 def test_workspace_size(lib):
-    # B=2, H_q=4, d_v=128, 16 pages = 8 tiles, 2 tiles per split -> 4 splits
+    # B=2, H_q=4, d_v=128, 16 pages = 8 tiles, 2 tiles per split -> 4 splits: fp32 partial
+    # outputs and (m, l) pairs, each padded to 256 B, then 640 B of query image per query head
     o = 2 * 4 * 4 * 128 * 4
-    assert bdfp4.bdfp4_decode_workspace_size(2, 4, 128, 16, 2) == ((o + 255) // 256) * 256 + 2 * 4 * 4 * 2 * 4
+    ml = 2 * 4 * 4 * 2 * 4
+    q = 2 * 4 * 640
+    pad = lambda n: (n + 255) // 256 * 256  # noqa: E731
+    assert bdfp4.bdfp4_decode_workspace_size(2, 4, 128, 16, 2) == pad(o) + pad(ml) + q
+    # one split per sequence: only the query images
+    assert bdfp4.bdfp4_decode_workspace_size(2, 4, 128, 16, 8) == q
     assert bdfp4.bdfp4_decode_workspace_size(0, 4, 128, 16, 2) == 0
 
 
