@@ -326,12 +326,7 @@ extern "C" int bdfp4_decode_plan(const int32_t* host_seq_lens, int B, int H_kv, 
         total_tiles += (int64_t)t * H_kv;
         max_tiles = std::max(max_tiles, t);
     }
-    // about 16 work items per SM keeps the tail short; at least 4 tiles per
-    // split keeps the merge traffic small next to the KV bytes
-    int64_t chunk = (total_tiles + 16LL * num_sms - 1) / (16LL * num_sms);
-    chunk = std::max<int64_t>(chunk, 4);
-    chunk = std::min<int64_t>(chunk, max_tiles);
-    return (int)std::max<int64_t>(chunk, 1);
+    return plan_chunk_tiles(total_tiles, max_tiles, num_sms);
 }
 
 template <int FMT, int DK, int DV>
@@ -388,8 +383,7 @@ extern "C" int bdfp4_decode(const void* q, const void* k_pages, const void* k_sc
             return BDFP4_ERR_CUDA;
         const int ntiles = (max_pages_per_seq * kPageSlots + kTileTokens - 1) / kTileTokens;
         const int64_t total = (int64_t)B * H_kv * ntiles;
-        const int64_t chunk = std::max<int64_t>(4, (total + 16LL * sms - 1) / (16LL * sms));
-        chunk_tiles = (int)std::min<int64_t>(chunk, ntiles);
+        chunk_tiles = plan_chunk_tiles(total, ntiles, sms);
     }
     DecodeArgs a{};
     a.max_splits = max_splits_for(max_pages_per_seq, chunk_tiles);
@@ -470,8 +464,7 @@ extern "C" int bdfp4_decode_noalloc(const void* q, const void* k_pages, const vo
             return BDFP4_ERR_CUDA;
         const int ntiles = (max_pages_per_seq * kPageSlots + kTileTokens - 1) / kTileTokens;
         const int64_t total = (int64_t)B * (H_kv > 0 ? H_kv : 1) * ntiles;
-        const int64_t chunk = std::max<int64_t>(4, (total + 16LL * sms - 1) / (16LL * sms));
-        chunk_tiles = (int)std::min<int64_t>(chunk, ntiles);
+        chunk_tiles = plan_chunk_tiles(total, ntiles, sms);
     }
     if (bdfp4_decode_workspace_size(B, H_q, d_v, max_pages_per_seq, chunk_tiles) > BDFP4_NOALLOC_SCRATCH_BYTES)
         return BDFP4_ERR_WORKSPACE;

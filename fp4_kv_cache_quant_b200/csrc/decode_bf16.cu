@@ -475,8 +475,7 @@ extern "C" int bdfp4_bf16_decode(const void* q, const void* k_pages, const void*
             return BDFP4_ERR_CUDA;
         const int ntiles = (max_pages_per_seq * kPageSlots + kTileTokens - 1) / kTileTokens;
         const int64_t total = (int64_t)B * H_kv * ntiles;
-        const int64_t chunk = std::max<int64_t>(4, (total + 16LL * sms - 1) / (16LL * sms));
-        chunk_tiles = (int)std::min<int64_t>(chunk, ntiles);
+        chunk_tiles = plan_chunk_tiles(total, ntiles, sms);
     }
     Bf16Args a{};
     const int ntiles_max = (max_pages_per_seq * kPageSlots + kTileTokens - 1) / kTileTokens;

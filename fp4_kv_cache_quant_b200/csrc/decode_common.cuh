@@ -38,6 +38,18 @@ __host__ __device__ __forceinline__ int num_splits(int N, int chunk_tiles) {
     return (ntiles + chunk_tiles - 1) / chunk_tiles;
 }
 
+// Tiles per split for total_tiles work tiles (all sequences x KV heads) on
+// num_sms SMs: about 12 CTAs' worth of tiles per SM, kept within [16, 40] tiles
+// (shorter splits repeat per-CTA setup and merge traffic; longer ones leave a
+// ragged tail on variable-length batches), at most the longest sequence.
+inline int plan_chunk_tiles(int64_t total_tiles, int max_tiles, int num_sms) {
+    const int64_t per = 12LL * (num_sms > 0 ? num_sms : 1);
+    int64_t chunk = (total_tiles + per - 1) / per;
+    chunk = chunk < 16 ? 16 : (chunk > 40 ? 40 : chunk);
+    if (chunk > max_tiles) chunk = max_tiles;
+    return chunk < 1 ? 1 : (int)chunk;
+}
+
 // tcgen05 decode for d_k = d_v = 128 (decode_tc.cu); returns a host status.
 int launch_decode_tc(const DecodeArgs& a, int fmt, int G, cudaStream_t st);
 

@@ -152,8 +152,9 @@ BDFP4_API int bdfp4_quantize_q(const void* q, int B, int H_q, int H_kv, int d_k,
                      void* stream);
 
 /*
- * Split plan for bdfp4_decode: tiles (128 tokens) per split so that the
- * (sequence, KV head, split) work items fill num_sms SMs several times over.
+ * Split plan for bdfp4_decode: tiles (128 tokens) per split, about twelve
+ * (sequence, KV head, split) work items per SM, each of 16 to 40 tiles (at most
+ * the longest sequence's tiles).
  * host_seq_lens [B] is a HOST array.  Returns chunk_tiles >= 1, or a negative
  * status.  Sequence b then has ceil(ceil(N_b / 128) / chunk_tiles) splits.
  */

@@ -44,14 +44,17 @@ def test_status_strings(lib):
 
 
 def test_decode_plan_host_logic(lib):
-    # 16 sequences of 32768 tokens, 8 KV heads, 148 SMs: 256 tiles each,
-    # 32768 work tiles -> ceil(32768 / (16 * 148)) = 14 tiles per split
-    assert bdfp4.bdfp4_decode_plan(np.full(16, 32768), 8, 148) == 14
-    # at least 4 tiles per split, at most the longest sequence
-    assert bdfp4.bdfp4_decode_plan(np.array([1000]), 1, 148) == 4
+    # 16 sequences of 32768 tokens, 8 KV heads, 148 SMs: 256 tiles each, 32768
+    # work tiles -> ceil(32768 / (12 * 148)) = 19 tiles per split
+    assert bdfp4.bdfp4_decode_plan(np.full(16, 32768), 8, 148) == 19
+    # at least 16 tiles per split, at most the longest sequence
+    assert bdfp4.bdfp4_decode_plan(np.array([1000]), 1, 148) == 8
+    assert bdfp4.bdfp4_decode_plan(np.array([5000]), 1, 148) == 16
     assert bdfp4.bdfp4_decode_plan(np.array([100]), 1, 148) == 1
-    # 64 sequences of 131072 tokens x 4 heads = 262144 tiles -> 111 per split
-    assert bdfp4.bdfp4_decode_plan(np.full(64, 131072), 4, 148) == 111
+    # 64 sequences of 131072 tokens x 4 heads = 262144 tiles -> 148 per SM-slot, at most 40
+    assert bdfp4.bdfp4_decode_plan(np.full(64, 131072), 4, 148) == 40
+    # 16 x 65536 tokens x 8 heads = 65536 tiles -> ceil(65536 / 1776) = 37
+    assert bdfp4.bdfp4_decode_plan(np.full(16, 65536), 8, 148) == 37
     assert bdfp4.bdfp4_decode_plan(np.array([0, 0]), 2, 148) == 1
     with pytest.raises(bdfp4.BDFP4Error):
         bdfp4.bdfp4_decode_plan(np.array([10]), 0, 148)
