@@ -1,9 +1,10 @@
 """Benchmark of the FP4 paged decode-attention step on B200.
 
 One step = one decode step of a serving batch through the whole hot path:
-append-quantize each sequence's open value block (its newest token and the
-earlier tokens of the same 16/32-slot block, kept in bf16 by the caller) into
-the paged FP4 cache, then decode attention for one query token per sequence
+append-quantize each sequence's newest key and its open value block (the
+newest token and the earlier tokens of the same 16/32-slot block, kept in bf16
+by the caller) into the paged FP4 cache, then decode attention for one query
+token per sequence
 (query transform + dual-residual FP4, paged tile fetch, QK^T, transposed
 softmax with fused underflow-aware P quantization, P.V, split merge).
 
@@ -140,7 +141,7 @@ def setup_ours(sp, fmt, rank, device, with_bf16: bool = False):
     cache = bdfp4.FP4Cache.empty(wl.num_pages, sp.H_kv, sp.d_k, sp.d_v, fmt, device=device)
     status = torch.zeros(1, dtype=torch.int32, device=device)
     bcache = bdfp4.BF16Cache.empty(wl.num_pages, sp.H_kv, sp.d_k, device=device) if with_bf16 else None
-    tails_k, tails_v, tails_sm = [], [], []
+    tails_k, tails_v, tails_sm, new_sm = [], [], [], []
     q_bytes = 0
     t_quant, quant_bytes = 0.0, 0
     for b in range(sp.B):
@@ -160,14 +161,16 @@ def setup_ours(sp, fmt, rank, device, with_bf16: bool = False):
                                                                   sp.d_v // beta)
         # the open value block of the newest token, kept in bf16 for the next append
         r = ((n - 1) % beta) + 1 if n > 0 else 0
-        tails_k.append(k[n - r:].clone())
+        tails_k.append(k[n - 1:].clone())        # the newest token's key
         tails_v.append(v[n - r:].clone())
         tails_sm.append(sm[n - r:].clone())
+        new_sm.append(sm[n - 1:].clone())
         del k, v
     assert int(status.item()) == 0
     tail_k = torch.cat(tails_k)
     tail_v = torch.cat(tails_v)
     tail_sm = torch.cat(tails_sm)
+    new_k, new_sm = tail_k, torch.cat(new_sm)
     q = wl.queries(device)
     bt = torch.from_numpy(wl.block_table).to(device)
     sl = torch.from_numpy(wl.seq_lens).to(device)
@@ -175,7 +178,8 @@ def setup_ours(sp, fmt, rank, device, with_bf16: bool = False):
     chunk = bdfp4.bdfp4_decode_plan(wl.seq_lens, sp.H_kv, num_sms)
     ws = bdfp4.workspace_for(sp.B, sp.H_q, sp.d_v, wl.max_pages, chunk, device=device)
     out = torch.empty((sp.B, sp.H_q, sp.d_v), dtype=torch.bfloat16, device=device)
-    return dict(wl=wl, kv=kv, cache=cache, status=status, tail_k=tail_k, tail_v=tail_v, tail_sm=tail_sm, q=q, bt=bt,
+    return dict(wl=wl, kv=kv, cache=cache, status=status, new_k=new_k, new_sm=new_sm, tail_v=tail_v, tail_sm=tail_sm,
+                q=q, bt=bt,
                 sl=sl, chunk=chunk, ws=ws, out=out, quant_gbs=quant_bytes / t_quant / 1e9, num_sms=num_sms,
                 bcache=bcache)
 
@@ -199,8 +203,13 @@ def run_ours(args, sp, fmt):
     wl, kv, cache = S["wl"], S["kv"], S["cache"]
     stream = torch.cuda.current_stream(device)
 
+    def append():
+        # the newest token's key, and the open value block it joins (kept in bf16 by the caller)
+        bdfp4.bdfp4_quantize_k(S["new_k"], S["new_sm"], kv, cache, dev_status=S["status"])
+        bdfp4.bdfp4_quantize_v(S["tail_v"], S["tail_sm"], kv, cache)
+
     def step(q):
-        bdfp4.bdfp4_quantize_kv(S["tail_k"], S["tail_v"], S["tail_sm"], kv, cache, dev_status=S["status"])
+        append()
         bdfp4.bdfp4_decode(q, cache, S["bt"], S["sl"], kv, sp.sm_scale, S["chunk"], S["ws"], S["out"],
                            dev_status=S["status"])
 
@@ -219,7 +228,7 @@ def run_ours(args, sp, fmt):
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for i in range(args.steps):
-        bdfp4.bdfp4_quantize_kv(S["tail_k"], S["tail_v"], S["tail_sm"], kv, cache, dev_status=S["status"])
+        append()
         ev[i][0].record(stream)
         bdfp4.bdfp4_decode(S["q"], cache, S["bt"], S["sl"], kv, sp.sm_scale, S["chunk"], S["ws"], S["out"],
                            dev_status=S["status"])
@@ -257,7 +266,7 @@ def run_ours(args, sp, fmt):
     # end to end through the C ABI with host buffers: H2D of q and the tail rows,
     # D2H of the output, every step
     q_host = S["q"].cpu().pin_memory()
-    tk_host = S["tail_k"].cpu().pin_memory()
+    tk_host = S["new_k"].cpu().pin_memory()
     tv_host = S["tail_v"].cpu().pin_memory()
     out_host = torch.empty(S["out"].shape, dtype=S["out"].dtype).pin_memory()
     q_dev = torch.empty_like(S["q"])
@@ -269,7 +278,7 @@ def run_ours(args, sp, fmt):
             s1 = torch.cuda.Event(enable_timing=True)
             s0.record(stream)
         q_dev.copy_(q_host, non_blocking=True)
-        S["tail_k"].copy_(tk_host, non_blocking=True)
+        S["new_k"].copy_(tk_host, non_blocking=True)
         S["tail_v"].copy_(tv_host, non_blocking=True)
         step(q_dev)
         out_host.copy_(S["out"], non_blocking=True)
@@ -283,7 +292,8 @@ def run_ours(args, sp, fmt):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         step_s, dec_s, e2e_s, bf16_s = t.tolist()
         tokens *= world
-    launches_per_step = 2 + 1 + (1 if S["chunk"] < (wl.max_pages * 64 + 127) // 128 else 0)
+    # append K and V; query images + tensor-core decode (d = 128) or one CUDA-core decode; merge when split
+    launches_per_step = 2 + (2 if sp.d_k == 128 else 1) + (1 if S["chunk"] < (wl.max_pages * 64 + 127) // 128 else 0)
     alg = algorithmic_bytes(sp, wl.seq_lens, fmt)
     peaks_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(peaks_path):

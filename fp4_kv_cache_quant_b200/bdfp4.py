@@ -28,7 +28,7 @@ PAGE_SLOTS = 64
 TILE_TOKENS = 128
 
 #: names of every entry point declared in include/bdfp4.h
-ENTRY_POINTS = ("bdfp4_calibrate", "bdfp4_quantize_kv", "bdfp4_quantize_q", "bdfp4_decode_plan",
+ENTRY_POINTS = ("bdfp4_calibrate", "bdfp4_quantize_kv", "bdfp4_quantize_k", "bdfp4_quantize_v", "bdfp4_quantize_q", "bdfp4_decode_plan",
                 "bdfp4_decode_workspace_size", "bdfp4_decode", "bdfp4_decode_noalloc", "bdfp4_status_string", "bdfp4_last_error")
 #: names of every entry point declared in include/bdfp4_bf16.h
 BF16_ENTRY_POINTS = ("bdfp4_bf16_append", "bdfp4_bf16_decode")
@@ -62,6 +62,10 @@ def load() -> ctypes.CDLL:
     L.bdfp4_calibrate.restype = i
     L.bdfp4_quantize_kv.argtypes = [p, p, p, i, i, i, i, i, i, kvp, p, p, p, p, i64, p, p]
     L.bdfp4_quantize_kv.restype = i
+    L.bdfp4_quantize_k.argtypes = [p, p, i, i, i, i, i, kvp, p, p, i64, p, p]
+    L.bdfp4_quantize_k.restype = i
+    L.bdfp4_quantize_v.argtypes = [p, p, i, i, i, i, kvp, p, p, i64, p]
+    L.bdfp4_quantize_v.restype = i
     L.bdfp4_quantize_q.argtypes = [p, i, i, i, i, i, i, p, p, p, p, p, p, p]
     L.bdfp4_quantize_q.restype = i
     L.bdfp4_decode_plan.argtypes = [p, i, i, i]
@@ -173,6 +177,23 @@ def bdfp4_quantize_kv(k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tens
                                   _ptr(cache.v_pages), _ptr(cache.v_scales), cache.num_pages, _ptr(dev_status),
                                   _stream(stream))
     _check(rc, "bdfp4_quantize_kv")
+
+
+def bdfp4_quantize_k(k: torch.Tensor, slot_mapping: torch.Tensor, kv: KVParams, cache: FP4Cache, flags: int = 0,
+                     dev_status: torch.Tensor | None = None, stream=None) -> None:
+    c = kv._c()
+    rc = load().bdfp4_quantize_k(_ptr(k), _ptr(slot_mapping), k.shape[0], cache.H_kv, cache.d_k, cache.fmt, flags,
+                                 ctypes.byref(c), _ptr(cache.k_pages), _ptr(cache.k_scales), cache.num_pages,
+                                 _ptr(dev_status), _stream(stream))
+    _check(rc, "bdfp4_quantize_k")
+
+
+def bdfp4_quantize_v(v: torch.Tensor, slot_mapping: torch.Tensor, kv: KVParams, cache: FP4Cache, stream=None) -> None:
+    c = kv._c()
+    rc = load().bdfp4_quantize_v(_ptr(v), _ptr(slot_mapping), v.shape[0], cache.H_kv, cache.d_v, cache.fmt,
+                                 ctypes.byref(c), _ptr(cache.v_pages), _ptr(cache.v_scales), cache.num_pages,
+                                 _stream(stream))
+    _check(rc, "bdfp4_quantize_v")
 
 
 def bdfp4_quantize_q(q: torch.Tensor, H_kv: int, fmt: int, smooth: torch.Tensor, flags: int = 0,

@@ -405,6 +405,61 @@ extern "C" int bdfp4_quantize_kv(const void* k, const void* v, const int64_t* sl
     return launch_status();
 }
 
+// The key half and the value half of bdfp4_quantize_kv on their own token lists.
+extern "C" int bdfp4_quantize_k(const void* k, const int64_t* slot_mapping, int T, int H_kv, int d_k, bdfp4_fmt fmt,
+                                int flags, const bdfp4_kv_params* kv, void* k_pages, void* k_scales,
+                                int64_t num_pages, int32_t* dev_status, void* stream) {
+    if (T < 0 || H_kv <= 0 || num_pages < 0) return BDFP4_ERR_ARG;
+    if (fmt != BDFP4_NVFP4 && fmt != BDFP4_MXFP4) return BDFP4_ERR_ARG;
+    if (d_k != 128 && d_k != 576) return BDFP4_ERR_UNSUPPORTED;
+    if (T == 0) return BDFP4_OK;
+    if (!k || !slot_mapping || !kv || !kv->smooth || !k_pages || !k_scales) return BDFP4_ERR_ARG;
+    if (fmt == BDFP4_NVFP4 && !kv->k_gscale) return BDFP4_ERR_ARG;
+    if (!aligned(k, 16) || !aligned(k_pages, 128) || !aligned(k_scales, 128)) return BDFP4_ERR_ALIGN;
+    cudaStream_t st = (cudaStream_t)stream;
+    const int64_t rows = (int64_t)T * H_kv;
+    auto launch = [&](auto kernel, int R) {
+        kernel<<<(unsigned)((rows + R - 1) / R), 256, 0, st>>>((const __nv_bfloat16*)k, slot_mapping, T, H_kv,
+                                                              kv->smooth, kv->k_gscale, (uint8_t*)k_pages,
+                                                              (uint8_t*)k_scales, num_pages, flags, dev_status);
+    };
+    if (fmt == BDFP4_NVFP4) {
+        if (d_k == 128) launch(quantize_k_kernel<BDFP4_NVFP4, 128>, KGeom<BDFP4_NVFP4, 128>::R);
+        else launch(quantize_k_kernel<BDFP4_NVFP4, 576>, KGeom<BDFP4_NVFP4, 576>::R);
+    } else {
+        if (d_k == 128) launch(quantize_k_kernel<BDFP4_MXFP4, 128>, KGeom<BDFP4_MXFP4, 128>::R);
+        else launch(quantize_k_kernel<BDFP4_MXFP4, 576>, KGeom<BDFP4_MXFP4, 576>::R);
+    }
+    return launch_status();
+}
+
+extern "C" int bdfp4_quantize_v(const void* v, const int64_t* slot_mapping, int T, int H_kv, int d_v, bdfp4_fmt fmt,
+                                const bdfp4_kv_params* kv, void* v_pages, void* v_scales, int64_t num_pages,
+                                void* stream) {
+    if (T < 0 || H_kv <= 0 || num_pages < 0) return BDFP4_ERR_ARG;
+    if (fmt != BDFP4_NVFP4 && fmt != BDFP4_MXFP4) return BDFP4_ERR_ARG;
+    if (d_v != 128 && d_v != 512) return BDFP4_ERR_UNSUPPORTED;
+    if (T == 0) return BDFP4_OK;
+    if (!v || !slot_mapping || !kv || !v_pages || !v_scales) return BDFP4_ERR_ARG;
+    if (fmt == BDFP4_NVFP4 && !kv->v_gscale) return BDFP4_ERR_ARG;
+    if (!aligned(v, 16) || !aligned(v_pages, 128) || !aligned(v_scales, 128)) return BDFP4_ERR_ALIGN;
+    cudaStream_t st = (cudaStream_t)stream;
+    const int64_t rows = (int64_t)T * H_kv;
+    auto launch = [&](auto kernel, int RPC, int CPR) {
+        kernel<<<(unsigned)((rows + RPC - 1) / RPC * CPR), 256, 0, st>>>((const __nv_bfloat16*)v, slot_mapping, T,
+                                                                        H_kv, kv->v_gscale, (uint8_t*)v_pages,
+                                                                        (uint8_t*)v_scales, num_pages);
+    };
+    if (fmt == BDFP4_NVFP4) {
+        if (d_v == 128) launch(quantize_v_kernel<BDFP4_NVFP4, 128>, VGeom<128>::RPC, VGeom<128>::CPR);
+        else launch(quantize_v_kernel<BDFP4_NVFP4, 512>, VGeom<512>::RPC, VGeom<512>::CPR);
+    } else {
+        if (d_v == 128) launch(quantize_v_kernel<BDFP4_MXFP4, 128>, VGeom<128>::RPC, VGeom<128>::CPR);
+        else launch(quantize_v_kernel<BDFP4_MXFP4, 512>, VGeom<512>::RPC, VGeom<512>::CPR);
+    }
+    return launch_status();
+}
+
 template <int FMT, int DK>
 static void launch_quantize_q(const void* q, int rows, int H_q, int G, const float* smooth, int flags, uint8_t* q1c,
                               uint8_t* q1s, uint8_t* q2c, uint8_t* q2s, float* gq, cudaStream_t st) {

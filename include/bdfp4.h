@@ -138,6 +138,22 @@ BDFP4_API int bdfp4_quantize_kv(const void* k, const void* v, const int64_t* slo
                       void* v_pages, void* v_scales, int64_t num_pages, int32_t* dev_status, void* stream);
 
 /*
+ * The two halves of bdfp4_quantize_kv, each on its own token list (same
+ * arguments, layouts, rules and results as the corresponding half there).
+ * A decode step appends the new token's key with bdfp4_quantize_k, and
+ * re-quantizes the open value block (the new token and the earlier tokens of
+ * its beta-slot block, kept in bf16 by the caller) with bdfp4_quantize_v: a
+ * key is quantized per token, so stored keys never need touching again.
+ * bdfp4_quantize_v reports nothing through a status word (bad slots are
+ * skipped; bdfp4_quantize_k reports them).
+ */
+BDFP4_API int bdfp4_quantize_k(const void* k, const int64_t* slot_mapping, int T, int H_kv, int d_k, bdfp4_fmt fmt,
+                    int flags, const bdfp4_kv_params* kv, void* k_pages, void* k_scales, int64_t num_pages,
+                    int32_t* dev_status, void* stream);
+BDFP4_API int bdfp4_quantize_v(const void* v, const int64_t* slot_mapping, int T, int H_kv, int d_v, bdfp4_fmt fmt,
+                    const bdfp4_kv_params* kv, void* v_pages, void* v_scales, int64_t num_pages, void* stream);
+
+/*
  * Dual-Residual Query Quantization on its own (Article Summary; the French
  * page: the second FP4 tensor encodes the residual of the first), exactly as
  * the decode prologue performs it.  q [B][H_q][d_k] bf16.  Query transform:

@@ -61,6 +61,39 @@ def test_quantize_kv_bit_exact(ora, lib, name, flags):
     assert_bytes_equal(cache_to_np(gcache), ocache)
 
 
+@pytest.mark.parametrize("name", ["tiny_nv", "tiny_mx", "ragged_g8_nv", "ragged_g8_mx", "mla_nv"])
+def test_decode_step_append_matches_oracle(ora, lib, name):
+    """Prefill all but the newest token with bdfp4_quantize_kv, then append the newest
+    token's key with bdfp4_quantize_k and its open value block with bdfp4_quantize_v:
+    the cache must equal the oracle's quantization of every token at once."""
+    sp, fmt = SMALL[name]
+    wl = Workload(sp, seed=7)
+    smooth, kg, vg = oracle_calibration(ora, wl)
+    ocache = ora.empty_cache(wl.num_pages, sp.H_kv, sp.d_k, sp.d_v, fmt)
+    ora.quantize_kv(wl.all_keys(), wl.all_values(), wl.slot_mapping_all(), ocache, sp.H_kv, fmt, smooth, kg, vg,
+                    wl.num_pages)
+    kvp = kv_params_gpu(smooth, kg, vg)
+    gcache = bdfp4.FP4Cache.empty(wl.num_pages, sp.H_kv, sp.d_k, sp.d_v, fmt)
+    for name_ in ("k_pages", "k_scales", "v_pages", "v_scales"):
+        getattr(gcache, name_).zero_()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    beta = 16 if fmt == NV else 32
+    for b in range(sp.B):
+        n = int(wl.seq_lens[b])
+        if n == 0:
+            continue
+        k, v = wl.keys(b).cuda(), wl.values(b).cuda()
+        sm = torch.from_numpy(wl.slot_mapping(b)).cuda()
+        if n > 1:
+            bdfp4.bdfp4_quantize_kv(k[:n - 1], v[:n - 1], sm[:n - 1], kvp, gcache, dev_status=status)
+        bdfp4.bdfp4_quantize_k(k[n - 1:], sm[n - 1:], kvp, gcache, dev_status=status)
+        r = (n - 1) % beta + 1   # the open block: the newest token and the earlier ones of its block
+        bdfp4.bdfp4_quantize_v(v[n - r:], sm[n - r:], kvp, gcache)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert_bytes_equal(cache_to_np(gcache), ocache)
+
+
 @pytest.mark.parametrize("fmt", [NV, MX])
 def test_quantize_kv_adversarial_values(ora, lib, fmt):
     """Exact E2M1 midpoints (ties), zero blocks, tiny and huge values, runs
