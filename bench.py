@@ -1,12 +1,12 @@
 """Benchmark of the FP4 paged decode-attention step on B200.
 
-One step = one decode step of a serving batch through the whole hot path:
-append-quantize each sequence's newest key and its open value block (the
-newest token and the earlier tokens of the same 16/32-slot block, kept in bf16
-by the caller) into the paged FP4 cache, then decode attention for one query
-token per sequence
-(query transform + dual-residual FP4, paged tile fetch, QK^T, transposed
-softmax with fused underflow-aware P quantization, P.V, split merge).
+One step = one decode step of a serving batch through the whole hot path, in
+one bdfp4_decode_step call: append-quantize each sequence's newest key and its
+open value block (the newest token and the earlier tokens of the same
+16/32-slot block, kept in bf16 on the device) into the paged FP4 cache, then
+decode attention for one query token per sequence (query transform +
+dual-residual FP4, paged tile fetch, QK^T, transposed softmax with fused
+underflow-aware P quantization, P.V, split merge).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config qwen3_4b]
                   [--fmt nvfp4|mxfp4] [--impl ours|reference]
@@ -57,7 +57,8 @@ def algorithmic_bytes(sp, seq_lens, fmt: int) -> int:
     return tok * per_tok + pages * 4 + sp.B * sp.H_q * (sp.d_k + sp.d_v) * 2
 
 
-DECODE_SOURCES = ("decode_tc.cu", "tc_ptx.cuh", "bdfp4_device.cuh", "quant_device.cuh", "decode_common.cuh")
+DECODE_SOURCES = ("decode_tc.cu", "tc_ptx.cuh", "bdfp4_device.cuh", "quant_device.cuh", "decode_common.cuh",
+                  "append_device.cuh")
 
 
 def decode_source_hash() -> str:
@@ -141,7 +142,10 @@ def setup_ours(sp, fmt, rank, device, with_bf16: bool = False):
     cache = bdfp4.FP4Cache.empty(wl.num_pages, sp.H_kv, sp.d_k, sp.d_v, fmt, device=device)
     status = torch.zeros(1, dtype=torch.int32, device=device)
     bcache = bdfp4.BF16Cache.empty(wl.num_pages, sp.H_kv, sp.d_k, device=device) if with_bf16 else None
-    tails_k, tails_v, tails_sm, new_sm = [], [], [], []
+    # decode-step inputs: the newest token of each sequence and the open value block it joins
+    new_k = torch.zeros((sp.B, sp.H_kv, sp.d_k), dtype=torch.bfloat16, device=device)
+    new_v = torch.zeros((sp.B, sp.H_kv, sp.d_v), dtype=torch.bfloat16, device=device)
+    v_open = torch.zeros((sp.B, beta, sp.H_kv, sp.d_v), dtype=torch.bfloat16, device=device)
     q_bytes = 0
     t_quant, quant_bytes = 0.0, 0
     for b in range(sp.B):
@@ -159,18 +163,13 @@ def setup_ours(sp, fmt, rank, device, with_bf16: bool = False):
         t_quant += e0.elapsed_time(e1) / 1e3
         quant_bytes += (k.numel() + v.numel()) * 2 + n * sp.H_kv * (sp.d_k // 2 + sp.d_k // beta + sp.d_v // 2 +
                                                                   sp.d_v // beta)
-        # the open value block of the newest token, kept in bf16 for the next append
-        r = ((n - 1) % beta) + 1 if n > 0 else 0
-        tails_k.append(k[n - 1:].clone())        # the newest token's key
-        tails_v.append(v[n - r:].clone())
-        tails_sm.append(sm[n - r:].clone())
-        new_sm.append(sm[n - 1:].clone())
+        if n > 0:
+            last = (n - 1) % beta   # row of the newest token in its open value block
+            new_k[b] = k[n - 1]
+            new_v[b] = v[n - 1]
+            v_open[b, :last] = v[n - 1 - last:n - 1]
         del k, v
     assert int(status.item()) == 0
-    tail_k = torch.cat(tails_k)
-    tail_v = torch.cat(tails_v)
-    tail_sm = torch.cat(tails_sm)
-    new_k, new_sm = tail_k, torch.cat(new_sm)
     q = wl.queries(device)
     bt = torch.from_numpy(wl.block_table).to(device)
     sl = torch.from_numpy(wl.seq_lens).to(device)
@@ -178,8 +177,7 @@ def setup_ours(sp, fmt, rank, device, with_bf16: bool = False):
     chunk = bdfp4.bdfp4_decode_plan(wl.seq_lens, sp.H_kv, num_sms)
     ws = bdfp4.workspace_for(sp.B, sp.H_q, sp.d_v, wl.max_pages, chunk, device=device)
     out = torch.empty((sp.B, sp.H_q, sp.d_v), dtype=torch.bfloat16, device=device)
-    return dict(wl=wl, kv=kv, cache=cache, status=status, new_k=new_k, new_sm=new_sm, tail_v=tail_v, tail_sm=tail_sm,
-                q=q, bt=bt,
+    return dict(wl=wl, kv=kv, cache=cache, status=status, new_k=new_k, new_v=new_v, v_open=v_open, q=q, bt=bt,
                 sl=sl, chunk=chunk, ws=ws, out=out, quant_gbs=quant_bytes / t_quant / 1e9, num_sms=num_sms,
                 bcache=bcache)
 
@@ -203,22 +201,20 @@ def run_ours(args, sp, fmt):
     wl, kv, cache = S["wl"], S["kv"], S["cache"]
     stream = torch.cuda.current_stream(device)
 
-    def append():
-        # the newest token's key, and the open value block it joins (kept in bf16 by the caller)
-        bdfp4.bdfp4_quantize_k(S["new_k"], S["new_sm"], kv, cache, dev_status=S["status"])
-        bdfp4.bdfp4_quantize_v(S["tail_v"], S["tail_sm"], kv, cache)
+    def step(q, k_new, v_new):
+        # one call: append each sequence's newest token (key, and the open value
+        # block it joins) into the FP4 cache, then decode over the updated cache
+        bdfp4.bdfp4_decode_step(q, k_new, v_new, S["v_open"], cache, S["bt"], S["sl"], kv, sp.sm_scale, S["chunk"],
+                                S["ws"], S["out"], dev_status=S["status"])
 
-    def step(q):
-        append()
-        bdfp4.bdfp4_decode(q, cache, S["bt"], S["sl"], kv, sp.sm_scale, S["chunk"], S["ws"], S["out"],
+    def decode_only():
+        bdfp4.bdfp4_decode(S["q"], cache, S["bt"], S["sl"], kv, sp.sm_scale, S["chunk"], S["ws"], S["out"],
                            dev_status=S["status"])
 
     for _ in range(max(args.warmup, 3)):
-        step(S["q"])
+        step(S["q"], S["new_k"], S["new_v"])
     torch.cuda.synchronize()
 
-    # per-launch decode timing (events on the launching stream) inside the timed region
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     clocks = ClockSampler(local)
     if world > 1:
         dist.barrier()
@@ -228,12 +224,16 @@ def run_ours(args, sp, fmt):
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for i in range(args.steps):
-        append()
-        ev[i][0].record(stream)
-        bdfp4.bdfp4_decode(S["q"], cache, S["bt"], S["sl"], kv, sp.sm_scale, S["chunk"], S["ws"], S["out"],
-                           dev_status=S["status"])
-        ev[i][1].record(stream)
+        step(S["q"], S["new_k"], S["new_v"])
     t1.record(stream)
+    torch.cuda.synchronize()
+    # the decode on its own (query images, decode kernel, merge), per call, for the roofline:
+    # the same number of calls on the same stream right after the steps, still under the clock sampler
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        decode_only()
+        ev[i][1].record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
     if world > 1:
@@ -263,13 +263,15 @@ def run_ours(args, sp, fmt):
         bf16_s = statistics.mean(a.elapsed_time(b) for a, b in bev) / 1e3
         assert int(S["status"].item()) == 0, "device status set"
 
-    # end to end through the C ABI with host buffers: H2D of q and the tail rows,
-    # D2H of the output, every step
+    # end to end through the C ABI with host buffers: H2D of q and the new keys and
+    # values, D2H of the output, every step
     q_host = S["q"].cpu().pin_memory()
     tk_host = S["new_k"].cpu().pin_memory()
-    tv_host = S["tail_v"].cpu().pin_memory()
+    tv_host = S["new_v"].cpu().pin_memory()
     out_host = torch.empty(S["out"].shape, dtype=S["out"].dtype).pin_memory()
     q_dev = torch.empty_like(S["q"])
+    k_dev = torch.empty_like(S["new_k"])
+    v_dev = torch.empty_like(S["new_v"])
     e2e_steps = max(3, args.steps // 2)
     for it in range(2 + e2e_steps):
         if it == 2:
@@ -278,9 +280,9 @@ def run_ours(args, sp, fmt):
             s1 = torch.cuda.Event(enable_timing=True)
             s0.record(stream)
         q_dev.copy_(q_host, non_blocking=True)
-        S["new_k"].copy_(tk_host, non_blocking=True)
-        S["tail_v"].copy_(tv_host, non_blocking=True)
-        step(q_dev)
+        k_dev.copy_(tk_host, non_blocking=True)
+        v_dev.copy_(tv_host, non_blocking=True)
+        step(q_dev, k_dev, v_dev)
         out_host.copy_(S["out"], non_blocking=True)
     s1.record(stream)
     torch.cuda.synchronize()
@@ -292,8 +294,9 @@ def run_ours(args, sp, fmt):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         step_s, dec_s, e2e_s, bf16_s = t.tolist()
         tokens *= world
-    # append K and V; query images + tensor-core decode (d = 128) or one CUDA-core decode; merge when split
-    launches_per_step = 2 + (2 if sp.d_k == 128 else 1) + (1 if S["chunk"] < (wl.max_pages * 64 + 127) // 128 else 0)
+    # one prologue (append + query images) and the tensor-core decode (d = 128), or the
+    # append and one CUDA-core decode; merge when a sequence can split
+    launches_per_step = 2 + (1 if S["chunk"] < (wl.max_pages * 64 + 127) // 128 else 0)
     alg = algorithmic_bytes(sp, wl.seq_lens, fmt)
     peaks_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(peaks_path):
@@ -331,7 +334,9 @@ def run_ours(args, sp, fmt):
         "quantize_prefill_gbs": S["quant_gbs"],
         "roofline": {"bound": "hbm", "achieved": alg / dec_s / 1e9, "peak": peak, "unit": "GB/s",
                      "frac": alg / dec_s / 1e9 / peak, "traffic": traffic,
-                     "kernel": "decode_fp4_kernel + merge_splits_kernel (events bracket both)",
+                     "kernel": ("bdfp4_decode calls (query images, decode_tc_kernel, merge_splits_kernel), "
+                                "events around each of K calls right after the step loop"
+                                if sp.d_k == 128 else "bdfp4_decode calls (decode_fp4_kernel, merge_splits_kernel)"),
                      "peak_source": f"{peak_src} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
                      "algorithmic_bytes_per_launch": alg},
         "e2e": {"value": tokens / e2e_s, "unit": "tokens/s",

@@ -29,7 +29,8 @@ TILE_TOKENS = 128
 
 #: names of every entry point declared in include/bdfp4.h
 ENTRY_POINTS = ("bdfp4_calibrate", "bdfp4_quantize_kv", "bdfp4_quantize_k", "bdfp4_quantize_v", "bdfp4_quantize_q", "bdfp4_decode_plan",
-                "bdfp4_decode_workspace_size", "bdfp4_decode", "bdfp4_decode_noalloc", "bdfp4_status_string", "bdfp4_last_error")
+                "bdfp4_decode_workspace_size", "bdfp4_decode", "bdfp4_decode_step", "bdfp4_decode_noalloc",
+                "bdfp4_status_string", "bdfp4_last_error")
 #: names of every entry point declared in include/bdfp4_bf16.h
 BF16_ENTRY_POINTS = ("bdfp4_bf16_append", "bdfp4_bf16_decode")
 
@@ -74,6 +75,9 @@ def load() -> ctypes.CDLL:
     L.bdfp4_decode_workspace_size.restype = sz
     L.bdfp4_decode.argtypes = [p, p, p, p, p, p, p, i, i, i, i, i, i, i64, i, i, kvp, f, i, p, sz, p, p, p]
     L.bdfp4_decode.restype = i
+    L.bdfp4_decode_step.argtypes = [p, p, p, p, p, p, p, p, p, p, i, i, i, i, i, i, i64, i, i, kvp, f, i, p, sz, p, p,
+                                    p]
+    L.bdfp4_decode_step.restype = i
     L.bdfp4_decode_noalloc.argtypes = [p, p, p, p, p, p, p, i, i, i, i, i, i, i64, i, i, kvp, f, i, p, p, p]
     L.bdfp4_decode_noalloc.restype = i
     L.bdfp4_status_string.argtypes = [i]
@@ -238,6 +242,26 @@ def bdfp4_decode(q: torch.Tensor, cache: FP4Cache, block_table: torch.Tensor, se
                              float(sm_scale), int(chunk_tiles), _ptr(workspace), ws_bytes, _ptr(out),
                              _ptr(dev_status), _stream(stream))
     _check(rc, "bdfp4_decode")
+    return out
+
+
+def bdfp4_decode_step(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, v_open: torch.Tensor,
+                      cache: FP4Cache, block_table: torch.Tensor, seq_lens: torch.Tensor, kv: KVParams,
+                      sm_scale: float, chunk_tiles: int, workspace: torch.Tensor | None, out: torch.Tensor,
+                      flags: int = 0, dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Append each sequence's new token (k_new, v_new [B, H_kv, d]) at position
+    seq_lens[b] - 1, keeping the open value block in v_open [B, beta, H_kv, d_v],
+    then decode q over the updated cache (bdfp4_decode_step in bdfp4.h)."""
+    B, H_q, d_k = q.shape
+    c = kv._c()
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = load().bdfp4_decode_step(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(v_open), _ptr(cache.k_pages),
+                                  _ptr(cache.k_scales), _ptr(cache.v_pages), _ptr(cache.v_scales), _ptr(block_table),
+                                  _ptr(seq_lens), B, H_q, cache.H_kv, d_k, cache.d_v, block_table.shape[1],
+                                  cache.num_pages, cache.fmt, flags, ctypes.byref(c), float(sm_scale),
+                                  int(chunk_tiles), _ptr(workspace), ws_bytes, _ptr(out), _ptr(dev_status),
+                                  _stream(stream))
+    _check(rc, "bdfp4_decode_step")
     return out
 
 

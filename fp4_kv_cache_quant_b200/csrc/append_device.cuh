@@ -1,0 +1,247 @@
+// append_device.cuh -- the KV-append quantizers as CTA-level device functions
+// (BitDecoding-FP4, Article Summary: Outlier-Aware Key Quantization; values
+// take the plain block rule), shared by the stand-alone append kernels and the
+// fused decode-step prologue.  Each function does the work of one CTA of 256
+// threads, given its block index inside its own role.
+#pragma once
+
+#include "bdfp4_device.cuh"
+#include "quant_device.cuh"
+
+namespace bdfp4 {
+
+// ---------------------------------------------------------------- keys
+// Work split of the K append: every scale block of a row gets NC lanes, one per
+// candidate code of its search window (10 for NVFP4, 2 for MXFP4, padded), so
+// the window is searched in parallel; R rows share a 256-thread CTA.
+template <int FMT, int DK>
+struct KGeom {
+    using RG = RowGeom<FMT, DK>;
+    static constexpr int B = RG::beta;
+    static constexpr int NB = DK / B;                                  // scale blocks per row
+    static constexpr int NC = FMT == BDFP4_NVFP4 ? 16 : 2;             // candidate lanes per block
+    static constexpr int R = 256 / (NB * NC) >= 1 ? 256 / (NB * NC) : 1;
+    static constexpr int PAIRS = R * NB * NC;                           // (block, candidate) pairs
+    static constexpr int PAIRS_PAD = (PAIRS + 255) / 256 * 256;
+    static constexpr int T1 = (R * RG::rt + 31) / 32 * 32;             // transform threads (whole warps)
+    static_assert(T1 <= 256, "transform threads exceed the CTA");
+};
+
+// Slot of token t from a slot mapping (page * 64 + slot, negative = skip);
+// slots past the cache are reported and skipped.
+struct MappedSlot {
+    const int64_t* slot_mapping;
+    int64_t num_pages;
+    int32_t* dev_status;
+    __device__ __forceinline__ int64_t operator()(int t, bool report) const {
+        const int64_t sm = __ldg(slot_mapping + t);
+        if (sm >= num_pages * kPageSlots) {
+            if (report) set_status(dev_status, BDFP4_DEV_BAD_SLOT);
+            return -1;
+        }
+        return sm;
+    }
+};
+
+// Slot of the newest token of sequence t in a decode step: position N - 1 of
+// the sequence (N = seq_lens[t] counts the new token), through its block table
+// row.  Empty or over-long sequences append nothing (the decode reports the
+// latter); a page id outside the cache is reported and skipped.
+struct NewestSlot {
+    const int32_t* block_table;
+    const int32_t* seq_lens;
+    int max_pages;
+    int64_t num_pages;
+    int32_t* dev_status;
+    __device__ __forceinline__ int64_t operator()(int t, bool report) const {
+        const int N = __ldg(seq_lens + t);
+        if (N <= 0 || N > max_pages * kPageSlots) return -1;
+        const int pg = __ldg(block_table + (int64_t)t * max_pages + (N - 1) / kPageSlots);
+        if (pg < 0 || pg >= num_pages) {
+            if (report) set_status(dev_status, BDFP4_DEV_BAD_PAGE);
+            return -1;
+        }
+        return (int64_t)pg * kPageSlots + (N - 1) % kPageSlots;
+    }
+};
+
+// Key rows [blk * R, blk * R + R) of k [rows / H_kv][H_kv][DK] (row = token *
+// H_kv + head).  Phase 1 transforms the rows into shared memory (thread per
+// block, butterflies across the row's threads); phase 2 quantizes every block
+// under every code of its window and keeps the fp64 squared errors (each
+// summed left to right); phase 3 scans each window from its largest code down,
+// keeping the first least error, and stores the winner.  The choice is the
+// sequential search's.
+template <int FMT, int DK, class SlotOf>
+__device__ __forceinline__ void append_k_cta(int blk, const __nv_bfloat16* __restrict__ k, int64_t rows, int H_kv,
+                                             const SlotOf& slot_of, const float* __restrict__ smooth,
+                                             const float* __restrict__ k_gscale, uint8_t* k_pages,
+                                             uint8_t* k_scales, int flags) {
+    using KG = KGeom<FMT, DK>;
+    using RG = typename KG::RG;
+    constexpr int B = KG::B, NB = KG::NB, NC = KG::NC, R = KG::R;
+    __shared__ float xs[R][DK];
+    __shared__ double errs[KG::PAIRS_PAD];
+    __shared__ uint32_t pks[KG::PAIRS_PAD][B / 8];
+    __shared__ int win[R * NB];            // hi << 16 | lo
+    __shared__ long long slots[R];
+    __shared__ float gs[R];                // tensor scale of the row's head
+    const int tid = threadIdx.x;
+    const int64_t row0 = (int64_t)blk * R;
+
+    if (tid < KG::T1) {
+        const int r = tid / RG::rt, j = tid % RG::rt;
+        const int64_t row = row0 + r;
+        const bool in_range = r < R && row < rows;
+        const int t = (int)(in_range ? row / H_kv : 0);
+        const int h = (int)(in_range ? row % H_kv : 0);
+        const int64_t sm = in_range ? slot_of(t, j == 0) : -1;
+        // whole warps stay converged through the shuffles; inactive rows compute on zeros
+        // the row is loaded whatever its slot id, so the two loads overlap
+        float x[B];
+        if (in_range && j < RG::tpr) {
+            load_bf16_block<B>(k + ((int64_t)t * H_kv + h) * DK, j * B, x);
+        } else {
+#pragma unroll
+            for (int i = 0; i < B; ++i) x[i] = 0.0f;
+        }
+        if (sm < 0) {
+#pragma unroll
+            for (int i = 0; i < B; ++i) x[i] = 0.0f;
+        }
+        const bool active = sm >= 0 && j < RG::tpr;
+        transform_block<FMT, DK, true>(x, smooth + (int64_t)h * DK, j, !(flags & BDFP4_FLAG_NO_HADAMARD));
+        if (active) {
+#pragma unroll
+            for (int i = 0; i < B; ++i) xs[r][j * B + i] = x[i];
+        }
+        if (r < R && j == 0) {
+            slots[r] = sm;
+            gs[r] = FMT == BDFP4_NVFP4 ? __ldg(k_gscale + h) : 1.0f;
+        }
+    }
+    __syncthreads();
+
+    for (int p = tid; p < KG::PAIRS; p += 256) {
+        const int r = p / (NB * NC), bk = (p / NC) % NB, ci = p % NC;
+        if (slots[r] < 0) continue;
+        const float g = gs[r];
+        float x[B];
+#pragma unroll
+        for (int i = 0; i < B; ++i) x[i] = xs[r][bk * B + i];
+        const float amax = block_amax<B>(x);
+        const int c0 = (int)plain_scale_code<FMT>(amax, g);
+        int hi = c0, lo = c0;   // all-zero blocks and the plain rule keep c0
+        if (amax != 0.0f && !(flags & BDFP4_FLAG_NO_SCALE_SEARCH)) {
+            const int top = FMT == BDFP4_NVFP4 ? 126 : 254;
+            hi = min(c0 + (FMT == BDFP4_NVFP4 ? 7 : 1), top);
+            lo = max(c0 - (FMT == BDFP4_NVFP4 ? 2 : 0), 0);
+        }
+        if (ci == 0) win[r * NB + bk] = (hi << 16) | lo;
+        const int c = hi - ci;
+        if (c >= lo) errs[p] = quantize_block<B>(x, block_sigma<FMT>((uint32_t)c, g), pks[p]);
+    }
+    __syncthreads();
+
+    for (int q = tid; q < R * NB; q += 256) {
+        const int r = q / NB, bk = q % NB;
+        const int64_t sm = slots[r];
+        if (sm < 0) continue;
+        const int h = (int)((row0 + r) % H_kv);
+        const int hi = win[q] >> 16, lo = win[q] & 0xffff;
+        const int base = q * NC;
+        int best = 0;
+        double best_err = errs[base];
+        for (int ci = 1; ci <= hi - lo; ++ci) {
+            if (errs[base + ci] < best_err) {
+                best = ci;
+                best_err = errs[base + ci];
+            }
+        }
+        const int64_t page = sm / kPageSlots;
+        const int slot = (int)(sm % kPageSlots);
+        uint8_t* kp = k_pages + (page * H_kv + h) * (int64_t)(kPageSlots * DK / 2);
+        uint8_t* dst = kp + k_nib_offset(DK, slot, bk * B);
+        const uint32_t* pk = pks[base + best];
+        if constexpr (B == 16) {
+            *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
+        } else {
+            *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+        uint8_t* ks = k_scales + (page * H_kv + h) * (int64_t)k_scale_page_bytes(DK, B);
+        ks[k_scale_offset<B>(DK, slot, bk)] = (uint8_t)(hi - best);
+    }
+}
+
+// ---------------------------------------------------------------- values
+// One thread per (row, channel): TPR threads of a row per CTA, RPC rows per
+// CTA, CPR CTAs per row.
+template <int DV>
+struct VGeom {
+    static constexpr int TPR = DV < 256 ? DV : 256;   // threads of a row in one CTA
+    static constexpr int RPC = 256 / TPR;             // rows per CTA
+    static constexpr int CPR = DV / TPR;              // CTAs per row
+};
+
+// Decode-step value append for rows (sequence b, head h) = blk's rows of the
+// [B][H_kv] grid.  v_open [B][beta][H_kv][DV] bf16 holds each sequence's open
+// beta-token block (row i = slot first + i of the block that holds position
+// N - 1): the new value v_new [B][H_kv][DV] goes into row (N - 1) % beta, and
+// the block is quantized from rows 0 .. (N - 1) % beta (later slots of the
+// block become zero), exactly as the append of that run of tokens.
+template <int FMT, int DV>
+__device__ __forceinline__ void append_v_open_cta(int blk, const __nv_bfloat16* __restrict__ v_new,
+                                                  __nv_bfloat16* v_open, const NewestSlot& slot_of, int nseq,
+                                                  int H_kv, const float* __restrict__ v_gscale, uint8_t* v_pages,
+                                                  uint8_t* v_scales) {
+    constexpr int B = Fmt<FMT>::beta;
+    using VG = VGeom<DV>;
+    const int64_t row = (int64_t)(blk / VG::CPR) * VG::RPC + threadIdx.x / VG::TPR;
+    const int c = (int)(blk % VG::CPR) * VG::TPR + threadIdx.x % VG::TPR;
+    if (row >= (int64_t)nseq * H_kv) return;
+    const int b = (int)(row / H_kv), h = (int)(row % H_kv);
+    // the whole open block and the new value are loaded with the slot lookup in flight
+    const unsigned short* ob = reinterpret_cast<const unsigned short*>(v_open);
+    const unsigned short vn = __ldg(reinterpret_cast<const unsigned short*>(v_new) + row * DV + c);
+    uint32_t raw[B];
+#pragma unroll
+    for (int i = 0; i < B; ++i) raw[i] = ob[(((int64_t)b * B + i) * H_kv + h) * DV + c];
+    const int64_t sm = slot_of(b, false);
+    if (sm < 0) return;
+    const int slot = (int)(sm % kPageSlots);
+    const int last = slot % B;   // row of the new value in the open block
+    const int first = slot - last;
+    reinterpret_cast<unsigned short*>(v_open)[(((int64_t)b * B + last) * H_kv + h) * DV + c] = vn;
+    float x[B];
+#pragma unroll
+    for (int i = 0; i < B; ++i) {
+        const uint32_t w = i == last ? (uint32_t)vn : raw[i];
+        x[i] = i <= last ? __uint_as_float(w << 16) : 0.0f;
+    }
+    const float g = FMT == BDFP4_NVFP4 ? __ldg(v_gscale + h) : 1.0f;
+    const uint32_t code = plain_scale_code<FMT>(block_amax<B>(x), g);
+    uint32_t packed[B / 8];
+    quantize_block<B>(x, block_sigma<FMT>(code, g), packed);
+    const int64_t page = sm / kPageSlots;
+    uint8_t* vp = v_pages + (page * H_kv + h) * (int64_t)(DV * kPageSlots / 2);
+    uint8_t* vs = v_scales + (page * H_kv + h) * (int64_t)(DV * kPageSlots / B);
+    uint8_t* dst = vp + v_nib_offset(c, first);
+    if constexpr (B == 16) {
+        *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+    } else {
+        *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    }
+    vs[v_scale_offset<B>(c, first / B)] = (uint8_t)code;
+}
+
+// CTAs of each append role for nrows (token, head) rows.
+template <int FMT, int DK>
+__host__ __device__ constexpr int64_t k_append_ctas(int64_t nrows) {
+    return (nrows + KGeom<FMT, DK>::R - 1) / KGeom<FMT, DK>::R;
+}
+template <int DV>
+__host__ __device__ constexpr int64_t v_append_ctas(int64_t nrows) {
+    return (nrows + VGeom<DV>::RPC - 1) / VGeom<DV>::RPC * VGeom<DV>::CPR;
+}
+
+}  // namespace bdfp4

@@ -330,15 +330,19 @@ extern "C" int bdfp4_decode_plan(const int32_t* host_seq_lens, int B, int H_kv, 
 }
 
 template <int FMT, int DK, int DV>
-static int launch_decode(const DecodeArgs& a, int G, cudaStream_t st) {
+static int launch_decode(const DecodeArgs& a, int G, cudaStream_t st, const StepArgs* step) {
     if (DK == 128 && G <= 16) {
-        // tensor-core path (decode_tc.cu)
-        const int rc = launch_decode_tc(a, FMT, G, st);
+        // tensor-core path (decode_tc.cu); a step's append runs in its prologue grid
+        const int rc = launch_decode_tc(a, FMT, G, st, step);
         if (rc != BDFP4_OK) return rc;
         if (a.max_splits > 1)
             merge_splits_kernel<DV><<<a.B * a.H_q, 128, merge_smem(a.max_splits), st>>>(
                 a.ws_o, a.ws_ml, a.seq_lens, a.H_q, a.max_pages, a.chunk_tiles, a.max_splits, a.out);
         return launch_status();
+    }
+    if (step) {
+        const int rc = launch_step_append(a, *step, FMT, DK, st);
+        if (rc != BDFP4_OK) return rc;
     }
     int hg = G >= 16 ? 16 : G;
     dim3 grid(a.max_splits, a.H_kv * (G / hg), a.B);
@@ -356,11 +360,11 @@ static int launch_decode(const DecodeArgs& a, int G, cudaStream_t st) {
     return launch_status();
 }
 
-extern "C" int bdfp4_decode(const void* q, const void* k_pages, const void* k_scales, const void* v_pages,
-                            const void* v_scales, const int32_t* block_table, const int32_t* seq_lens, int B, int H_q,
-                            int H_kv, int d_k, int d_v, int max_pages_per_seq, int64_t num_pages, bdfp4_fmt fmt,
-                            int flags, const bdfp4_kv_params* kv, float sm_scale, int chunk_tiles, void* workspace,
-                            size_t workspace_bytes, void* out, int32_t* dev_status, void* stream) {
+static int run_decode(const void* q, const void* k_pages, const void* k_scales, const void* v_pages,
+                      const void* v_scales, const int32_t* block_table, const int32_t* seq_lens, int B, int H_q,
+                      int H_kv, int d_k, int d_v, int max_pages_per_seq, int64_t num_pages, bdfp4_fmt fmt, int flags,
+                      const bdfp4_kv_params* kv, float sm_scale, int chunk_tiles, void* workspace,
+                      size_t workspace_bytes, void* out, int32_t* dev_status, void* stream, StepArgs* step) {
     if (B < 0 || H_q <= 0 || H_kv <= 0 || max_pages_per_seq <= 0 || num_pages < 0) return BDFP4_ERR_ARG;
     if (fmt != BDFP4_NVFP4 && fmt != BDFP4_MXFP4) return BDFP4_ERR_ARG;
     if (H_q % H_kv) return BDFP4_ERR_SHAPE;
@@ -416,10 +420,46 @@ extern "C" int bdfp4_decode(const void* q, const void* k_pages, const void* k_sc
     a.flags = flags;
     a.chunk_tiles = chunk_tiles;
     a.sm_scale = sm_scale;
+    a.append_wait = step != nullptr;
+    if (step) {
+        step->k_pages = (uint8_t*)k_pages;
+        step->k_scales = (uint8_t*)k_scales;
+        step->v_pages = (uint8_t*)v_pages;
+        step->v_scales = (uint8_t*)v_scales;
+    }
     cudaStream_t st = (cudaStream_t)stream;
     if (fmt == BDFP4_NVFP4)
-        return d_k == 128 ? launch_decode<BDFP4_NVFP4, 128, 128>(a, G, st) : launch_decode<BDFP4_NVFP4, 576, 512>(a, G, st);
-    return d_k == 128 ? launch_decode<BDFP4_MXFP4, 128, 128>(a, G, st) : launch_decode<BDFP4_MXFP4, 576, 512>(a, G, st);
+        return d_k == 128 ? launch_decode<BDFP4_NVFP4, 128, 128>(a, G, st, step)
+                          : launch_decode<BDFP4_NVFP4, 576, 512>(a, G, st, step);
+    return d_k == 128 ? launch_decode<BDFP4_MXFP4, 128, 128>(a, G, st, step)
+                      : launch_decode<BDFP4_MXFP4, 576, 512>(a, G, st, step);
+}
+
+extern "C" int bdfp4_decode(const void* q, const void* k_pages, const void* k_scales, const void* v_pages,
+                            const void* v_scales, const int32_t* block_table, const int32_t* seq_lens, int B, int H_q,
+                            int H_kv, int d_k, int d_v, int max_pages_per_seq, int64_t num_pages, bdfp4_fmt fmt,
+                            int flags, const bdfp4_kv_params* kv, float sm_scale, int chunk_tiles, void* workspace,
+                            size_t workspace_bytes, void* out, int32_t* dev_status, void* stream) {
+    return run_decode(q, k_pages, k_scales, v_pages, v_scales, block_table, seq_lens, B, H_q, H_kv, d_k, d_v,
+                      max_pages_per_seq, num_pages, fmt, flags, kv, sm_scale, chunk_tiles, workspace,
+                      workspace_bytes, out, dev_status, stream, nullptr);
+}
+
+extern "C" int bdfp4_decode_step(const void* q, const void* k_new, const void* v_new, void* v_open, void* k_pages,
+                                 void* k_scales, void* v_pages, void* v_scales, const int32_t* block_table,
+                                 const int32_t* seq_lens, int B, int H_q, int H_kv, int d_k, int d_v,
+                                 int max_pages_per_seq, int64_t num_pages, bdfp4_fmt fmt, int flags,
+                                 const bdfp4_kv_params* kv, float sm_scale, int chunk_tiles, void* workspace,
+                                 size_t workspace_bytes, void* out, int32_t* dev_status, void* stream) {
+    if (B > 0 && (!k_new || !v_new || !v_open)) return BDFP4_ERR_ARG;
+    if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(v_open, 16)) return BDFP4_ERR_ALIGN;
+    StepArgs s{};
+    s.k_new = (const __nv_bfloat16*)k_new;
+    s.v_new = (const __nv_bfloat16*)v_new;
+    s.v_open = (__nv_bfloat16*)v_open;
+    return run_decode(q, k_pages, k_scales, v_pages, v_scales, block_table, seq_lens, B, H_q, H_kv, d_k, d_v,
+                      max_pages_per_seq, num_pages, fmt, flags, kv, sm_scale, chunk_tiles, workspace,
+                      workspace_bytes, out, dev_status, stream, &s);
 }
 
 // ---------------------------------------------------------------- no-allocation variant

@@ -25,8 +25,22 @@ struct DecodeArgs {
     __nv_bfloat16* out;
     int32_t* dev_status;
     int B, H_q, H_kv, max_pages, flags, chunk_tiles, max_splits;
+    int append_wait;   // 1: a decode-step prologue grid writes each sequence's last page (tensor-core path)
     int64_t num_pages;
     float sm_scale;
+};
+
+// The new token of each sequence in a decode step: its key and value, and the
+// bf16 values of each sequence's open beta-token value block, all appended
+// into the cache (through these writable views of it) before the decode.
+struct StepArgs {
+    const __nv_bfloat16* k_new;   // [B][H_kv][d_k]
+    const __nv_bfloat16* v_new;   // [B][H_kv][d_v]
+    __nv_bfloat16* v_open;        // [B][beta][H_kv][d_v]
+    uint8_t* k_pages;
+    uint8_t* k_scales;
+    uint8_t* v_pages;
+    uint8_t* v_scales;
 };
 
 constexpr int kThreads = 128;
@@ -51,6 +65,11 @@ inline int plan_chunk_tiles(int64_t total_tiles, int max_tiles, int num_sms) {
 }
 
 // tcgen05 decode for d_k = d_v = 128 (decode_tc.cu); returns a host status.
-int launch_decode_tc(const DecodeArgs& a, int fmt, int G, cudaStream_t st);
+// With a step, one prologue grid appends the new tokens and builds the query
+// images, and the decode overlaps it (programmatic dependent launch).
+int launch_decode_tc(const DecodeArgs& a, int fmt, int G, cudaStream_t st, const StepArgs* step = nullptr);
+
+// Decode-step append on its own (quantize.cu), for the CUDA-core decode path.
+int launch_step_append(const DecodeArgs& a, const StepArgs& s, int fmt, int d_k, cudaStream_t st);
 
 }  // namespace bdfp4

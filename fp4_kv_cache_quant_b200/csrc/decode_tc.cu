@@ -21,6 +21,7 @@
 //               each tile's O into registers with the online-softmax rescale.
 // Every wait is bounded; a timeout sets BDFP4_DEV_TIMEOUT and the CTA unwinds.
 
+#include "append_device.cuh"
 #include "bdfp4_device.cuh"
 #include "decode_common.cuh"
 #include "host_common.h"
@@ -123,19 +124,18 @@ constexpr long long kWaitLimit = 1LL << 32;   // clock cycles (about 2 s)
 // one TMEM load; element e -> chunk e/32, byte (e%32)/2; then the scale codes
 // [NQ][8] and the logit scales sm_scale g_q g_k log2(e) per head).  Every split of
 // the sequence copies it instead of recomputing it.
+// One CTA (at least QTHREADS threads) builds the image of (sequence b, KV head hk).
 template <int FMT, int G>
-__global__ void __launch_bounds__(TcCfg<FMT, G>::QTHREADS) prep_query_kernel(const DecodeArgs a) {
+__device__ __forceinline__ void query_image_cta(const DecodeArgs& a, int hk, int b) {
     using C = TcCfg<FMT, G>;
     using RG = RowGeom<FMT, 128>;
     constexpr int B = C::B, HG = C::HG;
-    // the decode grid may start now; it waits for this grid before copying the image
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     __shared__ __align__(16) uint8_t img[C::QPACK];
     __shared__ int row_amax[G];
     uint8_t* q_op = img;
     uint8_t* qsc = img + C::Q_BYTES;
     float* lsc = reinterpret_cast<float*>(img + C::Q_BYTES + C::NQ * 8);
-    const int tid = threadIdx.x, hk = blockIdx.x, b = blockIdx.y, h0 = hk * G;
+    const int tid = threadIdx.x, h0 = hk * G;
     const bool hadamard = !(a.flags & BDFP4_FLAG_NO_HADAMARD);
     const bool dual = !(a.flags & BDFP4_FLAG_SINGLE_QUERY);
     for (int i = tid; i < C::QPACK / 16; i += blockDim.x) reinterpret_cast<uint4*>(img)[i] = make_uint4(0, 0, 0, 0);
@@ -176,6 +176,35 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::QTHREADS) prep_query_kernel(con
     __syncthreads();
     uint4* out = reinterpret_cast<uint4*>(a.qpack + ((int64_t)b * a.H_kv + hk) * C::QPACK);
     for (int i = tid; i < C::QPACK / 16; i += blockDim.x) out[i] = reinterpret_cast<const uint4*>(img)[i];
+}
+
+template <int FMT, int G>
+__global__ void __launch_bounds__(TcCfg<FMT, G>::QTHREADS) prep_query_kernel(const DecodeArgs a) {
+    // the decode grid may start now; it waits for this grid before copying the image
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    query_image_cta<FMT, G>(a, blockIdx.x, blockIdx.y);
+}
+
+// Decode-step prologue: one grid whose CTAs take three roles side by side --
+// the key append of every sequence's new token, the value append of its open
+// block, and the query images -- so a step costs one launch ahead of the
+// decode.  The decode grid starts as soon as every CTA here has started.
+template <int FMT, int G>
+__global__ void __launch_bounds__(256) prep_step_kernel(const DecodeArgs a, const StepArgs s) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int64_t rows = (int64_t)a.B * a.H_kv;
+    const NewestSlot slot{a.block_table, a.seq_lens, a.max_pages, a.num_pages, a.dev_status};
+    const int nk = (int)k_append_ctas<FMT, 128>(rows), nv = (int)v_append_ctas<128>(rows);
+    const int blk = blockIdx.x;
+    if (blk < nk) {
+        append_k_cta<FMT, 128>(blk, s.k_new, rows, a.H_kv, slot, a.smooth, a.k_gscale, s.k_pages, s.k_scales, a.flags);
+    } else if (blk < nk + nv) {
+        append_v_open_cta<FMT, 128>(blk - nk, s.v_new, s.v_open, slot, a.B, a.H_kv, a.v_gscale, s.v_pages,
+                                    s.v_scales);
+    } else {
+        const int qi = blk - nk - nv;
+        query_image_cta<FMT, G>(a, qi % a.H_kv, qi / a.H_kv);
+    }
 }
 
 template <int FMT, int G>
@@ -292,6 +321,9 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                 // slots lane and 32 + lane of each page and scale group into row lane of the
                 // group's tcgen05.cp source, then arrives on the stage barrier once they land
                 if (do_k) {
+                    // the step prologue writes the new token into the sequence's last page:
+                    // that tile's copies wait until the prologue grid has finished
+                    if (a.append_wait && tile0 + k == ntiles - 1) asm volatile("griddepcontrol.wait;" ::: "memory");
                     if (lane == 0) {
                         if (k >= C::NSK && !tc::mbar_wait(&kempty[ks], ((k / C::NSK) - 1) & 1, abort_flag, kWaitLimit))
                             ok = false;
@@ -679,7 +711,7 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
 }
 
 template <int FMT, int G>
-static int launch_tc(const DecodeArgs& a, cudaStream_t st) {
+static int launch_tc(const DecodeArgs& a, cudaStream_t st, const StepArgs* step) {
     using C = TcCfg<FMT, G>;
     static bool attr_set = false;
     if (!attr_set) {
@@ -691,7 +723,13 @@ static int launch_tc(const DecodeArgs& a, cudaStream_t st) {
         }
         attr_set = true;
     }
-    prep_query_kernel<FMT, G><<<dim3(a.H_kv, a.B), C::QTHREADS, 0, st>>>(a);
+    if (step) {
+        const int64_t rows = (int64_t)a.B * a.H_kv;
+        const int64_t ctas = k_append_ctas<FMT, 128>(rows) + v_append_ctas<128>(rows) + rows;
+        prep_step_kernel<FMT, G><<<(unsigned)ctas, 256, 0, st>>>(a, *step);
+    } else {
+        prep_query_kernel<FMT, G><<<dim3(a.H_kv, a.B), C::QTHREADS, 0, st>>>(a);
+    }
     const int rc = launch_status();
     if (rc != BDFP4_OK) return rc;
     // programmatic dependent launch: the decode CTAs start (TMEM, barriers, K/V
@@ -714,22 +752,22 @@ static int launch_tc(const DecodeArgs& a, cudaStream_t st) {
     return launch_status();
 }
 
-int launch_decode_tc(const DecodeArgs& a, int fmt, int G, cudaStream_t st) {
+int launch_decode_tc(const DecodeArgs& a, int fmt, int G, cudaStream_t st, const StepArgs* step) {
     if (fmt == BDFP4_NVFP4) {
         switch (G) {
-            case 1: return launch_tc<BDFP4_NVFP4, 1>(a, st);
-            case 2: return launch_tc<BDFP4_NVFP4, 2>(a, st);
-            case 4: return launch_tc<BDFP4_NVFP4, 4>(a, st);
-            case 8: return launch_tc<BDFP4_NVFP4, 8>(a, st);
-            case 16: return launch_tc<BDFP4_NVFP4, 16>(a, st);
+            case 1: return launch_tc<BDFP4_NVFP4, 1>(a, st, step);
+            case 2: return launch_tc<BDFP4_NVFP4, 2>(a, st, step);
+            case 4: return launch_tc<BDFP4_NVFP4, 4>(a, st, step);
+            case 8: return launch_tc<BDFP4_NVFP4, 8>(a, st, step);
+            case 16: return launch_tc<BDFP4_NVFP4, 16>(a, st, step);
         }
     } else {
         switch (G) {
-            case 1: return launch_tc<BDFP4_MXFP4, 1>(a, st);
-            case 2: return launch_tc<BDFP4_MXFP4, 2>(a, st);
-            case 4: return launch_tc<BDFP4_MXFP4, 4>(a, st);
-            case 8: return launch_tc<BDFP4_MXFP4, 8>(a, st);
-            case 16: return launch_tc<BDFP4_MXFP4, 16>(a, st);
+            case 1: return launch_tc<BDFP4_MXFP4, 1>(a, st, step);
+            case 2: return launch_tc<BDFP4_MXFP4, 2>(a, st, step);
+            case 4: return launch_tc<BDFP4_MXFP4, 4>(a, st, step);
+            case 8: return launch_tc<BDFP4_MXFP4, 8>(a, st, step);
+            case 16: return launch_tc<BDFP4_MXFP4, 16>(a, st, step);
         }
     }
     return BDFP4_ERR_UNSUPPORTED;

@@ -13,31 +13,12 @@
 #include "bdfp4_device.cuh"
 #include "host_common.h"
 #include "quant_device.cuh"
+#include "append_device.cuh"
+#include "decode_common.cuh"
 
 namespace bdfp4 {
 
-// ---------------------------------------------------------------- K append
-// Work split of the K append: every scale block of a row gets NC lanes, one per
-// candidate code of its search window (10 for NVFP4, 2 for MXFP4, padded), so
-// the window is searched in parallel; R rows share a 256-thread CTA.
-template <int FMT, int DK>
-struct KGeom {
-    using RG = RowGeom<FMT, DK>;
-    static constexpr int B = RG::beta;
-    static constexpr int NB = DK / B;                                  // scale blocks per row
-    static constexpr int NC = FMT == BDFP4_NVFP4 ? 16 : 2;             // candidate lanes per block
-    static constexpr int R = 256 / (NB * NC) >= 1 ? 256 / (NB * NC) : 1;
-    static constexpr int PAIRS = R * NB * NC;                           // (block, candidate) pairs
-    static constexpr int PAIRS_PAD = (PAIRS + 255) / 256 * 256;
-    static constexpr int T1 = (R * RG::rt + 31) / 32 * 32;             // transform threads (whole warps)
-    static_assert(T1 <= 256, "transform threads exceed the CTA");
-};
-
-// Phase 1 transforms R rows into shared memory (thread per block, butterflies
-// across the row's threads); phase 2 quantizes every block under every code of
-// its window and keeps the fp64 squared errors (each summed left to right);
-// phase 3 scans each window from its largest code down, keeping the first
-// least error, and stores the winner.  The choice is the sequential search's.
+// ---------------------------------------------------------------- KV append
 template <int FMT, int DK>
 __global__ void __launch_bounds__(256) quantize_k_kernel(const __nv_bfloat16* __restrict__ k,
                                                          const int64_t* __restrict__ slot_mapping, int T, int H_kv,
@@ -45,118 +26,13 @@ __global__ void __launch_bounds__(256) quantize_k_kernel(const __nv_bfloat16* __
                                                          const float* __restrict__ k_gscale, uint8_t* k_pages,
                                                          uint8_t* k_scales, int64_t num_pages, int flags,
                                                          int32_t* dev_status) {
-    using KG = KGeom<FMT, DK>;
-    using RG = typename KG::RG;
-    constexpr int B = KG::B, NB = KG::NB, NC = KG::NC, R = KG::R;
-    __shared__ float xs[R][DK];
-    __shared__ double errs[KG::PAIRS_PAD];
-    __shared__ uint32_t pks[KG::PAIRS_PAD][B / 8];
-    __shared__ int win[R * NB];            // hi << 16 | lo
-    __shared__ long long slots[R];
-    __shared__ float gs[R];                // tensor scale of the row's head
-    const int tid = threadIdx.x;
-    const int64_t rows = (int64_t)T * H_kv;
-    const int64_t row0 = (int64_t)blockIdx.x * R;
-
-    if (tid < KG::T1) {
-        const int r = tid / RG::rt, j = tid % RG::rt;
-        const int64_t row = row0 + r;
-        const bool in_range = r < R && row < rows;
-        const int t = (int)(in_range ? row / H_kv : 0);
-        const int h = (int)(in_range ? row % H_kv : 0);
-        int64_t sm = in_range ? __ldg(slot_mapping + t) : -1;
-        if (sm >= num_pages * kPageSlots) {
-            if (j == 0) set_status(dev_status, BDFP4_DEV_BAD_SLOT);
-            sm = -1;
-        }
-        // whole warps stay converged through the shuffles; inactive rows compute on zeros
-        // the row is loaded whatever its slot id, so the two loads overlap
-        float x[B];
-        if (in_range && j < RG::tpr) {
-            load_bf16_block<B>(k + ((int64_t)t * H_kv + h) * DK, j * B, x);
-        } else {
-#pragma unroll
-            for (int i = 0; i < B; ++i) x[i] = 0.0f;
-        }
-        if (sm < 0) {
-#pragma unroll
-            for (int i = 0; i < B; ++i) x[i] = 0.0f;
-        }
-        const bool active = sm >= 0 && j < RG::tpr;
-        transform_block<FMT, DK, true>(x, smooth + (int64_t)h * DK, j, !(flags & BDFP4_FLAG_NO_HADAMARD));
-        if (active) {
-#pragma unroll
-            for (int i = 0; i < B; ++i) xs[r][j * B + i] = x[i];
-        }
-        if (r < R && j == 0) {
-            slots[r] = sm;
-            gs[r] = FMT == BDFP4_NVFP4 ? __ldg(k_gscale + h) : 1.0f;
-        }
-    }
-    __syncthreads();
-
-    for (int p = tid; p < KG::PAIRS; p += 256) {
-        const int r = p / (NB * NC), bk = (p / NC) % NB, ci = p % NC;
-        if (slots[r] < 0) continue;
-        const float g = gs[r];
-        float x[B];
-#pragma unroll
-        for (int i = 0; i < B; ++i) x[i] = xs[r][bk * B + i];
-        const float amax = block_amax<B>(x);
-        const int c0 = (int)plain_scale_code<FMT>(amax, g);
-        int hi = c0, lo = c0;   // all-zero blocks and the plain rule keep c0
-        if (amax != 0.0f && !(flags & BDFP4_FLAG_NO_SCALE_SEARCH)) {
-            const int top = FMT == BDFP4_NVFP4 ? 126 : 254;
-            hi = min(c0 + (FMT == BDFP4_NVFP4 ? 7 : 1), top);
-            lo = max(c0 - (FMT == BDFP4_NVFP4 ? 2 : 0), 0);
-        }
-        if (ci == 0) win[r * NB + bk] = (hi << 16) | lo;
-        const int c = hi - ci;
-        if (c >= lo) errs[p] = quantize_block<B>(x, block_sigma<FMT>((uint32_t)c, g), pks[p]);
-    }
-    __syncthreads();
-
-    for (int q = tid; q < R * NB; q += 256) {
-        const int r = q / NB, bk = q % NB;
-        const int64_t sm = slots[r];
-        if (sm < 0) continue;
-        const int h = (int)((row0 + r) % H_kv);
-        const int hi = win[q] >> 16, lo = win[q] & 0xffff;
-        const int base = q * NC;
-        int best = 0;
-        double best_err = errs[base];
-        for (int ci = 1; ci <= hi - lo; ++ci) {
-            if (errs[base + ci] < best_err) {
-                best = ci;
-                best_err = errs[base + ci];
-            }
-        }
-        const int64_t page = sm / kPageSlots;
-        const int slot = (int)(sm % kPageSlots);
-        uint8_t* kp = k_pages + (page * H_kv + h) * (int64_t)(kPageSlots * DK / 2);
-        uint8_t* dst = kp + k_nib_offset(DK, slot, bk * B);
-        const uint32_t* pk = pks[base + best];
-        if constexpr (B == 16) {
-            *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
-        } else {
-            *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        }
-        uint8_t* ks = k_scales + (page * H_kv + h) * (int64_t)k_scale_page_bytes(DK, B);
-        ks[k_scale_offset<B>(DK, slot, bk)] = (uint8_t)(hi - best);
-    }
+    append_k_cta<FMT, DK>(blockIdx.x, k, (int64_t)T * H_kv, H_kv, MappedSlot{slot_mapping, num_pages, dev_status},
+                          smooth, k_gscale, k_pages, k_scales, flags);
 }
 
-// ---------------------------------------------------------------- V append
 // One thread per (token, head, channel); only the first token of each run
 // within a beta-slot block does work (see bdfp4_quantize_kv in bdfp4.h), for
 // the whole block of its channel.
-template <int DV>
-struct VGeom {
-    static constexpr int TPR = DV < 256 ? DV : 256;   // threads of a row in one CTA
-    static constexpr int RPC = 256 / TPR;             // rows per CTA
-    static constexpr int CPR = DV / TPR;              // CTAs per row
-};
-
 template <int FMT, int DV>
 __global__ void __launch_bounds__(256) quantize_v_kernel(const __nv_bfloat16* __restrict__ v,
                                                          const int64_t* __restrict__ slot_mapping, int T, int H_kv,
@@ -216,6 +92,37 @@ __global__ void __launch_bounds__(256) quantize_v_kernel(const __nv_bfloat16* __
         *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
     }
     vs[v_scale_offset<B>(c, first / B)] = (uint8_t)code;
+}
+
+// Decode-step append: key CTAs first, then value CTAs, one (sequence, KV
+// head) row per new token.
+template <int FMT, int DK, int DV>
+__global__ void __launch_bounds__(256) step_append_kernel(const DecodeArgs a, const StepArgs s) {
+    const int64_t rows = (int64_t)a.B * a.H_kv;
+    const NewestSlot slot{a.block_table, a.seq_lens, a.max_pages, a.num_pages, a.dev_status};
+    const int nk = (int)k_append_ctas<FMT, DK>(rows);
+    if ((int)blockIdx.x < nk)
+        append_k_cta<FMT, DK>(blockIdx.x, s.k_new, rows, a.H_kv, slot, a.smooth, a.k_gscale, s.k_pages, s.k_scales,
+                              a.flags);
+    else
+        append_v_open_cta<FMT, DV>(blockIdx.x - nk, s.v_new, s.v_open, slot, a.B, a.H_kv, a.v_gscale, s.v_pages,
+                                   s.v_scales);
+}
+
+template <int FMT, int DK, int DV>
+static int launch_step_append_t(const DecodeArgs& a, const StepArgs& s, cudaStream_t st) {
+    const int64_t rows = (int64_t)a.B * a.H_kv;
+    const int64_t ctas = k_append_ctas<FMT, DK>(rows) + v_append_ctas<DV>(rows);
+    step_append_kernel<FMT, DK, DV><<<(unsigned)ctas, 256, 0, st>>>(a, s);
+    return launch_status();
+}
+
+int launch_step_append(const DecodeArgs& a, const StepArgs& s, int fmt, int d_k, cudaStream_t st) {
+    if (fmt == BDFP4_NVFP4)
+        return d_k == 128 ? launch_step_append_t<BDFP4_NVFP4, 128, 128>(a, s, st)
+                          : launch_step_append_t<BDFP4_NVFP4, 576, 512>(a, s, st);
+    return d_k == 128 ? launch_step_append_t<BDFP4_MXFP4, 128, 128>(a, s, st)
+                      : launch_step_append_t<BDFP4_MXFP4, 576, 512>(a, s, st);
 }
 
 template <int FMT, int DK>

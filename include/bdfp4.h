@@ -207,6 +207,34 @@ BDFP4_API int bdfp4_decode(const void* q, const void* k_pages, const void* k_sca
                  size_t workspace_bytes, void* out, int32_t* dev_status, void* stream);
 
 /*
+ * One decode step in one call: append each sequence's new token to the FP4
+ * cache, then decode (the paper's generation loop -- the KV-append
+ * quantization of the Article Summary's kernel followed by its decode
+ * attention).  seq_lens[b] = N_b counts the new token, which goes to position
+ * N_b - 1, i.e. slot (N_b - 1) % 64 of page block_table[b][(N_b - 1) / 64].
+ *   k_new [B][H_kv][d_k], v_new [B][H_kv][d_v] bf16: the new keys and values.
+ *   v_open [B][beta][H_kv][d_v] bf16, caller-owned and kept across steps: the
+ *     open value block of each sequence, row i = slot (N_b - 1) - (N_b - 1) %
+ *     beta + i.  The call writes v_new into row (N_b - 1) % beta and re-
+ *     quantizes the block from rows 0 .. (N_b - 1) % beta (the rows before it
+ *     must hold the block's earlier tokens: written by earlier steps, or by
+ *     the caller after a prefill); the block's later slots become zero.
+ * The cache bytes after the call equal those of bdfp4_quantize_k on the new
+ * keys plus bdfp4_quantize_v on each open block's run of tokens; the output
+ * is bdfp4_decode's over the updated cache.  Sequences with N_b = 0 append
+ * nothing.  Other arguments, the workspace and the status bits are those of
+ * bdfp4_decode (k_new and v_new 16-byte aligned).  On the d_k = 128 path the
+ * append and the query images run in one prologue grid that the decode
+ * overlaps; only each sequence's last tile waits for it.
+ */
+BDFP4_API int bdfp4_decode_step(const void* q, const void* k_new, const void* v_new, void* v_open, void* k_pages,
+                                void* k_scales, void* v_pages, void* v_scales, const int32_t* block_table,
+                                const int32_t* seq_lens, int B, int H_q, int H_kv, int d_k, int d_v,
+                                int max_pages_per_seq, int64_t num_pages, bdfp4_fmt fmt, int flags,
+                                const bdfp4_kv_params* kv, float sm_scale, int chunk_tiles, void* workspace,
+                                size_t workspace_bytes, void* out, int32_t* dev_status, void* stream);
+
+/*
  * bdfp4_decode without a caller-provided workspace.  The paper has no
  * counterpart: this entry point exists for callers that cannot allocate
  * device memory themselves -- for example an operator plugged into a host

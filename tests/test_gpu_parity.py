@@ -94,6 +94,70 @@ def test_decode_step_append_matches_oracle(ora, lib, name):
     assert_bytes_equal(cache_to_np(gcache), ocache)
 
 
+@pytest.mark.parametrize("chunk", [0, 1])
+@pytest.mark.parametrize("name", ["tiny_nv", "tiny_mx", "ragged_g8_nv", "ragged_g8_mx", "g16_nv", "mla_nv", "mla_mx"])
+def test_decode_step_matches_oracle(ora, lib, name, chunk):
+    """bdfp4_decode_step after a prefill of all but each sequence's newest token:
+    the cache must equal the oracle's quantization of every token, the open
+    value block must hold the new value, and the output must match the oracle's
+    decode (and equal bdfp4_decode on the updated cache bit for bit).  Rows of
+    the open block past the new token hold large noise the step must ignore."""
+    sp, fmt = SMALL[name]
+    wl = Workload(sp, seed=8)
+    smooth, kg, vg = oracle_calibration(ora, wl)
+    ocache = ora.empty_cache(wl.num_pages, sp.H_kv, sp.d_k, sp.d_v, fmt)
+    ora.quantize_kv(wl.all_keys(), wl.all_values(), wl.slot_mapping_all(), ocache, sp.H_kv, fmt, smooth, kg, vg,
+                    wl.num_pages)
+    kvp = kv_params_gpu(smooth, kg, vg)
+    gcache = bdfp4.FP4Cache.empty(wl.num_pages, sp.H_kv, sp.d_k, sp.d_v, fmt)
+    for name_ in ("k_pages", "k_scales", "v_pages", "v_scales"):
+        getattr(gcache, name_).zero_()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    beta = 16 if fmt == NV else 32
+    gen = torch.Generator().manual_seed(9)
+    k_new = torch.randn((sp.B, sp.H_kv, sp.d_k), generator=gen).to(torch.bfloat16)
+    v_new = torch.randn((sp.B, sp.H_kv, sp.d_v), generator=gen).to(torch.bfloat16)
+    v_open = (1e4 * torch.randn((sp.B, beta, sp.H_kv, sp.d_v), generator=gen)).to(torch.bfloat16)
+    lasts = []
+    for b in range(sp.B):
+        n = int(wl.seq_lens[b])
+        lasts.append((n - 1) % beta if n > 0 else -1)
+        if n == 0:
+            continue
+        k, v = wl.keys(b), wl.values(b)
+        if n > 1:
+            sm = torch.from_numpy(wl.slot_mapping(b)).cuda()
+            bdfp4.bdfp4_quantize_kv(k[:n - 1].cuda(), v[:n - 1].cuda(), sm[:n - 1], kvp, gcache, dev_status=status)
+        last = lasts[-1]
+        k_new[b] = k[n - 1]
+        v_new[b] = v[n - 1]
+        v_open[b, :last] = v[n - 1 - last:n - 1]
+    q = wl.queries()
+    if chunk <= 0:
+        chunk = bdfp4.bdfp4_decode_plan(wl.seq_lens, sp.H_kv, torch.cuda.get_device_properties(0).multi_processor_count)
+    sl = torch.from_numpy(wl.seq_lens).cuda()
+    bt = torch.from_numpy(wl.block_table).cuda()
+    out = torch.empty((sp.B, sp.H_q, sp.d_v), dtype=torch.bfloat16, device="cuda")
+    ws = bdfp4.workspace_for(sp.B, sp.H_q, sp.d_v, bt.shape[1], chunk)
+    v_open_g = v_open.cuda()
+    bdfp4.bdfp4_decode_step(q.cuda(), k_new.cuda(), v_new.cuda(), v_open_g, gcache, bt, sl, kvp, sp.sm_scale, chunk,
+                            ws, out, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert_bytes_equal(cache_to_np(gcache), ocache)
+    vo = v_open_g.cpu()
+    for b, last in enumerate(lasts):
+        if last >= 0:
+            assert torch.equal(vo[b, last], v_new[b])
+    ref16, _ = ora.decode(q, ocache, wl.block_table, wl.seq_lens, sp.H_kv, sp.d_v, fmt, smooth, kg, vg, sp.sm_scale,
+                          chunk, wl.num_pages)
+    got = out_to_np(out)
+    max_abs, rel = compare_outputs(got, bf16_to_np(ref16))
+    assert max_abs <= MAX_ABS and rel <= REL_L2, (max_abs, rel)
+    again, st2 = run_gpu_decode(wl, gcache, q, kvp, chunk)
+    assert st2 == 0 and torch.equal(again, out)
+
+
 @pytest.mark.parametrize("fmt", [NV, MX])
 def test_quantize_kv_adversarial_values(ora, lib, fmt):
     """Exact E2M1 midpoints (ties), zero blocks, tiny and huge values, runs
