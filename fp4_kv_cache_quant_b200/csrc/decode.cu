@@ -294,8 +294,8 @@ static int max_splits_for(int max_pages, int chunk_tiles) {
 
 // Workspace regions: split partials (fp32 O, then (m, l)) when a sequence can
 // have more than one split, then the query images of the tensor-core path
-// (at most kQueryImageBytes per query head).
-constexpr size_t kQueryImageBytes = 640;
+// (at most kQueryImageBytes per query head: 640 at d_k = 128, 652 for MLA).
+constexpr size_t kQueryImageBytes = 656;
 
 struct WorkspaceMap {
     size_t o_bytes, ml_bytes, q_off, total;
@@ -334,6 +334,15 @@ static int launch_decode(const DecodeArgs& a, int G, cudaStream_t st, const Step
     if (DK == 128 && G <= 16) {
         // tensor-core path (decode_tc.cu); a step's append runs in its prologue grid
         const int rc = launch_decode_tc(a, FMT, G, st, step);
+        if (rc != BDFP4_OK) return rc;
+        if (a.max_splits > 1)
+            merge_splits_kernel<DV><<<a.B * a.H_q, 128, merge_smem(a.max_splits), st>>>(
+                a.ws_o, a.ws_ml, a.seq_lens, a.H_q, a.max_pages, a.chunk_tiles, a.max_splits, a.out);
+        return launch_status();
+    }
+    if (DK == 576 && mla_tc_supported(DK, DV, G)) {
+        // tensor-core path for MLA shapes (decode_mla_tc.cu); a step's append runs in its prologue grid
+        const int rc = launch_decode_mla_tc(a, FMT, G, st, step);
         if (rc != BDFP4_OK) return rc;
         if (a.max_splits > 1)
             merge_splits_kernel<DV><<<a.B * a.H_q, 128, merge_smem(a.max_splits), st>>>(
@@ -391,7 +400,7 @@ static int run_decode(const void* q, const void* k_pages, const void* k_scales, 
     }
     DecodeArgs a{};
     a.max_splits = max_splits_for(max_pages_per_seq, chunk_tiles);
-    const bool tensor_core_path = d_k == 128 && G <= 16;
+    const bool tensor_core_path = (d_k == 128 && G <= 16) || mla_tc_supported(d_k, d_v, G);
     if (a.max_splits > 1 || tensor_core_path) {
         const WorkspaceMap m = workspace_map(B, H_q, d_v, a.max_splits);
         if (!workspace || workspace_bytes < m.total) return BDFP4_ERR_WORKSPACE;

@@ -69,6 +69,13 @@ inline int plan_chunk_tiles(int64_t total_tiles, int max_tiles, int num_sms) {
 // images, and the decode overlaps it (programmatic dependent launch).
 int launch_decode_tc(const DecodeArgs& a, int fmt, int G, cudaStream_t st, const StepArgs* step = nullptr);
 
+// tcgen05 decode for MLA shapes (d_k = 576, d_v = 512, G in {16, 32, 64, 128};
+// decode_mla_tc.cu): a prologue grid (query images, and a step's append) and
+// the decode, overlapped the same way.
+bool mla_tc_supported(int d_k, int d_v, int G);
+int mla_query_image_bytes(int fmt, int G);
+int launch_decode_mla_tc(const DecodeArgs& a, int fmt, int G, cudaStream_t st, const StepArgs* step = nullptr);
+
 // Decode-step append on its own (quantize.cu), for the CUDA-core decode path.
 int launch_step_append(const DecodeArgs& a, const StepArgs& s, int fmt, int d_k, cudaStream_t st);
 

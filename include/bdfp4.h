@@ -178,9 +178,10 @@ BDFP4_API int bdfp4_decode_plan(const int32_t* host_seq_lens, int B, int H_kv, i
 
 /* Bytes of workspace bdfp4_decode needs for this shape and chunk_tiles: the
  * fp32 partial outputs and (m, l) pairs of the splits (when a sequence can
- * have more than one), then 640 bytes per query head for the query images the
- * d_k = 128 path computes once per (sequence, KV head) before the decode
- * kernel reads them.  Contents need no initialisation; calls that run at the
+ * have more than one), then 656 bytes per query head for the query images the
+ * tensor-core paths (d_k = 128; MLA d_k = 576 with G = 16, 32, 64 or 128)
+ * compute once per (sequence, KV head, head slice) before the decode kernel
+ * reads them.  Contents need no initialisation; calls that run at the
  * same time must not share a workspace. */
 BDFP4_API size_t bdfp4_decode_workspace_size(int B, int H_q, int d_v, int max_pages_per_seq, int chunk_tiles);
 
@@ -198,7 +199,8 @@ BDFP4_API size_t bdfp4_decode_workspace_size(int B, int H_q, int d_v, int max_pa
  * O accumulates P^ V; splits merge by log-sum-exp.  An empty sequence gives
  * zeros.  chunk_tiles <= 0 picks a plan from device seq_lens' upper bound
  * (max_pages_per_seq * 64).  workspace: >= bdfp4_decode_workspace_size bytes
- * (required for d_k = 128 and whenever a sequence can have several splits).
+ * (required on the tensor-core paths and whenever a sequence can have several
+ * splits).
  */
 BDFP4_API int bdfp4_decode(const void* q, const void* k_pages, const void* k_scales, const void* v_pages,
                  const void* v_scales, const int32_t* block_table, const int32_t* seq_lens, int B, int H_q, int H_kv,

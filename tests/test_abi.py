@@ -62,10 +62,10 @@ def test_decode_plan_host_logic(lib):
 
 def test_workspace_size(lib):
     # B=2, H_q=4, d_v=128, 16 pages = 8 tiles, 2 tiles per split -> 4 splits: fp32 partial
-    # outputs and (m, l) pairs, each padded to 256 B, then 640 B of query image per query head
+    # outputs and (m, l) pairs, each padded to 256 B, then 656 B of query image per query head
     o = 2 * 4 * 4 * 128 * 4
     ml = 2 * 4 * 4 * 2 * 4
-    q = 2 * 4 * 640
+    q = 2 * 4 * 656
     pad = lambda n: (n + 255) // 256 * 256  # noqa: E731
     assert bdfp4.bdfp4_decode_workspace_size(2, 4, 128, 16, 2) == pad(o) + pad(ml) + q
     # one split per sequence: only the query images
@@ -132,3 +132,15 @@ def test_bf16_entry_points_reject_bad_arguments(lib):
                                None) == -1
     assert L.bdfp4_bf16_append(None, None, None, -1, 1, 128, None, None, 1, None, None) == -1
     assert L.bdfp4_bf16_append(None, None, None, 0, 1, 128, None, None, 1, None, None) == 0
+
+
+def test_output_comparison_counts_one_bf16_step_as_agreement():
+    """The parity comparison: differences of one bf16 step (the two sides
+    rounding across a boundary) agree; anything larger counts at full size."""
+    from _util import compare_outputs
+
+    assert compare_outputs(np.array([16.0]), np.array([16.125]))[0] == 0.0     # one step at [16, 32)
+    assert compare_outputs(np.array([16.0]), np.array([16.25]))[0] == 0.25     # two steps
+    assert compare_outputs(np.array([1.0]), np.array([1.0078125]))[0] == 0.0   # one step at [1, 2)
+    assert abs(compare_outputs(np.array([0.5]), np.array([0.52]))[0] - 0.02) < 1e-12
+    assert compare_outputs(np.array([3.0]), np.array([3.0]))[1] == 0.0
