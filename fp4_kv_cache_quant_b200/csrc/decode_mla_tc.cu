@@ -13,8 +13,8 @@
 // O stays in TMEM: when a head's running maximum rises, the softmax warps that
 // own the head rescale its O columns after the previous tile's PV completed and
 // before this tile's PV is issued -- the online-softmax update, in place.
-//   warps 0 .. 4 NSG - 1   softmax: group g owns heads HG g .. HG g + HG - 1 (HG = 16
-//                          or 32), its warp q the tokens (TMEM lanes) 32 q .. 32 q + 31
+//   warps 0 .. 4 NSG - 1   softmax: group g owns heads 16 g .. 16 g + 15, its warp q
+//                          the tokens (TMEM lanes) 32 q .. 32 q + 31
 //   warp  4 NSG            producer: K and V pages by bulk copy, K scales by cp.async
 //   warp  4 NSG + 1        MMA issuer (one lane) and TMEM owner
 // Every wait is bounded; a timeout sets BDFP4_DEV_TIMEOUT and the CTA unwinds.
@@ -40,9 +40,7 @@ struct MlaCfg {
     static constexpr int NKG = (NBLK + 3) / 4;         // 4-block key scale groups per token
     static constexpr int KPG = MX ? 2 : 1;             // K steps per key scale group
     static constexpr int MT = DV / 128;                // 128-channel M tiles of O^T
-    // heads per softmax group: two groups of up to 32 (at most ten warps, so no
-    // SM sub-partition holds more than three and each thread may use 168 registers)
-    static constexpr int HG = GH >= 32 ? GH / 2 : GH;
+    static constexpr int HG = 16;                      // heads per softmax group
     static constexpr int NSG = GH / HG;                // softmax groups
     static constexpr int NSW = 4 * NSG;                // softmax warps
     static constexpr int PRODUCER = NSW, MMA_WARP = NSW + 1;
@@ -77,9 +75,12 @@ struct MlaCfg {
     static constexpr int SM_P = (SM_Q + QPACK + 127) / 128 * 128;
     static constexpr int SM_PSF = SM_P + 2 * P_BUF;    // [2 buf][2 page][32 rows][16 B] P scales
     static constexpr int SM_RED = SM_PSF + 2 * 2 * 512;
-    // per softmax warp: the running maxima and the last corrections of its group's heads
+    // per softmax warp and head of its group: the tile's softmax terms for the warp's two
+    // token blocks {logit scale, exponent base, correction, 1 / block scale} x 2, the two
+    // block-scale codes, and an output scale
+    static constexpr int WST_WARP = HG * 32 + HG * 4 + HG * 4;
     static constexpr int SM_WST = SM_RED + 2 * RED_BUF * 4;
-    static constexpr int SM_BARS = SM_WST + NSW * HG * 2 * 4;
+    static constexpr int SM_BARS = SM_WST + NSW * WST_WARP;
     static constexpr int NBARS = 2 * NSK + 2 * NSV + 8;
     static constexpr int SM_MISC = SM_BARS + NBARS * 8;   // tmem slot, abort flags
     static constexpr int SMEM = SM_MISC + 32;
@@ -200,7 +201,7 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
     uint8_t* p_op = smem + C::SM_P;
     uint8_t* psf = smem + C::SM_PSF;
     float* red = reinterpret_cast<float*>(smem + C::SM_RED);
-    float* wst = reinterpret_cast<float*>(smem + C::SM_WST);
+    uint8_t* wst = smem + C::SM_WST;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SM_BARS);
     uint64_t* kfull = bars;                   // [NSK] K tile landed -> MMA
     uint64_t* kempty = kfull + C::NSK;        // [NSK] QK done -> producer
@@ -489,13 +490,14 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
         tc::named_bar_sync(1 + C::NSG, 32 * C::NSW);   // psf zeroed before any tile writes it
         if (lane == 0) tc::mbar_arrive(q_ready);
 
-        // the running maxima (in scaled log2 units) and this tile's corrections live in the
-        // warp's own shared-memory slots (every warp of a group computes the same values):
-        // only the partial sums of l stay in registers
-        float* const m_run = wst + warp * HG * 2;
-        float* const corr = m_run + HG;
-        if (lane < HG) m_run[lane] = -INFINITY;
-        __syncwarp();
+        // Running maxima (scaled log2 units) are kept one head per lane: lane g of every warp
+        // of the group tracks head gb + g and posts, per tile, the terms every lane of the
+        // warp needs for that head to the warp's own shared-memory slots.
+        float4* const wterm = reinterpret_cast<float4*>(wst + warp * C::WST_WARP);   // [HG][2 blocks]
+        uint32_t* const wcode = reinterpret_cast<uint32_t*>(wst + warp * C::WST_WARP + HG * 32);   // [HG]
+        float* const wout = reinterpret_cast<float*>(wst + warp * C::WST_WARP + HG * 36);          // [HG]
+        float m_lane = -INFINITY;                   // running maximum of head gb + lane
+        const float ls_lane = lane < HG ? lsc[gb + lane] : 0.0f;
         float l_part[HG];
 #pragma unroll
         for (int g = 0; g < HG; ++g) l_part[g] = 0.0f;
@@ -540,103 +542,105 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
             if (bad || *abort_flag) sm_abort[grp] = 1;
             tc::named_bar_sync(bar_id, 128);
             if (sm_abort[grp]) break;
-            // running maxima: the correction of each head, applied to l here and to O below
-            bool rescale = false;
-            {
-#pragma unroll
-                for (int g = 0; g < HG; ++g) {
-                    const float* w = rw + (gb + g) * 8;
-                    const float4 w0 = *reinterpret_cast<const float4*>(w);
-                    const float4 w1 = *reinterpret_cast<const float4*>(w + 4);
-                    const float mt = fmaxf(fmaxf(fmaxf(w0.x, w0.y), fmaxf(w0.z, w0.w)),
-                                           fmaxf(fmaxf(w1.x, w1.y), fmaxf(w1.z, w1.w)));
-                    const float mo = m_run[g];
-                    const float mn = fmaxf(mo, mt * lsc[gb + g]);
-                    const float mz = mn == -INFINITY ? 0.0f : mn;
-                    const float cg = tc::ex2_approx(mo - mz);   // 0 on the split's first tile
-                    rescale |= mn != mo;
-                    l_part[g] *= cg;
-                    __syncwarp();
-                    if (lane == 0) {
-                        m_run[g] = mn;
-                        corr[g] = cg;
-                    }
+            // new running maxima, one head per lane, and the scales of the warp's two token
+            // blocks: the block maximum of alpha p is 2^(x_b ls - base) for the block's largest
+            // logit x_b, so the scale is the one the block's largest member picks
+            bool rose = false;
+            if (lane < HG) {
+                const float* w = rw + (gb + lane) * 8;
+                const float4 w0 = *reinterpret_cast<const float4*>(w);
+                const float4 w1 = *reinterpret_cast<const float4*>(w + 4);
+                const float mt = fmaxf(fmaxf(fmaxf(w0.x, w0.y), fmaxf(w0.z, w0.w)),
+                                       fmaxf(fmaxf(w1.x, w1.y), fmaxf(w1.z, w1.w)));
+                const float mn = fmaxf(m_lane, mt * ls_lane);
+                const float mz = mn == -INFINITY ? 0.0f : mn;
+                const float corr = tc::ex2_approx(m_lane - mz);   // 0 on the split's first tile
+                const float base = mz - la;
+                rose = mn != m_lane;
+                m_lane = mn;
+                const float bm_lo = w[qd * 2], bm_hi = w[qd * 2 + 1];
+                // per block: NVFP4 {ls, base, corr, 1 / scale}, the element is alpha p / scale;
+                // MXFP4 {ls, base + e, corr, 2^e} for the scale 2^e, the element is 2^(x ls - base - e)
+                // (the exponent's argument stays small, as the OCP rule's element) and p its 2^e multiple
+                float r_lo, r_hi, b_lo = base, b_hi = base;
+                uint32_t codes;
+                if constexpr (!MX) {
+                    const float a_lo = tc::ex2_approx(fmaf(bm_lo, ls_lane, -base));
+                    const float a_hi = tc::ex2_approx(fmaf(bm_hi, ls_lane, -base));
+                    codes = tc::e4m3x2_encode(__fmul_rn(a_lo, 1.0f / 6.0f), __fmul_rn(a_hi, 1.0f / 6.0f));
+                    const float2 sg = tc::e4m3x2_value(codes);
+                    // a zero scale zeroes the whole block inside the MMA, whatever the element codes
+                    r_lo = tc::rcp_approx(sg.x);
+                    r_hi = tc::rcp_approx(sg.y);
+                } else {
+                    // one 32-token block per warp; the OCP MX shared exponent in the log domain:
+                    // the block maximum is 2^d with d = x_b ls - m <= 0, so floor(log2) = floor(d)
+                    // and the element is p 2^(127 - c) for the E8M0 code c
+                    const float d = __fsub_rn(__fmul_rn(fmaxf(bm_lo, bm_hi), ls_lane), mz);
+                    const int c = max(__float2int_rd(fmaxf(d, -256.0f)) + 125, 0);
+                    codes = (uint32_t)c | ((uint32_t)c << 8);
+                    b_lo = b_hi = mz + (float)(c - 127);
+                    r_lo = r_hi = __uint_as_float(c > 0 ? (uint32_t)c << 23 : 0x00400000u);   // 2^(c - 127)
                 }
-                __syncwarp();
-                // O^T rescale of the group's heads once the previous tile's PV has completed;
-                // the group's warps decide alike, having read the same maxima
-                if (j > 0 && rescale) {
-                    if (!tc::mbar_wait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, kWaitLimitMla))
-                        bad = true;
-                    tc::tc_fence_after();
+                wterm[lane * 2 + 0] = make_float4(ls_lane, b_lo, corr, r_lo);
+                wterm[lane * 2 + 1] = make_float4(ls_lane, b_hi, corr, r_hi);
+                wcode[lane] = codes;
+            }
+            const uint32_t rmask = j > 0 ? __ballot_sync(0xffffffffu, rose) : 0u;
+            __syncwarp();
+            // O^T rescale of the heads whose maximum rose, once the previous tile's PV has
+            // completed; the group's warps decide alike, having read the same maxima
+            if (rmask) {
+                if (!tc::mbar_wait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, kWaitLimitMla)) bad = true;
+                tc::tc_fence_after();
+                uint32_t rem = rmask;
+                while (rem) {
+                    // up to four heads per round trip: their columns in the four M tiles
+                    int hs_[4];
+                    uint32_t ov[4][MT];
 #pragma unroll
-                    for (int t = 0; t < MT; ++t) {
+                    for (int k = 0; k < 4; ++k) {
+                        hs_[k] = rem ? __ffs(rem) - 1 : -1;
+                        if (rem) rem &= rem - 1;
+                        if (hs_[k] >= 0) {
 #pragma unroll
-                        for (int h8 = 0; h8 < HG; h8 += 8) {
-                            uint32_t ov[8];
-                            tc::tmem_ld<8>(tq + C::T_O + t * GH + gb + h8, ov);
-                            tc::tmem_wait_ld();
-#pragma unroll
-                            for (int g = 0; g < 8; ++g)
-                                ov[g] = __float_as_uint(__uint_as_float(ov[g]) * corr[h8 + g]);
-                            tc::tmem_st8(tq + C::T_O + t * GH + gb + h8, ov);
+                            for (int t = 0; t < MT; ++t) tc::tmem_ld<1>(tq + C::T_O + t * GH + gb + hs_[k], &ov[k][t]);
                         }
                     }
-                    tc::tmem_wait_st();
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        if (hs_[k] < 0) continue;
+                        const float c = wterm[hs_[k] * 2].z;
+#pragma unroll
+                        for (int t = 0; t < MT; ++t)
+                            tc::tmem_st1(tq + C::T_O + t * GH + gb + hs_[k], __float_as_uint(__uint_as_float(ov[k][t]) * c));
+                    }
                 }
+                tc::tmem_wait_st();
             }
             // probabilities and their FP4 quantization, two heads per conversion
             uint8_t* const pb = pbyte + (j & 1) * C::P_BUF;
             uint8_t* const sfb = sfbase + (j & 1) * 2 * 512;
+            const int half = lo_half ? 0 : 1;
 #pragma unroll
             for (int g = 0; g < HG; g += 2) {
-                float y[2], am[2];
-                uint32_t mxc[2];
+                float q[2];
 #pragma unroll
                 for (int u = 0; u < 2; ++u) {
-                    const int hh = g + u;
-                    const float ls = lsc[gb + hh];
-                    const float mz = m_run[hh] == -INFINITY ? 0.0f : m_run[hh];
-                    const float base = mz - la;
-                    const float x = valid ? __uint_as_float(sr[hh]) : -INFINITY;
-                    y[u] = tc::ex2_approx(fmaf(x, ls, -base));   // 0 for masked tokens
-                    l_part[hh] += y[u];                           // l in units of alpha
-                    const float* w = rw + (gb + hh) * 8;
-                    const float hm_lo = w[qd * 2], hm_hi = w[qd * 2 + 1];
-                    if constexpr (!MX) {
-                        // a 16-token block is this half warp
-                        const float bm = lo_half ? hm_lo : hm_hi;
-                        am[u] = tc::ex2_approx(fmaf(bm, ls, -base));
-                        mxc[u] = 0u;
-                    } else {
-                        // a 32-token block is this warp; the OCP MX shared exponent is taken in
-                        // the log domain, as in the d = 128 kernel
-                        const float bm = fmaxf(hm_lo, hm_hi);
-                        const float d = __fsub_rn(__fmul_rn(bm, ls), mz);
-                        const int c = max(__float2int_rd(fmaxf(d, -256.0f)) + 125, 0);
-                        mxc[u] = (uint32_t)c;
-                        am[u] = tc::ex2_approx(fmaf(x, ls, -(mz + (float)(c - 127))));
-                    }
+                    const float4 v = wterm[(g + u) * 2 + half];
+                    const float x = valid ? __uint_as_float(sr[g + u]) : -INFINITY;
+                    const float e = tc::ex2_approx(fmaf(x, v.x, -v.y));   // 0 for masked tokens
+                    const float y = MX ? e * v.w : e;                     // alpha p
+                    l_part[g + u] = fmaf(l_part[g + u], v.z, y);          // l in units of alpha
+                    q[u] = MX ? e : e * v.w;
                 }
-                uint32_t codes;
-                float q0, q1;
-                if constexpr (FMT == BDFP4_NVFP4) {
-                    codes = tc::e4m3x2_encode(__fmul_rn(am[0], 1.0f / 6.0f), __fmul_rn(am[1], 1.0f / 6.0f));
-                    const float2 sg = tc::e4m3x2_value(codes);
-                    // a zero scale zeroes the whole block inside the MMA, whatever the element codes
-                    q0 = y[0] * tc::rcp_approx(sg.x);
-                    q1 = y[1] * tc::rcp_approx(sg.y);
-                } else {
-                    codes = mxc[0] | (mxc[1] << 8);
-                    q0 = am[0];    // the element already divided by its block scale
-                    q1 = am[1];
-                }
-                const uint32_t mine = e2m1x2_encode(q0, q1);   // head g in bits 0..3, head g + 1 in 4..7
+                const uint32_t mine = e2m1x2_encode(q[0], q[1]);   // head g in bits 0..3, head g + 1 in 4..7
                 const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
                 const uint32_t wv = __byte_perm(mine, other, psel) >> (4 * hsel);
                 const int hr = gb + g + hsel;
                 pb[(hr >> 3) * 256 + (hr & 7) * 16] = (uint8_t)((wv & 0xfu) | ((wv >> 4) & 0xf0u));
-                if (sfstore) sfb[(hr & 31) * 16 + (hr >> 5) * 4] = (uint8_t)(codes >> (8 * hsel));
+                if (sfstore) sfb[(hr & 31) * 16 + (hr >> 5) * 4] = (uint8_t)(wcode[g + hsel] >> (8 * half));
             }
             // V scale factors (group 0): blocks past the sequence end are zeroed (NVFP4, in the
             // stage before its TMEM copy) or masked (MXFP4, stored into TMEM by these warps)
@@ -710,13 +714,19 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
             tc::named_bar_sync(bar_id, 128);
             // O and l both carry the factor alpha (P^ is alpha p quantized), so it cancels
             const float oscale = FMT == BDFP4_NVFP4 ? a.v_gscale[hk] : 1.0f;
-            float l[HG];
-#pragma unroll
-            for (int g = 0; g < HG; ++g) {
-                const float4 r4 = *reinterpret_cast<const float4*>(rl + (gb + g) * 4);
-                l[g] = r4.x + r4.y + r4.z + r4.w;
+            // lane g: the output scale and (m, l) of head gb + g, through the warp's slots
+            if (lane < HG) {
+                const float4 r4 = *reinterpret_cast<const float4*>(rl + (gb + lane) * 4);
+                const float l = r4.x + r4.y + r4.z + r4.w;
+                wout[lane] = nspl == 1 ? (l > 0.0f ? oscale / l : 0.0f) : oscale;
+                if (nspl > 1 && qd == 0) {
+                    const int64_t row = (int64_t)b * a.H_q + h0 + gb + lane;
+                    a.ws_ml[(row * a.max_splits + split) * 2 + 0] = m_lane;
+                    a.ws_ml[(row * a.max_splits + split) * 2 + 1] = l;
+                }
             }
-#pragma unroll
+            __syncwarp();
+#pragma unroll 1
             for (int t = 0; t < MT; ++t) {
                 uint32_t ov[HG];
                 tc::tmem_ld<HG>(tq + C::T_O + t * GH + gb, ov);
@@ -725,16 +735,9 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
 #pragma unroll
                 for (int g = 0; g < HG; ++g) {
                     const int64_t row = (int64_t)b * a.H_q + h0 + gb + g;
-                    const float o = __uint_as_float(ov[g]);
-                    if (nspl == 1) {
-                        a.out[row * C::DV + chan] = __float2bfloat16(l[g] > 0.0f ? o * oscale / l[g] : 0.0f);
-                    } else {
-                        a.ws_o[(row * a.max_splits + split) * C::DV + chan] = o * oscale;
-                        if (chan == 0) {
-                            a.ws_ml[(row * a.max_splits + split) * 2 + 0] = m_run[g];
-                            a.ws_ml[(row * a.max_splits + split) * 2 + 1] = l[g];
-                        }
-                    }
+                    const float o = __uint_as_float(ov[g]) * wout[g];
+                    if (nspl == 1) a.out[row * C::DV + chan] = __float2bfloat16(o);
+                    else a.ws_o[(row * a.max_splits + split) * C::DV + chan] = o;
                 }
             }
         }
