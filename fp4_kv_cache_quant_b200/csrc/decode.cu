@@ -24,6 +24,8 @@ namespace bdfp4 {
 
 template <int FMT, int DK, int DV, int HG>
 __global__ void __launch_bounds__(kThreads) decode_fp4_kernel(const DecodeArgs a) {
+    // the split merge (a programmatic dependent) may be scheduled as CTAs of this grid retire
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     constexpr int B = Fmt<FMT>::beta;
     constexpr int NCH = DV / kThreads;   // value channels per thread
     using RG = RowGeom<FMT, DK>;
@@ -329,25 +331,33 @@ extern "C" int bdfp4_decode_plan(const int32_t* host_seq_lens, int B, int H_kv, 
     return plan_chunk_tiles(total_tiles, max_tiles, num_sms);
 }
 
+// The split merge after a decode grid (nothing when no sequence can split).
+template <int DV>
+static int merge_splits(const DecodeArgs& a, cudaStream_t st) {
+    const int rc = launch_status();
+    if (rc != BDFP4_OK || a.max_splits <= 1) return rc;
+    const cudaError_t e = launch_merge<DV>(a.ws_o, a.ws_ml, a.seq_lens, a.B, a.H_q, a.max_pages, a.chunk_tiles,
+                                           a.max_splits, a.out, st);
+    if (e != cudaSuccess) {
+        record_cuda_error(e);
+        return BDFP4_ERR_CUDA;
+    }
+    return launch_status();
+}
+
 template <int FMT, int DK, int DV>
 static int launch_decode(const DecodeArgs& a, int G, cudaStream_t st, const StepArgs* step) {
     if (DK == 128 && G <= 16) {
         // tensor-core path (decode_tc.cu); a step's append runs in its prologue grid
         const int rc = launch_decode_tc(a, FMT, G, st, step);
         if (rc != BDFP4_OK) return rc;
-        if (a.max_splits > 1)
-            merge_splits_kernel<DV><<<a.B * a.H_q, 128, merge_smem(a.max_splits), st>>>(
-                a.ws_o, a.ws_ml, a.seq_lens, a.H_q, a.max_pages, a.chunk_tiles, a.max_splits, a.out);
-        return launch_status();
+        return merge_splits<DV>(a, st);
     }
     if (DK == 576 && mla_tc_supported(DK, DV, G)) {
         // tensor-core path for MLA shapes (decode_mla_tc.cu); a step's append runs in its prologue grid
         const int rc = launch_decode_mla_tc(a, FMT, G, st, step);
         if (rc != BDFP4_OK) return rc;
-        if (a.max_splits > 1)
-            merge_splits_kernel<DV><<<a.B * a.H_q, 128, merge_smem(a.max_splits), st>>>(
-                a.ws_o, a.ws_ml, a.seq_lens, a.H_q, a.max_pages, a.chunk_tiles, a.max_splits, a.out);
-        return launch_status();
+        return merge_splits<DV>(a, st);
     }
     if (step) {
         const int rc = launch_step_append(a, *step, FMT, DK, st);
@@ -363,10 +373,7 @@ static int launch_decode(const DecodeArgs& a, int G, cudaStream_t st, const Step
         case 16: decode_fp4_kernel<FMT, DK, DV, 16><<<grid, kThreads, 0, st>>>(a); break;
         default: return BDFP4_ERR_UNSUPPORTED;
     }
-    if (a.max_splits > 1)
-        merge_splits_kernel<DV><<<a.B * a.H_q, 128, merge_smem(a.max_splits), st>>>(
-            a.ws_o, a.ws_ml, a.seq_lens, a.H_q, a.max_pages, a.chunk_tiles, a.max_splits, a.out);
-    return launch_status();
+    return merge_splits<DV>(a, st);
 }
 
 static int run_decode(const void* q, const void* k_pages, const void* k_scales, const void* v_pages,

@@ -116,6 +116,8 @@ struct Bf16Args {
 template <int G>
 __global__ void __launch_bounds__(Bf16Cfg<G>::THREADS, 1) decode_bf16_kernel(const Bf16Args a) {
     using C = Bf16Cfg<G>;
+    // the split merge (a programmatic dependent) may be scheduled as CTAs of this grid retire
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     constexpr int HG = C::HG;
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t* q_op = smem + C::SM_Q;
@@ -433,8 +435,12 @@ static int launch_bf16(const Bf16Args& a, cudaStream_t st) {
     decode_bf16_kernel<G><<<grid, C::THREADS, C::SMEM, st>>>(a);
     const int rc = launch_status();
     if (rc != BDFP4_OK || a.max_splits <= 1) return rc;
-    merge_splits_kernel<C::D><<<a.B * a.H_q, 128, merge_smem(a.max_splits), st>>>(
-        a.ws_o, a.ws_ml, a.seq_lens, a.H_q, a.max_pages, a.chunk_tiles, a.max_splits, a.out);
+    const cudaError_t e = launch_merge<C::D>(a.ws_o, a.ws_ml, a.seq_lens, a.B, a.H_q, a.max_pages, a.chunk_tiles,
+                                             a.max_splits, a.out, st);
+    if (e != cudaSuccess) {
+        record_cuda_error(e);
+        return BDFP4_ERR_CUDA;
+    }
     return launch_status();
 }
 

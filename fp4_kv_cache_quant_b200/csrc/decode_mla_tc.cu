@@ -192,6 +192,8 @@ __global__ void __launch_bounds__(256) prep_mla_kernel(const DecodeArgs a, const
 template <int FMT, int GH>
 __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_kernel(const DecodeArgs a) {
     using C = MlaCfg<FMT, GH>;
+    // the split merge (a programmatic dependent) may be scheduled as CTAs of this grid retire
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     constexpr bool MX = C::MX;
     constexpr int B = C::B, HG = C::HG, MT = C::MT;
     extern __shared__ __align__(1024) uint8_t smem[];

@@ -210,6 +210,8 @@ __global__ void __launch_bounds__(256) prep_step_kernel(const DecodeArgs a, cons
 template <int FMT, int G>
 __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTAS) decode_tc_kernel(const DecodeArgs a) {
     using C = TcCfg<FMT, G>;
+    // the split merge (a programmatic dependent) may be scheduled as CTAs of this grid retire
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     constexpr bool MX = FMT == BDFP4_MXFP4;
     constexpr int B = C::B;
     constexpr int HG = C::HG;

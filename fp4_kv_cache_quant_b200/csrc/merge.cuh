@@ -17,6 +17,8 @@ __global__ void __launch_bounds__(128) merge_splits_kernel(const float* __restri
                                                            const int32_t* __restrict__ seq_lens, int H_q,
                                                            int max_pages, int chunk_tiles, int max_splits,
                                                            __nv_bfloat16* out) {
+    // launched as a programmatic dependent of the decode grid: wait for its partials
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int row = blockIdx.x;
     const int b = row / H_q;
     int N = seq_lens[b];
@@ -55,5 +57,26 @@ __global__ void __launch_bounds__(128) merge_splits_kernel(const float* __restri
 
 // Dynamic shared memory of merge_splits_kernel: a weight per split and L.
 inline size_t merge_smem(int max_splits) { return ((size_t)max_splits + 1) * sizeof(float); }
+
+// Launches the merge as a programmatic dependent of the decode grid just before
+// it on the stream: its CTAs are scheduled as the decode's last CTAs retire and
+// wait (griddepcontrol.wait) for the whole decode grid, so the launch latency
+// overlaps the decode's tail.  Returns the CUDA launch status.
+template <int DV>
+inline cudaError_t launch_merge(const float* ws_o, const float* ws_ml, const int32_t* seq_lens, int B, int H_q,
+                                int max_pages, int chunk_tiles, int max_splits, __nv_bfloat16* out, cudaStream_t st) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(B * H_q);
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = merge_smem(max_splits);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, merge_splits_kernel<DV>, ws_o, ws_ml, seq_lens, H_q, max_pages, chunk_tiles,
+                              max_splits, out);
+}
 
 }  // namespace bdfp4
