@@ -57,15 +57,20 @@ def algorithmic_bytes(sp, seq_lens, fmt: int) -> int:
     return tok * per_tok + pages * 4 + sp.B * sp.H_q * (sp.d_k + sp.d_v) * 2
 
 
-DECODE_SOURCES = ("decode_tc.cu", "tc_ptx.cuh", "bdfp4_device.cuh", "quant_device.cuh", "decode_common.cuh",
-                  "append_device.cuh")
+# sources of each tensor-core decode kernel: its file and the headers it includes
+DECODE_SOURCES = {
+    128: ("decode_tc.cu", "tc_ptx.cuh", "bdfp4_device.cuh", "quant_device.cuh", "decode_common.cuh",
+          "append_device.cuh"),
+    576: ("decode_mla_tc.cu", "tc_ptx.cuh", "bdfp4_device.cuh", "quant_device.cuh", "decode_common.cuh",
+          "append_device.cuh"),
+}
 
 
-def decode_source_hash() -> str:
-    """sha256 over the sources of the tensor-core decode kernel."""
+def decode_source_hash(d_k: int = 128) -> str:
+    """sha256 over the sources of the tensor-core decode kernel for head dim d_k."""
     import hashlib
     h = hashlib.sha256()
-    for name in DECODE_SOURCES:
+    for name in DECODE_SOURCES[d_k]:
         with open(os.path.join(ROOT, "fp4_kv_cache_quant_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
@@ -313,7 +318,7 @@ def run_ours(args, sp, fmt):
     if os.path.exists(tr_path):
         rec = json.load(open(tr_path)).get(f"{args.config}_{args.fmt}")
         # the counters describe the kernel as captured: null once its sources changed
-        if rec and rec.get("source_sha256") == decode_source_hash():
+        if rec and rec.get("source_sha256") == decode_source_hash(sp.d_k):
             traffic = rec.get("bytes_per_launch")
     result = {
         "metric": "FP4 paged decode-attn KV tokens/s",
