@@ -25,26 +25,28 @@ __global__ void __launch_bounds__(128) merge_splits_kernel(const float* __restri
     if (N < 0 || N > max_pages * kPageSlots) N = 0;
     const int ns = num_splits(N, chunk_tiles);
     if (ns <= 1) return;   // written by the decode kernel
-    // split weights 2^(m_s - M) through shared memory: the (m, l) pairs load in
-    // parallel, one per thread, instead of one dependent load per split
-    extern __shared__ float sw[];   // [ns] weights, then L
+    // split weights 2^(m_s - M) and L = sum_s 2^(m_s - M) l_s, every split's (m, l) pair
+    // loaded by its own thread (the loads overlap instead of following one another)
+    extern __shared__ float sw[];   // [ns] weights
+    __shared__ float red[2][4];
     const float* ml = ws_ml + (int64_t)row * max_splits * 2;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     float M = -INFINITY;
     for (int s = threadIdx.x; s < ns; s += blockDim.x) M = fmaxf(M, ml[2 * s]);
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    __shared__ float wmax[4];
-    if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = M;
+    if (lane == 0) red[0][wid] = M;
     __syncthreads();
-    M = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
-    for (int s = threadIdx.x; s < ns; s += blockDim.x) sw[s] = exp2f(ml[2 * s] - M);
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        float L = 0.0f;
-        for (int s = 0; s < ns; ++s) L += ml[2 * s + 1] * sw[s];
-        sw[ns] = L;
+    M = fmaxf(fmaxf(red[0][0], red[0][1]), fmaxf(red[0][2], red[0][3]));
+    float Lp = 0.0f;
+    for (int s = threadIdx.x; s < ns; s += blockDim.x) {
+        const float w = exp2f(ml[2 * s] - M);
+        sw[s] = w;
+        Lp += ml[2 * s + 1] * w;
     }
+    for (int off = 16; off > 0; off >>= 1) Lp += __shfl_xor_sync(0xffffffffu, Lp, off);
+    if (lane == 0) red[1][wid] = Lp;
     __syncthreads();
-    const float L = sw[ns];
+    const float L = (red[1][0] + red[1][1]) + (red[1][2] + red[1][3]);
     const float inv = L > 0.0f ? 1.0f / L : 0.0f;
     for (int c = threadIdx.x; c < DV; c += blockDim.x) {
         const float* o = ws_o + (int64_t)row * max_splits * DV + c;
@@ -55,8 +57,8 @@ __global__ void __launch_bounds__(128) merge_splits_kernel(const float* __restri
     }
 }
 
-// Dynamic shared memory of merge_splits_kernel: a weight per split and L.
-inline size_t merge_smem(int max_splits) { return ((size_t)max_splits + 1) * sizeof(float); }
+// Dynamic shared memory of merge_splits_kernel: a weight per split.
+inline size_t merge_smem(int max_splits) { return (size_t)max_splits * sizeof(float); }
 
 // Launches the merge as a programmatic dependent of the decode grid just before
 // it on the stream: its CTAs are scheduled as the decode's last CTAs retire and
