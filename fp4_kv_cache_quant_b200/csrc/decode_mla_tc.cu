@@ -19,6 +19,8 @@
 //   warp  4 NSG + 1        MMA issuer (one lane) and TMEM owner
 // Every wait is bounded; a timeout sets BDFP4_DEV_TIMEOUT and the CTA unwinds.
 
+#include <type_traits>
+
 #include "append_device.cuh"
 #include "bdfp4_device.cuh"
 #include "decode_common.cuh"
@@ -83,7 +85,8 @@ struct MlaCfg {
     static constexpr int SM_BARS = SM_WST + NSW * WST_WARP;
     static constexpr int NBARS = 2 * NSK + 2 * NSV + 8;
     static constexpr int SM_MISC = SM_BARS + NBARS * 8;   // tmem slot, abort flags
-    static constexpr int SMEM = SM_MISC + 32;
+    static constexpr int SM_PFLAG = SM_MISC + 32;   // [64] page flags of the split's tiles, any-bad
+    static constexpr int SMEM = SM_PFLAG + 64 + 16;
     // TMEM column map
     static constexpr int T_S = 0;
     static constexpr int T_O = GH;                     // M tile t at T_O + t GH
@@ -456,6 +459,32 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
         const float alpha = (FMT == BDFP4_NVFP4 && !(a.flags & BDFP4_FLAG_NO_UNDERFLOW)) ? kAlphaNV : 1.0f;
         bool bad = false;
 
+        // Pages the block table gets wrong (the producer reports them and copies nothing) are
+        // skipped like tokens past the end: their logits are masked and their V scales zeroed.
+        // Before the first tile the softmax threads note, per tile of the split, whether both
+        // of its pages are good (bit 0: first page, bit 1: second) and whether any is not;
+        // splits longer than 64 tiles look tiles 64 on up in the block table as they go.
+        uint8_t* const pflag = smem + C::SM_PFLAG;
+        volatile int* const pflag_bad = reinterpret_cast<volatile int*>(smem + C::SM_PFLAG + 64);
+        auto page_flags = [&](int jt) -> uint32_t {
+            uint32_t r = 3u;
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                const int pi = (tile0 + jt) * 2 + p;
+                if (pi * kPageSlots < N) {   // pages past the end are masked anyway
+                    const int v = __ldg(a.block_table + (int64_t)b * a.max_pages + pi);
+                    if (v < 0 || v >= a.num_pages) r &= ~(1u << p);
+                }
+            }
+            return r;
+        };
+        if (tid == 0) *pflag_bad = n > 64 ? 1 : 0;
+        tc::named_bar_sync(1 + C::NSG, 32 * C::NSW);
+        if (tid < 64 && tid < n) {
+            const uint32_t f = page_flags(tid);
+            pflag[tid] = (uint8_t)f;
+            if (f != 3u) *pflag_bad = 1;
+        }
         // the query image arrives in one bulk copy from the prologue grid, which this
         // grid may overlap: griddepcontrol.wait holds the copy until its writes are visible
         if (tid == 0) {
@@ -489,7 +518,8 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
         }
         tc::tc_fence_before();
         tc::fence_proxy_async_smem();
-        tc::named_bar_sync(1 + C::NSG, 32 * C::NSW);   // psf zeroed before any tile writes it
+        tc::named_bar_sync(1 + C::NSG, 32 * C::NSW);   // psf zeroed and page flags set before any tile
+        const bool any_bad_page = *pflag_bad != 0;
         if (lane == 0) tc::mbar_arrive(q_ready);
 
         // Running maxima (scaled log2 units) are kept one head per lane: lane g of every warp
@@ -519,182 +549,196 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
         uint8_t* const pbyte = p_op + page_of_thread * C::P_PAGE + (qd & 1) * 128 + (lane >> 1);
         uint8_t* const sfbase = psf + page_of_thread * 512 + pos_in_page / B;
 
-        for (int j = 0; j < n; ++j) {
-            const int tile = tile0 + j;
-            if (!tc::mbar_wait(s_full, j & 1, abort_flag, kWaitLimitMla)) bad = true;
-            tc::tc_fence_after();
-            uint32_t sr[HG];
-            tc::tmem_ld<HG>(tq + C::T_S + gb, sr);
-            tc::tmem_wait_ld();
-            // S may be overwritten by the next QK once every softmax warp has it in registers
-            tc::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(s_free);
-            const int token = tile * kTileTokens + tok_in_tile;
-            const bool valid = token < N;
-            // raw logits (q1 + q2).k; maxima over each half warp (16 consecutive slots)
-            float* rw = red + (j & 1) * C::RED_BUF;
-#pragma unroll
-            for (int g = 0; g < HG; ++g) {
-                const float x = valid ? __uint_as_float(sr[g]) : -INFINITY;
-                const float lo = tc::redux_max_f32(lo_half ? x : -INFINITY, 0xffffffffu);
-                const float hi = tc::redux_max_f32(lo_half ? -INFINITY : x, 0xffffffffu);
-                if (lane == 0) *reinterpret_cast<float2*>(rw + ((gb + g) * 4 + qd) * 2) = make_float2(lo, hi);
-            }
-            if (bad || *abort_flag) sm_abort[grp] = 1;
-            tc::named_bar_sync(bar_id, 128);
-            if (sm_abort[grp]) break;
-            // new running maxima, one head per lane, and the scales of the warp's two token
-            // blocks: the block maximum of alpha p is 2^(x_b ls - base) for the block's largest
-            // logit x_b, so the scale is the one the block's largest member picks
-            bool rose = false;
-            if (lane < HG) {
-                const float* w = rw + (gb + lane) * 8;
-                const float4 w0 = *reinterpret_cast<const float4*>(w);
-                const float4 w1 = *reinterpret_cast<const float4*>(w + 4);
-                const float mt = fmaxf(fmaxf(fmaxf(w0.x, w0.y), fmaxf(w0.z, w0.w)),
-                                       fmaxf(fmaxf(w1.x, w1.y), fmaxf(w1.z, w1.w)));
-                const float mn = fmaxf(m_lane, mt * ls_lane);
-                const float mz = mn == -INFINITY ? 0.0f : mn;
-                const float corr = tc::ex2_approx(m_lane - mz);   // 0 on the split's first tile
-                const float base = mz - la;
-                rose = mn != m_lane;
-                m_lane = mn;
-                const float bm_lo = w[qd * 2], bm_hi = w[qd * 2 + 1];
-                // per block: NVFP4 {ls, base, corr, 1 / scale}, the element is alpha p / scale;
-                // MXFP4 {ls, base + e, corr, 2^e} for the scale 2^e, the element is 2^(x ls - base - e)
-                // (the exponent's argument stays small, as the OCP rule's element) and p its 2^e multiple
-                float r_lo, r_hi, b_lo = base, b_hi = base;
-                uint32_t codes;
-                if constexpr (!MX) {
-                    const float a_lo = tc::ex2_approx(fmaf(bm_lo, ls_lane, -base));
-                    const float a_hi = tc::ex2_approx(fmaf(bm_hi, ls_lane, -base));
-                    codes = tc::e4m3x2_encode(__fmul_rn(a_lo, 1.0f / 6.0f), __fmul_rn(a_hi, 1.0f / 6.0f));
-                    const float2 sg = tc::e4m3x2_value(codes);
-                    // a zero scale zeroes the whole block inside the MMA, whatever the element codes
-                    r_lo = tc::rcp_approx(sg.x);
-                    r_hi = tc::rcp_approx(sg.y);
-                } else {
-                    // one 32-token block per warp; the OCP MX shared exponent in the log domain:
-                    // the block maximum is 2^d with d = x_b ls - m <= 0, so floor(log2) = floor(d)
-                    // and the element is p 2^(127 - c) for the E8M0 code c
-                    const float d = __fsub_rn(__fmul_rn(fmaxf(bm_lo, bm_hi), ls_lane), mz);
-                    const int c = max(__float2int_rd(fmaxf(d, -256.0f)) + 125, 0);
-                    codes = (uint32_t)c | ((uint32_t)c << 8);
-                    b_lo = b_hi = mz + (float)(c - 127);
-                    r_lo = r_hi = __uint_as_float(c > 0 ? (uint32_t)c << 23 : 0x00400000u);   // 2^(c - 127)
+        // The tile loop, in two copies: the page checks exist only in the copy a split with a
+        // bad page runs, so the normal copy carries no extra live registers.
+        auto tiles = [&](auto masked) {
+            for (int j = 0; j < n; ++j) {
+                const int tile = tile0 + j;
+                bool pok0 = true, pok1 = true;
+                if constexpr (decltype(masked)::value) {
+                    const uint32_t f = j < 64 ? pflag[j] : page_flags(j);
+                    pok0 = (f & 1u) != 0;
+                    pok1 = (f & 2u) != 0;
                 }
-                wterm[lane * 2 + 0] = make_float4(ls_lane, b_lo, corr, r_lo);
-                wterm[lane * 2 + 1] = make_float4(ls_lane, b_hi, corr, r_hi);
-                wcode[lane] = codes;
-            }
-            const uint32_t rmask = j > 0 ? __ballot_sync(0xffffffffu, rose) : 0u;
-            __syncwarp();
-            // O^T rescale of the heads whose maximum rose, once the previous tile's PV has
-            // completed; the group's warps decide alike, having read the same maxima
-            if (rmask) {
-                if (!tc::mbar_wait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, kWaitLimitMla)) bad = true;
+                if (!tc::mbar_wait(s_full, j & 1, abort_flag, kWaitLimitMla)) bad = true;
                 tc::tc_fence_after();
-                uint32_t rem = rmask;
-                while (rem) {
-                    // up to four heads per round trip: their columns in the four M tiles
-                    int hs_[4];
-                    uint32_t ov[4][MT];
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        hs_[k] = rem ? __ffs(rem) - 1 : -1;
-                        if (rem) rem &= rem - 1;
-                        if (hs_[k] >= 0) {
-#pragma unroll
-                            for (int t = 0; t < MT; ++t) tc::tmem_ld<1>(tq + C::T_O + t * GH + gb + hs_[k], &ov[k][t]);
+                uint32_t sr[HG];
+                tc::tmem_ld<HG>(tq + C::T_S + gb, sr);
+                tc::tmem_wait_ld();
+                // S may be overwritten by the next QK once every softmax warp has it in registers
+                tc::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(s_free);
+                const int token = tile * kTileTokens + tok_in_tile;
+                const bool valid = token < N && (page_of_thread ? pok1 : pok0);
+                // raw logits (q1 + q2).k; maxima over each half warp (16 consecutive slots)
+                float* rw = red + (j & 1) * C::RED_BUF;
+    #pragma unroll
+                for (int g = 0; g < HG; ++g) {
+                    const float x = valid ? __uint_as_float(sr[g]) : -INFINITY;
+                    const float lo = tc::redux_max_f32(lo_half ? x : -INFINITY, 0xffffffffu);
+                    const float hi = tc::redux_max_f32(lo_half ? -INFINITY : x, 0xffffffffu);
+                    if (lane == 0) *reinterpret_cast<float2*>(rw + ((gb + g) * 4 + qd) * 2) = make_float2(lo, hi);
+                }
+                if (bad || *abort_flag) sm_abort[grp] = 1;
+                tc::named_bar_sync(bar_id, 128);
+                if (sm_abort[grp]) break;
+                // new running maxima, one head per lane, and the scales of the warp's two token
+                // blocks: the block maximum of alpha p is 2^(x_b ls - base) for the block's largest
+                // logit x_b, so the scale is the one the block's largest member picks
+                bool rose = false;
+                if (lane < HG) {
+                    const float* w = rw + (gb + lane) * 8;
+                    const float4 w0 = *reinterpret_cast<const float4*>(w);
+                    const float4 w1 = *reinterpret_cast<const float4*>(w + 4);
+                    const float mt = fmaxf(fmaxf(fmaxf(w0.x, w0.y), fmaxf(w0.z, w0.w)),
+                                           fmaxf(fmaxf(w1.x, w1.y), fmaxf(w1.z, w1.w)));
+                    const float mn = fmaxf(m_lane, mt * ls_lane);
+                    const float mz = mn == -INFINITY ? 0.0f : mn;
+                    const float corr = tc::ex2_approx(m_lane - mz);   // 0 on the split's first tile
+                    const float base = mz - la;
+                    rose = mn != m_lane;
+                    m_lane = mn;
+                    const float bm_lo = w[qd * 2], bm_hi = w[qd * 2 + 1];
+                    // per block: NVFP4 {ls, base, corr, 1 / scale}, the element is alpha p / scale;
+                    // MXFP4 {ls, base + e, corr, 2^e} for the scale 2^e, the element is 2^(x ls - base - e)
+                    // (the exponent's argument stays small, as the OCP rule's element) and p its 2^e multiple
+                    float r_lo, r_hi, b_lo = base, b_hi = base;
+                    uint32_t codes;
+                    if constexpr (!MX) {
+                        const float a_lo = tc::ex2_approx(fmaf(bm_lo, ls_lane, -base));
+                        const float a_hi = tc::ex2_approx(fmaf(bm_hi, ls_lane, -base));
+                        codes = tc::e4m3x2_encode(__fmul_rn(a_lo, 1.0f / 6.0f), __fmul_rn(a_hi, 1.0f / 6.0f));
+                        const float2 sg = tc::e4m3x2_value(codes);
+                        // a zero scale zeroes the whole block inside the MMA, whatever the element codes
+                        r_lo = tc::rcp_approx(sg.x);
+                        r_hi = tc::rcp_approx(sg.y);
+                    } else {
+                        // one 32-token block per warp; the OCP MX shared exponent in the log domain:
+                        // the block maximum is 2^d with d = x_b ls - m <= 0, so floor(log2) = floor(d)
+                        // and the element is p 2^(127 - c) for the E8M0 code c
+                        const float d = __fsub_rn(__fmul_rn(fmaxf(bm_lo, bm_hi), ls_lane), mz);
+                        const int c = max(__float2int_rd(fmaxf(d, -256.0f)) + 125, 0);
+                        codes = (uint32_t)c | ((uint32_t)c << 8);
+                        b_lo = b_hi = mz + (float)(c - 127);
+                        r_lo = r_hi = __uint_as_float(c > 0 ? (uint32_t)c << 23 : 0x00400000u);   // 2^(c - 127)
+                    }
+                    wterm[lane * 2 + 0] = make_float4(ls_lane, b_lo, corr, r_lo);
+                    wterm[lane * 2 + 1] = make_float4(ls_lane, b_hi, corr, r_hi);
+                    wcode[lane] = codes;
+                }
+                const uint32_t rmask = j > 0 ? __ballot_sync(0xffffffffu, rose) : 0u;
+                __syncwarp();
+                // O^T rescale of the heads whose maximum rose, once the previous tile's PV has
+                // completed; the group's warps decide alike, having read the same maxima
+                if (rmask) {
+                    if (!tc::mbar_wait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, kWaitLimitMla)) bad = true;
+                    tc::tc_fence_after();
+                    uint32_t rem = rmask;
+                    while (rem) {
+                        // up to four heads per round trip: their columns in the four M tiles
+                        int hs_[4];
+                        uint32_t ov[4][MT];
+    #pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            hs_[k] = rem ? __ffs(rem) - 1 : -1;
+                            if (rem) rem &= rem - 1;
+                            if (hs_[k] >= 0) {
+    #pragma unroll
+                                for (int t = 0; t < MT; ++t) tc::tmem_ld<1>(tq + C::T_O + t * GH + gb + hs_[k], &ov[k][t]);
+                            }
+                        }
+                        tc::tmem_wait_ld();
+    #pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            if (hs_[k] < 0) continue;
+                            const float c = wterm[hs_[k] * 2].z;
+    #pragma unroll
+                            for (int t = 0; t < MT; ++t)
+                                tc::tmem_st1(tq + C::T_O + t * GH + gb + hs_[k], __float_as_uint(__uint_as_float(ov[k][t]) * c));
                         }
                     }
-                    tc::tmem_wait_ld();
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        if (hs_[k] < 0) continue;
-                        const float c = wterm[hs_[k] * 2].z;
-#pragma unroll
-                        for (int t = 0; t < MT; ++t)
-                            tc::tmem_st1(tq + C::T_O + t * GH + gb + hs_[k], __float_as_uint(__uint_as_float(ov[k][t]) * c));
+                    tc::tmem_wait_st();
+                }
+                // probabilities and their FP4 quantization, two heads per conversion
+                uint8_t* const pb = pbyte + (j & 1) * C::P_BUF;
+                uint8_t* const sfb = sfbase + (j & 1) * 2 * 512;
+                const int half = lo_half ? 0 : 1;
+    #pragma unroll
+                for (int g = 0; g < HG; g += 2) {
+                    float q[2];
+    #pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const float4 v = wterm[(g + u) * 2 + half];
+                        const float x = valid ? __uint_as_float(sr[g + u]) : -INFINITY;
+                        const float e = tc::ex2_approx(fmaf(x, v.x, -v.y));   // 0 for masked tokens
+                        const float y = MX ? e * v.w : e;                     // alpha p
+                        l_part[g + u] = fmaf(l_part[g + u], v.z, y);          // l in units of alpha
+                        q[u] = MX ? e : e * v.w;
                     }
+                    const uint32_t mine = e2m1x2_encode(q[0], q[1]);   // head g in bits 0..3, head g + 1 in 4..7
+                    const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
+                    const uint32_t wv = __byte_perm(mine, other, psel) >> (4 * hsel);
+                    const int hr = gb + g + hsel;
+                    pb[(hr >> 3) * 256 + (hr & 7) * 16] = (uint8_t)((wv & 0xfu) | ((wv >> 4) & 0xf0u));
+                    if (sfstore) sfb[(hr & 31) * 16 + (hr >> 5) * 4] = (uint8_t)(wcode[g + hsel] >> (8 * half));
                 }
-                tc::tmem_wait_st();
-            }
-            // probabilities and their FP4 quantization, two heads per conversion
-            uint8_t* const pb = pbyte + (j & 1) * C::P_BUF;
-            uint8_t* const sfb = sfbase + (j & 1) * 2 * 512;
-            const int half = lo_half ? 0 : 1;
-#pragma unroll
-            for (int g = 0; g < HG; g += 2) {
-                float q[2];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const float4 v = wterm[(g + u) * 2 + half];
-                    const float x = valid ? __uint_as_float(sr[g + u]) : -INFINITY;
-                    const float e = tc::ex2_approx(fmaf(x, v.x, -v.y));   // 0 for masked tokens
-                    const float y = MX ? e * v.w : e;                     // alpha p
-                    l_part[g + u] = fmaf(l_part[g + u], v.z, y);          // l in units of alpha
-                    q[u] = MX ? e : e * v.w;
-                }
-                const uint32_t mine = e2m1x2_encode(q[0], q[1]);   // head g in bits 0..3, head g + 1 in 4..7
-                const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
-                const uint32_t wv = __byte_perm(mine, other, psel) >> (4 * hsel);
-                const int hr = gb + g + hsel;
-                pb[(hr >> 3) * 256 + (hr & 7) * 16] = (uint8_t)((wv & 0xfu) | ((wv >> 4) & 0xf0u));
-                if (sfstore) sfb[(hr & 31) * 16 + (hr >> 5) * 4] = (uint8_t)(wcode[g + hsel] >> (8 * half));
-            }
-            // V scale factors (group 0): blocks past the sequence end are zeroed (NVFP4, in the
-            // stage before its TMEM copy) or masked (MXFP4, stored into TMEM by these warps)
-            if (grp == 0) {
-                const int s = j % C::NSV;
-                const bool tail = (tile + 1) * kTileTokens > N;
-                uint8_t* vs = smem + C::SM_VST + s * C::VSTAGE + C::OFF_VS;
-                if constexpr (!MX) {
-                    if (tail) {
+                // V scale factors (group 0): blocks past the sequence end are zeroed (NVFP4, in the
+                // stage before its TMEM copy) or masked (MXFP4, stored into TMEM by these warps)
+                if (grp == 0) {
+                    const int s = j % C::NSV;
+                    const bool tail = (tile + 1) * kTileTokens > N;
+                    uint8_t* vs = smem + C::SM_VST + s * C::VSTAGE + C::OFF_VS;
+                    if constexpr (!MX) {
+                        if (tail || !pok0 || !pok1) {
+                            if (!tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, kWaitLimitMla)) bad = true;
+    #pragma unroll
+                            for (int p = 0; p < 2; ++p) {
+                                const int t0 = tile * kTileTokens + p * kPageSlots;
+                                int nvb = (N - t0 + B - 1) / B;
+                                nvb = nvb < 0 ? 0 : (nvb > C::SPB ? C::SPB : nvb);
+                                if (!(p ? pok1 : pok0)) nvb = 0;
+                                for (int bb = nvb; bb < C::SPB; ++bb)
+    #pragma unroll
+                                    for (int t = 0; t < MT; ++t)
+                                        vs[p * C::VS_PAGE + t * C::VS_TILE + lane * 16 + qd * 4 + bb] = 0;
+                            }
+                        }
+                    } else {
                         if (!tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, kWaitLimitMla)) bad = true;
-#pragma unroll
+                        uint32_t mask[2];
+    #pragma unroll
                         for (int p = 0; p < 2; ++p) {
                             const int t0 = tile * kTileTokens + p * kPageSlots;
                             int nvb = (N - t0 + B - 1) / B;
                             nvb = nvb < 0 ? 0 : (nvb > C::SPB ? C::SPB : nvb);
-                            for (int bb = nvb; bb < C::SPB; ++bb)
-#pragma unroll
-                                for (int t = 0; t < MT; ++t)
-                                    vs[p * C::VS_PAGE + t * C::VS_TILE + lane * 16 + qd * 4 + bb] = 0;
+                            if (!(p ? pok1 : pok0)) nvb = 0;
+                            mask[p] = nvb >= 2 ? 0xffffu : ((1u << (8 * nvb)) - 1u);
                         }
-                    }
-                } else {
-                    if (!tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, kWaitLimitMla)) bad = true;
-                    uint32_t mask[2];
-#pragma unroll
-                    for (int p = 0; p < 2; ++p) {
-                        const int t0 = tile * kTileTokens + p * kPageSlots;
-                        int nvb = (N - t0 + B - 1) / B;
-                        nvb = nvb < 0 ? 0 : (nvb > C::SPB ? C::SPB : nvb);
-                        mask[p] = nvb >= 2 ? 0xffffu : ((1u << (8 * nvb)) - 1u);
-                    }
-#pragma unroll
-                    for (int t = 0; t < MT; ++t) {
-                        uint32_t v[8];
-#pragma unroll
-                        for (int p = 0; p < 2; ++p) {
-                            const uint2 w = *reinterpret_cast<const uint2*>(vs + p * C::VS_PAGE + t * C::VS_TILE + 8 * lane);
-                            v[p * 4 + 0] = w.x & mask[p];
-                            v[p * 4 + 1] = (w.x >> 16) & mask[p];
-                            v[p * 4 + 2] = w.y & mask[p];
-                            v[p * 4 + 3] = (w.y >> 16) & mask[p];
+    #pragma unroll
+                        for (int t = 0; t < MT; ++t) {
+                            uint32_t v[8];
+    #pragma unroll
+                            for (int p = 0; p < 2; ++p) {
+                                const uint2 w = *reinterpret_cast<const uint2*>(vs + p * C::VS_PAGE + t * C::VS_TILE + 8 * lane);
+                                v[p * 4 + 0] = w.x & mask[p];
+                                v[p * 4 + 1] = (w.x >> 16) & mask[p];
+                                v[p * 4 + 2] = w.y & mask[p];
+                                v[p * 4 + 3] = (w.y >> 16) & mask[p];
+                            }
+                            tc::tmem_st8(tq + C::T_SFV + ((j & 1) * MT + t) * 8, v);
                         }
-                        tc::tmem_st8(tq + C::T_SFV + ((j & 1) * MT + t) * 8, v);
+                        tc::tmem_wait_st();
                     }
-                    tc::tmem_wait_st();
                 }
+                tc::tc_fence_before();
+                tc::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&p_ready[j & 1]);
             }
-            tc::tc_fence_before();
-            tc::fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&p_ready[j & 1]);
-        }
+        };
+        if (any_bad_page) tiles(std::true_type{});
+        else tiles(std::false_type{});
         if (!sm_abort[grp]) {
             if (!tc::mbar_wait(&o_done[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag, kWaitLimitMla)) bad = true;
             tc::tc_fence_after();

@@ -21,6 +21,8 @@
 //               each tile's O into registers with the online-softmax rescale.
 // Every wait is bounded; a timeout sets BDFP4_DEV_TIMEOUT and the CTA unwinds.
 
+#include <type_traits>
+
 #include "append_device.cuh"
 #include "bdfp4_device.cuh"
 #include "decode_common.cuh"
@@ -28,9 +30,6 @@
 #include "quant_device.cuh"
 #include "tc_ptx.cuh"
 
-#ifndef BDFP4_TC_MIN_CTAS
-#define BDFP4_TC_MIN_CTAS 3
-#endif
 
 namespace bdfp4 {
 
@@ -41,10 +40,14 @@ struct TcCfg {
     static constexpr int NQ = (2 * G < 8) ? 8 : 2 * G;  // N of the QK MMA (q1 rows, q2 rows, padding)
     static constexpr int NP = (G < 8) ? 8 : G;          // N of the PV MMA
     static constexpr int KS = DK / 64;                   // MMA K steps of QK
+    // CTAs per SM the register budget is shaped for: four for up to four heads
+    // (4 x 10 warps at 48 registers), three for more (3 x 10 warps at 64)
+    static constexpr int MIN_CTAS = G <= 4 ? 4 : 3;
     // two shared-memory rings: K stages are released when QK completes, V stages
-    // when PV completes, so K (needed first) is prefetched further ahead
-    static constexpr int NSK = 4;
-    static constexpr int NSV = 3;
+    // when PV completes, so K (needed first) is prefetched further ahead; with four
+    // CTAs per SM the rings are shallower (the SM holds as many tiles in flight)
+    static constexpr int NSK = MIN_CTAS == 4 ? 3 : 4;
+    static constexpr int NSV = MIN_CTAS == 4 ? 2 : 3;
     // softmax warpgroups: warps w and w + 4 read the same TMEM lanes (tokens), so
     // two groups split the query heads of every tile between them
     static constexpr int NSG = G >= 2 ? 2 : 1;
@@ -52,9 +55,6 @@ struct TcCfg {
     static constexpr int NSW = 4 * NSG;                  // softmax warps
     static constexpr int PRODUCER = NSW, MMA_WARP = NSW + 1;
     static constexpr int THREADS = 32 * (NSW + 2);
-    // CTAs per SM the register budget is shaped for (3 x 10 warps fit in 64 K
-    // registers at 64 per thread)
-    static constexpr int MIN_CTAS = BDFP4_TC_MIN_CTAS;
     static constexpr int K_PAGE = kPageSlots * DK / 2;   // 4096
     static constexpr int NKG = (DK / B + 3) / 4;         // 4-block K scale groups per token (2 / 1)
     static constexpr int KPG = KS / NKG;                 // K steps per scale group (1 NVFP4, 2 MXFP4)
@@ -94,7 +94,8 @@ struct TcCfg {
     static constexpr int SM_BARS = (SM_RED + 2 * RED_BUF * 4 + 7) / 8 * 8;
     static constexpr int NBARS = 2 * NSK + 2 * NSV + 8;
     static constexpr int SM_MISC = SM_BARS + NBARS * 8;                  // tmem slot, abort flags
-    static constexpr int SMEM = SM_MISC + 16;
+    static constexpr int SM_PFLAG = SM_MISC + 16;                        // [64] page flags of the split's tiles, any-bad
+    static constexpr int SMEM = SM_PFLAG + 64 + 16;
     // TMEM column map
     static constexpr int T_S = 0;
     static constexpr int T_O = 2 * NQ;
@@ -460,6 +461,32 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
         const float alpha = (FMT == BDFP4_NVFP4 && !(a.flags & BDFP4_FLAG_NO_UNDERFLOW)) ? kAlphaNV : 1.0f;
         bool bad = false;
 
+        // Pages the block table gets wrong (the producer reports them and copies nothing) are
+        // skipped like tokens past the end: their logits are masked and their V scales zeroed.
+        // Before the first tile the softmax threads note, per tile of the split, whether both
+        // of its pages are good (bit 0: first page, bit 1: second) and whether any is not;
+        // splits longer than 64 tiles look tiles 64 on up in the block table as they go.
+        uint8_t* const pflag = smem + C::SM_PFLAG;
+        volatile int* const pflag_bad = reinterpret_cast<volatile int*>(smem + C::SM_PFLAG + 64);
+        auto page_flags = [&](int jt) -> uint32_t {
+            uint32_t r = 3u;
+#pragma unroll
+            for (int p = 0; p < 2; ++p) {
+                const int pi = (tile0 + jt) * 2 + p;
+                if (pi * kPageSlots < N) {   // pages past the end are masked anyway
+                    const int v = __ldg(a.block_table + (int64_t)b * a.max_pages + pi);
+                    if (v < 0 || v >= a.num_pages) r &= ~(1u << p);
+                }
+            }
+            return r;
+        };
+        if (tid == 0) *pflag_bad = n > 64 ? 1 : 0;
+        tc::named_bar_sync(1 + C::NSG, 32 * C::NSW);
+        if (tid < 64 && tid < n) {
+            const uint32_t f = page_flags(tid);
+            pflag[tid] = (uint8_t)f;
+            if (f != 3u) *pflag_bad = 1;
+        }
         // the query image (QK operand, scale codes, logit scales) of this (sequence, KV head)
         // arrives in one bulk copy from prep_query_kernel, which this grid may overlap:
         // griddepcontrol.wait holds the copy until that grid's writes are visible
@@ -486,7 +513,8 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
         }
         tc::tc_fence_before();
         tc::fence_proxy_async_smem();
-        tc::named_bar_sync(1 + C::NSG, 32 * C::NSW);   // psf zeroed before any tile writes it
+        tc::named_bar_sync(1 + C::NSG, 32 * C::NSW);   // psf zeroed and page flags set before any tile
+        const bool any_bad_page = *pflag_bad != 0;
         if (lane == 0) tc::mbar_arrive(q_ready);
         float m_run[HG], l_part[HG], o_acc[HG], corr_prev[HG];
 #pragma unroll
@@ -531,141 +559,154 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
         uint8_t* const pbyte = p_op + page_of_thread * C::P_PAGE + (qd & 1) * 128 + (lane >> 1) + hsel * 16;
         uint8_t* const sfbyte = psf + page_of_thread * 512 + pos_in_page / B + hsel * 16;
 
-        for (int j = 0; j < n; ++j) {
-            const int buf = j & 1, tile = tile0 + j;
-            // logits of this thread's token for the group's heads (q1 then q2 columns)
-            if (!tc::mbar_wait(&s_full[buf], (j >> 1) & 1, abort_flag, kWaitLimit)) bad = true;
-            tc::tc_fence_after();
-            uint32_t sr[2 * HG];
-            tc::tmem_ld<2 * HG>(tq + C::T_S + buf * C::NQ + 2 * gb, sr);
-            tc::tmem_wait_ld();
-            const int token = tile * kTileTokens + tok_in_tile;
-            // (a page the block table gets wrong is reported through BDFP4_DEV_BAD_PAGE)
-            const bool valid = token < N;
-            // raw logits q1.k + q2.k (the positive factor lsc is applied later, so maxima
-            // commute with it) and their maxima over each half warp (16 consecutive slots)
-            float t[HG], hm_lo[HG], hm_hi[HG];
-#pragma unroll
-            for (int g = 0; g < HG; ++g) {
-                t[g] = valid ? __uint_as_float(sr[g]) + __uint_as_float(sr[HG + g]) : -INFINITY;
-                hm_lo[g] = tc::redux_max_f32(lo_half ? t[g] : -INFINITY, 0xffffffffu);
-                hm_hi[g] = tc::redux_max_f32(lo_half ? -INFINITY : t[g], 0xffffffffu);
-            }
-            float* rw = red + buf * C::RED_BUF;
-            if (lane == 0) {
-#pragma unroll
+        // The tile loop, in two copies: the page checks exist only in the copy a split with a
+        // bad page runs, so the normal copy carries no extra live registers.
+        auto tiles = [&](auto masked) {
+            for (int j = 0; j < n; ++j) {
+                const int buf = j & 1, tile = tile0 + j;
+                bool pok0 = true, pok1 = true;
+                if constexpr (decltype(masked)::value) {
+                    const uint32_t f = j < 64 ? pflag[j] : page_flags(j);
+                    pok0 = (f & 1u) != 0;
+                    pok1 = (f & 2u) != 0;
+                }
+                // logits of this thread's token for the group's heads (q1 then q2 columns)
+                if (!tc::mbar_wait(&s_full[buf], (j >> 1) & 1, abort_flag, kWaitLimit)) bad = true;
+                tc::tc_fence_after();
+                uint32_t sr[2 * HG];
+                tc::tmem_ld<2 * HG>(tq + C::T_S + buf * C::NQ + 2 * gb, sr);
+                tc::tmem_wait_ld();
+                const int token = tile * kTileTokens + tok_in_tile;
+                const bool valid = token < N && (page_of_thread ? pok1 : pok0);
+                // raw logits q1.k + q2.k (the positive factor lsc is applied later, so maxima
+                // commute with it) and their maxima over each half warp (16 consecutive slots)
+                float t[HG], hm_lo[HG], hm_hi[HG];
+    #pragma unroll
                 for (int g = 0; g < HG; ++g) {
-                    rw[(gb + g) * 4 + qd] = fmaxf(hm_lo[g], hm_hi[g]);
+                    t[g] = valid ? __uint_as_float(sr[g]) + __uint_as_float(sr[HG + g]) : -INFINITY;
+                    hm_lo[g] = tc::redux_max_f32(lo_half ? t[g] : -INFINITY, 0xffffffffu);
+                    hm_hi[g] = tc::redux_max_f32(lo_half ? -INFINITY : t[g], 0xffffffffu);
                 }
-            }
-            // one decision for the group's four warps: its flag is written only before this barrier
-            if (bad || *abort_flag) sm_abort[grp] = 1;
-            tc::named_bar_sync(bar_id, 128);
-            if (sm_abort[grp]) break;
-            float y[HG], am[HG], corr[HG];
-            uint32_t mxc[HG];   // MXFP4 block scale codes
-#pragma unroll
-            for (int g = 0; g < HG; ++g) {
-                const float4 w4 = *reinterpret_cast<const float4*>(rw + (gb + g) * 4);
-                const float mt = fmaxf(fmaxf(w4.x, w4.y), fmaxf(w4.z, w4.w));
-                const float mn = fmaxf(m_run[g], mt * lsr[g]);
-                const float mz = mn == -INFINITY ? 0.0f : mn;
-                corr[g] = tc::ex2_approx(m_run[g] - mz);   // 0 on the split's first tile
-                m_run[g] = mn;
-                const float base = mz - la;
-                // the same two instructions give a token's scaled probability and its block's
-                // maximum, so the block scale is the one its largest member picks
-                y[g] = tc::ex2_approx(fmaf(t[g], lsr[g], -base));   // 0 for masked tokens
-                l_part[g] = fmaf(l_part[g], corr[g], y[g]);         // l in units of alpha (cancels at the end)
-                if constexpr (!MX) {
-                    // a 16-token block is this half warp
-                    const float bm = lo_half ? hm_lo[g] : hm_hi[g];
-                    am[g] = tc::ex2_approx(fmaf(bm, lsr[g], -base));
-                } else {
-                    // a 32-token block is this warp.  The OCP MX shared exponent is taken in the
-                    // log domain: the block maximum is 2^d with d = x_b - m, so floor(log2) =
-                    // floor(d) exactly (d = 0 for the tile's largest logit), and the element is
-                    // 2^(x - m - e) for the scale 2^e
-                    const float bm = fmaxf(hm_lo[g], hm_hi[g]);
-                    const float d = __fsub_rn(__fmul_rn(bm, lsr[g]), mz);
-                    const int c = max(__float2int_rd(fmaxf(d, -256.0f)) + 125, 0);
-                    mxc[g] = (uint32_t)c;
-                    am[g] = tc::ex2_approx(fmaf(t[g], lsr[g], -(mz + (float)(c - 127))));
+                float* rw = red + buf * C::RED_BUF;
+                if (lane == 0) {
+    #pragma unroll
+                    for (int g = 0; g < HG; ++g) {
+                        rw[(gb + g) * 4 + qd] = fmaxf(hm_lo[g], hm_hi[g]);
+                    }
                 }
-            }
-            // fused FP4 quantization of the probabilities, two heads per conversion
-            uint8_t* const pb = pbyte + buf * C::P_BUF;
-            uint8_t* const sfb = sfbyte + buf * 2 * 512;
-#pragma unroll
-            for (int g = 0; g < HG; g += 2) {
-                const int g1 = HG >= 2 ? g + 1 : g;
-                uint32_t codes;
-                float q0, q1;
-                if constexpr (FMT == BDFP4_NVFP4) {
-                    codes = tc::e4m3x2_encode(__fmul_rn(am[g], 1.0f / 6.0f), __fmul_rn(am[g1], 1.0f / 6.0f));
-                    const float2 sg = tc::e4m3x2_value(codes);
-                    // a zero scale zeroes the whole block inside the MMA, whatever the element codes
-                    q0 = y[g] * tc::rcp_approx(sg.x);
-                    q1 = y[g1] * tc::rcp_approx(sg.y);
-                } else {
-                    codes = mxc[g] | (mxc[g1] << 8);
-                    q0 = am[g];    // the element already divided by its block scale
-                    q1 = am[g1];
+                // one decision for the group's four warps: its flag is written only before this barrier
+                if (bad || *abort_flag) sm_abort[grp] = 1;
+                tc::named_bar_sync(bar_id, 128);
+                if (sm_abort[grp]) break;
+                float y[HG], am[HG], corr[HG];
+                uint32_t mxc[HG];   // MXFP4 block scale codes
+    #pragma unroll
+                for (int g = 0; g < HG; ++g) {
+                    const float4 w4 = *reinterpret_cast<const float4*>(rw + (gb + g) * 4);
+                    const float mt = fmaxf(fmaxf(w4.x, w4.y), fmaxf(w4.z, w4.w));
+                    const float mn = fmaxf(m_run[g], mt * lsr[g]);
+                    const float mz = mn == -INFINITY ? 0.0f : mn;
+                    corr[g] = tc::ex2_approx(m_run[g] - mz);   // 0 on the split's first tile
+                    m_run[g] = mn;
+                    const float base = mz - la;
+                    // the same two instructions give a token's scaled probability and its block's
+                    // maximum, so the block scale is the one its largest member picks
+                    y[g] = tc::ex2_approx(fmaf(t[g], lsr[g], -base));   // 0 for masked tokens
+                    l_part[g] = fmaf(l_part[g], corr[g], y[g]);         // l in units of alpha (cancels at the end)
+                    if constexpr (!MX) {
+                        // a 16-token block is this half warp
+                        const float bm = lo_half ? hm_lo[g] : hm_hi[g];
+                        am[g] = tc::ex2_approx(fmaf(bm, lsr[g], -base));
+                    } else {
+                        // a 32-token block is this warp.  The OCP MX shared exponent is taken in the
+                        // log domain: the block maximum is 2^d with d = x_b - m, so floor(log2) =
+                        // floor(d) exactly (d = 0 for the tile's largest logit), and the element is
+                        // 2^(x - m - e) for the scale 2^e
+                        const float bm = fmaxf(hm_lo[g], hm_hi[g]);
+                        const float d = __fsub_rn(__fmul_rn(bm, lsr[g]), mz);
+                        const int c = max(__float2int_rd(fmaxf(d, -256.0f)) + 125, 0);
+                        mxc[g] = (uint32_t)c;
+                        am[g] = tc::ex2_approx(fmaf(t[g], lsr[g], -(mz + (float)(c - 127))));
+                    }
                 }
-                const uint32_t mine = e2m1x2_encode(q0, q1);   // head g in bits 0..3, head g1 in 4..7
-                const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
-                const uint32_t w = __byte_perm(mine, other, psel) >> (4 * hsel);
-                const int hr = gb + g;
-                if (pstore) pb[(hr >> 3) * 256 + (hr & 7) * 16] = (uint8_t)((w & 0xfu) | ((w >> 4) & 0xf0u));
-                if (sfstore) sfb[hr * 16] = (uint8_t)(codes >> (8 * hsel));   // SFB rows hr, hr + 1
-            }
-            // V scale factors (group 0): blocks past the sequence end are zeroed, so the
-            // bytes a page holds there are never multiplied.  The V stage can not be
-            // refilled before this tile's PV, so waiting for it here is safe.
-            if (grp == 0) {
-                const int s = j % C::NSV;
-                const bool tail = (tile + 1) * kTileTokens > N;
-                uint8_t* vs = smem + C::SM_VST + s * C::VSTAGE + C::OFF_VS;
-                if constexpr (B == 16) {
-                    if (tail) {
+                // fused FP4 quantization of the probabilities, two heads per conversion
+                uint8_t* const pb = pbyte + buf * C::P_BUF;
+                uint8_t* const sfb = sfbyte + buf * 2 * 512;
+    #pragma unroll
+                for (int g = 0; g < HG; g += 2) {
+                    const int g1 = HG >= 2 ? g + 1 : g;
+                    uint32_t codes;
+                    float q0, q1;
+                    if constexpr (FMT == BDFP4_NVFP4) {
+                        codes = tc::e4m3x2_encode(__fmul_rn(am[g], 1.0f / 6.0f), __fmul_rn(am[g1], 1.0f / 6.0f));
+                        const float2 sg = tc::e4m3x2_value(codes);
+                        // a zero scale zeroes the whole block inside the MMA, whatever the element codes
+                        q0 = y[g] * tc::rcp_approx(sg.x);
+                        q1 = y[g1] * tc::rcp_approx(sg.y);
+                    } else {
+                        codes = mxc[g] | (mxc[g1] << 8);
+                        q0 = am[g];    // the element already divided by its block scale
+                        q1 = am[g1];
+                    }
+                    const uint32_t mine = e2m1x2_encode(q0, q1);   // head g in bits 0..3, head g1 in 4..7
+                    const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
+                    const uint32_t w = __byte_perm(mine, other, psel) >> (4 * hsel);
+                    const int hr = gb + g;
+                    if (pstore) pb[(hr >> 3) * 256 + (hr & 7) * 16] = (uint8_t)((w & 0xfu) | ((w >> 4) & 0xf0u));
+                    if (sfstore) sfb[hr * 16] = (uint8_t)(codes >> (8 * hsel));   // SFB rows hr, hr + 1
+                }
+                // V scale factors (group 0): blocks past the sequence end are zeroed, so the
+                // bytes a page holds there are never multiplied.  The V stage can not be
+                // refilled before this tile's PV, so waiting for it here is safe.
+                if (grp == 0) {
+                    const int s = j % C::NSV;
+                    const bool tail = (tile + 1) * kTileTokens > N;
+                    uint8_t* vs = smem + C::SM_VST + s * C::VSTAGE + C::OFF_VS;
+                    if constexpr (B == 16) {
+                        if (tail || !pok0 || !pok1) {
+                            if (!tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, kWaitLimit)) bad = true;
+    #pragma unroll
+                            for (int p = 0; p < 2; ++p) {
+                                const int t0 = tile * kTileTokens + p * kPageSlots;
+                                int nvb = (N - t0 + B - 1) / B;
+                                nvb = nvb < 0 ? 0 : (nvb > C::SPB ? C::SPB : nvb);
+                                if (!(p ? pok1 : pok0)) nvb = 0;
+                                for (int bb = nvb; bb < C::SPB; ++bb)
+                                    vs[p * C::VS_PAGE + (chan & 31) * 16 + (chan >> 5) * 4 + bb] = 0;
+                            }
+                        }
+                    } else {
                         if (!tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, kWaitLimit)) bad = true;
-#pragma unroll
+                        uint32_t v[8];
+    #pragma unroll
                         for (int p = 0; p < 2; ++p) {
                             const int t0 = tile * kTileTokens + p * kPageSlots;
                             int nvb = (N - t0 + B - 1) / B;
                             nvb = nvb < 0 ? 0 : (nvb > C::SPB ? C::SPB : nvb);
-                            for (int bb = nvb; bb < C::SPB; ++bb)
-                                vs[p * C::VS_PAGE + (chan & 31) * 16 + (chan >> 5) * 4 + bb] = 0;
+                            if (!(p ? pok1 : pok0)) nvb = 0;
+                            const uint32_t mask = nvb >= 2 ? 0xffffu : ((1u << (8 * nvb)) - 1u);
+                            const uint2 w = *reinterpret_cast<const uint2*>(vs + p * C::VS_PAGE + 8 * lane);
+                            v[p * 4 + 0] = w.x & mask;
+                            v[p * 4 + 1] = (w.x >> 16) & mask;
+                            v[p * 4 + 2] = w.y & mask;
+                            v[p * 4 + 3] = (w.y >> 16) & mask;
                         }
+                        tc::tmem_st8(tq + C::T_SFV + buf * 8, v);
+                        tc::tmem_wait_st();
+                        tc::tc_fence_before();
                     }
-                } else {
-                    if (!tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, kWaitLimit)) bad = true;
-                    uint32_t v[8];
-#pragma unroll
-                    for (int p = 0; p < 2; ++p) {
-                        const int t0 = tile * kTileTokens + p * kPageSlots;
-                        int nvb = (N - t0 + B - 1) / B;
-                        nvb = nvb < 0 ? 0 : (nvb > C::SPB ? C::SPB : nvb);
-                        const uint32_t mask = nvb >= 2 ? 0xffffu : ((1u << (8 * nvb)) - 1u);
-                        const uint2 w = *reinterpret_cast<const uint2*>(vs + p * C::VS_PAGE + 8 * lane);
-                        v[p * 4 + 0] = w.x & mask;
-                        v[p * 4 + 1] = (w.x >> 16) & mask;
-                        v[p * 4 + 2] = w.y & mask;
-                        v[p * 4 + 3] = (w.y >> 16) & mask;
-                    }
-                    tc::tmem_st8(tq + C::T_SFV + buf * 8, v);
-                    tc::tmem_wait_st();
-                    tc::tc_fence_before();
                 }
+                tc::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&p_ready[buf]);
+                // fold the previous tile's O into registers
+                if (j >= 1) bad |= !fold_o(j - 1);
+    #pragma unroll
+                for (int g = 0; g < HG; ++g) corr_prev[g] = corr[g];
             }
-            tc::fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&p_ready[buf]);
-            // fold the previous tile's O into registers
-            if (j >= 1) bad |= !fold_o(j - 1);
-#pragma unroll
-            for (int g = 0; g < HG; ++g) corr_prev[g] = corr[g];
-        }
+        };
+        if (any_bad_page) tiles(std::true_type{});
+        else tiles(std::false_type{});
         if (!sm_abort[grp] && !fold_o(n - 1)) bad = true;
         if (bad || *abort_flag) sm_abort[grp] = 1;
 
