@@ -99,7 +99,7 @@ struct TcCfg {
     // TMEM column map
     static constexpr int T_S = 0;
     static constexpr int T_O = 2 * NQ;
-    static constexpr int T_SFK = ((T_O + 2 * NP + 3) / 4) * 4;   // 2 x (4 per K scale group x NKG)
+    static constexpr int T_SFK = ((T_O + NP + 3) / 4) * 4;       // 2 x (4 per K scale group x NKG)
     static constexpr int T_SFV = T_SFK + 2 * 4 * NKG;            // 2 x (4 per page x 2 pages)
     // every scale-factor operand starts on a 4-column boundary (one 32-bit
     // column per 32 rows of a 128-row chunk), B operands included
@@ -230,7 +230,7 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
     uint64_t* vempty = vfull + C::NSV;        // [NSV] PV done -> producer
     uint64_t* s_full = vempty + C::NSV;       // [2] QK done -> softmax
     uint64_t* p_ready = s_full + 2;           // [2] P + scale factors ready -> MMA
-    uint64_t* o_full = p_ready + 2;           // [2] PV done -> softmax
+    uint64_t* o_full = p_ready + 2;           // [2] PV done -> softmax (rescale, epilogue)
     uint64_t* q_ready = o_full + 2;           // query operand and its scale factors -> MMA
     uint64_t* q_full = q_ready + 1;           // query image landed -> softmax
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SM_MISC);
@@ -442,9 +442,12 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                 }
 #pragma unroll
                 for (int p = 0; p < 2; ++p) {
-                    tc::mma_fp4<MX>(tbase + C::T_O + buf * C::NP, tc::smem_desc(vt + p * C::V_PAGE, 128, 256),
+                    // O^T accumulates across the split's tiles (the softmax warps rescale it in
+                    // place when a running maximum rises)
+                    tc::mma_fp4<MX>(tbase + C::T_O, tc::smem_desc(vt + p * C::V_PAGE, 128, 256),
                                     tc::smem_desc(p_addr + buf * C::P_BUF + p * C::P_PAGE, 128, 256), idesc_pv,
-                                    tbase + C::T_SFV + buf * 8 + p * 4, tbase + C::T_SFP + (buf * 2 + p) * 4, p > 0);
+                                    tbase + C::T_SFV + buf * 8 + p * 4, tbase + C::T_SFP + (buf * 2 + p) * 4,
+                                    (j > 0 || p > 0) ? 1u : 0u);
                 }
                 tc::mma_commit(&o_full[buf]);
                 tc::mma_commit(&vempty[s]);
@@ -516,13 +519,11 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
         tc::named_bar_sync(1 + C::NSG, 32 * C::NSW);   // psf zeroed and page flags set before any tile
         const bool any_bad_page = *pflag_bad != 0;
         if (lane == 0) tc::mbar_arrive(q_ready);
-        float m_run[HG], l_part[HG], o_acc[HG], corr_prev[HG];
+        float m_run[HG], l_part[HG];
 #pragma unroll
         for (int g = 0; g < HG; ++g) {
             m_run[g] = -INFINITY;
             l_part[g] = 0.0f;
-            o_acc[g] = 0.0f;
-            corr_prev[g] = 0.0f;
         }
         // TMEM lane 32 qd + lane holds token 32 qd + lane of the tile: slot 32 (qd % 2) + lane
         // of page qd / 2, so a warp owns 32 consecutive slots of one page
@@ -530,16 +531,6 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
         const int pos_in_page = 32 * (qd & 1) + lane;
         const int tok_in_tile = 32 * qd + lane;
         const int chan = 32 * qd + lane;   // O^T lane = value channel
-        auto fold_o = [&](int j) -> bool {
-            if (!tc::mbar_wait(&o_full[j & 1], (j >> 1) & 1, abort_flag, kWaitLimit)) return false;
-            tc::tc_fence_after();
-            uint32_t ov[HG];
-            tc::tmem_ld<HG>(tq + C::T_O + (j & 1) * C::NP + gb, ov);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int g = 0; g < HG; ++g) o_acc[g] = o_acc[g] * corr_prev[g] + __uint_as_float(ov[g]);
-            return true;
-        };
 
         // log2 of alpha: alpha * 2^(x - m) is evaluated as 2^(x - (m - log2 alpha))
         const float la = alpha == kAlphaNV ? 11.0f : 0.0f;
@@ -600,6 +591,7 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                 if (sm_abort[grp]) break;
                 float y[HG], am[HG], corr[HG];
                 uint32_t mxc[HG];   // MXFP4 block scale codes
+                bool rose = false;   // a running maximum of the group rose (alike in its four warps)
     #pragma unroll
                 for (int g = 0; g < HG; ++g) {
                     const float4 w4 = *reinterpret_cast<const float4*>(rw + (gb + g) * 4);
@@ -607,6 +599,7 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                     const float mn = fmaxf(m_run[g], mt * lsr[g]);
                     const float mz = mn == -INFINITY ? 0.0f : mn;
                     corr[g] = tc::ex2_approx(m_run[g] - mz);   // 0 on the split's first tile
+                    rose |= mn != m_run[g];
                     m_run[g] = mn;
                     const float base = mz - la;
                     // the same two instructions give a token's scaled probability and its block's
@@ -655,6 +648,20 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                     if (pstore) pb[(hr >> 3) * 256 + (hr & 7) * 16] = (uint8_t)((w & 0xfu) | ((w >> 4) & 0xf0u));
                     if (sfstore) sfb[hr * 16] = (uint8_t)(codes >> (8 * hsel));   // SFB rows hr, hr + 1
                 }
+                // O^T rescale of the group's heads once the previous tile's PV has completed,
+                // before this tile's PV is issued (the online-softmax update, in TMEM)
+                if (j > 0 && rose) {
+                    if (!tc::mbar_wait(&o_full[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, kWaitLimit)) bad = true;
+                    tc::tc_fence_after();
+                    uint32_t ov[HG];
+                    tc::tmem_ld<HG>(tq + C::T_O + gb, ov);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int g = 0; g < HG; ++g) ov[g] = __float_as_uint(__uint_as_float(ov[g]) * corr[g]);
+                    tc::tmem_st_n<HG>(tq + C::T_O + gb, ov);
+                    tc::tmem_wait_st();
+                    tc::tc_fence_before();
+                }
                 // V scale factors (group 0): blocks past the sequence end are zeroed, so the
                 // bytes a page holds there are never multiplied.  The V stage can not be
                 // refilled before this tile's PV, so waiting for it here is safe.
@@ -699,15 +706,20 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                 tc::fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&p_ready[buf]);
-                // fold the previous tile's O into registers
-                if (j >= 1) bad |= !fold_o(j - 1);
-    #pragma unroll
-                for (int g = 0; g < HG; ++g) corr_prev[g] = corr[g];
             }
         };
         if (any_bad_page) tiles(std::true_type{});
         else tiles(std::false_type{});
-        if (!sm_abort[grp] && !fold_o(n - 1)) bad = true;
+        // the split's O^T once its last PV has completed
+        uint32_t o_fin[HG];
+#pragma unroll
+        for (int g = 0; g < HG; ++g) o_fin[g] = 0u;
+        if (!sm_abort[grp]) {
+            if (!tc::mbar_wait(&o_full[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag, kWaitLimit)) bad = true;
+            tc::tc_fence_after();
+            tc::tmem_ld<HG>(tq + C::T_O + gb, o_fin);
+            tc::tmem_wait_ld();
+        }
         if (bad || *abort_flag) sm_abort[grp] = 1;
 
         // ------------------------------------------------------------ epilogue (thread = channel)
@@ -732,9 +744,10 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                 const float l = rl[hh * 8] + rl[hh * 8 + 1] + rl[hh * 8 + 2] + rl[hh * 8 + 3];
                 const int64_t row = (int64_t)b * a.H_q + h0 + hh;
                 if (nspl == 1) {
-                    a.out[row * C::DV + ch] = __float2bfloat16(l > 0.0f ? o_acc[g] * oscale / l : 0.0f);
+                    a.out[row * C::DV + ch] =
+                        __float2bfloat16(l > 0.0f ? __uint_as_float(o_fin[g]) * oscale / l : 0.0f);
                 } else {
-                    a.ws_o[(row * a.max_splits + split) * C::DV + ch] = o_acc[g] * oscale;
+                    a.ws_o[(row * a.max_splits + split) * C::DV + ch] = __uint_as_float(o_fin[g]) * oscale;
                     if (chan == 0) {
                         a.ws_ml[(row * a.max_splits + split) * 2 + 0] = m_run[g];
                         a.ws_ml[(row * a.max_splits + split) * 2 + 1] = l;

@@ -161,6 +161,16 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* v) {
         : "memory");
 }
 
+// 32 lanes x N columns of 32 bits from registers (N = 1, 2, 4, 8 or 16).
+template <int N>
+__device__ __forceinline__ void tmem_st_n(uint32_t taddr, const uint32_t* v) {
+    if constexpr (N == 1) tmem_st1(taddr, v[0]);
+    else if constexpr (N == 2) tmem_st2(taddr, v[0], v[1]);
+    else if constexpr (N == 4) tmem_st4(taddr, v[0], v[1], v[2], v[3]);
+    else if constexpr (N == 8) tmem_st8(taddr, v);
+    else tmem_st16(taddr, v);
+}
+
 // ------------------------------------------------------------------ MMA
 // Shared-memory matrix descriptor, K-major, no swizzle: 8-row x 16-byte core
 // blocks; lbo = byte distance between the two 16-byte K chunks of one MMA K
