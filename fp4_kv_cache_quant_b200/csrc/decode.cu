@@ -320,15 +320,9 @@ extern "C" size_t bdfp4_decode_workspace_size(int B, int H_q, int d_v, int max_p
 
 extern "C" int bdfp4_decode_plan(const int32_t* host_seq_lens, int B, int H_kv, int num_sms) {
     if (!host_seq_lens || B <= 0 || H_kv <= 0 || num_sms <= 0) return BDFP4_ERR_ARG;
-    int64_t total_tiles = 0;
-    int max_tiles = 1;
-    for (int b = 0; b < B; ++b) {
-        const int n = host_seq_lens[b] > 0 ? host_seq_lens[b] : 0;
-        const int t = (n + kTileTokens - 1) / kTileTokens;
-        total_tiles += (int64_t)t * H_kv;
-        max_tiles = std::max(max_tiles, t);
-    }
-    return plan_chunk_tiles(total_tiles, max_tiles, num_sms);
+    return plan_chunk_tiles(
+        B, [&](int b) { return ((host_seq_lens[b] > 0 ? host_seq_lens[b] : 0) + kTileTokens - 1) / kTileTokens; },
+        H_kv, num_sms);
 }
 
 // The split merge after a decode grid (nothing when no sequence can split).
@@ -402,8 +396,7 @@ static int run_decode(const void* q, const void* k_pages, const void* k_scales, 
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return BDFP4_ERR_CUDA;
         const int ntiles = (max_pages_per_seq * kPageSlots + kTileTokens - 1) / kTileTokens;
-        const int64_t total = (int64_t)B * H_kv * ntiles;
-        chunk_tiles = plan_chunk_tiles(total, ntiles, sms);
+        chunk_tiles = plan_chunk_tiles(B, [&](int) { return ntiles; }, H_kv, sms);
     }
     DecodeArgs a{};
     a.max_splits = max_splits_for(max_pages_per_seq, chunk_tiles);
@@ -519,8 +512,7 @@ extern "C" int bdfp4_decode_noalloc(const void* q, const void* k_pages, const vo
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return BDFP4_ERR_CUDA;
         const int ntiles = (max_pages_per_seq * kPageSlots + kTileTokens - 1) / kTileTokens;
-        const int64_t total = (int64_t)B * (H_kv > 0 ? H_kv : 1) * ntiles;
-        chunk_tiles = plan_chunk_tiles(total, ntiles, sms);
+        chunk_tiles = plan_chunk_tiles(B, [&](int) { return ntiles; }, (H_kv > 0 ? H_kv : 1), sms);
     }
     if (bdfp4_decode_workspace_size(B, H_q, d_v, max_pages_per_seq, chunk_tiles) > BDFP4_NOALLOC_SCRATCH_BYTES)
         return BDFP4_ERR_WORKSPACE;

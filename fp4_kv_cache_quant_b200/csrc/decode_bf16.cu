@@ -480,8 +480,7 @@ extern "C" int bdfp4_bf16_decode(const void* q, const void* k_pages, const void*
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return BDFP4_ERR_CUDA;
         const int ntiles = (max_pages_per_seq * kPageSlots + kTileTokens - 1) / kTileTokens;
-        const int64_t total = (int64_t)B * H_kv * ntiles;
-        chunk_tiles = plan_chunk_tiles(total, ntiles, sms);
+        chunk_tiles = plan_chunk_tiles(B, [&](int) { return ntiles; }, H_kv, sms);
     }
     Bf16Args a{};
     const int ntiles_max = (max_pages_per_seq * kPageSlots + kTileTokens - 1) / kTileTokens;

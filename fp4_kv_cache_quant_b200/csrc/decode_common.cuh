@@ -52,16 +52,32 @@ __host__ __device__ __forceinline__ int num_splits(int N, int chunk_tiles) {
     return (ntiles + chunk_tiles - 1) / chunk_tiles;
 }
 
-// Tiles per split for total_tiles work tiles (all sequences x KV heads) on
-// num_sms SMs: about 12 CTAs' worth of tiles per SM, kept within [16, 40] tiles
-// (shorter splits repeat per-CTA setup and merge traffic; longer ones leave a
-// ragged tail on variable-length batches), at most the longest sequence.
-inline int plan_chunk_tiles(int64_t total_tiles, int max_tiles, int num_sms) {
-    const int64_t per = 12LL * (num_sms > 0 ? num_sms : 1);
-    int64_t chunk = (total_tiles + per - 1) / per;
-    chunk = chunk < 16 ? 16 : (chunk > 40 ? 40 : chunk);
-    if (chunk > max_tiles) chunk = max_tiles;
-    return chunk < 1 ? 1 : (int)chunk;
+// Tiles per split.  Each split of c tiles is one CTA; at four CTAs per SM the grid
+// runs in ceil(CTAs / (4 num_sms)) waves of about c + 3 tile-times (the 3: a CTA's
+// set-up, its partial write and the merge work it adds).  The plan takes the c in
+// [16, 64] -- at most the longest sequence's tile count -- that minimises that
+// product, the longer c on a tie (fewer partials); tiles_of(b) is sequence b's tile
+// count, every sequence has H_kv KV heads.  Sweeps on the GQA shapes put this pick
+// at or next to the fastest measured split length.
+template <class TilesOf>
+inline int plan_chunk_tiles(int B, const TilesOf& tiles_of, int H_kv, int num_sms) {
+    int max_tiles = 0;
+    for (int b = 0; b < B; ++b) max_tiles = tiles_of(b) > max_tiles ? tiles_of(b) : max_tiles;
+    if (max_tiles <= 16) return max_tiles < 1 ? 1 : max_tiles;
+    const int64_t slots = 4LL * (num_sms > 0 ? num_sms : 1);
+    int best = 16;
+    int64_t best_cost = -1;
+    for (int c = 16; c <= 64 && c <= max_tiles; ++c) {
+        int64_t ctas = 0;
+        for (int b = 0; b < B; ++b) ctas += (tiles_of(b) + c - 1) / c;
+        ctas *= H_kv;
+        const int64_t cost = (ctas + slots - 1) / slots * (c + 3);
+        if (best_cost < 0 || cost <= best_cost) {
+            best_cost = cost;
+            best = c;
+        }
+    }
+    return best;
 }
 
 // tcgen05 decode for d_k = d_v = 128 (decode_tc.cu); returns a host status.

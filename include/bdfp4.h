@@ -168,9 +168,10 @@ BDFP4_API int bdfp4_quantize_q(const void* q, int B, int H_q, int H_kv, int d_k,
                      void* stream);
 
 /*
- * Split plan for bdfp4_decode: tiles (128 tokens) per split, about twelve
- * (sequence, KV head, split) work items per SM, each of 16 to 40 tiles (at most
- * the longest sequence's tiles).
+ * Split plan for bdfp4_decode: tiles (128 tokens) per split.  Each split is
+ * one CTA; at four CTAs per SM a grid runs in ceil(CTAs / (4 num_sms)) waves of
+ * about c + 3 tile-times.  The plan is the c in [16, 64] (at most the longest
+ * sequence's tiles) minimising that product, the longer c on ties.
  * host_seq_lens [B] is a HOST array.  Returns chunk_tiles >= 1, or a negative
  * status.  Sequence b then has ceil(ceil(N_b / 128) / chunk_tiles) splits.
  */

@@ -44,17 +44,19 @@ def test_status_strings(lib):
 
 
 def test_decode_plan_host_logic(lib):
-    # 16 sequences of 32768 tokens, 8 KV heads, 148 SMs: 256 tiles each, 32768
-    # work tiles -> ceil(32768 / (12 * 148)) = 19 tiles per split
-    assert bdfp4.bdfp4_decode_plan(np.full(16, 32768), 8, 148) == 19
-    # at least 16 tiles per split, at most the longest sequence
+    # the split length c in [16, 64] (at most the longest sequence) minimising
+    # ceil(CTAs / (4 * SMs)) * (c + 3), CTAs = KV heads * sum over sequences of ceil(tiles / c)
+    # 16 sequences of 32768 tokens (256 tiles), 8 KV heads, 148 SMs: c = 29 gives 9 splits per
+    # sequence, 1152 CTAs = 2 waves of 592 -> 2 * 32 = 64, the least over 16 .. 64
+    assert bdfp4.bdfp4_decode_plan(np.full(16, 32768), 8, 148) == 29
+    # at most the longest sequence; one wave of 3 CTAs at c = 16 beats longer splits
     assert bdfp4.bdfp4_decode_plan(np.array([1000]), 1, 148) == 8
     assert bdfp4.bdfp4_decode_plan(np.array([5000]), 1, 148) == 16
     assert bdfp4.bdfp4_decode_plan(np.array([100]), 1, 148) == 1
-    # 64 sequences of 131072 tokens x 4 heads = 262144 tiles -> 148 per SM-slot, at most 40
-    assert bdfp4.bdfp4_decode_plan(np.full(64, 131072), 4, 148) == 40
-    # 16 x 65536 tokens x 8 heads = 65536 tiles -> ceil(65536 / 1776) = 37
-    assert bdfp4.bdfp4_decode_plan(np.full(16, 65536), 8, 148) == 37
+    # 64 x 131072 tokens x 4 heads: 1024 tiles each; c = 64 -> 4096 CTAs = 7 waves * 67 = 469
+    assert bdfp4.bdfp4_decode_plan(np.full(64, 131072), 4, 148) == 64
+    # 16 x 65536 tokens x 8 heads: 512 tiles each; c = 57 -> 10 splits, 1280 CTAs = 3 waves * 60
+    assert bdfp4.bdfp4_decode_plan(np.full(16, 65536), 8, 148) == 57
     assert bdfp4.bdfp4_decode_plan(np.array([0, 0]), 2, 148) == 1
     with pytest.raises(bdfp4.BDFP4Error):
         bdfp4.bdfp4_decode_plan(np.array([10]), 0, 148)
