@@ -179,7 +179,7 @@ def setup_ours(sp, fmt, rank, device, with_bf16: bool = False):
     bt = torch.from_numpy(wl.block_table).to(device)
     sl = torch.from_numpy(wl.seq_lens).to(device)
     num_sms = torch.cuda.get_device_properties(device).multi_processor_count
-    chunk = bdfp4.bdfp4_decode_plan(wl.seq_lens, sp.H_kv, num_sms)
+    chunk = bdfp4.bdfp4_decode_plan_for(wl.seq_lens, sp.H_q, sp.H_kv, sp.d_k, sp.d_v, num_sms)
     ws = bdfp4.workspace_for(sp.B, sp.H_q, sp.d_v, wl.max_pages, chunk, device=device)
     out = torch.empty((sp.B, sp.H_q, sp.d_v), dtype=torch.bfloat16, device=device)
     return dict(wl=wl, kv=kv, cache=cache, status=status, new_k=new_k, new_v=new_v, v_open=v_open, q=q, bt=bt,

@@ -29,6 +29,7 @@ TILE_TOKENS = 128
 
 #: names of every entry point declared in include/bdfp4.h
 ENTRY_POINTS = ("bdfp4_calibrate", "bdfp4_quantize_kv", "bdfp4_quantize_k", "bdfp4_quantize_v", "bdfp4_quantize_q", "bdfp4_decode_plan",
+                "bdfp4_decode_plan_for",
                 "bdfp4_decode_workspace_size", "bdfp4_decode", "bdfp4_decode_step", "bdfp4_decode_noalloc",
                 "bdfp4_status_string", "bdfp4_last_error")
 #: names of every entry point declared in include/bdfp4_bf16.h
@@ -71,6 +72,8 @@ def load() -> ctypes.CDLL:
     L.bdfp4_quantize_q.restype = i
     L.bdfp4_decode_plan.argtypes = [p, i, i, i]
     L.bdfp4_decode_plan.restype = i
+    L.bdfp4_decode_plan_for.argtypes = [p, i, i, i, i, i, i]
+    L.bdfp4_decode_plan_for.restype = i
     L.bdfp4_decode_workspace_size.argtypes = [i, i, i, i, i]
     L.bdfp4_decode_workspace_size.restype = sz
     L.bdfp4_decode.argtypes = [p, p, p, p, p, p, p, i, i, i, i, i, i, i64, i, i, kvp, f, i, p, sz, p, p, p]
@@ -223,6 +226,15 @@ def bdfp4_decode_plan(host_seq_lens, H_kv: int, num_sms: int) -> int:
     rc = load().bdfp4_decode_plan(ctypes.c_void_p(sl.ctypes.data), sl.shape[0], H_kv, num_sms)
     if rc < 0:
         _check(rc, "bdfp4_decode_plan")
+    return rc
+
+
+def bdfp4_decode_plan_for(host_seq_lens, H_q: int, H_kv: int, d_k: int, d_v: int, num_sms: int) -> int:
+    import numpy as np
+    sl = np.ascontiguousarray(host_seq_lens, dtype=np.int32)
+    rc = load().bdfp4_decode_plan_for(ctypes.c_void_p(sl.ctypes.data), sl.shape[0], H_q, H_kv, d_k, d_v, num_sms)
+    if rc < 0:
+        _check(rc, "bdfp4_decode_plan_for")
     return rc
 
 

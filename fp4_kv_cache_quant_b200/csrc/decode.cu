@@ -318,11 +318,23 @@ extern "C" size_t bdfp4_decode_workspace_size(int B, int H_q, int d_v, int max_p
     return workspace_map(B, H_q, d_v, max_splits_for(max_pages_per_seq, chunk_tiles)).total;
 }
 
+static int host_tiles(const int32_t* host_seq_lens, int b) {
+    return ((host_seq_lens[b] > 0 ? host_seq_lens[b] : 0) + kTileTokens - 1) / kTileTokens;
+}
+
 extern "C" int bdfp4_decode_plan(const int32_t* host_seq_lens, int B, int H_kv, int num_sms) {
     if (!host_seq_lens || B <= 0 || H_kv <= 0 || num_sms <= 0) return BDFP4_ERR_ARG;
-    return plan_chunk_tiles(
-        B, [&](int b) { return ((host_seq_lens[b] > 0 ? host_seq_lens[b] : 0) + kTileTokens - 1) / kTileTokens; },
-        H_kv, num_sms);
+    return plan_chunk_tiles(B, [&](int b) { return host_tiles(host_seq_lens, b); }, H_kv, num_sms, 4);
+}
+
+extern "C" int bdfp4_decode_plan_for(const int32_t* host_seq_lens, int B, int H_q, int H_kv, int d_k, int d_v,
+                                     int num_sms) {
+    if (!host_seq_lens || B <= 0 || H_q <= 0 || H_kv <= 0 || num_sms <= 0) return BDFP4_ERR_ARG;
+    if (H_q % H_kv) return BDFP4_ERR_SHAPE;
+    if (!supported_dims(d_k, d_v)) return BDFP4_ERR_UNSUPPORTED;
+    const DecodeShape ks = decode_shape(d_k, d_v, H_q / H_kv);
+    return plan_chunk_tiles(B, [&](int b) { return host_tiles(host_seq_lens, b); }, H_kv * ks.items_per_kv_head,
+                            num_sms, ks.ctas_per_sm);
 }
 
 // The split merge after a decode grid (nothing when no sequence can split).
@@ -396,7 +408,9 @@ static int run_decode(const void* q, const void* k_pages, const void* k_scales, 
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return BDFP4_ERR_CUDA;
         const int ntiles = (max_pages_per_seq * kPageSlots + kTileTokens - 1) / kTileTokens;
-        chunk_tiles = plan_chunk_tiles(B, [&](int) { return ntiles; }, H_kv, sms);
+        const DecodeShape ks = decode_shape(d_k, d_v, G);
+        chunk_tiles = plan_chunk_tiles(B, [&](int) { return ntiles; }, H_kv * ks.items_per_kv_head, sms,
+                                       ks.ctas_per_sm);
     }
     DecodeArgs a{};
     a.max_splits = max_splits_for(max_pages_per_seq, chunk_tiles);
@@ -512,7 +526,9 @@ extern "C" int bdfp4_decode_noalloc(const void* q, const void* k_pages, const vo
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return BDFP4_ERR_CUDA;
         const int ntiles = (max_pages_per_seq * kPageSlots + kTileTokens - 1) / kTileTokens;
-        chunk_tiles = plan_chunk_tiles(B, [&](int) { return ntiles; }, (H_kv > 0 ? H_kv : 1), sms);
+        const DecodeShape ks = decode_shape(d_k, d_v, H_kv > 0 && H_q % H_kv == 0 ? H_q / H_kv : 1);
+        chunk_tiles = plan_chunk_tiles(B, [&](int) { return ntiles; }, (H_kv > 0 ? H_kv : 1) * ks.items_per_kv_head,
+                                       sms, ks.ctas_per_sm);
     }
     if (bdfp4_decode_workspace_size(B, H_q, d_v, max_pages_per_seq, chunk_tiles) > BDFP4_NOALLOC_SCRATCH_BYTES)
         return BDFP4_ERR_WORKSPACE;

@@ -480,7 +480,7 @@ extern "C" int bdfp4_bf16_decode(const void* q, const void* k_pages, const void*
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return BDFP4_ERR_CUDA;
         const int ntiles = (max_pages_per_seq * kPageSlots + kTileTokens - 1) / kTileTokens;
-        chunk_tiles = plan_chunk_tiles(B, [&](int) { return ntiles; }, H_kv, sms);
+        chunk_tiles = plan_chunk_tiles(B, [&](int) { return ntiles; }, H_kv, sms, 1);   // one CTA per SM
     }
     Bf16Args a{};
     const int ntiles_max = (max_pages_per_seq * kPageSlots + kTileTokens - 1) / kTileTokens;

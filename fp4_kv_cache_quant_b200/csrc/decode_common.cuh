@@ -52,25 +52,26 @@ __host__ __device__ __forceinline__ int num_splits(int N, int chunk_tiles) {
     return (ntiles + chunk_tiles - 1) / chunk_tiles;
 }
 
-// Tiles per split.  Each split of c tiles is one CTA; at four CTAs per SM the grid
-// runs in ceil(CTAs / (4 num_sms)) waves of about c + 3 tile-times (the 3: a CTA's
-// set-up, its partial write and the merge work it adds).  The plan takes the c in
-// [16, 64] -- at most the longest sequence's tile count -- that minimises that
+// Tiles per split.  Each split of c tiles of a sequence is `items` CTAs (one per
+// KV head and head slice); at ctas_per_sm resident CTAs per SM the grid runs in
+// ceil(CTAs / (ctas_per_sm num_sms)) waves of about c + 3 tile-times (the 3: a
+// CTA's set-up, its partial write and the merge work it adds).  The plan takes the
+// c in [16, 64] -- at most the longest sequence's tile count -- that minimises that
 // product, the longer c on a tie (fewer partials); tiles_of(b) is sequence b's tile
-// count, every sequence has H_kv KV heads.  Sweeps on the GQA shapes put this pick
-// at or next to the fastest measured split length.
+// count.  Sweeps on the GQA and MLA shapes put this pick at or next to the fastest
+// measured split length.
 template <class TilesOf>
-inline int plan_chunk_tiles(int B, const TilesOf& tiles_of, int H_kv, int num_sms) {
+inline int plan_chunk_tiles(int B, const TilesOf& tiles_of, int items, int num_sms, int ctas_per_sm) {
     int max_tiles = 0;
     for (int b = 0; b < B; ++b) max_tiles = tiles_of(b) > max_tiles ? tiles_of(b) : max_tiles;
     if (max_tiles <= 16) return max_tiles < 1 ? 1 : max_tiles;
-    const int64_t slots = 4LL * (num_sms > 0 ? num_sms : 1);
+    const int64_t slots = (int64_t)(ctas_per_sm > 0 ? ctas_per_sm : 1) * (num_sms > 0 ? num_sms : 1);
     int best = 16;
     int64_t best_cost = -1;
     for (int c = 16; c <= 64 && c <= max_tiles; ++c) {
         int64_t ctas = 0;
         for (int b = 0; b < B; ++b) ctas += (tiles_of(b) + c - 1) / c;
-        ctas *= H_kv;
+        ctas *= items;
         const int64_t cost = (ctas + slots - 1) / slots * (c + 3);
         if (best_cost < 0 || cost <= best_cost) {
             best_cost = cost;
@@ -78,6 +79,18 @@ inline int plan_chunk_tiles(int B, const TilesOf& tiles_of, int H_kv, int num_sm
         }
     }
     return best;
+}
+
+// CTAs per SM and CTAs per (sequence, split, KV head) of the decode kernel that
+// bdfp4_decode runs for this shape.
+struct DecodeShape {
+    int ctas_per_sm, items_per_kv_head;
+};
+inline DecodeShape decode_shape(int d_k, int d_v, int G) {
+    if (d_k == 128 && d_v == 128 && G <= 16) return {G <= 4 ? 4 : 3, 1};              // decode_tc.cu
+    if (d_k == 576 && d_v == 512 && (G == 16 || G == 32 || G == 64 || G == 128))
+        return {1, G > 64 ? G / 64 : 1};                                                  // decode_mla_tc.cu
+    return {8, G >= 16 ? G / 16 : 1};                                                     // CUDA-core decode
 }
 
 // tcgen05 decode for d_k = d_v = 128 (decode_tc.cu); returns a host status.

@@ -177,6 +177,18 @@ BDFP4_API int bdfp4_quantize_q(const void* q, int B, int H_q, int H_kv, int d_k,
  */
 BDFP4_API int bdfp4_decode_plan(const int32_t* host_seq_lens, int B, int H_kv, int num_sms);
 
+/*
+ * The same plan for the kernel bdfp4_decode runs on this shape (H_q query heads,
+ * head dims d_k / d_v): its CTAs per SM (4 for d = 128 with up to four query
+ * heads per KV head, 3 up to sixteen, 1 for the MLA tensor-core kernel) and its
+ * CTAs per split (one per KV head, times the 64-head slices of the MLA kernel).
+ * bdfp4_decode_plan is this with four CTAs per SM and one CTA per KV head.
+ * Returns chunk_tiles >= 1, or a negative status (BDFP4_ERR_SHAPE if H_q is not a
+ * multiple of H_kv, BDFP4_ERR_UNSUPPORTED for head dims outside the compiled set).
+ */
+BDFP4_API int bdfp4_decode_plan_for(const int32_t* host_seq_lens, int B, int H_q, int H_kv, int d_k, int d_v,
+                                    int num_sms);
+
 /* Bytes of workspace bdfp4_decode needs for this shape and chunk_tiles: the
  * fp32 partial outputs and (m, l) pairs of the splits (when a sequence can
  * have more than one), then 656 bytes per query head for the query images the

@@ -58,6 +58,21 @@ def test_decode_plan_host_logic(lib):
     # 16 x 65536 tokens x 8 heads: 512 tiles each; c = 57 -> 10 splits, 1280 CTAs = 3 waves * 60
     assert bdfp4.bdfp4_decode_plan(np.full(16, 65536), 8, 148) == 57
     assert bdfp4.bdfp4_decode_plan(np.array([0, 0]), 2, 148) == 1
+
+
+def test_decode_plan_for_kernel_shapes(lib):
+    # d = 128 with four query heads per KV head: four CTAs per SM, as bdfp4_decode_plan
+    assert bdfp4.bdfp4_decode_plan_for(np.full(16, 32768), 32, 8, 128, 128, 148) == 29
+    # eight heads per KV head: three CTAs per SM; 16 x 512 tiles x 8 heads: c = 52 -> 10 splits,
+    # 1280 CTAs = 3 waves of 444 -> 3 * 55 = 165, the least over 16 .. 64
+    assert bdfp4.bdfp4_decode_plan_for(np.full(16, 65536), 64, 8, 128, 128, 148) == 52
+    # MLA, 128 heads over one latent head: two 64-head slices per split, one CTA per SM;
+    # 32 x 128 tiles: c = 64 -> 128 CTAs in one wave of 148 -> 67
+    assert bdfp4.bdfp4_decode_plan_for(np.full(32, 16384), 128, 1, 576, 512, 148) == 64
+    with pytest.raises(bdfp4.BDFP4Error):
+        bdfp4.bdfp4_decode_plan_for(np.array([10]), 6, 4, 128, 128, 148)   # 6 query heads over 4 KV heads
+    with pytest.raises(bdfp4.BDFP4Error):
+        bdfp4.bdfp4_decode_plan_for(np.array([10]), 4, 4, 64, 64, 148)     # head dims outside the set
     with pytest.raises(bdfp4.BDFP4Error):
         bdfp4.bdfp4_decode_plan(np.array([10]), 0, 148)
 
