@@ -277,6 +277,32 @@ def test_device_status_on_bad_block_table(ora, lib):
     assert status & bdfp4.DEV_BAD_SEQLEN
 
 
+@pytest.mark.parametrize("name", ["ragged_g8_nv", "ragged_g8_mx", "mla32_mx", "mla128_nv"])
+def test_bad_page_leaves_other_sequences_exact(ora, lib, name):
+    """A page id outside the cache in one sequence is reported, that sequence's output
+    stays finite (its page's tokens are skipped), and every other sequence of the batch
+    matches the oracle run on the intact block table, split plan included."""
+    sp, fmt = SMALL[name]
+    wl = Workload(sp, seed=11)
+    smooth, kg, vg = oracle_calibration(ora, wl)
+    gcache, ocache = quantize_both(ora, wl, fmt, smooth, kg, vg)
+    q = wl.queries()
+    chunk = 1   # many splits: the bad page's split and its neighbours all run
+    ref16, _ = ora.decode(q, ocache, wl.block_table, wl.seq_lens, sp.H_kv, sp.d_v, fmt, smooth, kg, vg, sp.sm_scale,
+                          chunk, wl.num_pages)
+    bad_seq = int(np.argmax(wl.seq_lens))
+    bt = wl.block_table.copy()
+    bt[bad_seq, 1] = -7   # the second page of the longest sequence
+    out, status = run_gpu_decode(wl, gcache, q, kv_params_gpu(smooth, kg, vg), chunk, block_table=bt)
+    assert status & bdfp4.DEV_BAD_PAGE
+    got = out_to_np(out)
+    assert np.isfinite(got).all()
+    ref = bf16_to_np(ref16)
+    others = [b for b in range(sp.B) if b != bad_seq]
+    max_abs, rel = compare_outputs(got[others], ref[others])
+    assert max_abs <= MAX_ABS and rel <= REL_L2, (max_abs, rel)
+
+
 def test_quantize_then_decode_end_to_end(ora, lib):
     """GPU quantizer -> GPU decode against oracle quantizer -> oracle decode."""
     sp, fmt = SMALL["ragged_g8_nv"]
