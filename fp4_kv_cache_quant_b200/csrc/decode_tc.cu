@@ -48,6 +48,10 @@ struct TcCfg {
     // CTAs per SM the rings are shallower (the SM holds as many tiles in flight)
     static constexpr int NSK = MIN_CTAS == 4 ? 3 : 4;
     static constexpr int NSV = MIN_CTAS == 4 ? 2 : 3;
+    // tiles the V copies trail the K copies by: one (only PV needs V, and K is needed
+    // first), except for MXFP4 with the three-stage V ring, whose softmax warps also read
+    // each tile's V scales (2% faster on the 30B shape; with two V stages it was slower)
+    static constexpr int VLAG = (FMT == BDFP4_MXFP4 && NSV == 3) ? 0 : 1;
     // softmax warpgroups: warps w and w + 4 read the same TMEM lanes (tokens), so
     // two groups split the query heads of every tile between them
     static constexpr int NSG = G >= 2 ? 2 : 1;
@@ -289,8 +293,8 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
 
     if (warp == C::PRODUCER) {
         // ------------------------------------------------------------ producer
-        // Step k issues the K half of tile k and the V half of tile k - 1, each
-        // into its own ring, so K runs one tile ahead of V.  The warp reads the
+        // Step k issues the K half of tile k and the V half of tile k - VLAG, each
+        // into its own ring, so K runs VLAG tiles ahead of V.  The warp reads the
         // page ids of 32 tiles at once (one tile per lane), so the dependent
         // block-table load is off the per-tile path; lane 0 then waits for free
         // stages, and one lane per bulk copy issues a step's copies together (a
@@ -317,8 +321,10 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                 const int k = j0 + kk;
                 const int pg0 = __shfl_sync(0xffffffffu, pg_l[0], kk);
                 const int pg1 = __shfl_sync(0xffffffffu, pg_l[1], kk);
-                const bool do_k = k < n, do_v = k >= 1;
-                const int ks = k % C::NSK, v = k - 1, vsi = (k + C::NSV - 1) % C::NSV;
+                const int v = k - C::VLAG;   // the tile whose V half this step issues
+                const bool do_k = k < n, do_v = v >= 0 && v < n;
+                const int ks = k % C::NSK, vsi = (v + C::NSV) % C::NSV;
+                const int pv0_ = C::VLAG ? pv0 : pg0, pv1_ = C::VLAG ? pv1 : pg1;
                 // K half: lane 0 claims the stage and posts the byte count; lanes 0-1 bulk-copy
                 // the two K pages and every lane copies, with cp.async, the 8 scale bytes of
                 // slots lane and 32 + lane of each page and scale group into row lane of the
@@ -353,20 +359,20 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                     }
                     tc::cp_async_mbar_arrive_noinc(&kfull[ks]);
                 }
-                // V half of the previous tile: lanes 0-1 copy the V pages, 2-3 their scales
+                // V half of tile v: lanes 0-1 copy the V pages, 2-3 their scales
                 if (do_v) {
                     if (lane == 0) {
                         if (v >= C::NSV && !tc::mbar_wait(&vempty[vsi], ((v / C::NSV) - 1) & 1, abort_flag, kWaitLimit))
                             ok = false;
                         else
-                            tc::mbar_arrive_expect_tx(&vfull[vsi], (pv0 >= 0 ? C::V_PAGE + C::VS_PAGE : 0) +
-                                                                       (pv1 >= 0 ? C::V_PAGE + C::VS_PAGE : 0));
+                            tc::mbar_arrive_expect_tx(&vfull[vsi], (pv0_ >= 0 ? C::V_PAGE + C::VS_PAGE : 0) +
+                                                                       (pv1_ >= 0 ? C::V_PAGE + C::VS_PAGE : 0));
                     }
                     ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (!ok) break;
                     uint8_t* stg = smem + C::SM_VST + vsi * C::VSTAGE;
                     if (lane < 4) {
-                        const int p = lane & 1, pg = p ? pv1 : pv0;
+                        const int p = lane & 1, pg = p ? pv1_ : pv0_;
                         if (pg >= 0) {
                             const int64_t ph = (int64_t)pg * a.H_kv + hk;
                             if (lane < 2)
