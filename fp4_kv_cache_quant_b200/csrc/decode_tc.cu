@@ -3,22 +3,26 @@
 // transposed softmax with fused probability quantization, dual-residual
 // query, underflow-aware probability scaling), for d_k = d_v = 128.
 //
-// One CTA per (sequence, KV head, split); six warps:
-//   warp 4      producer: reads the block table and bulk-copies each 128-token
-//               tile (two pages: K nibbles, K scales, V nibbles, V scales) into
-//               a 4-stage shared-memory ring (mbarrier complete_tx);
-//   warp 5      MMA issuer (one lane) and TMEM owner:
+// One CTA per (sequence, KV head, split), four (up to four heads per KV head)
+// or three per SM; ten warps (six for a single head):
+//   producer    reads the block table and bulk-copies each 128-token tile (two
+//               pages: K nibbles, K scales, V nibbles, V scales) into a K ring
+//               and a V ring (mbarrier complete_tx);
+//   MMA         one lane issues, the warp owns TMEM:
 //                 S^T[token, q-row] = K_tile . [q1; q2]^T   (M = 128 tokens,
 //                 N = 2G stacked query rows, block-scaled E2M1, fp32 in TMEM),
 //                 O^T[chan, head]  += V^T . P^T             (M = 128 channels,
-//                 N = G heads, K = the tile's tokens, one MMA per page);
-//   warps 0..3  softmax: thread t owns token t of the tile (TMEM lane t), so
-//               the softmax is transposed -- per-head maxima are warp
-//               reductions, the FP4 quantization of P (beta-token blocks) is a
-//               shuffle max over the lanes of a block, and the P codes go
+//                 N = G heads, K = the tile's tokens, one MMA per page),
+//               O^T accumulating across the split's tiles;
+//   softmax     two groups of four warps (one for a single head), each group
+//               half of the heads: thread t owns token t of the tile (TMEM lane
+//               t), so the softmax is transposed -- per-head maxima are warp
+//               reductions, the FP4 quantization of P (beta-token blocks) takes
+//               the maximum over the lanes of a block, and the P codes go
 //               straight into the shared-memory operand of the PV MMA.  The
-//               same threads write the block-scale factors into TMEM and fold
-//               each tile's O into registers with the online-softmax rescale.
+//               same threads write the block-scale factors into TMEM and, when
+//               a running maximum rises, rescale their heads' O^T columns in
+//               TMEM between the previous tile's PV and this one's.
 // Every wait is bounded; a timeout sets BDFP4_DEV_TIMEOUT and the CTA unwinds.
 
 #include <type_traits>
