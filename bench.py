@@ -76,6 +76,16 @@ def decode_source_hash(d_k: int = 128) -> str:
     return h.hexdigest()
 
 
+def slowest_rank(times, device):
+    """Each of the per-rank device times (seconds) replaced by its maximum over the
+    process group's ranks: a replica job is as fast as its slowest rank."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(times, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
 class ClockSampler:
     """SM clock and clock-event (throttle) reasons polled through NVML in a
     background thread during the timed region (read-only queries)."""
@@ -333,9 +343,7 @@ def run_ours(args, sp, fmt):
 
     tokens = float(np.sum(wl.seq_lens))
     if world > 1:
-        t = torch.tensor([step_s, dec_s, e2e_s, bf16_s], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_s, dec_s, e2e_s, bf16_s = t.tolist()
+        step_s, dec_s, e2e_s, bf16_s = slowest_rank([step_s, dec_s, e2e_s, bf16_s], device)
         tokens *= world
     # one prologue (append + query images) and the tensor-core decode (d = 128), or the
     # append and one CUDA-core decode; merge when a sequence can split
