@@ -32,6 +32,9 @@ SMALL = {
     "mla128_mx": (spec("mla", B=2, ctx=("list", (300, 130))), MX),
     "mla64_nv": (spec("mla", B=2, H_q=64, ctx=("list", (1000, 77))), NV),
     "mla32_mx": (spec("mla", B=3, H_q=32, ctx=("list", (129, 0, 700))), MX),
+    # shapes the tensor-core kernels do not take run the CUDA-core decode
+    "g32_cuda_nv": (spec("tiny", B=2, H_q=32, H_kv=1, ctx=("list", (300, 77))), NV),
+    "mla8_cuda_mx": (spec("mla", B=2, H_q=8, ctx=("list", (200, 65))), MX),
 }
 
 
@@ -100,7 +103,7 @@ def test_decode_step_append_matches_oracle(ora, lib, name):
 
 @pytest.mark.parametrize("chunk", [0, 1])
 @pytest.mark.parametrize("name", ["tiny_nv", "tiny_mx", "ragged_g8_nv", "ragged_g8_mx", "g16_nv", "mla_nv", "mla_mx",
-                                  "mla128_nv", "mla32_mx"])
+                                  "mla128_nv", "mla32_mx", "g32_cuda_nv", "mla8_cuda_mx"])
 def test_decode_step_matches_oracle(ora, lib, name, chunk):
     """bdfp4_decode_step after a prefill of all but each sequence's newest token:
     the cache must equal the oracle's quantization of every token, the open
