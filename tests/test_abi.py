@@ -161,3 +161,24 @@ def test_output_comparison_counts_one_bf16_step_as_agreement():
     assert compare_outputs(np.array([1.0]), np.array([1.0078125]))[0] == 0.0   # one step at [1, 2)
     assert abs(compare_outputs(np.array([0.5]), np.array([0.52]))[0] - 0.02) < 1e-12
     assert compare_outputs(np.array([3.0]), np.array([3.0]))[1] == 0.0
+
+
+def test_decode_plan_minimises_the_documented_wave_cost(lib):
+    """On random batches the plan is the split length the header's rule names:
+    c in [16, 64] (at most the longest sequence) minimising ceil(CTAs / slots) * (c + 3),
+    the longer c on ties."""
+    rng = np.random.default_rng(5)
+    for _ in range(40):
+        B = int(rng.integers(1, 48))
+        lens = rng.integers(0, 200_000, size=B)
+        H_kv = int(rng.choice([1, 2, 4, 8]))
+        sms = int(rng.choice([132, 148]))
+        tiles = [(int(n) + 127) // 128 for n in lens]
+        got = bdfp4.bdfp4_decode_plan(lens, H_kv, sms)
+        mx = max(tiles)
+        if mx <= 16:
+            assert got == max(mx, 1)
+            continue
+        cost = {c: -(-H_kv * sum(-(-t // c) for t in tiles) // (4 * sms)) * (c + 3) for c in range(16, min(64, mx) + 1)}
+        best = min(cost.values())
+        assert cost[got] == best and got == max(c for c, v in cost.items() if v == best)
