@@ -124,6 +124,27 @@ def test_decode_argument_errors(lib):
     assert call(chunk=1, ws=_p(0x20000), ws_bytes=n - 1) == -6
 
 
+def test_decode_step_and_append_halves_argument_errors(lib):
+    kv = bdfp4._KVParams(0x1000, 0x2000, 0x3000)
+    a = _p(0x10000)
+
+    def step(k_new=a, v_new=a, v_open=a, H_q=8, H_kv=2, d_k=128, d_v=128):
+        return lib.bdfp4_decode_step(a, k_new, v_new, v_open, a, a, a, a, a, a, 2, H_q, H_kv, d_k, d_v, 4, 16, 0, 0,
+                                     ctypes.byref(kv), 0.1, 8, None, 0, a, None, None)
+    assert step(k_new=None) == -1
+    assert step(v_open=None) == -1
+    assert step(v_new=_p(0x10002)) == -3
+    assert step(H_q=7) == -2
+    assert step(d_k=64, d_v=64) == -4
+    # the K and V halves of the append
+    assert lib.bdfp4_quantize_k(a, a, 10, 2, 64, 0, 0, ctypes.byref(kv), a, a, 4, None, None) == -4
+    assert lib.bdfp4_quantize_k(None, a, 10, 2, 128, 0, 0, ctypes.byref(kv), a, a, 4, None, None) == -1
+    assert lib.bdfp4_quantize_k(a, a, 0, 2, 128, 0, 0, ctypes.byref(kv), a, a, 4, None, None) == 0
+    assert lib.bdfp4_quantize_v(a, a, 10, 2, 64, 0, ctypes.byref(kv), a, a, 4, None) == -4
+    assert lib.bdfp4_quantize_v(a, None, 10, 2, 128, 0, ctypes.byref(kv), a, a, 4, None) == -1
+    assert lib.bdfp4_quantize_v(a, a, 10, 2, 128, 3, ctypes.byref(kv), a, a, 4, None) == -1
+
+
 def test_product_code_does_not_touch_the_oracle():
     """The CUDA library and its binding share no code with the oracle."""
     pkg = os.path.join(ROOT, "fp4_kv_cache_quant_b200")
