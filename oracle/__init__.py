@@ -28,6 +28,7 @@ FLAG_NO_SCALE_SEARCH = 2
 FLAG_SINGLE_QUERY = 4
 FLAG_NO_UNDERFLOW = 8
 FLAG_EXACT_P = 16
+FLAG_DYNAMIC_ALPHA = 32
 
 PAGE_SLOTS = 64
 TILE_TOKENS = 128
@@ -86,6 +87,8 @@ def lib():
         L.ora_plain_scale_code.argtypes = [i, f, f]
         L.ora_search_scale_code.restype = i
         L.ora_search_scale_code.argtypes = [i, p, i, f]
+        L.ora_dynamic_alpha_exp.restype = i
+        L.ora_dynamic_alpha_exp.argtypes = [d]
         L.ora_dequant_key_row.restype = None
         L.ora_dequant_key_row.argtypes = [p, p, i, i64, i, i, i, i, p]
         L.ora_dequant_value_row.restype = None
@@ -168,6 +171,11 @@ def plain_scale_code(fmt: int, amax: float, g: float) -> int:
 def search_scale_code(fmt: int, x: np.ndarray, g: float) -> int:
     x = np.ascontiguousarray(x, np.float32)
     return lib().ora_search_scale_code(fmt, _ptr(x), x.shape[0], float(g))
+
+
+def dynamic_alpha_exp(p_max: float) -> int:
+    """Exponent of the per-tile probability pre-scale of the dynamic variant."""
+    return lib().ora_dynamic_alpha_exp(float(p_max))
 
 
 def dequant_key_row(cache: dict, fmt: int, page: int, head: int, H_kv: int, d_k: int, slot: int) -> np.ndarray:

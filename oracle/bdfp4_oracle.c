@@ -56,6 +56,7 @@
 #define ORA_FLAG_NO_UNDERFLOW    8   /* ablation: alpha = 1 (vanilla P scaling)    */
 #define ORA_FLAG_EXACT_P        16   /* oracle only: probabilities left unquantized,
                                         to pin the softmax against textbook attention */
+#define ORA_FLAG_DYNAMIC_ALPHA  32   /* variant: alpha chosen per tile and head     */
 
 #define PAGE_SLOTS 64   /* tokens per KV page                       */
 #define TILE_TOKENS 128 /* tokens per online-softmax step (2 pages) */
@@ -667,6 +668,14 @@ int ora_quantize_q(const uint16_t* q, int B, int H_q, int H_kv, int d_k, int fmt
  *   exactly: scale code c = E4M3(amax_y / 6), code 0 = collapsed block,
  *   e_t = E2M1(y_t / E4M3(c)), P^_t = e_t E4M3(c) / alpha.  Vanilla ablation:
  *   alpha = 1.  MXFP4 (E8M0 scale, no underflow at these magnitudes): alpha = 1.
+ *   Dynamic variant (NVFP4): the pages place the underflow at long contexts,
+ *   where a tile far below the running maximum has only tiny probabilities.
+ *   Reading: per tile and head, alpha = 2^E with E the largest integer such
+ *   that p_max 2^E <= 2688 (= 6 x 448, so the largest block scale still fits
+ *   E4M3), p_max the tile's largest p, E clamped to [11, 64] (64 also for
+ *   p_max = 0); P^ is divided by that tile's alpha, so O needs no other change.
+ *   A tile that raises the running maximum has p_max = 1 and E = 11, the
+ *   static choice.
  *   merge: m* = max m_s, O = sum_s O_s e^(m_s - m*) / sum_s l_s e^(m_s - m*),
  *   rounded to bf16.  An empty sequence gives 0.
  * The probabilities' codes are decided in fp64 here (the GPU decides them in
@@ -709,6 +718,18 @@ void ora_dequant_value_row(const uint8_t* v_pages, const uint8_t* v_scales, int 
     for (int c = 0; c < d_v; ++c) out[c] = deq_value(v_pages, v_scales, fmt, page, head, H_kv, d_v, c, slot);
 }
 
+/* Exponent E of the per-tile alpha = 2^E of the dynamic variant: the largest
+ * integer with p_max 2^E <= 2688, clamped to [11, 64]; every product here is
+ * exact in fp64 (a power-of-two scaling). */
+int ora_dynamic_alpha_exp(double p_max)
+{
+    if (!(p_max > 0.0)) return 64;
+    int E = 11;
+    while (E < 64 && ldexp(p_max, E + 1) <= 2688.0) ++E;
+    while (E > 11 && ldexp(p_max, E) > 2688.0) --E;
+    return E;
+}
+
 /* FP4 quantization of one block of probabilities y (already times alpha),
  * decided in fp64; returns the dequantized values (still times alpha). */
 static void quantize_probs(int fmt, const double* y, int n, double* yq)
@@ -748,6 +769,8 @@ int ora_decode(const uint16_t* q, const uint8_t* k_pages, const uint8_t* k_scale
     int hadamard = !(flags & ORA_FLAG_NO_HADAMARD);
     int dual = !(flags & ORA_FLAG_SINGLE_QUERY);
     double alpha = (fmt == ORA_NVFP4 && !(flags & ORA_FLAG_NO_UNDERFLOW)) ? 2048.0 : 1.0;
+    if ((flags & ORA_FLAG_DYNAMIC_ALPHA) && (flags & ORA_FLAG_NO_UNDERFLOW)) return -1;
+    int dynamic = fmt == ORA_NVFP4 && (flags & ORA_FLAG_DYNAMIC_ALPHA);
 
     /* One (sequence, KV head) at a time; the G query heads of the group each
      * run the steps above.  A tile's keys and values are dequantized once
@@ -825,11 +848,15 @@ int ora_decode(const uint16_t* q, const uint8_t* k_pages, const uint8_t* k_scale
                         }
                         double m_new = m[j] > m_tile ? m[j] : m_tile;
                         double corr = exp(m[j] - m_new);   /* 0 on a split's first tile */
-                        double psum = 0.0;
+                        double psum = 0.0, p_max = 0.0;
                         for (int jt = 0; jt < TILE_TOKENS; ++jt) {
-                            double p = valid[jt] ? exp(s[jt] - m_new) : 0.0;
-                            psum += p;
-                            y[jt] = p * alpha;
+                            y[jt] = valid[jt] ? exp(s[jt] - m_new) : 0.0;
+                            if (y[jt] > p_max) p_max = y[jt];
+                        }
+                        double alpha_t = dynamic ? ldexp(1.0, ora_dynamic_alpha_exp(p_max)) : alpha;
+                        for (int jt = 0; jt < TILE_TOKENS; ++jt) {
+                            psum += y[jt];
+                            y[jt] *= alpha_t;
                         }
                         if (flags & ORA_FLAG_EXACT_P) memcpy(yq, y, sizeof(y));
                         else
@@ -838,7 +865,7 @@ int ora_decode(const uint16_t* q, const uint8_t* k_pages, const uint8_t* k_scale
                         for (int c = 0; c < d_v; ++c) oj[c] *= corr;
                         for (int jt = 0; jt < TILE_TOKENS; ++jt) {
                             if (!valid[jt] || yq[jt] == 0.0) continue;
-                            double w = yq[jt] / alpha;
+                            double w = yq[jt] / alpha_t;
                             for (int c = 0; c < d_v; ++c) oj[c] += w * vt[(size_t)jt * d_v + c];
                         }
                         m[j] = m_new;

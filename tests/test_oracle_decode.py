@@ -139,8 +139,8 @@ def test_uniform_logits_closed_form(ora, fmt, flags, pscale):
         assert np.allclose(o64[0, h], expect, rtol=1e-12, atol=1e-12)
 
 
-def _sink_case(ora, fmt, flags, N=300, chunk=1000):
-    """One key with logit 10, the rest 0: p = 1 and e^-10 per token."""
+def _sink_case(ora, fmt, flags, N=300, chunk=1000, logit=10.0):
+    """One key with logit 10 (or `logit`), the rest 0: p = 1 and e^-10 per token."""
     rng = np.random.default_rng(7)
     H_kv, G, d = 1, 2, 128
     q = np.zeros((1, G, d), np.float32)
@@ -153,7 +153,7 @@ def _sink_case(ora, fmt, flags, N=300, chunk=1000):
     g = np.ones(H_kv, np.float32)
     cache = ora.empty_cache(num_pages, H_kv, d, d, fmt)
     ora.quantize_kv(_bf16(k), _bf16(v), sm, cache, H_kv, fmt, ones, g, g, num_pages, flags=ora.FLAG_NO_HADAMARD)
-    o16, o64 = ora.decode(_bf16(q), cache, bt, np.array([N]), H_kv, d, fmt, ones, g, g, 10.0 / 36.0, chunk,
+    o16, o64 = ora.decode(_bf16(q), cache, bt, np.array([N]), H_kv, d, fmt, ones, g, g, logit / 36.0, chunk,
                           num_pages, flags=ora.FLAG_NO_HADAMARD | flags)
     return o64, v[:, 0].astype(np.float64)
 
@@ -185,6 +185,57 @@ def test_split_kv_quantizes_probabilities_per_split(ora):
     tail = 6 * 2.0 ** -6 / 2048
     expect = (1.03125 * v[0] + tail * v[16:128].sum(0) + 1.03125 * math.exp(-10.0) * v[128:].sum(0)) / l
     assert np.allclose(o[0, 0], expect, rtol=1e-5, atol=1e-9)
+
+
+@pytest.mark.parametrize("p_max,E", [
+    (1.0, 11),                                    # 2688 / 1 = 2^11.39: the static alpha
+    (2688.0 * 2.0 ** -20, 20),                    # p_max 2^20 = 2688 exactly: still allowed
+    (np.nextafter(2688.0 * 2.0 ** -20, 1.0), 19),  # one ulp above: 2^20 p_max > 2688
+    (2.0 ** -20, 31),                             # 2^-20 2^31 = 2048 <= 2688 < 4096
+    (math.exp(-10.0), 25),                        # 2^25 e^-10 = 1523.3, 2^26 e^-10 = 3046.6
+    (math.exp(-20.0), 40),                        # 2^40 e^-20 = 2266.3, 2^41 e^-20 = 4532.6
+    (2.0 ** -100, 64),                            # clamped
+    (0.0, 64),                                    # empty tile
+])
+def test_dynamic_alpha_exponent_hand_values(ora, p_max, E):
+    assert ora.dynamic_alpha_exp(p_max) == E
+
+
+def test_dynamic_alpha_closed_form(ora):
+    """Sink logit 20: with alpha = 2^11 every block without the sink collapses
+    (E4M3(e^-20 2^11 / 6) = 0).  The dynamic variant keeps alpha = 2^11 on the
+    sink's tile (p_max = 1) but takes 2^40 on the two later tiles, whose p_max
+    is e^-20: E4M3(e^-20 2^40 / 6 = 377.7) = 384, E2M1(2266.3 / 384 = 5.90) = 6,
+    so each of their tokens gets P^ = 6 x 384 / 2^40."""
+    N = 300
+    l = 1.0 + (N - 1) * math.exp(-20.0)
+    o_st, v = _sink_case(ora, 0, 0, N, logit=20.0)
+    assert np.allclose(o_st[0, 0], 1.03125 * v[0] / l, rtol=1e-12, atol=1e-15)
+    o_dy, _ = _sink_case(ora, 0, ora.FLAG_DYNAMIC_ALPHA, N, logit=20.0)
+    tail = 6 * 384 * 2.0 ** -40 * v[128:].sum(0) / l
+    assert np.abs(tail).max() > 1e-9
+    # (the difference of two outputs of size ~10 carries ~1e-15 of cancellation)
+    assert np.allclose(o_dy[0, 0] - o_st[0, 0], tail, rtol=1e-9, atol=1e-13)
+    # unquantized P carries the tail as e^-20 per token (the sink's logit holds
+    # the fp32 rounding of g_q, so e^-20 only to ~1e-7, and l with it)
+    o_ex, _ = _sink_case(ora, 0, ora.FLAG_EXACT_P, N, logit=20.0)
+    exact_tail = (o_ex[0, 0] - v[0] / l)
+    assert np.allclose(exact_tail, math.exp(-20.0) * v[1:].sum(0) / l, rtol=1e-5, atol=1e-10)
+
+
+def test_dynamic_alpha_reduces_to_static_alpha(ora):
+    """Every split's first tile has p_max = 1 (alpha = 2^11): with one tile per
+    split the variant is the static method; MXFP4 has no alpha to choose."""
+    for logit in (10.0, 20.0):
+        o_st, _ = _sink_case(ora, 0, 0, 300, chunk=1, logit=logit)
+        o_dy, _ = _sink_case(ora, 0, ora.FLAG_DYNAMIC_ALPHA, 300, chunk=1, logit=logit)
+        assert np.array_equal(o_st, o_dy)
+        o_st, _ = _sink_case(ora, 1, 0, 300, logit=logit)
+        o_dy, _ = _sink_case(ora, 1, ora.FLAG_DYNAMIC_ALPHA, 300, logit=logit)
+        assert np.array_equal(o_st, o_dy)
+    # the variant and the vanilla ablation exclude each other
+    with pytest.raises(AssertionError):
+        _sink_case(ora, 0, ora.FLAG_DYNAMIC_ALPHA | ora.FLAG_NO_UNDERFLOW, 300)
 
 
 def test_quantized_probabilities_stay_close_on_random_data(ora):
