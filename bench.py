@@ -216,15 +216,17 @@ def run_ours(args, sp, fmt):
     wl, kv, cache = S["wl"], S["kv"], S["cache"]
     stream = torch.cuda.current_stream(device)
 
+    flags = bdfp4.FLAG_DYNAMIC_ALPHA if args.dynamic_alpha else 0
+
     def step(q, k_new, v_new, out=None):
         # one call: append each sequence's newest token (key, and the open value
         # block it joins) into the FP4 cache, then decode over the updated cache
         bdfp4.bdfp4_decode_step(q, k_new, v_new, S["v_open"], cache, S["bt"], S["sl"], kv, sp.sm_scale, S["chunk"],
-                                S["ws"], S["out"] if out is None else out, dev_status=S["status"])
+                                S["ws"], S["out"] if out is None else out, flags=flags, dev_status=S["status"])
 
     def decode_only():
         bdfp4.bdfp4_decode(S["q"], cache, S["bt"], S["sl"], kv, sp.sm_scale, S["chunk"], S["ws"], S["out"],
-                           dev_status=S["status"])
+                           flags=flags, dev_status=S["status"])
 
     for _ in range(max(args.warmup, 3)):
         step(S["q"], S["new_k"], S["new_v"])
@@ -356,7 +358,8 @@ def run_ours(args, sp, fmt):
         peak, peak_src = 6650.0, "fallback"
     traffic = None
     tr_path = os.path.join(ROOT, "profiles", "decode_traffic.json")
-    if os.path.exists(tr_path):
+    cuda_core = fmt == 0 and args.dynamic_alpha   # the variant runs on the CUDA-core decode
+    if os.path.exists(tr_path) and not cuda_core:
         rec = json.load(open(tr_path)).get(f"{args.config}_{args.fmt}")
         # the counters describe the kernel as captured: null once its sources changed
         if rec and rec.get("source_sha256") == decode_source_hash(sp.d_k):
@@ -379,15 +382,19 @@ def run_ours(args, sp, fmt):
                    "kv_tokens_per_step_per_gpu": int(tokens / world), "chunk_tiles": S["chunk"],
                    "parallelism": f"replicas x{world} (no data-path collective)",
                    "l2": f"inputs larger than L2 (FP4 cache {cache.nbytes() / 1e6:.0f} MB per GPU)",
-                   "accumulate": "fp32"},
+                   "accumulate": "fp32",
+                   "probability_prescale": "dynamic per tile" if args.dynamic_alpha else "static 2^11"},
         "hbm_gbs": alg / dec_s / 1e9,
         "decode_us": dec_s * 1e6,
         "quantize_prefill_gbs": S["quant_gbs"],
         "roofline": {"bound": "hbm", "achieved": alg / dec_s / 1e9, "peak": peak, "unit": "GB/s",
                      "frac": alg / dec_s / 1e9 / peak, "traffic": traffic,
-                     "kernel": ("bdfp4_decode calls (query images, decode_tc_kernel, merge_splits_kernel): "
-                                "K back-to-back calls right after the step loop, one event pair"
-                                if sp.d_k == 128 else "bdfp4_decode calls (decode_fp4_kernel, merge_splits_kernel)"),
+                     "kernel": ("bdfp4_decode calls (" +
+                                ("decode_fp4_kernel" if cuda_core else
+                                 "prep_query_kernel, decode_tc_kernel" if sp.d_k == 128 else
+                                 "prep_mla_kernel, decode_mla_tc_kernel") +
+                                ", merge_splits_kernel): K back-to-back calls right after the step loop, "
+                                "one event pair"),
                      "peak_source": f"{peak_src} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
                      "algorithmic_bytes_per_launch": alg},
         "e2e": {"value": tokens / e2e_s, "unit": "tokens/s",
@@ -405,7 +412,7 @@ def run_ours(args, sp, fmt):
             "frac": b_alg / bf16_s / 1e9 / peak, "algorithmic_bytes_per_launch": b_alg,
             "fp4_decode_speedup": bf16_s / dec_s}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(sp, fmt, budget_s=args.cpu_budget)
+        result["cpu_baseline"] = cpu_baseline(sp, fmt, budget_s=args.cpu_budget, flags=flags)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -413,7 +420,7 @@ def run_ours(args, sp, fmt):
         print(json.dumps(result), flush=True)
 
 
-def cpu_baseline(sp, fmt, budget_s: float = 15.0, seed: int = 0) -> dict:
+def cpu_baseline(sp, fmt, budget_s: float = 15.0, seed: int = 0, flags: int = 0) -> dict:
     """The oracle as it stands, timed on this host's cores on a bounded sample
     of the same workload: decode (with the tail append) of the first few
     sequences; prefill of the sample is untimed setup."""
@@ -436,7 +443,7 @@ def cpu_baseline(sp, fmt, budget_s: float = 15.0, seed: int = 0) -> dict:
         t0 = time.perf_counter()
         oracle.quantize_kv(k[n - r:], v[n - r:], sm[n - r:], cache, sp.H_kv, fmt, smooth, kg, vg, wl.num_pages)
         oracle.decode(q_all[b:b + 1], cache, wl.block_table[b:b + 1], wl.seq_lens[b:b + 1], sp.H_kv, sp.d_v, fmt,
-                      smooth, kg, vg, sp.sm_scale, 1 << 20, wl.num_pages)
+                      smooth, kg, vg, sp.sm_scale, 1 << 20, wl.num_pages, flags=flags)
         elapsed += time.perf_counter() - t0
         done_tokens += n
         nseq += 1
@@ -467,11 +474,12 @@ def run_reference(args, sp, fmt):
     cache = oracle.empty_cache(wl.num_pages, sp.H_kv, sp.d_k, sp.d_v, fmt)
     oracle.quantize_kv(k, v, sm, cache, sp.H_kv, fmt, smooth, kg, vg, wl.num_pages)
     r = ((n - 1) % beta) + 1
+    flags = oracle.FLAG_DYNAMIC_ALPHA if args.dynamic_alpha else 0
 
     def step():
         oracle.quantize_kv(k[n - r:], v[n - r:], sm[n - r:], cache, sp.H_kv, fmt, smooth, kg, vg, wl.num_pages)
         oracle.decode(q_all[b:b + 1], cache, wl.block_table[b:b + 1], wl.seq_lens[b:b + 1], sp.H_kv, sp.d_v, fmt,
-                      smooth, kg, vg, sp.sm_scale, 1 << 20, wl.num_pages)
+                      smooth, kg, vg, sp.sm_scale, 1 << 20, wl.num_pages, flags=flags)
 
     for _ in range(args.warmup):
         step()
@@ -485,7 +493,8 @@ def run_reference(args, sp, fmt):
         "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": el * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic",
-        "config": {"workload": CONFIG_TEXT[args.config], "name": args.config, "fmt": args.fmt},
+        "config": {"workload": CONFIG_TEXT[args.config], "name": args.config, "fmt": args.fmt,
+                   "probability_prescale": "dynamic per tile" if args.dynamic_alpha else "static 2^11"},
         "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
                          "sample": f"sequence 0 of {sp.B} ({n} KV tokens, all heads) per step: tail append + decode"},
         "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -503,6 +512,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-bf16", action="store_true", help="skip the BF16-KV comparator")
+    ap.add_argument("--dynamic-alpha", action="store_true",
+                    help="the per-tile probability pre-scale variant (NVFP4: CUDA-core decode)")
     args = ap.parse_args()
     from fp4_kv_cache_quant_b200.workloads import spec
     sp = spec(args.config)

@@ -21,6 +21,7 @@ FLAG_NO_HADAMARD = 1
 FLAG_NO_SCALE_SEARCH = 2
 FLAG_SINGLE_QUERY = 4
 FLAG_NO_UNDERFLOW = 8
+FLAG_DYNAMIC_ALPHA = 32
 
 DEV_BAD_PAGE, DEV_BAD_SEQLEN, DEV_BAD_SLOT, DEV_TIMEOUT = 1, 2, 4, 8
 

@@ -22,6 +22,21 @@
 
 namespace bdfp4 {
 
+// Exponent E of the per-tile pre-scale alpha = 2^E of the dynamic variant: the
+// largest integer with p_max 2^E <= 2688 (6 x 448: the tile's largest block
+// scale still fits E4M3), clamped to [11, 64].  With p_max = m 2^e, m in [1, 2),
+// and 2688 = 1.3125 x 2^11: E = 11 - e, less one when m > 1.3125 -- read from
+// the bits, so the decision is exact in fp32.  p_max <= 0, NaN or subnormal
+// (below 2^-126, where E > 64 anyway) gives 64.
+__device__ __forceinline__ int dynamic_alpha_exp(float p_max) {
+    if (!(p_max > 0.0f)) return 64;
+    const uint32_t u = __float_as_uint(p_max);
+    const int ebits = (int)((u >> 23) & 0xffu);
+    if (ebits == 0) return 64;
+    const int E = 11 - (ebits - 127) - ((u & 0x7fffffu) > 0x280000u ? 1 : 0);
+    return E < 11 ? 11 : (E > 64 ? 64 : E);
+}
+
 template <int FMT, int DK, int DV, int HG>
 __global__ void __launch_bounds__(kThreads) decode_fp4_kernel(const DecodeArgs a) {
     // the split merge (a programmatic dependent) may be scheduled as CTAs of this grid retire
@@ -100,6 +115,8 @@ __global__ void __launch_bounds__(kThreads) decode_fp4_kernel(const DecodeArgs a
     }
 
     const float alpha = (FMT == BDFP4_NVFP4 && !(a.flags & BDFP4_FLAG_NO_UNDERFLOW)) ? kAlphaNV : 1.0f;
+    // dynamic variant: each tile's alpha is divided out of its probabilities
+    const bool dyn = FMT == BDFP4_NVFP4 && (a.flags & BDFP4_FLAG_DYNAMIC_ALPHA);
     const float vg = FMT == BDFP4_NVFP4 ? a.v_gscale[hk] : 1.0f;
     const int64_t kv_stride_k = (int64_t)kPageSlots * DK / 2, kv_stride_ks = k_scale_page_bytes(DK, B);
     const int64_t kv_stride_v = (int64_t)DV * kPageSlots / 2, kv_stride_vs = (int64_t)DV * kPageSlots / B;
@@ -191,8 +208,14 @@ __global__ void __launch_bounds__(kThreads) decode_fp4_kernel(const DecodeArgs a
             m_run[g] = mn;
             p[g] = valid ? exp2f(s[g] - mn) : 0.0f;
             l_part[g] = l_part[g] * corr[g] + p[g];
+            float ag = alpha, ig = 1.0f;
+            if (dyn) {
+                const int E = dynamic_alpha_exp(exp2f(mt - mn));   // the tile's largest p
+                ag = __int_as_float((127 + E) << 23);
+                ig = __int_as_float((127 - E) << 23);
+            }
             // fused probability quantization over beta-token blocks of lanes
-            const float y = p[g] * alpha;
+            const float y = p[g] * ag;
             float am = y;
 #pragma unroll
             for (int off = B / 2; off > 0; off >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, off));
@@ -203,7 +226,7 @@ __global__ void __launch_bounds__(kThreads) decode_fp4_kernel(const DecodeArgs a
                 sigma = e8m0_value(mx_scale_code(am));
             }
             const uint32_t e = sigma > 0.0f ? e2m1_encode(__fdiv_rn(y, sigma)) : 0u;
-            ph[g][tid] = e2m1_value(e) * sigma;
+            ph[g][tid] = e2m1_value(e) * sigma * ig;
         }
         __syncthreads();
         // ------------------------------------------------ P.V (thread = value channel)
@@ -262,7 +285,7 @@ __global__ void __launch_bounds__(kThreads) decode_fp4_kernel(const DecodeArgs a
         if (lane == 0) lsum[warp][g] = v;
     }
     __syncthreads();
-    const float oscale = vg / alpha;
+    const float oscale = dyn ? vg : vg / alpha;
     const bool single = nspl == 1;
 #pragma unroll
     for (int g = 0; g < HG; ++g) {
@@ -353,13 +376,15 @@ static int merge_splits(const DecodeArgs& a, cudaStream_t st) {
 
 template <int FMT, int DK, int DV>
 static int launch_decode(const DecodeArgs& a, int G, cudaStream_t st, const StepArgs* step) {
-    if (DK == 128 && G <= 16) {
+    // the dynamic probability pre-scale runs on the CUDA-core decode (MXFP4 has no alpha)
+    const bool tc_ok = !(FMT == BDFP4_NVFP4 && (a.flags & BDFP4_FLAG_DYNAMIC_ALPHA));
+    if (tc_ok && DK == 128 && G <= 16) {
         // tensor-core path (decode_tc.cu); a step's append runs in its prologue grid
         const int rc = launch_decode_tc(a, FMT, G, st, step);
         if (rc != BDFP4_OK) return rc;
         return merge_splits<DV>(a, st);
     }
-    if (DK == 576 && mla_tc_supported(DK, DV, G)) {
+    if (tc_ok && DK == 576 && mla_tc_supported(DK, DV, G)) {
         // tensor-core path for MLA shapes (decode_mla_tc.cu); a step's append runs in its prologue grid
         const int rc = launch_decode_mla_tc(a, FMT, G, st, step);
         if (rc != BDFP4_OK) return rc;
@@ -398,6 +423,7 @@ static int run_decode(const void* q, const void* k_pages, const void* k_scales, 
         !kv->smooth)
         return BDFP4_ERR_ARG;
     if (fmt == BDFP4_NVFP4 && (!kv->k_gscale || !kv->v_gscale)) return BDFP4_ERR_ARG;
+    if ((flags & BDFP4_FLAG_DYNAMIC_ALPHA) && (flags & BDFP4_FLAG_NO_UNDERFLOW)) return BDFP4_ERR_ARG;
     if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_pages, 128) || !aligned(k_scales, 128) ||
         !aligned(v_pages, 128) || !aligned(v_scales, 128))
         return BDFP4_ERR_ALIGN;
@@ -414,7 +440,8 @@ static int run_decode(const void* q, const void* k_pages, const void* k_scales, 
     }
     DecodeArgs a{};
     a.max_splits = max_splits_for(max_pages_per_seq, chunk_tiles);
-    const bool tensor_core_path = (d_k == 128 && G <= 16) || mla_tc_supported(d_k, d_v, G);
+    const bool tensor_core_path = !(fmt == BDFP4_NVFP4 && (flags & BDFP4_FLAG_DYNAMIC_ALPHA)) &&
+                                  ((d_k == 128 && G <= 16) || mla_tc_supported(d_k, d_v, G));
     if (a.max_splits > 1 || tensor_core_path) {
         const WorkspaceMap m = workspace_map(B, H_q, d_v, a.max_splits);
         if (!workspace || workspace_bytes < m.total) return BDFP4_ERR_WORKSPACE;

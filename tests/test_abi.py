@@ -111,9 +111,9 @@ def test_decode_argument_errors(lib):
     kv = bdfp4._KVParams(0x1000, 0x2000, 0x3000)
     a = _p(0x10000)
 
-    def call(H_q=8, H_kv=2, d_k=128, d_v=128, chunk=1, ws=None, ws_bytes=0, q=a, max_pages=4):
-        return lib.bdfp4_decode(q, a, a, a, a, a, a, 2, H_q, H_kv, d_k, d_v, max_pages, 16, 0, 0, ctypes.byref(kv),
-                                0.1, chunk, ws, ws_bytes, a, None, None)
+    def call(H_q=8, H_kv=2, d_k=128, d_v=128, chunk=1, ws=None, ws_bytes=0, q=a, max_pages=4, flags=0):
+        return lib.bdfp4_decode(q, a, a, a, a, a, a, 2, H_q, H_kv, d_k, d_v, max_pages, 16, 0, flags,
+                                ctypes.byref(kv), 0.1, chunk, ws, ws_bytes, a, None, None)
     assert call(H_q=6, H_kv=2) == -4      # group of 3
     assert call(H_q=7, H_kv=2) == -2      # not a multiple
     assert call(d_k=256) == -4
@@ -122,6 +122,8 @@ def test_decode_argument_errors(lib):
     assert call(chunk=1) == -6            # 2 splits need a workspace
     n = bdfp4.bdfp4_decode_workspace_size(2, 8, 128, 4, 1)
     assert call(chunk=1, ws=_p(0x20000), ws_bytes=n - 1) == -6
+    # the dynamic probability pre-scale and the vanilla alpha = 1 ablation exclude each other
+    assert call(flags=bdfp4.FLAG_DYNAMIC_ALPHA | bdfp4.FLAG_NO_UNDERFLOW) == -1
 
 
 def test_decode_step_and_append_halves_argument_errors(lib):

@@ -251,6 +251,63 @@ def test_decode_ablation_flags_match_oracle(ora, lib, name, flags):
     assert max_abs <= MAX_ABS and rel <= REL_L2, (max_abs, rel)
 
 
+@pytest.mark.parametrize("chunk", [0, 2])
+@pytest.mark.parametrize("name", ["tiny_nv", "ragged_g8_nv", "g16_nv", "g32_cuda_nv", "mla_nv", "mla64_nv",
+                                  "tiny_mx", "mla_mx"])
+def test_decode_dynamic_alpha_matches_oracle(ora, lib, name, chunk):
+    got, ref, _ = _decode_case(ora, name, chunk, bdfp4.FLAG_DYNAMIC_ALPHA)
+    max_abs, rel = compare_outputs(got, ref)
+    assert max_abs <= MAX_ABS and rel <= REL_L2, (max_abs, rel)
+
+
+def test_dynamic_alpha_keeps_a_deep_sink_tail(ora, lib):
+    """One key with logit 14 and 131071 with logit 0, one split: with alpha = 2^11
+    every block without the sink collapses (E4M3(e^-14 2^11 / 6) = 0), a tenth of
+    the attention mass; the per-tile pre-scale keeps it.  Both arms match the
+    oracle; against the unquantized-P output both keep the sink block's own
+    error (P^ = 1.03125 p on 90% of the mass, about 2.5%), and the static arm
+    adds the lost tail (about 7% in all)."""
+    N, H_kv, G, d = 131072, 1, 2, 128
+    rng = np.random.default_rng(11)
+    q = np.zeros((1, G, d), np.float32)
+    q[0, :, 0] = 6.0
+    k = np.zeros((N, H_kv, d), np.float32)
+    k[0, 0, 0] = 6.0
+    v = rng.uniform(0.5, 1.5, (N, H_kv, d)).astype(np.float32)
+    npages = N // 64
+    bt = rng.permutation(npages).astype(np.int32)[None, :]
+    t = np.arange(N)
+    slots = bt[0, t // 64].astype(np.int64) * 64 + t % 64
+    ones = np.ones((H_kv, d), np.float32)
+    g = np.ones(H_kv, np.float32)
+    ocache = ora.empty_cache(npages, H_kv, d, d, NV)
+    qb = torch.from_numpy(q).to(torch.bfloat16)
+    ora.quantize_kv(torch.from_numpy(k).to(torch.bfloat16), torch.from_numpy(v).to(torch.bfloat16), slots, ocache,
+                    H_kv, NV, ones, g, g, npages, flags=bdfp4.FLAG_NO_HADAMARD)
+    gcache = cache_from_np(ocache, npages, H_kv, d, d, NV)
+    sl = np.array([N], np.int32)
+    sm_scale, chunk = 14.0 / 36.0, N // 128
+    outs = {}
+    for name, fl in (("static", 0), ("dynamic", bdfp4.FLAG_DYNAMIC_ALPHA)):
+        fl |= bdfp4.FLAG_NO_HADAMARD
+        ref16, _ = ora.decode(qb, ocache, bt, sl, H_kv, d, NV, ones, g, g, sm_scale, chunk, npages, flags=fl)
+        out = torch.empty((1, G, d), dtype=torch.bfloat16, device="cuda")
+        ws = bdfp4.workspace_for(1, G, d, npages, chunk)
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        bdfp4.bdfp4_decode(qb.cuda(), gcache, torch.from_numpy(bt).cuda(), torch.from_numpy(sl).cuda(),
+                           kv_params_gpu(ones, g, g), sm_scale, chunk, ws, out, flags=fl, dev_status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 0
+        got = out_to_np(out)
+        max_abs, rel = compare_outputs(got, bf16_to_np(ref16))
+        assert max_abs <= MAX_ABS and rel <= REL_L2, (name, max_abs, rel)
+        outs[name] = got.astype(np.float64)
+    _, exact = ora.decode(qb, ocache, bt, sl, H_kv, d, NV, ones, g, g, sm_scale, chunk, npages,
+                          flags=bdfp4.FLAG_NO_HADAMARD | ora.FLAG_EXACT_P)
+    err = {n: np.linalg.norm(o - exact) / np.linalg.norm(exact) for n, o in outs.items()}
+    assert err["dynamic"] < 0.03 and err["static"] > err["dynamic"] + 0.04, err
+
+
 def test_decode_empty_and_single_token(ora, lib):
     sp = spec("tiny", B=3, ctx=("list", (0, 1, 65)))
     SMALL["edge"] = (sp, NV)
