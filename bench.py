@@ -60,7 +60,7 @@ def algorithmic_bytes(sp, seq_lens, fmt: int) -> int:
 # sources of each tensor-core decode kernel: its file and the headers it includes
 DECODE_SOURCES = {
     128: ("decode_tc.cu", "tc_ptx.cuh", "bdfp4_device.cuh", "quant_device.cuh", "decode_common.cuh",
-          "append_device.cuh"),
+          "append_device.cuh", "prob_scale.cuh"),
     576: ("decode_mla_tc.cu", "tc_ptx.cuh", "bdfp4_device.cuh", "quant_device.cuh", "decode_common.cuh",
           "append_device.cuh"),
 }
@@ -358,9 +358,10 @@ def run_ours(args, sp, fmt):
         peak, peak_src = 6650.0, "fallback"
     traffic = None
     tr_path = os.path.join(ROOT, "profiles", "decode_traffic.json")
-    cuda_core = fmt == 0 and args.dynamic_alpha   # the variant runs on the CUDA-core decode
+    # the variant runs on the tensor-core decode at d = 128, on the CUDA-core decode for MLA
+    cuda_core = fmt == 0 and args.dynamic_alpha and sp.d_k != 128
     if os.path.exists(tr_path) and not cuda_core:
-        rec = json.load(open(tr_path)).get(f"{args.config}_{args.fmt}")
+        rec = json.load(open(tr_path)).get(f"{args.config}_{args.fmt}" + ("_dynamic" if args.dynamic_alpha and fmt == 0 else ""))
         # the counters describe the kernel as captured: null once its sources changed
         if rec and rec.get("source_sha256") == decode_source_hash(sp.d_k):
             traffic = rec.get("bytes_per_launch")
@@ -513,7 +514,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-bf16", action="store_true", help="skip the BF16-KV comparator")
     ap.add_argument("--dynamic-alpha", action="store_true",
-                    help="the per-tile probability pre-scale variant (NVFP4: CUDA-core decode)")
+                    help="the per-tile probability pre-scale variant (NVFP4)")
     args = ap.parse_args()
     from fp4_kv_cache_quant_b200.workloads import spec
     sp = spec(args.config)

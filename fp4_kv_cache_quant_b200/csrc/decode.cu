@@ -19,23 +19,9 @@
 #include "quant_device.cuh"
 #include "decode_common.cuh"
 #include "merge.cuh"
+#include "prob_scale.cuh"
 
 namespace bdfp4 {
-
-// Exponent E of the per-tile pre-scale alpha = 2^E of the dynamic variant: the
-// largest integer with p_max 2^E <= 2688 (6 x 448: the tile's largest block
-// scale still fits E4M3), clamped to [11, 64].  With p_max = m 2^e, m in [1, 2),
-// and 2688 = 1.3125 x 2^11: E = 11 - e, less one when m > 1.3125 -- read from
-// the bits, so the decision is exact in fp32.  p_max <= 0, NaN or subnormal
-// (below 2^-126, where E > 64 anyway) gives 64.
-__device__ __forceinline__ int dynamic_alpha_exp(float p_max) {
-    if (!(p_max > 0.0f)) return 64;
-    const uint32_t u = __float_as_uint(p_max);
-    const int ebits = (int)((u >> 23) & 0xffu);
-    if (ebits == 0) return 64;
-    const int E = 11 - (ebits - 127) - ((u & 0x7fffffu) > 0x280000u ? 1 : 0);
-    return E < 11 ? 11 : (E > 64 ? 64 : E);
-}
 
 template <int FMT, int DK, int DV, int HG>
 __global__ void __launch_bounds__(kThreads) decode_fp4_kernel(const DecodeArgs a) {
@@ -211,8 +197,8 @@ __global__ void __launch_bounds__(kThreads) decode_fp4_kernel(const DecodeArgs a
             float ag = alpha, ig = 1.0f;
             if (dyn) {
                 const int E = dynamic_alpha_exp(exp2f(mt - mn));   // the tile's largest p
-                ag = __int_as_float((127 + E) << 23);
-                ig = __int_as_float((127 - E) << 23);
+                ag = pow2f(E);
+                ig = pow2f(-E);
             }
             // fused probability quantization over beta-token blocks of lanes
             const float y = p[g] * ag;
@@ -376,15 +362,16 @@ static int merge_splits(const DecodeArgs& a, cudaStream_t st) {
 
 template <int FMT, int DK, int DV>
 static int launch_decode(const DecodeArgs& a, int G, cudaStream_t st, const StepArgs* step) {
-    // the dynamic probability pre-scale runs on the CUDA-core decode (MXFP4 has no alpha)
-    const bool tc_ok = !(FMT == BDFP4_NVFP4 && (a.flags & BDFP4_FLAG_DYNAMIC_ALPHA));
-    if (tc_ok && DK == 128 && G <= 16) {
+    // the dynamic probability pre-scale runs on the d = 128 tensor-core decode and, for
+    // MLA shapes, on the CUDA-core decode (MXFP4 has no alpha to choose)
+    const bool mla_tc_ok = !(FMT == BDFP4_NVFP4 && (a.flags & BDFP4_FLAG_DYNAMIC_ALPHA));
+    if (DK == 128 && G <= 16) {
         // tensor-core path (decode_tc.cu); a step's append runs in its prologue grid
         const int rc = launch_decode_tc(a, FMT, G, st, step);
         if (rc != BDFP4_OK) return rc;
         return merge_splits<DV>(a, st);
     }
-    if (tc_ok && DK == 576 && mla_tc_supported(DK, DV, G)) {
+    if (mla_tc_ok && DK == 576 && mla_tc_supported(DK, DV, G)) {
         // tensor-core path for MLA shapes (decode_mla_tc.cu); a step's append runs in its prologue grid
         const int rc = launch_decode_mla_tc(a, FMT, G, st, step);
         if (rc != BDFP4_OK) return rc;
@@ -440,8 +427,9 @@ static int run_decode(const void* q, const void* k_pages, const void* k_scales, 
     }
     DecodeArgs a{};
     a.max_splits = max_splits_for(max_pages_per_seq, chunk_tiles);
-    const bool tensor_core_path = !(fmt == BDFP4_NVFP4 && (flags & BDFP4_FLAG_DYNAMIC_ALPHA)) &&
-                                  ((d_k == 128 && G <= 16) || mla_tc_supported(d_k, d_v, G));
+    const bool tensor_core_path = (d_k == 128 && G <= 16) ||
+                                  (!(fmt == BDFP4_NVFP4 && (flags & BDFP4_FLAG_DYNAMIC_ALPHA)) &&
+                                   mla_tc_supported(d_k, d_v, G));
     if (a.max_splits > 1 || tensor_core_path) {
         const WorkspaceMap m = workspace_map(B, H_q, d_v, a.max_splits);
         if (!workspace || workspace_bytes < m.total) return BDFP4_ERR_WORKSPACE;

@@ -23,6 +23,8 @@
 //               same threads write the block-scale factors into TMEM and, when
 //               a running maximum rises, rescale their heads' O^T columns in
 //               TMEM between the previous tile's PV and this one's.
+// The dynamic variant (DYN, NVFP4) picks the probability pre-scale per tile and
+// head and folds a change of it into that same rescale.
 // Every wait is bounded; a timeout sets BDFP4_DEV_TIMEOUT and the CTA unwinds.
 
 #include <type_traits>
@@ -31,6 +33,7 @@
 #include "bdfp4_device.cuh"
 #include "decode_common.cuh"
 #include "host_common.h"
+#include "prob_scale.cuh"
 #include "quant_device.cuh"
 #include "tc_ptx.cuh"
 
@@ -216,7 +219,7 @@ __global__ void __launch_bounds__(256) prep_step_kernel(const DecodeArgs a, cons
     }
 }
 
-template <int FMT, int G>
+template <int FMT, int G, bool DYN = false>
 __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTAS) decode_tc_kernel(const DecodeArgs a) {
     using C = TcCfg<FMT, G>;
     // the split merge (a programmatic dependent) may be scheduled as CTAs of this grid retire
@@ -530,10 +533,13 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
         const bool any_bad_page = *pflag_bad != 0;
         if (lane == 0) tc::mbar_arrive(q_ready);
         float m_run[HG], l_part[HG];
+        // DYN: log2 of each head's current pre-scale; O^T and l are held in its units
+        int e_run[DYN ? HG : 1];
 #pragma unroll
         for (int g = 0; g < HG; ++g) {
             m_run[g] = -INFINITY;
             l_part[g] = 0.0f;
+            if constexpr (DYN) e_run[g] = 11;
         }
         // TMEM lane 32 qd + lane holds token 32 qd + lane of the tile: slot 32 (qd % 2) + lane
         // of page qd / 2, so a warp owns 32 consecutive slots of one page
@@ -611,7 +617,16 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                     corr[g] = tc::ex2_approx(m_run[g] - mz);   // 0 on the split's first tile
                     rose |= mn != m_run[g];
                     m_run[g] = mn;
-                    const float base = mz - la;
+                    float base = mz - la;
+                    if constexpr (DYN) {
+                        // this tile's pre-scale from its largest probability; the accumulators
+                        // move to its units (an exact power of two, folded into corr)
+                        const int e = dynamic_alpha_exp(tc::ex2_approx(mt * lsr[g] - mz));
+                        corr[g] *= pow2f(e - e_run[g]);
+                        rose |= e != e_run[g];
+                        e_run[g] = e;
+                        base = mz - (float)e;
+                    }
                     // the same two instructions give a token's scaled probability and its block's
                     // maximum, so the block scale is the one its largest member picks
                     y[g] = tc::ex2_approx(fmaf(t[g], lsr[g], -base));   // 0 for masked tokens
@@ -757,10 +772,12 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                     a.out[row * C::DV + ch] =
                         __float2bfloat16(l > 0.0f ? __uint_as_float(o_fin[g]) * oscale / l : 0.0f);
                 } else {
-                    a.ws_o[(row * a.max_splits + split) * C::DV + ch] = __uint_as_float(o_fin[g]) * oscale;
+                    // DYN: splits end in different units; the partials leave in the units of p
+                    const float un = DYN ? pow2f(-e_run[DYN ? g : 0]) : 1.0f;
+                    a.ws_o[(row * a.max_splits + split) * C::DV + ch] = __uint_as_float(o_fin[g]) * oscale * un;
                     if (chan == 0) {
                         a.ws_ml[(row * a.max_splits + split) * 2 + 0] = m_run[g];
-                        a.ws_ml[(row * a.max_splits + split) * 2 + 1] = l;
+                        a.ws_ml[(row * a.max_splits + split) * 2 + 1] = l * un;
                     }
                 }
             }
@@ -776,13 +793,13 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
     }
 }
 
-template <int FMT, int G>
+template <int FMT, int G, bool DYN = false>
 static int launch_tc(const DecodeArgs& a, cudaStream_t st, const StepArgs* step) {
     using C = TcCfg<FMT, G>;
     static bool attr_set = false;
     if (!attr_set) {
-        const cudaError_t e =
-            cudaFuncSetAttribute(decode_tc_kernel<FMT, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_LAUNCH);
+        const cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<FMT, G, DYN>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_LAUNCH);
         if (e != cudaSuccess) {
             record_cuda_error(e);
             return BDFP4_ERR_CUDA;
@@ -810,7 +827,7 @@ static int launch_tc(const DecodeArgs& a, cudaStream_t st, const StepArgs* step)
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<FMT, G>, a);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<FMT, G, DYN>, a);
     if (e != cudaSuccess) {
         record_cuda_error(e);
         return BDFP4_ERR_CUDA;
@@ -819,7 +836,15 @@ static int launch_tc(const DecodeArgs& a, cudaStream_t st, const StepArgs* step)
 }
 
 int launch_decode_tc(const DecodeArgs& a, int fmt, int G, cudaStream_t st, const StepArgs* step) {
-    if (fmt == BDFP4_NVFP4) {
+    if (fmt == BDFP4_NVFP4 && (a.flags & BDFP4_FLAG_DYNAMIC_ALPHA)) {
+        switch (G) {
+            case 1: return launch_tc<BDFP4_NVFP4, 1, true>(a, st, step);
+            case 2: return launch_tc<BDFP4_NVFP4, 2, true>(a, st, step);
+            case 4: return launch_tc<BDFP4_NVFP4, 4, true>(a, st, step);
+            case 8: return launch_tc<BDFP4_NVFP4, 8, true>(a, st, step);
+            case 16: return launch_tc<BDFP4_NVFP4, 16, true>(a, st, step);
+        }
+    } else if (fmt == BDFP4_NVFP4) {
         switch (G) {
             case 1: return launch_tc<BDFP4_NVFP4, 1>(a, st, step);
             case 2: return launch_tc<BDFP4_NVFP4, 2>(a, st, step);

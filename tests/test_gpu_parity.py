@@ -110,6 +110,16 @@ def test_decode_step_matches_oracle(ora, lib, name, chunk):
     value block must hold the new value, and the output must match the oracle's
     decode (and equal bdfp4_decode on the updated cache bit for bit).  Rows of
     the open block past the new token hold large noise the step must ignore."""
+    _decode_step_case(ora, name, chunk, 0)
+
+
+@pytest.mark.parametrize("chunk", [0, 1])
+@pytest.mark.parametrize("name", ["tiny_nv", "ragged_g8_nv", "mla_nv"])
+def test_decode_step_dynamic_alpha_matches_oracle(ora, lib, name, chunk):
+    _decode_step_case(ora, name, chunk, bdfp4.FLAG_DYNAMIC_ALPHA)
+
+
+def _decode_step_case(ora, name, chunk, flags):
     sp, fmt = SMALL[name]
     wl = Workload(sp, seed=8)
     smooth, kg, vg = oracle_calibration(ora, wl)
@@ -149,7 +159,7 @@ def test_decode_step_matches_oracle(ora, lib, name, chunk):
     ws = bdfp4.workspace_for(sp.B, sp.H_q, sp.d_v, bt.shape[1], chunk)
     v_open_g = v_open.cuda()
     bdfp4.bdfp4_decode_step(q.cuda(), k_new.cuda(), v_new.cuda(), v_open_g, gcache, bt, sl, kvp, sp.sm_scale, chunk,
-                            ws, out, dev_status=status)
+                            ws, out, flags=flags, dev_status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     assert_bytes_equal(cache_to_np(gcache), ocache)
@@ -158,11 +168,11 @@ def test_decode_step_matches_oracle(ora, lib, name, chunk):
         if last >= 0:
             assert torch.equal(vo[b, last], v_new[b])
     ref16, _ = ora.decode(q, ocache, wl.block_table, wl.seq_lens, sp.H_kv, sp.d_v, fmt, smooth, kg, vg, sp.sm_scale,
-                          chunk, wl.num_pages)
+                          chunk, wl.num_pages, flags=flags)
     got = out_to_np(out)
     max_abs, rel = compare_outputs(got, bf16_to_np(ref16))
     assert max_abs <= MAX_ABS and rel <= REL_L2, (max_abs, rel)
-    again, st2 = run_gpu_decode(wl, gcache, q, kvp, chunk)
+    again, st2 = run_gpu_decode(wl, gcache, q, kvp, chunk, flags)
     assert st2 == 0 and torch.equal(again, out)
 
 
