@@ -89,6 +89,12 @@ def lib():
         L.ora_search_scale_code.argtypes = [i, p, i, f]
         L.ora_dynamic_alpha_exp.restype = i
         L.ora_dynamic_alpha_exp.argtypes = [d]
+        L.ora_search_scale_code_weighted.restype = i
+        L.ora_search_scale_code_weighted.argtypes = [i, p, i, f, p]
+        L.ora_key_weights.restype = i
+        L.ora_key_weights.argtypes = [p, i, i, i, i, i, p, p]
+        L.ora_quantize_kv_weighted.restype = i
+        L.ora_quantize_kv_weighted.argtypes = [p, p, p, i, i, i, i, i, i, p, p, p, p, p, p, p, p, i64]
         L.ora_dequant_key_row.restype = None
         L.ora_dequant_key_row.argtypes = [p, p, i, i64, i, i, i, i, p]
         L.ora_dequant_value_row.restype = None
@@ -168,9 +174,12 @@ def plain_scale_code(fmt: int, amax: float, g: float) -> int:
     return lib().ora_plain_scale_code(fmt, float(amax), float(g))
 
 
-def search_scale_code(fmt: int, x: np.ndarray, g: float) -> int:
+def search_scale_code(fmt: int, x: np.ndarray, g: float, w=None) -> int:
     x = np.ascontiguousarray(x, np.float32)
-    return lib().ora_search_scale_code(fmt, _ptr(x), x.shape[0], float(g))
+    if w is None:
+        return lib().ora_search_scale_code(fmt, _ptr(x), x.shape[0], float(g))
+    w = np.ascontiguousarray(w, np.float32)
+    return lib().ora_search_scale_code_weighted(fmt, _ptr(x), x.shape[0], float(g), _ptr(w))
 
 
 def dynamic_alpha_exp(p_max: float) -> int:
@@ -242,8 +251,9 @@ def empty_cache(num_pages: int, H_kv: int, d_k: int, d_v: int, fmt: int) -> dict
 
 
 def quantize_kv(k, v, slot_mapping, cache: dict, H_kv: int, fmt: int, smooth, k_g, v_g,
-                num_pages: int, flags: int = 0) -> dict:
-    """Append-quantize tokens into ``cache`` (in place) and return it."""
+                num_pages: int, flags: int = 0, k_weight=None) -> dict:
+    """Append-quantize tokens into ``cache`` (in place) and return it.  ``k_weight``
+    ([H_kv, d_k]) selects the attention-aware key scale search."""
     kb, vb = _bits(k), _bits(v)
     T, _, d_k = kb.shape
     d_v = vb.shape[2]
@@ -251,11 +261,27 @@ def quantize_kv(k, v, slot_mapping, cache: dict, H_kv: int, fmt: int, smooth, k_
     s = np.ascontiguousarray(smooth, np.float32)
     kg = np.ascontiguousarray(k_g, np.float32)
     vg = np.ascontiguousarray(v_g, np.float32)
-    rc = lib().ora_quantize_kv(_ptr(kb), _ptr(vb), _ptr(sm), T, H_kv, d_k, d_v, fmt, flags,
-                               _ptr(s), _ptr(kg), _ptr(vg), _ptr(cache["k_pages"]), _ptr(cache["k_scales"]),
-                               _ptr(cache["v_pages"]), _ptr(cache["v_scales"]), num_pages)
+    pages = (_ptr(cache["k_pages"]), _ptr(cache["k_scales"]), _ptr(cache["v_pages"]), _ptr(cache["v_scales"]))
+    if k_weight is None:
+        rc = lib().ora_quantize_kv(_ptr(kb), _ptr(vb), _ptr(sm), T, H_kv, d_k, d_v, fmt, flags,
+                                   _ptr(s), _ptr(kg), _ptr(vg), *pages, num_pages)
+    else:
+        w = np.ascontiguousarray(k_weight, np.float32).reshape(H_kv, d_k)
+        rc = lib().ora_quantize_kv_weighted(_ptr(kb), _ptr(vb), _ptr(sm), T, H_kv, d_k, d_v, fmt, flags,
+                                            _ptr(s), _ptr(kg), _ptr(vg), _ptr(w), *pages, num_pages)
     assert rc == 0, rc
     return cache
+
+
+def key_weights(q_cal, H_q: int, H_kv: int, smooth, flags: int = 0) -> np.ndarray:
+    """[H_kv, d_k] channel weights of the attention-aware key scale search."""
+    q = _bits(q_cal)
+    Tq, _, d_k = q.shape
+    s = np.ascontiguousarray(smooth, np.float32)
+    w = np.empty((H_kv, d_k), np.float32)
+    rc = lib().ora_key_weights(_ptr(q), Tq, H_q, H_kv, d_k, flags, _ptr(s), _ptr(w))
+    assert rc == 0, rc
+    return w
 
 
 def quantize_q(q, H_kv: int, fmt: int, smooth, flags: int = 0) -> dict:

@@ -403,6 +403,41 @@ int ora_search_scale_code(int fmt, const float* x, int n, float g)
     return best;
 }
 
+/* Attention-aware variant of the search (the pages leave its objective open):
+ * the same window and tie rule, with each element's squared error weighted by
+ * w_i, the calibration queries' mean square of that transformed channel -- for
+ * independent channels, the expected square of the logit error q'.(k' - k^')
+ * the block adds.  w = NULL is the plain objective (a weight of 1 changes no
+ * sum).  Sums run left to right in fp64. */
+int ora_search_scale_code_weighted(int fmt, const float* x, int n, float g, const float* w)
+{
+    if (!w) return ora_search_scale_code(fmt, x, n, g);
+    float amax = block_amax(x, n);
+    int c0 = ora_plain_scale_code(fmt, amax, g);
+    if (amax == 0.0f) return c0;
+    int top = (fmt == ORA_NVFP4) ? 126 : 254;
+    int hi = (fmt == ORA_NVFP4) ? c0 + 7 : c0 + 1;
+    int lo = (fmt == ORA_NVFP4) ? c0 - 2 : c0;
+    if (hi > top) hi = top;
+    if (lo < 0) lo = 0;
+    int best = hi;
+    double best_err = 0.0;
+    for (int c = hi; c >= lo; --c) {
+        float sigma = ora_block_sigma(fmt, c, g);
+        double err = 0.0;
+        for (int i = 0; i < n; ++i) {
+            int e = sigma != 0.0f ? ora_e2m1_encode((double)(x[i] / sigma)) : 0;
+            double d = (double)x[i] - ora_e2m1_value(e) * (double)sigma;
+            err = err + (double)w[i] * (d * d);
+        }
+        if (c == hi || err < best_err) {
+            best = c;
+            best_err = err;
+        }
+    }
+    return best;
+}
+
 static int fmt_beta(int fmt) { return fmt == ORA_NVFP4 ? 16 : 32; }
 
 /* =========================================================================
@@ -475,6 +510,31 @@ int ora_calibrate(const uint16_t* k_cal, const uint16_t* q_cal, const uint16_t* 
     return 0;
 }
 
+/* Channel weights of the attention-aware search: per KV head h and channel c
+ * of the transformed key space, the mean over the calibration queries of the
+ * KV group (Tq tokens x G heads) of q'_c^2, q' = the query transform (smoothing
+ * and rotation as the decode applies them).  fp64 sums, stored as fp32. */
+int ora_key_weights(const uint16_t* q_cal, int Tq, int H_q, int H_kv, int d_k, int flags, const float* smooth,
+                    float* w)
+{
+    if (H_kv <= 0 || H_q % H_kv != 0 || d_k > 1024 || d_k % 64 || Tq <= 0) return -1;
+    int G = H_q / H_kv;
+    int hadamard = !(flags & ORA_FLAG_NO_HADAMARD);
+    for (int h = 0; h < H_kv; ++h) {
+        double acc[1024];
+        for (int c = 0; c < d_k; ++c) acc[c] = 0.0;
+        for (int t = 0; t < Tq; ++t)
+            for (int j = 0; j < G; ++j) {
+                float in[1024], x[1024];
+                for (int c = 0; c < d_k; ++c) in[c] = bf16_to_f32(q_cal[((size_t)t * H_q + h * G + j) * d_k + c]);
+                ora_transform(in, smooth + (size_t)h * d_k, d_k, 0, hadamard, x);
+                for (int c = 0; c < d_k; ++c) acc[c] += (double)x[c] * (double)x[c];
+            }
+        for (int c = 0; c < d_k; ++c) w[(size_t)h * d_k + c] = (float)(acc[c] / ((double)Tq * G));
+    }
+    return 0;
+}
+
 /* =========================================================================
  * 6. KV-append quantization into the paged cache.
  *
@@ -491,7 +551,7 @@ int ora_calibrate(const uint16_t* k_cal, const uint16_t* q_cal, const uint16_t* 
  * zero.  slot_mapping[t] = page * 64 + slot, or -1 to skip the token.
  * ========================================================================= */
 
-static void quantize_key_row(const float* x, int d_k, int fmt, int search, float g,
+static void quantize_key_row(const float* x, int d_k, int fmt, int search, float g, const float* w,
                              int64_t page, int head, int H_kv, int slot,
                              uint8_t* k_pages, uint8_t* k_scales)
 {
@@ -499,7 +559,7 @@ static void quantize_key_row(const float* x, int d_k, int fmt, int search, float
     uint8_t codes[64];
     for (int b = 0; b < d_k / beta; ++b) {
         const float* xb = x + b * beta;
-        int sc = search ? ora_search_scale_code(fmt, xb, beta, g)
+        int sc = search ? ora_search_scale_code_weighted(fmt, xb, beta, g, w ? w + b * beta : NULL)
                         : ora_plain_scale_code(fmt, block_amax(xb, beta), g);
         ora_quantize_block(xb, beta, ora_block_sigma(fmt, sc, g), codes);
         k_scales[k_scale_byte(page, head, H_kv, d_k, beta, slot, b)] = (uint8_t)sc;
@@ -510,11 +570,13 @@ static void quantize_key_row(const float* x, int d_k, int fmt, int search, float
     }
 }
 
-int ora_quantize_kv(const uint16_t* k, const uint16_t* v, const int64_t* slot_mapping, int T,
-                    int H_kv, int d_k, int d_v, int fmt, int flags,
-                    const float* smooth, const float* k_g, const float* v_g,
-                    uint8_t* k_pages, uint8_t* k_scales, uint8_t* v_pages, uint8_t* v_scales,
-                    int64_t num_pages)
+/* k_weight: [H_kv][d_k] channel weights of the attention-aware search, or
+ * NULL for the plain objective (ora_quantize_kv). */
+int ora_quantize_kv_weighted(const uint16_t* k, const uint16_t* v, const int64_t* slot_mapping, int T,
+                             int H_kv, int d_k, int d_v, int fmt, int flags,
+                             const float* smooth, const float* k_g, const float* v_g, const float* k_weight,
+                             uint8_t* k_pages, uint8_t* k_scales, uint8_t* v_pages, uint8_t* v_scales,
+                             int64_t num_pages)
 {
     init_tables();
     if (d_k % 64 || d_v % 128 || d_k > 1024 || (fmt != ORA_NVFP4 && fmt != ORA_MXFP4)) return -1;
@@ -536,7 +598,8 @@ int ora_quantize_kv(const uint16_t* k, const uint16_t* v, const int64_t* slot_ma
             for (int c = 0; c < d_k; ++c) in[c] = bf16_to_f32(k[((size_t)t * H_kv + h) * d_k + c]);
             ora_transform(in, smooth + (size_t)h * d_k, d_k, 1, hadamard, x);
             float g = fmt == ORA_NVFP4 ? k_g[h] : 1.0f;
-            quantize_key_row(x, d_k, fmt, search, g, page, h, H_kv, slot, k_pages, k_scales);
+            quantize_key_row(x, d_k, fmt, search, g, k_weight ? k_weight + (size_t)h * d_k : NULL, page, h, H_kv,
+                             slot, k_pages, k_scales);
         }
     }
 
@@ -573,6 +636,16 @@ int ora_quantize_kv(const uint16_t* k, const uint16_t* v, const int64_t* slot_ma
         }
     }
     return 0;
+}
+
+int ora_quantize_kv(const uint16_t* k, const uint16_t* v, const int64_t* slot_mapping, int T,
+                    int H_kv, int d_k, int d_v, int fmt, int flags,
+                    const float* smooth, const float* k_g, const float* v_g,
+                    uint8_t* k_pages, uint8_t* k_scales, uint8_t* v_pages, uint8_t* v_scales,
+                    int64_t num_pages)
+{
+    return ora_quantize_kv_weighted(k, v, slot_mapping, T, H_kv, d_k, d_v, fmt, flags, smooth, k_g, v_g, NULL,
+                                    k_pages, k_scales, v_pages, v_scales, num_pages);
 }
 
 /* =========================================================================

@@ -179,3 +179,129 @@ def test_dual_residual_never_worse_elementwise(ora, fmt):
     if fmt == 0:
         # g_q is the per-head amax / 2688
         assert np.array_equal(out["g_q"], (np.abs(out["xq"]).max(-1) / np.float32(2688)).astype(np.float32))
+
+
+def _np_block_w(x, sigma, w):
+    """_np_block with each squared error weighted (fp64, left to right)."""
+    x = np.asarray(x, np.float32)
+    if sigma == 0:
+        vals = np.zeros_like(x, dtype=np.float64)
+    else:
+        vals = (x / np.float32(sigma)).astype(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    err = 0.0
+    for i in range(x.shape[0]):
+        d = float(x[i]) - vals[i] * float(sigma)
+        err = err + float(np.float32(w[i])) * (d * d)
+    return err
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_weighted_search_against_brute_force(ora, fmt):
+    """The attention-aware search keeps the plain search's window and tie rule
+    (larger code) and minimises the weighted block error: checked against every
+    code of the window, errors re-derived with ml_dtypes."""
+    rng = np.random.default_rng(20 + fmt)
+    n = 16 if fmt == 0 else 32
+    g = np.float32(0.0123) if fmt == 0 else np.float32(1.0)
+    changed = 0
+    for trial in range(300):
+        x = (rng.standard_normal(n) * rng.choice([1.0, 0.3, 3.0])).astype(np.float32)
+        if trial % 3 == 0:
+            x[rng.integers(n)] *= 8.0
+        w = (10.0 ** rng.uniform(-3, 3, n)).astype(np.float32)
+        if trial % 5 == 0:
+            w[rng.integers(n)] = 0.0
+        code = ora.search_scale_code(fmt, x, float(g), w)
+        c0 = ora.plain_scale_code(fmt, float(np.abs(x).max()), float(g))
+        if fmt == 0:
+            window = [c for c in range(c0 + 7, c0 - 3, -1) if 0 <= c <= 126]
+        else:
+            window = [c for c in (c0 + 1, c0) if 0 <= c <= 254]
+        errs = {c: _np_block_w(x, _sigma(fmt, c, g), w) for c in window}
+        assert code == min(window, key=lambda c: (errs[c], -c)), trial
+        changed += code != ora.search_scale_code(fmt, x, float(g))
+    if fmt == 0:
+        assert changed > 0   # the weights do move the choice
+
+
+def test_weighted_search_reductions(ora):
+    """Unit weights are the plain objective (bit for bit, through the cache);
+    scaling all weights by a power of two changes no choice; one dominant
+    weight makes that element's error the first criterion."""
+    rng = np.random.default_rng(23)
+    for trial in range(200):
+        x = (rng.standard_normal(16) * 2).astype(np.float32)
+        assert ora.search_scale_code(0, x, 0.01, np.ones(16, np.float32)) == ora.search_scale_code(0, x, 0.01)
+        w = rng.uniform(0.1, 10, 16).astype(np.float32)
+        assert ora.search_scale_code(0, x, 0.01, w) == ora.search_scale_code(0, x, 0.01, w * np.float32(2.0 ** -7))
+        i = int(rng.integers(16))
+        wd = np.ones(16, np.float32)
+        wd[i] = 1e12
+        code = ora.search_scale_code(0, x, 0.01, wd)
+        c0 = ora.plain_scale_code(0, float(np.abs(x).max()), 0.01)
+        window = [c for c in range(c0 + 7, c0 - 3, -1) if 0 <= c <= 126]
+
+        def elem_err(c):
+            s = _sigma(0, c, np.float32(0.01))
+            v = float(np.float32(x[i] / s).astype(ml_dtypes.float4_e2m1fn)) if s else 0.0
+            return abs(float(x[i]) - v * float(s))
+        assert elem_err(code) == min(elem_err(c) for c in window), trial
+    # through the cache: unit weights give the same bytes as the plain quantizer
+    H_kv, d, T = 2, 128, 40
+    k = _bf16(rng.standard_normal((T, H_kv, d)) * 3)
+    v = _bf16(rng.standard_normal((T, H_kv, d)))
+    ones = np.ones((H_kv, d), np.float32)
+    g = np.full(H_kv, 0.004, np.float32)
+    a = ora.quantize_kv(k, v, np.arange(T), ora.empty_cache(1, H_kv, d, d, 0), H_kv, 0, ones, g, g, 1)
+    b = ora.quantize_kv(k, v, np.arange(T), ora.empty_cache(1, H_kv, d, d, 0), H_kv, 0, ones, g, g, 1,
+                        k_weight=ones)
+    for name in a:
+        assert np.array_equal(a[name], b[name]), name
+
+
+def test_key_weights_hand_values(ora):
+    """Mean square of the transformed calibration queries per channel.  Without
+    rotation: q' = q s, so 2 queries with q_0 = 3, 5 and s_0 = 2 give
+    w_0 = ((6^2) + (10^2)) / 2 = 68.  With rotation (d = 128, query scale
+    2^-3), one query 4 e_0 becomes 4/8 = 0.5 in every channel: w = 0.25."""
+    d, H_kv = 128, 1
+    q = np.zeros((2, 1, d), np.float32)
+    q[0, 0, 0], q[1, 0, 0] = 3.0, 5.0
+    q[0, 0, 7] = -1.0
+    s = np.ones((H_kv, d), np.float32)
+    s[0, 0] = 2.0
+    w = ora.key_weights(_bf16(q), 1, H_kv, s, flags=ora.FLAG_NO_HADAMARD)
+    expect = np.zeros(d)
+    expect[0], expect[7] = 68.0, 0.5
+    assert np.array_equal(w[0], expect.astype(np.float32))
+    q1 = np.zeros((1, 2, d), np.float32)   # two query heads of one KV head
+    q1[0, 0, 0] = 4.0
+    q1[0, 1, 0] = 4.0
+    w = ora.key_weights(_bf16(q1), 2, 1, np.ones((1, d), np.float32))
+    assert np.array_equal(w[0], np.full(d, 0.25, np.float32))
+
+
+def test_attention_aware_search_lowers_logit_error(ora):
+    """With query energy concentrated on a few channels (no rotation, which
+    would spread it), weighting the search by it lowers the squared logit error
+    q.(k - k^) over fresh queries of the same distribution (a sanity bound)."""
+    rng = np.random.default_rng(31)
+    H_kv, d, T = 1, 128, 256
+    k = rng.standard_normal((T, H_kv, d)).astype(np.float32)
+    std = np.where(np.arange(d) % 16 < 2, 8.0, 0.25)
+    qc = (rng.standard_normal((512, 1, d)) * std).astype(np.float32)
+    qt = (rng.standard_normal((512, d)) * std).astype(np.float32)
+    ones = np.ones((H_kv, d), np.float32)
+    kb = _bf16(k)
+    xt = kb.float().numpy()[:, 0]
+    g = np.array([np.abs(xt).max() / 2688], np.float32)
+    w = ora.key_weights(_bf16(qc), 1, H_kv, ones, flags=ora.FLAG_NO_HADAMARD)
+    errs = {}
+    for name, kw in (("plain", None), ("weighted", w)):
+        cache = ora.quantize_kv(kb, _bf16(np.zeros_like(k)), np.arange(T), ora.empty_cache(4, H_kv, d, d, 0), H_kv,
+                                0, ones, g, g, 4, flags=ora.FLAG_NO_HADAMARD, k_weight=kw)
+        deq = np.stack([ora.dequant_key_row(cache, 0, 0, 0, H_kv, d, t) for t in range(64)]) * g[0]
+        deq = np.concatenate([deq] + [np.stack([ora.dequant_key_row(cache, 0, p, 0, H_kv, d, t)
+                                                for t in range(64)]) * g[0] for p in (1, 2, 3)])
+        errs[name] = float((((deq - xt) @ qt.T) ** 2).mean())
+    assert errs["weighted"] < 0.9 * errs["plain"], errs
