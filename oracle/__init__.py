@@ -319,6 +319,27 @@ def decode(q, cache: dict, block_table, seq_lens, H_kv: int, d_v: int, fmt: int,
     return out16, out64
 
 
+def decode_multi(q, cache: dict, block_table, seq_lens, H_kv: int, d_v: int, fmt: int, smooth, k_g, v_g,
+                 sm_scale: float, chunk_tiles: int, num_pages: int, flags: int = 0):
+    """Multi-token queries (speculative or chunked decode): q [B, T_q, H_q, d_k]
+    holds each sequence's T_q newest tokens, already in the cache.  Query token i
+    attends causally to the first seq_lens[b] - T_q + 1 + i tokens and runs the
+    single-token decode on that prefix, with the same tile and split boundaries
+    (splits cut at multiples of chunk_tiles from the sequence start).  Returns
+    (bf16 bits, fp64) outputs [B, T_q, H_q, d_v]."""
+    qb = _bits(q)
+    B, T_q, H_q, d_k = qb.shape
+    bt = np.ascontiguousarray(block_table, dtype=np.int32)
+    sl = np.asarray(seq_lens, dtype=np.int64)
+    if np.any(sl < T_q):
+        raise ValueError("every sequence must hold its T_q query tokens")
+    rows_sl = (sl[:, None] - T_q + 1 + np.arange(T_q)[None, :]).reshape(-1).astype(np.int32)
+    rows_bt = np.repeat(bt, T_q, axis=0)
+    o16, o64 = decode(np.ascontiguousarray(qb.reshape(B * T_q, H_q, d_k)), cache, rows_bt, rows_sl, H_kv, d_v, fmt, smooth, k_g, v_g, sm_scale, chunk_tiles,
+                      num_pages, flags=flags)
+    return o16.reshape(B, T_q, H_q, d_v), o64.reshape(B, T_q, H_q, d_v)
+
+
 def attention_ref(q, k, v, cu_seqlens, H_kv: int, sm_scale: float) -> np.ndarray:
     """fp64 softmax(q k^T * sm_scale) v on the unquantized bf16 inputs."""
     qb, kb, vb = _bits(q), _bits(k), _bits(v)

@@ -255,3 +255,43 @@ def test_quantized_probabilities_stay_close_on_random_data(ora):
     _, quant = ora.decode(*args, flags=ora.FLAG_NO_HADAMARD)
     rel = np.linalg.norm(quant - exact) / np.linalg.norm(exact)
     assert 0 < rel < 0.1
+
+
+@pytest.mark.parametrize("T_q,seq_lens", [(4, [300, 4, 129]), (1, [77, 200]), (16, [1000])])
+def test_multi_token_queries_match_causal_textbook_attention(ora, T_q, seq_lens):
+    """Multi-token queries on FP4-exact inputs with unquantized P equal causal
+    fp64 attention written out in numpy (query token i of a sequence of N sees
+    keys 0 .. N - T_q + i); with T_q = 1 the call is the single-token decode."""
+    rng = np.random.default_rng(40 + T_q)
+    H_kv, G, d = 2, 4, 128
+    H_q = G * H_kv
+    _, k, v = _exact_case(rng, seq_lens, H_q, H_kv, d)
+    q = _exact_fp4(rng, (len(seq_lens), T_q, H_q), 16, d)
+    bt, num_pages, sm = _pages(seq_lens, rng)
+    ones = np.ones((H_kv, d), np.float32)
+    g = np.ones(H_kv, np.float32)
+    cache = ora.empty_cache(num_pages, H_kv, d, d, ora.NVFP4)
+    fl = ora.FLAG_NO_HADAMARD
+    ora.quantize_kv(_bf16(k), _bf16(v), sm, cache, H_kv, ora.NVFP4, ones, g, g, num_pages, flags=fl)
+    sm_scale = 1 / math.sqrt(d) / 8
+    qf = _bf16(q).float().numpy().astype(np.float64)
+    kf, vf = k.astype(np.float64), v.astype(np.float64)
+    for chunk in (1, 3):
+        _, o64 = ora.decode_multi(_bf16(q), cache, bt, np.array(seq_lens), H_kv, d, ora.NVFP4, ones, g, g,
+                                  sm_scale, chunk, num_pages, flags=fl | ora.FLAG_EXACT_P)
+        off = 0
+        for b, n in enumerate(seq_lens):
+            for i in range(T_q):
+                vis = n - T_q + 1 + i
+                for h in range(H_q):
+                    s = kf[off:off + vis, h // G] @ qf[b, i, h] * sm_scale
+                    p = np.exp(s - s.max())
+                    ref = p @ vf[off:off + vis, h // G] / p.sum()
+                    assert np.allclose(o64[b, i, h], ref, rtol=0, atol=1e-6 * (np.abs(ref).max() + 1e-30))
+            off += n
+    if T_q == 1:
+        o16m, _ = ora.decode_multi(_bf16(q), cache, bt, np.array(seq_lens), H_kv, d, ora.NVFP4, ones, g, g,
+                                   sm_scale, 2, num_pages, flags=fl)
+        o16, _ = ora.decode(_bf16(q[:, 0]), cache, bt, np.array(seq_lens), H_kv, d, ora.NVFP4, ones, g, g,
+                            sm_scale, 2, num_pages, flags=fl)
+        assert np.array_equal(o16m[:, 0], o16)
