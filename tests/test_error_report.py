@@ -15,7 +15,8 @@ these are the errors of the GPU results too:
   underflow-aware alpha = 2^11 and with alpha = 1, for near-uniform logits
   (keys N(0, 0.05^2)) and for a batch with a planted sink token per 4096 tokens
   (logit +12 over a N(0, 1.5^2)-logit bulk), where alpha = 1 collapses the
-  small probabilities.
+  small probabilities, and the per-tile alpha variant on these and on a deep
+  sink (logit +16 in 131072 tokens), where alpha = 2^11 collapses them too.
 
 Each test asserts the ordering the method must show and records its numbers;
 with BDFP4_REPORT=<path> the collected figures are written there as JSON."""
@@ -32,6 +33,7 @@ from fp4_kv_cache_quant_b200.workloads import Workload, spec
 
 NV, MX = 0, 1
 FLAG_NO_HADAMARD, FLAG_NO_SCALE_SEARCH, FLAG_SINGLE_QUERY, FLAG_NO_UNDERFLOW, FLAG_EXACT_P = 1, 2, 4, 8, 16
+FLAG_DYNAMIC_ALPHA = 32
 
 REPORT = {}
 
@@ -140,9 +142,10 @@ def test_output_error_against_bf16_kv(ora, fmt):
     assert errs["method"] <= errs["single_query"]
 
 
-def _sink_workload(seed: int, n: int, period: int = 4096):
-    """One KV head, G = 1: bulk logits N(0, 1.5^2), one sink token (logit +12) per `period`
-    tokens; bulk values mu + 0.3 N(0, 1) around a common mu, sink values N(0, 1)."""
+def _sink_workload(seed: int, n: int, period: int = 4096, sink_logit: float = 12.0):
+    """One KV head, G = 1: bulk logits N(0, 1.5^2), one sink token (logit +12, or
+    `sink_logit`) per `period` tokens; bulk values mu + 0.3 N(0, 1) around a common
+    mu, sink values N(0, 1)."""
     rng = np.random.default_rng(seed)
     d = 128
     sm = 1.0 / math.sqrt(d)
@@ -153,7 +156,8 @@ def _sink_workload(seed: int, n: int, period: int = 4096):
     z -= np.outer(z @ qn, qn)
     along = rng.standard_normal(n) * 1.5 / (sm * np.linalg.norm(q))
     k = z + np.outer(along, qn)
-    k[::period] = z[::period] + np.outer(np.full(len(range(0, n, period)), 12.0 / (sm * np.linalg.norm(q))), qn)
+    k[::period] = z[::period] + np.outer(np.full(len(range(0, n, period)), sink_logit / (sm * np.linalg.norm(q))),
+                                         qn)
     # the bulk's values share a direction, so the mass in its small probabilities
     # carries signal (random values would let a dropped bulk cancel out)
     mu = rng.standard_normal(d)
@@ -200,8 +204,27 @@ def test_underflow_alpha_sink_stress(ora):
     q, k, v, sm = _sink_workload(24, 16384)
     ref = _decode_pages(ora, q, k, v, sm, NV, FLAG_EXACT_P)
     errs = {name: _rel(_decode_pages(ora, q, k, v, sm, NV, flags), ref)
-            for name, flags in (("alpha_2^11", 0), ("alpha_1", FLAG_NO_UNDERFLOW))}
+            for name, flags in (("alpha_2^11", 0), ("alpha_1", FLAG_NO_UNDERFLOW),
+                                ("alpha_per_tile", FLAG_DYNAMIC_ALPHA))}
     REPORT["underflow_sink_stress_nvfp4"] = errs
     print(f"\nsink stress, 16384 tokens, error added by P quantization: alpha=2^11 {errs['alpha_2^11']:.5f}, "
-          f"alpha=1 {errs['alpha_1']:.5f}")
+          f"alpha=1 {errs['alpha_1']:.5f}, per-tile alpha {errs['alpha_per_tile']:.5f}")
     assert errs["alpha_2^11"] < errs["alpha_1"] / 2
+    assert errs["alpha_per_tile"] <= errs["alpha_2^11"] * 1.05
+
+
+def test_underflow_deep_sink_per_tile_alpha(ora):
+    """One sink of logit +16 in 131072 tokens: the bulk's blocks fall below the
+    smallest E4M3 scale even at alpha = 2^11 (block maxima near e^-13 x 2^11 / 6),
+    while holding about 5% of the attention mass; the per-tile alpha of the tiles
+    without the sink keeps them.  What remains (about 0.03) is the sink block's
+    own error: P^ = 1.03125 p on 95% of the mass, the same in both arms."""
+    q, k, v, sm = _sink_workload(25, 131072, period=131072, sink_logit=16.0)
+    ref = _decode_pages(ora, q, k, v, sm, NV, FLAG_EXACT_P)
+    errs = {name: _rel(_decode_pages(ora, q, k, v, sm, NV, flags), ref)
+            for name, flags in (("alpha_2^11", 0), ("alpha_1", FLAG_NO_UNDERFLOW),
+                                ("alpha_per_tile", FLAG_DYNAMIC_ALPHA))}
+    REPORT["underflow_deep_sink_nvfp4"] = errs
+    print(f"\ndeep sink, 131072 tokens, error added by P quantization: alpha=2^11 {errs['alpha_2^11']:.5f}, "
+          f"alpha=1 {errs['alpha_1']:.5f}, per-tile alpha {errs['alpha_per_tile']:.5f}")
+    assert errs["alpha_per_tile"] < 0.8 * errs["alpha_2^11"]
