@@ -205,3 +205,19 @@ def test_decode_plan_minimises_the_documented_wave_cost(lib):
         cost = {c: -(-H_kv * sum(-(-t // c) for t in tiles) // (4 * sms)) * (c + 3) for c in range(16, min(64, mx) + 1)}
         best = min(cost.values())
         assert cost[got] == best and got == max(c for c, v in cost.items() if v == best)
+
+
+def test_binding_and_oracle_constants_match_the_header():
+    """Every flag and device-status bit of include/bdfp4.h has the same value in
+    the binding, and the oracle's flags of the same arms share it (the parity
+    tests pass one integer to both sides); the oracle-only flag collides with none."""
+    import oracle
+    hdr = open(os.path.join(ROOT, "include", "bdfp4.h")).read()
+    defs = {m.group(1): int(m.group(2)) for m in re.finditer(r"#define BDFP4_((?:FLAG|DEV)_\w+) (\d+)", hdr)}
+    assert {"FLAG_NO_HADAMARD", "FLAG_DYNAMIC_ALPHA", "DEV_TIMEOUT"} <= set(defs)
+    for name, val in defs.items():
+        assert getattr(bdfp4, name) == val, name
+        if name.startswith("FLAG_"):
+            assert getattr(oracle, name) == val, name
+    assert oracle.FLAG_EXACT_P not in defs.values()
+    assert sorted(v for k, v in defs.items() if k.startswith("FLAG_")) == [1, 2, 4, 8, 32]
