@@ -188,14 +188,17 @@ def test_underflow_alpha_near_uniform(ora):
     q = wl.queries("cpu")
     cache, smooth, kg, vg = _quantized_cache(ora, wl, NV)
     outs = {}
-    for name, flags in (("exact_p", FLAG_EXACT_P), ("alpha_2^11", 0), ("alpha_1", FLAG_NO_UNDERFLOW)):
+    for name, flags in (("exact_p", FLAG_EXACT_P), ("alpha_2^11", 0), ("alpha_1", FLAG_NO_UNDERFLOW),
+                        ("alpha_per_tile", FLAG_DYNAMIC_ALPHA)):
         _, outs[name] = ora.decode(q, cache, wl.block_table, wl.seq_lens, sp.H_kv, sp.d_v, NV, smooth, kg, vg,
                                    sp.sm_scale, 1 << 20, wl.num_pages, flags=flags)
-    errs = {name: _rel(outs[name], outs["exact_p"]) for name in ("alpha_2^11", "alpha_1")}
+    errs = {name: _rel(outs[name], outs["exact_p"]) for name in ("alpha_2^11", "alpha_1", "alpha_per_tile")}
     REPORT["underflow_near_uniform_nvfp4"] = errs
     print(f"\nnear-uniform logits, 16384 tokens, error added by P quantization: alpha=2^11 "
-          f"{errs['alpha_2^11']:.5f}, alpha=1 {errs['alpha_1']:.5f}")
+          f"{errs['alpha_2^11']:.5f}, alpha=1 {errs['alpha_1']:.5f}, per-tile alpha {errs['alpha_per_tile']:.5f}")
     assert abs(errs["alpha_2^11"] - errs["alpha_1"]) <= 0.1 * errs["alpha_1"] + 1e-4
+    # every tile's largest p stays above 2688 / 4096 of the running maximum: the per-tile exponent is 11
+    assert np.array_equal(outs["alpha_per_tile"], outs["alpha_2^11"])
 
 
 def test_underflow_alpha_sink_stress(ora):
