@@ -51,8 +51,12 @@ def test_reference_arm_json_line():
 def test_reference_arm_under_torchrun_prints_once():
     """Launched as the driver launches it for N = 2: rank 0 alone runs the
     reference arm and prints its line; the other rank exits 0 without work."""
+    import socket
+    with socket.socket() as sock:
+        sock.bind(("127.0.0.1", 0))
+        port = sock.getsockname()[1]
     cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
-           "--master-addr", "127.0.0.1", "--master-port", "29531", os.path.join(ROOT, "bench.py"),
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.join(ROOT, "bench.py"),
            "--impl", "reference", "--config", "tiny", "--steps", "1", "--warmup", "0", "--gpus", "2"]
     out = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT)
     assert out.returncode == 0, out.stderr[-2000:]
