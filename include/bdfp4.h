@@ -217,7 +217,8 @@ BDFP4_API size_t bdfp4_decode_workspace_size(int B, int H_q, int d_v, int max_pa
  * into splits of chunk_tiles tiles; per tile p_t = exp(s_t - m_new), l sums the
  * unquantized p, and P is quantized in beta-token blocks (NVFP4: alpha = 2^11
  * underflow-aware pre-scale, divided out exactly; E4M3 block scale of
- * amax(alpha p) / 6, code 0 collapses the block; MXFP4: E8M0, alpha = 1);
+ * amax(alpha p) / 6, code 0 collapses the block; MXFP4: E8M0, alpha = 1;
+ * BDFP4_FLAG_DYNAMIC_ALPHA: alpha per tile and head, see the flag);
  * O accumulates P^ V; splits merge by log-sum-exp.  An empty sequence gives
  * zeros.  chunk_tiles <= 0 picks a plan from device seq_lens' upper bound
  * (max_pages_per_seq * 64).  workspace: >= bdfp4_decode_workspace_size bytes
