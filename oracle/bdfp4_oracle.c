@@ -741,8 +741,9 @@ int ora_quantize_q(const uint16_t* q, int B, int H_q, int H_kv, int d_k, int fmt
  *   exactly: scale code c = E4M3(amax_y / 6), code 0 = collapsed block,
  *   e_t = E2M1(y_t / E4M3(c)), P^_t = e_t E4M3(c) / alpha.  Vanilla ablation:
  *   alpha = 1.  MXFP4 (E8M0 scale, no underflow at these magnitudes): alpha = 1.
- *   Dynamic variant (NVFP4): the pages place the underflow at long contexts,
- *   where a tile far below the running maximum has only tiny probabilities.
+ *   Dynamic variant (NVFP4): the pages place the underflow at long contexts
+ *   ([BLOG] What is actually new; [SNS] Analyse approfondie), where a tile far
+ *   below the running maximum has only tiny probabilities.
  *   Reading: per tile and head, alpha = 2^E with E the largest integer such
  *   that p_max 2^E <= 2688 (= 6 x 448, so the largest block scale still fits
  *   E4M3), p_max the tile's largest p, E clamped to [11, 64] (64 also for
