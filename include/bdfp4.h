@@ -90,8 +90,11 @@ typedef enum { BDFP4_NVFP4 = 0, BDFP4_MXFP4 = 1 } bdfp4_fmt;
 #define BDFP4_FLAG_NO_SCALE_SEARCH 2 /* keys use the plain amax scale rule                               */
 #define BDFP4_FLAG_SINGLE_QUERY 4    /* vanilla single-FP4 query (q2 = 0)                               */
 #define BDFP4_FLAG_NO_UNDERFLOW 8    /* vanilla probability scaling (alpha = 1)                         */
-/* variant of the Underflow-Aware Probability Scaling (decode, NVFP4): the
- * probability pre-scale alpha = 2^E is chosen per 128-token tile and query head,
+/* Variant of the Underflow-Aware Probability Scaling (decode, NVFP4).  The
+ * collapse it guards against sits at long contexts ("FP4 KV Cache Done Right",
+ * What is actually new; "BitDecoding-FP4 : décodage natif du KV cache FP4",
+ * Analyse approfondie).  The probability pre-scale alpha = 2^E is chosen per
+ * 128-token tile and query head,
  * E the largest integer with p_max 2^E <= 2688 (p_max the tile's largest
  * probability relative to the running maximum), clamped to [11, 64]; each
  * tile's alpha is divided out of its quantized probabilities.  A tile that
