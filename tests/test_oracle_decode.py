@@ -289,6 +289,9 @@ def test_multi_token_queries_match_causal_textbook_attention(ora, T_q, seq_lens)
                     ref = p @ vf[off:off + vis, h // G] / p.sum()
                     assert np.allclose(o64[b, i, h], ref, rtol=0, atol=1e-6 * (np.abs(ref).max() + 1e-30))
             off += n
+    with pytest.raises(ValueError):   # a sequence shorter than its query tokens
+        ora.decode_multi(_bf16(q), cache, bt, np.full(len(seq_lens), T_q - 1), H_kv, d, ora.NVFP4, ones, g, g,
+                         sm_scale, 1, num_pages, flags=fl)
     if T_q == 1:
         o16m, _ = ora.decode_multi(_bf16(q), cache, bt, np.array(seq_lens), H_kv, d, ora.NVFP4, ones, g, g,
                                    sm_scale, 2, num_pages, flags=fl)
