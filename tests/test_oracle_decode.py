@@ -298,3 +298,28 @@ def test_multi_token_queries_match_causal_textbook_attention(ora, T_q, seq_lens)
         o16, _ = ora.decode(_bf16(q[:, 0]), cache, bt, np.array(seq_lens), H_kv, d, ora.NVFP4, ones, g, g,
                             sm_scale, 2, num_pages, flags=fl)
         assert np.array_equal(o16m[:, 0], o16)
+
+
+def test_kernel_exponent_bit_rule_equals_the_definition(ora):
+    """The decode kernels decide the per-tile exponent from p_max's fp32 bits
+    (p_max = m 2^e: E = 11 - e, less one when m > 1.3125, i.e. mantissa bits above
+    0x280000; clamped to [11, 64]; 64 for zero or subnormal p_max).  That rule,
+    written out here from its statement, equals the oracle's fp64 definition
+    for every fp32 exponent at the mantissas around the threshold."""
+    def bit_rule(p32):
+        u = int(np.float32(p32).view(np.uint32))
+        eb = (u >> 23) & 0xFF
+        if p32 <= 0 or eb == 0:
+            return 64
+        E = 11 - (eb - 127) - (1 if (u & 0x7FFFFF) > 0x280000 else 0)
+        return min(max(E, 11), 64)
+    rng = np.random.default_rng(3)
+    mants = [0, 1, 0x27FFFF, 0x280000, 0x280001, 0x400000, 0x7FFFFF] + list(rng.integers(0, 1 << 23, 8))
+    for eb in range(1, 128):          # p_max in [2^-126, 2^0]: every normal fp32 up to 1
+        for mt in mants:
+            if eb == 127 and mt:
+                continue              # p_max never exceeds 1
+            p = np.array([(eb << 23) | int(mt)], np.uint32).view(np.float32)[0]
+            assert bit_rule(p) == ora.dynamic_alpha_exp(float(p)), (eb, hex(int(mt)))
+    for p in (0.0, 1e-45, 1e-40):     # zero and subnormals
+        assert bit_rule(np.float32(p)) == ora.dynamic_alpha_exp(float(np.float32(p))) == 64
