@@ -8,12 +8,17 @@ decode attention for one query token per sequence (query transform +
 dual-residual FP4, paged tile fetch, QK^T, transposed softmax with fused
 underflow-aware P quantization, P.V, split merge).
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--config qwen3_4b]
-                  [--fmt nvfp4|mxfp4] [--impl ours|reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config qwen3_30b_a3b]
+                  [--fmt nvfp4|mxfp4] [--impl ours|reference] [--extra qwen3_4b,...]
 
 `value` is KV tokens per second (sum of context lengths per step / step
 time), device-timed with CUDA events; under torchrun each rank runs its own
 batch (weak scaling) and rank 0 reports the whole job over the slowest rank.
+Each timed block is exactly K steps between one CUDA event pair; blocks are
+repeated until they cover at least --min-region seconds (so the clock record
+holds many samples) and the median block is reported.  The default workload
+is the largest single-GPU one (Qwen3-30B-A3B-shaped); --extra adds decode
+figures of other workloads under "extra".
 `--impl reference` times the CPU oracle on a bounded sample instead.
 """
 from __future__ import annotations
@@ -84,6 +89,29 @@ def slowest_rank(times, device):
     t = torch.tensor(times, dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return t.tolist()
+
+
+def timed_blocks(fn, steps: int, stream, min_region_s: float, max_blocks: int = 1000) -> list:
+    """Seconds of blocks of exactly `steps` back-to-back calls of fn, each block
+    between one CUDA event pair on `stream` with a synchronize after it; blocks
+    repeat until together they cover min_region_s (at most max_blocks)."""
+    import torch
+    times = []
+    while True:
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) / 1e3)
+        if sum(times) >= min_region_s or len(times) >= max_blocks:
+            return times
+
+
+def median_step(times, steps: int) -> float:
+    return statistics.median(times) / steps
 
 
 class ClockSampler:
@@ -197,6 +225,59 @@ def setup_ours(sp, fmt, rank, device, with_bf16: bool = False):
                 bcache=bcache)
 
 
+def _peak():
+    peaks_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(peaks_path):
+        return json.load(open(peaks_path))["hbm_gbs"], "measured"
+    return 6650.0, "fallback"
+
+
+def measure_extra(args, name, fmt, flags, device, stream) -> dict:
+    """Decode figures of a second workload in the same run: the step, the decode
+    call and the BF16-KV comparator, each timed like the headline."""
+    import torch
+
+    from fp4_kv_cache_quant_b200 import bdfp4
+    from fp4_kv_cache_quant_b200.workloads import spec
+    sp = spec(name)
+    S = setup_ours(sp, fmt, 0, device, with_bf16=not args.no_bf16 and sp.d_k == 128)
+
+    def step():
+        bdfp4.bdfp4_decode_step(S["q"], S["new_k"], S["new_v"], S["v_open"], S["cache"], S["bt"], S["sl"], S["kv"],
+                                sp.sm_scale, S["chunk"], S["ws"], S["out"], flags=flags, dev_status=S["status"])
+
+    def decode_only():
+        bdfp4.bdfp4_decode(S["q"], S["cache"], S["bt"], S["sl"], S["kv"], sp.sm_scale, S["chunk"], S["ws"], S["out"],
+                           flags=flags, dev_status=S["status"])
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+        decode_only()
+    step_s = median_step(timed_blocks(step, args.steps, stream, args.min_region), args.steps)
+    dec_s = median_step(timed_blocks(decode_only, args.steps, stream, args.min_region), args.steps)
+    assert int(S["status"].item()) == 0, "device status set"
+    tokens = float(np.sum(S["wl"].seq_lens))
+    alg = algorithmic_bytes(sp, S["wl"].seq_lens, fmt)
+    peak, _ = _peak()
+    r = {"workload": CONFIG_TEXT[name], "name": name, "fmt": "nvfp4" if fmt == 0 else "mxfp4",
+         "chunk_tiles": S["chunk"], "kv_tokens_per_s": tokens / step_s, "ms_per_step": step_s * 1e3,
+         "decode_us": dec_s * 1e6, "hbm_gbs": alg / dec_s / 1e9, "frac": alg / dec_s / 1e9 / peak,
+         "algorithmic_bytes_per_launch": alg}
+    if S["bcache"] is not None:
+        bout = torch.empty_like(S["out"])
+
+        def bf16_decode():
+            bdfp4.bdfp4_bf16_decode(S["q"], S["bcache"], S["bt"], S["sl"], sp.sm_scale, S["chunk"], S["ws"], bout,
+                                    dev_status=S["status"])
+
+        for _ in range(max(args.warmup, 3)):
+            bf16_decode()
+        bf16_s = median_step(timed_blocks(bf16_decode, args.steps, stream, args.min_region), args.steps)
+        r["bf16_kv"] = {"decode_us": bf16_s * 1e6, "frac": bf16_algorithmic_bytes(sp, S["wl"].seq_lens) / bf16_s / 1e9
+                        / peak, "fp4_decode_speedup": bf16_s / dec_s}
+    return r
+
+
 def run_ours(args, sp, fmt):
     import torch
     import torch.distributed as dist
@@ -238,28 +319,17 @@ def run_ours(args, sp, fmt):
         dist.barrier()
     torch.cuda.synchronize()
     clocks.start()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for i in range(args.steps):
-        step(S["q"], S["new_k"], S["new_v"])
-    t1.record(stream)
-    torch.cuda.synchronize()
-    # the decode on its own (query images, decode kernel, merge) for the roofline: the same
-    # number of back-to-back calls on the same stream right after the steps, bracketed by one
-    # event pair like the steps, still under the clock sampler
-    d0 = torch.cuda.Event(enable_timing=True)
-    d1 = torch.cuda.Event(enable_timing=True)
-    d0.record(stream)
-    for i in range(args.steps):
-        decode_only()
-    d1.record(stream)
-    torch.cuda.synchronize()
+    # the steps: blocks of exactly K steps, repeated until they cover --min-region seconds
+    step_blocks = timed_blocks(lambda: step(S["q"], S["new_k"], S["new_v"]), args.steps, stream, args.min_region)
+    # the decode on its own (query images, decode kernel, merge) for the roofline: blocks of
+    # K back-to-back calls on the same stream right after the steps, still under the clock sampler
+    dec_blocks = timed_blocks(decode_only, args.steps, stream, args.min_region)
     clk = clocks.stop()
+    torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    step_s = t0.elapsed_time(t1) / 1e3 / args.steps
-    dec_s = d0.elapsed_time(d1) / 1e3 / args.steps
+    step_s = median_step(step_blocks, args.steps)
+    dec_s = median_step(dec_blocks, args.steps)
     assert int(S["status"].item()) == 0, "device status set"
 
     # the BF16-KV comparator on the same workload: decode calls timed alone
@@ -274,15 +344,8 @@ def run_ours(args, sp, fmt):
         for _ in range(max(args.warmup, 3)):
             bf16_decode()
         torch.cuda.synchronize()
-        # timed like the FP4 decode calls: K back-to-back calls, one event pair
-        b0 = torch.cuda.Event(enable_timing=True)
-        b1 = torch.cuda.Event(enable_timing=True)
-        b0.record(stream)
-        for i in range(args.steps):
-            bf16_decode()
-        b1.record(stream)
-        torch.cuda.synchronize()
-        bf16_s = b0.elapsed_time(b1) / 1e3 / args.steps
+        # timed like the FP4 decode calls
+        bf16_s = median_step(timed_blocks(bf16_decode, args.steps, stream, args.min_region), args.steps)
         assert int(S["status"].item()) == 0, "device status set"
 
     # end to end through the C ABI with host buffers: every step uploads its q and new keys
@@ -351,11 +414,7 @@ def run_ours(args, sp, fmt):
     # append and one CUDA-core decode; merge when a sequence can split
     launches_per_step = 2 + (1 if S["chunk"] < (wl.max_pages * 64 + 127) // 128 else 0)
     alg = algorithmic_bytes(sp, wl.seq_lens, fmt)
-    peaks_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(peaks_path):
-        peak, peak_src = json.load(open(peaks_path))["hbm_gbs"], "measured"
-    else:
-        peak, peak_src = 6650.0, "fallback"
+    peak, peak_src = _peak()
     traffic = None
     tr_path = os.path.join(ROOT, "profiles", "decode_traffic.json")
     # the variant runs on the tensor-core decode at d = 128, on the CUDA-core decode for MLA
@@ -383,6 +442,8 @@ def run_ours(args, sp, fmt):
                    "kv_tokens_per_step_per_gpu": int(tokens / world), "chunk_tiles": S["chunk"],
                    "parallelism": f"replicas x{world} (no data-path collective)",
                    "l2": f"inputs larger than L2 (FP4 cache {cache.nbytes() / 1e6:.0f} MB per GPU)",
+                   "timing": f"median of {len(step_blocks)} blocks of exactly {args.steps} steps (each block one "
+                             f"CUDA event pair), {sum(step_blocks):.3f} s of steps timed",
                    "accumulate": "fp32",
                    "probability_prescale": "dynamic per tile" if args.dynamic_alpha else "static 2^11"},
         "hbm_gbs": alg / dec_s / 1e9,
@@ -394,8 +455,8 @@ def run_ours(args, sp, fmt):
                                 ("decode_fp4_kernel" if cuda_core else
                                  "prep_query_kernel, decode_tc_kernel" if sp.d_k == 128 else
                                  "prep_mla_kernel, decode_mla_tc_kernel") +
-                                ", merge_splits_kernel): K back-to-back calls right after the step loop, "
-                                "one event pair"),
+                                ", merge_splits_kernel): median of blocks of K back-to-back calls right after the "
+                                "step blocks, one event pair per block"),
                      "peak_source": f"{peak_src} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
                      "algorithmic_bytes_per_launch": alg},
         "e2e": {"value": tokens / e2e_s, "unit": "tokens/s",
@@ -412,6 +473,11 @@ def run_ours(args, sp, fmt):
             "decode_us": bf16_s * 1e6, "kv_tokens_per_s": tokens / bf16_s, "hbm_gbs": b_alg / bf16_s / 1e9,
             "frac": b_alg / bf16_s / 1e9 / peak, "algorithmic_bytes_per_launch": b_alg,
             "fp4_decode_speedup": bf16_s / dec_s}
+    extra_names = [n for n in (args.extra.split(",") if args.extra else []) if n and n != args.config]
+    if rank == 0 and world == 1 and extra_names:
+        del S, cache, kv, wl
+        torch.cuda.empty_cache()
+        result["extra"] = [measure_extra(args, n, fmt, flags, device, stream) for n in extra_names]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(sp, fmt, budget_s=args.cpu_budget, flags=flags)
     if world > 1:
@@ -507,7 +573,11 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="qwen3_4b", choices=list(CONFIG_TEXT))
+    ap.add_argument("--config", default="qwen3_30b_a3b", choices=list(CONFIG_TEXT))
+    ap.add_argument("--extra", default="qwen3_4b",
+                    help="comma-separated workloads whose decode figures go under \"extra\" (N = 1 only)")
+    ap.add_argument("--min-region", type=float, default=0.5,
+                    help="seconds the repeated blocks of K timed steps cover at least")
     ap.add_argument("--fmt", default="nvfp4", choices=["nvfp4", "mxfp4"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0)

@@ -1,6 +1,11 @@
-"""Builds the in-tree CUDA library libbdfp4.so for B200 (sm_100a) with nvcc."""
+"""Builds the in-tree CUDA library libbdfp4.so for B200 (sm_100a) with nvcc.
+
+Each translation unit compiles to an object of its own, in parallel (one nvcc
+process per .cu file, under _build/ beside this file), and nvcc links them
+into the shared library."""
 from __future__ import annotations
 
+import concurrent.futures
 import glob
 import os
 import subprocess
@@ -9,23 +14,39 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libbdfp4.so")
+OBJ = os.path.join(HERE, "_build")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
-FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17", "-shared",
-         "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr"]
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+FLAGS = [*ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
+         "--expt-relaxed-constexpr"]
 
 
 def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
+def _headers() -> list[str]:
+    return glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) + \
+        glob.glob(os.path.join(HERE, "..", "include", "*.h"))
+
+
 def _stale() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) + \
-        glob.glob(os.path.join(HERE, "..", "include", "*.h"))
-    return any(os.path.getmtime(p) > t for p in deps)
+    return any(os.path.getmtime(p) > t for p in sources() + _headers())
+
+
+def _compile(src: str, extra: list[str], verbose: bool) -> tuple[str, str]:
+    obj = os.path.join(OBJ, os.path.basename(src)[:-3] + ".o")
+    cmd = [NVCC, *FLAGS, *extra, "-c", "-o", obj, src]
+    if verbose:
+        print(" ".join(cmd), flush=True)
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    if r.returncode != 0:
+        raise RuntimeError(f"nvcc failed on {os.path.basename(src)}:\n{r.stdout}{r.stderr}")
+    return obj, r.stdout + r.stderr
 
 
 def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None, out: str | None = None) -> str:
@@ -33,9 +54,15 @@ def build(force: bool = False, verbose: bool = False, extra: list[str] | None = 
     target = out or LIB
     if not force and out is None and not _stale():
         return LIB
-    cmd = [NVCC, *FLAGS, *(extra or []), "-o", target + ".tmp", *sources()]
+    os.makedirs(OBJ, exist_ok=True)
+    srcs = sources()
+    with concurrent.futures.ThreadPoolExecutor(max_workers=max(1, min(len(srcs), os.cpu_count() or 1))) as ex:
+        results = list(ex.map(lambda s: _compile(s, extra or [], verbose), srcs))
     if verbose:
-        print(" ".join(cmd), flush=True)
+        for _, log in results:
+            if log.strip():
+                print(log, end="", flush=True)
+    cmd = [NVCC, *ARCH, "-shared", "-Xcompiler", "-fPIC", "-o", target + ".tmp", *[o for o, _ in results]]
     subprocess.run(cmd, check=True)
     os.replace(target + ".tmp", target)
     return target

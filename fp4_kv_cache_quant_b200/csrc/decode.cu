@@ -190,13 +190,16 @@ __global__ void __launch_bounds__(kThreads) decode_fp4_kernel(const DecodeArgs a
         for (int g = 0; g < HG; ++g) {
             const float mt = fmaxf(fmaxf(red[0][g], red[1][g]), fmaxf(red[2][g], red[3][g]));
             const float mn = fmaxf(m_run[g], mt);
-            corr[g] = exp2f(m_run[g] - mn);   // 0 on the split's first tile
+            // a split whose tiles so far hold only masked tokens (bad pages) keeps m = -inf:
+            // take 0 as the reference there, so corr and p are 0 rather than NaN
+            const float mz = mn == -INFINITY ? 0.0f : mn;
+            corr[g] = exp2f(m_run[g] - mz);   // 0 on the split's first tile
             m_run[g] = mn;
-            p[g] = valid ? exp2f(s[g] - mn) : 0.0f;
+            p[g] = valid ? exp2f(s[g] - mz) : 0.0f;
             l_part[g] = l_part[g] * corr[g] + p[g];
             float ag = alpha, ig = 1.0f;
             if (dyn) {
-                const int E = dynamic_alpha_exp(exp2f(mt - mn));   // the tile's largest p
+                const int E = dynamic_alpha_exp(exp2f(mt - mz));   // the tile's largest p
                 ag = pow2f(E);
                 ig = pow2f(-E);
             }
@@ -305,8 +308,7 @@ static int max_splits_for(int max_pages, int chunk_tiles) {
 
 // Workspace regions: split partials (fp32 O, then (m, l)) when a sequence can
 // have more than one split, then the query images of the tensor-core path
-// (at most kQueryImageBytes per query head: 640 at d_k = 128, 652 for MLA).
-constexpr size_t kQueryImageBytes = 656;
+// (at most kQueryImageBytes per query head: 592 at d_k = 128, 652 for MLA).
 
 struct WorkspaceMap {
     size_t o_bytes, ml_bytes, q_off, total;
@@ -318,7 +320,7 @@ static WorkspaceMap workspace_map(int B, int H_q, int d_v, int max_splits) {
     m.o_bytes = (size_t)B * H_q * ms * d_v * sizeof(float);
     m.ml_bytes = (size_t)B * H_q * ms * 2 * sizeof(float);
     m.q_off = ((m.o_bytes + 255) / 256) * 256 + ((m.ml_bytes + 255) / 256) * 256;
-    m.total = m.q_off + (size_t)B * H_q * kQueryImageBytes;
+    m.total = m.q_off + (size_t)B * H_q * (size_t)kQueryImageBytes;
     return m;
 }
 

@@ -46,6 +46,11 @@ struct StepArgs {
 constexpr int kThreads = 128;
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Workspace bytes reserved per query head for the query images of the
+// tensor-core decodes (an image of a (sequence, KV head) or head slice of h
+// heads takes at most h times this; each layout static_asserts it).
+constexpr int kQueryImageBytes = 656;
+
 // Splits of a sequence of N tokens.
 __host__ __device__ __forceinline__ int num_splits(int N, int chunk_tiles) {
     const int ntiles = (N + kTileTokens - 1) / kTileTokens;

@@ -101,6 +101,8 @@ struct MlaCfg {
     static_assert(T_USED <= T_ALLOC, "TMEM budget");
     static_assert(SMEM <= 232448 && SMEM > 232448 / 2, "one CTA per SM");
     static_assert(QPACK % 16 == 0, "query image copied in 16-byte units");
+    // the image of a head slice fits the workspace region reserved for its heads
+    static_assert(QPACK <= kQueryImageBytes * GH, "query image larger than its workspace share");
     static_assert(NSG + 2 <= 16, "named barriers");
 };
 

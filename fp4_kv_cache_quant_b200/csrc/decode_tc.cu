@@ -125,6 +125,9 @@ struct TcCfg {
     static constexpr int MAX_CTAS = 512 / T_ALLOC;
     static constexpr int SMEM_MIN = 233472 / (MAX_CTAS + 1) - 1024 + 16;
     static constexpr int SMEM_LAUNCH = SMEM > SMEM_MIN ? SMEM : SMEM_MIN;
+    // the query image of a (sequence, KV head) fits the workspace region reserved for it
+    static_assert(QPACK <= kQueryImageBytes * G, "query image larger than its workspace share");
+    static_assert(QPACK % 16 == 0, "query image copied in 16-byte units");
 };
 
 constexpr long long kWaitLimit = 1LL << 32;   // clock cycles (about 2 s)

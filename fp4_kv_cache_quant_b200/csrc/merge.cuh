@@ -37,6 +37,10 @@ __global__ void __launch_bounds__(128) merge_splits_kernel(const float* __restri
     if (lane == 0) red[0][wid] = M;
     __syncthreads();
     M = fmaxf(fmaxf(red[0][0], red[0][1]), fmaxf(red[0][2], red[0][3]));
+    // every split saw only masked tokens (all of the sequence's pages bad): m = -inf
+    // everywhere, so take 0 as the reference -- the weights become 0, L = 0 and the
+    // row is written as zeros, as a single-split row is
+    if (M == -INFINITY) M = 0.0f;
     float Lp = 0.0f;
     for (int s = threadIdx.x; s < ns; s += blockDim.x) {
         const float w = exp2f(ml[2 * s] - M);

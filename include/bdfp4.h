@@ -279,6 +279,9 @@ BDFP4_API int bdfp4_decode_step(const void* q, const void* k_new, const void* v_
  *  - The first call on each device looks up the scratch array's device
  *    address (cudaGetSymbolAddress) with that device current; make that first
  *    call before any stream capture.  A failed lookup returns BDFP4_ERR_CUDA.
+ *    The address is kept for the life of the process: it does not survive a
+ *    cudaDeviceReset (or any other teardown of the device's primary context),
+ *    after which this entry point must not be called again in that process.
  *  - All calls share the one array and it keeps the last call's contents (no
  *    part of it needs to start at zero: every partial is written before it is
  *    read).  Calls that overlap on the GPU -- on different streams, or from

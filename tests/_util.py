@@ -29,21 +29,39 @@ def bf16_ulp(x: np.ndarray) -> np.ndarray:
 
 
 def compare_outputs(gpu: np.ndarray, ref: np.ndarray):
-    """-> (max_abs, rel_l2) of bf16 outputs against the oracle's bf16 outputs.
+    """-> (max_abs, rel_l2, step_frac) of bf16 outputs against the oracle's bf16 outputs.
 
     Both sides round an fp32 / fp64 result to bf16 at the end, so two results
     that straddle a bf16 rounding boundary land one bf16 step apart; above
     magnitude 2 that step is larger than the 1e-2 bound (2^-6 at [2, 4), 2^-3 at
     [16, 32) -- the MLA workload's outlier value channels reach there).  An
     element one step or less from the oracle's therefore counts as agreeing;
-    max_abs is the largest difference among the others."""
+    max_abs is the largest difference among the others, and step_frac is the
+    fraction of elements that needed that allowance (more than 1e-2 apart but
+    within one step)."""
     g = gpu.astype(np.float64)
     r = ref.astype(np.float64)
     d = np.abs(g - r)
-    d = np.where(d <= bf16_ulp(r), 0.0, d)
+    step = d <= bf16_ulp(r)
+    d = np.where(step, 0.0, d)
     max_abs = float(np.max(d)) if g.size else 0.0
     rel = float(np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-30))
-    return max_abs, rel
+    step_frac = float(np.count_nonzero(step & (np.abs(g - r) > MAX_ABS)) / g.size) if g.size else 0.0
+    return max_abs, rel, step_frac
+
+
+# Largest fraction of elements that may use the one-bf16-step allowance of
+# compare_outputs: a rounding straddle is rare, so a kernel off by one step on
+# many large outputs fails even though each element alone would pass.
+STEP_FRAC = 1e-3
+
+
+def assert_close(gpu: np.ndarray, ref: np.ndarray, *ctx):
+    """The decode bound: max-abs 1e-2 (one-step allowance as in compare_outputs),
+    relative L2 5e-3, and at most STEP_FRAC of the elements on the allowance."""
+    max_abs, rel, step_frac = compare_outputs(gpu, ref)
+    assert max_abs <= MAX_ABS and rel <= REL_L2 and step_frac <= STEP_FRAC, (*ctx, max_abs, rel, step_frac)
+    return max_abs, rel, step_frac
 
 
 def kv_params_np(kv: bdfp4.KVParams):

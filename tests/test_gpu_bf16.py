@@ -9,7 +9,7 @@ import numpy as np
 import pytest
 import torch
 
-from _util import MAX_ABS, REL_L2, compare_outputs, out_to_np
+from _util import assert_close, out_to_np
 from fp4_kv_cache_quant_b200 import bdfp4
 from fp4_kv_cache_quant_b200.workloads import Workload, spec
 
@@ -83,8 +83,7 @@ def test_bf16_decode_matches_oracle(ora, name, chunk):
     got = out_to_np(out)
     ref = ora.attention_ref(q, wl.all_keys(), wl.all_values(), wl.cu_seqlens, sp.H_kv, sp.sm_scale)
     assert np.all(np.isfinite(got))
-    max_abs, rel = compare_outputs(got, ref)
-    assert max_abs <= MAX_ABS and rel <= REL_L2, (max_abs, rel)
+    assert_close(got, ref)
     for b, n in enumerate(wl.seq_lens):
         if n == 0:
             assert np.all(got[b] == 0)
@@ -116,5 +115,4 @@ def test_bf16_decode_full_size_sampled(ora):
         n = int(wl.seq_lens[b])
         ref = ora.attention_ref(q[b:b + 1], wl.keys(b), wl.values(b), np.array([0, n], np.int64), sp.H_kv,
                                 sp.sm_scale)
-        max_abs, rel = compare_outputs(got[b:b + 1], ref)
-        assert max_abs <= MAX_ABS and rel <= REL_L2, (b, max_abs, rel)
+        assert_close(got[b:b + 1], ref, b)

@@ -44,10 +44,13 @@ def _pages(seq_lens, rng):
     return bt, num_pages, np.concatenate(slots) if slots else np.zeros(0, np.int64)
 
 
-def _exact_case(rng, seq_lens, H_q, H_kv, d, fmt=0):
+def _exact_case(rng, seq_lens, H_q, H_kv, d, fmt=0, d_v=None):
+    """q [B, H_q, d], k [T, H_kv, d] and v [T, H_kv, d_v] (d_v = d unless given)
+    that the format represents exactly with unit tensor scales."""
     beta = 16 if fmt == 0 else 32
+    d_k, d = d, (d if d_v is None else d_v)
     T = int(sum(seq_lens))
-    k = _exact_fp4(rng, (T, H_kv), beta, d)
+    k = _exact_fp4(rng, (T, H_kv), beta, d_k)
     # V blocks run along tokens: build per (head, channel) along the token axis,
     # block-aligned per sequence (pages start at token 0 of each sequence)
     v = np.zeros((T, H_kv, d), np.float32)
@@ -68,7 +71,7 @@ def _exact_case(rng, seq_lens, H_q, H_kv, d, fmt=0):
                         blk[h, c, 0] = val
             v[off: off + n] = np.transpose(vv, (2, 0, 1))[:n]
         off += n
-    q = _exact_fp4(rng, (len(seq_lens), H_q), beta, d)
+    q = _exact_fp4(rng, (len(seq_lens), H_q), beta, d_k)
     return q, k, v
 
 
@@ -109,6 +112,39 @@ def test_exact_inputs_match_textbook_attention(ora, G, seq_lens):
     for b, n in enumerate(seq_lens):
         if n == 0:
             assert np.all(outs[0][b] == 0)
+
+
+@pytest.mark.parametrize("fmt", [0, 1])
+def test_exact_inputs_match_textbook_attention_latent_geometry(ora, fmt):
+    """The MLA geometry: keys of d_k = 576 (512 latent + 64 rope channels), values of
+    d_v = 512, sixteen query heads over one KV head.  An index slip between d_k and
+    d_v (key rows, value rows, their scale bytes) breaks the equality."""
+    rng = np.random.default_rng(576 + fmt)
+    seq_lens = [130, 0, 300]
+    H_kv, H_q, d_k, d_v = 1, 16, 576, 512
+    q, k, v = _exact_case(rng, seq_lens, H_q, H_kv, d_k, fmt, d_v=d_v)
+    bt, num_pages, sm = _pages(seq_lens, rng)
+    ones = np.ones((H_kv, d_k), np.float32)
+    g = np.ones(H_kv, np.float32)
+    cache = ora.empty_cache(num_pages, H_kv, d_k, d_v, fmt)
+    fl = ora.FLAG_NO_HADAMARD
+    ora.quantize_kv(_bf16(k), _bf16(v), sm, cache, H_kv, fmt, ones, g, g, num_pages, flags=fl)
+    t = 0
+    for b, n in enumerate(seq_lens):
+        for i in range(0, n, 29):
+            page, slot = bt[b, i // 64], i % 64
+            assert np.array_equal(ora.dequant_key_row(cache, fmt, page, 0, H_kv, d_k, slot), k[t + i, 0])
+            assert np.array_equal(ora.dequant_value_row(cache, fmt, page, 0, H_kv, d_v, slot), v[t + i, 0])
+        t += n
+    sm_scale = 1 / math.sqrt(d_k) / 8
+    cu = np.concatenate([[0], np.cumsum(seq_lens)])
+    ref = ora.attention_ref(_bf16(q), _bf16(k), _bf16(v), cu, H_kv, sm_scale)
+    assert ref.shape == (len(seq_lens), H_q, d_v)
+    for chunk in (1, 1000):
+        _, o64 = ora.decode(_bf16(q), cache, bt, np.array(seq_lens), H_kv, d_v, fmt, ones, g, g, sm_scale, chunk,
+                            num_pages, flags=fl | ora.FLAG_EXACT_P)
+        assert np.max(np.abs(o64 - ref)) <= 1e-6 * (np.abs(ref).max() + 1e-30), chunk
+        assert np.all(o64[1] == 0)
 
 
 def _uniform_case(ora, fmt, flags):
