@@ -29,7 +29,7 @@ PAGE_SLOTS = 64
 TILE_TOKENS = 128
 
 #: names of every entry point declared in include/bdfp4.h
-ENTRY_POINTS = ("bdfp4_calibrate", "bdfp4_quantize_kv", "bdfp4_quantize_k", "bdfp4_quantize_v", "bdfp4_quantize_q", "bdfp4_decode_plan",
+ENTRY_POINTS = ("bdfp4_calibrate", "bdfp4_key_weights", "bdfp4_quantize_kv", "bdfp4_quantize_k", "bdfp4_quantize_v", "bdfp4_quantize_q", "bdfp4_decode_plan",
                 "bdfp4_decode_plan_for",
                 "bdfp4_decode_workspace_size", "bdfp4_decode", "bdfp4_decode_step", "bdfp4_decode_noalloc",
                 "bdfp4_status_string", "bdfp4_last_error")
@@ -45,7 +45,8 @@ class BDFP4Error(RuntimeError):
 
 
 class _KVParams(ctypes.Structure):
-    _fields_ = [("smooth", ctypes.c_void_p), ("k_gscale", ctypes.c_void_p), ("v_gscale", ctypes.c_void_p)]
+    _fields_ = [("smooth", ctypes.c_void_p), ("k_gscale", ctypes.c_void_p), ("v_gscale", ctypes.c_void_p),
+                ("k_weight", ctypes.c_void_p)]
 
 
 _lib = None
@@ -63,6 +64,8 @@ def load() -> ctypes.CDLL:
     kvp = ctypes.POINTER(_KVParams)
     L.bdfp4_calibrate.argtypes = [p, p, p, i, i, i, i, i, i, i, p, p, p, p]
     L.bdfp4_calibrate.restype = i
+    L.bdfp4_key_weights.argtypes = [p, i, i, i, i, i, p, p, p]
+    L.bdfp4_key_weights.restype = i
     L.bdfp4_quantize_kv.argtypes = [p, p, p, i, i, i, i, i, i, kvp, p, p, p, p, i64, p, p]
     L.bdfp4_quantize_kv.restype = i
     L.bdfp4_quantize_k.argtypes = [p, p, i, i, i, i, i, kvp, p, p, i64, p, p]
@@ -129,13 +132,16 @@ def beta(fmt: int) -> int:
 
 @dataclass
 class KVParams:
-    """Static per-layer parameters: smoothing factors and FP32 tensor scales."""
+    """Static per-layer parameters: smoothing factors, FP32 tensor scales and,
+    optionally, the channel weights of the attention-aware key scale search."""
     smooth: torch.Tensor    # [H_kv, d_k] fp32
     k_gscale: torch.Tensor  # [H_kv] fp32
     v_gscale: torch.Tensor  # [H_kv] fp32
+    k_weight: torch.Tensor | None = None   # [H_kv, d_k] fp32 (bdfp4_key_weights) or None
 
     def _c(self) -> _KVParams:
-        return _KVParams(self.smooth.data_ptr(), self.k_gscale.data_ptr(), self.v_gscale.data_ptr())
+        return _KVParams(self.smooth.data_ptr(), self.k_gscale.data_ptr(), self.v_gscale.data_ptr(),
+                         None if self.k_weight is None else self.k_weight.data_ptr())
 
 
 @dataclass
@@ -174,6 +180,17 @@ def bdfp4_calibrate(k_cal: torch.Tensor, q_cal: torch.Tensor, v_cal: torch.Tenso
                                 _ptr(kv.smooth), _ptr(kv.k_gscale), _ptr(kv.v_gscale), _stream(stream))
     _check(rc, "bdfp4_calibrate")
     return kv
+
+
+def bdfp4_key_weights(q_cal: torch.Tensor, H_kv: int, smooth: torch.Tensor, flags: int = 0,
+                      stream=None) -> torch.Tensor:
+    """[H_kv, d_k] channel weights of the attention-aware key scale search from
+    calibration queries q_cal [Tq, H_q, d_k] (bdfp4_key_weights in bdfp4.h)."""
+    Tq, H_q, d_k = q_cal.shape
+    w = torch.empty((H_kv, d_k), dtype=torch.float32, device=q_cal.device)
+    rc = load().bdfp4_key_weights(_ptr(q_cal), Tq, H_q, H_kv, d_k, flags, _ptr(smooth), _ptr(w), _stream(stream))
+    _check(rc, "bdfp4_key_weights")
+    return w
 
 
 def bdfp4_quantize_kv(k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor, kv: KVParams, cache: FP4Cache,

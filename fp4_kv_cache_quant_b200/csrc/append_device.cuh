@@ -11,20 +11,16 @@
 namespace bdfp4 {
 
 // ---------------------------------------------------------------- keys
-// Work split of the K append: every scale block of a row gets NC lanes, one per
-// candidate code of its search window (10 for NVFP4, 2 for MXFP4, padded), so
-// the window is searched in parallel; R rows share a 256-thread CTA.
+// Work split of the K append: one thread per scale block of a row (its beta
+// channels), R rows per 256-thread CTA; the thread transforms its block and
+// searches the block's whole window itself, so nothing leaves registers.
 template <int FMT, int DK>
 struct KGeom {
     using RG = RowGeom<FMT, DK>;
     static constexpr int B = RG::beta;
     static constexpr int NB = DK / B;                                  // scale blocks per row
-    static constexpr int NC = FMT == BDFP4_NVFP4 ? 16 : 2;             // candidate lanes per block
-    static constexpr int R = 256 / (NB * NC) >= 1 ? 256 / (NB * NC) : 1;
-    static constexpr int PAIRS = R * NB * NC;                           // (block, candidate) pairs
-    static constexpr int PAIRS_PAD = (PAIRS + 255) / 256 * 256;
-    static constexpr int T1 = (R * RG::rt + 31) / 32 * 32;             // transform threads (whole warps)
-    static_assert(T1 <= 256, "transform threads exceed the CTA");
+    static constexpr int R = 256 / RG::rt;                             // rows per CTA
+    static_assert(256 % RG::rt == 0, "rows tile the CTA");
 };
 
 // Slot of token t from a slot mapping (page * 64 + slot, negative = skip);
@@ -66,111 +62,66 @@ struct NewestSlot {
 };
 
 // Key rows [blk * R, blk * R + R) of k [rows / H_kv][H_kv][DK] (row = token *
-// H_kv + head).  Phase 1 transforms the rows into shared memory (thread per
-// block, butterflies across the row's threads); phase 2 quantizes every block
-// under every code of its window and keeps the fp64 squared errors (each
-// summed left to right); phase 3 scans each window from its largest code down,
-// keeping the first least error, and stores the winner.  The choice is the
-// sequential search's.
+// H_kv + head).  Each thread transforms its scale block (butterflies across
+// the row's threads, which share a warp), then quantizes the block under every
+// code of its window in turn, keeping the least fp64 squared error (summed left
+// to right; with k_weight, each element's term weighted by its channel's
+// weight) and the larger code on a tie -- the sequential search -- and stores
+// the winner.  k_weight [H_kv][DK] or null (the plain objective).
 template <int FMT, int DK, class SlotOf>
 __device__ __forceinline__ void append_k_cta(int blk, const __nv_bfloat16* __restrict__ k, int64_t rows, int H_kv,
                                              const SlotOf& slot_of, const float* __restrict__ smooth,
-                                             const float* __restrict__ k_gscale, uint8_t* k_pages,
-                                             uint8_t* k_scales, int flags) {
+                                             const float* __restrict__ k_gscale, const float* __restrict__ k_weight,
+                                             uint8_t* k_pages, uint8_t* k_scales, int flags) {
     using KG = KGeom<FMT, DK>;
     using RG = typename KG::RG;
-    constexpr int B = KG::B, NB = KG::NB, NC = KG::NC, R = KG::R;
-    __shared__ float xs[R][DK];
-    __shared__ double errs[KG::PAIRS_PAD];
-    __shared__ uint32_t pks[KG::PAIRS_PAD][B / 8];
-    __shared__ int win[R * NB];            // hi << 16 | lo
-    __shared__ long long slots[R];
-    __shared__ float gs[R];                // tensor scale of the row's head
-    const int tid = threadIdx.x;
-    const int64_t row0 = (int64_t)blk * R;
-
-    if (tid < KG::T1) {
-        const int r = tid / RG::rt, j = tid % RG::rt;
-        const int64_t row = row0 + r;
-        const bool in_range = r < R && row < rows;
-        const int t = (int)(in_range ? row / H_kv : 0);
-        const int h = (int)(in_range ? row % H_kv : 0);
-        const int64_t sm = in_range ? slot_of(t, j == 0) : -1;
-        // whole warps stay converged through the shuffles; inactive rows compute on zeros
-        // the row is loaded whatever its slot id, so the two loads overlap
-        float x[B];
-        if (in_range && j < RG::tpr) {
-            load_bf16_block<B>(k + ((int64_t)t * H_kv + h) * DK, j * B, x);
-        } else {
+    constexpr int B = KG::B;
+    const int r = threadIdx.x / RG::rt, j = threadIdx.x % RG::rt;
+    const int64_t row = (int64_t)blk * KG::R + r;
+    const bool in_range = row < rows;
+    const int t = (int)(in_range ? row / H_kv : 0);
+    const int h = (int)(in_range ? row % H_kv : 0);
+    const int64_t sm = in_range ? slot_of(t, j == 0) : -1;
+    // whole warps stay converged through the shuffles; inactive rows compute on zeros.
+    // The row is loaded whatever its slot id, so the two loads overlap
+    float x[B];
+    if (in_range && j < RG::tpr) {
+        load_bf16_block<B>(k + ((int64_t)t * H_kv + h) * DK, j * B, x);
+    } else {
 #pragma unroll
-            for (int i = 0; i < B; ++i) x[i] = 0.0f;
-        }
-        if (sm < 0) {
-#pragma unroll
-            for (int i = 0; i < B; ++i) x[i] = 0.0f;
-        }
-        const bool active = sm >= 0 && j < RG::tpr;
-        transform_block<FMT, DK, true>(x, smooth + (int64_t)h * DK, j, !(flags & BDFP4_FLAG_NO_HADAMARD));
-        if (active) {
-#pragma unroll
-            for (int i = 0; i < B; ++i) xs[r][j * B + i] = x[i];
-        }
-        if (r < R && j == 0) {
-            slots[r] = sm;
-            gs[r] = FMT == BDFP4_NVFP4 ? __ldg(k_gscale + h) : 1.0f;
-        }
+        for (int i = 0; i < B; ++i) x[i] = 0.0f;
     }
-    __syncthreads();
-
-    for (int p = tid; p < KG::PAIRS; p += 256) {
-        const int r = p / (NB * NC), bk = (p / NC) % NB, ci = p % NC;
-        if (slots[r] < 0) continue;
-        const float g = gs[r];
-        float x[B];
+    if (sm < 0) {
 #pragma unroll
-        for (int i = 0; i < B; ++i) x[i] = xs[r][bk * B + i];
-        const float amax = block_amax<B>(x);
-        const int c0 = (int)plain_scale_code<FMT>(amax, g);
-        int hi = c0, lo = c0;   // all-zero blocks and the plain rule keep c0
-        if (amax != 0.0f && !(flags & BDFP4_FLAG_NO_SCALE_SEARCH)) {
-            const int top = FMT == BDFP4_NVFP4 ? 126 : 254;
-            hi = min(c0 + (FMT == BDFP4_NVFP4 ? 7 : 1), top);
-            lo = max(c0 - (FMT == BDFP4_NVFP4 ? 2 : 0), 0);
-        }
-        if (ci == 0) win[r * NB + bk] = (hi << 16) | lo;
-        const int c = hi - ci;
-        if (c >= lo) errs[p] = quantize_block<B>(x, block_sigma<FMT>((uint32_t)c, g), pks[p]);
+        for (int i = 0; i < B; ++i) x[i] = 0.0f;
     }
-    __syncthreads();
-
-    for (int q = tid; q < R * NB; q += 256) {
-        const int r = q / NB, bk = q % NB;
-        const int64_t sm = slots[r];
-        if (sm < 0) continue;
-        const int h = (int)((row0 + r) % H_kv);
-        const int hi = win[q] >> 16, lo = win[q] & 0xffff;
-        const int base = q * NC;
-        int best = 0;
-        double best_err = errs[base];
-        for (int ci = 1; ci <= hi - lo; ++ci) {
-            if (errs[base + ci] < best_err) {
-                best = ci;
-                best_err = errs[base + ci];
-            }
-        }
-        const int64_t page = sm / kPageSlots;
-        const int slot = (int)(sm % kPageSlots);
-        uint8_t* kp = k_pages + (page * H_kv + h) * (int64_t)(kPageSlots * DK / 2);
-        uint8_t* dst = kp + k_nib_offset(DK, slot, bk * B);
-        const uint32_t* pk = pks[base + best];
-        if constexpr (B == 16) {
-            *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
-        } else {
-            *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        }
-        uint8_t* ks = k_scales + (page * H_kv + h) * (int64_t)k_scale_page_bytes(DK, B);
-        ks[k_scale_offset<B>(DK, slot, bk)] = (uint8_t)(hi - best);
+    transform_block<FMT, DK, true>(x, smooth + (int64_t)h * DK, j, !(flags & BDFP4_FLAG_NO_HADAMARD));
+    if (sm < 0 || j >= RG::tpr) return;
+    const float g = FMT == BDFP4_NVFP4 ? __ldg(k_gscale + h) : 1.0f;
+    uint32_t pk[B / 8];
+    uint32_t code;
+    if (flags & BDFP4_FLAG_NO_SCALE_SEARCH) {
+        code = plain_scale_code<FMT>(block_amax<B>(x), g);
+        quantize_block<B>(x, block_sigma<FMT>(code, g), pk);
+    } else if (k_weight) {
+        float w[B];
+#pragma unroll
+        for (int i = 0; i < B; ++i) w[i] = __ldg(k_weight + (int64_t)h * DK + j * B + i);
+        code = search_scale<FMT, true>(x, g, w, pk);
+    } else {
+        code = search_scale<FMT, false>(x, g, nullptr, pk);
     }
+    const int64_t page = sm / kPageSlots;
+    const int slot = (int)(sm % kPageSlots);
+    uint8_t* kp = k_pages + (page * H_kv + h) * (int64_t)(kPageSlots * DK / 2);
+    uint8_t* dst = kp + k_nib_offset(DK, slot, j * B);
+    if constexpr (B == 16) {
+        *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
+    } else {
+        *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    }
+    uint8_t* ks = k_scales + (page * H_kv + h) * (int64_t)k_scale_page_bytes(DK, B);
+    ks[k_scale_offset<B>(DK, slot, j)] = (uint8_t)code;
 }
 
 // ---------------------------------------------------------------- values

@@ -450,6 +450,7 @@ static int run_decode(const void* q, const void* k_pages, const void* k_scales, 
     a.smooth = kv->smooth;
     a.k_gscale = kv->k_gscale;
     a.v_gscale = kv->v_gscale;
+    a.k_weight = kv->k_weight;
     a.out = (__nv_bfloat16*)out;
     a.dev_status = dev_status;
     a.B = B;

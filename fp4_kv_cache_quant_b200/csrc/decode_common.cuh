@@ -19,6 +19,7 @@ struct DecodeArgs {
     const float* smooth;
     const float* k_gscale;
     const float* v_gscale;
+    const float* k_weight;   // [H_kv][d_k] channel weights of the key scale search, or null
     float* ws_o;   // [B][H_q][max_splits][d_v] unnormalised partial outputs
     float* ws_ml;  // [B][H_q][max_splits][2]  (m in log2 units, l)
     uint8_t* qpack;  // [B][H_kv] query images of the tensor-core path (written before the decode)

@@ -172,7 +172,7 @@ __global__ void __launch_bounds__(256) prep_mla_kernel(const DecodeArgs a, const
         const NewestSlot slot{a.block_table, a.seq_lens, a.max_pages, a.num_pages, a.dev_status};
         const int nk = (int)k_append_ctas<FMT, 576>(rows), nv = (int)v_append_ctas<512>(rows);
         if (blk < nk) {
-            append_k_cta<FMT, 576>(blk, s.k_new, rows, a.H_kv, slot, a.smooth, a.k_gscale, s.k_pages, s.k_scales,
+            append_k_cta<FMT, 576>(blk, s.k_new, rows, a.H_kv, slot, a.smooth, a.k_gscale, a.k_weight, s.k_pages, s.k_scales,
                                    a.flags);
             return;
         }

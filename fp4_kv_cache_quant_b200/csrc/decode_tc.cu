@@ -212,7 +212,8 @@ __global__ void __launch_bounds__(256) prep_step_kernel(const DecodeArgs a, cons
     const int nk = (int)k_append_ctas<FMT, 128>(rows), nv = (int)v_append_ctas<128>(rows);
     const int blk = blockIdx.x;
     if (blk < nk) {
-        append_k_cta<FMT, 128>(blk, s.k_new, rows, a.H_kv, slot, a.smooth, a.k_gscale, s.k_pages, s.k_scales, a.flags);
+        append_k_cta<FMT, 128>(blk, s.k_new, rows, a.H_kv, slot, a.smooth, a.k_gscale, a.k_weight, s.k_pages, s.k_scales,
+                               a.flags);
     } else if (blk < nk + nv) {
         append_v_open_cta<FMT, 128>(blk - nk, s.v_new, s.v_open, slot, a.B, a.H_kv, a.v_gscale, s.v_pages,
                                     s.v_scales);

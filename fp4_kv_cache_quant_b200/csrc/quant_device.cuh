@@ -73,20 +73,28 @@ __device__ __forceinline__ void transform_block(float* x, const float* smooth_ro
 
 // E2M1 codes of x / sigma (sigma = 0 -> zeros), packed two per byte (even
 // element low), and the block's squared error summed left to right in fp64.
-template <int B>
-__device__ __forceinline__ double quantize_block(const float* x, float sigma, uint32_t* packed /* B/8 words */) {
+// With W, element i's squared error is weighted: w[i] * (d_i * d_i).
+template <int B, bool W = false>
+__device__ __forceinline__ double quantize_block(const float* x, float sigma, uint32_t* packed /* B/8 words */,
+                                                 const float* w = nullptr) {
     double err = 0.0;
 #pragma unroll
-    for (int w = 0; w < B / 8; ++w) packed[w] = 0u;
+    for (int k = 0; k < B / 8; ++k) packed[k] = 0u;
 #pragma unroll
     for (int i = 0; i < B; i += 2) {
         uint32_t pair = 0u;
         if (sigma != 0.0f) pair = e2m1x2_encode(__fdiv_rn(x[i], sigma), __fdiv_rn(x[i + 1], sigma));
         packed[i / 8] |= pair << (4 * (i % 8));
-        double d0 = __dsub_rn((double)x[i], __dmul_rn((double)e2m1_value(pair & 15u), (double)sigma));
-        err = __dadd_rn(err, __dmul_rn(d0, d0));
-        double d1 = __dsub_rn((double)x[i + 1], __dmul_rn((double)e2m1_value(pair >> 4), (double)sigma));
-        err = __dadd_rn(err, __dmul_rn(d1, d1));
+        // e sigma is exact in fp64, so x - e sigma rounds once either way
+        const double d0 = __dsub_rn((double)x[i], __dmul_rn((double)e2m1_value(pair & 15u), (double)sigma));
+        const double d1 = __dsub_rn((double)x[i + 1], __dmul_rn((double)e2m1_value(pair >> 4), (double)sigma));
+        if constexpr (W) {
+            err = __dadd_rn(err, __dmul_rn((double)w[i], __dmul_rn(d0, d0)));
+            err = __dadd_rn(err, __dmul_rn((double)w[i + 1], __dmul_rn(d1, d1)));
+        } else {
+            err = __dadd_rn(err, __dmul_rn(d0, d0));
+            err = __dadd_rn(err, __dmul_rn(d1, d1));
+        }
     }
     return err;
 }
@@ -99,15 +107,19 @@ __device__ __forceinline__ float block_amax(const float* x) {
     return a;
 }
 
-// Scale search window: NVFP4 c0+7 .. c0-2 (E4M3 codes, within [0, 126]);
-// MXFP4 c0+1, c0 (E8M0, within [0, 254]); least squared error, ties to the
-// larger code.  All-zero blocks keep code 0.
-template <int FMT>
-__device__ __forceinline__ uint32_t search_scale(const float* x, float g) {
+// Scale search of one key block: the window NVFP4 c0+7 .. c0-2 (E4M3 codes,
+// within [0, 126]) or MXFP4 c0+1, c0 (E8M0, within [0, 254]) around the plain
+// code c0; least (W: weighted) squared error, ties to the larger code.  An
+// all-zero block keeps c0.  Returns the code; `packed` gets its E2M1 codes.
+template <int FMT, bool W>
+__device__ __forceinline__ uint32_t search_scale(const float* x, float g, const float* w, uint32_t* packed) {
     constexpr int B = Fmt<FMT>::beta;
     const float amax = block_amax<B>(x);
     const int c0 = (int)plain_scale_code<FMT>(amax, g);
-    if (amax == 0.0f) return (uint32_t)c0;
+    if (amax == 0.0f) {
+        quantize_block<B>(x, block_sigma<FMT>((uint32_t)c0, g), packed);
+        return (uint32_t)c0;
+    }
     const int top = FMT == BDFP4_NVFP4 ? 126 : 254;
     int hi = c0 + (FMT == BDFP4_NVFP4 ? 7 : 1);
     int lo = c0 - (FMT == BDFP4_NVFP4 ? 2 : 0);
@@ -115,12 +127,14 @@ __device__ __forceinline__ uint32_t search_scale(const float* x, float g) {
     lo = lo < 0 ? 0 : lo;
     int best = hi;
     double best_err = 0.0;
-    uint32_t scratch[B / 8];
     for (int c = hi; c >= lo; --c) {
-        double err = quantize_block<B>(x, block_sigma<FMT>((uint32_t)c, g), scratch);
+        uint32_t cand[B / 8];
+        const double err = quantize_block<B, W>(x, block_sigma<FMT>((uint32_t)c, g), cand, w);
         if (c == hi || err < best_err) {
             best = c;
             best_err = err;
+#pragma unroll
+            for (int k = 0; k < B / 8; ++k) packed[k] = cand[k];
         }
     }
     return (uint32_t)best;

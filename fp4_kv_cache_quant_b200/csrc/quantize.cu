@@ -23,11 +23,12 @@ template <int FMT, int DK>
 __global__ void __launch_bounds__(256) quantize_k_kernel(const __nv_bfloat16* __restrict__ k,
                                                          const int64_t* __restrict__ slot_mapping, int T, int H_kv,
                                                          const float* __restrict__ smooth,
-                                                         const float* __restrict__ k_gscale, uint8_t* k_pages,
+                                                         const float* __restrict__ k_gscale,
+                                                         const float* __restrict__ k_weight, uint8_t* k_pages,
                                                          uint8_t* k_scales, int64_t num_pages, int flags,
                                                          int32_t* dev_status) {
     append_k_cta<FMT, DK>(blockIdx.x, k, (int64_t)T * H_kv, H_kv, MappedSlot{slot_mapping, num_pages, dev_status},
-                          smooth, k_gscale, k_pages, k_scales, flags);
+                          smooth, k_gscale, k_weight, k_pages, k_scales, flags);
 }
 
 // One thread per (token, head, channel); only the first token of each run
@@ -102,7 +103,7 @@ __global__ void __launch_bounds__(256) step_append_kernel(const DecodeArgs a, co
     const NewestSlot slot{a.block_table, a.seq_lens, a.max_pages, a.num_pages, a.dev_status};
     const int nk = (int)k_append_ctas<FMT, DK>(rows);
     if ((int)blockIdx.x < nk)
-        append_k_cta<FMT, DK>(blockIdx.x, s.k_new, rows, a.H_kv, slot, a.smooth, a.k_gscale, s.k_pages, s.k_scales,
+        append_k_cta<FMT, DK>(blockIdx.x, s.k_new, rows, a.H_kv, slot, a.smooth, a.k_gscale, a.k_weight, s.k_pages, s.k_scales,
                               a.flags);
     else
         append_v_open_cta<FMT, DV>(blockIdx.x - nk, s.v_new, s.v_open, slot, a.B, a.H_kv, a.v_gscale, s.v_pages,
@@ -244,6 +245,65 @@ __global__ void calibrate_kernel(const __nv_bfloat16* __restrict__ k_cal, const 
     }
 }
 
+// ---------------------------------------------------------------- key weights
+// Channel weights of the attention-aware key scale search, one CTA per KV
+// head.  Each pass transforms R calibration query rows of the head's group
+// (a thread per 16-channel block, butterflies across the row's threads) into
+// shared memory; then the thread owning channel c adds the rows' squares of
+// that channel in query order (token, then head) to its fp64 sum.
+template <int DK>
+__global__ void __launch_bounds__(256) key_weights_kernel(const __nv_bfloat16* __restrict__ q_cal, int Tq, int H_q,
+                                                          int H_kv, int flags, const float* __restrict__ smooth,
+                                                          float* w) {
+    using RG = RowGeom<BDFP4_NVFP4, DK>;
+    constexpr int B = RG::beta;
+    constexpr int R = 256 / RG::rt;
+    constexpr int NCH = (DK + 255) / 256;   // channels per thread: threadIdx.x + 256 i
+    __shared__ float xs[R][DK];
+    const int hk = blockIdx.x, G = H_q / H_kv;
+    const int r = threadIdx.x / RG::rt, j = threadIdx.x % RG::rt;
+    const int64_t nrows = (int64_t)Tq * G;
+    const bool hadamard = !(flags & BDFP4_FLAG_NO_HADAMARD);
+    double acc[NCH];
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) acc[i] = 0.0;
+    for (int64_t q0 = 0; q0 < nrows; q0 += R) {
+        const int64_t qi = q0 + r;
+        const bool act = qi < nrows && j < RG::tpr;
+        float x[B];
+        if (act) {
+            const int64_t t = qi / G, jg = qi % G;
+            load_bf16_block<B>(q_cal + (t * H_q + (int64_t)hk * G + jg) * DK, j * B, x);
+        } else {
+#pragma unroll
+            for (int i = 0; i < B; ++i) x[i] = 0.0f;
+        }
+        transform_block<BDFP4_NVFP4, DK, false>(x, smooth + (int64_t)hk * DK, j, hadamard);
+        __syncthreads();   // the previous pass's rows have been read
+        if (act) {
+#pragma unroll
+            for (int i = 0; i < B; ++i) xs[r][j * B + i] = x[i];
+        }
+        __syncthreads();
+        const int nr = (int)(nrows - q0 < R ? nrows - q0 : R);
+#pragma unroll
+        for (int i = 0; i < NCH; ++i) {
+            const int c = threadIdx.x + 256 * i;
+            if (c < DK)
+                for (int rr = 0; rr < nr; ++rr) {
+                    const double v = (double)xs[rr][c];
+                    acc[i] = __dadd_rn(acc[i], __dmul_rn(v, v));
+                }
+        }
+    }
+    const double n = (double)Tq * (double)G;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+        const int c = threadIdx.x + 256 * i;
+        if (c < DK) w[(int64_t)hk * DK + c] = __double2float_rn(__ddiv_rn(acc[i], n));
+    }
+}
+
 }  // namespace bdfp4
 
 using namespace bdfp4;
@@ -263,6 +323,20 @@ extern "C" int bdfp4_calibrate(const void* k_cal, const void* q_cal, const void*
     return launch_status();
 }
 
+extern "C" int bdfp4_key_weights(const void* q_cal, int Tq, int H_q, int H_kv, int d_k, int flags,
+                                 const float* smooth, float* w, void* stream) {
+    if (!q_cal || !smooth || !w || Tq <= 0 || H_q <= 0 || H_kv <= 0) return BDFP4_ERR_ARG;
+    if (H_q % H_kv) return BDFP4_ERR_SHAPE;
+    if (d_k != 128 && d_k != 576) return BDFP4_ERR_UNSUPPORTED;
+    if (!aligned(q_cal, 16)) return BDFP4_ERR_ALIGN;
+    cudaStream_t st = (cudaStream_t)stream;
+    if (d_k == 128)
+        key_weights_kernel<128><<<H_kv, 256, 0, st>>>((const __nv_bfloat16*)q_cal, Tq, H_q, H_kv, flags, smooth, w);
+    else
+        key_weights_kernel<576><<<H_kv, 256, 0, st>>>((const __nv_bfloat16*)q_cal, Tq, H_q, H_kv, flags, smooth, w);
+    return launch_status();
+}
+
 template <int FMT, int DK, int DV>
 static void launch_quantize_kv(const void* k, const void* v, const int64_t* slot_mapping, int T, int H_kv,
                                const bdfp4_kv_params* kv, void* k_pages, void* k_scales, void* v_pages,
@@ -270,7 +344,7 @@ static void launch_quantize_kv(const void* k, const void* v, const int64_t* slot
     const int64_t rows = (int64_t)T * H_kv;
     const int64_t kblocks = (rows + KGeom<FMT, DK>::R - 1) / KGeom<FMT, DK>::R;
     quantize_k_kernel<FMT, DK><<<(unsigned)kblocks, 256, 0, st>>>(
-        (const __nv_bfloat16*)k, slot_mapping, T, H_kv, kv->smooth, kv->k_gscale, (uint8_t*)k_pages,
+        (const __nv_bfloat16*)k, slot_mapping, T, H_kv, kv->smooth, kv->k_gscale, kv->k_weight, (uint8_t*)k_pages,
         (uint8_t*)k_scales, num_pages, flags, dev_status);
     using VG = VGeom<DV>;
     const int64_t vblocks = (rows + VG::RPC - 1) / VG::RPC * VG::CPR;
@@ -327,7 +401,8 @@ extern "C" int bdfp4_quantize_k(const void* k, const int64_t* slot_mapping, int 
     const int64_t rows = (int64_t)T * H_kv;
     auto launch = [&](auto kernel, int R) {
         kernel<<<(unsigned)((rows + R - 1) / R), 256, 0, st>>>((const __nv_bfloat16*)k, slot_mapping, T, H_kv,
-                                                              kv->smooth, kv->k_gscale, (uint8_t*)k_pages,
+                                                              kv->smooth, kv->k_gscale, kv->k_weight,
+                                                              (uint8_t*)k_pages,
                                                               (uint8_t*)k_scales, num_pages, flags, dev_status);
     };
     if (fmt == BDFP4_NVFP4) {

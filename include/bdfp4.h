@@ -104,11 +104,15 @@ typedef enum { BDFP4_NVFP4 = 0, BDFP4_MXFP4 = 1 } bdfp4_fmt;
 #define BDFP4_FLAG_DYNAMIC_ALPHA 32
 
 /* Static per-layer quantization parameters (device pointers), produced by
- * bdfp4_calibrate or supplied by the caller. */
+ * bdfp4_calibrate (and bdfp4_key_weights) or supplied by the caller. */
 typedef struct {
     const float* smooth;   /* [H_kv][d_k]: s_c, each a power of two; keys are divided by s_c, queries multiplied */
     const float* k_gscale; /* [H_kv]: NVFP4 FP32 tensor scale of keys (unused for MXFP4)   */
     const float* v_gscale; /* [H_kv]: NVFP4 FP32 tensor scale of values (unused for MXFP4) */
+    /* [H_kv][d_k] channel weights of the attention-aware key scale search
+     * (bdfp4_key_weights), or NULL for the plain objective.  Only the key
+     * appends read it (bdfp4_quantize_kv, bdfp4_quantize_k, bdfp4_decode_step). */
+    const float* k_weight;
 } bdfp4_kv_params;
 
 /*
@@ -127,6 +131,26 @@ BDFP4_API int bdfp4_calibrate(const void* k_cal, const void* q_cal, const void* 
                     int d_k, int d_v, int flags, float* smooth, float* k_gscale, float* v_gscale, void* stream);
 
 /*
+ * Channel weights of the attention-aware key scale search, a variant of the
+ * Outlier-Aware Key Quantization's scale search: the pages say the search
+ * picks a better scale per group of keys but not by what measure ("FP4 KV
+ * Cache Done Right", What is actually new; "BitDecoding-FP4 : décodage natif du
+ * KV cache FP4", Analyse approfondie).  This measure weights each element's
+ * squared error by what it costs the logits: for channel c of KV head h,
+ * w[h][c] = the mean over the calibration queries of the group (Tq tokens x G
+ * heads, G = H_q / H_kv) of x_c^2, x = the query transform (smoothing and, unless
+ * BDFP4_FLAG_NO_HADAMARD, rotation, as the decode applies them) -- with
+ * independent channels, the expected square of the logit error q'.(k' - k^)
+ * the block adds.  Sums in fp64 in query order (token, then head), stored as
+ * fp32 (the sum divided by Tq G).
+ * q_cal [Tq][H_q][d_k] bf16, smooth [H_kv][d_k] (from bdfp4_calibrate), out w
+ * [H_kv][d_k] fp32.  Pass w as bdfp4_kv_params.k_weight to select the weighted
+ * search.  d_k in {128, 576}.
+ */
+BDFP4_API int bdfp4_key_weights(const void* q_cal, int Tq, int H_q, int H_kv, int d_k, int flags, const float* smooth,
+                                float* w, void* stream);
+
+/*
  * KV-append quantization into the paged cache (Outlier-Aware Key Quantization,
  * Article Summary; "Analyse approfondie" of the French page for what each
  * part does).  k [T][H_kv][d_k], v [T][H_kv][d_v] bf16; slot_mapping [T] int64
@@ -136,7 +160,9 @@ BDFP4_API int bdfp4_calibrate(const void* k_cal, const void* q_cal, const void* 
  * per block of beta channels a scale code is searched (NVFP4: E4M3 codes
  * c0+7 .. c0-2 around the plain code c0 = E4M3(amax / (6 g_k)); MXFP4: E8M0
  * codes c0+1, c0 around the OCP MX rule) minimising the block's squared error
- * (fp64, left to right), ties to the larger code; elements are E2M1(x / sigma),
+ * (fp64, left to right; with kv->k_weight, element i's term is w_i d_i^2, the
+ * channel weights of the attention-aware variant), ties to the larger code;
+ * elements are E2M1(x / sigma),
  * sigma = fp32(E4M3(c) g_k) or 2^(c-127).
  * Values: the beta-slot blocks of the call's tokens are (re)quantized with the
  * plain rule; a block's tokens must form one run of consecutive tokens with

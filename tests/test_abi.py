@@ -36,6 +36,25 @@ def test_exports_every_declared_entry_point(lib):
         assert hasattr(lib, n), n
 
 
+def test_kv_params_struct_matches_the_header(lib):
+    """bdfp4_kv_params: four device pointers in the header's order."""
+    hdr = open(os.path.join(ROOT, "include", "bdfp4.h")).read()
+    body = re.search(r"typedef struct \{(.*?)\} bdfp4_kv_params;", hdr, re.S).group(1)
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    fields = re.findall(r"const float\*\s*(\w+);", body)
+    assert fields == [f for f, _ in bdfp4._KVParams._fields_] == ["smooth", "k_gscale", "v_gscale", "k_weight"]
+    assert ctypes.sizeof(bdfp4._KVParams) == 4 * ctypes.sizeof(ctypes.c_void_p)
+
+
+def test_key_weights_argument_errors(lib):
+    a = _p(0x10000)
+    assert lib.bdfp4_key_weights(a, 8, 8, 2, 64, 0, a, a, None) == -4      # head dim outside the set
+    assert lib.bdfp4_key_weights(a, 8, 6, 4, 128, 0, a, a, None) == -2     # 6 query heads over 4 KV heads
+    assert lib.bdfp4_key_weights(None, 8, 8, 2, 128, 0, a, a, None) == -1
+    assert lib.bdfp4_key_weights(a, 0, 8, 2, 128, 0, a, a, None) == -1
+    assert lib.bdfp4_key_weights(_p(0x10001), 8, 8, 2, 128, 0, a, a, None) == -3
+
+
 def test_status_strings(lib):
     for code in range(-6, 1):
         s = bdfp4.bdfp4_status_string(code)

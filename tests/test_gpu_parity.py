@@ -75,6 +75,50 @@ def test_quantize_kv_bit_exact(ora, lib, name, flags):
     assert_bytes_equal(cache_to_np(gcache), ocache)
 
 
+@pytest.mark.parametrize("flags", [0, bdfp4.FLAG_NO_HADAMARD])
+@pytest.mark.parametrize("name", list(SMALL))
+def test_key_weights_bit_exact(ora, lib, name, flags):
+    """Channel weights of the attention-aware key scale search (bdfp4_key_weights)."""
+    sp, fmt = SMALL[name]
+    wl = Workload(sp, seed=14)
+    smooth, _, _ = oracle_calibration(ora, wl, flags)
+    _, qc, _ = wl.calibration("cpu")
+    ref = ora.key_weights(qc, sp.H_q, sp.H_kv, smooth, flags=flags)
+    got = bdfp4.bdfp4_key_weights(qc.cuda(), sp.H_kv, torch.from_numpy(smooth).cuda(), flags=flags)
+    torch.cuda.synchronize()
+    assert np.array_equal(got.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("flags", [0, bdfp4.FLAG_NO_HADAMARD])
+@pytest.mark.parametrize("name", list(SMALL))
+def test_quantize_kv_weighted_search_bit_exact(ora, lib, name, flags):
+    """The attention-aware key scale search: the cache bytes equal the oracle's
+    weighted quantization.  Without the rotation the calibration queries' energy
+    is uneven across channels (smoothing moves it), so the weighted search must
+    pick other codes than the plain one somewhere -- the path is exercised."""
+    sp, fmt = SMALL[name]
+    wl = Workload(sp, seed=15)
+    smooth, kg, vg = oracle_calibration(ora, wl, flags)
+    _, qc, _ = wl.calibration("cpu")
+    w = ora.key_weights(qc, sp.H_q, sp.H_kv, smooth, flags=flags)
+    k, v, sm = wl.all_keys(), wl.all_values(), wl.slot_mapping_all()
+    ocache = ora.empty_cache(wl.num_pages, sp.H_kv, sp.d_k, sp.d_v, fmt)
+    ora.quantize_kv(k, v, sm, ocache, sp.H_kv, fmt, smooth, kg, vg, wl.num_pages, flags=flags, k_weight=w)
+    kvp = kv_params_gpu(smooth, kg, vg)
+    kvp.k_weight = torch.from_numpy(w).cuda()
+    gcache = bdfp4.FP4Cache.empty(wl.num_pages, sp.H_kv, sp.d_k, sp.d_v, fmt)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    bdfp4.bdfp4_quantize_kv(k.cuda(), v.cuda(), torch.from_numpy(sm).cuda(), kvp, gcache, flags=flags,
+                            dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert_bytes_equal(cache_to_np(gcache), ocache)
+    if flags & bdfp4.FLAG_NO_HADAMARD and fmt == NV:
+        plain = ora.empty_cache(wl.num_pages, sp.H_kv, sp.d_k, sp.d_v, fmt)
+        ora.quantize_kv(k, v, sm, plain, sp.H_kv, fmt, smooth, kg, vg, wl.num_pages, flags=flags)
+        assert not np.array_equal(plain["k_scales"], ocache["k_scales"])
+
+
 @pytest.mark.parametrize("name", ["tiny_nv", "tiny_mx", "ragged_g8_nv", "ragged_g8_mx", "mla_nv"])
 def test_decode_step_append_matches_oracle(ora, lib, name):
     """Prefill all but the newest token with bdfp4_quantize_kv, then append the newest
@@ -126,14 +170,26 @@ def test_decode_step_dynamic_alpha_matches_oracle(ora, lib, name, chunk):
     _decode_step_case(ora, name, chunk, bdfp4.FLAG_DYNAMIC_ALPHA)
 
 
-def _decode_step_case(ora, name, chunk, flags):
+@pytest.mark.parametrize("name", ["ragged_g8_nv", "ragged_g8_mx", "mla_nv", "mla8_cuda_mx"])
+def test_decode_step_weighted_search_matches_oracle(ora, lib, name):
+    """The step's key append takes the attention-aware search when the parameters carry weights."""
+    _decode_step_case(ora, name, 1, 0, weighted=True)
+
+
+def _decode_step_case(ora, name, chunk, flags, weighted=False):
     sp, fmt = SMALL[name]
     wl = Workload(sp, seed=8)
     smooth, kg, vg = oracle_calibration(ora, wl)
+    w = None
+    if weighted:
+        _, qc, _ = wl.calibration("cpu")
+        w = ora.key_weights(qc, sp.H_q, sp.H_kv, smooth)
     ocache = ora.empty_cache(wl.num_pages, sp.H_kv, sp.d_k, sp.d_v, fmt)
     ora.quantize_kv(wl.all_keys(), wl.all_values(), wl.slot_mapping_all(), ocache, sp.H_kv, fmt, smooth, kg, vg,
-                    wl.num_pages)
+                    wl.num_pages, k_weight=w)
     kvp = kv_params_gpu(smooth, kg, vg)
+    if weighted:
+        kvp.k_weight = torch.from_numpy(w).cuda()
     gcache = bdfp4.FP4Cache.empty(wl.num_pages, sp.H_kv, sp.d_k, sp.d_v, fmt)
     for name_ in ("k_pages", "k_scales", "v_pages", "v_scales"):
         getattr(gcache, name_).zero_()
