@@ -53,13 +53,14 @@ def bf16_algorithmic_bytes(sp, seq_lens) -> int:
     return tok * sp.H_kv * 2 * (sp.d_k + sp.d_v) + pages * 4 + sp.B * sp.H_q * (sp.d_k + sp.d_v) * 2
 
 
-def algorithmic_bytes(sp, seq_lens, fmt: int) -> int:
-    """Packed KV + scales + block table + Q and O in bf16 for one decode."""
+def algorithmic_bytes(sp, seq_lens, fmt: int, T_q: int = 1) -> int:
+    """Packed KV + scales + block table + Q and O in bf16 for one decode (T_q query
+    tokens per sequence: the cache is read once, Q and O T_q times)."""
     beta = 16 if fmt == 0 else 32
     tok = int(np.sum(seq_lens))
     per_tok = sp.H_kv * (sp.d_k // 2 + sp.d_k // beta + sp.d_v // 2 + sp.d_v // beta)
     pages = int(np.sum((np.asarray(seq_lens) + 63) // 64))
-    return tok * per_tok + pages * 4 + sp.B * sp.H_q * (sp.d_k + sp.d_v) * 2
+    return tok * per_tok + pages * 4 + sp.B * T_q * sp.H_q * (sp.d_k + sp.d_v) * 2
 
 
 # sources of each tensor-core decode kernel: its file and the headers it includes
@@ -275,6 +276,30 @@ def measure_extra(args, name, fmt, flags, device, stream) -> dict:
         bf16_s = median_step(timed_blocks(bf16_decode, args.steps, stream, args.min_region), args.steps)
         r["bf16_kv"] = {"decode_us": bf16_s * 1e6, "frac": bf16_algorithmic_bytes(sp, S["wl"].seq_lens) / bf16_s / 1e9
                         / peak, "fp4_decode_speedup": bf16_s / dec_s}
+    if args.multi_tokens > 1 and sp.d_k == 128:
+        # several query tokens per sequence (the newest T_q, causal), one bdfp4_decode_multi call
+        T = args.multi_tokens
+        g = torch.Generator(device=device)
+        g.manual_seed(7)
+        qm = torch.randn((sp.B, T, sp.H_q, sp.d_k), generator=g, device=device).to(torch.bfloat16)
+        outm = torch.empty((sp.B, T, sp.H_q, sp.d_v), dtype=torch.bfloat16, device=device)
+        cm = bdfp4.bdfp4_decode_multi_plan(S["wl"].seq_lens, T, sp.H_q, sp.H_kv, sp.d_k, sp.d_v, S["num_sms"])
+        wsm = bdfp4.workspace_for(sp.B * T, sp.H_q, sp.d_v, S["wl"].max_pages, cm, device=device)
+
+        def multi():
+            bdfp4.bdfp4_decode_multi(qm, S["cache"], S["bt"], S["sl"], S["kv"], sp.sm_scale, cm, wsm, outm,
+                                     flags=flags, dev_status=S["status"])
+
+        for _ in range(max(args.warmup, 3)):
+            multi()
+        mt_s = median_step(timed_blocks(multi, args.steps, stream, args.min_region), args.steps)
+        assert int(S["status"].item()) == 0, "device status set"
+        m_alg = algorithmic_bytes(sp, S["wl"].seq_lens, fmt, T)
+        r["multi_token"] = {"T_q": T, "kernel": "bdfp4_decode_multi (query images + tensor-core decode + merge)"
+                            if sp.H_q // sp.H_kv * T <= 16 else "bdfp4_decode_multi (CUDA-core decode + merge)",
+                            "chunk_tiles": cm, "decode_us": mt_s * 1e6, "kv_tokens_per_s": tokens / mt_s,
+                            "query_tokens_per_s": sp.B * T / mt_s, "hbm_gbs": m_alg / mt_s / 1e9,
+                            "frac": m_alg / mt_s / 1e9 / peak, "algorithmic_bytes_per_launch": m_alg}
     return r
 
 
@@ -576,6 +601,8 @@ def main():
     ap.add_argument("--config", default="qwen3_30b_a3b", choices=list(CONFIG_TEXT))
     ap.add_argument("--extra", default="qwen3_4b",
                     help="comma-separated workloads whose decode figures go under \"extra\" (N = 1 only)")
+    ap.add_argument("--multi-tokens", type=int, default=4,
+                    help="query tokens per sequence of the multi-token decode figure under extra (1: none)")
     ap.add_argument("--min-region", type=float, default=0.5,
                     help="seconds the repeated blocks of K timed steps cover at least")
     ap.add_argument("--fmt", default="nvfp4", choices=["nvfp4", "mxfp4"])

@@ -30,8 +30,9 @@ TILE_TOKENS = 128
 
 #: names of every entry point declared in include/bdfp4.h
 ENTRY_POINTS = ("bdfp4_calibrate", "bdfp4_key_weights", "bdfp4_quantize_kv", "bdfp4_quantize_k", "bdfp4_quantize_v", "bdfp4_quantize_q", "bdfp4_decode_plan",
-                "bdfp4_decode_plan_for",
-                "bdfp4_decode_workspace_size", "bdfp4_decode", "bdfp4_decode_step", "bdfp4_decode_noalloc",
+                "bdfp4_decode_plan_for", "bdfp4_decode_multi_plan",
+                "bdfp4_decode_workspace_size", "bdfp4_decode", "bdfp4_decode_step", "bdfp4_decode_multi",
+                "bdfp4_decode_noalloc",
                 "bdfp4_status_string", "bdfp4_last_error")
 #: names of every entry point declared in include/bdfp4_bf16.h
 BF16_ENTRY_POINTS = ("bdfp4_bf16_append", "bdfp4_bf16_decode")
@@ -78,6 +79,8 @@ def load() -> ctypes.CDLL:
     L.bdfp4_decode_plan.restype = i
     L.bdfp4_decode_plan_for.argtypes = [p, i, i, i, i, i, i]
     L.bdfp4_decode_plan_for.restype = i
+    L.bdfp4_decode_multi_plan.argtypes = [p, i, i, i, i, i, i, i]
+    L.bdfp4_decode_multi_plan.restype = i
     L.bdfp4_decode_workspace_size.argtypes = [i, i, i, i, i]
     L.bdfp4_decode_workspace_size.restype = sz
     L.bdfp4_decode.argtypes = [p, p, p, p, p, p, p, i, i, i, i, i, i, i64, i, i, kvp, f, i, p, sz, p, p, p]
@@ -85,6 +88,8 @@ def load() -> ctypes.CDLL:
     L.bdfp4_decode_step.argtypes = [p, p, p, p, p, p, p, p, p, p, i, i, i, i, i, i, i64, i, i, kvp, f, i, p, sz, p, p,
                                     p]
     L.bdfp4_decode_step.restype = i
+    L.bdfp4_decode_multi.argtypes = [p, p, p, p, p, p, p, i, i, i, i, i, i, i, i64, i, i, kvp, f, i, p, sz, p, p, p]
+    L.bdfp4_decode_multi.restype = i
     L.bdfp4_decode_noalloc.argtypes = [p, p, p, p, p, p, p, i, i, i, i, i, i, i64, i, i, kvp, f, i, p, p, p]
     L.bdfp4_decode_noalloc.restype = i
     L.bdfp4_status_string.argtypes = [i]
@@ -256,6 +261,16 @@ def bdfp4_decode_plan_for(host_seq_lens, H_q: int, H_kv: int, d_k: int, d_v: int
     return rc
 
 
+def bdfp4_decode_multi_plan(host_seq_lens, T_q: int, H_q: int, H_kv: int, d_k: int, d_v: int, num_sms: int) -> int:
+    import numpy as np
+    sl = np.ascontiguousarray(host_seq_lens, dtype=np.int32)
+    rc = load().bdfp4_decode_multi_plan(ctypes.c_void_p(sl.ctypes.data), sl.shape[0], T_q, H_q, H_kv, d_k, d_v,
+                                        num_sms)
+    if rc < 0:
+        _check(rc, "bdfp4_decode_multi_plan")
+    return rc
+
+
 def bdfp4_decode_workspace_size(B: int, H_q: int, d_v: int, max_pages_per_seq: int, chunk_tiles: int) -> int:
     return int(load().bdfp4_decode_workspace_size(B, H_q, d_v, max_pages_per_seq, chunk_tiles))
 
@@ -272,6 +287,24 @@ def bdfp4_decode(q: torch.Tensor, cache: FP4Cache, block_table: torch.Tensor, se
                              float(sm_scale), int(chunk_tiles), _ptr(workspace), ws_bytes, _ptr(out),
                              _ptr(dev_status), _stream(stream))
     _check(rc, "bdfp4_decode")
+    return out
+
+
+def bdfp4_decode_multi(q: torch.Tensor, cache: FP4Cache, block_table: torch.Tensor, seq_lens: torch.Tensor,
+                       kv: KVParams, sm_scale: float, chunk_tiles: int, workspace: torch.Tensor | None,
+                       out: torch.Tensor, flags: int = 0, dev_status: torch.Tensor | None = None,
+                       stream=None) -> torch.Tensor:
+    """Causal decode of each sequence's T_q newest tokens: q [B, T_q, H_q, d_k],
+    out [B, T_q, H_q, d_v] (bdfp4_decode_multi in bdfp4.h)."""
+    B, T_q, H_q, d_k = q.shape
+    c = kv._c()
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = load().bdfp4_decode_multi(_ptr(q), _ptr(cache.k_pages), _ptr(cache.k_scales), _ptr(cache.v_pages),
+                                   _ptr(cache.v_scales), _ptr(block_table), _ptr(seq_lens), B, T_q, H_q, cache.H_kv,
+                                   d_k, cache.d_v, block_table.shape[1], cache.num_pages, cache.fmt, flags,
+                                   ctypes.byref(c), float(sm_scale), int(chunk_tiles), _ptr(workspace), ws_bytes,
+                                   _ptr(out), _ptr(dev_status), _stream(stream))
+    _check(rc, "bdfp4_decode_multi")
     return out
 
 

@@ -41,23 +41,28 @@ __global__ void __launch_bounds__(kThreads) decode_fp4_kernel(const DecodeArgs a
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int split = blockIdx.x;
-    const int G = a.H_q / a.H_kv;
-    const int chunks = G / HG;
+    // the rows of a (sequence, KV head): the group's G query heads, for each of the T_q
+    // query tokens (token-major, stacked_row); this CTA takes HG of them from v0
+    const int G = a.H_q / a.H_kv, T = a.T_q;
+    const int chunks = G * T / HG;
     const int hk = blockIdx.y / chunks;
-    const int h0 = hk * G + (blockIdx.y % chunks) * HG;   // first query head of this CTA
+    const int v0 = (blockIdx.y % chunks) * HG;
     const int b = blockIdx.z;
+    auto row_of = [&](int r) -> int64_t { return stacked_row(a, b, hk, v0 + r); };
 
     int N = a.seq_lens[b];
     if (N < 0 || N > a.max_pages * kPageSlots) {
         if (tid == 0 && split == 0) set_status(a.dev_status, BDFP4_DEV_BAD_SEQLEN);
         N = 0;
     }
+    // several query tokens: the sequence must hold them (rows that see no token give zeros)
+    if (T > 1 && N > 0 && N < T && tid == 0 && split == 0 && blockIdx.y == 0)
+        set_status(a.dev_status, BDFP4_DEV_BAD_SEQLEN);
     const int ntiles = (N + kTileTokens - 1) / kTileTokens;
     const int nspl = (ntiles + a.chunk_tiles - 1) / a.chunk_tiles;
     if (split > 0 && split >= nspl) return;
     if (N == 0) {  // empty sequence: zeros
-        for (int i = tid; i < HG * DV; i += kThreads)
-            a.out[((int64_t)b * a.H_q + h0 + i / DV) * DV + i % DV] = __float2bfloat16(0.0f);
+        for (int i = tid; i < HG * DV; i += kThreads) a.out[row_of(i / DV) * DV + i % DV] = __float2bfloat16(0.0f);
         return;
     }
 
@@ -72,7 +77,7 @@ __global__ void __launch_bounds__(kThreads) decode_fp4_kernel(const DecodeArgs a
         row_amax[tid] = 0;
         float x[B];
         if (active) {
-            load_bf16_block<B>(a.q + ((int64_t)b * a.H_q + h0 + r) * DK, j * B, x);
+            load_bf16_block<B>(a.q + row_of(r) * DK, j * B, x);
         } else {
 #pragma unroll
             for (int i = 0; i < B; ++i) x[i] = 0.0f;
@@ -175,6 +180,12 @@ __global__ void __launch_bounds__(kThreads) decode_fp4_kernel(const DecodeArgs a
             }
 #pragma unroll
             for (int g = 0; g < HG; ++g) s[g] = acc[g] * lsc[g];
+            // query token i of the stacked row sees the first N - T + 1 + i tokens
+            if (T > 1) {
+#pragma unroll
+                for (int g = 0; g < HG; ++g)
+                    if (token >= N - T + 1 + (v0 + g) / G) s[g] = -INFINITY;
+            }
         }
         // ------------------------------------------------ transposed online softmax
         float p[HG], corr[HG];
@@ -195,7 +206,7 @@ __global__ void __launch_bounds__(kThreads) decode_fp4_kernel(const DecodeArgs a
             const float mz = mn == -INFINITY ? 0.0f : mn;
             corr[g] = exp2f(m_run[g] - mz);   // 0 on the split's first tile
             m_run[g] = mn;
-            p[g] = valid ? exp2f(s[g] - mz) : 0.0f;
+            p[g] = valid && s[g] != -INFINITY ? exp2f(s[g] - mz) : 0.0f;
             l_part[g] = l_part[g] * corr[g] + p[g];
             float ag = alpha, ig = 1.0f;
             if (dyn) {
@@ -279,7 +290,7 @@ __global__ void __launch_bounds__(kThreads) decode_fp4_kernel(const DecodeArgs a
 #pragma unroll
     for (int g = 0; g < HG; ++g) {
         const float l = lsum[0][g] + lsum[1][g] + lsum[2][g] + lsum[3][g];
-        const int64_t row = (int64_t)b * a.H_q + h0 + g;
+        const int64_t row = row_of(g);
 #pragma unroll
         for (int c = 0; c < NCH; ++c) {
             const int ch = tid + c * kThreads;
@@ -340,21 +351,27 @@ extern "C" int bdfp4_decode_plan(const int32_t* host_seq_lens, int B, int H_kv, 
 
 extern "C" int bdfp4_decode_plan_for(const int32_t* host_seq_lens, int B, int H_q, int H_kv, int d_k, int d_v,
                                      int num_sms) {
-    if (!host_seq_lens || B <= 0 || H_q <= 0 || H_kv <= 0 || num_sms <= 0) return BDFP4_ERR_ARG;
+    return bdfp4_decode_multi_plan(host_seq_lens, B, 1, H_q, H_kv, d_k, d_v, num_sms);
+}
+
+extern "C" int bdfp4_decode_multi_plan(const int32_t* host_seq_lens, int B, int T_q, int H_q, int H_kv, int d_k,
+                                       int d_v, int num_sms) {
+    if (!host_seq_lens || B <= 0 || T_q <= 0 || H_q <= 0 || H_kv <= 0 || num_sms <= 0) return BDFP4_ERR_ARG;
     if (H_q % H_kv) return BDFP4_ERR_SHAPE;
     if (!supported_dims(d_k, d_v)) return BDFP4_ERR_UNSUPPORTED;
-    const DecodeShape ks = decode_shape(d_k, d_v, H_q / H_kv);
+    const DecodeShape ks = decode_shape(d_k, d_v, H_q / H_kv, T_q);
     return plan_chunk_tiles(B, [&](int b) { return host_tiles(host_seq_lens, b); }, H_kv * ks.items_per_kv_head,
                             num_sms, ks.ctas_per_sm);
 }
 
-// The split merge after a decode grid (nothing when no sequence can split).
+// The split merge after a decode grid (nothing when no sequence can split).  Its
+// rows are the [B][T_q][H_q] output rows; a sequence's T_q H_q rows share its length.
 template <int DV>
 static int merge_splits(const DecodeArgs& a, cudaStream_t st) {
     const int rc = launch_status();
     if (rc != BDFP4_OK || a.max_splits <= 1) return rc;
-    const cudaError_t e = launch_merge<DV>(a.ws_o, a.ws_ml, a.seq_lens, a.B, a.H_q, a.max_pages, a.chunk_tiles,
-                                           a.max_splits, a.out, st);
+    const cudaError_t e = launch_merge<DV>(a.ws_o, a.ws_ml, a.seq_lens, a.B, a.H_q * a.T_q, a.max_pages,
+                                           a.chunk_tiles, a.max_splits, a.out, st);
     if (e != cudaSuccess) {
         record_cuda_error(e);
         return BDFP4_ERR_CUDA;
@@ -364,16 +381,16 @@ static int merge_splits(const DecodeArgs& a, cudaStream_t st) {
 
 template <int FMT, int DK, int DV>
 static int launch_decode(const DecodeArgs& a, int G, cudaStream_t st, const StepArgs* step) {
-    // the dynamic probability pre-scale runs on the d = 128 tensor-core decode and, for
-    // MLA shapes, on the CUDA-core decode (MXFP4 has no alpha to choose)
-    const bool mla_tc_ok = !(FMT == BDFP4_NVFP4 && (a.flags & BDFP4_FLAG_DYNAMIC_ALPHA));
-    if (DK == 128 && G <= 16) {
-        // tensor-core path (decode_tc.cu); a step's append runs in its prologue grid
-        const int rc = launch_decode_tc(a, FMT, G, st, step);
+    const bool dyn_mla = FMT == BDFP4_NVFP4 && (a.flags & BDFP4_FLAG_DYNAMIC_ALPHA);
+    const DecodePath path = decode_path(DK, DV, G, a.T_q, dyn_mla);
+    if (path == DecodePath::kTensorCore128) {
+        // tensor-core path (decode_tc.cu) on the G T_q stacked rows; a step's append runs in
+        // its prologue grid
+        const int rc = launch_decode_tc(a, FMT, G * a.T_q, st, step);
         if (rc != BDFP4_OK) return rc;
         return merge_splits<DV>(a, st);
     }
-    if (mla_tc_ok && DK == 576 && mla_tc_supported(DK, DV, G)) {
+    if (path == DecodePath::kTensorCoreMla) {
         // tensor-core path for MLA shapes (decode_mla_tc.cu); a step's append runs in its prologue grid
         const int rc = launch_decode_mla_tc(a, FMT, G, st, step);
         if (rc != BDFP4_OK) return rc;
@@ -383,8 +400,8 @@ static int launch_decode(const DecodeArgs& a, int G, cudaStream_t st, const Step
         const int rc = launch_step_append(a, *step, FMT, DK, st);
         if (rc != BDFP4_OK) return rc;
     }
-    int hg = G >= 16 ? 16 : G;
-    dim3 grid(a.max_splits, a.H_kv * (G / hg), a.B);
+    const int rows = G * a.T_q, hg = cuda_core_rows(rows);
+    dim3 grid(a.max_splits, a.H_kv * (rows / hg), a.B);
     switch (hg) {
         case 1: decode_fp4_kernel<FMT, DK, DV, 1><<<grid, kThreads, 0, st>>>(a); break;
         case 2: decode_fp4_kernel<FMT, DK, DV, 2><<<grid, kThreads, 0, st>>>(a); break;
@@ -397,16 +414,17 @@ static int launch_decode(const DecodeArgs& a, int G, cudaStream_t st, const Step
 }
 
 static int run_decode(const void* q, const void* k_pages, const void* k_scales, const void* v_pages,
-                      const void* v_scales, const int32_t* block_table, const int32_t* seq_lens, int B, int H_q,
-                      int H_kv, int d_k, int d_v, int max_pages_per_seq, int64_t num_pages, bdfp4_fmt fmt, int flags,
-                      const bdfp4_kv_params* kv, float sm_scale, int chunk_tiles, void* workspace,
+                      const void* v_scales, const int32_t* block_table, const int32_t* seq_lens, int B, int T_q,
+                      int H_q, int H_kv, int d_k, int d_v, int max_pages_per_seq, int64_t num_pages, bdfp4_fmt fmt,
+                      int flags, const bdfp4_kv_params* kv, float sm_scale, int chunk_tiles, void* workspace,
                       size_t workspace_bytes, void* out, int32_t* dev_status, void* stream, StepArgs* step) {
-    if (B < 0 || H_q <= 0 || H_kv <= 0 || max_pages_per_seq <= 0 || num_pages < 0) return BDFP4_ERR_ARG;
+    if (B < 0 || T_q <= 0 || H_q <= 0 || H_kv <= 0 || max_pages_per_seq <= 0 || num_pages < 0) return BDFP4_ERR_ARG;
     if (fmt != BDFP4_NVFP4 && fmt != BDFP4_MXFP4) return BDFP4_ERR_ARG;
     if (H_q % H_kv) return BDFP4_ERR_SHAPE;
     if (!supported_dims(d_k, d_v)) return BDFP4_ERR_UNSUPPORTED;
     const int G = H_q / H_kv;
     if (G > 16 ? (G % 16 != 0 || G > 128) : (G & (G - 1)) != 0) return BDFP4_ERR_UNSUPPORTED;
+    if ((int64_t)G * T_q > 4096) return BDFP4_ERR_UNSUPPORTED;
     if (B == 0) return BDFP4_OK;
     if (!q || !k_pages || !k_scales || !v_pages || !v_scales || !block_table || !seq_lens || !out || !kv ||
         !kv->smooth)
@@ -416,6 +434,7 @@ static int run_decode(const void* q, const void* k_pages, const void* k_scales, 
     if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_pages, 128) || !aligned(k_scales, 128) ||
         !aligned(v_pages, 128) || !aligned(v_scales, 128))
         return BDFP4_ERR_ALIGN;
+    const bool dyn_mla = fmt == BDFP4_NVFP4 && (flags & BDFP4_FLAG_DYNAMIC_ALPHA);
     if (chunk_tiles <= 0) {
         // no host sequence lengths: plan for the longest possible sequence
         int dev = 0, sms = 148;
@@ -423,17 +442,15 @@ static int run_decode(const void* q, const void* k_pages, const void* k_scales, 
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return BDFP4_ERR_CUDA;
         const int ntiles = (max_pages_per_seq * kPageSlots + kTileTokens - 1) / kTileTokens;
-        const DecodeShape ks = decode_shape(d_k, d_v, G);
+        const DecodeShape ks = decode_shape(d_k, d_v, G, T_q, dyn_mla);
         chunk_tiles = plan_chunk_tiles(B, [&](int) { return ntiles; }, H_kv * ks.items_per_kv_head, sms,
                                        ks.ctas_per_sm);
     }
     DecodeArgs a{};
     a.max_splits = max_splits_for(max_pages_per_seq, chunk_tiles);
-    const bool tensor_core_path = (d_k == 128 && G <= 16) ||
-                                  (!(fmt == BDFP4_NVFP4 && (flags & BDFP4_FLAG_DYNAMIC_ALPHA)) &&
-                                   mla_tc_supported(d_k, d_v, G));
+    const bool tensor_core_path = decode_path(d_k, d_v, G, T_q, dyn_mla) != DecodePath::kCudaCore;
     if (a.max_splits > 1 || tensor_core_path) {
-        const WorkspaceMap m = workspace_map(B, H_q, d_v, a.max_splits);
+        const WorkspaceMap m = workspace_map(B * T_q, H_q, d_v, a.max_splits);
         if (!workspace || workspace_bytes < m.total) return BDFP4_ERR_WORKSPACE;
         if (!aligned(workspace, 128)) return BDFP4_ERR_ALIGN;
         a.ws_o = (float*)workspace;
@@ -454,6 +471,7 @@ static int run_decode(const void* q, const void* k_pages, const void* k_scales, 
     a.out = (__nv_bfloat16*)out;
     a.dev_status = dev_status;
     a.B = B;
+    a.T_q = T_q;
     a.H_q = H_q;
     a.H_kv = H_kv;
     a.max_pages = max_pages_per_seq;
@@ -481,7 +499,7 @@ extern "C" int bdfp4_decode(const void* q, const void* k_pages, const void* k_sc
                             int H_kv, int d_k, int d_v, int max_pages_per_seq, int64_t num_pages, bdfp4_fmt fmt,
                             int flags, const bdfp4_kv_params* kv, float sm_scale, int chunk_tiles, void* workspace,
                             size_t workspace_bytes, void* out, int32_t* dev_status, void* stream) {
-    return run_decode(q, k_pages, k_scales, v_pages, v_scales, block_table, seq_lens, B, H_q, H_kv, d_k, d_v,
+    return run_decode(q, k_pages, k_scales, v_pages, v_scales, block_table, seq_lens, B, 1, H_q, H_kv, d_k, d_v,
                       max_pages_per_seq, num_pages, fmt, flags, kv, sm_scale, chunk_tiles, workspace,
                       workspace_bytes, out, dev_status, stream, nullptr);
 }
@@ -498,9 +516,20 @@ extern "C" int bdfp4_decode_step(const void* q, const void* k_new, const void* v
     s.k_new = (const __nv_bfloat16*)k_new;
     s.v_new = (const __nv_bfloat16*)v_new;
     s.v_open = (__nv_bfloat16*)v_open;
-    return run_decode(q, k_pages, k_scales, v_pages, v_scales, block_table, seq_lens, B, H_q, H_kv, d_k, d_v,
+    return run_decode(q, k_pages, k_scales, v_pages, v_scales, block_table, seq_lens, B, 1, H_q, H_kv, d_k, d_v,
                       max_pages_per_seq, num_pages, fmt, flags, kv, sm_scale, chunk_tiles, workspace,
                       workspace_bytes, out, dev_status, stream, &s);
+}
+
+extern "C" int bdfp4_decode_multi(const void* q, const void* k_pages, const void* k_scales, const void* v_pages,
+                                  const void* v_scales, const int32_t* block_table, const int32_t* seq_lens, int B,
+                                  int T_q, int H_q, int H_kv, int d_k, int d_v, int max_pages_per_seq,
+                                  int64_t num_pages, bdfp4_fmt fmt, int flags, const bdfp4_kv_params* kv,
+                                  float sm_scale, int chunk_tiles, void* workspace, size_t workspace_bytes, void* out,
+                                  int32_t* dev_status, void* stream) {
+    return run_decode(q, k_pages, k_scales, v_pages, v_scales, block_table, seq_lens, B, T_q, H_q, H_kv, d_k, d_v,
+                      max_pages_per_seq, num_pages, fmt, flags, kv, sm_scale, chunk_tiles, workspace,
+                      workspace_bytes, out, dev_status, stream, nullptr);
 }
 
 // ---------------------------------------------------------------- no-allocation variant
@@ -544,7 +573,8 @@ extern "C" int bdfp4_decode_noalloc(const void* q, const void* k_pages, const vo
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return BDFP4_ERR_CUDA;
         const int ntiles = (max_pages_per_seq * kPageSlots + kTileTokens - 1) / kTileTokens;
-        const DecodeShape ks = decode_shape(d_k, d_v, H_kv > 0 && H_q % H_kv == 0 ? H_q / H_kv : 1);
+        const DecodeShape ks = decode_shape(d_k, d_v, H_kv > 0 && H_q % H_kv == 0 ? H_q / H_kv : 1, 1,
+                                            fmt == BDFP4_NVFP4 && (flags & BDFP4_FLAG_DYNAMIC_ALPHA));
         chunk_tiles = plan_chunk_tiles(B, [&](int) { return ntiles; }, (H_kv > 0 ? H_kv : 1) * ks.items_per_kv_head,
                                        sms, ks.ctas_per_sm);
     }

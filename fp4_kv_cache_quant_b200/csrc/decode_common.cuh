@@ -27,6 +27,7 @@ struct DecodeArgs {
     int32_t* dev_status;
     int B, H_q, H_kv, max_pages, flags, chunk_tiles, max_splits;
     int append_wait;   // 1: a decode-step prologue grid writes each sequence's last page (tensor-core path)
+    int T_q;           // query tokens per sequence (1: single-token decode); q, out are [B][T_q][H_q][d]
     int64_t num_pages;
     float sm_scale;
 };
@@ -51,6 +52,14 @@ constexpr float kLog2e = 1.4426950408889634f;
 // tensor-core decodes (an image of a (sequence, KV head) or head slice of h
 // heads takes at most h times this; each layout static_asserts it).
 constexpr int kQueryImageBytes = 656;
+
+// Row of the query, output and split-partial arrays ([B][T_q][H_q]) of stacked
+// query row v of (sequence b, KV head hk): the T_q tokens' query heads of the
+// KV group stack token-major, v = i G + g for token i and head g of the group.
+__device__ __forceinline__ int64_t stacked_row(const DecodeArgs& a, int b, int hk, int v) {
+    const int G = a.H_q / a.H_kv;
+    return ((int64_t)b * a.T_q + v / G) * a.H_q + (int64_t)hk * G + v % G;
+}
 
 // Splits of a sequence of N tokens.
 __host__ __device__ __forceinline__ int num_splits(int N, int chunk_tiles) {
@@ -87,16 +96,37 @@ inline int plan_chunk_tiles(int B, const TilesOf& tiles_of, int items, int num_s
     return best;
 }
 
+// Which decode kernel runs a shape: G query heads per KV head, T query tokens
+// per sequence (their G T rows stack per (sequence, KV head)), head dims d_k /
+// d_v; dyn_mla: the per-tile probability pre-scale with NVFP4 on MLA shapes.
+enum class DecodePath { kTensorCore128, kTensorCoreMla, kCudaCore };
+inline DecodePath decode_path(int d_k, int d_v, int G, int T, bool dyn_mla) {
+    const int rows = G * T;
+    if (d_k == 128 && d_v == 128 && rows <= 16 && (rows & (rows - 1)) == 0) return DecodePath::kTensorCore128;
+    if (d_k == 576 && d_v == 512 && T == 1 && !dyn_mla && (G == 16 || G == 32 || G == 64 || G == 128))
+        return DecodePath::kTensorCoreMla;
+    return DecodePath::kCudaCore;
+}
+
+// Rows per CTA of the CUDA-core decode for `rows` stacked rows: the largest
+// power of two up to 16 that divides them.
+inline int cuda_core_rows(int rows) {
+    int hg = 16;
+    while (rows % hg) hg >>= 1;
+    return hg;
+}
+
 // CTAs per SM and CTAs per (sequence, split, KV head) of the decode kernel that
-// bdfp4_decode runs for this shape.
+// runs this shape (decode_path).
 struct DecodeShape {
     int ctas_per_sm, items_per_kv_head;
 };
-inline DecodeShape decode_shape(int d_k, int d_v, int G) {
-    if (d_k == 128 && d_v == 128 && G <= 16) return {G <= 4 ? 4 : 3, 1};              // decode_tc.cu
-    if (d_k == 576 && d_v == 512 && (G == 16 || G == 32 || G == 64 || G == 128))
-        return {1, G > 64 ? G / 64 : 1};                                                  // decode_mla_tc.cu
-    return {8, G >= 16 ? G / 16 : 1};                                                     // CUDA-core decode
+inline DecodeShape decode_shape(int d_k, int d_v, int G, int T = 1, bool dyn_mla = false) {
+    switch (decode_path(d_k, d_v, G, T, dyn_mla)) {
+        case DecodePath::kTensorCore128: return {G * T <= 4 ? 4 : 3, 1};                  // decode_tc.cu
+        case DecodePath::kTensorCoreMla: return {1, G > 64 ? G / 64 : 1};                   // decode_mla_tc.cu
+        default: return {8, G * T / cuda_core_rows(G * T)};                                 // CUDA-core decode
+    }
 }
 
 // tcgen05 decode for d_k = d_v = 128 (decode_tc.cu); returns a host status.

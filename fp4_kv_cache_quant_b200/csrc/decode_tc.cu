@@ -140,7 +140,9 @@ constexpr long long kWaitLimit = 1LL << 32;   // clock cycles (about 2 s)
 // [NQ][8] and the logit scales sm_scale g_q g_k log2(e) per head).  Every split of
 // the sequence copies it instead of recomputing it.
 // One CTA (at least QTHREADS threads) builds the image of (sequence b, KV head hk).
-template <int FMT, int G>
+// MT (several query tokens per sequence): the G stacked rows are the T_q
+// tokens' query heads of the group, token-major (stacked_row).
+template <int FMT, int G, bool MT = false>
 __device__ __forceinline__ void query_image_cta(const DecodeArgs& a, int hk, int b) {
     using C = TcCfg<FMT, G>;
     using RG = RowGeom<FMT, 128>;
@@ -160,7 +162,8 @@ __device__ __forceinline__ void query_image_cta(const DecodeArgs& a, int hk, int
     const bool active = r < G && j < RG::tpr;
     float x[B];
     if (active) {
-        load_bf16_block<B>(a.q + ((int64_t)b * a.H_q + h0 + r) * C::DK, j * B, x);
+        const int64_t qrow = MT ? stacked_row(a, b, hk, r) : (int64_t)b * a.H_q + h0 + r;
+        load_bf16_block<B>(a.q + qrow * C::DK, j * B, x);
     } else {
 #pragma unroll
         for (int i = 0; i < B; ++i) x[i] = 0.0f;
@@ -193,11 +196,11 @@ __device__ __forceinline__ void query_image_cta(const DecodeArgs& a, int hk, int
     for (int i = tid; i < C::QPACK / 16; i += blockDim.x) out[i] = reinterpret_cast<const uint4*>(img)[i];
 }
 
-template <int FMT, int G>
+template <int FMT, int G, bool MT = false>
 __global__ void __launch_bounds__(TcCfg<FMT, G>::QTHREADS) prep_query_kernel(const DecodeArgs a) {
     // the decode grid may start now; it waits for this grid before copying the image
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    query_image_cta<FMT, G>(a, blockIdx.x, blockIdx.y);
+    query_image_cta<FMT, G, MT>(a, blockIdx.x, blockIdx.y);
 }
 
 // Decode-step prologue: one grid whose CTAs take three roles side by side --
@@ -223,7 +226,9 @@ __global__ void __launch_bounds__(256) prep_step_kernel(const DecodeArgs a, cons
     }
 }
 
-template <int FMT, int G, bool DYN = false>
+// MT: several query tokens per sequence (a.T_q), their query heads stacked as
+// the G rows (token-major); query token i sees the first N - T_q + 1 + i tokens.
+template <int FMT, int G, bool DYN = false, bool MT = false>
 __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTAS) decode_tc_kernel(const DecodeArgs a) {
     using C = TcCfg<FMT, G>;
     // the split merge (a programmatic dependent) may be scheduled as CTAs of this grid retire
@@ -261,12 +266,18 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
         if (tid == 0 && split == 0) set_status(a.dev_status, BDFP4_DEV_BAD_SEQLEN);
         N = 0;
     }
+    // MT: a sequence must hold its T_q query tokens (rows that would see no token give zeros)
+    if (MT && N > 0 && N < a.T_q && tid == 0 && split == 0) set_status(a.dev_status, BDFP4_DEV_BAD_SEQLEN);
+    // output / partial row of stacked row v
+    auto row_of = [&](int v) -> int64_t {
+        if constexpr (MT) return stacked_row(a, b, hk, v);
+        else return (int64_t)b * a.H_q + h0 + v;
+    };
     const int ntiles = (N + kTileTokens - 1) / kTileTokens;
     const int nspl = (ntiles + a.chunk_tiles - 1) / a.chunk_tiles;
     if (split > 0 && split >= nspl) return;
     if (N == 0) {
-        for (int i = tid; i < G * C::DV; i += blockDim.x)
-            a.out[((int64_t)b * a.H_q + h0 + i / C::DV) * C::DV + i % C::DV] = __float2bfloat16(0.0f);
+        for (int i = tid; i < G * C::DV; i += blockDim.x) a.out[row_of(i / C::DV) * C::DV + i % C::DV] = __float2bfloat16(0.0f);
         return;
     }
     const int tile0 = split * a.chunk_tiles;
@@ -589,12 +600,16 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                 tc::tmem_wait_ld();
                 const int token = tile * kTileTokens + tok_in_tile;
                 const bool valid = token < N && (page_of_thread ? pok1 : pok0);
+                // MT: the token is visible to query token i iff token <= N - T_q + i, i.e. to the
+                // stacked rows v = i G + g >= (token - (N - T_q)) G: rows g >= vis of this group
+                int vis = 0;
+                if constexpr (MT) vis = (token - (N - a.T_q)) * (a.H_q / a.H_kv) - gb;
                 // raw logits q1.k + q2.k (the positive factor lsc is applied later, so maxima
                 // commute with it) and their maxima over each half warp (16 consecutive slots)
                 float t[HG], hm_lo[HG], hm_hi[HG];
     #pragma unroll
                 for (int g = 0; g < HG; ++g) {
-                    t[g] = valid ? __uint_as_float(sr[g]) + __uint_as_float(sr[HG + g]) : -INFINITY;
+                    t[g] = (valid && (!MT || g >= vis)) ? __uint_as_float(sr[g]) + __uint_as_float(sr[HG + g]) : -INFINITY;
                     hm_lo[g] = tc::redux_max_f32(lo_half ? t[g] : -INFINITY, 0xffffffffu);
                     hm_hi[g] = tc::redux_max_f32(lo_half ? -INFINITY : t[g], 0xffffffffu);
                 }
@@ -771,7 +786,7 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
             for (int g = 0; g < HG; ++g) {
                 const int hh = gb + g;
                 const float l = rl[hh * 8] + rl[hh * 8 + 1] + rl[hh * 8 + 2] + rl[hh * 8 + 3];
-                const int64_t row = (int64_t)b * a.H_q + h0 + hh;
+                const int64_t row = row_of(hh);
                 if (nspl == 1) {
                     a.out[row * C::DV + ch] =
                         __float2bfloat16(l > 0.0f ? __uint_as_float(o_fin[g]) * oscale / l : 0.0f);
@@ -797,12 +812,12 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
     }
 }
 
-template <int FMT, int G, bool DYN = false>
+template <int FMT, int G, bool DYN = false, bool MT = false>
 static int launch_tc(const DecodeArgs& a, cudaStream_t st, const StepArgs* step) {
     using C = TcCfg<FMT, G>;
     static bool attr_set = false;
     if (!attr_set) {
-        const cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<FMT, G, DYN>,
+        const cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<FMT, G, DYN, MT>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_LAUNCH);
         if (e != cudaSuccess) {
             record_cuda_error(e);
@@ -810,12 +825,17 @@ static int launch_tc(const DecodeArgs& a, cudaStream_t st, const StepArgs* step)
         }
         attr_set = true;
     }
-    if (step) {
-        const int64_t rows = (int64_t)a.B * a.H_kv;
-        const int64_t ctas = k_append_ctas<FMT, 128>(rows) + v_append_ctas<128>(rows) + rows;
-        prep_step_kernel<FMT, G><<<(unsigned)ctas, 256, 0, st>>>(a, *step);
+    if constexpr (!MT) {
+        if (step) {
+            const int64_t rows = (int64_t)a.B * a.H_kv;
+            const int64_t ctas = k_append_ctas<FMT, 128>(rows) + v_append_ctas<128>(rows) + rows;
+            prep_step_kernel<FMT, G><<<(unsigned)ctas, 256, 0, st>>>(a, *step);
+        } else {
+            prep_query_kernel<FMT, G><<<dim3(a.H_kv, a.B), C::QTHREADS, 0, st>>>(a);
+        }
     } else {
-        prep_query_kernel<FMT, G><<<dim3(a.H_kv, a.B), C::QTHREADS, 0, st>>>(a);
+        if (step) return BDFP4_ERR_UNSUPPORTED;   // a step appends one token per sequence
+        prep_query_kernel<FMT, G, true><<<dim3(a.H_kv, a.B), C::QTHREADS, 0, st>>>(a);
     }
     const int rc = launch_status();
     if (rc != BDFP4_OK) return rc;
@@ -831,7 +851,7 @@ static int launch_tc(const DecodeArgs& a, cudaStream_t st, const StepArgs* step)
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<FMT, G, DYN>, a);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<FMT, G, DYN, MT>, a);
     if (e != cudaSuccess) {
         record_cuda_error(e);
         return BDFP4_ERR_CUDA;
@@ -839,33 +859,40 @@ static int launch_tc(const DecodeArgs& a, cudaStream_t st, const StepArgs* step)
     return launch_status();
 }
 
-int launch_decode_tc(const DecodeArgs& a, int fmt, int G, cudaStream_t st, const StepArgs* step) {
+template <bool MT>
+static int dispatch_tc(const DecodeArgs& a, int fmt, int G, cudaStream_t st, const StepArgs* step) {
     if (fmt == BDFP4_NVFP4 && (a.flags & BDFP4_FLAG_DYNAMIC_ALPHA)) {
         switch (G) {
-            case 1: return launch_tc<BDFP4_NVFP4, 1, true>(a, st, step);
-            case 2: return launch_tc<BDFP4_NVFP4, 2, true>(a, st, step);
-            case 4: return launch_tc<BDFP4_NVFP4, 4, true>(a, st, step);
-            case 8: return launch_tc<BDFP4_NVFP4, 8, true>(a, st, step);
-            case 16: return launch_tc<BDFP4_NVFP4, 16, true>(a, st, step);
+            case 1: if constexpr (!MT) return launch_tc<BDFP4_NVFP4, 1, true, false>(a, st, step); break;
+            case 2: return launch_tc<BDFP4_NVFP4, 2, true, MT>(a, st, step);
+            case 4: return launch_tc<BDFP4_NVFP4, 4, true, MT>(a, st, step);
+            case 8: return launch_tc<BDFP4_NVFP4, 8, true, MT>(a, st, step);
+            case 16: return launch_tc<BDFP4_NVFP4, 16, true, MT>(a, st, step);
         }
     } else if (fmt == BDFP4_NVFP4) {
         switch (G) {
-            case 1: return launch_tc<BDFP4_NVFP4, 1>(a, st, step);
-            case 2: return launch_tc<BDFP4_NVFP4, 2>(a, st, step);
-            case 4: return launch_tc<BDFP4_NVFP4, 4>(a, st, step);
-            case 8: return launch_tc<BDFP4_NVFP4, 8>(a, st, step);
-            case 16: return launch_tc<BDFP4_NVFP4, 16>(a, st, step);
+            case 1: if constexpr (!MT) return launch_tc<BDFP4_NVFP4, 1, false, false>(a, st, step); break;
+            case 2: return launch_tc<BDFP4_NVFP4, 2, false, MT>(a, st, step);
+            case 4: return launch_tc<BDFP4_NVFP4, 4, false, MT>(a, st, step);
+            case 8: return launch_tc<BDFP4_NVFP4, 8, false, MT>(a, st, step);
+            case 16: return launch_tc<BDFP4_NVFP4, 16, false, MT>(a, st, step);
         }
     } else {
         switch (G) {
-            case 1: return launch_tc<BDFP4_MXFP4, 1>(a, st, step);
-            case 2: return launch_tc<BDFP4_MXFP4, 2>(a, st, step);
-            case 4: return launch_tc<BDFP4_MXFP4, 4>(a, st, step);
-            case 8: return launch_tc<BDFP4_MXFP4, 8>(a, st, step);
-            case 16: return launch_tc<BDFP4_MXFP4, 16>(a, st, step);
+            case 1: if constexpr (!MT) return launch_tc<BDFP4_MXFP4, 1, false, false>(a, st, step); break;
+            case 2: return launch_tc<BDFP4_MXFP4, 2, false, MT>(a, st, step);
+            case 4: return launch_tc<BDFP4_MXFP4, 4, false, MT>(a, st, step);
+            case 8: return launch_tc<BDFP4_MXFP4, 8, false, MT>(a, st, step);
+            case 16: return launch_tc<BDFP4_MXFP4, 16, false, MT>(a, st, step);
         }
     }
     return BDFP4_ERR_UNSUPPORTED;
+}
+
+// G = rows stacked per (sequence, KV head): the query heads of the group, times
+// the query tokens per sequence when a.T_q > 1 (which then takes the MT kernels)
+int launch_decode_tc(const DecodeArgs& a, int fmt, int G, cudaStream_t st, const StepArgs* step) {
+    return a.T_q > 1 ? dispatch_tc<true>(a, fmt, G, st, step) : dispatch_tc<false>(a, fmt, G, st, step);
 }
 
 }  // namespace bdfp4

@@ -227,6 +227,13 @@ BDFP4_API int bdfp4_decode_plan(const int32_t* host_seq_lens, int B, int H_kv, i
 BDFP4_API int bdfp4_decode_plan_for(const int32_t* host_seq_lens, int B, int H_q, int H_kv, int d_k, int d_v,
                                     int num_sms);
 
+/* The plan for bdfp4_decode_multi with T_q query tokens per sequence (T_q = 1
+ * is bdfp4_decode_plan_for): the kernel that runs G T_q stacked rows per KV head
+ * -- the d = 128 tensor-core decode at up to 16 rows, three (four up to four
+ * rows) CTAs per SM; the CUDA-core decode otherwise. */
+BDFP4_API int bdfp4_decode_multi_plan(const int32_t* host_seq_lens, int B, int T_q, int H_q, int H_kv, int d_k,
+                                      int d_v, int num_sms);
+
 /* Bytes of workspace bdfp4_decode needs for this shape and chunk_tiles: the
  * fp32 partial outputs and (m, l) pairs of the splits (when a sequence can
  * have more than one), then 656 bytes per query head for the query images the
@@ -287,6 +294,33 @@ BDFP4_API int bdfp4_decode_step(const void* q, const void* k_new, const void* v_
                                 int max_pages_per_seq, int64_t num_pages, bdfp4_fmt fmt, int flags,
                                 const bdfp4_kv_params* kv, float sm_scale, int chunk_tiles, void* workspace,
                                 size_t workspace_bytes, void* out, int32_t* dev_status, void* stream);
+
+/*
+ * Decode attention for several query tokens per sequence: speculative
+ * verification or chunked decode, the T_q newest tokens of each sequence
+ * (already appended to the cache) attending causally.  The pages describe one
+ * query token per step; this extends their stacked-query MMA ("BitDecoding-FP4:
+ * Native FP4 KV Cache Decoding via Algorithm-System Co-Design", Article
+ * Summary: query operations stacked over the paged cache; "BitDecoding-FP4 :
+ * décodage natif du KV cache FP4", Analyse approfondie) from the G heads of a
+ * KV group to the G T_q (token, head) rows, which share each K/V tile read.
+ * q [B][T_q][H_q][d_k] bf16, out [B][T_q][H_q][d_v] bf16.  Query token i of
+ * sequence b (N_b = seq_lens[b] tokens, the last T_q of them the query tokens)
+ * sees the first N_b - T_q + 1 + i tokens and gets exactly bdfp4_decode's
+ * arithmetic on that prefix, with the same 128-token tiles and chunk_tiles
+ * splits from the sequence start.  A sequence with 0 < N_b < T_q sets
+ * BDFP4_DEV_BAD_SEQLEN (its rows that would see no token give zeros); N_b = 0
+ * gives zeros.  workspace: >= bdfp4_decode_workspace_size(B * T_q, H_q, d_v,
+ * max_pages_per_seq, chunk_tiles) bytes; chunk_tiles from
+ * bdfp4_decode_multi_plan (<= 0 plans from max_pages_per_seq).  Flags,
+ * layouts and other arguments as bdfp4_decode; T_q = 1 is bdfp4_decode.
+ */
+BDFP4_API int bdfp4_decode_multi(const void* q, const void* k_pages, const void* k_scales, const void* v_pages,
+                                 const void* v_scales, const int32_t* block_table, const int32_t* seq_lens, int B,
+                                 int T_q, int H_q, int H_kv, int d_k, int d_v, int max_pages_per_seq,
+                                 int64_t num_pages, bdfp4_fmt fmt, int flags, const bdfp4_kv_params* kv,
+                                 float sm_scale, int chunk_tiles, void* workspace, size_t workspace_bytes, void* out,
+                                 int32_t* dev_status, void* stream);
 
 /*
  * bdfp4_decode without a caller-provided workspace.  The paper has no

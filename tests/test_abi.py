@@ -145,6 +145,30 @@ def test_decode_argument_errors(lib):
     assert call(flags=bdfp4.FLAG_DYNAMIC_ALPHA | bdfp4.FLAG_NO_UNDERFLOW) == -1
 
 
+def test_decode_multi_argument_errors_and_plan(lib):
+    kv = bdfp4._KVParams(0x1000, 0x2000, 0x3000)
+    a = _p(0x10000)
+
+    def call(T=2, H_q=8, H_kv=2, chunk=1, ws=None, ws_bytes=0):
+        return lib.bdfp4_decode_multi(a, a, a, a, a, a, a, 2, T, H_q, H_kv, 128, 128, 4, 16, 0, 0, ctypes.byref(kv),
+                                      0.1, chunk, ws, ws_bytes, a, None, None)
+    assert call(T=0) == -1
+    assert call(H_q=7) == -2
+    # the workspace holds B T_q rows of partials and query images
+    n1 = bdfp4.bdfp4_decode_workspace_size(2, 8, 128, 4, 1)
+    n2 = bdfp4.bdfp4_decode_workspace_size(2 * 2, 8, 128, 4, 1)
+    assert n2 > n1 and call(ws=_p(0x20000), ws_bytes=n1) == -6
+    # plan: T_q = 1 is the single-token plan; four query tokens of four heads per KV head stack
+    # sixteen rows, planned as sixteen heads per KV head are
+    lens = np.full(16, 32768)
+    assert bdfp4.bdfp4_decode_multi_plan(lens, 1, 32, 8, 128, 128, 148) == \
+        bdfp4.bdfp4_decode_plan_for(lens, 32, 8, 128, 128, 148) == 29
+    assert bdfp4.bdfp4_decode_multi_plan(lens, 4, 32, 8, 128, 128, 148) == \
+        bdfp4.bdfp4_decode_plan_for(lens, 128, 8, 128, 128, 148)
+    with pytest.raises(bdfp4.BDFP4Error):
+        bdfp4.bdfp4_decode_multi_plan(lens, 0, 32, 8, 128, 128, 148)
+
+
 def test_decode_step_and_append_halves_argument_errors(lib):
     kv = bdfp4._KVParams(0x1000, 0x2000, 0x3000)
     a = _p(0x10000)
