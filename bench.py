@@ -442,9 +442,7 @@ def run_ours(args, sp, fmt):
     peak, peak_src = _peak()
     traffic = None
     tr_path = os.path.join(ROOT, "profiles", "decode_traffic.json")
-    # the variant runs on the tensor-core decode at d = 128, on the CUDA-core decode for MLA
-    cuda_core = fmt == 0 and args.dynamic_alpha and sp.d_k != 128
-    if os.path.exists(tr_path) and not cuda_core:
+    if os.path.exists(tr_path):
         rec = json.load(open(tr_path)).get(f"{args.config}_{args.fmt}" + ("_dynamic" if args.dynamic_alpha and fmt == 0 else ""))
         # the counters describe the kernel as captured: null once its sources changed
         if rec and rec.get("source_sha256") == decode_source_hash(sp.d_k):
@@ -477,8 +475,7 @@ def run_ours(args, sp, fmt):
         "roofline": {"bound": "hbm", "achieved": alg / dec_s / 1e9, "peak": peak, "unit": "GB/s",
                      "frac": alg / dec_s / 1e9 / peak, "traffic": traffic,
                      "kernel": ("bdfp4_decode calls (" +
-                                ("decode_fp4_kernel" if cuda_core else
-                                 "prep_query_kernel, decode_tc_kernel" if sp.d_k == 128 else
+                                ("prep_query_kernel, decode_tc_kernel" if sp.d_k == 128 else
                                  "prep_mla_kernel, decode_mla_tc_kernel") +
                                 ", merge_splits_kernel): median of blocks of K back-to-back calls right after the "
                                 "step blocks, one event pair per block"),
@@ -603,6 +600,8 @@ def main():
                     help="comma-separated workloads whose decode figures go under \"extra\" (N = 1 only)")
     ap.add_argument("--multi-tokens", type=int, default=4,
                     help="query tokens per sequence of the multi-token decode figure under extra (1: none)")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="sequences per GPU instead of the workload's batch (small profiling captures)")
     ap.add_argument("--min-region", type=float, default=0.5,
                     help="seconds the repeated blocks of K timed steps cover at least")
     ap.add_argument("--fmt", default="nvfp4", choices=["nvfp4", "mxfp4"])
@@ -614,7 +613,7 @@ def main():
                     help="the per-tile probability pre-scale variant (NVFP4)")
     args = ap.parse_args()
     from fp4_kv_cache_quant_b200.workloads import spec
-    sp = spec(args.config)
+    sp = spec(args.config, **({"B": args.batch} if args.batch > 0 else {}))
     fmt = 0 if args.fmt == "nvfp4" else 1
     if args.impl == "reference":
         run_reference(args, sp, fmt)

@@ -381,8 +381,7 @@ static int merge_splits(const DecodeArgs& a, cudaStream_t st) {
 
 template <int FMT, int DK, int DV>
 static int launch_decode(const DecodeArgs& a, int G, cudaStream_t st, const StepArgs* step) {
-    const bool dyn_mla = FMT == BDFP4_NVFP4 && (a.flags & BDFP4_FLAG_DYNAMIC_ALPHA);
-    const DecodePath path = decode_path(DK, DV, G, a.T_q, dyn_mla);
+    const DecodePath path = decode_path(DK, DV, G, a.T_q);
     if (path == DecodePath::kTensorCore128) {
         // tensor-core path (decode_tc.cu) on the G T_q stacked rows; a step's append runs in
         // its prologue grid
@@ -434,7 +433,6 @@ static int run_decode(const void* q, const void* k_pages, const void* k_scales, 
     if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_pages, 128) || !aligned(k_scales, 128) ||
         !aligned(v_pages, 128) || !aligned(v_scales, 128))
         return BDFP4_ERR_ALIGN;
-    const bool dyn_mla = fmt == BDFP4_NVFP4 && (flags & BDFP4_FLAG_DYNAMIC_ALPHA);
     if (chunk_tiles <= 0) {
         // no host sequence lengths: plan for the longest possible sequence
         int dev = 0, sms = 148;
@@ -442,13 +440,13 @@ static int run_decode(const void* q, const void* k_pages, const void* k_scales, 
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return BDFP4_ERR_CUDA;
         const int ntiles = (max_pages_per_seq * kPageSlots + kTileTokens - 1) / kTileTokens;
-        const DecodeShape ks = decode_shape(d_k, d_v, G, T_q, dyn_mla);
+        const DecodeShape ks = decode_shape(d_k, d_v, G, T_q);
         chunk_tiles = plan_chunk_tiles(B, [&](int) { return ntiles; }, H_kv * ks.items_per_kv_head, sms,
                                        ks.ctas_per_sm);
     }
     DecodeArgs a{};
     a.max_splits = max_splits_for(max_pages_per_seq, chunk_tiles);
-    const bool tensor_core_path = decode_path(d_k, d_v, G, T_q, dyn_mla) != DecodePath::kCudaCore;
+    const bool tensor_core_path = decode_path(d_k, d_v, G, T_q) != DecodePath::kCudaCore;
     if (a.max_splits > 1 || tensor_core_path) {
         const WorkspaceMap m = workspace_map(B * T_q, H_q, d_v, a.max_splits);
         if (!workspace || workspace_bytes < m.total) return BDFP4_ERR_WORKSPACE;
@@ -573,8 +571,7 @@ extern "C" int bdfp4_decode_noalloc(const void* q, const void* k_pages, const vo
             cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return BDFP4_ERR_CUDA;
         const int ntiles = (max_pages_per_seq * kPageSlots + kTileTokens - 1) / kTileTokens;
-        const DecodeShape ks = decode_shape(d_k, d_v, H_kv > 0 && H_q % H_kv == 0 ? H_q / H_kv : 1, 1,
-                                            fmt == BDFP4_NVFP4 && (flags & BDFP4_FLAG_DYNAMIC_ALPHA));
+        const DecodeShape ks = decode_shape(d_k, d_v, H_kv > 0 && H_q % H_kv == 0 ? H_q / H_kv : 1);
         chunk_tiles = plan_chunk_tiles(B, [&](int) { return ntiles; }, (H_kv > 0 ? H_kv : 1) * ks.items_per_kv_head,
                                        sms, ks.ctas_per_sm);
     }

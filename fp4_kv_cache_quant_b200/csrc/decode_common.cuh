@@ -98,12 +98,12 @@ inline int plan_chunk_tiles(int B, const TilesOf& tiles_of, int items, int num_s
 
 // Which decode kernel runs a shape: G query heads per KV head, T query tokens
 // per sequence (their G T rows stack per (sequence, KV head)), head dims d_k /
-// d_v; dyn_mla: the per-tile probability pre-scale with NVFP4 on MLA shapes.
+// d_v.
 enum class DecodePath { kTensorCore128, kTensorCoreMla, kCudaCore };
-inline DecodePath decode_path(int d_k, int d_v, int G, int T, bool dyn_mla) {
+inline DecodePath decode_path(int d_k, int d_v, int G, int T) {
     const int rows = G * T;
     if (d_k == 128 && d_v == 128 && rows <= 16 && (rows & (rows - 1)) == 0) return DecodePath::kTensorCore128;
-    if (d_k == 576 && d_v == 512 && T == 1 && !dyn_mla && (G == 16 || G == 32 || G == 64 || G == 128))
+    if (d_k == 576 && d_v == 512 && T == 1 && (G == 16 || G == 32 || G == 64 || G == 128))
         return DecodePath::kTensorCoreMla;
     return DecodePath::kCudaCore;
 }
@@ -121,8 +121,8 @@ inline int cuda_core_rows(int rows) {
 struct DecodeShape {
     int ctas_per_sm, items_per_kv_head;
 };
-inline DecodeShape decode_shape(int d_k, int d_v, int G, int T = 1, bool dyn_mla = false) {
-    switch (decode_path(d_k, d_v, G, T, dyn_mla)) {
+inline DecodeShape decode_shape(int d_k, int d_v, int G, int T = 1) {
+    switch (decode_path(d_k, d_v, G, T)) {
         case DecodePath::kTensorCore128: return {G * T <= 4 ? 4 : 3, 1};                  // decode_tc.cu
         case DecodePath::kTensorCoreMla: return {1, G > 64 ? G / 64 : 1};                   // decode_mla_tc.cu
         default: return {8, G * T / cuda_core_rows(G * T)};                                 // CUDA-core decode

@@ -25,6 +25,7 @@
 #include "bdfp4_device.cuh"
 #include "decode_common.cuh"
 #include "host_common.h"
+#include "prob_scale.cuh"
 #include "quant_device.cuh"
 #include "tc_ptx.cuh"
 
@@ -194,7 +195,10 @@ __global__ void __launch_bounds__(256) prep_mla_kernel(const DecodeArgs a, const
 }
 
 // ---------------------------------------------------------------- decode
-template <int FMT, int GH>
+// DYN (NVFP4): the probability pre-scale alpha = 2^E per tile and head; a head's
+// O^T and l are held in units of its current tile's alpha, so a change of E joins
+// the running-maximum correction as the exact factor 2^(E - E_prev).
+template <int FMT, int GH, bool DYN = false>
 __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_kernel(const DecodeArgs a) {
     using C = MlaCfg<FMT, GH>;
     // the split merge (a programmatic dependent) may be scheduled as CTAs of this grid retire
@@ -531,6 +535,7 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
         uint32_t* const wcode = reinterpret_cast<uint32_t*>(wst + warp * C::WST_WARP + HG * 32);   // [HG]
         float* const wout = reinterpret_cast<float*>(wst + warp * C::WST_WARP + HG * 36);          // [HG]
         float m_lane = -INFINITY;                   // running maximum of head gb + lane
+        int e_lane = 11;                            // DYN: log2 of head gb + lane's current pre-scale
         const float ls_lane = lane < HG ? lsc[gb + lane] : 0.0f;
         float l_part[HG];
 #pragma unroll
@@ -597,10 +602,19 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
                                            fmaxf(fmaxf(w1.x, w1.y), fmaxf(w1.z, w1.w)));
                     const float mn = fmaxf(m_lane, mt * ls_lane);
                     const float mz = mn == -INFINITY ? 0.0f : mn;
-                    const float corr = tc::ex2_approx(m_lane - mz);   // 0 on the split's first tile
-                    const float base = mz - la;
+                    float corr = tc::ex2_approx(m_lane - mz);   // 0 on the split's first tile
+                    float base = mz - la;
                     rose = mn != m_lane;
                     m_lane = mn;
+                    if constexpr (DYN) {
+                        // this tile's pre-scale from its largest probability; O^T and l move to
+                        // its units (an exact power of two, folded into corr)
+                        const int e = dynamic_alpha_exp(tc::ex2_approx(fmaf(mt, ls_lane, -mz)));
+                        corr *= pow2f(e - e_lane);
+                        rose |= e != e_lane;
+                        e_lane = e;
+                        base = mz - (float)e;
+                    }
                     const float bm_lo = w[qd * 2], bm_hi = w[qd * 2 + 1];
                     // per block: NVFP4 {ls, base, corr, 1 / scale}, the element is alpha p / scale;
                     // MXFP4 {ls, base + e, corr, 2^e} for the scale 2^e, the element is 2^(x ls - base - e)
@@ -766,11 +780,13 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
             if (lane < HG) {
                 const float4 r4 = *reinterpret_cast<const float4*>(rl + (gb + lane) * 4);
                 const float l = r4.x + r4.y + r4.z + r4.w;
-                wout[lane] = nspl == 1 ? (l > 0.0f ? oscale / l : 0.0f) : oscale;
+                // DYN: splits end in different units; the partials leave in the units of p
+                const float un = DYN ? pow2f(-e_lane) : 1.0f;
+                wout[lane] = nspl == 1 ? (l > 0.0f ? oscale / l : 0.0f) : oscale * un;
                 if (nspl > 1 && qd == 0) {
                     const int64_t row = (int64_t)b * a.H_q + h0 + gb + lane;
                     a.ws_ml[(row * a.max_splits + split) * 2 + 0] = m_lane;
-                    a.ws_ml[(row * a.max_splits + split) * 2 + 1] = l;
+                    a.ws_ml[(row * a.max_splits + split) * 2 + 1] = l * un;
                 }
             }
             __syncwarp();
@@ -800,14 +816,14 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
     }
 }
 
-template <int FMT, int GH>
+template <int FMT, int GH, bool DYN = false>
 static int launch_mla(const DecodeArgs& a, cudaStream_t st, const StepArgs* step) {
     using C = MlaCfg<FMT, GH>;
     using RG = RowGeom<FMT, 576>;
     static bool attr_set = false;
     if (!attr_set) {
-        const cudaError_t e =
-            cudaFuncSetAttribute(decode_mla_tc_kernel<FMT, GH>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        const cudaError_t e = cudaFuncSetAttribute(decode_mla_tc_kernel<FMT, GH, DYN>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
         if (e != cudaSuccess) {
             record_cuda_error(e);
             return BDFP4_ERR_CUDA;
@@ -839,7 +855,7 @@ static int launch_mla(const DecodeArgs& a, cudaStream_t st, const StepArgs* step
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_mla_tc_kernel<FMT, GH>, a);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_mla_tc_kernel<FMT, GH, DYN>, a);
     if (e != cudaSuccess) {
         record_cuda_error(e);
         return BDFP4_ERR_CUDA;
@@ -861,7 +877,13 @@ int mla_query_image_bytes(int fmt, int G) {
 
 int launch_decode_mla_tc(const DecodeArgs& a, int fmt, int G, cudaStream_t st, const StepArgs* step) {
     const int gh = G < 64 ? G : 64;
-    if (fmt == BDFP4_NVFP4) {
+    if (fmt == BDFP4_NVFP4 && (a.flags & BDFP4_FLAG_DYNAMIC_ALPHA)) {
+        switch (gh) {
+            case 16: return launch_mla<BDFP4_NVFP4, 16, true>(a, st, step);
+            case 32: return launch_mla<BDFP4_NVFP4, 32, true>(a, st, step);
+            case 64: return launch_mla<BDFP4_NVFP4, 64, true>(a, st, step);
+        }
+    } else if (fmt == BDFP4_NVFP4) {
         switch (gh) {
             case 16: return launch_mla<BDFP4_NVFP4, 16>(a, st, step);
             case 32: return launch_mla<BDFP4_NVFP4, 32>(a, st, step);

@@ -98,9 +98,10 @@ typedef enum { BDFP4_NVFP4 = 0, BDFP4_MXFP4 = 1 } bdfp4_fmt;
  * E the largest integer with p_max 2^E <= 2688 (p_max the tile's largest
  * probability relative to the running maximum), clamped to [11, 64]; each
  * tile's alpha is divided out of its quantized probabilities.  A tile that
- * raises the running maximum keeps the static 2^11.  Runs on the tensor-core
- * decode at d = 128 and on the CUDA-core decode for MLA shapes; with MXFP4 it
- * changes nothing; with BDFP4_FLAG_NO_UNDERFLOW it is BDFP4_ERR_ARG. */
+ * raises the running maximum keeps the static 2^11.  Runs in every decode
+ * kernel (the tensor-core decodes at d = 128 and for MLA shapes, the CUDA-core
+ * decode); with MXFP4 it changes nothing; with BDFP4_FLAG_NO_UNDERFLOW it is
+ * BDFP4_ERR_ARG. */
 #define BDFP4_FLAG_DYNAMIC_ALPHA 32
 
 /* Static per-layer quantization parameters (device pointers), produced by

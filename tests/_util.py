@@ -37,23 +37,28 @@ def compare_outputs(gpu: np.ndarray, ref: np.ndarray):
     [16, 32) -- the MLA workload's outlier value channels reach there).  An
     element one step or less from the oracle's therefore counts as agreeing;
     max_abs is the largest difference among the others, and step_frac is the
-    fraction of elements that needed that allowance (more than 1e-2 apart but
-    within one step)."""
+    fraction of the elements where the allowance can apply at all (one step
+    larger than 1e-2) that needed it (more than 1e-2 apart)."""
     g = gpu.astype(np.float64)
     r = ref.astype(np.float64)
     d = np.abs(g - r)
-    step = d <= bf16_ulp(r)
+    ulp = bf16_ulp(r)
+    step = d <= ulp
     d = np.where(step, 0.0, d)
     max_abs = float(np.max(d)) if g.size else 0.0
     rel = float(np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-30))
-    step_frac = float(np.count_nonzero(step & (np.abs(g - r) > MAX_ABS)) / g.size) if g.size else 0.0
+    large = ulp > MAX_ABS
+    used = np.count_nonzero(step & (np.abs(g - r) > MAX_ABS))
+    step_frac = float(used / np.count_nonzero(large)) if used else 0.0
     return max_abs, rel, step_frac
 
 
-# Largest fraction of elements that may use the one-bf16-step allowance of
-# compare_outputs: a rounding straddle is rare, so a kernel off by one step on
-# many large outputs fails even though each element alone would pass.
-STEP_FRAC = 1e-3
+# Largest fraction of the large elements (one bf16 step above 1e-2) that may use
+# the one-step allowance.  Two results a relative distance e apart straddle a
+# bf16 rounding boundary with probability about e / 2^-8; at the relative-L2
+# errors these decodes reach (about 1e-3) that is a few in a hundred, so a kernel
+# off by one step on most large outputs fails, though each element alone passes.
+STEP_FRAC = 0.5
 
 
 def assert_close(gpu: np.ndarray, ref: np.ndarray, *ctx):

@@ -227,6 +227,24 @@ def test_output_comparison_counts_one_bf16_step_as_agreement():
     assert compare_outputs(np.array([1.0]), np.array([1.0078125]))[0] == 0.0   # one step at [1, 2)
     assert abs(compare_outputs(np.array([0.5]), np.array([0.52]))[0] - 0.02) < 1e-12
     assert compare_outputs(np.array([3.0]), np.array([3.0]))[1] == 0.0
+    # the allowance counts among the elements it can apply to (one step above 1e-2)
+    assert compare_outputs(np.array([16.0, 0.5, 3.0]), np.array([16.125, 0.5, 3.0]))[2] == 0.5
+
+
+def test_decode_bound_rejects_a_kernel_a_step_off_on_most_large_outputs():
+    """Every element one bf16 step off passes max-abs alone; the bound on the
+    allowance's use among large outputs fails it, while a rare straddle passes."""
+    from _util import assert_close, bf16_ulp
+
+    rng = np.random.default_rng(0)
+    ref = np.concatenate([rng.uniform(2.0, 30.0, 400), rng.uniform(-0.5, 0.5, 4000)])
+    ref = (ref.astype(np.float32).view(np.uint32) & 0xFFFF0000).view(np.float32).astype(np.float64)   # bf16 values
+    off = ref + np.where(np.abs(ref) >= 2.0, bf16_ulp(ref), 0.0)
+    with pytest.raises(AssertionError):
+        assert_close(off, ref)
+    rare = ref.copy()
+    rare[:10] += bf16_ulp(ref[:10])
+    assert_close(rare, ref)
 
 
 def test_decode_plan_minimises_the_documented_wave_cost(lib):

@@ -329,6 +329,39 @@ def test_decode_dynamic_alpha_matches_oracle(ora, lib, name, chunk):
     assert_close(got, ref)
 
 
+@pytest.mark.parametrize("name", ["mla_nv", "mla64_nv", "mla128_nv"])
+def test_dynamic_alpha_runs_on_the_mla_tensor_core_kernel(ora, lib, name):
+    """MLA shapes with the per-tile pre-scale take the tensor-core kernel: it needs a
+    workspace for its query images even with one split, which the CUDA-core decode
+    does not, so a workspace-less single-split call is refused before any launch."""
+    sp, fmt = SMALL[name]
+    wl = Workload(sp, seed=5)
+    smooth, kg, vg = oracle_calibration(ora, wl)
+    gcache = bdfp4.FP4Cache.empty(wl.num_pages, sp.H_kv, sp.d_k, sp.d_v, fmt)
+    one_split = (wl.max_pages * 64 + 127) // 128
+    out = torch.empty((sp.B, sp.H_q, sp.d_v), dtype=torch.bfloat16, device="cuda")
+    args = (wl.queries().cuda(), gcache, torch.from_numpy(wl.block_table).cuda(), torch.from_numpy(wl.seq_lens).cuda(),
+            kv_params_gpu(smooth, kg, vg), sp.sm_scale, one_split, None, out)
+    with pytest.raises(bdfp4.BDFP4Error, match="workspace"):
+        bdfp4.bdfp4_decode(*args, flags=bdfp4.FLAG_DYNAMIC_ALPHA)
+    # a shape the tensor-core kernels do not take runs without one
+    sp8, _ = SMALL["mla8_cuda_mx"]
+    wl8 = Workload(sp8, seed=5)
+    s8, k8, v8 = oracle_calibration(ora, wl8)
+    c8 = bdfp4.FP4Cache.empty(wl8.num_pages, sp8.H_kv, sp8.d_k, sp8.d_v, NV)
+    o8 = torch.empty((sp8.B, sp8.H_q, sp8.d_v), dtype=torch.bfloat16, device="cuda")
+    bdfp4.bdfp4_decode(wl8.queries().cuda(), c8, torch.from_numpy(wl8.block_table).cuda(),
+                       torch.from_numpy(wl8.seq_lens).cuda(), kv_params_gpu(s8, k8, v8), sp8.sm_scale,
+                       (wl8.max_pages * 64 + 127) // 128, None, o8, flags=bdfp4.FLAG_DYNAMIC_ALPHA)
+    torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("chunk", [0, 1])
+@pytest.mark.parametrize("name", ["mla_nv", "mla128_nv"])
+def test_decode_step_dynamic_alpha_mla_matches_oracle(ora, lib, name, chunk):
+    _decode_step_case(ora, name, chunk, bdfp4.FLAG_DYNAMIC_ALPHA)
+
+
 def test_dynamic_alpha_keeps_a_deep_sink_tail(ora, lib):
     """One key with logit 14 and 131071 with logit 0, one split: with alpha = 2^11
     every block without the sink collapses (E4M3(e^-14 2^11 / 6) = 0), a tenth of
