@@ -55,10 +55,8 @@ struct TcCfg {
     // CTAs per SM the rings are shallower (the SM holds as many tiles in flight)
     static constexpr int NSK = MIN_CTAS == 4 ? 3 : 4;
     static constexpr int NSV = MIN_CTAS == 4 ? 2 : 3;
-    // tiles the V copies trail the K copies by: one (only PV needs V, and K is needed
-    // first), except for MXFP4 with the three-stage V ring, whose softmax warps also read
-    // each tile's V scales (2% faster on the 30B shape; with two V stages it was slower)
-    static constexpr int VLAG = (FMT == BDFP4_MXFP4 && NSV == 3) ? 0 : 1;
+    // tiles the V copies trail the K copies by: one (only PV needs V, and K is needed first)
+    static constexpr int VLAG = 1;
     // softmax warpgroups: warps w and w + 4 read the same TMEM lanes (tokens), so
     // two groups split the query heads of every tile between them
     static constexpr int NSG = G >= 2 ? 2 : 1;
@@ -99,9 +97,11 @@ struct TcCfg {
     static constexpr int SM_LSC = SM_QSC + NQ * 8;
     static constexpr int SM_P = SM_Q + QPACK;
     static constexpr int SM_PSF = (SM_P + 2 * P_BUF + 127) / 128 * 128;  // [2 buf][2 page][32 rows][16 B] P scales
+    // MXFP4: [2 buf][32 rows][16 B] V scales of a tile's two pages, interleaved by the MMA warp
+    static constexpr int SM_VSF = SM_PSF + 2 * 2 * 512;
     // per S buffer: [G][4] warp maxima (floats)
     static constexpr int RED_BUF = 4 * G;
-    static constexpr int SM_RED = SM_PSF + 2 * 2 * 512;
+    static constexpr int SM_RED = SM_VSF + (FMT == BDFP4_MXFP4 ? 2 * 512 : 0);
     static constexpr int SM_BARS = (SM_RED + 2 * RED_BUF * 4 + 7) / 8 * 8;
     static constexpr int NBARS = 2 * NSK + 2 * NSV + 8;
     static constexpr int SM_MISC = SM_BARS + NBARS * 8;                  // tmem slot, abort flags
@@ -111,7 +111,9 @@ struct TcCfg {
     static constexpr int T_S = 0;
     static constexpr int T_O = 2 * NQ;
     static constexpr int T_SFK = ((T_O + NP + 3) / 4) * 4;       // 2 x (4 per K scale group x NKG)
-    static constexpr int T_SFV = T_SFK + 2 * 4 * NKG;            // 2 x (4 per page x 2 pages)
+    // 2 x (4 per page x 2 pages); MXFP4 2 x 4: a column holds a channel's 2 scale bytes of
+    // each page, page 0 in bytes 0-1 and page 1 in bytes 2-3 (scale-factor id 2)
+    static constexpr int T_SFV = T_SFK + 2 * 4 * NKG;
     // every scale-factor operand starts on a 4-column boundary (one 32-bit
     // column per 32 rows of a 128-row chunk), B operands included
     static constexpr int T_SFQ = T_SFV + 2 * 8;                  // KS x 4 columns
@@ -413,75 +415,134 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
         if (!ok && lane == 0) *abort_flag = 1;
     } else if (warp == C::MMA_WARP) {
         // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc_qk = tc::idesc_fp4(C::NQ, MX);
-            constexpr uint32_t idesc_pv = tc::idesc_fp4(C::NP, MX);
-            const uint32_t q_addr = tc::smem_u32(q_op);
-            const uint32_t p_addr = tc::smem_u32(p_op);
-            const uint32_t kst_addr = tc::smem_u32(smem + C::SM_KST);
-            const uint32_t vst_addr = tc::smem_u32(smem + C::SM_VST);
-            const uint32_t psf_addr = tc::smem_u32(psf);
-            auto issue_qk = [&](int j) -> bool {
+        // Lane 0 issues every tcgen05 operation and takes the waits; the warp follows it
+        // through the loop, and with MXFP4 all its lanes wait for each V stage and build the
+        // tile's V scale-factor source: per channel group, the 2 bytes of page 0 and of page 1
+        // side by side, so one tcgen05.cp serves both pages' MMAs (scale-factor ids 0 and 2).
+        const bool leader = lane == 0;
+        constexpr uint32_t idesc_qk = tc::idesc_fp4(C::NQ, MX);
+        constexpr uint32_t idesc_pv = tc::idesc_fp4(C::NP, MX);
+        const uint32_t q_addr = tc::smem_u32(q_op);
+        const uint32_t p_addr = tc::smem_u32(p_op);
+        const uint32_t kst_addr = tc::smem_u32(smem + C::SM_KST);
+        const uint32_t vst_addr = tc::smem_u32(smem + C::SM_VST);
+        const uint32_t psf_addr = tc::smem_u32(psf);
+        const uint32_t vsf_addr = tc::smem_u32(smem + C::SM_VSF);
+        auto issue_qk = [&](int j) -> bool {
+            bool ok = true;
+            if (leader) {
                 const int s = j % C::NSK, buf = j & 1;
-                if (!tc::mbar_wait(&kfull[s], (j / C::NSK) & 1, abort_flag, kWaitLimit)) return false;
-                tc::tc_fence_after();
-                // the scale rows came through cp.async (generic proxy); tcgen05.cp reads them
-                // through the async proxy
-                tc::fence_proxy_async_smem();
-                const uint32_t kt = kst_addr + s * C::KSTAGE + C::OFF_K;
-                // K scale factors: each 512-byte group chunk is the 32 x 16-byte copy source
+                ok = tc::mbar_wait(&kfull[s], (j / C::NSK) & 1, abort_flag, kWaitLimit);
+                if (ok) {
+                    tc::tc_fence_after();
+                    // the scale rows came through cp.async (generic proxy); tcgen05.cp reads them
+                    // through the async proxy
+                    tc::fence_proxy_async_smem();
+                    const uint32_t kt = kst_addr + s * C::KSTAGE + C::OFF_K;
+                    // K scale factors: each 512-byte group chunk is the 32 x 16-byte copy source
 #pragma unroll
-                for (int kg = 0; kg < C::NKG; ++kg)
-                    tc::tmem_cp_32x128b_x4(tbase + C::T_SFK + (buf * C::NKG + kg) * 4,
-                                           tc::smem_desc(kt - C::OFF_K + C::OFF_KS + kg * 512, 128, 128));
+                    for (int kg = 0; kg < C::NKG; ++kg)
+                        tc::tmem_cp_32x128b_x4(tbase + C::T_SFK + (buf * C::NKG + kg) * 4,
+                                               tc::smem_desc(kt - C::OFF_K + C::OFF_KS + kg * 512, 128, 128));
 #pragma unroll
-                for (int ks = 0; ks < C::KS; ++ks) {
-                    // MXFP4 packs two K steps per scale column: byte offset 2 (sf id) for the odd step
-                    const uint32_t sfid = (uint32_t)(ks % C::KPG) * 2u;
-                    tc::mma_fp4<MX>(tbase + C::T_S + buf * C::NQ, tc::smem_desc(kt + ks * 256, 128, 512),
-                                    tc::smem_desc(q_addr + ks * 256, 128, 512), idesc_qk | (sfid << 29),
-                                    (tbase + C::T_SFK + (buf * C::NKG + ks / C::KPG) * 4) | (sfid << 30),
-                                    tbase + C::T_SFQ + ks * 4, ks > 0);
+                    for (int ks = 0; ks < C::KS; ++ks) {
+                        // MXFP4 packs two K steps per scale column: byte offset 2 (sf id) for the odd step
+                        const uint32_t sfid = (uint32_t)(ks % C::KPG) * 2u;
+                        tc::mma_fp4<MX>(tbase + C::T_S + buf * C::NQ, tc::smem_desc(kt + ks * 256, 128, 512),
+                                        tc::smem_desc(q_addr + ks * 256, 128, 512), idesc_qk | (sfid << 29),
+                                        (tbase + C::T_SFK + (buf * C::NKG + ks / C::KPG) * 4) | (sfid << 30),
+                                        tbase + C::T_SFQ + ks * 4, ks > 0);
+                    }
+                    tc::mma_commit(&s_full[buf]);
+                    tc::mma_commit(&kempty[s]);   // the K stage is free once QK has read it
                 }
-                tc::mma_commit(&s_full[buf]);
-                tc::mma_commit(&kempty[s]);   // the K stage is free once QK has read it
-                return true;
-            };
-            // the softmax warps quantize the query into shared memory and TMEM first
-            bool ok = tc::mbar_wait(q_ready, 0, abort_flag, kWaitLimit);
-            if (ok) tc::tc_fence_after();
-            ok = ok && issue_qk(0);
-            for (int j = 0; ok && j < n; ++j) {
-                if (j + 1 < n && !(ok = issue_qk(j + 1))) break;
-                const int s = j % C::NSV, buf = j & 1;
-                if (!(ok = tc::mbar_wait(&p_ready[buf], (j >> 1) & 1, abort_flag, kWaitLimit))) break;
-                if (!(ok = tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, kWaitLimit))) break;
-                tc::tc_fence_after();
-                const uint32_t vt = vst_addr + s * C::VSTAGE + C::OFF_V;
-                // scale factors of P (written by the softmax warps) and, for NVFP4, of V
-                // (the page's scale block is already in the 32 x 16-byte copy layout)
-#pragma unroll
-                for (int p = 0; p < 2; ++p) {
-                    tc::tmem_cp_32x128b_x4(tbase + C::T_SFP + (buf * 2 + p) * 4,
-                                           tc::smem_desc(psf_addr + (buf * 2 + p) * 512, 128, 128));
-                    if constexpr (!MX)
-                        tc::tmem_cp_32x128b_x4(tbase + C::T_SFV + buf * 8 + p * 4,
-                                               tc::smem_desc(vt - C::OFF_V + C::OFF_VS + p * C::VS_PAGE, 128, 128));
-                }
-#pragma unroll
-                for (int p = 0; p < 2; ++p) {
-                    // O^T accumulates across the split's tiles (the softmax warps rescale it in
-                    // place when a running maximum rises)
-                    tc::mma_fp4<MX>(tbase + C::T_O, tc::smem_desc(vt + p * C::V_PAGE, 128, 256),
-                                    tc::smem_desc(p_addr + buf * C::P_BUF + p * C::P_PAGE, 128, 256), idesc_pv,
-                                    tbase + C::T_SFV + buf * 8 + p * 4, tbase + C::T_SFP + (buf * 2 + p) * 4,
-                                    (j > 0 || p > 0) ? 1u : 0u);
-                }
-                tc::mma_commit(&o_full[buf]);
-                tc::mma_commit(&vempty[s]);
             }
-            if (!ok) *abort_flag = 1;
+            return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        };
+        // the softmax warps quantize the query into shared memory and TMEM first (every lane
+        // waits: with MXFP4 the lanes read the page flags those warps wrote before)
+        bool ok = __all_sync(0xffffffffu, tc::mbar_wait(q_ready, 0, abort_flag, kWaitLimit));
+        if (ok) tc::tc_fence_after();
+        // MXFP4: the split's page flags (written by the softmax warps before q_ready)
+        const bool any_bad_page = MX && ok && *reinterpret_cast<volatile int*>(smem + C::SM_PFLAG + 64) != 0;
+        ok = ok && issue_qk(0);
+        for (int j = 0; ok && j < n; ++j) {
+            if (j + 1 < n && !(ok = issue_qk(j + 1))) break;
+            const int s = j % C::NSV, buf = j & 1;
+            bool w = true;
+            if (leader) w = tc::mbar_wait(&p_ready[buf], (j >> 1) & 1, abort_flag, kWaitLimit);
+            if (!(ok = __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0)) break;
+            if constexpr (MX) {
+                w = tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, kWaitLimit);
+                if (!(ok = __all_sync(0xffffffffu, w))) break;
+                // row `lane` of the source: TMEM lane `lane`, column c <- channel 32 c + lane;
+                // blocks past the sequence end and blocks of pages the block table gets wrong
+                // are zeroed (their bytes are never multiplied)
+                const int tile = tile0 + j;
+                const uint8_t* vs = smem + C::SM_VST + s * C::VSTAGE + C::OFF_VS;
+                const uint2 w0 = *reinterpret_cast<const uint2*>(vs + 8 * lane);
+                const uint2 w1 = *reinterpret_cast<const uint2*>(vs + C::VS_PAGE + 8 * lane);
+                uint32_t msk[2];
+#pragma unroll
+                for (int p = 0; p < 2; ++p) {
+                    int nvb = (N - (tile * kTileTokens + p * kPageSlots) + B - 1) / B;
+                    nvb = nvb < 0 ? 0 : (nvb > C::SPB ? C::SPB : nvb);
+                    if (any_bad_page) {
+                        const uint32_t f = j < 64 ? (smem + C::SM_PFLAG)[j] : 0u;
+                        if (j >= 64) {
+                            const int pi = tile * 2 + p;
+                            const int v = pi * kPageSlots < N ? __ldg(a.block_table + (int64_t)b * a.max_pages + pi) : 0;
+                            if (v < 0 || v >= a.num_pages) nvb = 0;
+                        } else if (!(f & (1u << p))) {
+                            nvb = 0;
+                        }
+                    }
+                    const uint32_t m16 = nvb >= 2 ? 0xffffu : ((1u << (8 * nvb)) - 1u);
+                    msk[p] = m16 | (m16 << 16);
+                }
+                const uint32_t x0 = w0.x & msk[0], x1 = w0.y & msk[0], y0 = w1.x & msk[1], y1 = w1.y & msk[1];
+                *reinterpret_cast<uint4*>(smem + C::SM_VSF + buf * 512 + 16 * lane) =
+                    make_uint4(__byte_perm(x0, y0, 0x5410), __byte_perm(x0, y0, 0x7632), __byte_perm(x1, y1, 0x5410),
+                               __byte_perm(x1, y1, 0x7632));
+                tc::fence_proxy_async_smem();
+                __syncwarp();
+            }
+            if (leader) {
+                if constexpr (!MX) ok = tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, kWaitLimit);
+                if (ok) {
+                    tc::tc_fence_after();
+                    const uint32_t vt = vst_addr + s * C::VSTAGE + C::OFF_V;
+                    // scale factors of P (written by the softmax warps) and of V: NVFP4 a page's scale
+                    // block is already in the 32 x 16-byte copy layout, MXFP4 the interleaved rows
+#pragma unroll
+                    for (int p = 0; p < 2; ++p) {
+                        tc::tmem_cp_32x128b_x4(tbase + C::T_SFP + (buf * 2 + p) * 4,
+                                               tc::smem_desc(psf_addr + (buf * 2 + p) * 512, 128, 128));
+                        if constexpr (!MX)
+                            tc::tmem_cp_32x128b_x4(tbase + C::T_SFV + buf * 8 + p * 4,
+                                                   tc::smem_desc(vt - C::OFF_V + C::OFF_VS + p * C::VS_PAGE, 128, 128));
+                    }
+                    if constexpr (MX)
+                        tc::tmem_cp_32x128b_x4(tbase + C::T_SFV + buf * 4, tc::smem_desc(vsf_addr + buf * 512, 128, 128));
+#pragma unroll
+                    for (int p = 0; p < 2; ++p) {
+                        // O^T accumulates across the split's tiles (the softmax warps rescale it in
+                        // place when a running maximum rises)
+                        const uint32_t sfid = MX ? (uint32_t)p * 2u : 0u;
+                        const uint32_t sfa = MX ? (tbase + C::T_SFV + buf * 4) | (sfid << 30)
+                                                : tbase + C::T_SFV + buf * 8 + p * 4;
+                        tc::mma_fp4<MX>(tbase + C::T_O, tc::smem_desc(vt + p * C::V_PAGE, 128, 256),
+                                        tc::smem_desc(p_addr + buf * C::P_BUF + p * C::P_PAGE, 128, 256),
+                                        idesc_pv | (sfid << 29), sfa, tbase + C::T_SFP + (buf * 2 + p) * 4,
+                                        (j > 0 || p > 0) ? 1u : 0u);
+                    }
+                    tc::mma_commit(&o_full[buf]);
+                    tc::mma_commit(&vempty[s]);
+                }
+            }
+            if (!(ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0)) break;
         }
+        if (!ok && leader) *abort_flag = 1;
     } else {
         // ------------------------------------------------------------ softmax warps
         const int grp = warp >> 2;                 // head group
@@ -706,14 +767,15 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                     tc::tmem_wait_st();
                     tc::tc_fence_before();
                 }
-                // V scale factors (group 0): blocks past the sequence end are zeroed, so the
+                // NVFP4 V scale factors (group 0): blocks past the sequence end are zeroed, so the
                 // bytes a page holds there are never multiplied.  The V stage can not be
-                // refilled before this tile's PV, so waiting for it here is safe.
-                if (grp == 0) {
-                    const int s = j % C::NSV;
-                    const bool tail = (tile + 1) * kTileTokens > N;
-                    uint8_t* vs = smem + C::SM_VST + s * C::VSTAGE + C::OFF_VS;
-                    if constexpr (B == 16) {
+                // refilled before this tile's PV, so waiting for it here is safe.  (MXFP4: the
+                // MMA warp builds the tile's V scale rows and masks them.)
+                if constexpr (B == 16) {
+                    if (grp == 0) {
+                        const int s = j % C::NSV;
+                        const bool tail = (tile + 1) * kTileTokens > N;
+                        uint8_t* vs = smem + C::SM_VST + s * C::VSTAGE + C::OFF_VS;
                         if (tail || !pok0 || !pok1) {
                             if (!tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, kWaitLimit)) bad = true;
     #pragma unroll
@@ -726,25 +788,6 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                                     vs[p * C::VS_PAGE + (chan & 31) * 16 + (chan >> 5) * 4 + bb] = 0;
                             }
                         }
-                    } else {
-                        if (!tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, kWaitLimit)) bad = true;
-                        uint32_t v[8];
-    #pragma unroll
-                        for (int p = 0; p < 2; ++p) {
-                            const int t0 = tile * kTileTokens + p * kPageSlots;
-                            int nvb = (N - t0 + B - 1) / B;
-                            nvb = nvb < 0 ? 0 : (nvb > C::SPB ? C::SPB : nvb);
-                            if (!(p ? pok1 : pok0)) nvb = 0;
-                            const uint32_t mask = nvb >= 2 ? 0xffffu : ((1u << (8 * nvb)) - 1u);
-                            const uint2 w = *reinterpret_cast<const uint2*>(vs + p * C::VS_PAGE + 8 * lane);
-                            v[p * 4 + 0] = w.x & mask;
-                            v[p * 4 + 1] = (w.x >> 16) & mask;
-                            v[p * 4 + 2] = w.y & mask;
-                            v[p * 4 + 3] = (w.y >> 16) & mask;
-                        }
-                        tc::tmem_st8(tq + C::T_SFV + buf * 8, v);
-                        tc::tmem_wait_st();
-                        tc::tc_fence_before();
                     }
                 }
                 tc::fence_proxy_async_smem();
