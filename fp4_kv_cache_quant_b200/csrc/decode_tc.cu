@@ -415,26 +415,34 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
         if (!ok && lane == 0) *abort_flag = 1;
     } else if (warp == C::MMA_WARP) {
         // ------------------------------------------------------------ MMA issuer
-        // Lane 0 issues every tcgen05 operation and takes the waits; the warp follows it
-        // through the loop, and with MXFP4 all its lanes wait for each V stage and build the
-        // tile's V scale-factor source: per channel group, the 2 bytes of page 0 and of page 1
-        // side by side, so one tcgen05.cp serves both pages' MMAs (scale-factor ids 0 and 2).
-        const bool leader = lane == 0;
-        constexpr uint32_t idesc_qk = tc::idesc_fp4(C::NQ, MX);
-        constexpr uint32_t idesc_pv = tc::idesc_fp4(C::NP, MX);
-        const uint32_t q_addr = tc::smem_u32(q_op);
-        const uint32_t p_addr = tc::smem_u32(p_op);
-        const uint32_t kst_addr = tc::smem_u32(smem + C::SM_KST);
-        const uint32_t vst_addr = tc::smem_u32(smem + C::SM_VST);
-        const uint32_t psf_addr = tc::smem_u32(psf);
-        const uint32_t vsf_addr = tc::smem_u32(smem + C::SM_VSF);
-        auto issue_qk = [&](int j) -> bool {
-            bool ok = true;
-            if (leader) {
+        // Lane 0 issues every tcgen05 operation.  NVFP4: the other lanes leave (a lane that
+        // spins alone while the rest of its warp waits for it costs issue slots).  MXFP4: all
+        // lanes run every wait themselves, converged, because they also build each tile's V
+        // scale-factor source: per channel group, the 2 bytes of page 0 and of page 1 side by
+        // side, so one tcgen05.cp serves both pages' MMAs (scale-factor ids 0 and 2).
+        if (MX || lane == 0) {
+            const bool leader = lane == 0;
+            // a decision every lane inside takes alike
+            auto all = [&](bool v) -> bool {
+                if constexpr (MX) return __all_sync(0xffffffffu, v);
+                else return v;
+            };
+            auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+                return all(tc::mbar_wait(bar, parity, abort_flag, kWaitLimit));
+            };
+            constexpr uint32_t idesc_qk = tc::idesc_fp4(C::NQ, MX);
+            constexpr uint32_t idesc_pv = tc::idesc_fp4(C::NP, MX);
+            const uint32_t q_addr = tc::smem_u32(q_op);
+            const uint32_t p_addr = tc::smem_u32(p_op);
+            const uint32_t kst_addr = tc::smem_u32(smem + C::SM_KST);
+            const uint32_t vst_addr = tc::smem_u32(smem + C::SM_VST);
+            const uint32_t psf_addr = tc::smem_u32(psf);
+            const uint32_t vsf_addr = tc::smem_u32(smem + C::SM_VSF);
+            auto issue_qk = [&](int j) -> bool {
                 const int s = j % C::NSK, buf = j & 1;
-                ok = tc::mbar_wait(&kfull[s], (j / C::NSK) & 1, abort_flag, kWaitLimit);
-                if (ok) {
-                    tc::tc_fence_after();
+                if (!wait(&kfull[s], (j / C::NSK) & 1)) return false;
+                tc::tc_fence_after();
+                if (leader) {
                     // the scale rows came through cp.async (generic proxy); tcgen05.cp reads them
                     // through the async proxy
                     tc::fence_proxy_async_smem();
@@ -456,61 +464,54 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                     tc::mma_commit(&s_full[buf]);
                     tc::mma_commit(&kempty[s]);   // the K stage is free once QK has read it
                 }
-            }
-            return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        };
-        // the softmax warps quantize the query into shared memory and TMEM first (every lane
-        // waits: with MXFP4 the lanes read the page flags those warps wrote before)
-        bool ok = __all_sync(0xffffffffu, tc::mbar_wait(q_ready, 0, abort_flag, kWaitLimit));
-        if (ok) tc::tc_fence_after();
-        // MXFP4: the split's page flags (written by the softmax warps before q_ready)
-        const bool any_bad_page = MX && ok && *reinterpret_cast<volatile int*>(smem + C::SM_PFLAG + 64) != 0;
-        ok = ok && issue_qk(0);
-        for (int j = 0; ok && j < n; ++j) {
-            if (j + 1 < n && !(ok = issue_qk(j + 1))) break;
-            const int s = j % C::NSV, buf = j & 1;
-            bool w = true;
-            if (leader) w = tc::mbar_wait(&p_ready[buf], (j >> 1) & 1, abort_flag, kWaitLimit);
-            if (!(ok = __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0)) break;
-            if constexpr (MX) {
-                w = tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, kWaitLimit);
-                if (!(ok = __all_sync(0xffffffffu, w))) break;
-                // row `lane` of the source: TMEM lane `lane`, column c <- channel 32 c + lane;
-                // blocks past the sequence end and blocks of pages the block table gets wrong
-                // are zeroed (their bytes are never multiplied)
-                const int tile = tile0 + j;
-                const uint8_t* vs = smem + C::SM_VST + s * C::VSTAGE + C::OFF_VS;
-                const uint2 w0 = *reinterpret_cast<const uint2*>(vs + 8 * lane);
-                const uint2 w1 = *reinterpret_cast<const uint2*>(vs + C::VS_PAGE + 8 * lane);
-                uint32_t msk[2];
+                if constexpr (MX) __syncwarp();
+                return true;
+            };
+            // the softmax warps quantize the query into shared memory and TMEM first (MXFP4: the
+            // lanes then read the page flags those warps wrote before)
+            bool ok = wait(q_ready, 0);
+            if (ok) tc::tc_fence_after();
+            const bool any_bad_page = MX && ok && *reinterpret_cast<volatile int*>(smem + C::SM_PFLAG + 64) != 0;
+            ok = ok && issue_qk(0);
+            for (int j = 0; ok && j < n; ++j) {
+                if (j + 1 < n && !(ok = issue_qk(j + 1))) break;
+                const int s = j % C::NSV, buf = j & 1;
+                if (!(ok = wait(&p_ready[buf], (j >> 1) & 1))) break;
+                if (!(ok = wait(&vfull[s], (j / C::NSV) & 1))) break;
+                tc::tc_fence_after();
+                if constexpr (MX) {
+                    // row `lane` of the source: TMEM lane `lane`, column c <- channel 32 c + lane;
+                    // blocks past the sequence end and blocks of pages the block table gets wrong
+                    // are zeroed (their bytes are never multiplied)
+                    const int tile = tile0 + j;
+                    const uint8_t* vs = smem + C::SM_VST + s * C::VSTAGE + C::OFF_VS;
+                    const uint2 w0 = *reinterpret_cast<const uint2*>(vs + 8 * lane);
+                    const uint2 w1 = *reinterpret_cast<const uint2*>(vs + C::VS_PAGE + 8 * lane);
+                    uint32_t msk[2];
 #pragma unroll
-                for (int p = 0; p < 2; ++p) {
-                    int nvb = (N - (tile * kTileTokens + p * kPageSlots) + B - 1) / B;
-                    nvb = nvb < 0 ? 0 : (nvb > C::SPB ? C::SPB : nvb);
-                    if (any_bad_page) {
-                        const uint32_t f = j < 64 ? (smem + C::SM_PFLAG)[j] : 0u;
-                        if (j >= 64) {
+                    for (int p = 0; p < 2; ++p) {
+                        int nvb = (N - (tile * kTileTokens + p * kPageSlots) + B - 1) / B;
+                        nvb = nvb < 0 ? 0 : (nvb > C::SPB ? C::SPB : nvb);
+                        if (any_bad_page) {
                             const int pi = tile * 2 + p;
-                            const int v = pi * kPageSlots < N ? __ldg(a.block_table + (int64_t)b * a.max_pages + pi) : 0;
-                            if (v < 0 || v >= a.num_pages) nvb = 0;
-                        } else if (!(f & (1u << p))) {
-                            nvb = 0;
+                            if (j < 64) {
+                                if (!((smem + C::SM_PFLAG)[j] & (1u << p))) nvb = 0;
+                            } else if (pi * kPageSlots < N) {
+                                const int v = __ldg(a.block_table + (int64_t)b * a.max_pages + pi);
+                                if (v < 0 || v >= a.num_pages) nvb = 0;
+                            }
                         }
+                        const uint32_t m16 = nvb >= 2 ? 0xffffu : ((1u << (8 * nvb)) - 1u);
+                        msk[p] = m16 | (m16 << 16);
                     }
-                    const uint32_t m16 = nvb >= 2 ? 0xffffu : ((1u << (8 * nvb)) - 1u);
-                    msk[p] = m16 | (m16 << 16);
+                    const uint32_t x0 = w0.x & msk[0], x1 = w0.y & msk[0], y0 = w1.x & msk[1], y1 = w1.y & msk[1];
+                    *reinterpret_cast<uint4*>(smem + C::SM_VSF + buf * 512 + 16 * lane) =
+                        make_uint4(__byte_perm(x0, y0, 0x5410), __byte_perm(x0, y0, 0x7632),
+                                   __byte_perm(x1, y1, 0x5410), __byte_perm(x1, y1, 0x7632));
+                    tc::fence_proxy_async_smem();
+                    __syncwarp();
                 }
-                const uint32_t x0 = w0.x & msk[0], x1 = w0.y & msk[0], y0 = w1.x & msk[1], y1 = w1.y & msk[1];
-                *reinterpret_cast<uint4*>(smem + C::SM_VSF + buf * 512 + 16 * lane) =
-                    make_uint4(__byte_perm(x0, y0, 0x5410), __byte_perm(x0, y0, 0x7632), __byte_perm(x1, y1, 0x5410),
-                               __byte_perm(x1, y1, 0x7632));
-                tc::fence_proxy_async_smem();
-                __syncwarp();
-            }
-            if (leader) {
-                if constexpr (!MX) ok = tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, kWaitLimit);
-                if (ok) {
-                    tc::tc_fence_after();
+                if (leader) {
                     const uint32_t vt = vst_addr + s * C::VSTAGE + C::OFF_V;
                     // scale factors of P (written by the softmax warps) and of V: NVFP4 a page's scale
                     // block is already in the 32 x 16-byte copy layout, MXFP4 the interleaved rows
@@ -539,10 +540,10 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                     tc::mma_commit(&o_full[buf]);
                     tc::mma_commit(&vempty[s]);
                 }
+                if constexpr (MX) __syncwarp();
             }
-            if (!(ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0)) break;
+            if (!ok && leader) *abort_flag = 1;
         }
-        if (!ok && leader) *abort_flag = 1;
     } else {
         // ------------------------------------------------------------ softmax warps
         const int grp = warp >> 2;                 // head group
