@@ -35,13 +35,21 @@ struct Fmt<BDFP4_MXFP4> {
 };
 
 // ------------------------------------------------------------------ E2M1
-// Value of a 4-bit E2M1 code (sign bit 3): 0, 0.5, 1, 1.5, 2, 3, 4, 6.
+// Value of a 4-bit E2M1 code (sign bit 3): 0, 0.5, 1, 1.5, 2, 3, 4, 6.  The
+// normal codes m = 2..7 (1, 1.5, 2, 3, 4, 6) step by 2^22 in their fp32 bits,
+// 0x3F000000 + m 2^22; code 1 is 0.5 = 0x3F000000.
 __device__ __forceinline__ float e2m1_value(uint32_t code) {
-    uint32_t m = code & 7u;
-    uint32_t e = m >> 1, f = m & 1u;
-    // e == 0: 0.5 * f; else (1 + 0.5 f) * 2^(e-1)
-    float mag = (e == 0) ? 0.5f * (float)f : __uint_as_float(((e + 126u) << 23) | (f << 22));
-    return (code & 8u) ? -mag : mag;
+    const uint32_t m = code & 7u;
+    const uint32_t mag = m >= 2u ? 0x3F000000u + (m << 22) : (m ? 0x3F000000u : 0u);
+    return __uint_as_float(mag | ((code & 8u) << 28));
+}
+
+// The same value as an fp64: the high word of codes 2..7 steps by 2^19 from
+// 0x3FE00000 (0.5, code 1).
+__device__ __forceinline__ double e2m1_value_f64(uint32_t code) {
+    const uint32_t m = code & 7u;
+    const uint32_t hi = m >= 2u ? 0x3FE00000u + (m << 19) : (m ? 0x3FE00000u : 0u);
+    return __hiloint2double((int)(hi | ((code & 8u) << 28)), 0);
 }
 
 // Round two fp32 values to E2M1 (nearest, ties to even, saturating at +-6,

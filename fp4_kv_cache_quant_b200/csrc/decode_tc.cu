@@ -257,7 +257,6 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
     uint64_t* q_full = q_ready + 1;           // query image landed -> softmax
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SM_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::SM_MISC + 4);   // any role gave up
-    volatile int* sm_abort = reinterpret_cast<volatile int*>(smem + C::SM_MISC + 8);     // [NSG] group decisions
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int split = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
@@ -302,8 +301,6 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
         tc::mbar_init(q_ready, C::NSW);
         tc::mbar_init(q_full, 1);
         *abort_flag = 0;
-        sm_abort[0] = 0;
-        sm_abort[1] = 0;
         tc::fence_mbar_init();
     }
     if (warp == C::MMA_WARP) {
@@ -553,6 +550,7 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
         const uint32_t tq = tbase + ((uint32_t)(32 * qd) << 16);
         const float alpha = (FMT == BDFP4_NVFP4 && !(a.flags & BDFP4_FLAG_NO_UNDERFLOW)) ? kAlphaNV : 1.0f;
         bool bad = false;
+        bool grp_abort = false;   // the group's four warps gave up (alike in all of them)
 
         // Pages the block table gets wrong (the producer reports them and copies nothing) are
         // skipped like tokens past the end: their logits are masked and their V scales zeroed.
@@ -682,10 +680,12 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                         rw[(gb + g) * 4 + qd] = fmaxf(hm_lo[g], hm_hi[g]);
                     }
                 }
-                // one decision for the group's four warps: its flag is written only before this barrier
-                if (bad || *abort_flag) sm_abort[grp] = 1;
-                tc::named_bar_sync(bar_id, 128);
-                if (sm_abort[grp]) break;
+                // one decision for the group's four warps, taken by the barrier itself (a role
+                // that gave up leaves a wait here unfinished, and the wait sees its abort flag)
+                if (tc::named_bar_or(bar_id, 128, bad)) {
+                    grp_abort = true;
+                    break;
+                }
                 float y[HG], am[HG], corr[HG];
                 uint32_t mxc[HG];   // MXFP4 block scale codes
                 bool rose = false;   // a running maximum of the group rose (alike in its four warps)
@@ -802,18 +802,17 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
         uint32_t o_fin[HG];
 #pragma unroll
         for (int g = 0; g < HG; ++g) o_fin[g] = 0u;
-        if (!sm_abort[grp]) {
+        if (!grp_abort) {
             if (!tc::mbar_wait(&o_full[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag, kWaitLimit)) bad = true;
             tc::tc_fence_after();
             tc::tmem_ld<HG>(tq + C::T_O + gb, o_fin);
             tc::tmem_wait_ld();
         }
-        if (bad || *abort_flag) sm_abort[grp] = 1;
 
         // ------------------------------------------------------------ epilogue (thread = channel)
-        tc::named_bar_sync(bar_id, 128);
-        if (sm_abort[grp]) *abort_flag = 1;
-        if (!sm_abort[grp]) {
+        grp_abort = tc::named_bar_or(bar_id, 128, grp_abort || bad || *abort_flag);
+        if (grp_abort) *abort_flag = 1;
+        if (!grp_abort) {
             float* rl = red;   // [G][8] partial sums (the tile maxima are no longer read)
 #pragma unroll
             for (int g = 0; g < HG; ++g) {

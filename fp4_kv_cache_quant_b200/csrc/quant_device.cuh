@@ -73,21 +73,28 @@ __device__ __forceinline__ void transform_block(float* x, const float* smooth_ro
 
 // E2M1 codes of x / sigma (sigma = 0 -> zeros), packed two per byte (even
 // element low), and the block's squared error summed left to right in fp64.
-// With W, element i's squared error is weighted: w[i] * (d_i * d_i).
-template <int B, bool W = false>
+// With W, element i's squared error is weighted: w[i] * (d_i * d_i).  POW2:
+// sigma is a power of two and inv = 1 / sigma (exact), so x / sigma rounded to
+// fp32 is x * inv rounded (both are the correctly rounded value of the same
+// real quotient).
+template <int B, bool W = false, bool POW2 = false>
 __device__ __forceinline__ double quantize_block(const float* x, float sigma, uint32_t* packed /* B/8 words */,
-                                                 const float* w = nullptr) {
+                                                 const float* w = nullptr, float inv = 0.0f) {
     double err = 0.0;
 #pragma unroll
     for (int k = 0; k < B / 8; ++k) packed[k] = 0u;
+    const double sd = (double)sigma;
 #pragma unroll
     for (int i = 0; i < B; i += 2) {
         uint32_t pair = 0u;
-        if (sigma != 0.0f) pair = e2m1x2_encode(__fdiv_rn(x[i], sigma), __fdiv_rn(x[i + 1], sigma));
+        if (sigma != 0.0f) {
+            if constexpr (POW2) pair = e2m1x2_encode(__fmul_rn(x[i], inv), __fmul_rn(x[i + 1], inv));
+            else pair = e2m1x2_encode(__fdiv_rn(x[i], sigma), __fdiv_rn(x[i + 1], sigma));
+        }
         packed[i / 8] |= pair << (4 * (i % 8));
         // e sigma is exact in fp64, so x - e sigma rounds once either way
-        const double d0 = __dsub_rn((double)x[i], __dmul_rn((double)e2m1_value(pair & 15u), (double)sigma));
-        const double d1 = __dsub_rn((double)x[i + 1], __dmul_rn((double)e2m1_value(pair >> 4), (double)sigma));
+        const double d0 = __dsub_rn((double)x[i], __dmul_rn(e2m1_value_f64(pair & 15u), sd));
+        const double d1 = __dsub_rn((double)x[i + 1], __dmul_rn(e2m1_value_f64(pair >> 4), sd));
         if constexpr (W) {
             err = __dadd_rn(err, __dmul_rn((double)w[i], __dmul_rn(d0, d0)));
             err = __dadd_rn(err, __dmul_rn((double)w[i + 1], __dmul_rn(d1, d1)));
@@ -107,10 +114,56 @@ __device__ __forceinline__ float block_amax(const float* x) {
     return a;
 }
 
+// Exact scoring of window codes hi .. lo (those whose bit k = hi - c is set in
+// `take`, taken from the largest code down): least (W: weighted) fp64 squared
+// error, ties to the larger code.  Returns the code (-1 if none), `packed` its
+// E2M1 codes.  The loop walks the thread's own set bits, so a warp whose
+// threads take different codes runs as many iterations as its busiest thread.
+template <int FMT, bool W>
+__device__ __forceinline__ int search_exact(const float* x, float g, const float* w, int hi, uint32_t take,
+                                            uint32_t* packed) {
+    constexpr int B = Fmt<FMT>::beta;
+    int best = -1;
+    double best_err = 0.0;
+#pragma unroll 1
+    while (take) {
+        const int c = hi - (__ffs(take) - 1);
+        take &= take - 1u;
+        uint32_t cand[B / 8];
+        const float sg = block_sigma<FMT>((uint32_t)c, g);
+        double err;
+        if constexpr (FMT == BDFP4_MXFP4) {
+            // sigma = 2^(c - 127): dividing by it is multiplying by 2^(127 - c), exactly
+            const float inv = __uint_as_float(c == 254 ? 0x00400000u : (uint32_t)(254 - c) << 23);
+            err = quantize_block<B, W, true>(x, sg, cand, w, inv);
+        } else {
+            err = quantize_block<B, W>(x, sg, cand, w);
+        }
+        if (best < 0 || err < best_err) {
+            best = c;
+            best_err = err;
+#pragma unroll
+            for (int k = 0; k < B / 8; ++k) packed[k] = cand[k];
+        }
+    }
+    return best;
+}
+
 // Scale search of one key block: the window NVFP4 c0+7 .. c0-2 (E4M3 codes,
 // within [0, 126]) or MXFP4 c0+1, c0 (E8M0, within [0, 254]) around the plain
-// code c0; least (W: weighted) squared error, ties to the larger code.  An
-// all-zero block keeps c0.  Returns the code; `packed` gets its E2M1 codes.
+// code c0; least (W: weighted) squared error in fp64 summed left to right, ties
+// to the larger code.  An all-zero block keeps c0.  Returns the code; `packed`
+// gets its E2M1 codes.
+//
+// NVFP4 scores every candidate cheaply first: x times the rounded 1 / sigma
+// for the codes, the squared error in fp32.  Against the exact score (fp32 RN
+// division, fp64 sums) the cheap one moves an element's code only within a few
+// ulps of a rounding midpoint, where the two codes' errors agree to 1e-5
+// relative, and rounds the sum to about 1e-6 relative, so the exact winner
+// always scores within 2^-10 (relative) of the cheapest candidate.  Only those
+// candidates are scored exactly, in window order -- the same winner as scoring
+// all of them exactly.  A candidate whose 1 / sigma is not finite is always
+// scored exactly.
 template <int FMT, bool W>
 __device__ __forceinline__ uint32_t search_scale(const float* x, float g, const float* w, uint32_t* packed) {
     constexpr int B = Fmt<FMT>::beta;
@@ -125,19 +178,46 @@ __device__ __forceinline__ uint32_t search_scale(const float* x, float g, const 
     int lo = c0 - (FMT == BDFP4_NVFP4 ? 2 : 0);
     hi = hi > top ? top : hi;
     lo = lo < 0 ? 0 : lo;
-    int best = hi;
-    double best_err = 0.0;
-    for (int c = hi; c >= lo; --c) {
-        uint32_t cand[B / 8];
-        const double err = quantize_block<B, W>(x, block_sigma<FMT>((uint32_t)c, g), cand, w);
-        if (c == hi || err < best_err) {
-            best = c;
-            best_err = err;
+    const uint32_t all = (1u << (hi - lo + 1)) - 1u;
+    if constexpr (FMT == BDFP4_MXFP4) {
+        return (uint32_t)search_exact<FMT, W>(x, g, w, hi, all, packed);
+    } else {
+        constexpr int NW = 10;   // window length
+        float score[NW];
+        uint32_t force = 0u;
+        float best = INFINITY;
 #pragma unroll
-            for (int k = 0; k < B / 8; ++k) packed[k] = cand[k];
+        for (int k = 0; k < NW; ++k) {
+            const int c = hi - k;
+            score[k] = INFINITY;
+            if (c < lo) continue;
+            const float sg = block_sigma<FMT>((uint32_t)c, g);
+            const float r = __frcp_rn(sg);
+            if (!(sg > 0.0f) || !(r < INFINITY)) {
+                force |= 1u << k;
+                continue;
+            }
+            float e = 0.0f;
+#pragma unroll
+            for (int i = 0; i < B; i += 2) {
+                const uint32_t pair = e2m1x2_encode(x[i] * r, x[i + 1] * r);
+                const float d0 = fmaf(-e2m1_value(pair & 15u), sg, x[i]);
+                const float d1 = fmaf(-e2m1_value(pair >> 4), sg, x[i + 1]);
+                e = fmaf(W ? w[i] * d0 : d0, d0, e);
+                e = fmaf(W ? w[i + 1] * d1 : d1, d1, e);
+            }
+            score[k] = e;
+            best = fminf(best, e);
         }
+        const float lim = best + best * (1.0f / 1024.0f);
+        uint32_t take = force;
+#pragma unroll
+        for (int k = 0; k < NW; ++k)
+            if (score[k] <= lim) take |= 1u << k;
+        take &= all;
+        // nothing comparable (non-finite scores): score the whole window exactly
+        return (uint32_t)search_exact<FMT, W>(x, g, w, hi, take ? take : all, packed);
     }
-    return (uint32_t)best;
 }
 
 // ---------------------------------------------------------------- query
