@@ -36,6 +36,8 @@ ENTRY_POINTS = ("bdfp4_calibrate", "bdfp4_key_weights", "bdfp4_quantize_kv", "bd
                 "bdfp4_status_string", "bdfp4_last_error")
 #: names of every entry point declared in include/bdfp4_bf16.h
 BF16_ENTRY_POINTS = ("bdfp4_bf16_append", "bdfp4_bf16_decode")
+#: names of every entry point declared in include/bdfp4_debug.h (test hooks)
+DEBUG_ENTRY_POINTS = ("bdfp4_debug_decode_wait_test",)
 
 #: size of the library's built-in scratch used by bdfp4_decode_noalloc
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -96,6 +98,9 @@ def load() -> ctypes.CDLL:
     L.bdfp4_status_string.restype = ctypes.c_char_p
     L.bdfp4_last_error.argtypes = []
     L.bdfp4_last_error.restype = ctypes.c_char_p
+    L.bdfp4_debug_decode_wait_test.argtypes = [p, p, p, p, p, p, p, i, i, i, i, i, i, i64, i, i, kvp, f, i, p, sz, p,
+                                               p, ctypes.c_longlong, i, p]
+    L.bdfp4_debug_decode_wait_test.restype = i
     L.bdfp4_bf16_append.argtypes = [p, p, p, i, i, i, p, p, i64, p, p]
     L.bdfp4_bf16_append.restype = i
     L.bdfp4_bf16_decode.argtypes = [p, p, p, p, p, i, i, i, i, i, i64, f, i, p, sz, p, p, p]
@@ -325,6 +330,25 @@ def bdfp4_decode_step(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
                                   int(chunk_tiles), _ptr(workspace), ws_bytes, _ptr(out), _ptr(dev_status),
                                   _stream(stream))
     _check(rc, "bdfp4_decode_step")
+    return out
+
+
+def bdfp4_debug_decode_wait_test(q: torch.Tensor, cache: FP4Cache, block_table: torch.Tensor, seq_lens: torch.Tensor,
+                                 kv: KVParams, sm_scale: float, chunk_tiles: int, workspace: torch.Tensor | None,
+                                 out: torch.Tensor, wait_limit_cycles: int, stall: bool, flags: int = 0,
+                                 dev_status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Test hook (include/bdfp4_debug.h): bdfp4_decode with a short in-kernel wait
+    bound and, with stall, every CTA's first K tile withheld so its waits run out."""
+    B, H_q, d_k = q.shape
+    c = kv._c()
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = load().bdfp4_debug_decode_wait_test(_ptr(q), _ptr(cache.k_pages), _ptr(cache.k_scales), _ptr(cache.v_pages),
+                                             _ptr(cache.v_scales), _ptr(block_table), _ptr(seq_lens), B, H_q,
+                                             cache.H_kv, d_k, cache.d_v, block_table.shape[1], cache.num_pages,
+                                             cache.fmt, flags, ctypes.byref(c), float(sm_scale), int(chunk_tiles),
+                                             _ptr(workspace), ws_bytes, _ptr(out), _ptr(dev_status),
+                                             int(wait_limit_cycles), 1 if stall else 0, _stream(stream))
+    _check(rc, "bdfp4_debug_decode_wait_test")
     return out
 
 

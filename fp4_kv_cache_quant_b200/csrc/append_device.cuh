@@ -124,6 +124,127 @@ __device__ __forceinline__ void append_k_cta(int blk, const __nv_bfloat16* __res
     ks[k_scale_offset<B>(DK, slot, j)] = (uint8_t)code;
 }
 
+// Low-latency K append for few rows (a decode step's new tokens): every scale
+// block of a row gets NC lanes, one per candidate code of its search window, so
+// the window is scored in parallel -- each lane quantizes the block under its
+// code exactly (fp32 RN division, fp64 error left to right) -- and a shuffle
+// argmin over the block's lanes keeps the least error, the larger code on a
+// tie, as the sequential search.  R rows share a 256-thread CTA.
+template <int FMT, int DK>
+struct KWideGeom {
+    using RG = RowGeom<FMT, DK>;
+    static constexpr int B = RG::beta;
+    static constexpr int NB = DK / B;                                  // scale blocks per row
+    static constexpr int NC = FMT == BDFP4_NVFP4 ? 16 : 2;             // candidate lanes per block (10 or 2 used)
+    static constexpr int R = 256 / (NB * NC) >= 1 ? 256 / (NB * NC) : 1;
+    static constexpr int PAIRS = R * NB * NC;                          // (block, candidate) lanes
+    static constexpr int T1 = (R * RG::rt + 31) / 32 * 32;             // transform threads (whole warps)
+    static_assert(T1 <= 256 && 32 % NC == 0, "work split");
+};
+
+template <int FMT, int DK, class SlotOf>
+__device__ __forceinline__ void append_k_cta_wide(int blk, const __nv_bfloat16* __restrict__ k, int64_t rows,
+                                                  int H_kv, const SlotOf& slot_of, const float* __restrict__ smooth,
+                                                  const float* __restrict__ k_gscale,
+                                                  const float* __restrict__ k_weight, uint8_t* k_pages,
+                                                  uint8_t* k_scales, int flags) {
+    using KG = KWideGeom<FMT, DK>;
+    using RG = typename KG::RG;
+    constexpr int B = KG::B, NB = KG::NB, NC = KG::NC, R = KG::R;
+    __shared__ float xs[R][DK];
+    __shared__ long long slots[R];
+    __shared__ float gs[R];
+    const int tid = threadIdx.x;
+    const int64_t row0 = (int64_t)blk * R;
+    // phase 1: the rows' transform into shared memory (thread per block)
+    if (tid < KG::T1) {
+        const int r = tid / RG::rt, j = tid % RG::rt;
+        const int64_t row = row0 + r;
+        const bool in_range = r < R && row < rows;
+        const int t = (int)(in_range ? row / H_kv : 0);
+        const int h = (int)(in_range ? row % H_kv : 0);
+        const int64_t sm = in_range ? slot_of(t, j == 0) : -1;
+        float x[B];
+        if (in_range && j < RG::tpr) {
+            load_bf16_block<B>(k + ((int64_t)t * H_kv + h) * DK, j * B, x);
+        } else {
+#pragma unroll
+            for (int i = 0; i < B; ++i) x[i] = 0.0f;
+        }
+        if (sm < 0) {
+#pragma unroll
+            for (int i = 0; i < B; ++i) x[i] = 0.0f;
+        }
+        transform_block<FMT, DK, true>(x, smooth + (int64_t)h * DK, j, !(flags & BDFP4_FLAG_NO_HADAMARD));
+        if (sm >= 0 && j < RG::tpr) {
+#pragma unroll
+            for (int i = 0; i < B; ++i) xs[r][j * B + i] = x[i];
+        }
+        if (r < R && j == 0) {
+            slots[r] = sm;
+            gs[r] = FMT == BDFP4_NVFP4 ? __ldg(k_gscale + h) : 1.0f;
+        }
+    }
+    __syncthreads();
+    // phase 2: lane (row, block, candidate); whole warps take part in the shuffles
+    for (int p0 = 0; p0 < KG::PAIRS; p0 += 256) {
+        const int p = p0 + tid;
+        const bool live = p < KG::PAIRS;
+        const int r = live ? p / (NB * NC) : 0, bk = live ? (p / NC) % NB : 0, ci = p % NC;
+        const int64_t sm = live ? slots[r] : -1;
+        const float g = gs[r];
+        float x[B];
+#pragma unroll
+        for (int i = 0; i < B; ++i) x[i] = xs[r][bk * B + i];
+        const int h = (int)((row0 + r) % H_kv);
+        const float amax = block_amax<B>(x);
+        const int c0 = (int)plain_scale_code<FMT>(amax, g);
+        int hi = c0, lo = c0;   // all-zero blocks and the plain rule keep c0
+        if (amax != 0.0f && !(flags & BDFP4_FLAG_NO_SCALE_SEARCH)) {
+            const int top = FMT == BDFP4_NVFP4 ? 126 : 254;
+            hi = min(c0 + (FMT == BDFP4_NVFP4 ? 7 : 1), top);
+            lo = max(c0 - (FMT == BDFP4_NVFP4 ? 2 : 0), 0);
+        }
+        const int c = hi - ci;
+        uint32_t pk[B / 8];
+        double err = INFINITY;
+        if (sm >= 0 && c >= lo) {
+            if (k_weight) {
+                float w[B];
+#pragma unroll
+                for (int i = 0; i < B; ++i) w[i] = __ldg(k_weight + (int64_t)h * DK + bk * B + i);
+                err = quantize_block<B, true>(x, block_sigma<FMT>((uint32_t)c, g), pk, w);
+            } else {
+                err = quantize_block<B>(x, block_sigma<FMT>((uint32_t)c, g), pk);
+            }
+        }
+        // argmin over the block's NC lanes: least error, then smallest ci (the larger code)
+        double be = err;
+        int bci = ci;
+#pragma unroll
+        for (int off = NC / 2; off > 0; off >>= 1) {
+            const double oe = __shfl_xor_sync(0xffffffffu, be, off);
+            const int oc = __shfl_xor_sync(0xffffffffu, bci, off);
+            if (oe < be || (oe == be && oc < bci)) {
+                be = oe;
+                bci = oc;
+            }
+        }
+        if (sm >= 0 && ci == bci) {
+            const int64_t page = sm / kPageSlots;
+            const int slot = (int)(sm % kPageSlots);
+            uint8_t* dst = k_pages + (page * H_kv + h) * (int64_t)(kPageSlots * DK / 2) + k_nib_offset(DK, slot, bk * B);
+            if constexpr (B == 16) {
+                *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
+            } else {
+                *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+            k_scales[(page * H_kv + h) * (int64_t)k_scale_page_bytes(DK, B) + k_scale_offset<B>(DK, slot, bk)] =
+                (uint8_t)c;
+        }
+    }
+}
+
 // ---------------------------------------------------------------- values
 // One thread per (row, channel): TPR threads of a row per CTA, RPC rows per
 // CTA, CPR CTAs per row.
@@ -189,6 +310,10 @@ __device__ __forceinline__ void append_v_open_cta(int blk, const __nv_bfloat16* 
 template <int FMT, int DK>
 __host__ __device__ constexpr int64_t k_append_ctas(int64_t nrows) {
     return (nrows + KGeom<FMT, DK>::R - 1) / KGeom<FMT, DK>::R;
+}
+template <int FMT, int DK>
+__host__ __device__ constexpr int64_t k_append_ctas_wide(int64_t nrows) {
+    return (nrows + KWideGeom<FMT, DK>::R - 1) / KWideGeom<FMT, DK>::R;
 }
 template <int DV>
 __host__ __device__ constexpr int64_t v_append_ctas(int64_t nrows) {

@@ -14,6 +14,7 @@
 #include <cstdio>
 #include <mutex>
 
+#include "../../include/bdfp4_debug.h"
 #include "bdfp4_device.cuh"
 #include "host_common.h"
 #include "quant_device.cuh"
@@ -416,7 +417,8 @@ static int run_decode(const void* q, const void* k_pages, const void* k_scales, 
                       const void* v_scales, const int32_t* block_table, const int32_t* seq_lens, int B, int T_q,
                       int H_q, int H_kv, int d_k, int d_v, int max_pages_per_seq, int64_t num_pages, bdfp4_fmt fmt,
                       int flags, const bdfp4_kv_params* kv, float sm_scale, int chunk_tiles, void* workspace,
-                      size_t workspace_bytes, void* out, int32_t* dev_status, void* stream, StepArgs* step) {
+                      size_t workspace_bytes, void* out, int32_t* dev_status, void* stream, StepArgs* step,
+                      long long wait_limit = kWaitLimitDefault, int test_stall = 0) {
     if (B < 0 || T_q <= 0 || H_q <= 0 || H_kv <= 0 || max_pages_per_seq <= 0 || num_pages < 0) return BDFP4_ERR_ARG;
     if (fmt != BDFP4_NVFP4 && fmt != BDFP4_MXFP4) return BDFP4_ERR_ARG;
     if (H_q % H_kv) return BDFP4_ERR_SHAPE;
@@ -478,6 +480,8 @@ static int run_decode(const void* q, const void* k_pages, const void* k_scales, 
     a.chunk_tiles = chunk_tiles;
     a.sm_scale = sm_scale;
     a.append_wait = step != nullptr;
+    a.wait_limit = wait_limit;
+    a.test_stall = test_stall;
     if (step) {
         step->k_pages = (uint8_t*)k_pages;
         step->k_scales = (uint8_t*)k_scales;
@@ -528,6 +532,23 @@ extern "C" int bdfp4_decode_multi(const void* q, const void* k_pages, const void
     return run_decode(q, k_pages, k_scales, v_pages, v_scales, block_table, seq_lens, B, T_q, H_q, H_kv, d_k, d_v,
                       max_pages_per_seq, num_pages, fmt, flags, kv, sm_scale, chunk_tiles, workspace,
                       workspace_bytes, out, dev_status, stream, nullptr);
+}
+
+// ---------------------------------------------------------------- unwind test (bdfp4_debug.h)
+extern "C" int bdfp4_debug_decode_wait_test(const void* q, const void* k_pages, const void* k_scales,
+                                            const void* v_pages, const void* v_scales, const int32_t* block_table,
+                                            const int32_t* seq_lens, int B, int H_q, int H_kv, int d_k, int d_v,
+                                            int max_pages_per_seq, int64_t num_pages, bdfp4_fmt fmt, int flags,
+                                            const bdfp4_kv_params* kv, float sm_scale, int chunk_tiles,
+                                            void* workspace, size_t workspace_bytes, void* out,
+                                            int32_t* dev_status, long long wait_limit_cycles, int stall,
+                                            void* stream) {
+    // only the d = 128 tensor-core decode takes the switch
+    if (d_k != 128 || d_v != 128 || H_kv <= 0 || H_q % H_kv || H_q / H_kv > 16) return BDFP4_ERR_UNSUPPORTED;
+    if (wait_limit_cycles <= 0) return BDFP4_ERR_ARG;
+    return run_decode(q, k_pages, k_scales, v_pages, v_scales, block_table, seq_lens, B, 1, H_q, H_kv, d_k, d_v,
+                      max_pages_per_seq, num_pages, fmt, flags, kv, sm_scale, chunk_tiles, workspace,
+                      workspace_bytes, out, dev_status, stream, nullptr, wait_limit_cycles, stall ? 1 : 0);
 }
 
 // ---------------------------------------------------------------- no-allocation variant

@@ -28,6 +28,10 @@ struct DecodeArgs {
     int B, H_q, H_kv, max_pages, flags, chunk_tiles, max_splits;
     int append_wait;   // 1: a decode-step prologue grid writes each sequence's last page (tensor-core path)
     int T_q;           // query tokens per sequence (1: single-token decode); q, out are [B][T_q][H_q][d]
+    // d = 128 tensor-core decode: the bound of every in-kernel wait (clock cycles), and the
+    // unwind test's switch (1: every CTA withholds its first K tile, see bdfp4_debug.h)
+    long long wait_limit;
+    int test_stall;
     int64_t num_pages;
     float sm_scale;
 };
@@ -46,6 +50,7 @@ struct StepArgs {
 };
 
 constexpr int kThreads = 128;
+constexpr long long kWaitLimitDefault = 1LL << 32;   // clock cycles (about 2 s)
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Workspace bytes reserved per query head for the query images of the

@@ -171,9 +171,9 @@ __global__ void __launch_bounds__(256) prep_mla_kernel(const DecodeArgs a, const
     if (with_step) {
         const int64_t rows = (int64_t)a.B * a.H_kv;
         const NewestSlot slot{a.block_table, a.seq_lens, a.max_pages, a.num_pages, a.dev_status};
-        const int nk = (int)k_append_ctas<FMT, 576>(rows), nv = (int)v_append_ctas<512>(rows);
+        const int nk = (int)k_append_ctas_wide<FMT, 576>(rows), nv = (int)v_append_ctas<512>(rows);
         if (blk < nk) {
-            append_k_cta<FMT, 576>(blk, s.k_new, rows, a.H_kv, slot, a.smooth, a.k_gscale, a.k_weight, s.k_pages, s.k_scales,
+            append_k_cta_wide<FMT, 576>(blk, s.k_new, rows, a.H_kv, slot, a.smooth, a.k_gscale, a.k_weight, s.k_pages, s.k_scales,
                                    a.flags);
             return;
         }
@@ -837,7 +837,7 @@ static int launch_mla(const DecodeArgs& a, cudaStream_t st, const StepArgs* step
     StepArgs s{};
     if (step) {
         const int64_t rows = (int64_t)a.B * a.H_kv;
-        ctas += k_append_ctas<FMT, 576>(rows) + v_append_ctas<512>(rows);
+        ctas += k_append_ctas_wide<FMT, 576>(rows) + v_append_ctas<512>(rows);
         s = *step;
     }
     prep_mla_kernel<FMT, GH><<<(unsigned)ctas, 256, 0, st>>>(a, s, step ? 1 : 0);

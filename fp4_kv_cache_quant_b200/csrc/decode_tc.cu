@@ -132,7 +132,6 @@ struct TcCfg {
     static_assert(QPACK % 16 == 0, "query image copied in 16-byte units");
 };
 
-constexpr long long kWaitLimit = 1LL << 32;   // clock cycles (about 2 s)
 
 // Query image of one (sequence, KV head): smoothing + Hadamard transform and
 // dual-residual FP4 of its G query heads, laid out as the decode CTA keeps them
@@ -214,11 +213,11 @@ __global__ void __launch_bounds__(256) prep_step_kernel(const DecodeArgs a, cons
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int64_t rows = (int64_t)a.B * a.H_kv;
     const NewestSlot slot{a.block_table, a.seq_lens, a.max_pages, a.num_pages, a.dev_status};
-    const int nk = (int)k_append_ctas<FMT, 128>(rows), nv = (int)v_append_ctas<128>(rows);
+    const int nk = (int)k_append_ctas_wide<FMT, 128>(rows), nv = (int)v_append_ctas<128>(rows);
     const int blk = blockIdx.x;
     if (blk < nk) {
-        append_k_cta<FMT, 128>(blk, s.k_new, rows, a.H_kv, slot, a.smooth, a.k_gscale, a.k_weight, s.k_pages, s.k_scales,
-                               a.flags);
+        append_k_cta_wide<FMT, 128>(blk, s.k_new, rows, a.H_kv, slot, a.smooth, a.k_gscale, a.k_weight, s.k_pages,
+                                    s.k_scales, a.flags);
     } else if (blk < nk + nv) {
         append_v_open_cta<FMT, 128>(blk - nk, s.v_new, s.v_open, slot, a.B, a.H_kv, a.v_gscale, s.v_pages,
                                     s.v_scales);
@@ -323,6 +322,7 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
         // are consumed).
         bool ok = true;
         int pv0 = -1, pv1 = -1;   // pages of the previous tile (the V half of this step)
+        int k_last = -1, v_last = -1;   // the last tiles whose K / V halves were announced
         for (int j0 = 0; ok && j0 <= n; j0 += 32) {
             int pg_l[2] = {-1, -1};
             if (j0 + lane < n) {
@@ -350,12 +350,13 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                 // the two K pages and every lane copies, with cp.async, the 8 scale bytes of
                 // slots lane and 32 + lane of each page and scale group into row lane of the
                 // group's tcgen05.cp source, then arrives on the stage barrier once they land
-                if (do_k) {
+                // the unwind test withholds tile 0's K half: the MMA warp's wait for it runs out
+                if (do_k && !(a.test_stall && k == 0)) {
                     // the step prologue writes the new token into the sequence's last page:
                     // that tile's copies wait until the prologue grid has finished
                     if (a.append_wait && tile0 + k == ntiles - 1) asm volatile("griddepcontrol.wait;" ::: "memory");
                     if (lane == 0) {
-                        if (k >= C::NSK && !tc::mbar_wait(&kempty[ks], ((k / C::NSK) - 1) & 1, abort_flag, kWaitLimit))
+                        if (k >= C::NSK && !tc::mbar_wait(&kempty[ks], ((k / C::NSK) - 1) & 1, abort_flag, a.wait_limit))
                             ok = false;
                         else
                             tc::mbar_arrive_expect_tx(&kfull[ks], (pg0 >= 0 ? C::K_PAGE : 0) + (pg1 >= 0 ? C::K_PAGE : 0));
@@ -379,11 +380,12 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                             tc::cp_async_8(stg + C::OFF_KS + kg * 512 + lane * 16 + p * 8, ksrc + kg * 256);
                     }
                     tc::cp_async_mbar_arrive_noinc(&kfull[ks]);
+                    k_last = k;
                 }
                 // V half of tile v: lanes 0-1 copy the V pages, 2-3 their scales
                 if (do_v) {
                     if (lane == 0) {
-                        if (v >= C::NSV && !tc::mbar_wait(&vempty[vsi], ((v / C::NSV) - 1) & 1, abort_flag, kWaitLimit))
+                        if (v >= C::NSV && !tc::mbar_wait(&vempty[vsi], ((v / C::NSV) - 1) & 1, abort_flag, a.wait_limit))
                             ok = false;
                         else
                             tc::mbar_arrive_expect_tx(&vfull[vsi], (pv0_ >= 0 ? C::V_PAGE + C::VS_PAGE : 0) +
@@ -404,12 +406,32 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                                              C::VS_PAGE, &vfull[vsi]);
                         }
                     }
+                    v_last = v;
                 }
                 pv0 = pg0;
                 pv1 = pg1;
             }
         }
         if (!ok && lane == 0) *abort_flag = 1;
+        // Unwinding: before the CTA can exit, every copy this warp started must have landed.
+        // Each stage's last announced phase completes once its bytes (and the lanes' cp.async
+        // arrivals) are in; announced tiles run consecutively from the first one announced.
+        if (!ok || a.test_stall || *abort_flag) {
+            if (lane == 0) {
+                const int k_first = a.test_stall ? 1 : 0;
+                for (int s = 0; s < C::NSK; ++s) {
+                    if (k_last < s) continue;
+                    const int t = k_last - (k_last - s) % C::NSK;
+                    if (t >= k_first) tc::mbar_wait_drain(&kfull[s], (t / C::NSK) & 1, a.wait_limit);
+                }
+                for (int s = 0; s < C::NSV; ++s) {
+                    if (v_last < s) continue;
+                    const int t = v_last - (v_last - s) % C::NSV;
+                    tc::mbar_wait_drain(&vfull[s], (t / C::NSV) & 1, a.wait_limit);
+                }
+            }
+            __syncwarp();
+        }
     } else if (warp == C::MMA_WARP) {
         // ------------------------------------------------------------ MMA issuer
         // Lane 0 issues every tcgen05 operation.  NVFP4: the other lanes leave (a lane that
@@ -425,7 +447,7 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                 else return v;
             };
             auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
-                return all(tc::mbar_wait(bar, parity, abort_flag, kWaitLimit));
+                return all(tc::mbar_wait(bar, parity, abort_flag, a.wait_limit));
             };
             constexpr uint32_t idesc_qk = tc::idesc_fp4(C::NQ, MX);
             constexpr uint32_t idesc_pv = tc::idesc_fp4(C::NP, MX);
@@ -435,6 +457,9 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
             const uint32_t vst_addr = tc::smem_u32(smem + C::SM_VST);
             const uint32_t psf_addr = tc::smem_u32(psf);
             const uint32_t vsf_addr = tc::smem_u32(smem + C::SM_VSF);
+            // the last commit: its phase completes once every tcgen05 operation issued before it has
+            uint64_t* last_bar = nullptr;
+            uint32_t last_par = 0;
             auto issue_qk = [&](int j) -> bool {
                 const int s = j % C::NSK, buf = j & 1;
                 if (!wait(&kfull[s], (j / C::NSK) & 1)) return false;
@@ -460,6 +485,8 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                     }
                     tc::mma_commit(&s_full[buf]);
                     tc::mma_commit(&kempty[s]);   // the K stage is free once QK has read it
+                    last_bar = &kempty[s];
+                    last_par = (uint32_t)(j / C::NSK) & 1u;
                 }
                 if constexpr (MX) __syncwarp();
                 return true;
@@ -536,10 +563,17 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                     }
                     tc::mma_commit(&o_full[buf]);
                     tc::mma_commit(&vempty[s]);
+                    last_bar = &vempty[s];
+                    last_par = (uint32_t)(j / C::NSV) & 1u;
                 }
                 if constexpr (MX) __syncwarp();
             }
-            if (!ok && leader) *abort_flag = 1;
+            if (!ok && leader) {
+                *abort_flag = 1;
+                // unwinding: the tensor memory is freed below, so the MMAs and copies into it
+                // must have finished
+                if (last_bar) tc::mbar_wait_drain(last_bar, last_par, a.wait_limit);
+            }
         }
     } else {
         // ------------------------------------------------------------ softmax warps
@@ -588,7 +622,7 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
         }
         // the P scale-factor buffers: zero (rows of absent heads must stay zero)
         for (int i = tid; i < 2 * 2 * 512 / 16; i += 32 * C::NSW) reinterpret_cast<uint4*>(psf)[i] = make_uint4(0, 0, 0, 0);
-        if (!tc::mbar_wait(q_full, 0, abort_flag, kWaitLimit)) bad = true;
+        if (!tc::mbar_wait(q_full, 0, abort_flag, a.wait_limit)) bad = true;
         // query scale factors (SFB of QK): lane n <- row n, one 4-column chunk per K step
         if (grp == 0) {
 #pragma unroll
@@ -653,7 +687,7 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                     pok1 = (f & 2u) != 0;
                 }
                 // logits of this thread's token for the group's heads (q1 then q2 columns)
-                if (!tc::mbar_wait(&s_full[buf], (j >> 1) & 1, abort_flag, kWaitLimit)) bad = true;
+                if (!tc::mbar_wait(&s_full[buf], (j >> 1) & 1, abort_flag, a.wait_limit)) bad = true;
                 tc::tc_fence_after();
                 uint32_t sr[2 * HG];
                 tc::tmem_ld<2 * HG>(tq + C::T_S + buf * C::NQ + 2 * gb, sr);
@@ -757,7 +791,7 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                 // O^T rescale of the group's heads once the previous tile's PV has completed,
                 // before this tile's PV is issued (the online-softmax update, in TMEM)
                 if (j > 0 && rose) {
-                    if (!tc::mbar_wait(&o_full[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, kWaitLimit)) bad = true;
+                    if (!tc::mbar_wait(&o_full[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, a.wait_limit)) bad = true;
                     tc::tc_fence_after();
                     uint32_t ov[HG];
                     tc::tmem_ld<HG>(tq + C::T_O + gb, ov);
@@ -778,7 +812,7 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                         const bool tail = (tile + 1) * kTileTokens > N;
                         uint8_t* vs = smem + C::SM_VST + s * C::VSTAGE + C::OFF_VS;
                         if (tail || !pok0 || !pok1) {
-                            if (!tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, kWaitLimit)) bad = true;
+                            if (!tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, a.wait_limit)) bad = true;
     #pragma unroll
                             for (int p = 0; p < 2; ++p) {
                                 const int t0 = tile * kTileTokens + p * kPageSlots;
@@ -803,7 +837,7 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
 #pragma unroll
         for (int g = 0; g < HG; ++g) o_fin[g] = 0u;
         if (!grp_abort) {
-            if (!tc::mbar_wait(&o_full[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag, kWaitLimit)) bad = true;
+            if (!tc::mbar_wait(&o_full[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag, a.wait_limit)) bad = true;
             tc::tc_fence_after();
             tc::tmem_ld<HG>(tq + C::T_O + gb, o_fin);
             tc::tmem_wait_ld();
@@ -871,7 +905,7 @@ static int launch_tc(const DecodeArgs& a, cudaStream_t st, const StepArgs* step)
     if constexpr (!MT) {
         if (step) {
             const int64_t rows = (int64_t)a.B * a.H_kv;
-            const int64_t ctas = k_append_ctas<FMT, 128>(rows) + v_append_ctas<128>(rows) + rows;
+            const int64_t ctas = k_append_ctas_wide<FMT, 128>(rows) + v_append_ctas<128>(rows) + rows;
             prep_step_kernel<FMT, G><<<(unsigned)ctas, 256, 0, st>>>(a, *step);
         } else {
             prep_query_kernel<FMT, G><<<dim3(a.H_kv, a.B), C::QTHREADS, 0, st>>>(a);

@@ -31,18 +31,30 @@ __global__ void __launch_bounds__(256, FMT == BDFP4_NVFP4 ? 3 : 2) quantize_k_ke
                           smooth, k_gscale, k_weight, k_pages, k_scales, flags);
 }
 
-// One thread per (token, head, channel); only the first token of each run
-// within a beta-slot block does work (see bdfp4_quantize_kv in bdfp4.h), for
-// the whole block of its channel.
+// One thread per (token, head, group of VC channels: 8 for NVFP4, 4 for MXFP4);
+// only the first token of each run within a beta-slot block does work (see
+// bdfp4_quantize_kv in bdfp4.h), for the whole block of its VC channels.  A
+// warp covers whole (token, head) rows, so its threads are leaders or not
+// together; a leader loads its beta tokens' channels with one 16- or 8-byte
+// load per token.
+template <int FMT>
+struct VAppend {
+    static constexpr int B = Fmt<FMT>::beta;
+    static constexpr int VC = FMT == BDFP4_NVFP4 ? 8 : 4;   // channels per thread
+    static constexpr int W = VC / 2;                        // 32-bit words of a token's channels
+};
+
 template <int FMT, int DV>
 __global__ void __launch_bounds__(256) quantize_v_kernel(const __nv_bfloat16* __restrict__ v,
                                                          const int64_t* __restrict__ slot_mapping, int T, int H_kv,
                                                          const float* __restrict__ v_gscale, uint8_t* v_pages,
                                                          uint8_t* v_scales, int64_t num_pages) {
-    constexpr int B = Fmt<FMT>::beta;
-    using VG = VGeom<DV>;
-    const int64_t row = (int64_t)(blockIdx.x / VG::CPR) * VG::RPC + threadIdx.x / VG::TPR;
-    const int c = (int)(blockIdx.x % VG::CPR) * VG::TPR + threadIdx.x % VG::TPR;
+    using VA = VAppend<FMT>;
+    constexpr int B = VA::B, VC = VA::VC, W = VA::W;
+    constexpr int GPR = DV / VC;   // channel groups of a row
+    const int64_t gid = (int64_t)blockIdx.x * 256 + threadIdx.x;
+    const int64_t row = gid / GPR;
+    const int c0 = (int)(gid % GPR) * VC;
     if (row >= (int64_t)T * H_kv) return;
     const int t = (int)(row / H_kv), h = (int)(row % H_kv);
     // two rounds of independent loads: this token's and its predecessor's slot
@@ -56,11 +68,6 @@ __global__ void __launch_bounds__(256) quantize_v_kernel(const __nv_bfloat16* __
     int64_t sm_next[B - 1];
 #pragma unroll
     for (int i = 1; i < B; ++i) sm_next[i - 1] = t + i < T ? __ldg(slot_mapping + t + i) : -2;
-    const unsigned short* vb = reinterpret_cast<const unsigned short*>(v);
-    uint32_t raw[B];
-#pragma unroll
-    for (int i = 0; i < B; ++i) raw[i] = t + i < T ? (uint32_t)__ldg(vb + ((int64_t)(t + i) * H_kv + h) * DV + c) : 0u;
-    const float g = FMT == BDFP4_NVFP4 ? __ldg(v_gscale + h) : 1.0f;
     // run: the following tokens on consecutive slots of the same block
     int n = 1;
     bool run = true;
@@ -70,29 +77,51 @@ __global__ void __launch_bounds__(256) quantize_v_kernel(const __nv_bfloat16* __
         n += run ? 1 : 0;
     }
     const int first = slot - slot % B;
+    const int off = slot - first;   // block slot of token t
+    // raw[i]: the channels of block slot i (token t + i - off when it lies in the run)
+    uint32_t raw[B][W];
+#pragma unroll
+    for (int i = 0; i < B; ++i) {
+        const int jt = i - off;
+        const bool in = jt >= 0 && jt < n;
+        const __nv_bfloat16* src = v + ((int64_t)(t + (in ? jt : 0)) * H_kv + h) * DV + c0;
+        if constexpr (W == 4) {
+            uint4 u = in ? __ldg(reinterpret_cast<const uint4*>(src)) : make_uint4(0u, 0u, 0u, 0u);
+            raw[i][0] = u.x; raw[i][1] = u.y; raw[i][2] = u.z; raw[i][3] = u.w;
+        } else {
+            uint2 u = in ? __ldg(reinterpret_cast<const uint2*>(src)) : make_uint2(0u, 0u);
+            raw[i][0] = u.x; raw[i][1] = u.y;
+        }
+    }
+    const float g = FMT == BDFP4_NVFP4 ? __ldg(v_gscale + h) : 1.0f;
     const int64_t page = sm / kPageSlots;
     uint8_t* vp = v_pages + (page * H_kv + h) * (int64_t)(DV * kPageSlots / 2);
     uint8_t* vs = v_scales + (page * H_kv + h) * (int64_t)(DV * kPageSlots / B);
-    // slot first + i holds token t + (first + i - slot) when that lies in the run
-    float x[B];
 #pragma unroll
-    for (int i = 0; i < B; ++i) {
-        const int jt = first + i - slot;
-        uint32_t w = 0u;
+    for (int cc = 0; cc < VC; ++cc) {
+        float x[B];
 #pragma unroll
-        for (int u = 0; u < B; ++u) w = (u == jt) ? raw[u] : w;
-        x[i] = (jt >= 0 && jt < n) ? __uint_as_float(w << 16) : 0.0f;
+        for (int i = 0; i < B; ++i) {
+            const uint32_t w = raw[i][cc >> 1];
+            x[i] = __uint_as_float((cc & 1) ? (w & 0xffff0000u) : (w << 16));
+        }
+        const uint32_t code = plain_scale_code<FMT>(block_amax<B>(x), g);
+        uint32_t packed[B / 8];
+        if constexpr (FMT == BDFP4_MXFP4) {
+            // sigma = 2^(code - 127): dividing by it is multiplying by 2^(127 - code), exactly
+            const float inv = __uint_as_float(code == 254u ? 0x00400000u : (254u - code) << 23);
+            quantize_block<B, false, true>(x, block_sigma<FMT>(code, g), packed, nullptr, inv);
+        } else {
+            quantize_block<B>(x, block_sigma<FMT>(code, g), packed);
+        }
+        uint8_t* dst = vp + v_nib_offset(c0 + cc, first);
+        if constexpr (B == 16) {
+            *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
+        } else {
+            *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        }
+        vs[v_scale_offset<B>(c0 + cc, first / B)] = (uint8_t)code;
     }
-    const uint32_t code = plain_scale_code<FMT>(block_amax<B>(x), g);
-    uint32_t packed[B / 8];
-    quantize_block<B>(x, block_sigma<FMT>(code, g), packed);
-    uint8_t* dst = vp + v_nib_offset(c, first);
-    if constexpr (B == 16) {
-        *reinterpret_cast<uint2*>(dst) = make_uint2(packed[0], packed[1]);
-    } else {
-        *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-    }
-    vs[v_scale_offset<B>(c, first / B)] = (uint8_t)code;
 }
 
 // Decode-step append: key CTAs first, then value CTAs, one (sequence, KV
@@ -101,9 +130,9 @@ template <int FMT, int DK, int DV>
 __global__ void __launch_bounds__(256) step_append_kernel(const DecodeArgs a, const StepArgs s) {
     const int64_t rows = (int64_t)a.B * a.H_kv;
     const NewestSlot slot{a.block_table, a.seq_lens, a.max_pages, a.num_pages, a.dev_status};
-    const int nk = (int)k_append_ctas<FMT, DK>(rows);
+    const int nk = (int)k_append_ctas_wide<FMT, DK>(rows);
     if ((int)blockIdx.x < nk)
-        append_k_cta<FMT, DK>(blockIdx.x, s.k_new, rows, a.H_kv, slot, a.smooth, a.k_gscale, a.k_weight, s.k_pages, s.k_scales,
+        append_k_cta_wide<FMT, DK>(blockIdx.x, s.k_new, rows, a.H_kv, slot, a.smooth, a.k_gscale, a.k_weight, s.k_pages, s.k_scales,
                               a.flags);
     else
         append_v_open_cta<FMT, DV>(blockIdx.x - nk, s.v_new, s.v_open, slot, a.B, a.H_kv, a.v_gscale, s.v_pages,
@@ -113,7 +142,7 @@ __global__ void __launch_bounds__(256) step_append_kernel(const DecodeArgs a, co
 template <int FMT, int DK, int DV>
 static int launch_step_append_t(const DecodeArgs& a, const StepArgs& s, cudaStream_t st) {
     const int64_t rows = (int64_t)a.B * a.H_kv;
-    const int64_t ctas = k_append_ctas<FMT, DK>(rows) + v_append_ctas<DV>(rows);
+    const int64_t ctas = k_append_ctas_wide<FMT, DK>(rows) + v_append_ctas<DV>(rows);
     step_append_kernel<FMT, DK, DV><<<(unsigned)ctas, 256, 0, st>>>(a, s);
     return launch_status();
 }
@@ -346,11 +375,10 @@ static void launch_quantize_kv(const void* k, const void* v, const int64_t* slot
     quantize_k_kernel<FMT, DK><<<(unsigned)kblocks, 256, 0, st>>>(
         (const __nv_bfloat16*)k, slot_mapping, T, H_kv, kv->smooth, kv->k_gscale, kv->k_weight, (uint8_t*)k_pages,
         (uint8_t*)k_scales, num_pages, flags, dev_status);
-    using VG = VGeom<DV>;
-    const int64_t vblocks = (rows + VG::RPC - 1) / VG::RPC * VG::CPR;
-    quantize_v_kernel<FMT, DV><<<(unsigned)vblocks, 256, 0, st>>>((const __nv_bfloat16*)v, slot_mapping, T, H_kv,
-                                                                  kv->v_gscale, (uint8_t*)v_pages,
-                                                                  (uint8_t*)v_scales, num_pages);
+    const int64_t vthreads = rows * (DV / VAppend<FMT>::VC);
+    quantize_v_kernel<FMT, DV><<<(unsigned)((vthreads + 255) / 256), 256, 0, st>>>(
+        (const __nv_bfloat16*)v, slot_mapping, T, H_kv, kv->v_gscale, (uint8_t*)v_pages, (uint8_t*)v_scales,
+        num_pages);
 }
 
 extern "C" int bdfp4_quantize_kv(const void* k, const void* v, const int64_t* slot_mapping, int T, int H_kv, int d_k,
@@ -427,17 +455,18 @@ extern "C" int bdfp4_quantize_v(const void* v, const int64_t* slot_mapping, int 
     if (!aligned(v, 16) || !aligned(v_pages, 128) || !aligned(v_scales, 128)) return BDFP4_ERR_ALIGN;
     cudaStream_t st = (cudaStream_t)stream;
     const int64_t rows = (int64_t)T * H_kv;
-    auto launch = [&](auto kernel, int RPC, int CPR) {
-        kernel<<<(unsigned)((rows + RPC - 1) / RPC * CPR), 256, 0, st>>>((const __nv_bfloat16*)v, slot_mapping, T,
-                                                                        H_kv, kv->v_gscale, (uint8_t*)v_pages,
-                                                                        (uint8_t*)v_scales, num_pages);
+    auto launch = [&](auto kernel, int groups_per_row) {
+        const int64_t threads = rows * groups_per_row;
+        kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>((const __nv_bfloat16*)v, slot_mapping, T, H_kv,
+                                                                 kv->v_gscale, (uint8_t*)v_pages, (uint8_t*)v_scales,
+                                                                 num_pages);
     };
     if (fmt == BDFP4_NVFP4) {
-        if (d_v == 128) launch(quantize_v_kernel<BDFP4_NVFP4, 128>, VGeom<128>::RPC, VGeom<128>::CPR);
-        else launch(quantize_v_kernel<BDFP4_NVFP4, 512>, VGeom<512>::RPC, VGeom<512>::CPR);
+        if (d_v == 128) launch(quantize_v_kernel<BDFP4_NVFP4, 128>, 128 / VAppend<BDFP4_NVFP4>::VC);
+        else launch(quantize_v_kernel<BDFP4_NVFP4, 512>, 512 / VAppend<BDFP4_NVFP4>::VC);
     } else {
-        if (d_v == 128) launch(quantize_v_kernel<BDFP4_MXFP4, 128>, VGeom<128>::RPC, VGeom<128>::CPR);
-        else launch(quantize_v_kernel<BDFP4_MXFP4, 512>, VGeom<512>::RPC, VGeom<512>::CPR);
+        if (d_v == 128) launch(quantize_v_kernel<BDFP4_MXFP4, 128>, 128 / VAppend<BDFP4_MXFP4>::VC);
+        else launch(quantize_v_kernel<BDFP4_MXFP4, 512>, 512 / VAppend<BDFP4_MXFP4>::VC);
     }
     return launch_status();
 }

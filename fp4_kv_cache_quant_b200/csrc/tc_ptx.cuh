@@ -67,6 +67,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 #endif
 }
 
+// Bounded wait used while unwinding (the abort flag is already set): gives up
+// only after `limit` clock cycles.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, long long limit) {
+    if (mbar_try(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try(bar, parity)) return true;
+        if (clock64() - t0 > limit) return false;
+    }
+}
+
 // ------------------------------------------------------------------ bulk copy
 // Untiled bulk copy global -> shared completing on an mbarrier (16-byte
 // aligned addresses, size a multiple of 16).

@@ -32,6 +32,7 @@ def test_exports_every_declared_entry_point(lib):
     names = _declared()
     assert set(bdfp4.ENTRY_POINTS) <= set(names)
     assert set(bdfp4.BF16_ENTRY_POINTS) <= set(names)
+    assert set(bdfp4.DEBUG_ENTRY_POINTS) <= set(names)
     for n in names:
         assert hasattr(lib, n), n
 
