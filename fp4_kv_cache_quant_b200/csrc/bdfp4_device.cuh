@@ -69,6 +69,17 @@ __device__ __forceinline__ uint32_t e2m1x2_encode(float lo, float hi) {
 
 __device__ __forceinline__ uint32_t e2m1_encode(float x) { return e2m1x2_encode(x, 0.0f) & 0xfu; }
 
+// Values of the E2M1 pair lo | hi << 4 (as e2m1x2_encode packs it) through the
+// hardware conversion: .x the low code's, .y the high code's (exact: E2M1 is a
+// subset of fp16).
+__device__ __forceinline__ float2 e2m1x2_value(uint32_t pair) {
+    uint32_t h2;
+    asm("{\n .reg .b8 t;\n .reg .b16 u;\n cvt.u16.u32 u, %1;\n cvt.u8.u16 t, u;\n cvt.rn.f16x2.e2m1x2 %0, t;\n}\n"
+        : "=r"(h2)
+        : "r"(pair));
+    return __half22float2(*reinterpret_cast<const __half2*>(&h2));
+}
+
 // ------------------------------------------------------------------ E4M3
 // Value of an E4M3FN code (0..0x7e used; bias 7, subnormals m * 2^-9).
 __device__ __forceinline__ float e4m3_value(uint32_t code) {

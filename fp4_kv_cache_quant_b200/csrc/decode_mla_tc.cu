@@ -226,7 +226,6 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
     uint64_t* q_full = q_ready + 1;           // query image landed -> softmax
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SM_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::SM_MISC + 4);
-    volatile int* sm_abort = reinterpret_cast<volatile int*>(smem + C::SM_MISC + 8);   // [NSG]
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int split = blockIdx.x, slice = blockIdx.y, b = blockIdx.z;
@@ -269,7 +268,6 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
         tc::mbar_init(q_ready, C::NSW);
         tc::mbar_init(q_full, 1);
         *abort_flag = 0;
-        for (int g = 0; g < C::NSG; ++g) sm_abort[g] = 0;
         tc::fence_mbar_init();
     }
     if (warp == C::MMA_WARP) {
@@ -464,6 +462,7 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
         const uint32_t tq = tbase + ((uint32_t)(32 * qd) << 16);
         const float alpha = (FMT == BDFP4_NVFP4 && !(a.flags & BDFP4_FLAG_NO_UNDERFLOW)) ? kAlphaNV : 1.0f;
         bool bad = false;
+        bool grp_abort = false;   // the group's four warps gave up (alike in all of them)
 
         // Pages the block table gets wrong (the producer reports them and copies nothing) are
         // skipped like tokens past the end: their logits are masked and their V scales zeroed.
@@ -587,9 +586,12 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
                     const float hi = tc::redux_max_f32(lo_half ? -INFINITY : x, 0xffffffffu);
                     if (lane == 0) *reinterpret_cast<float2*>(rw + ((gb + g) * 4 + qd) * 2) = make_float2(lo, hi);
                 }
-                if (bad || *abort_flag) sm_abort[grp] = 1;
-                tc::named_bar_sync(bar_id, 128);
-                if (sm_abort[grp]) break;
+                // one decision for the group's four warps, taken by the barrier itself (a role
+                // that gave up leaves a wait here unfinished, and the wait sees its abort flag)
+                if (tc::named_bar_or(bar_id, 128, bad)) {
+                    grp_abort = true;
+                    break;
+                }
                 // new running maxima, one head per lane, and the scales of the warp's two token
                 // blocks: the block maximum of alpha p is 2^(x_b ls - base) for the block's largest
                 // logit x_b, so the scale is the one the block's largest member picks
@@ -755,16 +757,15 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
         };
         if (any_bad_page) tiles(std::true_type{});
         else tiles(std::false_type{});
-        if (!sm_abort[grp]) {
+        if (!grp_abort) {
             if (!tc::mbar_wait(&o_done[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag, kWaitLimitMla)) bad = true;
             tc::tc_fence_after();
         }
-        if (bad || *abort_flag) sm_abort[grp] = 1;
 
         // ------------------------------------------------------------ epilogue (thread = channel)
-        tc::named_bar_sync(bar_id, 128);
-        if (sm_abort[grp]) *abort_flag = 1;
-        if (!sm_abort[grp]) {
+        grp_abort = tc::named_bar_or(bar_id, 128, grp_abort || bad || *abort_flag);
+        if (grp_abort) *abort_flag = 1;
+        if (!grp_abort) {
             float* rl = red;   // [GH][4] partial sums (the tile maxima are no longer read)
 #pragma unroll
             for (int g = 0; g < HG; ++g) {

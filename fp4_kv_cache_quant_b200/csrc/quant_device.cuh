@@ -200,9 +200,9 @@ __device__ __forceinline__ uint32_t search_scale(const float* x, float g, const 
             float e = 0.0f;
 #pragma unroll
             for (int i = 0; i < B; i += 2) {
-                const uint32_t pair = e2m1x2_encode(x[i] * r, x[i + 1] * r);
-                const float d0 = fmaf(-e2m1_value(pair & 15u), sg, x[i]);
-                const float d1 = fmaf(-e2m1_value(pair >> 4), sg, x[i + 1]);
+                const float2 v = e2m1x2_value(e2m1x2_encode(x[i] * r, x[i + 1] * r));
+                const float d0 = fmaf(-v.x, sg, x[i]);
+                const float d1 = fmaf(-v.y, sg, x[i + 1]);
                 e = fmaf(W ? w[i] * d0 : d0, d0, e);
                 e = fmaf(W ? w[i + 1] * d1 : d1, d1, e);
             }
