@@ -543,8 +543,10 @@ extern "C" int bdfp4_debug_decode_wait_test(const void* q, const void* k_pages, 
                                             void* workspace, size_t workspace_bytes, void* out,
                                             int32_t* dev_status, long long wait_limit_cycles, int stall,
                                             void* stream) {
-    // only the d = 128 tensor-core decode takes the switch
-    if (d_k != 128 || d_v != 128 || H_kv <= 0 || H_q % H_kv || H_q / H_kv > 16) return BDFP4_ERR_UNSUPPORTED;
+    // only the d = 128 tensor-core decode's eight-head instantiation takes the switch
+    if (d_k != 128 || d_v != 128 || H_kv <= 0 || H_q % H_kv || H_q / H_kv != 8 ||
+        (flags & BDFP4_FLAG_DYNAMIC_ALPHA))
+        return BDFP4_ERR_UNSUPPORTED;
     if (wait_limit_cycles <= 0) return BDFP4_ERR_ARG;
     return run_decode(q, k_pages, k_scales, v_pages, v_scales, block_table, seq_lens, B, 1, H_q, H_kv, d_k, d_v,
                       max_pages_per_seq, num_pages, fmt, flags, kv, sm_scale, chunk_tiles, workspace,

@@ -229,9 +229,14 @@ __global__ void __launch_bounds__(256) prep_step_kernel(const DecodeArgs a, cons
 
 // MT: several query tokens per sequence (a.T_q), their query heads stacked as
 // the G rows (token-major); query token i sees the first N - T_q + 1 + i tokens.
-template <int FMT, int G, bool DYN = false, bool MT = false>
+// HOOK: the unwind test's instantiation (bdfp4_debug.h) -- its wait bound and
+// its first-tile stall come from the arguments; every other instantiation bounds
+// its waits at the compile-time kWaitLimitDefault.
+template <int FMT, int G, bool DYN = false, bool MT = false, bool HOOK = false>
 __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTAS) decode_tc_kernel(const DecodeArgs a) {
     using C = TcCfg<FMT, G>;
+    const long long wlim = HOOK ? a.wait_limit : kWaitLimitDefault;
+    const bool stall = HOOK && a.test_stall;
     // the split merge (a programmatic dependent) may be scheduled as CTAs of this grid retire
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     constexpr bool MX = FMT == BDFP4_MXFP4;
@@ -351,12 +356,12 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                 // slots lane and 32 + lane of each page and scale group into row lane of the
                 // group's tcgen05.cp source, then arrives on the stage barrier once they land
                 // the unwind test withholds tile 0's K half: the MMA warp's wait for it runs out
-                if (do_k && !(a.test_stall && k == 0)) {
+                if (do_k && !(stall && k == 0)) {
                     // the step prologue writes the new token into the sequence's last page:
                     // that tile's copies wait until the prologue grid has finished
                     if (a.append_wait && tile0 + k == ntiles - 1) asm volatile("griddepcontrol.wait;" ::: "memory");
                     if (lane == 0) {
-                        if (k >= C::NSK && !tc::mbar_wait(&kempty[ks], ((k / C::NSK) - 1) & 1, abort_flag, a.wait_limit))
+                        if (k >= C::NSK && !tc::mbar_wait(&kempty[ks], ((k / C::NSK) - 1) & 1, abort_flag, wlim))
                             ok = false;
                         else
                             tc::mbar_arrive_expect_tx(&kfull[ks], (pg0 >= 0 ? C::K_PAGE : 0) + (pg1 >= 0 ? C::K_PAGE : 0));
@@ -385,7 +390,7 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                 // V half of tile v: lanes 0-1 copy the V pages, 2-3 their scales
                 if (do_v) {
                     if (lane == 0) {
-                        if (v >= C::NSV && !tc::mbar_wait(&vempty[vsi], ((v / C::NSV) - 1) & 1, abort_flag, a.wait_limit))
+                        if (v >= C::NSV && !tc::mbar_wait(&vempty[vsi], ((v / C::NSV) - 1) & 1, abort_flag, wlim))
                             ok = false;
                         else
                             tc::mbar_arrive_expect_tx(&vfull[vsi], (pv0_ >= 0 ? C::V_PAGE + C::VS_PAGE : 0) +
@@ -416,18 +421,18 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
         // Unwinding: before the CTA can exit, every copy this warp started must have landed.
         // Each stage's last announced phase completes once its bytes (and the lanes' cp.async
         // arrivals) are in; announced tiles run consecutively from the first one announced.
-        if (!ok || a.test_stall || *abort_flag) {
+        if (!ok || stall || *abort_flag) {
             if (lane == 0) {
-                const int k_first = a.test_stall ? 1 : 0;
+                const int k_first = stall ? 1 : 0;
                 for (int s = 0; s < C::NSK; ++s) {
                     if (k_last < s) continue;
                     const int t = k_last - (k_last - s) % C::NSK;
-                    if (t >= k_first) tc::mbar_wait_drain(&kfull[s], (t / C::NSK) & 1, a.wait_limit);
+                    if (t >= k_first) tc::mbar_wait_drain(&kfull[s], (t / C::NSK) & 1, wlim);
                 }
                 for (int s = 0; s < C::NSV; ++s) {
                     if (v_last < s) continue;
                     const int t = v_last - (v_last - s) % C::NSV;
-                    tc::mbar_wait_drain(&vfull[s], (t / C::NSV) & 1, a.wait_limit);
+                    tc::mbar_wait_drain(&vfull[s], (t / C::NSV) & 1, wlim);
                 }
             }
             __syncwarp();
@@ -447,7 +452,7 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                 else return v;
             };
             auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
-                return all(tc::mbar_wait(bar, parity, abort_flag, a.wait_limit));
+                return all(tc::mbar_wait(bar, parity, abort_flag, wlim));
             };
             constexpr uint32_t idesc_qk = tc::idesc_fp4(C::NQ, MX);
             constexpr uint32_t idesc_pv = tc::idesc_fp4(C::NP, MX);
@@ -572,7 +577,7 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                 *abort_flag = 1;
                 // unwinding: the tensor memory is freed below, so the MMAs and copies into it
                 // must have finished
-                if (last_bar) tc::mbar_wait_drain(last_bar, last_par, a.wait_limit);
+                if (last_bar) tc::mbar_wait_drain(last_bar, last_par, wlim);
             }
         }
     } else {
@@ -622,7 +627,7 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
         }
         // the P scale-factor buffers: zero (rows of absent heads must stay zero)
         for (int i = tid; i < 2 * 2 * 512 / 16; i += 32 * C::NSW) reinterpret_cast<uint4*>(psf)[i] = make_uint4(0, 0, 0, 0);
-        if (!tc::mbar_wait(q_full, 0, abort_flag, a.wait_limit)) bad = true;
+        if (!tc::mbar_wait(q_full, 0, abort_flag, wlim)) bad = true;
         // query scale factors (SFB of QK): lane n <- row n, one 4-column chunk per K step
         if (grp == 0) {
 #pragma unroll
@@ -687,7 +692,7 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                     pok1 = (f & 2u) != 0;
                 }
                 // logits of this thread's token for the group's heads (q1 then q2 columns)
-                if (!tc::mbar_wait(&s_full[buf], (j >> 1) & 1, abort_flag, a.wait_limit)) bad = true;
+                if (!tc::mbar_wait(&s_full[buf], (j >> 1) & 1, abort_flag, wlim)) bad = true;
                 tc::tc_fence_after();
                 uint32_t sr[2 * HG];
                 tc::tmem_ld<2 * HG>(tq + C::T_S + buf * C::NQ + 2 * gb, sr);
@@ -791,7 +796,7 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                 // O^T rescale of the group's heads once the previous tile's PV has completed,
                 // before this tile's PV is issued (the online-softmax update, in TMEM)
                 if (j > 0 && rose) {
-                    if (!tc::mbar_wait(&o_full[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, a.wait_limit)) bad = true;
+                    if (!tc::mbar_wait(&o_full[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, wlim)) bad = true;
                     tc::tc_fence_after();
                     uint32_t ov[HG];
                     tc::tmem_ld<HG>(tq + C::T_O + gb, ov);
@@ -812,7 +817,7 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                         const bool tail = (tile + 1) * kTileTokens > N;
                         uint8_t* vs = smem + C::SM_VST + s * C::VSTAGE + C::OFF_VS;
                         if (tail || !pok0 || !pok1) {
-                            if (!tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, a.wait_limit)) bad = true;
+                            if (!tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, wlim)) bad = true;
     #pragma unroll
                             for (int p = 0; p < 2; ++p) {
                                 const int t0 = tile * kTileTokens + p * kPageSlots;
@@ -837,7 +842,7 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
 #pragma unroll
         for (int g = 0; g < HG; ++g) o_fin[g] = 0u;
         if (!grp_abort) {
-            if (!tc::mbar_wait(&o_full[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag, a.wait_limit)) bad = true;
+            if (!tc::mbar_wait(&o_full[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag, wlim)) bad = true;
             tc::tc_fence_after();
             tc::tmem_ld<HG>(tq + C::T_O + gb, o_fin);
             tc::tmem_wait_ld();
@@ -889,12 +894,12 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
     }
 }
 
-template <int FMT, int G, bool DYN = false, bool MT = false>
+template <int FMT, int G, bool DYN = false, bool MT = false, bool HOOK = false>
 static int launch_tc(const DecodeArgs& a, cudaStream_t st, const StepArgs* step) {
     using C = TcCfg<FMT, G>;
     static bool attr_set = false;
     if (!attr_set) {
-        const cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<FMT, G, DYN, MT>,
+        const cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<FMT, G, DYN, MT, HOOK>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_LAUNCH);
         if (e != cudaSuccess) {
             record_cuda_error(e);
@@ -928,7 +933,7 @@ static int launch_tc(const DecodeArgs& a, cudaStream_t st, const StepArgs* step)
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<FMT, G, DYN, MT>, a);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<FMT, G, DYN, MT, HOOK>, a);
     if (e != cudaSuccess) {
         record_cuda_error(e);
         return BDFP4_ERR_CUDA;
@@ -969,6 +974,12 @@ static int dispatch_tc(const DecodeArgs& a, int fmt, int G, cudaStream_t st, con
 // G = rows stacked per (sequence, KV head): the query heads of the group, times
 // the query tokens per sequence when a.T_q > 1 (which then takes the MT kernels)
 int launch_decode_tc(const DecodeArgs& a, int fmt, int G, cudaStream_t st, const StepArgs* step) {
+    if (a.test_stall || a.wait_limit != kWaitLimitDefault) {
+        // the unwind test's instantiation: eight heads per KV head, one query token, no step
+        if (G != 8 || a.T_q != 1 || step || (a.flags & BDFP4_FLAG_DYNAMIC_ALPHA)) return BDFP4_ERR_UNSUPPORTED;
+        return fmt == BDFP4_NVFP4 ? launch_tc<BDFP4_NVFP4, 8, false, false, true>(a, st, step)
+                                  : launch_tc<BDFP4_MXFP4, 8, false, false, true>(a, st, step);
+    }
     return a.T_q > 1 ? dispatch_tc<true>(a, fmt, G, st, step) : dispatch_tc<false>(a, fmt, G, st, step);
 }
 

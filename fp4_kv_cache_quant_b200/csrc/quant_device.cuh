@@ -123,6 +123,18 @@ template <int FMT, bool W>
 __device__ __forceinline__ int search_exact(const float* x, float g, const float* w, int hi, uint32_t take,
                                             uint32_t* packed) {
     constexpr int B = Fmt<FMT>::beta;
+    if (take && !(take & (take - 1u))) {
+        // one code left: nothing to compare, only its elements are needed
+        const int c = hi - (__ffs(take) - 1);
+        const float sg = block_sigma<FMT>((uint32_t)c, g);
+        if constexpr (FMT == BDFP4_MXFP4) {
+            const float inv = __uint_as_float(c == 254 ? 0x00400000u : (uint32_t)(254 - c) << 23);
+            quantize_block<B, false, true>(x, sg, packed, nullptr, inv);
+        } else {
+            quantize_block<B>(x, sg, packed);
+        }
+        return c;
+    }
     int best = -1;
     double best_err = 0.0;
 #pragma unroll 1

@@ -13,7 +13,8 @@ extern "C" {
 #endif
 
 /*
- * bdfp4_decode on the d = 128 tensor-core decode (H_q / H_kv <= 16) with every
+ * bdfp4_decode on the d = 128 tensor-core decode (H_q / H_kv = 8, static
+ * probability pre-scale: the one shape compiled with this switch) with every
  * in-kernel wait bounded by wait_limit_cycles clock cycles instead of about two
  * seconds, and, when stall is nonzero, each CTA's first K tile never announced
  * to its MMA warp.  The MMA warp's wait for that tile then runs out: the CTA

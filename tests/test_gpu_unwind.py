@@ -68,7 +68,7 @@ def test_a_wait_that_runs_out_unwinds_and_reports(ora, fmt, chunk):
 
 
 def test_the_hook_refuses_other_shapes(ora):
-    sp = spec("mla", B=1, H_q=16, ctx=("fixed", 64))
+    sp = spec("tiny", B=1, ctx=("fixed", 64))   # four heads per KV head
     wl = Workload(sp, seed=16)
     cache = bdfp4.FP4Cache.empty(wl.num_pages, sp.H_kv, sp.d_k, sp.d_v, bdfp4.NVFP4)
     smooth, kg, vg = oracle_calibration(ora, wl)
