@@ -68,7 +68,7 @@ DECODE_SOURCES = {
     128: ("decode_tc.cu", "tc_ptx.cuh", "bdfp4_device.cuh", "quant_device.cuh", "decode_common.cuh",
           "append_device.cuh", "prob_scale.cuh"),
     576: ("decode_mla_tc.cu", "tc_ptx.cuh", "bdfp4_device.cuh", "quant_device.cuh", "decode_common.cuh",
-          "append_device.cuh"),
+          "append_device.cuh", "prob_scale.cuh"),
 }
 
 

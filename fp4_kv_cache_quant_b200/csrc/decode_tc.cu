@@ -582,307 +582,312 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
         }
     } else {
         // ------------------------------------------------------------ softmax warps
-        const int grp = warp >> 2;                 // head group
-        const int qd = warp & 3;                   // TMEM lane quadrant = tokens 32 qd .. 32 qd + 31
-        const int gb = grp * HG;                   // first head of the group
-        const int bar_id = 1 + grp;                // named barrier of the group (128 threads)
-        const uint32_t tq = tbase + ((uint32_t)(32 * qd) << 16);
-        const float alpha = (FMT == BDFP4_NVFP4 && !(a.flags & BDFP4_FLAG_NO_UNDERFLOW)) ? kAlphaNV : 1.0f;
-        bool bad = false;
-        bool grp_abort = false;   // the group's four warps gave up (alike in all of them)
+        // the body is instantiated once per head group, so the group's offsets are constants
+        auto softmax_role = [&](auto grp_c) {
+            constexpr int grp = decltype(grp_c)::value;   // head group
+            const int qd = warp & 3;                   // TMEM lane quadrant = tokens 32 qd .. 32 qd + 31
+            constexpr int gb = grp * HG;               // first head of the group
+            constexpr int bar_id = 1 + grp;            // named barrier of the group (128 threads)
+            const uint32_t tq = tbase + ((uint32_t)(32 * qd) << 16);
+            const float alpha = (FMT == BDFP4_NVFP4 && !(a.flags & BDFP4_FLAG_NO_UNDERFLOW)) ? kAlphaNV : 1.0f;
+            bool bad = false;
+            bool grp_abort = false;   // the group's four warps gave up (alike in all of them)
 
-        // Pages the block table gets wrong (the producer reports them and copies nothing) are
-        // skipped like tokens past the end: their logits are masked and their V scales zeroed.
-        // Before the first tile the softmax threads note, per tile of the split, whether both
-        // of its pages are good (bit 0: first page, bit 1: second) and whether any is not;
-        // splits longer than 64 tiles look tiles 64 on up in the block table as they go.
-        uint8_t* const pflag = smem + C::SM_PFLAG;
-        volatile int* const pflag_bad = reinterpret_cast<volatile int*>(smem + C::SM_PFLAG + 64);
-        auto page_flags = [&](int jt) -> uint32_t {
-            uint32_t r = 3u;
-#pragma unroll
-            for (int p = 0; p < 2; ++p) {
-                const int pi = (tile0 + jt) * 2 + p;
-                if (pi * kPageSlots < N) {   // pages past the end are masked anyway
-                    const int v = __ldg(a.block_table + (int64_t)b * a.max_pages + pi);
-                    if (v < 0 || v >= a.num_pages) r &= ~(1u << p);
+            // Pages the block table gets wrong (the producer reports them and copies nothing) are
+            // skipped like tokens past the end: their logits are masked and their V scales zeroed.
+            // Before the first tile the softmax threads note, per tile of the split, whether both
+            // of its pages are good (bit 0: first page, bit 1: second) and whether any is not;
+            // splits longer than 64 tiles look tiles 64 on up in the block table as they go.
+            uint8_t* const pflag = smem + C::SM_PFLAG;
+            volatile int* const pflag_bad = reinterpret_cast<volatile int*>(smem + C::SM_PFLAG + 64);
+            auto page_flags = [&](int jt) -> uint32_t {
+                uint32_t r = 3u;
+    #pragma unroll
+                for (int p = 0; p < 2; ++p) {
+                    const int pi = (tile0 + jt) * 2 + p;
+                    if (pi * kPageSlots < N) {   // pages past the end are masked anyway
+                        const int v = __ldg(a.block_table + (int64_t)b * a.max_pages + pi);
+                        if (v < 0 || v >= a.num_pages) r &= ~(1u << p);
+                    }
                 }
-            }
-            return r;
+                return r;
         };
-        if (tid == 0) *pflag_bad = n > 64 ? 1 : 0;
-        tc::named_bar_sync(1 + C::NSG, 32 * C::NSW);
-        if (tid < 64 && tid < n) {
-            const uint32_t f = page_flags(tid);
-            pflag[tid] = (uint8_t)f;
-            if (f != 3u) *pflag_bad = 1;
-        }
-        // the query image (QK operand, scale codes, logit scales) of this (sequence, KV head)
-        // arrives in one bulk copy from prep_query_kernel, which this grid may overlap:
-        // griddepcontrol.wait holds the copy until that grid's writes are visible
-        if (tid == 0) {
-            asm volatile("griddepcontrol.wait;" ::: "memory");
-            tc::mbar_arrive_expect_tx(q_full, C::QPACK);
-            tc::bulk_g2s(q_op, a.qpack + ((int64_t)b * a.H_kv + hk) * C::QPACK, C::QPACK, q_full);
-        }
-        // the P scale-factor buffers: zero (rows of absent heads must stay zero)
-        for (int i = tid; i < 2 * 2 * 512 / 16; i += 32 * C::NSW) reinterpret_cast<uint4*>(psf)[i] = make_uint4(0, 0, 0, 0);
-        if (!tc::mbar_wait(q_full, 0, abort_flag, wlim)) bad = true;
-        // query scale factors (SFB of QK): lane n <- row n, one 4-column chunk per K step
-        if (grp == 0) {
-#pragma unroll
-            for (int ks = 0; ks < C::KS; ++ks) {
-                uint32_t v = 0;
-                if (lane < C::NQ) {
-                    if constexpr (B == 16) v = *reinterpret_cast<const uint32_t*>(qsc + lane * 8 + ks * 4);
-                    else v = (uint32_t)qsc[lane * 8 + ks * 2] | ((uint32_t)qsc[lane * 8 + ks * 2 + 1] << 8);
-                }
-                tc::tmem_st4(tq + C::T_SFQ + ks * 4, v, 0u, 0u, 0u);
+            if (tid == 0) *pflag_bad = n > 64 ? 1 : 0;
+            tc::named_bar_sync(1 + C::NSG, 32 * C::NSW);
+            if (tid < 64 && tid < n) {
+                const uint32_t f = page_flags(tid);
+                pflag[tid] = (uint8_t)f;
+                if (f != 3u) *pflag_bad = 1;
             }
-            tc::tmem_wait_st();
-        }
-        tc::tc_fence_before();
-        tc::fence_proxy_async_smem();
-        tc::named_bar_sync(1 + C::NSG, 32 * C::NSW);   // psf zeroed and page flags set before any tile
-        const bool any_bad_page = *pflag_bad != 0;
-        if (lane == 0) tc::mbar_arrive(q_ready);
-        float m_run[HG], l_part[HG];
-        // DYN: log2 of each head's current pre-scale; O^T and l are held in its units
-        int e_run[DYN ? HG : 1];
-#pragma unroll
-        for (int g = 0; g < HG; ++g) {
-            m_run[g] = -INFINITY;
-            l_part[g] = 0.0f;
-            if constexpr (DYN) e_run[g] = 11;
-        }
-        // TMEM lane 32 qd + lane holds token 32 qd + lane of the tile: slot 32 (qd % 2) + lane
-        // of page qd / 2, so a warp owns 32 consecutive slots of one page
-        const int page_of_thread = qd >> 1;
-        const int pos_in_page = 32 * (qd & 1) + lane;
-        const int tok_in_tile = 32 * qd + lane;
-        const int chan = 32 * qd + lane;   // O^T lane = value channel
+            // the query image (QK operand, scale codes, logit scales) of this (sequence, KV head)
+            // arrives in one bulk copy from prep_query_kernel, which this grid may overlap:
+            // griddepcontrol.wait holds the copy until that grid's writes are visible
+            if (tid == 0) {
+                asm volatile("griddepcontrol.wait;" ::: "memory");
+                tc::mbar_arrive_expect_tx(q_full, C::QPACK);
+                tc::bulk_g2s(q_op, a.qpack + ((int64_t)b * a.H_kv + hk) * C::QPACK, C::QPACK, q_full);
+            }
+            // the P scale-factor buffers: zero (rows of absent heads must stay zero)
+            for (int i = tid; i < 2 * 2 * 512 / 16; i += 32 * C::NSW) reinterpret_cast<uint4*>(psf)[i] = make_uint4(0, 0, 0, 0);
+            if (!tc::mbar_wait(q_full, 0, abort_flag, wlim)) bad = true;
+            // query scale factors (SFB of QK): lane n <- row n, one 4-column chunk per K step
+            if (grp == 0) {
+    #pragma unroll
+                for (int ks = 0; ks < C::KS; ++ks) {
+                    uint32_t v = 0;
+                    if (lane < C::NQ) {
+                        if constexpr (B == 16) v = *reinterpret_cast<const uint32_t*>(qsc + lane * 8 + ks * 4);
+                        else v = (uint32_t)qsc[lane * 8 + ks * 2] | ((uint32_t)qsc[lane * 8 + ks * 2 + 1] << 8);
+                    }
+                    tc::tmem_st4(tq + C::T_SFQ + ks * 4, v, 0u, 0u, 0u);
+                }
+                tc::tmem_wait_st();
+            }
+            tc::tc_fence_before();
+            tc::fence_proxy_async_smem();
+            tc::named_bar_sync(1 + C::NSG, 32 * C::NSW);   // psf zeroed and page flags set before any tile
+            const bool any_bad_page = *pflag_bad != 0;
+            if (lane == 0) tc::mbar_arrive(q_ready);
+            float m_run[HG], l_part[HG];
+            // DYN: log2 of each head's current pre-scale; O^T and l are held in its units
+            int e_run[DYN ? HG : 1];
+    #pragma unroll
+            for (int g = 0; g < HG; ++g) {
+                m_run[g] = -INFINITY;
+                l_part[g] = 0.0f;
+                if constexpr (DYN) e_run[g] = 11;
+            }
+            // TMEM lane 32 qd + lane holds token 32 qd + lane of the tile: slot 32 (qd % 2) + lane
+            // of page qd / 2, so a warp owns 32 consecutive slots of one page
+            const int page_of_thread = qd >> 1;
+            const int pos_in_page = 32 * (qd & 1) + lane;
+            const int tok_in_tile = 32 * qd + lane;
+            const int chan = 32 * qd + lane;   // O^T lane = value channel
 
-        // log2 of alpha: alpha * 2^(x - m) is evaluated as 2^(x - (m - log2 alpha))
-        const float la = alpha == kAlphaNV ? 11.0f : 0.0f;
-        float lsr[HG];
-#pragma unroll
-        for (int g = 0; g < HG; ++g) lsr[g] = lsc[gb + g];
-        const bool lo_half = lane < 16;
-        // P operand bytes: a lane pair (tokens 2i, 2i + 1 of a half warp) fills one byte of
-        // each head row; with two heads per pair step the even lane writes head g, the odd
-        // lane head g + 1.  Token pos of page p is K index pos: 16-byte chunk pos/32, byte (pos%32)/2
-        const int hsel = HG >= 2 ? (lane & 1) : 0;
-        const bool pstore = HG >= 2 || (lane & 1) == 0;
-        // the lanes that write a block's scale byte: the first (two) of the half warp
-        // (NVFP4, 16-token blocks) or of the warp (MXFP4, 32-token blocks)
-        const bool sfstore = (lane & (B - 1)) < (HG >= 2 ? 2 : 1);
-        const uint32_t psel = (lane & 1) ? 0x0004u : 0x0040u;   // byte 0 <- token 2i, byte 1 <- token 2i + 1
-        uint8_t* const pbyte = p_op + page_of_thread * C::P_PAGE + (qd & 1) * 128 + (lane >> 1) + hsel * 16;
-        uint8_t* const sfbyte = psf + page_of_thread * 512 + pos_in_page / B + hsel * 16;
+            // log2 of alpha: alpha * 2^(x - m) is evaluated as 2^(x - (m - log2 alpha))
+            const float la = alpha == kAlphaNV ? 11.0f : 0.0f;
+            float lsr[HG];
+    #pragma unroll
+            for (int g = 0; g < HG; ++g) lsr[g] = lsc[gb + g];
+            const bool lo_half = lane < 16;
+            // P operand bytes: a lane pair (tokens 2i, 2i + 1 of a half warp) fills one byte of
+            // each head row; with two heads per pair step the even lane writes head g, the odd
+            // lane head g + 1.  Token pos of page p is K index pos: 16-byte chunk pos/32, byte (pos%32)/2
+            const int hsel = HG >= 2 ? (lane & 1) : 0;
+            const bool pstore = HG >= 2 || (lane & 1) == 0;
+            // the lanes that write a block's scale byte: the first (two) of the half warp
+            // (NVFP4, 16-token blocks) or of the warp (MXFP4, 32-token blocks)
+            const bool sfstore = (lane & (B - 1)) < (HG >= 2 ? 2 : 1);
+            const uint32_t psel = (lane & 1) ? 0x0004u : 0x0040u;   // byte 0 <- token 2i, byte 1 <- token 2i + 1
+            uint8_t* const pbyte = p_op + page_of_thread * C::P_PAGE + (qd & 1) * 128 + (lane >> 1) + hsel * 16;
+            uint8_t* const sfbyte = psf + page_of_thread * 512 + pos_in_page / B + hsel * 16;
 
-        // The tile loop, in two copies: the page checks exist only in the copy a split with a
-        // bad page runs, so the normal copy carries no extra live registers.
-        auto tiles = [&](auto masked) {
-            for (int j = 0; j < n; ++j) {
-                const int buf = j & 1, tile = tile0 + j;
-                bool pok0 = true, pok1 = true;
-                if constexpr (decltype(masked)::value) {
-                    const uint32_t f = j < 64 ? pflag[j] : page_flags(j);
-                    pok0 = (f & 1u) != 0;
-                    pok1 = (f & 2u) != 0;
-                }
-                // logits of this thread's token for the group's heads (q1 then q2 columns)
-                if (!tc::mbar_wait(&s_full[buf], (j >> 1) & 1, abort_flag, wlim)) bad = true;
-                tc::tc_fence_after();
-                uint32_t sr[2 * HG];
-                tc::tmem_ld<2 * HG>(tq + C::T_S + buf * C::NQ + 2 * gb, sr);
-                tc::tmem_wait_ld();
-                const int token = tile * kTileTokens + tok_in_tile;
-                const bool valid = token < N && (page_of_thread ? pok1 : pok0);
-                // MT: the token is visible to query token i iff token <= N - T_q + i, i.e. to the
-                // stacked rows v = i G + g >= (token - (N - T_q)) G: rows g >= vis of this group
-                int vis = 0;
-                if constexpr (MT) vis = (token - (N - a.T_q)) * (a.H_q / a.H_kv) - gb;
-                // raw logits q1.k + q2.k (the positive factor lsc is applied later, so maxima
-                // commute with it) and their maxima over each half warp (16 consecutive slots)
-                float t[HG], hm_lo[HG], hm_hi[HG];
-    #pragma unroll
-                for (int g = 0; g < HG; ++g) {
-                    t[g] = (valid && (!MT || g >= vis)) ? __uint_as_float(sr[g]) + __uint_as_float(sr[HG + g]) : -INFINITY;
-                    hm_lo[g] = tc::redux_max_f32(lo_half ? t[g] : -INFINITY, 0xffffffffu);
-                    hm_hi[g] = tc::redux_max_f32(lo_half ? -INFINITY : t[g], 0xffffffffu);
-                }
-                float* rw = red + buf * C::RED_BUF;
-                if (lane == 0) {
-    #pragma unroll
-                    for (int g = 0; g < HG; ++g) {
-                        rw[(gb + g) * 4 + qd] = fmaxf(hm_lo[g], hm_hi[g]);
+            // The tile loop, in two copies: the page checks exist only in the copy a split with a
+            // bad page runs, so the normal copy carries no extra live registers.
+            auto tiles = [&](auto masked) {
+                for (int j = 0; j < n; ++j) {
+                    const int buf = j & 1, tile = tile0 + j;
+                    bool pok0 = true, pok1 = true;
+                    if constexpr (decltype(masked)::value) {
+                        const uint32_t f = j < 64 ? pflag[j] : page_flags(j);
+                        pok0 = (f & 1u) != 0;
+                        pok1 = (f & 2u) != 0;
                     }
-                }
-                // one decision for the group's four warps, taken by the barrier itself (a role
-                // that gave up leaves a wait here unfinished, and the wait sees its abort flag)
-                if (tc::named_bar_or(bar_id, 128, bad)) {
-                    grp_abort = true;
-                    break;
-                }
-                float y[HG], am[HG], corr[HG];
-                uint32_t mxc[HG];   // MXFP4 block scale codes
-                bool rose = false;   // a running maximum of the group rose (alike in its four warps)
-    #pragma unroll
-                for (int g = 0; g < HG; ++g) {
-                    const float4 w4 = *reinterpret_cast<const float4*>(rw + (gb + g) * 4);
-                    const float mt = fmaxf(fmaxf(w4.x, w4.y), fmaxf(w4.z, w4.w));
-                    const float mn = fmaxf(m_run[g], mt * lsr[g]);
-                    const float mz = mn == -INFINITY ? 0.0f : mn;
-                    corr[g] = tc::ex2_approx(m_run[g] - mz);   // 0 on the split's first tile
-                    rose |= mn != m_run[g];
-                    m_run[g] = mn;
-                    float base = mz - la;
-                    if constexpr (DYN) {
-                        // this tile's pre-scale from its largest probability; the accumulators
-                        // move to its units (an exact power of two, folded into corr)
-                        const int e = dynamic_alpha_exp(tc::ex2_approx(mt * lsr[g] - mz));
-                        corr[g] *= pow2f(e - e_run[g]);
-                        rose |= e != e_run[g];
-                        e_run[g] = e;
-                        base = mz - (float)e;
-                    }
-                    // the same two instructions give a token's scaled probability and its block's
-                    // maximum, so the block scale is the one its largest member picks
-                    y[g] = tc::ex2_approx(fmaf(t[g], lsr[g], -base));   // 0 for masked tokens
-                    l_part[g] = fmaf(l_part[g], corr[g], y[g]);         // l in units of alpha (cancels at the end)
-                    if constexpr (!MX) {
-                        // a 16-token block is this half warp
-                        const float bm = lo_half ? hm_lo[g] : hm_hi[g];
-                        am[g] = tc::ex2_approx(fmaf(bm, lsr[g], -base));
-                    } else {
-                        // a 32-token block is this warp.  The OCP MX shared exponent is taken in the
-                        // log domain: the block maximum is 2^d with d = x_b - m, so floor(log2) =
-                        // floor(d) exactly (d = 0 for the tile's largest logit), and the element is
-                        // 2^(x - m - e) for the scale 2^e
-                        const float bm = fmaxf(hm_lo[g], hm_hi[g]);
-                        const float d = __fsub_rn(__fmul_rn(bm, lsr[g]), mz);
-                        const int c = max(__float2int_rd(fmaxf(d, -256.0f)) + 125, 0);
-                        mxc[g] = (uint32_t)c;
-                        am[g] = tc::ex2_approx(fmaf(t[g], lsr[g], -(mz + (float)(c - 127))));
-                    }
-                }
-                // fused FP4 quantization of the probabilities, two heads per conversion
-                uint8_t* const pb = pbyte + buf * C::P_BUF;
-                uint8_t* const sfb = sfbyte + buf * 2 * 512;
-    #pragma unroll
-                for (int g = 0; g < HG; g += 2) {
-                    const int g1 = HG >= 2 ? g + 1 : g;
-                    uint32_t codes;
-                    float q0, q1;
-                    if constexpr (FMT == BDFP4_NVFP4) {
-                        codes = tc::e4m3x2_encode(__fmul_rn(am[g], 1.0f / 6.0f), __fmul_rn(am[g1], 1.0f / 6.0f));
-                        const float2 sg = tc::e4m3x2_value(codes);
-                        // a zero scale zeroes the whole block inside the MMA, whatever the element codes
-                        q0 = y[g] * tc::rcp_approx(sg.x);
-                        q1 = y[g1] * tc::rcp_approx(sg.y);
-                    } else {
-                        codes = mxc[g] | (mxc[g1] << 8);
-                        q0 = am[g];    // the element already divided by its block scale
-                        q1 = am[g1];
-                    }
-                    const uint32_t mine = e2m1x2_encode(q0, q1);   // head g in bits 0..3, head g1 in 4..7
-                    const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
-                    const uint32_t w = __byte_perm(mine, other, psel) >> (4 * hsel);
-                    const int hr = gb + g;
-                    if (pstore) pb[(hr >> 3) * 256 + (hr & 7) * 16] = (uint8_t)((w & 0xfu) | ((w >> 4) & 0xf0u));
-                    if (sfstore) sfb[hr * 16] = (uint8_t)(codes >> (8 * hsel));   // SFB rows hr, hr + 1
-                }
-                // O^T rescale of the group's heads once the previous tile's PV has completed,
-                // before this tile's PV is issued (the online-softmax update, in TMEM)
-                if (j > 0 && rose) {
-                    if (!tc::mbar_wait(&o_full[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, wlim)) bad = true;
+                    // logits of this thread's token for the group's heads (q1 then q2 columns)
+                    if (!tc::mbar_wait(&s_full[buf], (j >> 1) & 1, abort_flag, wlim)) bad = true;
                     tc::tc_fence_after();
-                    uint32_t ov[HG];
-                    tc::tmem_ld<HG>(tq + C::T_O + gb, ov);
+                    uint32_t sr[2 * HG];
+                    tc::tmem_ld<2 * HG>(tq + C::T_S + buf * C::NQ + 2 * gb, sr);
                     tc::tmem_wait_ld();
-#pragma unroll
-                    for (int g = 0; g < HG; ++g) ov[g] = __float_as_uint(__uint_as_float(ov[g]) * corr[g]);
-                    tc::tmem_st_n<HG>(tq + C::T_O + gb, ov);
-                    tc::tmem_wait_st();
-                    tc::tc_fence_before();
-                }
-                // NVFP4 V scale factors (group 0): blocks past the sequence end are zeroed, so the
-                // bytes a page holds there are never multiplied.  The V stage can not be
-                // refilled before this tile's PV, so waiting for it here is safe.  (MXFP4: the
-                // MMA warp builds the tile's V scale rows and masks them.)
-                if constexpr (B == 16) {
-                    if (grp == 0) {
-                        const int s = j % C::NSV;
-                        const bool tail = (tile + 1) * kTileTokens > N;
-                        uint8_t* vs = smem + C::SM_VST + s * C::VSTAGE + C::OFF_VS;
-                        if (tail || !pok0 || !pok1) {
-                            if (!tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, wlim)) bad = true;
+                    const int token = tile * kTileTokens + tok_in_tile;
+                    const bool valid = token < N && (page_of_thread ? pok1 : pok0);
+                    // MT: the token is visible to query token i iff token <= N - T_q + i, i.e. to the
+                    // stacked rows v = i G + g >= (token - (N - T_q)) G: rows g >= vis of this group
+                    int vis = 0;
+                    if constexpr (MT) vis = (token - (N - a.T_q)) * (a.H_q / a.H_kv) - gb;
+                    // raw logits q1.k + q2.k (the positive factor lsc is applied later, so maxima
+                    // commute with it) and their maxima over each half warp (16 consecutive slots)
+                    float t[HG], hm_lo[HG], hm_hi[HG];
+        #pragma unroll
+                    for (int g = 0; g < HG; ++g) {
+                        t[g] = (valid && (!MT || g >= vis)) ? __uint_as_float(sr[g]) + __uint_as_float(sr[HG + g]) : -INFINITY;
+                        hm_lo[g] = tc::redux_max_f32(lo_half ? t[g] : -INFINITY, 0xffffffffu);
+                        hm_hi[g] = tc::redux_max_f32(lo_half ? -INFINITY : t[g], 0xffffffffu);
+                    }
+                    float* rw = red + buf * C::RED_BUF;
+                    if (lane == 0) {
+        #pragma unroll
+                        for (int g = 0; g < HG; ++g) {
+                            rw[(gb + g) * 4 + qd] = fmaxf(hm_lo[g], hm_hi[g]);
+                        }
+                    }
+                    // one decision for the group's four warps, taken by the barrier itself (a role
+                    // that gave up leaves a wait here unfinished, and the wait sees its abort flag)
+                    if (tc::named_bar_or(bar_id, 128, bad)) {
+                        grp_abort = true;
+                        break;
+                    }
+                    float y[HG], am[HG], corr[HG];
+                    uint32_t mxc[HG];   // MXFP4 block scale codes
+                    bool rose = false;   // a running maximum of the group rose (alike in its four warps)
+        #pragma unroll
+                    for (int g = 0; g < HG; ++g) {
+                        const float4 w4 = *reinterpret_cast<const float4*>(rw + (gb + g) * 4);
+                        const float mt = fmaxf(fmaxf(w4.x, w4.y), fmaxf(w4.z, w4.w));
+                        const float mn = fmaxf(m_run[g], mt * lsr[g]);
+                        const float mz = mn == -INFINITY ? 0.0f : mn;
+                        corr[g] = tc::ex2_approx(m_run[g] - mz);   // 0 on the split's first tile
+                        rose |= mn != m_run[g];
+                        m_run[g] = mn;
+                        float base = mz - la;
+                        if constexpr (DYN) {
+                            // this tile's pre-scale from its largest probability; the accumulators
+                            // move to its units (an exact power of two, folded into corr)
+                            const int e = dynamic_alpha_exp(tc::ex2_approx(mt * lsr[g] - mz));
+                            corr[g] *= pow2f(e - e_run[g]);
+                            rose |= e != e_run[g];
+                            e_run[g] = e;
+                            base = mz - (float)e;
+                        }
+                        // the same two instructions give a token's scaled probability and its block's
+                        // maximum, so the block scale is the one its largest member picks
+                        y[g] = tc::ex2_approx(fmaf(t[g], lsr[g], -base));   // 0 for masked tokens
+                        l_part[g] = fmaf(l_part[g], corr[g], y[g]);         // l in units of alpha (cancels at the end)
+                        if constexpr (!MX) {
+                            // a 16-token block is this half warp
+                            const float bm = lo_half ? hm_lo[g] : hm_hi[g];
+                            am[g] = tc::ex2_approx(fmaf(bm, lsr[g], -base));
+                        } else {
+                            // a 32-token block is this warp.  The OCP MX shared exponent is taken in the
+                            // log domain: the block maximum is 2^d with d = x_b - m, so floor(log2) =
+                            // floor(d) exactly (d = 0 for the tile's largest logit), and the element is
+                            // 2^(x - m - e) for the scale 2^e
+                            const float bm = fmaxf(hm_lo[g], hm_hi[g]);
+                            const float d = __fsub_rn(__fmul_rn(bm, lsr[g]), mz);
+                            const int c = max(__float2int_rd(fmaxf(d, -256.0f)) + 125, 0);
+                            mxc[g] = (uint32_t)c;
+                            am[g] = tc::ex2_approx(fmaf(t[g], lsr[g], -(mz + (float)(c - 127))));
+                        }
+                    }
+                    // fused FP4 quantization of the probabilities, two heads per conversion
+                    uint8_t* const pb = pbyte + buf * C::P_BUF;
+                    uint8_t* const sfb = sfbyte + buf * 2 * 512;
+        #pragma unroll
+                    for (int g = 0; g < HG; g += 2) {
+                        const int g1 = HG >= 2 ? g + 1 : g;
+                        uint32_t codes;
+                        float q0, q1;
+                        if constexpr (FMT == BDFP4_NVFP4) {
+                            codes = tc::e4m3x2_encode(__fmul_rn(am[g], 1.0f / 6.0f), __fmul_rn(am[g1], 1.0f / 6.0f));
+                            const float2 sg = tc::e4m3x2_value(codes);
+                            // a zero scale zeroes the whole block inside the MMA, whatever the element codes
+                            q0 = y[g] * tc::rcp_approx(sg.x);
+                            q1 = y[g1] * tc::rcp_approx(sg.y);
+                        } else {
+                            codes = mxc[g] | (mxc[g1] << 8);
+                            q0 = am[g];    // the element already divided by its block scale
+                            q1 = am[g1];
+                        }
+                        const uint32_t mine = e2m1x2_encode(q0, q1);   // head g in bits 0..3, head g1 in 4..7
+                        const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
+                        const uint32_t w = __byte_perm(mine, other, psel) >> (4 * hsel);
+                        const int hr = gb + g;
+                        if (pstore) pb[(hr >> 3) * 256 + (hr & 7) * 16] = (uint8_t)((w & 0xfu) | ((w >> 4) & 0xf0u));
+                        if (sfstore) sfb[hr * 16] = (uint8_t)(codes >> (8 * hsel));   // SFB rows hr, hr + 1
+                    }
+                    // O^T rescale of the group's heads once the previous tile's PV has completed,
+                    // before this tile's PV is issued (the online-softmax update, in TMEM)
+                    if (j > 0 && rose) {
+                        if (!tc::mbar_wait(&o_full[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, wlim)) bad = true;
+                        tc::tc_fence_after();
+                        uint32_t ov[HG];
+                        tc::tmem_ld<HG>(tq + C::T_O + gb, ov);
+                        tc::tmem_wait_ld();
     #pragma unroll
-                            for (int p = 0; p < 2; ++p) {
-                                const int t0 = tile * kTileTokens + p * kPageSlots;
-                                int nvb = (N - t0 + B - 1) / B;
-                                nvb = nvb < 0 ? 0 : (nvb > C::SPB ? C::SPB : nvb);
-                                if (!(p ? pok1 : pok0)) nvb = 0;
-                                for (int bb = nvb; bb < C::SPB; ++bb)
-                                    vs[p * C::VS_PAGE + (chan & 31) * 16 + (chan >> 5) * 4 + bb] = 0;
+                        for (int g = 0; g < HG; ++g) ov[g] = __float_as_uint(__uint_as_float(ov[g]) * corr[g]);
+                        tc::tmem_st_n<HG>(tq + C::T_O + gb, ov);
+                        tc::tmem_wait_st();
+                        tc::tc_fence_before();
+                    }
+                    // NVFP4 V scale factors (group 0): blocks past the sequence end are zeroed, so the
+                    // bytes a page holds there are never multiplied.  The V stage can not be
+                    // refilled before this tile's PV, so waiting for it here is safe.  (MXFP4: the
+                    // MMA warp builds the tile's V scale rows and masks them.)
+                    if constexpr (B == 16) {
+                        if (grp == 0) {
+                            const int s = j % C::NSV;
+                            const bool tail = (tile + 1) * kTileTokens > N;
+                            uint8_t* vs = smem + C::SM_VST + s * C::VSTAGE + C::OFF_VS;
+                            if (tail || !pok0 || !pok1) {
+                                if (!tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, wlim)) bad = true;
+        #pragma unroll
+                                for (int p = 0; p < 2; ++p) {
+                                    const int t0 = tile * kTileTokens + p * kPageSlots;
+                                    int nvb = (N - t0 + B - 1) / B;
+                                    nvb = nvb < 0 ? 0 : (nvb > C::SPB ? C::SPB : nvb);
+                                    if (!(p ? pok1 : pok0)) nvb = 0;
+                                    for (int bb = nvb; bb < C::SPB; ++bb)
+                                        vs[p * C::VS_PAGE + (chan & 31) * 16 + (chan >> 5) * 4 + bb] = 0;
+                                }
                             }
                         }
                     }
+                    tc::fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(&p_ready[buf]);
                 }
-                tc::fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&p_ready[buf]);
+            };
+            if (any_bad_page) tiles(std::true_type{});
+            else tiles(std::false_type{});
+            // the split's O^T once its last PV has completed
+            uint32_t o_fin[HG];
+    #pragma unroll
+            for (int g = 0; g < HG; ++g) o_fin[g] = 0u;
+            if (!grp_abort) {
+                if (!tc::mbar_wait(&o_full[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag, wlim)) bad = true;
+                tc::tc_fence_after();
+                tc::tmem_ld<HG>(tq + C::T_O + gb, o_fin);
+                tc::tmem_wait_ld();
             }
-        };
-        if (any_bad_page) tiles(std::true_type{});
-        else tiles(std::false_type{});
-        // the split's O^T once its last PV has completed
-        uint32_t o_fin[HG];
-#pragma unroll
-        for (int g = 0; g < HG; ++g) o_fin[g] = 0u;
-        if (!grp_abort) {
-            if (!tc::mbar_wait(&o_full[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag, wlim)) bad = true;
-            tc::tc_fence_after();
-            tc::tmem_ld<HG>(tq + C::T_O + gb, o_fin);
-            tc::tmem_wait_ld();
-        }
 
-        // ------------------------------------------------------------ epilogue (thread = channel)
-        grp_abort = tc::named_bar_or(bar_id, 128, grp_abort || bad || *abort_flag);
-        if (grp_abort) *abort_flag = 1;
-        if (!grp_abort) {
-            float* rl = red;   // [G][8] partial sums (the tile maxima are no longer read)
-#pragma unroll
-            for (int g = 0; g < HG; ++g) {
-                float v = l_part[g];
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-                if (lane == 0) rl[(gb + g) * 8 + qd] = v;
-            }
-            tc::named_bar_sync(bar_id, 128);
-            // O and l both carry the factor alpha (P^ is alpha p quantized), so it cancels
-            const float oscale = FMT == BDFP4_NVFP4 ? a.v_gscale[hk] : 1.0f;
-            const int ch = chan;
-#pragma unroll
-            for (int g = 0; g < HG; ++g) {
-                const int hh = gb + g;
-                const float l = rl[hh * 8] + rl[hh * 8 + 1] + rl[hh * 8 + 2] + rl[hh * 8 + 3];
-                const int64_t row = row_of(hh);
-                if (nspl == 1) {
-                    a.out[row * C::DV + ch] =
-                        __float2bfloat16(l > 0.0f ? __uint_as_float(o_fin[g]) * oscale / l : 0.0f);
-                } else {
-                    // DYN: splits end in different units; the partials leave in the units of p
-                    const float un = DYN ? pow2f(-e_run[DYN ? g : 0]) : 1.0f;
-                    a.ws_o[(row * a.max_splits + split) * C::DV + ch] = __uint_as_float(o_fin[g]) * oscale * un;
-                    if (chan == 0) {
-                        a.ws_ml[(row * a.max_splits + split) * 2 + 0] = m_run[g];
-                        a.ws_ml[(row * a.max_splits + split) * 2 + 1] = l * un;
+            // ------------------------------------------------------------ epilogue (thread = channel)
+            grp_abort = tc::named_bar_or(bar_id, 128, grp_abort || bad || *abort_flag);
+            if (grp_abort) *abort_flag = 1;
+            if (!grp_abort) {
+                float* rl = red;   // [G][8] partial sums (the tile maxima are no longer read)
+    #pragma unroll
+                for (int g = 0; g < HG; ++g) {
+                    float v = l_part[g];
+    #pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+                    if (lane == 0) rl[(gb + g) * 8 + qd] = v;
+                }
+                tc::named_bar_sync(bar_id, 128);
+                // O and l both carry the factor alpha (P^ is alpha p quantized), so it cancels
+                const float oscale = FMT == BDFP4_NVFP4 ? a.v_gscale[hk] : 1.0f;
+                const int ch = chan;
+    #pragma unroll
+                for (int g = 0; g < HG; ++g) {
+                    const int hh = gb + g;
+                    const float l = rl[hh * 8] + rl[hh * 8 + 1] + rl[hh * 8 + 2] + rl[hh * 8 + 3];
+                    const int64_t row = row_of(hh);
+                    if (nspl == 1) {
+                        a.out[row * C::DV + ch] =
+                            __float2bfloat16(l > 0.0f ? __uint_as_float(o_fin[g]) * oscale / l : 0.0f);
+                    } else {
+                        // DYN: splits end in different units; the partials leave in the units of p
+                        const float un = DYN ? pow2f(-e_run[DYN ? g : 0]) : 1.0f;
+                        a.ws_o[(row * a.max_splits + split) * C::DV + ch] = __uint_as_float(o_fin[g]) * oscale * un;
+                        if (chan == 0) {
+                            a.ws_ml[(row * a.max_splits + split) * 2 + 0] = m_run[g];
+                            a.ws_ml[(row * a.max_splits + split) * 2 + 1] = l * un;
+                        }
                     }
                 }
             }
-        }
+        };
+        if (C::NSG == 1 || warp < 4) softmax_role(std::integral_constant<int, 0>{});
+        else softmax_role(std::integral_constant<int, (C::NSG > 1 ? 1 : 0)>{});
     }
 
     tc::tc_fence_before();

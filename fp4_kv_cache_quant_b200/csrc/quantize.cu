@@ -31,12 +31,13 @@ __global__ void __launch_bounds__(256, FMT == BDFP4_NVFP4 ? 3 : 2) quantize_k_ke
                           smooth, k_gscale, k_weight, k_pages, k_scales, flags);
 }
 
-// One thread per (token, head, group of VC channels: 8 for NVFP4, 4 for MXFP4);
-// only the first token of each run within a beta-slot block does work (see
-// bdfp4_quantize_kv in bdfp4.h), for the whole block of its VC channels.  A
-// warp covers whole (token, head) rows, so its threads are leaders or not
-// together; a leader loads its beta tokens' channels with one 16- or 8-byte
-// load per token.
+// One thread per (range of beta tokens, head, group of VC channels: 8 for
+// NVFP4, 4 for MXFP4): for each token of its range that leads a run within a
+// beta-slot block (see bdfp4_quantize_kv in bdfp4.h; usually the range's first
+// token) it quantizes the block of its VC channels, loading the run's tokens
+// with one 16- or 8-byte load each.  A warp covers whole (range, head) rows, so
+// its threads find the same leaders; a thread per token would leave 15 of 16
+// CTAs with nothing to do but start and exit.
 template <int FMT>
 struct VAppend {
     static constexpr int B = Fmt<FMT>::beta;
@@ -55,16 +56,19 @@ __global__ void __launch_bounds__(256) quantize_v_kernel(const __nv_bfloat16* __
     const int64_t gid = (int64_t)blockIdx.x * 256 + threadIdx.x;
     const int64_t row = gid / GPR;
     const int c0 = (int)(gid % GPR) * VC;
-    if (row >= (int64_t)T * H_kv) return;
-    const int t = (int)(row / H_kv), h = (int)(row % H_kv);
-    // two rounds of independent loads: this token's and its predecessor's slot
-    // ids (the leader test), then the next B - 1 slot ids with the B rows a run can cover
+    const int64_t nranges = ((int64_t)T + B - 1) / B;
+    if (row >= nranges * H_kv) return;
+    const int t0 = (int)(row / H_kv) * B, h = (int)(row % H_kv);
+    const int t1 = t0 + B < T ? t0 + B : T;
+    int64_t sm_prev = t0 > 0 ? __ldg(slot_mapping + t0 - 1) : -2;
+    for (int t = t0; t < t1; ++t) {
     const int64_t sm = __ldg(slot_mapping + t);
-    const int64_t sm_prev = t > 0 ? __ldg(slot_mapping + t - 1) : -2;
-    if (sm < 0 || sm >= num_pages * kPageSlots) return;  // bad slots are reported by the K kernel
+    const int64_t smp = sm_prev;
+    sm_prev = sm;
+    if (sm < 0 || sm >= num_pages * kPageSlots) continue;  // bad slots are reported by the K kernel
     const int slot = (int)(sm % kPageSlots);
-    const bool leader = (slot % B == 0) || t == 0 || sm_prev != sm - 1;
-    if (!leader) return;
+    const bool leader = (slot % B == 0) || t == 0 || smp != sm - 1;
+    if (!leader) continue;
     int64_t sm_next[B - 1];
 #pragma unroll
     for (int i = 1; i < B; ++i) sm_next[i - 1] = t + i < T ? __ldg(slot_mapping + t + i) : -2;
@@ -121,6 +125,7 @@ __global__ void __launch_bounds__(256) quantize_v_kernel(const __nv_bfloat16* __
             *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
         }
         vs[v_scale_offset<B>(c0 + cc, first / B)] = (uint8_t)code;
+    }
     }
 }
 
@@ -375,7 +380,7 @@ static void launch_quantize_kv(const void* k, const void* v, const int64_t* slot
     quantize_k_kernel<FMT, DK><<<(unsigned)kblocks, 256, 0, st>>>(
         (const __nv_bfloat16*)k, slot_mapping, T, H_kv, kv->smooth, kv->k_gscale, kv->k_weight, (uint8_t*)k_pages,
         (uint8_t*)k_scales, num_pages, flags, dev_status);
-    const int64_t vthreads = rows * (DV / VAppend<FMT>::VC);
+    const int64_t vthreads = ((int64_t)T + Fmt<FMT>::beta - 1) / Fmt<FMT>::beta * H_kv * (DV / VAppend<FMT>::VC);
     quantize_v_kernel<FMT, DV><<<(unsigned)((vthreads + 255) / 256), 256, 0, st>>>(
         (const __nv_bfloat16*)v, slot_mapping, T, H_kv, kv->v_gscale, (uint8_t*)v_pages, (uint8_t*)v_scales,
         num_pages);
@@ -454,9 +459,9 @@ extern "C" int bdfp4_quantize_v(const void* v, const int64_t* slot_mapping, int 
     if (fmt == BDFP4_NVFP4 && !kv->v_gscale) return BDFP4_ERR_ARG;
     if (!aligned(v, 16) || !aligned(v_pages, 128) || !aligned(v_scales, 128)) return BDFP4_ERR_ALIGN;
     cudaStream_t st = (cudaStream_t)stream;
-    const int64_t rows = (int64_t)T * H_kv;
     auto launch = [&](auto kernel, int groups_per_row) {
-        const int64_t threads = rows * groups_per_row;
+        const int beta = fmt == BDFP4_NVFP4 ? 16 : 32;
+        const int64_t threads = ((int64_t)T + beta - 1) / beta * H_kv * groups_per_row;
         kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>((const __nv_bfloat16*)v, slot_mapping, T, H_kv,
                                                                  kv->v_gscale, (uint8_t*)v_pages, (uint8_t*)v_scales,
                                                                  num_pages);
