@@ -1,22 +1,30 @@
 // decode_mla_tc.cu -- FP4 paged decode attention on the sm_100a tensor cores for
 // latent-KV (MLA) shapes: d_k = 576 (512-d latent + 64-d rope), d_v = 512 (the
 // latent), many query heads over one KV head (BitDecoding-FP4, Article Summary:
-// stacked query MMA on paged KV caches, transposed softmax with fused probability
-// quantization, dual-residual query, underflow-aware probability scaling; the
-// method is evaluated on GQA and MLA models).
+// stacked query MMA on paged KV caches, fused probability quantization,
+// dual-residual query, underflow-aware probability scaling; the method is
+// evaluated on GQA and MLA models).
 //
 // One CTA per (sequence, KV head, slice of GH <= 64 query heads, split), one
-// CTA per SM.  TMEM (512 columns) holds
-//   S^T [128 tokens][GH heads]         q1.k and q2.k accumulate into the same cells,
+// CTA per SM.  The query operand stacks the slice's dual-residual halves as
+// rows: row 2h holds q1 and row 2h + 1 holds q2 of head h.  TMEM (512 columns)
+// holds
+//   S [128 rows][128 tokens]           one QK MMA chain per tile (M = 128, N = 128),
 //   O^T [512 channels = 4 x 128 lanes][GH heads], accumulated across the tiles,
 //   and the scale factors of every MMA operand.
-// O stays in TMEM: when a head's running maximum rises, the softmax warps that
-// own the head rescale its O columns after the previous tile's PV completed and
-// before this tile's PV is issued -- the online-softmax update, in place.
-//   warps 0 .. 4 NSG - 1   softmax: group g owns heads 16 g .. 16 g + 15, its warp q
-//                          the tokens (TMEM lanes) 32 q .. 32 q + 31
-//   warp  4 NSG            producer: K and V pages by bulk copy, K scales by cp.async
-//   warp  4 NSG + 1        MMA issuer (one lane) and TMEM owner
+// A softmax lane owns one stacked row: its lane pair (q1, q2 of one head) adds
+// the two halves over 16 tokens each, so a 16-token probability block (the
+// NVFP4 block) is one lane's, and the 32-token MXFP4 block one lane pair's.
+// O stays in TMEM: when a head's running maximum rises, every softmax warp
+// rescales the head's O^T columns in its own lane quadrant and M tile, after
+// the previous tile's PV completed and before this tile's PV is issued -- the
+// online-softmax update, in place.
+//   warps 0 .. 15   softmax: warp w reads S lane quadrant w % 4 (heads
+//                   16 (w % 4) .. +15, when the slice has them) over tokens
+//                   32 (w / 4) .. +31 of each tile, and rescales and writes out
+//                   O^T M tile w / 4 of that lane quadrant
+//   warp  16        producer: K and V pages by bulk copy, K scales by cp.async
+//   warp  17        MMA issuer (one lane) and TMEM owner
 // Every wait is bounded; a timeout sets BDFP4_DEV_TIMEOUT and the CTA unwinds.
 
 #include <type_traits>
@@ -43,9 +51,9 @@ struct MlaCfg {
     static constexpr int NKG = (NBLK + 3) / 4;         // 4-block key scale groups per token
     static constexpr int KPG = MX ? 2 : 1;             // K steps per key scale group
     static constexpr int MT = DV / 128;                // 128-channel M tiles of O^T
-    static constexpr int HG = 16;                      // heads per softmax group
-    static constexpr int NSG = GH / HG;                // softmax groups
-    static constexpr int NSW = 4 * NSG;                // softmax warps
+    static constexpr int ROWS = 2 * GH;                // stacked query rows (q1, q2 of each head)
+    static constexpr int NQ = GH / 16;                 // S lane quadrants holding rows
+    static constexpr int NSW = 16;                     // softmax warps
     static constexpr int PRODUCER = NSW, MMA_WARP = NSW + 1;
     static constexpr int THREADS = 32 * (NSW + 2);
     static constexpr int NSK = 2, NSV = 2;             // K and V ring stages
@@ -57,54 +65,55 @@ struct MlaCfg {
     static constexpr int SPB = kPageSlots / B;         // token blocks per page
     static constexpr int SBO = DK / 32 * 128;          // 8-row group stride of the K and query operands
     // K stage: the two pages (MMA rows 0-63, 64-127), then per scale group the
-    // 32 x 16-byte tcgen05.cp source (row i: rows i, 32 + i, 64 + i, 96 + i)
+    // 32 x 16-byte tcgen05.cp source (row i: tokens i, 32 + i, 64 + i, 96 + i)
     static constexpr int OFF_KS = 2 * K_PAGE;
     static constexpr int KSTAGE = OFF_KS + NKG * 512;
     // V stage: the two pages, then their scale blocks
     static constexpr int OFF_VS = 2 * V_PAGE;
     static constexpr int VSTAGE = OFF_VS + 2 * VS_PAGE;
-    // query image: q1 and q2 operands [GH rows][DK] in K-major core blocks, their
-    // scale codes [2][GH][NBLK], the logit scales [GH] (fp32)
-    static constexpr int Q_OP = GH * DK / 2;
-    static constexpr int QSC = GH * NBLK;
-    static constexpr int QPACK = 2 * Q_OP + 2 * QSC + GH * 4;
+    // query image: the stacked operand [ROWS][DK] in K-major core blocks, its scale codes
+    // [ROWS][NBLK], the logit scales [GH] (fp32).  Shared memory holds the operand at its
+    // full 128 rows (rows past ROWS zero) and the codes and logit scales apart.
+    static constexpr int Q_OP = 128 * DK / 2;
+    static constexpr int QOP_IMG = ROWS * DK / 2;
+    static constexpr int QSC = ROWS * NBLK;
+    static constexpr int QMETA = QSC + GH * 4;
+    static constexpr int QPACK = QOP_IMG + QMETA;
     static constexpr int P_PAGE = GH / 8 * 256;        // P^T operand of one page: GH rows x 64 tokens
     static constexpr int P_BUF = 2 * P_PAGE;
-    static constexpr int RED_BUF = GH * 8;             // floats: [GH][4 quadrants][2 half warps]
     // shared memory map
     static constexpr int SM_KST = 0;
     static constexpr int SM_VST = SM_KST + NSK * KSTAGE;
     static constexpr int SM_Q = SM_VST + NSV * VSTAGE;
-    static constexpr int SM_P = (SM_Q + QPACK + 127) / 128 * 128;
-    static constexpr int SM_PSF = SM_P + 2 * P_BUF;    // [2 buf][2 page][32 rows][16 B] P scales
-    static constexpr int SM_RED = SM_PSF + 2 * 2 * 512;
-    // per softmax warp and head of its group: the tile's softmax terms for the warp's two
-    // token blocks {logit scale, exponent base, correction, 1 / block scale} x 2, the two
-    // block-scale codes, and an output scale
-    static constexpr int WST_WARP = HG * 32 + HG * 4 + HG * 4;
-    static constexpr int SM_WST = SM_RED + 2 * RED_BUF * 4;
-    static constexpr int SM_BARS = SM_WST + NSW * WST_WARP;
-    static constexpr int NBARS = 2 * NSK + 2 * NSV + 8;
+    static constexpr int SM_QM = SM_Q + Q_OP;
+    static constexpr int SM_P = (SM_QM + QMETA + 127) / 128 * 128;
+    static constexpr int SM_PSF = SM_P + 2 * P_BUF;       // [2 buf][2 page][32 rows][16 B] P scales
+    static constexpr int SM_VSF = SM_PSF + 2 * 2 * 512;   // MXFP4: [2 buf][MT][32 rows][16 B] V scales
+    static constexpr int SM_RED = SM_VSF + (MX ? 2 * MT * 512 : 0);   // [2][GH][4 quarters] tile maxima
+    static constexpr int SM_LRED = SM_RED + 2 * GH * 4 * 4;          // [GH][4 quarters] l partials
+    static constexpr int SM_COR = SM_LRED + GH * 4 * 4;              // [2][GH] corrections
+    static constexpr int SM_RISE = SM_COR + 2 * GH * 4;              // [2][4 quadrants] risen-head masks
+    static constexpr int SM_HEAD = SM_RISE + 2 * 4 * 4;              // [GH] output scales
+    static constexpr int SM_BARS = SM_HEAD + GH * 4;
+    static constexpr int NBARS = 2 * NSK + 2 * NSV + 10;
     static constexpr int SM_MISC = SM_BARS + NBARS * 8;   // tmem slot, abort flags
     static constexpr int SM_PFLAG = SM_MISC + 32;   // [64] page flags of the split's tiles, any-bad
     static constexpr int SMEM = SM_PFLAG + 64 + 16;
     // TMEM column map
-    static constexpr int T_S = 0;
-    static constexpr int T_O = GH;                     // M tile t at T_O + t GH
-    static constexpr int T_SFK = (T_O + MT * GH + 3) / 4 * 4;   // 2 buffers x NKG groups x 4
-    static constexpr int T_SFQ = T_SFK + 2 * NKG * 4;           // 2 operands x KS steps x 4
-    static constexpr int NSFV = MX ? 2 : 1;                     // V scale-factor buffers
-    static constexpr int T_SFV = T_SFQ + 2 * KS * 4;            // NSFV x MT tiles x 2 pages x 4
-    static constexpr int T_SFP = T_SFV + NSFV * MT * 8;         // 2 buffers x 2 pages x 4
+    static constexpr int T_S = 0;                      // 128 columns (tokens)
+    static constexpr int T_O = 128;                    // M tile t at T_O + t GH
+    static constexpr int T_SFK = (T_O + MT * GH + 3) / 4 * 4;   // NKG groups x 4
+    static constexpr int T_SFQ = T_SFK + NKG * 4;               // KS steps x 4
+    static constexpr int T_SFV = T_SFQ + KS * 4;                // NVFP4: MT tiles x 2 pages x 4; MXFP4: MT x 4
+    static constexpr int T_SFP = T_SFV + MT * (MX ? 4 : 8);     // 2 buffers x 2 pages x 4
     static constexpr int T_USED = T_SFP + 16;
     static constexpr int T_ALLOC = 512;
-    static_assert(GH % HG == 0 && GH <= 64, "head slice");
+    static_assert(GH % 16 == 0 && GH <= 64, "head slice");
     static_assert(T_USED <= T_ALLOC, "TMEM budget");
     static_assert(SMEM <= 232448 && SMEM > 232448 / 2, "one CTA per SM");
-    static_assert(QPACK % 16 == 0, "query image copied in 16-byte units");
+    static_assert(QOP_IMG % 16 == 0 && QMETA % 16 == 0, "query image copied in 16-byte units");
     // the image of a head slice fits the workspace region reserved for its heads
     static_assert(QPACK <= kQueryImageBytes * GH, "query image larger than its workspace share");
-    static_assert(NSG + 2 <= 16, "named barriers");
 };
 
 // ---------------------------------------------------------------- query image
@@ -148,14 +157,15 @@ __device__ __forceinline__ void mla_query_rows(const DecodeArgs& a, int img, int
 #pragma unroll
     for (int o = 0; o < 2; ++o) {
         const uint32_t* pk = o ? p2 : p1;
-        uint8_t* dst = im + o * C::Q_OP + (r >> 3) * C::SBO + (e0 >> 5) * 128 + (r & 7) * 16 + (e0 & 31) / 2;
+        const int sr = 2 * r + o;   // stacked row: q1 of head r at 2r, q2 at 2r + 1
+        uint8_t* dst = im + (sr >> 3) * C::SBO + (e0 >> 5) * 128 + (sr & 7) * 16 + (e0 & 31) / 2;
         if constexpr (B == 16) *reinterpret_cast<uint2*>(dst) = make_uint2(pk[0], pk[1]);
         else *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-        im[2 * C::Q_OP + o * C::QSC + r * C::NBLK + j] = (uint8_t)(o ? c2 : c1);
+        im[C::QOP_IMG + sr * C::NBLK + j] = (uint8_t)(o ? c2 : c1);
     }
     if (j == 0) {
         const float gk = FMT == BDFP4_NVFP4 ? a.k_gscale[hk] : 1.0f;
-        reinterpret_cast<float*>(im + 2 * C::Q_OP + 2 * C::QSC)[r] = a.sm_scale * gq * gk * kLog2e;
+        reinterpret_cast<float*>(im + C::QOP_IMG + C::QSC)[r] = a.sm_scale * gq * gk * kLog2e;
     }
 }
 
@@ -194,6 +204,7 @@ __global__ void __launch_bounds__(256) prep_mla_kernel(const DecodeArgs a, const
     mla_query_rows<FMT, GH>(a, img, hk * G + hs * GH + r0, r0);
 }
 
+
 // ---------------------------------------------------------------- decode
 // DYN (NVFP4): the probability pre-scale alpha = 2^E per tile and head; a head's
 // O^T and l are held in units of its current tile's alpha, so a change of E joins
@@ -204,26 +215,30 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
     // the split merge (a programmatic dependent) may be scheduled as CTAs of this grid retire
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     constexpr bool MX = C::MX;
-    constexpr int B = C::B, HG = C::HG, MT = C::MT;
+    constexpr int B = C::B, MT = C::MT;
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t* q_op = smem + C::SM_Q;
-    const uint8_t* qsc = q_op + 2 * C::Q_OP;
-    const float* lsc = reinterpret_cast<const float*>(q_op + 2 * C::Q_OP + 2 * C::QSC);
+    const uint8_t* qsc = smem + C::SM_QM;
+    const float* lsc = reinterpret_cast<const float*>(smem + C::SM_QM + C::QSC);
     uint8_t* p_op = smem + C::SM_P;
     uint8_t* psf = smem + C::SM_PSF;
     float* red = reinterpret_cast<float*>(smem + C::SM_RED);
-    uint8_t* wst = smem + C::SM_WST;
+    float* lred = reinterpret_cast<float*>(smem + C::SM_LRED);
+    float* cor = reinterpret_cast<float*>(smem + C::SM_COR);
+    uint32_t* rise = reinterpret_cast<uint32_t*>(smem + C::SM_RISE);
+    float* hscale = reinterpret_cast<float*>(smem + C::SM_HEAD);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SM_BARS);
     uint64_t* kfull = bars;                   // [NSK] K tile landed -> MMA
     uint64_t* kempty = kfull + C::NSK;        // [NSK] QK done -> producer
     uint64_t* vfull = kempty + C::NSK;        // [NSV] V tile landed -> MMA, softmax
     uint64_t* vempty = vfull + C::NSV;        // [NSV] PV done -> producer
     uint64_t* s_full = vempty + C::NSV;       // QK done -> softmax
-    uint64_t* s_free = s_full + 1;            // S read by every softmax warp -> MMA
-    uint64_t* p_ready = s_free + 1;           // [2] P, its scales and O rescaled -> MMA
+    uint64_t* s_free = s_full + 1;            // S read by every row-owning softmax warp -> MMA
+    uint64_t* p_ready = s_free + 1;           // [2] P, its scales, V scales and O rescaled -> MMA
     uint64_t* o_done = p_ready + 2;           // [2] PV done -> softmax (rescale, epilogue), MMA
     uint64_t* q_ready = o_done + 2;           // query operand and its scale factors -> MMA
     uint64_t* q_full = q_ready + 1;           // query image landed -> softmax
+    uint64_t* c_ready = q_full + 1;           // [2] the tile's corrections and risen heads posted -> softmax
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SM_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::SM_MISC + 4);
 
@@ -260,13 +275,15 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
             tc::mbar_init(&vempty[s], 1);
         }
         tc::mbar_init(s_full, 1);
-        tc::mbar_init(s_free, C::NSW);
+        tc::mbar_init(s_free, 4 * C::NQ);
         tc::mbar_init(&p_ready[0], C::NSW);
         tc::mbar_init(&p_ready[1], C::NSW);
         tc::mbar_init(&o_done[0], 1);
         tc::mbar_init(&o_done[1], 1);
         tc::mbar_init(q_ready, C::NSW);
         tc::mbar_init(q_full, 1);
+        tc::mbar_init(&c_ready[0], C::NQ);
+        tc::mbar_init(&c_ready[1], C::NQ);
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
@@ -285,6 +302,7 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
         // block-table reads of 32 tiles at a time, one per lane, as in the d = 128 kernel)
         bool ok = true;
         int pv0 = -1, pv1 = -1;
+        int k_last = -1, v_last = -1;   // the last tiles whose K / V halves were announced
         for (int j0 = 0; ok && j0 <= n; j0 += 32) {
             int pg_l[2] = {-1, -1};
             if (j0 + lane < n) {
@@ -334,6 +352,7 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
                             tc::cp_async_8(stg + C::OFF_KS + kg * 512 + lane * 16 + p * 8, ksrc + kg * 256);
                     }
                     tc::cp_async_mbar_arrive_noinc(&kfull[ks]);
+                    k_last = k;
                 }
                 if (do_v) {
                     if (lane == 0) {
@@ -357,51 +376,76 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
                                              C::VS_PAGE, &vfull[vsi]);
                         }
                     }
+                    v_last = v;
                 }
                 pv0 = pg0;
                 pv1 = pg1;
             }
         }
         if (!ok && lane == 0) *abort_flag = 1;
+        // Unwinding: before the CTA can exit, every copy this warp started must have landed.
+        // Each stage's last announced phase completes once its bytes (and the lanes' cp.async
+        // arrivals) are in; announced tiles run consecutively from the first.
+        if (!ok || *abort_flag) {
+            if (lane == 0) {
+                for (int s = 0; s < C::NSK; ++s) {
+                    if (k_last < s) continue;
+                    const int t = k_last - (k_last - s) % C::NSK;
+                    tc::mbar_wait_drain(&kfull[s], (t / C::NSK) & 1, kWaitLimitMla);
+                }
+                for (int s = 0; s < C::NSV; ++s) {
+                    if (v_last < s) continue;
+                    const int t = v_last - (v_last - s) % C::NSV;
+                    tc::mbar_wait_drain(&vfull[s], (t / C::NSV) & 1, kWaitLimitMla);
+                }
+            }
+            __syncwarp();
+        }
     } else if (warp == C::MMA_WARP) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc = tc::idesc_fp4(GH, MX);
+            constexpr uint32_t idesc_qk = tc::idesc_fp4(128, MX);
+            constexpr uint32_t idesc_pv = tc::idesc_fp4(GH, MX);
             const uint32_t q_addr = tc::smem_u32(q_op);
             const uint32_t p_addr = tc::smem_u32(p_op);
             const uint32_t kst_addr = tc::smem_u32(smem + C::SM_KST);
             const uint32_t vst_addr = tc::smem_u32(smem + C::SM_VST);
             const uint32_t psf_addr = tc::smem_u32(psf);
+            const uint32_t vsf_addr = tc::smem_u32(smem + C::SM_VSF);
+            uint64_t* last_bar = nullptr;   // the barrier of the last commit, and its phase
+            uint32_t last_par = 0;
+            // Descriptors and TMEM addresses are formed once; a K step, scale group or page moves
+            // a shared-memory descriptor by its byte offset / 16 (the address field), so each
+            // tcgen05 instruction costs the issuing lane an add or two.  The lane shares its
+            // sub-partition's issue slots with four softmax warps.
+            const uint64_t qdesc = tc::smem_desc(q_addr, 128, C::SBO);
+            const uint32_t t_s = tbase + C::T_S, t_o = tbase + C::T_O, t_sfk = tbase + C::T_SFK;
+            const uint32_t t_sfq = tbase + C::T_SFQ, t_sfv = tbase + C::T_SFV, t_sfp = tbase + C::T_SFP;
             auto issue_qk = [&](int j) -> bool {
-                const int s = j % C::NSK, buf = j & 1;
+                const int s = j % C::NSK;
                 if (!tc::mbar_wait(&kfull[s], (j / C::NSK) & 1, abort_flag, kWaitLimitMla)) return false;
                 tc::tc_fence_after();
                 // the scale rows came through cp.async (generic proxy); tcgen05.cp reads them
-                // through the async proxy
+                // through the async proxy.  One TMEM buffer: the previous QK completed before
+                // every softmax warp could read its S, which this issue waited for.
                 tc::fence_proxy_async_smem();
                 const uint32_t kt = kst_addr + s * C::KSTAGE;
+                const uint64_t kdesc = tc::smem_desc(kt, 128, C::SBO);
+                const uint64_t sdesc = tc::smem_desc(kt + C::OFF_KS, 128, 128);
 #pragma unroll
-                for (int kg = 0; kg < C::NKG; ++kg)
-                    tc::tmem_cp_32x128b_x4(tbase + C::T_SFK + (buf * C::NKG + kg) * 4,
-                                           tc::smem_desc(kt + C::OFF_KS + kg * 512, 128, 128));
-                // S^T = K (q1 + q2)^T: the q2 products accumulate onto the q1 ones (loops kept
-                // rolled: one lane issues them, and unrolled descriptors cost registers
-                // every warp of the CTA is sized for)
-#pragma unroll 1
-                for (int o = 0; o < 2; ++o) {
-#pragma unroll 1
-                    for (int ks = 0; ks < C::KS; ++ks) {
-                        // MXFP4 packs two K steps per key scale column: byte offset 2 for the odd step
-                        const uint32_t sfid = (uint32_t)(ks % C::KPG) * 2u;
-                        tc::mma_fp4<MX>(tbase + C::T_S, tc::smem_desc(kt + ks * 256, 128, C::SBO),
-                                        tc::smem_desc(q_addr + o * C::Q_OP + ks * 256, 128, C::SBO),
-                                        idesc | (sfid << 29),
-                                        (tbase + C::T_SFK + (buf * C::NKG + ks / C::KPG) * 4) | (sfid << 30),
-                                        tbase + C::T_SFQ + (o * C::KS + ks) * 4, (o > 0 || ks > 0) ? 1u : 0u);
-                    }
+                for (int kg = 0; kg < C::NKG; ++kg) tc::tmem_cp_32x128b_x4(t_sfk + kg * 4, sdesc + (uint64_t)(kg * 32));
+                // S = Q_stacked K^T: rows are (head, residual half), columns the tile's tokens
+#pragma unroll
+                for (int ks = 0; ks < C::KS; ++ks) {
+                    // MXFP4 packs two K steps per key scale column: byte offset 2 for the odd step
+                    const uint32_t sfid = (uint32_t)(ks % C::KPG) * 2u;
+                    tc::mma_fp4<MX>(t_s, qdesc + (uint64_t)(ks * 16), kdesc + (uint64_t)(ks * 16), idesc_qk | (sfid << 4),
+                                    t_sfq + ks * 4, (t_sfk + (ks / C::KPG) * 4) | (sfid << 30), ks > 0 ? 1u : 0u);
                 }
                 tc::mma_commit(s_full);
                 tc::mma_commit(&kempty[s]);   // the K stage is free once QK has read it
+                last_bar = &kempty[s];
+                last_par = (uint32_t)(j / C::NSK) & 1u;
                 return true;
             };
             bool ok = tc::mbar_wait(q_ready, 0, abort_flag, kWaitLimitMla);
@@ -417,52 +461,70 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
                 const int s = j % C::NSV, pb = j & 1;
                 if (!(ok = tc::mbar_wait(&p_ready[pb], (j >> 1) & 1, abort_flag, kWaitLimitMla))) break;
                 if (!(ok = tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, kWaitLimitMla))) break;
-                // NVFP4 V scale factors have one TMEM buffer: the previous PV must have read it
-                if (!MX && j > 0 && !(ok = tc::mbar_wait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag,
-                                                         kWaitLimitMla)))
+                // the V scale factors have one TMEM buffer: the previous PV must have read it
+                if (j > 0 && !(ok = tc::mbar_wait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, kWaitLimitMla)))
                     break;
                 tc::tc_fence_after();
                 const uint32_t vt = vst_addr + s * C::VSTAGE;
+                const uint64_t psd = tc::smem_desc(psf_addr + pb * 1024, 128, 128);
 #pragma unroll
-                for (int p = 0; p < 2; ++p)
-                    tc::tmem_cp_32x128b_x4(tbase + C::T_SFP + (pb * 2 + p) * 4,
-                                           tc::smem_desc(psf_addr + (pb * 2 + p) * 512, 128, 128));
+                for (int p = 0; p < 2; ++p) tc::tmem_cp_32x128b_x4(t_sfp + (pb * 2 + p) * 4, psd + (uint64_t)(p * 32));
                 if constexpr (!MX) {
                     // each M tile's scale block of a page is already the 32 x 16-byte copy source
+                    const uint64_t vsd = tc::smem_desc(vt + C::OFF_VS, 128, 128);
 #pragma unroll
                     for (int t = 0; t < MT; ++t)
 #pragma unroll
                         for (int p = 0; p < 2; ++p)
-                            tc::tmem_cp_32x128b_x4(tbase + C::T_SFV + t * 8 + p * 4,
-                                                   tc::smem_desc(vt + C::OFF_VS + p * C::VS_PAGE + t * C::VS_TILE,
-                                                                 128, 128));
+                            tc::tmem_cp_32x128b_x4(t_sfv + t * 8 + p * 4,
+                                                   vsd + (uint64_t)((p * C::VS_PAGE + t * C::VS_TILE) >> 4));
+                } else {
+                    // the two pages' blocks interleaved by the softmax warps (bytes 0-1 page 0, 2-3 page 1)
+                    const uint64_t vfd = tc::smem_desc(vsf_addr + pb * MT * 512, 128, 128);
+#pragma unroll
+                    for (int t = 0; t < MT; ++t) tc::tmem_cp_32x128b_x4(t_sfv + t * 4, vfd + (uint64_t)(t * 32));
                 }
-                const int vb = MX ? pb : 0;
-#pragma unroll 1
+                const uint64_t vd = tc::smem_desc(vt, 128, 256);
+                const uint64_t pd = tc::smem_desc(p_addr + pb * C::P_BUF, 128, 256);
+#pragma unroll
                 for (int t = 0; t < MT; ++t) {
 #pragma unroll
                     for (int p = 0; p < 2; ++p) {
-                        tc::mma_fp4<MX>(tbase + C::T_O + t * GH, tc::smem_desc(vt + p * C::V_PAGE + t * 4096, 128, 256),
-                                        tc::smem_desc(p_addr + pb * C::P_BUF + p * C::P_PAGE, 128, 256), idesc,
-                                        tbase + C::T_SFV + (vb * MT + t) * 8 + p * 4,
-                                        tbase + C::T_SFP + (pb * 2 + p) * 4, (j > 0 || p > 0) ? 1u : 0u);
+                        const uint32_t sfid = MX ? (uint32_t)p * 2u : 0u;
+                        const uint32_t sfa = MX ? (t_sfv + t * 4) | (sfid << 30) : t_sfv + t * 8 + p * 4;
+                        tc::mma_fp4<MX>(t_o + t * GH, vd + (uint64_t)((p * C::V_PAGE + t * 4096) >> 4),
+                                        pd + (uint64_t)((p * C::P_PAGE) >> 4), idesc_pv | (sfid << 29), sfa,
+                                        t_sfp + (pb * 2 + p) * 4, (j > 0 || p > 0) ? 1u : 0u);
                     }
                 }
                 tc::mma_commit(&o_done[j & 1]);
                 tc::mma_commit(&vempty[s]);
+                last_bar = &vempty[s];
+                last_par = (uint32_t)(j / C::NSV) & 1u;
             }
-            if (!ok) *abort_flag = 1;
+            if (!ok) {
+                *abort_flag = 1;
+                // unwinding: the tensor memory is freed below, so the MMAs and copies into it
+                // must have finished
+                if (last_bar) tc::mbar_wait_drain(last_bar, last_par, kWaitLimitMla);
+            }
         }
     } else {
         // ------------------------------------------------------------ softmax warps
-        const int grp = warp >> 2;                 // head group
-        const int qd = warp & 3;                   // TMEM lane quadrant = tokens 32 qd .. 32 qd + 31
-        const int gb = grp * HG;                   // first head of the group (within the CTA)
-        const int bar_id = 1 + grp;                // named barrier of the group (128 threads)
+        const int qd = warp & 3;                   // TMEM lane quadrant
+        const int t4 = warp >> 2;                  // token quarter of S; M tile of O^T
+        const bool rows_here = qd < C::NQ;         // the quadrant holds stacked query rows
+        const int odd = lane & 1;                  // 0: the q1 row, 1: the q2 row of the lane pair
+        const int h = 16 * qd + (lane >> 1);       // head (within the CTA) of the lane pair
         const uint32_t tq = tbase + ((uint32_t)(32 * qd) << 16);
         const float alpha = (FMT == BDFP4_NVFP4 && !(a.flags & BDFP4_FLAG_NO_UNDERFLOW)) ? kAlphaNV : 1.0f;
         bool bad = false;
-        bool grp_abort = false;   // the group's four warps gave up (alike in all of them)
+        bool grp_abort = false;   // the quadrant's four warps gave up (alike in all of them)
+        // a wait that gave up stops every role of the CTA
+        auto fail_wait = [&]() {
+            bad = true;
+            *abort_flag = 1;
+        };
 
         // Pages the block table gets wrong (the producer reports them and copies nothing) are
         // skipped like tokens past the end: their logits are masked and their V scales zeroed.
@@ -484,76 +546,68 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
             return r;
         };
         if (tid == 0) *pflag_bad = n > 64 ? 1 : 0;
-        tc::named_bar_sync(1 + C::NSG, 32 * C::NSW);
+        tc::named_bar_sync(5, 32 * C::NSW);
         if (tid < 64 && tid < n) {
             const uint32_t f = page_flags(tid);
             pflag[tid] = (uint8_t)f;
             if (f != 3u) *pflag_bad = 1;
         }
-        // the query image arrives in one bulk copy from the prologue grid, which this
-        // grid may overlap: griddepcontrol.wait holds the copy until its writes are visible
+        // the query image arrives in two bulk copies from the prologue grid, which this grid
+        // may overlap: griddepcontrol.wait holds the copies until its writes are visible
         if (tid == 0) {
             asm volatile("griddepcontrol.wait;" ::: "memory");
+            const uint8_t* im = a.qpack + (int64_t)img * C::QPACK;
             tc::mbar_arrive_expect_tx(q_full, C::QPACK);
-            tc::bulk_g2s(q_op, a.qpack + (int64_t)img * C::QPACK, C::QPACK, q_full);
+            tc::bulk_g2s(q_op, im, C::QOP_IMG, q_full);
+            tc::bulk_g2s(smem + C::SM_QM, im + C::QOP_IMG, C::QMETA, q_full);
         }
-        // the P scale-factor buffers: zero (columns past the heads must stay zero)
+        // the P scale-factor buffers: zero (rows past the heads must stay zero); operand rows
+        // past the slice's stacked rows: zero
         for (int i = tid; i < 2 * 2 * 512 / 16; i += 32 * C::NSW) reinterpret_cast<uint4*>(psf)[i] = make_uint4(0, 0, 0, 0);
-        if (!tc::mbar_wait(q_full, 0, abort_flag, kWaitLimitMla)) bad = true;
-        // query scale factors (SFB of QK): row n at lane n % 32, column n / 32 of each K step's chunk
-        if (grp == 0) {
+        for (int i = C::QOP_IMG / 16 + tid; i < C::Q_OP / 16; i += 32 * C::NSW)
+            reinterpret_cast<uint4*>(q_op)[i] = make_uint4(0, 0, 0, 0);
+        if (!tc::mbar_wait(q_full, 0, abort_flag, kWaitLimitMla)) fail_wait();
+        // query scale factors (SFA of QK): row r at lane r % 32, column r / 32 of each K step's
+        // chunk, in every lane quadrant
+        if (t4 == 0) {
+#pragma unroll 1
+            for (int ks = 0; ks < C::KS; ++ks) {
+                uint32_t v[4];
 #pragma unroll
-            for (int o = 0; o < 2; ++o) {
-#pragma unroll
-                for (int ks = 0; ks < C::KS; ++ks) {
-                    uint32_t v[2] = {0u, 0u};
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        const int r = 32 * c + lane;
-                        if (r < GH) {
-                            const uint8_t* q = qsc + o * C::QSC + r * C::NBLK;
-                            if constexpr (B == 16) v[c] = *reinterpret_cast<const uint32_t*>(q + ks * 4);
-                            else v[c] = (uint32_t)q[ks * 2] | ((uint32_t)q[ks * 2 + 1] << 8);
-                        }
+                for (int c = 0; c < 4; ++c) {
+                    const int r = 32 * c + lane;
+                    v[c] = 0u;
+                    if (r < C::ROWS) {
+                        const uint8_t* q = qsc + r * C::NBLK;
+                        if constexpr (B == 16) v[c] = *reinterpret_cast<const uint32_t*>(q + ks * 4);
+                        else v[c] = (uint32_t)q[ks * 2] | ((uint32_t)q[ks * 2 + 1] << 8);
                     }
-                    tc::tmem_st4(tq + C::T_SFQ + (o * C::KS + ks) * 4, v[0], v[1], 0u, 0u);
                 }
+                tc::tmem_st4(tq + C::T_SFQ + ks * 4, v[0], v[1], v[2], v[3]);
             }
             tc::tmem_wait_st();
         }
         tc::tc_fence_before();
         tc::fence_proxy_async_smem();
-        tc::named_bar_sync(1 + C::NSG, 32 * C::NSW);   // psf zeroed and page flags set before any tile
+        tc::named_bar_sync(5, 32 * C::NSW);   // psf and operand padding zeroed, page flags set before any tile
         const bool any_bad_page = *pflag_bad != 0;
         if (lane == 0) tc::mbar_arrive(q_ready);
 
-        // Running maxima (scaled log2 units) are kept one head per lane: lane g of every warp
-        // of the group tracks head gb + g and posts, per tile, the terms every lane of the
-        // warp needs for that head to the warp's own shared-memory slots.
-        float4* const wterm = reinterpret_cast<float4*>(wst + warp * C::WST_WARP);   // [HG][2 blocks]
-        uint32_t* const wcode = reinterpret_cast<uint32_t*>(wst + warp * C::WST_WARP + HG * 32);   // [HG]
-        float* const wout = reinterpret_cast<float*>(wst + warp * C::WST_WARP + HG * 36);          // [HG]
-        float m_lane = -INFINITY;                   // running maximum of head gb + lane
-        int e_lane = 11;                            // DYN: log2 of head gb + lane's current pre-scale
-        const float ls_lane = lane < HG ? lsc[gb + lane] : 0.0f;
-        float l_part[HG];
-#pragma unroll
-        for (int g = 0; g < HG; ++g) l_part[g] = 0.0f;
-        // TMEM lane 32 qd + lane holds token 32 qd + lane of the tile: slot 32 (qd % 2) + lane
-        // of page qd / 2
-        const int page_of_thread = qd >> 1;
-        const int pos_in_page = 32 * (qd & 1) + lane;
-        const int tok_in_tile = 32 * qd + lane;
+        // per-lane state: the running maximum of head h (scaled log2 units), l over the lane's
+        // tokens (in units of the current pre-scale), DYN: log2 of the head's current pre-scale
+        float m_run = -INFINITY, l_run = 0.0f;
+        int e_run = 11;
+        const float ls = rows_here ? lsc[h] : 0.0f;   // logit scale of head h
         // log2 of alpha: alpha * 2^(x - m) is evaluated as 2^(x - (m - log2 alpha))
         const float la = alpha == kAlphaNV ? 11.0f : 0.0f;
-        const bool lo_half = lane < 16;
-        // P^T operand bytes: a lane pair (tokens 2i, 2i + 1) fills one byte of each head
-        // row; per pair of heads the even lane writes the first, the odd lane the second
-        const int hsel = lane & 1;
-        const uint32_t psel = (lane & 1) ? 0x0004u : 0x0040u;   // byte 0 <- token 2i, byte 1 <- token 2i + 1
-        const bool sfstore = (lane & (B - 1)) < 2;             // first two lanes of a token block
-        uint8_t* const pbyte = p_op + page_of_thread * C::P_PAGE + (qd & 1) * 128 + (lane >> 1);
-        uint8_t* const sfbase = psf + page_of_thread * 512 + pos_in_page / B;
+        // the lane's 16 tokens: page t4 / 2 of the tile, slots 32 (t4 % 2) + 16 odd ..
+        const int page_of_lane = t4 >> 1;
+        const int tok_in_tile = 32 * t4 + 16 * odd;
+        // P^T operand bytes of the lane (head h, its 16 tokens: 8 bytes of the row's 16-byte K
+        // chunk t4 % 2) and its block-scale byte (NVFP4: block 2 (t4 % 2) + odd of the page;
+        // MXFP4: block t4 % 2, the lane pair's)
+        const int p_off = page_of_lane * C::P_PAGE + (h >> 3) * 256 + (t4 & 1) * 128 + (h & 7) * 16 + 8 * odd;
+        const int sf_off = page_of_lane * 512 + (h & 31) * 16 + (h >> 5) * 4 + (MX ? (t4 & 1) : 2 * (t4 & 1) + odd);
 
         // The tile loop, in two copies: the page checks exist only in the copy a split with a
         // bad page runs, so the normal copy carries no extra live registers.
@@ -566,185 +620,186 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
                     pok0 = (f & 1u) != 0;
                     pok1 = (f & 2u) != 0;
                 }
-                if (!tc::mbar_wait(s_full, j & 1, abort_flag, kWaitLimitMla)) bad = true;
-                tc::tc_fence_after();
-                uint32_t sr[HG];
-                tc::tmem_ld<HG>(tq + C::T_S + gb, sr);
-                tc::tmem_wait_ld();
-                // S may be overwritten by the next QK once every softmax warp has it in registers
-                tc::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(s_free);
-                const int token = tile * kTileTokens + tok_in_tile;
-                const bool valid = token < N && (page_of_thread ? pok1 : pok0);
-                // raw logits (q1 + q2).k; maxima over each half warp (16 consecutive slots)
-                float* rw = red + (j & 1) * C::RED_BUF;
-    #pragma unroll
-                for (int g = 0; g < HG; ++g) {
-                    const float x = valid ? __uint_as_float(sr[g]) : -INFINITY;
-                    const float lo = tc::redux_max_f32(lo_half ? x : -INFINITY, 0xffffffffu);
-                    const float hi = tc::redux_max_f32(lo_half ? -INFINITY : x, 0xffffffffu);
-                    if (lane == 0) *reinterpret_cast<float2*>(rw + ((gb + g) * 4 + qd) * 2) = make_float2(lo, hi);
-                }
-                // one decision for the group's four warps, taken by the barrier itself (a role
-                // that gave up leaves a wait here unfinished, and the wait sees its abort flag)
-                if (tc::named_bar_or(bar_id, 128, bad)) {
-                    grp_abort = true;
-                    break;
-                }
-                // new running maxima, one head per lane, and the scales of the warp's two token
-                // blocks: the block maximum of alpha p is 2^(x_b ls - base) for the block's largest
-                // logit x_b, so the scale is the one the block's largest member picks
-                bool rose = false;
-                if (lane < HG) {
-                    const float* w = rw + (gb + lane) * 8;
-                    const float4 w0 = *reinterpret_cast<const float4*>(w);
-                    const float4 w1 = *reinterpret_cast<const float4*>(w + 4);
-                    const float mt = fmaxf(fmaxf(fmaxf(w0.x, w0.y), fmaxf(w0.z, w0.w)),
-                                           fmaxf(fmaxf(w1.x, w1.y), fmaxf(w1.z, w1.w)));
-                    const float mn = fmaxf(m_lane, mt * ls_lane);
+                const int jb = j & 1;
+                if (rows_here) {
+                    if (!tc::mbar_wait(s_full, j & 1, abort_flag, kWaitLimitMla)) fail_wait();
+                    tc::tc_fence_after();
+                    uint32_t sv[32];
+                    tc::tmem_ld<32>(tq + C::T_S + 32 * t4, sv);
+                    tc::tmem_wait_ld();
+                    // S may be overwritten by the next QK once every row-owning warp has it in registers
+                    tc::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(s_free);
+                    // (q1 + q2).k over the lane's 16 tokens: the pair's even lane keeps the first
+                    // 16 of the quarter, the odd lane the last 16, each adding its partner's row
+                    float x[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float lo = __uint_as_float(sv[i]), hi = __uint_as_float(sv[16 + i]);
+                        const float give = odd ? lo : hi;
+                        x[i] = (odd ? hi : lo) + __shfl_xor_sync(0xffffffffu, give, 1);
+                    }
+                    const int tok0 = tile * kTileTokens + tok_in_tile;
+                    if (decltype(masked)::value || tok0 + 16 > N) {
+                        int nv = N - tok0;
+                        nv = nv < 0 ? 0 : (nv > 16 ? 16 : nv);
+                        if (!(page_of_lane ? pok1 : pok0)) nv = 0;
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) x[i] = i < nv ? x[i] : -INFINITY;
+                    }
+                    // block maximum (raw logits; the logit scale is positive), then the quarter's
+                    // maximum of the head over the lane pair, posted for the quadrant's warps
+                    float bm = x[0];
+#pragma unroll
+                    for (int i = 1; i < 16; ++i) bm = fmaxf(bm, x[i]);
+                    const float pm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
+                    float* rw = red + jb * GH * 4;
+                    if (!odd) rw[h * 4 + t4] = pm;
+                    // one decision for the quadrant's four warps, taken by the barrier itself (a
+                    // role that gave up leaves a wait unfinished, and the wait sees its abort flag)
+                    if (tc::named_bar_or(1 + qd, 128, bad)) {
+                        grp_abort = true;
+                        *abort_flag = 1;
+                        break;
+                    }
+                    const float4 w4 = *reinterpret_cast<const float4*>(rw + h * 4);
+                    const float mt = fmaxf(fmaxf(w4.x, w4.y), fmaxf(w4.z, w4.w));
+                    const float mn = fmaxf(m_run, mt * ls);
                     const float mz = mn == -INFINITY ? 0.0f : mn;
-                    float corr = tc::ex2_approx(m_lane - mz);   // 0 on the split's first tile
+                    float corr = tc::ex2_approx(m_run - mz);   // 0 on the split's first tile
                     float base = mz - la;
-                    rose = mn != m_lane;
-                    m_lane = mn;
+                    bool rose = mn != m_run;
+                    m_run = mn;
                     if constexpr (DYN) {
                         // this tile's pre-scale from its largest probability; O^T and l move to
                         // its units (an exact power of two, folded into corr)
-                        const int e = dynamic_alpha_exp(tc::ex2_approx(fmaf(mt, ls_lane, -mz)));
-                        corr *= pow2f(e - e_lane);
-                        rose |= e != e_lane;
-                        e_lane = e;
+                        const int e = dynamic_alpha_exp(tc::ex2_approx(fmaf(mt, ls, -mz)));
+                        corr *= pow2f(e - e_run);
+                        rose |= e != e_run;
+                        e_run = e;
                         base = mz - (float)e;
                     }
-                    const float bm_lo = w[qd * 2], bm_hi = w[qd * 2 + 1];
-                    // per block: NVFP4 {ls, base, corr, 1 / scale}, the element is alpha p / scale;
-                    // MXFP4 {ls, base + e, corr, 2^e} for the scale 2^e, the element is 2^(x ls - base - e)
-                    // (the exponent's argument stays small, as the OCP rule's element) and p its 2^e multiple
-                    float r_lo, r_hi, b_lo = base, b_hi = base;
-                    uint32_t codes;
+                    // the quadrant's corrections and risen heads, for every softmax warp's O^T rescale
+                    const uint32_t rb = __ballot_sync(0xffffffffu, rose) & 0x55555555u;
+                    if (t4 == 0) {
+                        if (!odd) cor[jb * GH + h] = rose ? corr : 1.0f;
+                        if (lane == 0) rise[jb * 4 + qd] = rb;
+                        __syncwarp();
+                        if (lane == 0) tc::mbar_arrive(&c_ready[jb]);
+                    }
+                    // probabilities and their FP4 quantization: NVFP4 one 16-token block per lane
+                    // with the E4M3 scale of its largest alpha p; MXFP4 one 32-token block per lane
+                    // pair, the OCP MX shared exponent taken in the log domain (the block maximum
+                    // is 2^d with d = x_b ls - m <= 0, so floor(log2) = floor(d)) and the element
+                    // 2^(x ls - m - (c - 127)), p its 2^(c - 127) multiple
+                    float rinv, eb;
+                    uint32_t code;
                     if constexpr (!MX) {
-                        const float a_lo = tc::ex2_approx(fmaf(bm_lo, ls_lane, -base));
-                        const float a_hi = tc::ex2_approx(fmaf(bm_hi, ls_lane, -base));
-                        codes = tc::e4m3x2_encode(__fmul_rn(a_lo, 1.0f / 6.0f), __fmul_rn(a_hi, 1.0f / 6.0f));
-                        const float2 sg = tc::e4m3x2_value(codes);
+                        const float ab = tc::ex2_approx(fmaf(bm, ls, -base));
+                        code = tc::e4m3x2_encode(__fmul_rn(ab, 1.0f / 6.0f), 0.0f) & 0xffu;
                         // a zero scale zeroes the whole block inside the MMA, whatever the element codes
-                        r_lo = tc::rcp_approx(sg.x);
-                        r_hi = tc::rcp_approx(sg.y);
+                        rinv = tc::rcp_approx(tc::e4m3x2_value(code).x);
+                        eb = base;
                     } else {
-                        // one 32-token block per warp; the OCP MX shared exponent in the log domain:
-                        // the block maximum is 2^d with d = x_b ls - m <= 0, so floor(log2) = floor(d)
-                        // and the element is p 2^(127 - c) for the E8M0 code c
-                        const float d = __fsub_rn(__fmul_rn(fmaxf(bm_lo, bm_hi), ls_lane), mz);
+                        const float d = __fsub_rn(__fmul_rn(pm, ls), mz);
                         const int c = max(__float2int_rd(fmaxf(d, -256.0f)) + 125, 0);
-                        codes = (uint32_t)c | ((uint32_t)c << 8);
-                        b_lo = b_hi = mz + (float)(c - 127);
-                        r_lo = r_hi = __uint_as_float(c > 0 ? (uint32_t)c << 23 : 0x00400000u);   // 2^(c - 127)
+                        code = (uint32_t)c;
+                        eb = base + (float)(c - 127);   // base = m here (alpha = 1)
+                        rinv = __uint_as_float(c > 0 ? (uint32_t)c << 23 : 0x00400000u);   // 2^(c - 127)
                     }
-                    wterm[lane * 2 + 0] = make_float4(ls_lane, b_lo, corr, r_lo);
-                    wterm[lane * 2 + 1] = make_float4(ls_lane, b_hi, corr, r_hi);
-                    wcode[lane] = codes;
-                }
-                const uint32_t rmask = j > 0 ? __ballot_sync(0xffffffffu, rose) : 0u;
-                __syncwarp();
-                // O^T rescale of the heads whose maximum rose, once the previous tile's PV has
-                // completed; the group's warps decide alike, having read the same maxima
-                if (rmask) {
-                    if (!tc::mbar_wait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, kWaitLimitMla)) bad = true;
-                    tc::tc_fence_after();
-                    uint32_t rem = rmask;
-                    while (rem) {
-                        // up to four heads per round trip: their columns in the four M tiles
-                        int hs_[4];
-                        uint32_t ov[4][MT];
-    #pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            hs_[k] = rem ? __ffs(rem) - 1 : -1;
-                            if (rem) rem &= rem - 1;
-                            if (hs_[k] >= 0) {
-    #pragma unroll
-                                for (int t = 0; t < MT; ++t) tc::tmem_ld<1>(tq + C::T_O + t * GH + gb + hs_[k], &ov[k][t]);
-                            }
-                        }
-                        tc::tmem_wait_ld();
-    #pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            if (hs_[k] < 0) continue;
-                            const float c = wterm[hs_[k] * 2].z;
-    #pragma unroll
-                            for (int t = 0; t < MT; ++t)
-                                tc::tmem_st1(tq + C::T_O + t * GH + gb + hs_[k], __float_as_uint(__uint_as_float(ov[k][t]) * c));
+                    float lsum = 0.0f;
+                    uint32_t pk[2] = {0u, 0u};
+#pragma unroll
+                    for (int i = 0; i < 16; i += 2) {
+                        const float e0 = tc::ex2_approx(fmaf(x[i], ls, -eb));   // 0 for masked tokens
+                        const float e1 = tc::ex2_approx(fmaf(x[i + 1], ls, -eb));
+                        if constexpr (!MX) {
+                            lsum += e0 + e1;   // alpha p
+                            pk[i / 8] |= e2m1x2_encode(e0 * rinv, e1 * rinv) << (4 * (i % 8));
+                        } else {
+                            lsum += (e0 + e1) * rinv;   // p
+                            pk[i / 8] |= e2m1x2_encode(e0, e1) << (4 * (i % 8));
                         }
                     }
-                    tc::tmem_wait_st();
+                    l_run = fmaf(l_run, corr, lsum);
+                    *reinterpret_cast<uint2*>(p_op + jb * C::P_BUF + p_off) = make_uint2(pk[0], pk[1]);
+                    if (MX ? !odd : true) psf[jb * 1024 + sf_off] = (uint8_t)code;
                 }
-                // probabilities and their FP4 quantization, two heads per conversion
-                uint8_t* const pb = pbyte + (j & 1) * C::P_BUF;
-                uint8_t* const sfb = sfbase + (j & 1) * 2 * 512;
-                const int half = lo_half ? 0 : 1;
-    #pragma unroll
-                for (int g = 0; g < HG; g += 2) {
-                    float q[2];
-    #pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const float4 v = wterm[(g + u) * 2 + half];
-                        const float x = valid ? __uint_as_float(sr[g + u]) : -INFINITY;
-                        const float e = tc::ex2_approx(fmaf(x, v.x, -v.y));   // 0 for masked tokens
-                        const float y = MX ? e * v.w : e;                     // alpha p
-                        l_part[g + u] = fmaf(l_part[g + u], v.z, y);          // l in units of alpha
-                        q[u] = MX ? e : e * v.w;
-                    }
-                    const uint32_t mine = e2m1x2_encode(q[0], q[1]);   // head g in bits 0..3, head g + 1 in 4..7
-                    const uint32_t other = __shfl_xor_sync(0xffffffffu, mine, 1);
-                    const uint32_t wv = __byte_perm(mine, other, psel) >> (4 * hsel);
-                    const int hr = gb + g + hsel;
-                    pb[(hr >> 3) * 256 + (hr & 7) * 16] = (uint8_t)((wv & 0xfu) | ((wv >> 4) & 0xf0u));
-                    if (sfstore) sfb[(hr & 31) * 16 + (hr >> 5) * 4] = (uint8_t)(wcode[g + hsel] >> (8 * half));
-                }
-                // V scale factors (group 0): blocks past the sequence end are zeroed (NVFP4, in the
-                // stage before its TMEM copy) or masked (MXFP4, stored into TMEM by these warps)
-                if (grp == 0) {
+                // V scale factors (warps of the first token quarter, lane quadrant qd: channels
+                // 32 qd .. +31 of each M tile): blocks past the sequence end or in a bad page
+                // are zeroed in the stage before its TMEM copy (NVFP4) or in the interleaved
+                // rows these warps build (MXFP4)
+                if (t4 == 0) {
                     const int s = j % C::NSV;
-                    const bool tail = (tile + 1) * kTileTokens > N;
                     uint8_t* vs = smem + C::SM_VST + s * C::VSTAGE + C::OFF_VS;
                     if constexpr (!MX) {
-                        if (tail || !pok0 || !pok1) {
-                            if (!tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, kWaitLimitMla)) bad = true;
-    #pragma unroll
+                        if ((tile + 1) * kTileTokens > N || !pok0 || !pok1) {
+                            if (!tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, kWaitLimitMla)) fail_wait();
+#pragma unroll
                             for (int p = 0; p < 2; ++p) {
                                 const int t0 = tile * kTileTokens + p * kPageSlots;
                                 int nvb = (N - t0 + B - 1) / B;
                                 nvb = nvb < 0 ? 0 : (nvb > C::SPB ? C::SPB : nvb);
                                 if (!(p ? pok1 : pok0)) nvb = 0;
                                 for (int bb = nvb; bb < C::SPB; ++bb)
-    #pragma unroll
+#pragma unroll
                                     for (int t = 0; t < MT; ++t)
                                         vs[p * C::VS_PAGE + t * C::VS_TILE + lane * 16 + qd * 4 + bb] = 0;
                             }
                         }
                     } else {
-                        if (!tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, kWaitLimitMla)) bad = true;
-                        uint32_t mask[2];
-    #pragma unroll
+                        if (!tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, kWaitLimitMla)) fail_wait();
+                        uint32_t msk[2];
+#pragma unroll
                         for (int p = 0; p < 2; ++p) {
                             const int t0 = tile * kTileTokens + p * kPageSlots;
                             int nvb = (N - t0 + B - 1) / B;
                             nvb = nvb < 0 ? 0 : (nvb > C::SPB ? C::SPB : nvb);
                             if (!(p ? pok1 : pok0)) nvb = 0;
-                            mask[p] = nvb >= 2 ? 0xffffu : ((1u << (8 * nvb)) - 1u);
+                            const uint32_t m16 = nvb >= 2 ? 0xffffu : ((1u << (8 * nvb)) - 1u);
+                            msk[p] = m16 | (m16 << 16);
                         }
-    #pragma unroll
-                        for (int t = 0; t < MT; ++t) {
-                            uint32_t v[8];
-    #pragma unroll
-                            for (int p = 0; p < 2; ++p) {
-                                const uint2 w = *reinterpret_cast<const uint2*>(vs + p * C::VS_PAGE + t * C::VS_TILE + 8 * lane);
-                                v[p * 4 + 0] = w.x & mask[p];
-                                v[p * 4 + 1] = (w.x >> 16) & mask[p];
-                                v[p * 4 + 2] = w.y & mask[p];
-                                v[p * 4 + 3] = (w.y >> 16) & mask[p];
+                        // M tile qd: lane i's 8 bytes of each page are channels 4 i .. 4 i + 3 of
+                        // the tile's copy rows; the row interleaves page 0's two blocks (bytes
+                        // 0-1) with page 1's (bytes 2-3)
+                        const uint2 w0 = *reinterpret_cast<const uint2*>(vs + qd * C::VS_TILE + 8 * lane);
+                        const uint2 w1 = *reinterpret_cast<const uint2*>(vs + C::VS_PAGE + qd * C::VS_TILE + 8 * lane);
+                        const uint32_t x0 = w0.x & msk[0], x1 = w0.y & msk[0], y0 = w1.x & msk[1], y1 = w1.y & msk[1];
+                        *reinterpret_cast<uint4*>(smem + C::SM_VSF + (jb * MT + qd) * 512 + 16 * lane) =
+                            make_uint4(__byte_perm(x0, y0, 0x5410), __byte_perm(x0, y0, 0x7632),
+                                       __byte_perm(x1, y1, 0x5410), __byte_perm(x1, y1, 0x7632));
+                    }
+                }
+                // O^T rescale of the heads whose maximum rose (any quadrant's), once the previous
+                // tile's PV has completed: this warp's lane quadrant of M tile t4
+                if (!tc::mbar_wait(&c_ready[jb], (j >> 1) & 1, abort_flag, kWaitLimitMla)) fail_wait();
+                if (j > 0) {
+                    uint32_t any = 0u;
+#pragma unroll
+                    for (int g = 0; g < C::NQ; ++g) any |= rise[jb * 4 + g];
+                    if (any) {
+                        if (!tc::mbar_wait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, kWaitLimitMla)) fail_wait();
+                        tc::tc_fence_after();
+                        const uint32_t ob = tq + C::T_O + t4 * GH;
+                        // per quadrant with a risen head: its 16 head columns in one round trip,
+                        // the heads that did not rise multiplied by exactly 1
+#pragma unroll 1
+                        for (int g = 0; g < C::NQ; ++g) {
+                            if (!rise[jb * 4 + g]) continue;
+                            uint32_t ov[16];
+                            tc::tmem_ld<16>(ob + 16 * g, ov);
+                            const float4* cg = reinterpret_cast<const float4*>(cor + jb * GH + 16 * g);
+                            tc::tmem_wait_ld();
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                const float4 c4 = cg[k];
+                                ov[4 * k + 0] = __float_as_uint(__uint_as_float(ov[4 * k + 0]) * c4.x);
+                                ov[4 * k + 1] = __float_as_uint(__uint_as_float(ov[4 * k + 1]) * c4.y);
+                                ov[4 * k + 2] = __float_as_uint(__uint_as_float(ov[4 * k + 2]) * c4.z);
+                                ov[4 * k + 3] = __float_as_uint(__uint_as_float(ov[4 * k + 3]) * c4.w);
                             }
-                            tc::tmem_st8(tq + C::T_SFV + ((j & 1) * MT + t) * 8, v);
+                            tc::tmem_st16(ob + 16 * g, ov);
                         }
                         tc::tmem_wait_st();
                     }
@@ -752,55 +807,53 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
                 tc::tc_fence_before();
                 tc::fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&p_ready[j & 1]);
+                if (lane == 0) tc::mbar_arrive(&p_ready[jb]);
+                // a warp without rows takes part in no barrier of the loop: it stops here
+                if (!rows_here && bad) break;
             }
         };
         if (any_bad_page) tiles(std::true_type{});
         else tiles(std::false_type{});
-        if (!grp_abort) {
-            if (!tc::mbar_wait(&o_done[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag, kWaitLimitMla)) bad = true;
+        if (!grp_abort && !bad) {
+            if (!tc::mbar_wait(&o_done[(n - 1) & 1], ((n - 1) >> 1) & 1, abort_flag, kWaitLimitMla)) fail_wait();
             tc::tc_fence_after();
         }
 
         // ------------------------------------------------------------ epilogue (thread = channel)
-        grp_abort = tc::named_bar_or(bar_id, 128, grp_abort || bad || *abort_flag);
-        if (grp_abort) *abort_flag = 1;
-        if (!grp_abort) {
-            float* rl = red;   // [GH][4] partial sums (the tile maxima are no longer read)
-#pragma unroll
-            for (int g = 0; g < HG; ++g) {
-                float v = l_part[g];
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-                if (lane == 0) rl[(gb + g) * 4 + qd] = v;
+        const bool fail = tc::named_bar_or(5, 32 * C::NSW, grp_abort || bad || *abort_flag);
+        if (fail) {
+            if (tid == 0) *abort_flag = 1;
+        } else {
+            if (rows_here) {
+                const float l2 = l_run + __shfl_xor_sync(0xffffffffu, l_run, 1);
+                if (!odd) lred[h * 4 + t4] = l2;
             }
-            tc::named_bar_sync(bar_id, 128);
+            tc::named_bar_sync(5, 32 * C::NSW);
             // O and l both carry the factor alpha (P^ is alpha p quantized), so it cancels
             const float oscale = FMT == BDFP4_NVFP4 ? a.v_gscale[hk] : 1.0f;
-            // lane g: the output scale and (m, l) of head gb + g, through the warp's slots
-            if (lane < HG) {
-                const float4 r4 = *reinterpret_cast<const float4*>(rl + (gb + lane) * 4);
+            if (rows_here && t4 == 0 && !odd) {
+                const float4 r4 = *reinterpret_cast<const float4*>(lred + h * 4);
                 const float l = r4.x + r4.y + r4.z + r4.w;
                 // DYN: splits end in different units; the partials leave in the units of p
-                const float un = DYN ? pow2f(-e_lane) : 1.0f;
-                wout[lane] = nspl == 1 ? (l > 0.0f ? oscale / l : 0.0f) : oscale * un;
-                if (nspl > 1 && qd == 0) {
-                    const int64_t row = (int64_t)b * a.H_q + h0 + gb + lane;
-                    a.ws_ml[(row * a.max_splits + split) * 2 + 0] = m_lane;
+                const float un = DYN ? pow2f(-e_run) : 1.0f;
+                hscale[h] = nspl == 1 ? (l > 0.0f ? oscale / l : 0.0f) : oscale * un;
+                if (nspl > 1) {
+                    const int64_t row = (int64_t)b * a.H_q + h0 + h;
+                    a.ws_ml[(row * a.max_splits + split) * 2 + 0] = m_run;
                     a.ws_ml[(row * a.max_splits + split) * 2 + 1] = l * un;
                 }
             }
-            __syncwarp();
+            tc::named_bar_sync(5, 32 * C::NSW);
+            const int chan = t4 * 128 + 32 * qd + lane;
 #pragma unroll 1
-            for (int t = 0; t < MT; ++t) {
-                uint32_t ov[HG];
-                tc::tmem_ld<HG>(tq + C::T_O + t * GH + gb, ov);
+            for (int c0 = 0; c0 < GH; c0 += 16) {
+                uint32_t ov[16];
+                tc::tmem_ld<16>(tq + C::T_O + t4 * GH + c0, ov);
                 tc::tmem_wait_ld();
-                const int chan = t * 128 + 32 * qd + lane;
 #pragma unroll
-                for (int g = 0; g < HG; ++g) {
-                    const int64_t row = (int64_t)b * a.H_q + h0 + gb + g;
-                    const float o = __uint_as_float(ov[g]) * wout[g];
+                for (int g = 0; g < 16; ++g) {
+                    const int64_t row = (int64_t)b * a.H_q + h0 + c0 + g;
+                    const float o = __uint_as_float(ov[g]) * hscale[c0 + g];
                     if (nspl == 1) a.out[row * C::DV + chan] = __float2bfloat16(o);
                     else a.ws_o[(row * a.max_splits + split) * C::DV + chan] = o;
                 }
