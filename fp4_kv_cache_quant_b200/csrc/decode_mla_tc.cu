@@ -88,8 +88,7 @@ struct MlaCfg {
     static constexpr int SM_QM = SM_Q + Q_OP;
     static constexpr int SM_P = (SM_QM + QMETA + 127) / 128 * 128;
     static constexpr int SM_PSF = SM_P + 2 * P_BUF;       // [2 buf][2 page][32 rows][16 B] P scales
-    static constexpr int SM_VSF = SM_PSF + 2 * 2 * 512;   // MXFP4: [2 buf][MT][32 rows][16 B] V scales
-    static constexpr int SM_RED = SM_VSF + (MX ? 2 * MT * 512 : 0);   // [2][GH][4 quarters] tile maxima
+    static constexpr int SM_RED = SM_PSF + 2 * 2 * 512;              // [2][GH][4 quarters] tile maxima
     static constexpr int SM_LRED = SM_RED + 2 * GH * 4 * 4;          // [GH][4 quarters] l partials
     static constexpr int SM_COR = SM_LRED + GH * 4 * 4;              // [2][GH] corrections
     static constexpr int SM_RISE = SM_COR + 2 * GH * 4;              // [2][4 quadrants] risen-head masks
@@ -233,7 +232,7 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
     uint64_t* vfull = kempty + C::NSK;        // [NSV] V tile landed -> MMA, softmax
     uint64_t* vempty = vfull + C::NSV;        // [NSV] PV done -> producer
     uint64_t* s_full = vempty + C::NSV;       // QK done -> softmax
-    uint64_t* s_free = s_full + 1;            // S read by every row-owning softmax warp -> MMA
+    uint64_t* s_free = s_full + 1;            // S read, the next tile's key scale factors stored -> MMA
     uint64_t* p_ready = s_free + 1;           // [2] P, its scales, V scales and O rescaled -> MMA
     uint64_t* o_done = p_ready + 2;           // [2] PV done -> softmax (rescale, epilogue), MMA
     uint64_t* q_ready = o_done + 2;           // query operand and its scale factors -> MMA
@@ -275,7 +274,7 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
             tc::mbar_init(&vempty[s], 1);
         }
         tc::mbar_init(s_full, 1);
-        tc::mbar_init(s_free, 4 * C::NQ);
+        tc::mbar_init(s_free, 3 * C::NQ + 4);   // row-owning warps, and second-quarter warps without rows
         tc::mbar_init(&p_ready[0], C::NSW);
         tc::mbar_init(&p_ready[1], C::NSW);
         tc::mbar_init(&o_done[0], 1);
@@ -411,7 +410,6 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
             const uint32_t kst_addr = tc::smem_u32(smem + C::SM_KST);
             const uint32_t vst_addr = tc::smem_u32(smem + C::SM_VST);
             const uint32_t psf_addr = tc::smem_u32(psf);
-            const uint32_t vsf_addr = tc::smem_u32(smem + C::SM_VSF);
             uint64_t* last_bar = nullptr;   // the barrier of the last commit, and its phase
             uint32_t last_par = 0;
             // Descriptors and TMEM addresses are formed once; a K step, scale group or page moves
@@ -425,15 +423,10 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
                 const int s = j % C::NSK;
                 if (!tc::mbar_wait(&kfull[s], (j / C::NSK) & 1, abort_flag, kWaitLimitMla)) return false;
                 tc::tc_fence_after();
-                // the scale rows came through cp.async (generic proxy); tcgen05.cp reads them
-                // through the async proxy.  One TMEM buffer: the previous QK completed before
-                // every softmax warp could read its S, which this issue waited for.
-                tc::fence_proxy_async_smem();
+                // the tile's key scale factors are in TMEM already: the softmax warps of the second
+                // token quarter stored them before their arrival on s_free (or on q_ready)
                 const uint32_t kt = kst_addr + s * C::KSTAGE;
                 const uint64_t kdesc = tc::smem_desc(kt, 128, C::SBO);
-                const uint64_t sdesc = tc::smem_desc(kt + C::OFF_KS, 128, 128);
-#pragma unroll
-                for (int kg = 0; kg < C::NKG; ++kg) tc::tmem_cp_32x128b_x4(t_sfk + kg * 4, sdesc + (uint64_t)(kg * 32));
                 // S = Q_stacked K^T: rows are (head, residual half), columns the tile's tokens
 #pragma unroll
                 for (int ks = 0; ks < C::KS; ++ks) {
@@ -461,29 +454,12 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
                 const int s = j % C::NSV, pb = j & 1;
                 if (!(ok = tc::mbar_wait(&p_ready[pb], (j >> 1) & 1, abort_flag, kWaitLimitMla))) break;
                 if (!(ok = tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, kWaitLimitMla))) break;
-                // the V scale factors have one TMEM buffer: the previous PV must have read it
-                if (j > 0 && !(ok = tc::mbar_wait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, kWaitLimitMla)))
-                    break;
                 tc::tc_fence_after();
                 const uint32_t vt = vst_addr + s * C::VSTAGE;
                 const uint64_t psd = tc::smem_desc(psf_addr + pb * 1024, 128, 128);
 #pragma unroll
                 for (int p = 0; p < 2; ++p) tc::tmem_cp_32x128b_x4(t_sfp + (pb * 2 + p) * 4, psd + (uint64_t)(p * 32));
-                if constexpr (!MX) {
-                    // each M tile's scale block of a page is already the 32 x 16-byte copy source
-                    const uint64_t vsd = tc::smem_desc(vt + C::OFF_VS, 128, 128);
-#pragma unroll
-                    for (int t = 0; t < MT; ++t)
-#pragma unroll
-                        for (int p = 0; p < 2; ++p)
-                            tc::tmem_cp_32x128b_x4(t_sfv + t * 8 + p * 4,
-                                                   vsd + (uint64_t)((p * C::VS_PAGE + t * C::VS_TILE) >> 4));
-                } else {
-                    // the two pages' blocks interleaved by the softmax warps (bytes 0-1 page 0, 2-3 page 1)
-                    const uint64_t vfd = tc::smem_desc(vsf_addr + pb * MT * 512, 128, 128);
-#pragma unroll
-                    for (int t = 0; t < MT; ++t) tc::tmem_cp_32x128b_x4(t_sfv + t * 4, vfd + (uint64_t)(t * 32));
-                }
+                // the V scale factors were stored by the softmax warps of the first token quarter
                 const uint64_t vd = tc::smem_desc(vt, 128, 256);
                 const uint64_t pd = tc::smem_desc(p_addr + pb * C::P_BUF, 128, 256);
 #pragma unroll
@@ -567,6 +543,22 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
         for (int i = C::QOP_IMG / 16 + tid; i < C::Q_OP / 16; i += 32 * C::NSW)
             reinterpret_cast<uint4*>(q_op)[i] = make_uint4(0, 0, 0, 0);
         if (!tc::mbar_wait(q_full, 0, abort_flag, kWaitLimitMla)) fail_wait();
+        // Key scale factors of tile jt (SFB of QK: token n at lane n % 32, column n / 32 of each
+        // group's chunk, in every lane quadrant), from the K stage into this warp's lane quadrant.
+        // The warps of the second token quarter store them once the tile's K stage landed and
+        // the previous QK, the buffer's only reader, completed.
+        auto write_sfk = [&](int jt) {
+            const int s = jt % C::NSK;
+            if (!tc::mbar_wait(&kfull[s], (jt / C::NSK) & 1, abort_flag, kWaitLimitMla)) fail_wait();
+            const uint8_t* src = smem + C::SM_KST + s * C::KSTAGE + C::OFF_KS + 16 * lane;
+#pragma unroll
+            for (int kg = 0; kg < C::NKG; ++kg) {
+                const uint4 w = *reinterpret_cast<const uint4*>(src + kg * 512);
+                tc::tmem_st4(tq + C::T_SFK + kg * 4, w.x, w.y, w.z, w.w);
+            }
+            tc::tmem_wait_st();
+        };
+        if (t4 == 1) write_sfk(0);
         // query scale factors (SFA of QK): row r at lane r % 32, column r / 32 of each K step's
         // chunk, in every lane quadrant
         if (t4 == 0) {
@@ -627,6 +619,7 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
                     uint32_t sv[32];
                     tc::tmem_ld<32>(tq + C::T_S + 32 * t4, sv);
                     tc::tmem_wait_ld();
+                    if (t4 == 1 && j + 1 < n) write_sfk(j + 1);
                     // S may be overwritten by the next QK once every row-owning warp has it in registers
                     tc::tc_fence_before();
                     __syncwarp();
@@ -725,51 +718,65 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
                     l_run = fmaf(l_run, corr, lsum);
                     *reinterpret_cast<uint2*>(p_op + jb * C::P_BUF + p_off) = make_uint2(pk[0], pk[1]);
                     if (MX ? !odd : true) psf[jb * 1024 + sf_off] = (uint8_t)code;
+                } else if (t4 == 1) {
+                    // a lane quadrant without rows: only the next tile's key scale factors
+                    if (!tc::mbar_wait(s_full, j & 1, abort_flag, kWaitLimitMla)) fail_wait();
+                    tc::tc_fence_after();
+                    if (j + 1 < n) write_sfk(j + 1);
+                    tc::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(s_free);
                 }
-                // V scale factors (warps of the first token quarter, lane quadrant qd: channels
-                // 32 qd .. +31 of each M tile): blocks past the sequence end or in a bad page
-                // are zeroed in the stage before its TMEM copy (NVFP4) or in the interleaved
-                // rows these warps build (MXFP4)
+                // V scale factors of the tile (SFA of PV: channel r of an M tile at lane r % 32,
+                // column r / 32 of its chunk, in every lane quadrant), stored by the warps of the
+                // first token quarter once the V stage landed and the previous PV, the buffer's
+                // reader, completed.  Blocks past the sequence end or in a bad page are zeroed.
+                // NVFP4: per M tile and page the stage holds the 32 x 16-byte rows as stored;
+                // MXFP4: a row interleaves page 0's two blocks (bytes 0-1) with page 1's (2-3).
                 if (t4 == 0) {
                     const int s = j % C::NSV;
-                    uint8_t* vs = smem + C::SM_VST + s * C::VSTAGE + C::OFF_VS;
-                    if constexpr (!MX) {
-                        if ((tile + 1) * kTileTokens > N || !pok0 || !pok1) {
-                            if (!tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, kWaitLimitMla)) fail_wait();
+                    if (!tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, kWaitLimitMla)) fail_wait();
+                    if (j > 0 && !tc::mbar_wait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, kWaitLimitMla))
+                        fail_wait();
+                    tc::tc_fence_after();
+                    const uint8_t* vs = smem + C::SM_VST + s * C::VSTAGE + C::OFF_VS;
+                    uint32_t msk[2];
 #pragma unroll
-                            for (int p = 0; p < 2; ++p) {
-                                const int t0 = tile * kTileTokens + p * kPageSlots;
-                                int nvb = (N - t0 + B - 1) / B;
-                                nvb = nvb < 0 ? 0 : (nvb > C::SPB ? C::SPB : nvb);
-                                if (!(p ? pok1 : pok0)) nvb = 0;
-                                for (int bb = nvb; bb < C::SPB; ++bb)
-#pragma unroll
-                                    for (int t = 0; t < MT; ++t)
-                                        vs[p * C::VS_PAGE + t * C::VS_TILE + lane * 16 + qd * 4 + bb] = 0;
-                            }
-                        }
-                    } else {
-                        if (!tc::mbar_wait(&vfull[s], (j / C::NSV) & 1, abort_flag, kWaitLimitMla)) fail_wait();
-                        uint32_t msk[2];
-#pragma unroll
-                        for (int p = 0; p < 2; ++p) {
-                            const int t0 = tile * kTileTokens + p * kPageSlots;
-                            int nvb = (N - t0 + B - 1) / B;
-                            nvb = nvb < 0 ? 0 : (nvb > C::SPB ? C::SPB : nvb);
-                            if (!(p ? pok1 : pok0)) nvb = 0;
+                    for (int p = 0; p < 2; ++p) {
+                        const int t0 = tile * kTileTokens + p * kPageSlots;
+                        int nvb = (N - t0 + B - 1) / B;
+                        nvb = nvb < 0 ? 0 : (nvb > C::SPB ? C::SPB : nvb);
+                        if (!(p ? pok1 : pok0)) nvb = 0;
+                        if constexpr (!MX) {
+                            msk[p] = nvb >= 4 ? 0xffffffffu : ((1u << (8 * nvb)) - 1u);
+                        } else {
                             const uint32_t m16 = nvb >= 2 ? 0xffffu : ((1u << (8 * nvb)) - 1u);
                             msk[p] = m16 | (m16 << 16);
                         }
-                        // M tile qd: lane i's 8 bytes of each page are channels 4 i .. 4 i + 3 of
-                        // the tile's copy rows; the row interleaves page 0's two blocks (bytes
-                        // 0-1) with page 1's (bytes 2-3)
-                        const uint2 w0 = *reinterpret_cast<const uint2*>(vs + qd * C::VS_TILE + 8 * lane);
-                        const uint2 w1 = *reinterpret_cast<const uint2*>(vs + C::VS_PAGE + qd * C::VS_TILE + 8 * lane);
-                        const uint32_t x0 = w0.x & msk[0], x1 = w0.y & msk[0], y0 = w1.x & msk[1], y1 = w1.y & msk[1];
-                        *reinterpret_cast<uint4*>(smem + C::SM_VSF + (jb * MT + qd) * 512 + 16 * lane) =
-                            make_uint4(__byte_perm(x0, y0, 0x5410), __byte_perm(x0, y0, 0x7632),
-                                       __byte_perm(x1, y1, 0x5410), __byte_perm(x1, y1, 0x7632));
                     }
+#pragma unroll
+                    for (int t = 0; t < MT; ++t) {
+                        if constexpr (!MX) {
+                            uint32_t w[8];
+#pragma unroll
+                            for (int p = 0; p < 2; ++p) {
+                                const uint4 x = *reinterpret_cast<const uint4*>(vs + p * C::VS_PAGE + t * C::VS_TILE + 16 * lane);
+                                w[4 * p + 0] = x.x & msk[p];
+                                w[4 * p + 1] = x.y & msk[p];
+                                w[4 * p + 2] = x.z & msk[p];
+                                w[4 * p + 3] = x.w & msk[p];
+                            }
+                            tc::tmem_st8(tq + C::T_SFV + t * 8, w);
+                        } else {
+                            // lane i's 8 bytes of each page are channels 4 i .. 4 i + 3 of the tile's rows
+                            const uint2 w0 = *reinterpret_cast<const uint2*>(vs + t * C::VS_TILE + 8 * lane);
+                            const uint2 w1 = *reinterpret_cast<const uint2*>(vs + C::VS_PAGE + t * C::VS_TILE + 8 * lane);
+                            const uint32_t x0 = w0.x & msk[0], x1 = w0.y & msk[0], y0 = w1.x & msk[1], y1 = w1.y & msk[1];
+                            tc::tmem_st4(tq + C::T_SFV + t * 4, __byte_perm(x0, y0, 0x5410), __byte_perm(x0, y0, 0x7632),
+                                         __byte_perm(x1, y1, 0x5410), __byte_perm(x1, y1, 0x7632));
+                        }
+                    }
+                    tc::tmem_wait_st();
                 }
                 // O^T rescale of the heads whose maximum rose (any quadrant's), once the previous
                 // tile's PV has completed: this warp's lane quadrant of M tile t4
