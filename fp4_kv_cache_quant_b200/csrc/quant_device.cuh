@@ -8,6 +8,36 @@
 
 namespace bdfp4 {
 
+// Packed fp32 pairs (sm_100 f32x2 instructions: each lane an IEEE fp32 operation, round
+// to nearest, subnormals kept) and an approximate reciprocal (the special-function unit,
+// relative error below 2^-22; subnormal inputs and results flushed to zero).
+using f32x2 = unsigned long long;
+__device__ __forceinline__ f32x2 f32x2_pack(float lo, float hi) {
+    f32x2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float2 f32x2_unpack(f32x2 v) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return make_float2(lo, hi);
+}
+__device__ __forceinline__ f32x2 f32x2_mul(f32x2 a, f32x2 b) {
+    f32x2 r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ f32x2 f32x2_fma(f32x2 a, f32x2 b, f32x2 c) {
+    f32x2 r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ float rcp_approx_ftz(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
 // Row geometry: threads per row (padded), active threads, segment split.
 template <int FMT, int DK>
 struct RowGeom {
@@ -48,7 +78,14 @@ __device__ __forceinline__ void transform_block(float* x, const float* smooth_ro
 #pragma unroll
     for (int i = 0; i < B; ++i) {
         float s = active ? __ldg(smooth_row + e0 + i) : 1.0f;
-        x[i] = IS_KEY ? __fdiv_rn(x[i], s) : __fmul_rn(x[i], s);
+        if constexpr (IS_KEY) {
+            // a power of two 2^k whose reciprocal is normal: x / 2^k and x * 2^-k round alike
+            const uint32_t u = __float_as_uint(s), e = (u >> 23) & 0xffu;
+            if ((u & 0x807fffffu) == 0u && e >= 1u && e <= 253u) x[i] = __fmul_rn(x[i], __uint_as_float((254u - e) << 23));
+            else x[i] = __fdiv_rn(x[i], s);
+        } else {
+            x[i] = __fmul_rn(x[i], s);
+        }
     }
     if (!hadamard) return;
     fwht_local<B>(x);
@@ -167,14 +204,16 @@ __device__ __forceinline__ int search_exact(const float* x, float g, const float
 // to the larger code.  An all-zero block keeps c0.  Returns the code; `packed`
 // gets its E2M1 codes.
 //
-// NVFP4 scores every candidate cheaply first: x times the rounded 1 / sigma
-// for the codes, the squared error in fp32.  Against the exact score (fp32 RN
-// division, fp64 sums) the cheap one moves an element's code only within a few
-// ulps of a rounding midpoint, where the two codes' errors agree to 1e-5
-// relative, and rounds the sum to about 1e-6 relative, so the exact winner
-// always scores within 2^-10 (relative) of the cheapest candidate.  Only those
-// candidates are scored exactly, in window order -- the same winner as scoring
-// all of them exactly.  A candidate whose 1 / sigma is not finite is always
+// NVFP4 scores every candidate cheaply first: x times an approximate 1 / sigma
+// (rcp.approx, relative error below 2^-22) for the codes, the squared error in
+// fp32, two elements per packed f32x2 instruction (two partial sums).  Against
+// the exact score (fp32 RN division, fp64 sums) the cheap one moves an
+// element's code only within a few ulps of a rounding midpoint, where the two
+// codes' errors agree to about 5e-5 relative, and rounds the sum to about 1e-6
+// relative, so the exact winner always scores within 2^-10 (relative) of the
+// cheapest candidate.  Only those candidates are scored exactly, in window
+// order -- the same winner as scoring all of them exactly.  A candidate whose
+// 1 / sigma is not finite (sigma zero or below the normal range) is always
 // scored exactly.
 template <int FMT, bool W>
 __device__ __forceinline__ uint32_t search_scale(const float* x, float g, const float* w, uint32_t* packed) {
@@ -204,20 +243,23 @@ __device__ __forceinline__ uint32_t search_scale(const float* x, float g, const 
             score[k] = INFINITY;
             if (c < lo) continue;
             const float sg = block_sigma<FMT>((uint32_t)c, g);
-            const float r = __frcp_rn(sg);
+            const float r = rcp_approx_ftz(sg);
             if (!(sg > 0.0f) || !(r < INFINITY)) {
                 force |= 1u << k;
                 continue;
             }
-            float e = 0.0f;
+            const f32x2 r2 = f32x2_pack(r, r), ns2 = f32x2_pack(-sg, -sg);
+            f32x2 e2 = f32x2_pack(0.0f, 0.0f);
 #pragma unroll
             for (int i = 0; i < B; i += 2) {
-                const float2 v = e2m1x2_value(e2m1x2_encode(x[i] * r, x[i + 1] * r));
-                const float d0 = fmaf(-v.x, sg, x[i]);
-                const float d1 = fmaf(-v.y, sg, x[i + 1]);
-                e = fmaf(W ? w[i] * d0 : d0, d0, e);
-                e = fmaf(W ? w[i + 1] * d1 : d1, d1, e);
+                const f32x2 xp = f32x2_pack(x[i], x[i + 1]);
+                const float2 y = f32x2_unpack(f32x2_mul(xp, r2));
+                const float2 v = e2m1x2_value(e2m1x2_encode(y.x, y.y));
+                const f32x2 dp = f32x2_fma(f32x2_pack(v.x, v.y), ns2, xp);   // x - v sigma
+                e2 = f32x2_fma(W ? f32x2_mul(f32x2_pack(w[i], w[i + 1]), dp) : dp, dp, e2);
             }
+            const float2 ep = f32x2_unpack(e2);
+            const float e = ep.x + ep.y;
             score[k] = e;
             best = fminf(best, e);
         }

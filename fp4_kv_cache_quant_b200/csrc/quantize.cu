@@ -20,7 +20,7 @@ namespace bdfp4 {
 
 // ---------------------------------------------------------------- KV append
 template <int FMT, int DK>
-__global__ void __launch_bounds__(256, FMT == BDFP4_NVFP4 ? 3 : 2) quantize_k_kernel(const __nv_bfloat16* __restrict__ k,
+__global__ void __launch_bounds__(256, FMT == BDFP4_NVFP4 ? 4 : 2) quantize_k_kernel(const __nv_bfloat16* __restrict__ k,
                                                          const int64_t* __restrict__ slot_mapping, int T, int H_kv,
                                                          const float* __restrict__ smooth,
                                                          const float* __restrict__ k_gscale,
