@@ -64,10 +64,25 @@ __device__ __forceinline__ uint32_t e2m1x2_encode(float lo, float hi) {
         "}\n"
         : "=r"(packed)
         : "f"(hi), "f"(lo));
-    return packed & 0xffu;
+    return packed;   // cvt.u32.u8 zero-extends
 }
 
 __device__ __forceinline__ uint32_t e2m1_encode(float x) { return e2m1x2_encode(x, 0.0f) & 0xfu; }
+
+// Eight fp32 values to E2M1 (nearest, ties to even, saturating at +-6, sign kept),
+// packed v[0] in bits 0..3 up to v[7] in bits 28..31 (the byte order of a K-major row).
+__device__ __forceinline__ uint32_t e2m1x8_encode(const float* v) {
+    uint32_t r;
+    asm("{\n .reg .b8 b0, b1, b2, b3;\n"
+        " cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n"
+        " cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n"
+        " cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n"
+        " cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n"
+        " mov.b32 %0, {b0, b1, b2, b3};\n}"
+        : "=r"(r)
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+    return r;
+}
 
 // Values of the E2M1 pair lo | hi << 4 (as e2m1x2_encode packs it) through the
 // hardware conversion: .x the low code's, .y the high code's (exact: E2M1 is a

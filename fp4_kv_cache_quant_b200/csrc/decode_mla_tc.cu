@@ -701,22 +701,23 @@ __global__ void __launch_bounds__(MlaCfg<FMT, GH>::THREADS, 1) decode_mla_tc_ker
                         eb = base + (float)(c - 127);   // base = m here (alpha = 1)
                         rinv = __uint_as_float(c > 0 ? (uint32_t)c << 23 : 0x00400000u);   // 2^(c - 127)
                     }
-                    float lsum = 0.0f;
-                    uint32_t pk[2] = {0u, 0u};
+                    float lsum = 0.0f, pq[16];
 #pragma unroll
                     for (int i = 0; i < 16; i += 2) {
                         const float e0 = tc::ex2_approx(fmaf(x[i], ls, -eb));   // 0 for masked tokens
                         const float e1 = tc::ex2_approx(fmaf(x[i + 1], ls, -eb));
                         if constexpr (!MX) {
                             lsum += e0 + e1;   // alpha p
-                            pk[i / 8] |= e2m1x2_encode(e0 * rinv, e1 * rinv) << (4 * (i % 8));
+                            pq[i] = e0 * rinv;
+                            pq[i + 1] = e1 * rinv;
                         } else {
                             lsum += (e0 + e1) * rinv;   // p
-                            pk[i / 8] |= e2m1x2_encode(e0, e1) << (4 * (i % 8));
+                            pq[i] = e0;
+                            pq[i + 1] = e1;
                         }
                     }
                     l_run = fmaf(l_run, corr, lsum);
-                    *reinterpret_cast<uint2*>(p_op + jb * C::P_BUF + p_off) = make_uint2(pk[0], pk[1]);
+                    *reinterpret_cast<uint2*>(p_op + jb * C::P_BUF + p_off) = make_uint2(e2m1x8_encode(pq), e2m1x8_encode(pq + 8));
                     if (MX ? !odd : true) psf[jb * 1024 + sf_off] = (uint8_t)code;
                 } else if (t4 == 1) {
                     // a lane quadrant without rows: only the next tile's key scale factors

@@ -648,15 +648,16 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
             tc::named_bar_sync(1 + C::NSG, 32 * C::NSW);   // psf zeroed and page flags set before any tile
             const bool any_bad_page = *pflag_bad != 0;
             if (lane == 0) tc::mbar_arrive(q_ready);
-            float m_run[HG], l_part[HG];
-            // DYN: log2 of each head's current pre-scale; O^T and l are held in its units
-            int e_run[DYN ? HG : 1];
+            // The running maximum of head gb + hl lives in the lanes hl, hl + HG, ... of each of the
+            // group's warps (hl = lane % HG); they compute the head's per-tile terms once, and the
+            // warp's lanes take them by shuffle.  DYN: e_l is log2 of the head's current pre-scale
+            // (O^T and l are held in its units).
+            const int hl = lane % HG;
+            float m_l = -INFINITY;
+            int e_l = 11;
+            float l_part[HG];
     #pragma unroll
-            for (int g = 0; g < HG; ++g) {
-                m_run[g] = -INFINITY;
-                l_part[g] = 0.0f;
-                if constexpr (DYN) e_run[g] = 11;
-            }
+            for (int g = 0; g < HG; ++g) l_part[g] = 0.0f;
             // TMEM lane 32 qd + lane holds token 32 qd + lane of the tile: slot 32 (qd % 2) + lane
             // of page qd / 2, so a warp owns 32 consecutive slots of one page
             const int page_of_thread = qd >> 1;
@@ -729,26 +730,35 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                     }
                     float y[HG], am[HG], corr[HG];
                     uint32_t mxc[HG];   // MXFP4 block scale codes
-                    bool rose = false;   // a running maximum of the group rose (alike in its four warps)
-        #pragma unroll
-                    for (int g = 0; g < HG; ++g) {
-                        const float4 w4 = *reinterpret_cast<const float4*>(rw + (gb + g) * 4);
+                    float corr_l, base_l, mz_l;
+                    bool rose_l;
+                    {
+                        const float4 w4 = *reinterpret_cast<const float4*>(rw + (gb + hl) * 4);
                         const float mt = fmaxf(fmaxf(w4.x, w4.y), fmaxf(w4.z, w4.w));
-                        const float mn = fmaxf(m_run[g], mt * lsr[g]);
-                        const float mz = mn == -INFINITY ? 0.0f : mn;
-                        corr[g] = tc::ex2_approx(m_run[g] - mz);   // 0 on the split's first tile
-                        rose |= mn != m_run[g];
-                        m_run[g] = mn;
-                        float base = mz - la;
+                        const float ls = lsc[gb + hl];
+                        const float mn = fmaxf(m_l, mt * ls);
+                        mz_l = mn == -INFINITY ? 0.0f : mn;
+                        corr_l = tc::ex2_approx(m_l - mz_l);   // 0 on the split's first tile
+                        rose_l = mn != m_l;
+                        m_l = mn;
+                        base_l = mz_l - la;
                         if constexpr (DYN) {
                             // this tile's pre-scale from its largest probability; the accumulators
                             // move to its units (an exact power of two, folded into corr)
-                            const int e = dynamic_alpha_exp(tc::ex2_approx(mt * lsr[g] - mz));
-                            corr[g] *= pow2f(e - e_run[g]);
-                            rose |= e != e_run[g];
-                            e_run[g] = e;
-                            base = mz - (float)e;
+                            const int e = dynamic_alpha_exp(tc::ex2_approx(mt * ls - mz_l));
+                            corr_l *= pow2f(e - e_l);
+                            rose_l |= e != e_l;
+                            e_l = e;
+                            base_l = mz_l - (float)e;
                         }
+                    }
+                    // a running maximum of the group rose (alike in its four warps)
+                    const bool rose = __any_sync(0xffffffffu, rose_l);
+        #pragma unroll
+                    for (int g = 0; g < HG; ++g) {
+                        corr[g] = __shfl_sync(0xffffffffu, corr_l, g);
+                        const float base = __shfl_sync(0xffffffffu, base_l, g);
+                        const float mz = MX ? __shfl_sync(0xffffffffu, mz_l, g) : 0.0f;
                         // the same two instructions give a token's scaled probability and its block's
                         // maximum, so the block scale is the one its largest member picks
                         y[g] = tc::ex2_approx(fmaf(t[g], lsr[g], -base));   // 0 for masked tokens
@@ -876,10 +886,11 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                             __float2bfloat16(l > 0.0f ? __uint_as_float(o_fin[g]) * oscale / l : 0.0f);
                     } else {
                         // DYN: splits end in different units; the partials leave in the units of p
-                        const float un = DYN ? pow2f(-e_run[DYN ? g : 0]) : 1.0f;
+                        const float un = DYN ? pow2f(-__shfl_sync(0xffffffffu, e_l, g)) : 1.0f;
+                        const float m_g = __shfl_sync(0xffffffffu, m_l, g);
                         a.ws_o[(row * a.max_splits + split) * C::DV + ch] = __uint_as_float(o_fin[g]) * oscale * un;
                         if (chan == 0) {
-                            a.ws_ml[(row * a.max_splits + split) * 2 + 0] = m_run[g];
+                            a.ws_ml[(row * a.max_splits + split) * 2 + 0] = m_g;
                             a.ws_ml[(row * a.max_splits + split) * 2 + 1] = l * un;
                         }
                     }
