@@ -72,13 +72,21 @@ DECODE_SOURCES = {
 }
 
 
+def _strip_comments(src: str) -> str:
+    """C/C++ source without its // and /* */ comments (string literals kept as they are)."""
+    import re
+    pat = re.compile(r'"(?:\\.|[^"\\])*"|//[^\n]*|/\*.*?\*/', re.S)
+    return pat.sub(lambda m: m.group(0) if m.group(0).startswith('"') else "", src)
+
+
 def decode_source_hash(d_k: int = 128) -> str:
-    """sha256 over the sources of the tensor-core decode kernel for head dim d_k."""
+    """sha256 over the sources of the tensor-core decode kernel for head dim d_k, comments
+    stripped: a recorded capture stays valid across comment edits, not across code edits."""
     import hashlib
     h = hashlib.sha256()
     for name in DECODE_SOURCES[d_k]:
-        with open(os.path.join(ROOT, "fp4_kv_cache_quant_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "fp4_kv_cache_quant_b200", "csrc", name), encoding="utf-8") as f:
+            h.update(_strip_comments(f.read()).encode())
     return h.hexdigest()
 
 

@@ -19,10 +19,12 @@
 //               t), so the softmax is transposed -- per-head maxima are warp
 //               reductions, the FP4 quantization of P (beta-token blocks) takes
 //               the maximum over the lanes of a block, and the P codes go
-//               straight into the shared-memory operand of the PV MMA.  The
-//               same threads write the block-scale factors into TMEM and, when
-//               a running maximum rises, rescale their heads' O^T columns in
-//               TMEM between the previous tile's PV and this one's.
+//               straight into the shared-memory operand of the PV MMA.  A
+//               head's running maximum and per-tile terms are computed once per
+//               warp, by the lanes that hold the head, and shuffled to the
+//               others.  The same threads write the block-scale factors of P
+//               and, when a running maximum rises, rescale their heads' O^T
+//               columns in TMEM between the previous tile's PV and this one's.
 // The dynamic variant (DYN, NVFP4) picks the probability pre-scale per tile and
 // head and folds a change of it into that same rescale.
 // Every wait is bounded; a timeout sets BDFP4_DEV_TIMEOUT and the CTA unwinds.

@@ -62,3 +62,14 @@ def test_reference_arm_under_torchrun_prints_once():
     assert out.returncode == 0, out.stderr[-2000:]
     lines = [json.loads(l) for l in out.stdout.splitlines() if l.startswith("{")]
     assert len(lines) == 1 and lines[0]["impl"] == "reference" and lines[0]["n_gpus"] == 2
+
+
+def test_source_hash_ignores_comments_only():
+    """The traffic records are keyed by a hash of the decode sources without comments: a comment
+    edit keeps a capture valid, a code edit (even inside a string literal) does not."""
+    import bench
+    src = 'int a = 1; // note\n/* block\n note */ asm("mov.b32 %0, 1; // kept");\n'
+    out = bench._strip_comments(src)
+    assert "note" not in out and "int a = 1;" in out and '"mov.b32 %0, 1; // kept"' in out
+    assert bench._strip_comments(src.replace("// note", "// other")) == out
+    assert bench._strip_comments(src.replace("a = 1", "a = 2")) != out
