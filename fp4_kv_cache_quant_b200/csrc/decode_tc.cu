@@ -731,8 +731,10 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                         break;
                     }
                     float y[HG], am[HG], corr[HG];
-                    uint32_t mxc[HG];   // MXFP4 block scale codes
+                    [[maybe_unused]] uint32_t mxc[HG];   // MXFP4 block scale codes
                     float corr_l, base_l, mz_l;
+                    [[maybe_unused]] float eb_l = 0.0f;   // MXFP4: head hl's element exponent base m + (c - 127)
+                    [[maybe_unused]] int c_l = 0;         // MXFP4: head hl's block scale code (the block is the warp)
                     bool rose_l;
                     {
                         const float4 w4 = *reinterpret_cast<const float4*>(rw + (gb + hl) * 4);
@@ -753,6 +755,18 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                             e_l = e;
                             base_l = mz_l - (float)e;
                         }
+                        if constexpr (MX) {
+                            // the OCP MX shared exponent of head hl's 32-token block (this warp), in
+                            // the log domain: the block maximum is 2^d with d = x_b - m, so floor(log2) =
+                            // floor(d) exactly (d = 0 for the tile's largest logit), and the element is
+                            // 2^(x - m - e) for the scale 2^e
+                            float bm = fmaxf(hm_lo[0], hm_hi[0]);
+        #pragma unroll
+                            for (int g = 1; g < HG; ++g) bm = hl == g ? fmaxf(hm_lo[g], hm_hi[g]) : bm;
+                            const float dd = __fsub_rn(__fmul_rn(bm, ls), mz_l);
+                            c_l = max(__float2int_rd(fmaxf(dd, -256.0f)) + 125, 0);
+                            eb_l = mz_l + (float)(c_l - 127);
+                        }
                     }
                     // a running maximum of the group rose (alike in its four warps)
                     const bool rose = __any_sync(0xffffffffu, rose_l);
@@ -760,7 +774,6 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                     for (int g = 0; g < HG; ++g) {
                         corr[g] = __shfl_sync(0xffffffffu, corr_l, g);
                         const float base = __shfl_sync(0xffffffffu, base_l, g);
-                        const float mz = MX ? __shfl_sync(0xffffffffu, mz_l, g) : 0.0f;
                         // the same two instructions give a token's scaled probability and its block's
                         // maximum, so the block scale is the one its largest member picks
                         y[g] = tc::ex2_approx(fmaf(t[g], lsr[g], -base));   // 0 for masked tokens
@@ -770,15 +783,9 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                             const float bm = lo_half ? hm_lo[g] : hm_hi[g];
                             am[g] = tc::ex2_approx(fmaf(bm, lsr[g], -base));
                         } else {
-                            // a 32-token block is this warp.  The OCP MX shared exponent is taken in the
-                            // log domain: the block maximum is 2^d with d = x_b - m, so floor(log2) =
-                            // floor(d) exactly (d = 0 for the tile's largest logit), and the element is
-                            // 2^(x - m - e) for the scale 2^e
-                            const float bm = fmaxf(hm_lo[g], hm_hi[g]);
-                            const float d = __fsub_rn(__fmul_rn(bm, lsr[g]), mz);
-                            const int c = max(__float2int_rd(fmaxf(d, -256.0f)) + 125, 0);
-                            mxc[g] = (uint32_t)c;
-                            am[g] = tc::ex2_approx(fmaf(t[g], lsr[g], -(mz + (float)(c - 127))));
+                            // a 32-token block is this warp: its exponent from the head's lanes
+                            mxc[g] = (uint32_t)__shfl_sync(0xffffffffu, c_l, g);
+                            am[g] = tc::ex2_approx(fmaf(t[g], lsr[g], -__shfl_sync(0xffffffffu, eb_l, g)));
                         }
                     }
                     // fused FP4 quantization of the probabilities, two heads per conversion
