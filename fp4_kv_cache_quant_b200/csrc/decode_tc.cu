@@ -730,11 +730,17 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                         grp_abort = true;
                         break;
                     }
-                    float y[HG], am[HG], corr[HG];
+                    float y[HG], corr[HG];
+                    [[maybe_unused]] float am[HG];   // block maxima of alpha p (NVFP4 up to two heads per group), MXFP4 elements
                     [[maybe_unused]] uint32_t mxc[HG];   // MXFP4 block scale codes
                     float corr_l, base_l, mz_l;
                     [[maybe_unused]] float eb_l = 0.0f;   // MXFP4: head hl's element exponent base m + (c - 127)
                     [[maybe_unused]] int c_l = 0;         // MXFP4: head hl's block scale code (the block is the warp)
+                    // NVFP4, four or more heads per group: the block scale of head hl over half warp
+                    // (lane / HG) % 2, its code and reciprocal (a 16-token block is a half warp)
+                    constexpr bool NV_LANE = !MX && HG >= 4;
+                    [[maybe_unused]] float rinv_l = 0.0f;
+                    [[maybe_unused]] uint32_t code_l = 0u;
                     bool rose_l;
                     {
                         const float4 w4 = *reinterpret_cast<const float4*>(rw + (gb + hl) * 4);
@@ -767,6 +773,16 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                             c_l = max(__float2int_rd(fmaxf(dd, -256.0f)) + 125, 0);
                             eb_l = mz_l + (float)(c_l - 127);
                         }
+                        if constexpr (NV_LANE) {
+                            const bool hh = ((lane / HG) & 1) != 0;
+                            float bm = hh ? hm_hi[0] : hm_lo[0];
+        #pragma unroll
+                            for (int g = 1; g < HG; ++g) bm = hl == g ? (hh ? hm_hi[g] : hm_lo[g]) : bm;
+                            const float ab = tc::ex2_approx(fmaf(bm, ls, -base_l));
+                            code_l = tc::e4m3x2_encode(__fmul_rn(ab, 1.0f / 6.0f), 0.0f) & 0xffu;
+                            // a zero scale zeroes the whole block inside the MMA, whatever the element codes
+                            rinv_l = tc::rcp_approx(tc::e4m3x2_value(code_l).x);
+                        }
                     }
                     // a running maximum of the group rose (alike in its four warps)
                     const bool rose = __any_sync(0xffffffffu, rose_l);
@@ -780,8 +796,10 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                         l_part[g] = fmaf(l_part[g], corr[g], y[g]);         // l in units of alpha (cancels at the end)
                         if constexpr (!MX) {
                             // a 16-token block is this half warp
-                            const float bm = lo_half ? hm_lo[g] : hm_hi[g];
-                            am[g] = tc::ex2_approx(fmaf(bm, lsr[g], -base));
+                            if constexpr (!NV_LANE) {
+                                const float bm = lo_half ? hm_lo[g] : hm_hi[g];
+                                am[g] = tc::ex2_approx(fmaf(bm, lsr[g], -base));
+                            }
                         } else {
                             // a 32-token block is this warp: its exponent from the head's lanes
                             mxc[g] = (uint32_t)__shfl_sync(0xffffffffu, c_l, g);
@@ -796,7 +814,13 @@ __global__ void __launch_bounds__(TcCfg<FMT, G>::THREADS, TcCfg<FMT, G>::MIN_CTA
                         const int g1 = HG >= 2 ? g + 1 : g;
                         uint32_t codes;
                         float q0, q1;
-                        if constexpr (FMT == BDFP4_NVFP4) {
+                        if constexpr (NV_LANE) {
+                            // the block scales of this half warp, from the lanes of heads g and g1
+                            const int ho = lo_half ? 0 : HG;
+                            q0 = y[g] * __shfl_sync(0xffffffffu, rinv_l, g + ho);
+                            q1 = y[g1] * __shfl_sync(0xffffffffu, rinv_l, g1 + ho);
+                            codes = __shfl_sync(0xffffffffu, code_l, g + hsel + ho) << (8 * hsel);
+                        } else if constexpr (FMT == BDFP4_NVFP4) {
                             codes = tc::e4m3x2_encode(__fmul_rn(am[g], 1.0f / 6.0f), __fmul_rn(am[g1], 1.0f / 6.0f));
                             const float2 sg = tc::e4m3x2_value(codes);
                             // a zero scale zeroes the whole block inside the MMA, whatever the element codes
